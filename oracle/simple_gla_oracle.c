@@ -1,0 +1,183 @@
+/*
+ * Simple GLA oracle: a plain, slow, fp64 CPU statement of what the GPU path
+ * computes.  TEST INFRASTRUCTURE ONLY -- the tests, the smoke check and the
+ * bench's CPU-baseline leg are the only callers; the product path never
+ * links, loads or calls this file.
+ *
+ * What it follows ("Simple GLA in flash-linear-attention: maths and kernels",
+ * xxqk.cn article; section numbers are the article's):
+ *   - section 1 (definition): one scalar forget gate per head and token, the
+ *     state update S_t = gate_t * S_{t-1} + k_t v_t^T, written in the naive
+ *     reference as "S = S * gate + kv";
+ *   - section 1 / 2: the gate arrives in log space (the API example feeds
+ *     logsigmoid outputs and the chunk path pre-scales by 1/ln2 to use exp2),
+ *     so the multiplier is exp(g_t);  g_gamma[h] is a data-independent
+ *     per-head log decay used instead of g (never both);
+ *   - section 1 (the tril mask includes the diagonal): the read-out uses the
+ *     state after the update, o_t = scale * S_t^T q_t;
+ *   - section 2: q,k [B,T,H,K], v,o [B,T,H,V], states [N,H,K,V]; scale
+ *     defaults to 1/sqrt(K) (the Python wrapper applies that default);
+ *     with cu_seqlens the batch is 1 and sequence n spans tokens
+ *     cu[n] .. cu[n+1]-1, each with its own initial and final state.
+ * Readings of the page where it is silent: neither g nor g_gamma means g == 0;
+ * a zero-length sequence returns its initial state unchanged.
+ *
+ * There is no chunking, blocking or reordering here: the loop is the
+ * recurrence itself, token by token, in fp64.  The chunked GPU method reaches
+ * the same numbers up to rounding by regrouping these sums.
+ *
+ * Parity pins for this file (brute force, closed forms, invariants) live in
+ * the tests; every function here is pinned.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { GATE_NONE = 0, GATE_PER_TOKEN = 1, GATE_PER_HEAD = 2 };
+
+/*
+ * One (sequence, head) pair: tokens [t_begin, t_end) of the flattened token
+ * axis.  Tensors are row-major [tokens, H, D].  S is K*V scratch (row k, col v).
+ */
+static void recur_one_head(const double *q, const double *k, const double *v,
+                           const double *g, const double *g_gamma, int gate_mode,
+                           double scale, const double *h0, double *o, double *hT,
+                           int64_t t_begin, int64_t t_end, int64_t h, int64_t H,
+                           int64_t K, int64_t V, double *S)
+{
+    if (h0)
+        memcpy(S, h0, (size_t)(K * V) * sizeof(double));
+    else
+        memset(S, 0, (size_t)(K * V) * sizeof(double));
+
+    for (int64_t t = t_begin; t < t_end; ++t) {
+        double a = 0.0;
+        if (gate_mode == GATE_PER_TOKEN)
+            a = g[t * H + h];
+        else if (gate_mode == GATE_PER_HEAD)
+            a = g_gamma[h];
+        const double decay = exp(a);
+        const double *qt = q + (t * H + h) * K;
+        const double *kt = k + (t * H + h) * K;
+        const double *vt = v + (t * H + h) * V;
+
+        /* S_t = exp(g_t) S_{t-1} + k_t v_t^T */
+        for (int64_t i = 0; i < K; ++i)
+            for (int64_t j = 0; j < V; ++j)
+                S[i * V + j] = decay * S[i * V + j] + kt[i] * vt[j];
+
+        /* o_t = scale * S_t^T q_t  (post-update state) */
+        double *ot = o + (t * H + h) * V;
+        for (int64_t j = 0; j < V; ++j) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < K; ++i)
+                acc += qt[i] * S[i * V + j];
+            ot[j] = scale * acc;
+        }
+    }
+    if (hT)
+        memcpy(hT, S, (size_t)(K * V) * sizeof(double));
+}
+
+static int gate_mode_of(const double *g, const double *g_gamma)
+{
+    if (g && g_gamma)
+        return -1;
+    return g ? GATE_PER_TOKEN : (g_gamma ? GATE_PER_HEAD : GATE_NONE);
+}
+
+/*
+ * Forward over a dense batch (cu_seqlens == NULL: N = B sequences of T tokens)
+ * or a packed variable-length batch (cu_seqlens != NULL: B must be 1, N
+ * sequences, cu_seqlens[N] == T).  h0 / hT are [N,H,K,V] or NULL.
+ * Returns 0 on success, a negative code on an invalid argument.
+ */
+int sgla_oracle_fwd(const double *q, const double *k, const double *v,
+                    const double *g, const double *g_gamma, double scale,
+                    const double *h0, double *o, double *hT,
+                    const int64_t *cu_seqlens, int64_t N,
+                    int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                    int nthreads)
+{
+    const int gate_mode = gate_mode_of(g, g_gamma);
+    if (gate_mode < 0)
+        return -1;
+    if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0)
+        return -2;
+    if (cu_seqlens) {
+        if (B != 1 || N < 1 || cu_seqlens[0] != 0 || cu_seqlens[N] != T)
+            return -3;
+        for (int64_t n = 0; n < N; ++n)
+            if (cu_seqlens[n + 1] < cu_seqlens[n])
+                return -4;
+    } else {
+        N = B;
+    }
+    const int64_t units = N * H;
+    int err = 0;
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+    for (int64_t u = 0; u < units; ++u) {
+        const int64_t n = u / H, h = u % H;
+        const int64_t t0 = cu_seqlens ? cu_seqlens[n] : n * T;
+        const int64_t t1 = cu_seqlens ? cu_seqlens[n + 1] : (n + 1) * T;
+        double *S = (double *)malloc((size_t)(K * V) * sizeof(double));
+        if (!S) {
+            err = -5;
+            continue;
+        }
+        const size_t state_off = (size_t)((n * H + h) * K * V);
+        recur_one_head(q, k, v, g, g_gamma, gate_mode, scale,
+                       h0 ? h0 + state_off : NULL, o, hT ? hT + state_off : NULL,
+                       t0, t1, h, H, K, V, S);
+        free(S);
+    }
+    return err;
+}
+
+/*
+ * One recurrent decode step for N independent sequences: the same update and
+ * read-out as one token of the forward, applied to a caller-held state that is
+ * updated in place.  q,k [N,H,K]; v,o [N,H,V]; g [N,H] or g_gamma [H] or
+ * neither; state [N,H,K,V].
+ */
+int sgla_oracle_decode_step(const double *q, const double *k, const double *v,
+                            const double *g, const double *g_gamma, double scale,
+                            double *state, double *o,
+                            int64_t N, int64_t H, int64_t K, int64_t V,
+                            int nthreads)
+{
+    const int gate_mode = gate_mode_of(g, g_gamma);
+    if (gate_mode < 0)
+        return -1;
+    if (N < 0 || H <= 0 || K <= 0 || V <= 0)
+        return -2;
+    const int64_t units = N * H;
+    int err = 0;
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+    for (int64_t u = 0; u < units; ++u) {
+        const int64_t n = u / H, h = u % H;
+        double *S = (double *)malloc((size_t)(K * V) * sizeof(double));
+        if (!S) {
+            err = -5;
+            continue;
+        }
+        double *st = state + (size_t)((n * H + h) * K * V);
+        /* token n of a length-N "sequence axis": one token per sequence */
+        recur_one_head(q, k, v, g, g_gamma, gate_mode, scale, st, o, st,
+                       n, n + 1, h, H, K, V, S);
+        free(S);
+    }
+    return err;
+}
