@@ -1,0 +1,218 @@
+"""B200 (sm_100a) Simple GLA: Python binding of libsimplegla.so.
+
+The operator is head-wise gated linear attention as stated in "Simple GLA in
+flash-linear-attention: maths and kernels" (xxqk.cn article): per head
+S_t = exp(g_t) S_{t-1} + k_t v_t^T and o_t = scale * q_t^T S_t (section 1), with
+the chunk_simple_gla argument conventions of section 2 and the chunked kernels
+of section 3.
+
+This module only marshals arguments: it checks tensor types and shapes, takes
+device memory (outputs, workspace) from PyTorch's caching allocator, passes raw
+pointers and the current CUDA stream to the C ABI declared in
+``include/simple_gla.h``, and maps status codes to exceptions.  Every step of the
+computation runs in the library's CUDA kernels; there is no fallback of any kind
+-- a missing library or a CPU tensor is an error.
+
+Public functions (same names as the C entry points):
+  simple_gla_fwd(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
+                 output_final_state=False, chunk_size=64) -> (o, final_state|None)
+  simple_gla_fwd_varlen(q, k, v, cu_seqlens, g=None, ...) -> (o, final_state|None)
+  simple_gla_decode_step(q, k, v, state, g=None, g_gamma=None, scale=None) -> o
+  chunk_simple_gla(...)  -- the article's entry-point name; dispatches on cu_seqlens.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from ._lib import (SGLA_BF16, SGLA_FP32, SGLA_OK, SglaError, lib, library_path,  # noqa: F401
+                   raise_for_status)
+
+__all__ = ["simple_gla_fwd", "simple_gla_fwd_varlen", "simple_gla_decode_step", "chunk_simple_gla",
+           "fwd_workspace_size", "varlen_workspace_size", "workspace_status", "library_path",
+           "SglaError"]
+
+_DTYPES = {torch.bfloat16: SGLA_BF16, torch.float32: SGLA_FP32}
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check_cuda(name, t, dtype=None, ndim=None):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
+
+
+def fwd_workspace_size(B, T, H, K, V, chunk_size=64, dtype=torch.bfloat16) -> int:
+    return int(lib().simple_gla_fwd_workspace_size(B, T, H, K, V, chunk_size, _DTYPES[dtype]))
+
+
+def varlen_workspace_size(N, T_total, H, K, V, chunk_size=64, dtype=torch.bfloat16) -> int:
+    return int(lib().simple_gla_fwd_varlen_workspace_size(N, T_total, H, K, V, chunk_size, _DTYPES[dtype]))
+
+
+def _workspace(nbytes, device, workspace):
+    if workspace is not None:
+        _check_cuda("workspace", workspace, torch.uint8)
+        if workspace.numel() < nbytes:
+            raise ValueError(f"workspace holds {workspace.numel()} bytes, {nbytes} needed")
+        return workspace
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def _common_checks(q, k, v, g, g_gamma, initial_state):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_cuda(name, t)
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"q,k,v must be bfloat16 or float32, got {q.dtype}")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k and v must share one dtype")
+    if g is not None and g_gamma is not None:
+        raise ValueError("only one of g and g_gamma may be provided")
+    _check_cuda("g", g, torch.float32)
+    _check_cuda("g_gamma", g_gamma, torch.float32, 1)
+    _check_cuda("initial_state", initial_state, torch.float32, 4)
+
+
+def simple_gla_fwd(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
+                   output_final_state=False, chunk_size=64, workspace=None):
+    """Dense chunked forward.  q,k [B,T,H,K]; v [B,T,H,V]; g [B,T,H] fp32 log gates or
+    g_gamma [H]; initial_state [B,H,K,V] fp32.  Returns (o [B,T,H,V], final_state)."""
+    _common_checks(q, k, v, g, g_gamma, initial_state)
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q,k must be [B,T,H,K] and v [B,T,H,V]")
+    B, T, H, K = q.shape
+    V = v.shape[3]
+    if g is not None and tuple(g.shape) != (B, T, H):
+        raise ValueError(f"g must be [B,T,H] = {(B, T, H)}, got {tuple(g.shape)}")
+    if g_gamma is not None and tuple(g_gamma.shape) != (H,):
+        raise ValueError(f"g_gamma must be [H] = ({H},)")
+    if initial_state is not None and tuple(initial_state.shape) != (B, H, K, V):
+        raise ValueError(f"initial_state must be [B,H,K,V] = {(B, H, K, V)}")
+    dt = _DTYPES[q.dtype]
+    o = torch.empty((B, T, H, V), dtype=q.dtype, device=q.device)
+    ht = torch.empty((B, H, K, V), dtype=torch.float32, device=q.device) if output_final_state else None
+    nbytes = int(lib().simple_gla_fwd_workspace_size(B, T, H, K, V, chunk_size, dt))
+    if nbytes == 0:
+        raise_for_status(_size_status(K, V, chunk_size), "simple_gla_fwd")
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().simple_gla_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma),
+                              ctypes.c_float(_scale(scale)), _ptr(initial_state), _ptr(o), _ptr(ht),
+                              B, T, H, K, V, chunk_size, dt, _ptr(ws), ws.numel(), _stream())
+    raise_for_status(st, "simple_gla_fwd")
+    return o, ht
+
+
+def simple_gla_fwd_varlen(q, k, v, cu_seqlens, g=None, g_gamma=None, scale=None, initial_state=None,
+                          output_final_state=False, chunk_size=64, workspace=None):
+    """Packed variable-length forward.  q,k [1,T,H,K] or [T,H,K]; v likewise with V;
+    cu_seqlens [N+1] int64 on the device; g [1,T,H] or [T,H]; initial_state [N,H,K,V]."""
+    _common_checks(q, k, v, g, g_gamma, initial_state)
+    _check_cuda("cu_seqlens", cu_seqlens, torch.int64, 1)
+    if q.dim() == 4:
+        if q.shape[0] != 1:
+            raise ValueError("with cu_seqlens the batch size must be 1 (flatten the batch first)")
+        q, k, v = q[0], k[0], v[0]
+        g = g[0] if g is not None else None
+        squeeze = True
+    else:
+        squeeze = False
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+        raise ValueError("q,k must be [T,H,K] and v [T,H,V] (or with a leading batch of 1)")
+    T, H, K = q.shape
+    V = v.shape[2]
+    N = cu_seqlens.shape[0] - 1
+    if N < 1:
+        raise ValueError("cu_seqlens must hold at least two entries")
+    if g is not None and tuple(g.shape) != (T, H):
+        raise ValueError("g must be [T,H] (or [1,T,H])")
+    if g_gamma is not None and tuple(g_gamma.shape) != (H,):
+        raise ValueError("g_gamma must be [H]")
+    if initial_state is not None and initial_state.shape[0] != N:
+        raise ValueError(f"the number of initial states must equal len(cu_seqlens) - 1 = {N}, "
+                         f"got {initial_state.shape[0]}")
+    if initial_state is not None and tuple(initial_state.shape) != (N, H, K, V):
+        raise ValueError(f"initial_state must be [N,H,K,V] = {(N, H, K, V)}")
+    dt = _DTYPES[q.dtype]
+    o = torch.empty((T, H, V), dtype=q.dtype, device=q.device)
+    ht = torch.empty((N, H, K, V), dtype=torch.float32, device=q.device) if output_final_state else None
+    nbytes = int(lib().simple_gla_fwd_varlen_workspace_size(N, T, H, K, V, chunk_size, dt))
+    if nbytes == 0:
+        raise_for_status(_size_status(K, V, chunk_size), "simple_gla_fwd_varlen")
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().simple_gla_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma),
+                                     ctypes.c_float(_scale(scale)), _ptr(cu_seqlens), N, T,
+                                     _ptr(initial_state), _ptr(o), _ptr(ht), H, K, V, chunk_size, dt,
+                                     _ptr(ws), ws.numel(), _stream())
+    raise_for_status(st, "simple_gla_fwd_varlen")
+    return (o.unsqueeze(0) if squeeze else o), ht
+
+
+def chunk_simple_gla(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
+                     output_final_state=False, cu_seqlens=None, chunk_size=64):
+    """The article's entry-point name (section 2): dense, or packed when cu_seqlens is given."""
+    if cu_seqlens is None:
+        return simple_gla_fwd(q, k, v, g, g_gamma, scale, initial_state, output_final_state, chunk_size)
+    return simple_gla_fwd_varlen(q, k, v, cu_seqlens, g, g_gamma, scale, initial_state,
+                                 output_final_state, chunk_size)
+
+
+def simple_gla_decode_step(q, k, v, state, g=None, g_gamma=None, scale=None, out=None):
+    """One recurrent step.  q,k [N,H,K]; v [N,H,V]; g [N,H] fp32 or g_gamma [H];
+    state [N,H,K,V] fp32 updated in place.  Returns o [N,H,V]."""
+    _common_checks(q, k, v, g, g_gamma, None)
+    _check_cuda("state", state, torch.float32, 4)
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+        raise ValueError("q,k must be [N,H,K] and v [N,H,V]")
+    N, H, K = q.shape
+    V = v.shape[2]
+    if tuple(state.shape) != (N, H, K, V):
+        raise ValueError(f"state must be [N,H,K,V] = {(N, H, K, V)}")
+    if g is not None and tuple(g.shape) != (N, H):
+        raise ValueError("g must be [N,H]")
+    if g_gamma is not None and tuple(g_gamma.shape) != (H,):
+        raise ValueError("g_gamma must be [H]")
+    o = out if out is not None else torch.empty((N, H, V), dtype=q.dtype, device=q.device)
+    _check_cuda("out", o, q.dtype, 3)
+    st = lib().simple_gla_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma),
+                                      ctypes.c_float(_scale(scale)), _ptr(state), _ptr(o), N, H, K, V,
+                                      _DTYPES[q.dtype], _stream())
+    raise_for_status(st, "simple_gla_decode_step")
+    return o
+
+
+def workspace_status(workspace) -> int:
+    """Device status word of the last forward that used ``workspace`` (synchronises)."""
+    out = ctypes.c_int(-1)
+    raise_for_status(lib().sgla_workspace_status(_ptr(workspace), ctypes.byref(out), _stream()),
+                     "sgla_workspace_status")
+    return out.value
+
+
+def _scale(scale):
+    return float("nan") if scale is None else float(scale)
+
+
+def _size_status(K, V, chunk_size):
+    # mirrors the library's size rules only to pick the exception type for a zero
+    # workspace query; the library itself decides by returning 0
+    if chunk_size <= 0 or chunk_size & (chunk_size - 1):
+        return 1
+    return 2

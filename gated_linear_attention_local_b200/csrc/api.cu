@@ -1,0 +1,339 @@
+// C ABI of libsimplegla.so: argument validation, planning, workspace carve-up and
+// launch order.  Declarations and the contract of each entry point are in
+// include/simple_gla.h; the operator is the one of "Simple GLA in
+// flash-linear-attention: maths and kernels" (xxqk.cn article), sections 1-3.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <atomic>
+#include <vector>
+
+#include "kernels.h"
+#include "simple_gla.h"
+#include "tc_path.h"
+
+namespace {
+
+using namespace sgla;
+
+thread_local char g_last_cuda_error[256] = "";
+
+sgla_status cuda_fail(cudaError_t e, const char *where) {
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", where, cudaGetErrorString(e));
+    return SGLA_ERR_CUDA;
+}
+
+#define SGLA_CUDA(call, where)                         \
+    do {                                               \
+        cudaError_t e_ = (call);                       \
+        if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+    } while (0)
+
+// ---- tracing: launch counter and optional per-kernel events -----------------
+std::atomic<uint64_t> g_launches{0};
+bool g_prof_on = false;
+struct ProfRec {
+    const char *name;
+    cudaEvent_t a, b;
+};
+std::vector<ProfRec> g_prof;
+
+void prof_mark(cudaStream_t st, cudaEvent_t *ev) {
+    *ev = nullptr;
+    if (!g_prof_on) return;
+    if (cudaEventCreate(ev) != cudaSuccess) { *ev = nullptr; return; }
+    cudaEventRecord(*ev, st);
+}
+
+void prof_push(const char *name, cudaEvent_t a, cudaEvent_t b) {
+    if (a && b) g_prof.push_back({name, a, b});
+    else {
+        if (a) cudaEventDestroy(a);
+        if (b) cudaEventDestroy(b);
+    }
+}
+
+// Launch one kernel through its launcher, counting it and (when recording) timing it.
+#define SGLA_LAUNCH(name, call)                                   \
+    do {                                                          \
+        cudaEvent_t ea_, eb_;                                     \
+        prof_mark(st, &ea_);                                      \
+        cudaError_t e_ = (call);                                  \
+        prof_mark(st, &eb_);                                      \
+        prof_push(name, ea_, eb_);                                \
+        if (e_ != cudaSuccess) return cuda_fail(e_, name);        \
+        g_launches.fetch_add(1, std::memory_order_relaxed);       \
+    } while (0)
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+constexpr int64_t kMaxTokens = (int64_t)1 << 31;
+
+// Everything derived from the sizes alone: path, segment length, grid bounds and
+// workspace offsets.  The workspace query and the launch both go through here.
+struct Plan {
+    bool valid = false;
+    sgla_status why = SGLA_ERR_INVALID_ARGUMENT;
+    bool tc = false;           // tensor-core (tcgen05) path
+    int C = 0, L = 1, NT = 0, NS = 0;
+    int64_t max_chunks = 0, max_segs = 0;
+    bool multi_seg = false;    // some sequence may have more than one segment
+    size_t off_chunk_off = 0, off_seg_off = 0, off_gcum = 0, off_seg_dec = 0, off_seg_state = 0;
+    size_t bytes = 0;
+};
+
+sgla_status check_sizes(int64_t H, int64_t K, int64_t V, int chunk_size) {
+    if (H < 1 || K < 1 || V < 1) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!is_pow2(chunk_size)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (chunk_size < 16 || chunk_size > 128) return SGLA_ERR_UNSUPPORTED;
+    if (K > 512 || V > 512 || K % 8 || V % 8) return SGLA_ERR_UNSUPPORTED;
+    if (H > 65535) return SGLA_ERR_UNSUPPORTED;
+    return SGLA_OK;
+}
+
+// varlen: N sequences, T = total tokens; dense: N = B, T = tokens per sequence.
+Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V, int C,
+               sgla_dtype dtype, bool per_token_gate) {
+    Plan p;
+    sgla_status st = check_sizes(H, K, V, C);
+    if (st != SGLA_OK) { p.why = st; return p; }
+    if (dtype != SGLA_BF16 && dtype != SGLA_FP32) return p;
+    if (N < (varlen ? 1 : 0) || T < 0) return p;
+    const int64_t tokens = varlen ? T : N * T;
+    if (tokens >= kMaxTokens || N >= kMaxTokens) { p.why = SGLA_ERR_UNSUPPORTED; return p; }
+    p.C = C;
+    p.tc = tc_path_supports(dtype == SGLA_BF16, (int)K, (int)V, C);
+    const int64_t chunks_est = varlen ? (T + C - 1) / C : N * ((T + C - 1) / C);
+    // Segment length: long enough to keep state round trips rare, short enough that
+    // (segments x heads x V tiles) still fills the 148 SMs a few times over.
+    const int64_t vtiles = p.tc ? tc_path_vtiles((int)K, (int)V) : (V + 31) / 32;
+    const int64_t target_ctas = p.tc ? tc_path_target_ctas() : 4 * 148;
+    int64_t L = std::max<int64_t>(1, (chunks_est * H * vtiles) / target_ctas);
+    if (!varlen) L = std::min<int64_t>(L, std::max<int64_t>(1, (T + C - 1) / C));
+    L = std::min<int64_t>(L, 1 << 20);
+    p.L = (int)L;
+    if (varlen) {
+        p.max_chunks = T / C + N;
+        p.max_segs = T / (C * L) + N;
+        p.multi_seg = true;
+    } else {
+        p.NT = (int)((T + C - 1) / C);
+        p.NS = (p.NT + p.L - 1) / p.L;
+        p.max_chunks = N * p.NT;
+        p.max_segs = N * p.NS;
+        p.multi_seg = p.NS > 1;
+    }
+    if (p.max_chunks >= kMaxTokens || p.max_segs * H >= kMaxTokens) { p.why = SGLA_ERR_UNSUPPORTED; return p; }
+    size_t off = 256;  // status word
+    if (varlen) {
+        p.off_chunk_off = off;
+        off = align_up(off + sizeof(int) * (size_t)(N + 1), 256);
+        p.off_seg_off = off;
+        off = align_up(off + sizeof(int) * (size_t)(N + 1), 256);
+    }
+    if (per_token_gate) {
+        p.off_gcum = off;
+        off = align_up(off + sizeof(float) * (size_t)tokens * H, 256);
+    }
+    if (p.multi_seg) {
+        p.off_seg_dec = off;
+        off = align_up(off + sizeof(float) * (size_t)p.max_segs * H, 256);
+        p.off_seg_state = off;
+        off = align_up(off + sizeof(float) * (size_t)p.max_segs * H * K * V, 256);
+    }
+    p.bytes = off;
+    p.valid = true;
+    return p;
+}
+
+sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v, const float *g,
+                        const float *g_gamma, float scale, const int64_t *cu, int64_t N, int64_t T,
+                        const float *h0, void *o, float *hT, int64_t H, int64_t K, int64_t V,
+                        int chunk_size, sgla_dtype dtype, void *workspace, size_t workspace_bytes,
+                        void *stream) {
+    if (g && g_gamma) return SGLA_ERR_INVALID_ARGUMENT;
+    const int64_t tokens = varlen ? T : N * T;
+    if (tokens > 0 && (!q || !k || !v || !o)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (varlen && !cu) return SGLA_ERR_INVALID_ARGUMENT;
+    for (const void *p : {q, k, v, (const void *)o, (const void *)h0, (const void *)hT})
+        if (!aligned(p, 16)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!aligned(g, 4) || !aligned(g_gamma, 4) || !aligned(cu, 8)) return SGLA_ERR_INVALID_ARGUMENT;
+    const bool per_token = g != nullptr;
+    Plan p = make_plan(varlen, N, T, H, K, V, chunk_size, dtype, per_token);
+    if (!p.valid) return p.why;
+    if (!workspace || workspace_bytes < p.bytes) return SGLA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!(scale > 0.f) || isnan(scale) || isinf(scale)) scale = 1.0f / sqrtf((float)K);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+
+    FwdArgs a{};
+    a.q = q; a.k = k; a.v = v; a.g = g; a.g_gamma = g_gamma; a.scale = scale;
+    a.h0 = h0; a.o = o; a.hT = hT;
+    a.H = (int)H; a.K = (int)K; a.V = (int)V;
+    a.gate_mode = g ? kGatePerToken : (g_gamma ? kGatePerHead : kGateNone);
+    a.bf16 = dtype == SGLA_BF16;
+    a.gcum = per_token ? reinterpret_cast<float *>(ws + p.off_gcum) : nullptr;
+    a.seg_dec = p.multi_seg ? reinterpret_cast<float *>(ws + p.off_seg_dec) : nullptr;
+    a.seg_state = p.multi_seg ? reinterpret_cast<float *>(ws + p.off_seg_state) : nullptr;
+    SeqLayout &lay = a.lay;
+    lay.cu = varlen ? cu : nullptr;
+    lay.chunk_off = varlen ? reinterpret_cast<int *>(ws + p.off_chunk_off) : nullptr;
+    lay.seg_off = varlen ? reinterpret_cast<int *>(ws + p.off_seg_off) : nullptr;
+    lay.status = reinterpret_cast<int *>(ws);
+    lay.T = T; lay.N = (int)N; lay.H = (int)H; lay.C = p.C; lay.L = p.L;
+    lay.NT = p.NT; lay.NS = p.NS;
+    lay.max_chunks = (int)p.max_chunks; lay.max_segs = (int)p.max_segs;
+
+    if (varlen) {
+        SGLA_LAUNCH("varlen_plan", launch_varlen_plan(cu, (int)N, T, p.C, p.L, const_cast<int *>(lay.chunk_off),
+                                                      const_cast<int *>(lay.seg_off),
+                                                      reinterpret_cast<int *>(ws), st));
+    } else {
+        SGLA_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), st), "status reset");
+    }
+    if (N == 0) return SGLA_OK;
+    if (per_token && tokens > 0) SGLA_LAUNCH("chunk_cumsum", launch_chunk_cumsum(g, a.gcum, lay, st));
+    if (p.multi_seg && p.max_segs > 0) {
+        if (p.tc) SGLA_LAUNCH("segment_state_tc", tc_launch_segment_state(a, st));
+        else SGLA_LAUNCH("segment_state_simt", launch_segment_state_simt(a, st));
+    }
+    const bool empty_dense = !varlen && p.NT == 0;
+    if (p.multi_seg || (empty_dense && hT)) SGLA_LAUNCH("segment_carry", launch_segment_carry(a, p.multi_seg, st));
+    if (tokens > 0 && p.max_segs > 0) {
+        if (p.tc) SGLA_LAUNCH("chunk_output_tc", tc_launch_chunk_output(a, st));
+        else SGLA_LAUNCH("chunk_output_simt", launch_chunk_output_simt(a, st));
+    }
+    return SGLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sgla_version(void) { return 100; }
+
+const char *sgla_status_string(int status) {
+    switch (status) {
+        case SGLA_OK: return "SGLA_OK";
+        case SGLA_ERR_INVALID_ARGUMENT: return "SGLA_ERR_INVALID_ARGUMENT";
+        case SGLA_ERR_UNSUPPORTED: return "SGLA_ERR_UNSUPPORTED";
+        case SGLA_ERR_CUDA: return "SGLA_ERR_CUDA";
+        case SGLA_ERR_WORKSPACE: return "SGLA_ERR_WORKSPACE";
+        case SGLA_ERR_DEVICE_CHECK: return "SGLA_ERR_DEVICE_CHECK";
+        default: return "SGLA_UNKNOWN_STATUS";
+    }
+}
+
+const char *sgla_last_cuda_error(void) { return g_last_cuda_error; }
+
+size_t simple_gla_fwd_workspace_size(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                                     int chunk_size, sgla_dtype dtype) {
+    Plan p = make_plan(false, B, T, H, K, V, chunk_size, dtype, true);
+    return p.valid ? p.bytes : 0;
+}
+
+size_t simple_gla_fwd_varlen_workspace_size(int64_t N, int64_t T_total, int64_t H, int64_t K,
+                                            int64_t V, int chunk_size, sgla_dtype dtype) {
+    Plan p = make_plan(true, N, T_total, H, K, V, chunk_size, dtype, true);
+    return p.valid ? p.bytes : 0;
+}
+
+sgla_status simple_gla_fwd(const void *q, const void *k, const void *v, const float *g,
+                           const float *g_gamma, float scale, const float *initial_state, void *o,
+                           float *final_state, int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                           int chunk_size, sgla_dtype dtype, void *workspace, size_t workspace_bytes,
+                           void *stream) {
+    if (B < 0 || T < 0) return SGLA_ERR_INVALID_ARGUMENT;
+    return run_forward(false, q, k, v, g, g_gamma, scale, nullptr, B, T, initial_state, o, final_state,
+                       H, K, V, chunk_size, dtype, workspace, workspace_bytes, stream);
+}
+
+sgla_status simple_gla_fwd_varlen(const void *q, const void *k, const void *v, const float *g,
+                                  const float *g_gamma, float scale, const int64_t *cu_seqlens,
+                                  int64_t N, int64_t T_total, const float *initial_state, void *o,
+                                  float *final_state, int64_t H, int64_t K, int64_t V, int chunk_size,
+                                  sgla_dtype dtype, void *workspace, size_t workspace_bytes,
+                                  void *stream) {
+    if (N < 1 || T_total < 0) return SGLA_ERR_INVALID_ARGUMENT;
+    return run_forward(true, q, k, v, g, g_gamma, scale, cu_seqlens, N, T_total, initial_state, o,
+                       final_state, H, K, V, chunk_size, dtype, workspace, workspace_bytes, stream);
+}
+
+sgla_status simple_gla_decode_step(const void *q, const void *k, const void *v, const float *g,
+                                   const float *g_gamma, float scale, float *state, void *o, int64_t N,
+                                   int64_t H, int64_t K, int64_t V, sgla_dtype dtype, void *stream) {
+    if (g && g_gamma) return SGLA_ERR_INVALID_ARGUMENT;
+    if (N < 0 || H < 1 || K < 1 || V < 1) return SGLA_ERR_INVALID_ARGUMENT;
+    if (dtype != SGLA_BF16 && dtype != SGLA_FP32) return SGLA_ERR_INVALID_ARGUMENT;
+    if (K > 1024 || V > 512 || V % 4) return SGLA_ERR_UNSUPPORTED;
+    if (N * H >= kMaxTokens) return SGLA_ERR_UNSUPPORTED;
+    if (N == 0) return SGLA_OK;
+    if (!q || !k || !v || !o || !state) return SGLA_ERR_INVALID_ARGUMENT;
+    for (const void *p : {q, k, v, (const void *)o, (const void *)state})
+        if (!aligned(p, 16)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!aligned(g, 4) || !aligned(g_gamma, 4)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!(scale > 0.f) || isnan(scale) || isinf(scale)) scale = 1.0f / sqrtf((float)K);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    SGLA_LAUNCH("decode_step", launch_decode_step(q, k, v, g, g_gamma, scale, state, o, N, (int)H, (int)K,
+                                                  (int)V, dtype == SGLA_BF16, st));
+    return SGLA_OK;
+}
+
+sgla_status sgla_workspace_status(const void *workspace, int *device_status, void *stream) {
+    if (!workspace || !device_status) return SGLA_ERR_INVALID_ARGUMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int host = -1;
+    SGLA_CUDA(cudaMemcpyAsync(&host, workspace, sizeof(int), cudaMemcpyDeviceToHost, st), "status read");
+    SGLA_CUDA(cudaStreamSynchronize(st), "status sync");
+    *device_status = host;
+    return SGLA_OK;
+}
+
+uint64_t sgla_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+sgla_status sgla_profile_begin(void) {
+    for (auto &r : g_prof) {
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    g_prof.clear();
+    g_prof_on = true;
+    return SGLA_OK;
+}
+
+sgla_status sgla_profile_end(char *names, int *launches, double *total_ms, int max_kernels, int *n_kernels) {
+    g_prof_on = false;
+    if (!names || !launches || !total_ms || !n_kernels || max_kernels < 0) return SGLA_ERR_INVALID_ARGUMENT;
+    int n = 0;
+    sgla_status status = SGLA_OK;
+    for (auto &r : g_prof) {
+        float ms = 0.f;
+        cudaError_t e = cudaEventSynchronize(r.b);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+        if (e != cudaSuccess) status = cuda_fail(e, "profile read");
+        int i = 0;
+        while (i < n && strncmp(names + 64 * i, r.name, 63) != 0) ++i;
+        if (i == n) {
+            if (n == max_kernels) continue;
+            strncpy(names + 64 * i, r.name, 63);
+            names[64 * i + 63] = 0;
+            launches[i] = 0;
+            total_ms[i] = 0.0;
+            ++n;
+        }
+        launches[i] += 1;
+        total_ms[i] += ms;
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    g_prof.clear();
+    *n_kernels = n;
+    return status;
+}
+
+}  // extern "C"

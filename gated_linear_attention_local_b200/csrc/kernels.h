@@ -1,0 +1,47 @@
+// Host-side launchers of the device kernels (internal to libsimplegla.so).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace sgla {
+
+struct FwdArgs {
+    const void *q, *k, *v;
+    const float *g, *g_gamma;
+    float scale;
+    const float *h0;
+    void *o;
+    float *hT;
+    int H, K, V;
+    int gate_mode;
+    bool bf16;
+    // workspace carve-up
+    float *gcum;     // [tokens, H] chunk-local cumsum of g in log2 units (per-token gates)
+    float *seg_dec;  // [max_segs, H] log2 total decay of each segment
+    float *seg_state;// [max_segs, H, K, V] segment states (local end state, then entering state)
+    SeqLayout lay;
+};
+
+// Plan for packed batches: validate cu_seqlens, fill chunk_off / seg_off, set status.
+cudaError_t launch_varlen_plan(const int64_t *cu, int N, int64_t T_total, int C, int L,
+                               int *chunk_off, int *seg_off, int *status, cudaStream_t st);
+
+// Chunk-local inclusive cumsum of g times 1/ln2 (warp-shuffle scan).
+cudaError_t launch_chunk_cumsum(const float *g, float *gcum, const SeqLayout &lay, cudaStream_t st);
+
+// Scalar-decay carry across segments (also writes final states of empty sequences).
+cudaError_t launch_segment_carry(const FwdArgs &a, bool need_carry, cudaStream_t st);
+
+// SIMT (fp32 FFMA) chunk path: segment states and the fused output walk.
+cudaError_t launch_segment_state_simt(const FwdArgs &a, cudaStream_t st);
+cudaError_t launch_chunk_output_simt(const FwdArgs &a, cudaStream_t st);
+
+// Recurrent decode step.
+cudaError_t launch_decode_step(const void *q, const void *k, const void *v, const float *g,
+                               const float *g_gamma, float scale, float *state, void *o,
+                               int64_t N, int H, int K, int V, bool bf16, cudaStream_t st);
+
+}  // namespace sgla

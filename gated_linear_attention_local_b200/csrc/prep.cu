@@ -1,0 +1,199 @@
+// Planning, chunk-local gate cumsum and the cross-segment state carry.
+//
+// "Simple GLA in flash-linear-attention: maths and kernels" (xxqk.cn article),
+// section 3, step 1: the per-head scalar gate is cumulated inside each chunk and
+// multiplied by 1/ln2, so later kernels evaluate decays with exp2.  Because the
+// gate is one scalar per head this is a 1-D scan per (chunk, head) -- here one
+// warp-shuffle scan per column of a [chunk x 32 heads] tile.
+#include "kernels.h"
+
+namespace sgla {
+
+// ---------------------------------------------------------------------------
+// varlen plan: one block.  Validates cu_seqlens and writes exclusive prefix sums
+// of chunks and segments per sequence.  On a malformed cu_seqlens every offset is
+// zero (so no kernel finds work) and the status word records the failure.
+// ---------------------------------------------------------------------------
+constexpr int kPlanThreads = 1024;
+
+__device__ __forceinline__ int block_exclusive_scan(int x, int &total, int *warp_sums) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = x;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = (lane < (int)(blockDim.x >> 5)) ? warp_sums[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, wi, off);
+            if (lane >= off) wi += y;
+        }
+        warp_sums[lane] = wi - w;  // exclusive prefix of warp totals
+        if (lane == 31) warp_sums[32] = wi;
+    }
+    __syncthreads();
+    const int excl = warp_sums[warp] + incl - x;
+    total = warp_sums[32];
+    __syncthreads();
+    return excl;
+}
+
+__global__ void __launch_bounds__(kPlanThreads)
+varlen_plan_kernel(const int64_t *__restrict__ cu, int N, int64_t T_total, int C, int L,
+                   int *__restrict__ chunk_off, int *__restrict__ seg_off, int *__restrict__ status) {
+    __shared__ int warp_sums[33];
+    __shared__ int bad;
+    if (threadIdx.x == 0) bad = (cu[0] != 0 || cu[N] != T_total) ? 1 : 0;
+    __syncthreads();
+    for (int n = threadIdx.x; n < N; n += blockDim.x)
+        if (cu[n + 1] < cu[n]) bad = 1;
+    __syncthreads();
+    const bool ok = (bad == 0);
+    int run_c = 0, run_s = 0;
+    for (int base = 0; base < N; base += blockDim.x) {
+        const int n = base + threadIdx.x;
+        int nc = 0, ns = 0;
+        if (ok && n < N) {
+            const int64_t len = cu[n + 1] - cu[n];
+            nc = (int)((len + C - 1) / C);
+            ns = (nc + L - 1) / L;
+        }
+        int tot_c, tot_s;
+        const int ec = block_exclusive_scan(nc, tot_c, warp_sums);
+        const int es = block_exclusive_scan(ns, tot_s, warp_sums);
+        if (n < N) {
+            chunk_off[n] = run_c + ec;
+            seg_off[n] = run_s + es;
+        }
+        run_c += tot_c;
+        run_s += tot_s;
+    }
+    if (threadIdx.x == 0) {
+        chunk_off[N] = run_c;
+        seg_off[N] = run_s;
+        *status = ok ? kDevOk : kDevBadCuSeqlens;
+    }
+}
+
+cudaError_t launch_varlen_plan(const int64_t *cu, int N, int64_t T_total, int C, int L,
+                               int *chunk_off, int *seg_off, int *status, cudaStream_t st) {
+    varlen_plan_kernel<<<1, kPlanThreads, 0, st>>>(cu, N, T_total, C, L, chunk_off, seg_off, status);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// chunk-local cumsum: block = one chunk x 32 heads; 8 warps, 4 heads each.
+// ---------------------------------------------------------------------------
+constexpr int kCumsumMaxC = 128;
+
+__global__ void __launch_bounds__(256)
+chunk_cumsum_kernel(const float *__restrict__ g, float *__restrict__ gcum, SeqLayout lay) {
+    __shared__ float tile[kCumsumMaxC][33];
+    if (device_failed(lay)) return;
+    int n, c;
+    if (!locate_chunk(lay, blockIdx.x, n, c)) return;
+    int64_t t0, t1;
+    seq_span(lay, n, t0, t1);
+    const int64_t ta = t0 + (int64_t)c * lay.C;
+    const int len = (int)min64(lay.C, t1 - ta);
+    const int H = lay.H, h0 = blockIdx.y * 32;
+    const int hw = min(32, H - h0);
+    // coalesced load: each row of 32 heads is contiguous
+    for (int e = threadIdx.x; e < len * 32; e += blockDim.x) {
+        const int i = e >> 5, j = e & 31;
+        tile[i][j] = (j < hw) ? fmaxf(g[(ta + i) * H + h0 + j], kMinLogGate) : 0.f;
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int R = max(1, lay.C >> 5);  // elements per lane (contiguous run)
+    for (int j = warp; j < hw; j += 8) {
+        float vals[kCumsumMaxC / 32];
+        float run = 0.f;
+#pragma unroll
+        for (int r = 0; r < kCumsumMaxC / 32; ++r) {
+            if (r < R) {
+                const int i = lane * R + r;
+                run += (i < len) ? tile[i][j] : 0.f;
+                vals[r] = run;
+            }
+        }
+        float incl = run;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        const float excl = incl - run;
+#pragma unroll
+        for (int r = 0; r < kCumsumMaxC / 32; ++r) {
+            const int i = lane * R + r;
+            if (r < R && i < len) tile[i][j] = (vals[r] + excl) * kRcpLn2;
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < len * 32; e += blockDim.x) {
+        const int i = e >> 5, j = e & 31;
+        if (j < hw) gcum[(ta + i) * H + h0 + j] = tile[i][j];
+    }
+}
+
+cudaError_t launch_chunk_cumsum(const float *g, float *gcum, const SeqLayout &lay, cudaStream_t st) {
+    if (lay.max_chunks == 0) return cudaSuccess;
+    dim3 grid(lay.max_chunks, (lay.H + 31) / 32);
+    chunk_cumsum_kernel<<<grid, 256, 0, st>>>(g, gcum, lay);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Cross-segment carry, one thread per 4 state elements of one (sequence, head).
+// seg_state[u] holds segment u's local end state (from zero) on entry and the
+// state ENTERING segment u+1 on exit; seg_dec[u] is segment u's log2 total decay.
+// Also writes final_state for empty sequences (initial state unchanged).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+segment_carry_kernel(FwdArgs a, bool need_carry) {
+    const SeqLayout &lay = a.lay;
+    if (device_failed(lay)) return;
+    const int n = blockIdx.x, h = blockIdx.y;
+    const int64_t KV = (int64_t)a.K * a.V;
+    const int64_t e = ((int64_t)blockIdx.z * blockDim.x + threadIdx.x) * 4;
+    if (e >= KV) return;
+    const int nseg = seq_segments(lay, n);
+    const int64_t sidx = ((int64_t)n * a.H + h) * KV + e;
+    if (nseg == 0) {
+        if (a.hT) {
+            float4 s0 = a.h0 ? *reinterpret_cast<const float4 *>(a.h0 + sidx) : make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4 *>(a.hT + sidx) = s0;
+        }
+        return;
+    }
+    if (!need_carry || nseg == 1) return;
+    const int first = seq_first_segment(lay, n);
+    float4 S = a.h0 ? *reinterpret_cast<const float4 *>(a.h0 + sidx) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s + 1 < nseg; ++s) {
+        const int64_t u = first + s;
+        float4 *slot = reinterpret_cast<float4 *>(a.seg_state + (u * a.H + h) * KV + e);
+        const float4 d = *slot;
+        const float dec = exp2f(a.seg_dec[u * a.H + h]);
+        S.x = fmaf(dec, S.x, d.x);
+        S.y = fmaf(dec, S.y, d.y);
+        S.z = fmaf(dec, S.z, d.z);
+        S.w = fmaf(dec, S.w, d.w);
+        *slot = S;
+    }
+}
+
+cudaError_t launch_segment_carry(const FwdArgs &a, bool need_carry, cudaStream_t st) {
+    const int64_t KV = (int64_t)a.K * a.V;
+    dim3 grid(a.lay.N, a.H, (unsigned)((KV / 4 + 255) / 256));
+    segment_carry_kernel<<<grid, 256, 0, st>>>(a, need_carry);
+    return cudaGetLastError();
+}
+
+}  // namespace sgla

@@ -1,0 +1,208 @@
+/*
+ * simple_gla.h -- C ABI of the B200 (sm_100a) Simple GLA library, libsimplegla.so.
+ *
+ * The operator is head-wise gated linear attention ("Simple GLA"), as stated in
+ * "Simple GLA in flash-linear-attention: maths and kernels" (xxqk.cn article):
+ *
+ *   section 1 (definition):  per head, one scalar forget gate per token,
+ *       S_t = exp(g_t) * S_{t-1} + k_t v_t^T          (S is K x V)
+ *       o_t = scale * q_t^T S_t                        (read-out after the update)
+ *   section 2 (API):  q,k [B,T,H,K]; v [B,T,H,V]; g [B,T,H] log-space gates or a
+ *       data-independent per-head log decay g_gamma [H] (at most one of the two);
+ *       scale defaults to 1/sqrt(K); initial/final state [N,H,K,V] with N = B, or
+ *       N = number of sequences when cu_seqlens [N+1] packs variable-length
+ *       sequences into a batch of 1; chunk_size is a power of two (default 64).
+ *   section 3 (chunk kernels):  g is cumulated inside each chunk and pre-scaled by
+ *       1/ln 2 so that the kernels use exp2; an inter-chunk state pass carries S by
+ *       the scalar chunk decay; the output combines q.S_prev with the intra-chunk
+ *       decay-masked q k^T.
+ *   section 2/4 (fused recurrent):  the single-token recurrent step used for
+ *       inference decode.
+ *
+ * Readings where the article is silent: with neither g nor g_gamma the gate is 1
+ * (g == 0); o has the dtype of v; states are fp32 (recurrent storage in fp32 with
+ * bf16 operands, as the NVIDIA ModelOpt linear-attention config page states for
+ * this family); a zero-length sequence returns its initial state.
+ *
+ * Conventions for every entry point
+ *   - All tensors are device pointers to dense, C-contiguous arrays in the layout
+ *     given, 16-byte aligned.  dtype selects the element type of q, k, v, o:
+ *     SGLA_BF16 (bfloat16) or SGLA_FP32.  g, g_gamma, states are always fp32;
+ *     cu_seqlens is int64.
+ *   - The caller owns every buffer.  The library never allocates or frees device
+ *     memory; scratch comes from the caller's workspace (size from the matching
+ *     *_workspace_size query).  Inputs are only read; outputs and the workspace
+ *     are written.  No buffer may alias another, except that a decode state is
+ *     updated in place.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and the call returns without synchronising.  Calls that share a workspace
+ *     must be ordered on the GPU (same stream or explicit events).
+ *   - Errors are status codes; nothing crosses the ABI as an exception.  A call
+ *     that returns an error before any launch has enqueued nothing and written
+ *     nothing.  SGLA_ERR_CUDA means a launch failed; the CUDA error string is
+ *     available from sgla_last_cuda_error().  Problems only visible on the device
+ *     (a malformed cu_seqlens) are recorded in the workspace and read back with
+ *     sgla_workspace_status(); the kernels then write no outputs.
+ *   - Not thread-safe with respect to sgla_last_cuda_error() only; everything else
+ *     is reentrant.
+ */
+#ifndef SIMPLE_GLA_H
+#define SIMPLE_GLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SGLA_API __attribute__((visibility("default")))
+#else
+#define SGLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SGLA_OK = 0,
+    SGLA_ERR_INVALID_ARGUMENT = 1, /* shape/pointer/alignment/exclusivity violation (the
+                                      article's ValueError cases among them) */
+    SGLA_ERR_UNSUPPORTED = 2,      /* well-formed but outside what the kernels handle */
+    SGLA_ERR_CUDA = 3,             /* a CUDA runtime call or launch failed */
+    SGLA_ERR_WORKSPACE = 4,        /* workspace NULL or smaller than the query returned */
+    SGLA_ERR_DEVICE_CHECK = 5      /* device-side validation failed (see sgla_workspace_status) */
+} sgla_status;
+
+typedef enum { SGLA_BF16 = 0, SGLA_FP32 = 1 } sgla_dtype;
+
+/* Device-side status words, as returned by sgla_workspace_status(). */
+#define SGLA_DEVICE_OK 0
+#define SGLA_DEVICE_BAD_CU_SEQLENS 1 /* cu_seqlens[0] != 0, decreasing, or cu[N] != T_total */
+
+/* Library version: major*10000 + minor*100 + patch. */
+SGLA_API int sgla_version(void);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+SGLA_API const char *sgla_status_string(int status);
+
+/* Message of the last CUDA error seen by this library in the calling process
+ * (static storage; "" if none). */
+SGLA_API const char *sgla_last_cuda_error(void);
+
+/*
+ * Workspace bytes needed by simple_gla_fwd for these sizes (0 if the sizes are
+ * invalid).  The value depends only on the arguments, so it may be cached.
+ */
+SGLA_API size_t simple_gla_fwd_workspace_size(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                                     int chunk_size, sgla_dtype dtype);
+
+/*
+ * Workspace bytes needed by simple_gla_fwd_varlen for N packed sequences of
+ * T_total tokens in all (an upper bound over every way of splitting T_total into
+ * N lengths, so it needs no access to cu_seqlens).
+ */
+SGLA_API size_t simple_gla_fwd_varlen_workspace_size(int64_t N, int64_t T_total, int64_t H, int64_t K,
+                                            int64_t V, int chunk_size, sgla_dtype dtype);
+
+/*
+ * Chunked Simple GLA forward over a dense batch (article sections 1-3; the
+ * chunk_simple_gla entry point of section 2).
+ *
+ *   q, k           [B,T,H,K]  dtype     queries, keys
+ *   v              [B,T,H,V]  dtype     values
+ *   g              [B,T,H]    fp32      log-space forget gates (e.g. logsigmoid
+ *                                       outputs), or NULL
+ *   g_gamma        [H]        fp32      per-head log decay, or NULL; g and g_gamma
+ *                                       both non-NULL -> SGLA_ERR_INVALID_ARGUMENT;
+ *                                       both NULL -> no decay
+ *   scale                              read-out scale; NaN or <= 0 selects 1/sqrt(K)
+ *   initial_state  [B,H,K,V]  fp32      or NULL (zeros)
+ *   o              [B,T,H,V]  dtype     output (written)
+ *   final_state    [B,H,K,V]  fp32      or NULL (not written): S after token T-1
+ *   chunk_size                          power of two; 16, 32, 64 or 128 are built,
+ *                                       other powers of two -> SGLA_ERR_UNSUPPORTED,
+ *                                       non-powers of two -> SGLA_ERR_INVALID_ARGUMENT.
+ *                                       It changes rounding only, never the result.
+ *   workspace      device scratch of at least simple_gla_fwd_workspace_size() bytes,
+ *                  256-byte aligned; its contents on entry do not matter.
+ *   stream         cudaStream_t
+ * Supported sizes: 1 <= K, V <= 512, both multiples of 8; H >= 1; B, T >= 0
+ * (B*T == 0 writes only final_state = initial_state).
+ */
+SGLA_API sgla_status simple_gla_fwd(const void *q, const void *k, const void *v,
+                           const float *g, const float *g_gamma, float scale,
+                           const float *initial_state, void *o, float *final_state,
+                           int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                           int chunk_size, sgla_dtype dtype,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Chunked Simple GLA forward over N variable-length sequences packed along the
+ * token axis (article section 2: cu_seqlens follows the FlashAttention
+ * convention, the batch dimension is 1, and initial_state holds one state per
+ * sequence).  Sequence n covers tokens cu_seqlens[n] .. cu_seqlens[n+1]-1; chunks
+ * never straddle two sequences.
+ *
+ *   q, k [T_total,H,K], v, o [T_total,H,V] (a batch of 1 with the leading 1 dropped),
+ *   g [T_total,H] or NULL, g_gamma [H] or NULL, initial_state / final_state
+ *   [N,H,K,V] fp32 or NULL, cu_seqlens: DEVICE pointer to N+1 int64, non-decreasing,
+ *   cu_seqlens[0] == 0 and cu_seqlens[N] == T_total.  A cu_seqlens that breaks this
+ *   is detected on the device: no output is written and sgla_workspace_status()
+ *   reports SGLA_DEVICE_BAD_CU_SEQLENS.  N >= 1.  Other arguments as simple_gla_fwd.
+ */
+SGLA_API sgla_status simple_gla_fwd_varlen(const void *q, const void *k, const void *v,
+                                  const float *g, const float *g_gamma, float scale,
+                                  const int64_t *cu_seqlens, int64_t N, int64_t T_total,
+                                  const float *initial_state, void *o, float *final_state,
+                                  int64_t H, int64_t K, int64_t V, int chunk_size,
+                                  sgla_dtype dtype, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/*
+ * One recurrent decode step for N independent sequences (the single-token case of
+ * fused_recurrent_simple_gla, article sections 2 and 4):
+ *   state <- exp(a) * state + k v^T ;  o = scale * state^T q   (post-update state)
+ * with a = g[n,h], or g_gamma[h], or 0.
+ *
+ *   q, k   [N,H,K] dtype;  v, o [N,H,V] dtype;  g [N,H] fp32 or NULL;
+ *   g_gamma [H] fp32 or NULL (not both);  scale as simple_gla_fwd;
+ *   state  [N,H,K,V] fp32, read and updated IN PLACE.
+ * Supported sizes: 1 <= K <= 1024, 1 <= V <= 512 with V a multiple of 4.
+ * No workspace.
+ */
+SGLA_API sgla_status simple_gla_decode_step(const void *q, const void *k, const void *v,
+                                   const float *g, const float *g_gamma, float scale,
+                                   float *state, void *o, int64_t N, int64_t H, int64_t K,
+                                   int64_t V, sgla_dtype dtype, void *stream);
+
+/*
+ * Read the device-side status word of the last forward call that used
+ * `workspace` (SGLA_DEVICE_OK or SGLA_DEVICE_*).  Synchronises `stream`.
+ * Returns SGLA_OK and fills *device_status, or an error status.
+ */
+SGLA_API sgla_status sgla_workspace_status(const void *workspace, int *device_status, void *stream);
+
+/*
+ * Tracing aids (no counterpart in the article; they observe, never change, the
+ * computation).
+ *
+ * sgla_kernel_launch_count: number of kernels this library has launched in the
+ * process so far, over every entry point.
+ *
+ * sgla_profile_begin / sgla_profile_end: while recording is on, every kernel
+ * launch is bracketed by two CUDA events on its stream.  sgla_profile_end stops
+ * recording, waits for the recorded events, and aggregates by kernel name: for
+ * i < *n_kernels, names + 64*i holds a NUL-terminated kernel name, launches[i]
+ * the number of launches and total_ms[i] their summed device time.  At most
+ * max_kernels distinct names are returned.  Recording is process-wide and not
+ * thread-safe; the events are the library's own (created and destroyed inside).
+ */
+SGLA_API uint64_t sgla_kernel_launch_count(void);
+SGLA_API sgla_status sgla_profile_begin(void);
+SGLA_API sgla_status sgla_profile_end(char *names, int *launches, double *total_ms, int max_kernels,
+                                      int *n_kernels);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SIMPLE_GLA_H */

@@ -1,0 +1,118 @@
+"""C ABI checks that need no GPU: the library loads, exports every entry point the
+header declares, sizes its workspace, and rejects invalid calls before touching
+the device (no kernel is launched by any call in this file)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from gated_linear_attention_local_b200 import _lib as L
+from gated_linear_attention_local_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "simple_gla.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w \*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "defined")))
+
+
+def test_header_declares_the_three_entry_points():
+    names = declared_functions()
+    for n in ("simple_gla_fwd", "simple_gla_fwd_varlen", "simple_gla_decode_step"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", L.library_path], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if " T " in line)
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    assert set(declared_functions()) == set(L._SIG), "binding signatures out of sync with the header"
+
+
+def test_status_strings(lib):
+    assert lib.sgla_status_string(0) == b"SGLA_OK"
+    assert lib.sgla_status_string(1) == b"SGLA_ERR_INVALID_ARGUMENT"
+    assert lib.sgla_status_string(99) == b"SGLA_UNKNOWN_STATUS"
+    assert lib.sgla_version() >= 100
+
+
+def test_workspace_sizes(lib):
+    ws = lib.simple_gla_fwd_workspace_size
+    assert ws(4, 2048, 4, 512, 512, 64, L.SGLA_BF16) > 0
+    assert ws(1, 256, 2, 64, 64, 64, L.SGLA_FP32) % 256 == 0
+    assert ws(1, 256, 2, 64, 64, 48, L.SGLA_FP32) == 0      # not a power of two
+    assert ws(1, 256, 2, 64, 64, 256, L.SGLA_FP32) == 0     # power of two, not built
+    assert ws(1, 256, 2, 1024, 64, 64, L.SGLA_FP32) == 0    # K too large
+    # the varlen bound does not depend on how T_total splits
+    vs = lib.simple_gla_fwd_varlen_workspace_size
+    assert vs(8, 18062, 16, 128, 128, 64, L.SGLA_BF16) >= ws(1, 18062, 16, 128, 128, 64, L.SGLA_BF16)
+    assert vs(0, 100, 16, 128, 128, 64, L.SGLA_BF16) == 0
+
+
+FAKE = 1 << 20  # an aligned non-NULL address: every call below must return before using it
+
+
+def _fwd(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=None, g_gamma=None, scale=float("nan"), h0=None, o=FAKE, hT=None,
+             B=1, T=64, H=2, K=64, V=64, C=64, dtype=L.SGLA_BF16, ws=FAKE, wsb=1 << 30, stream=None)
+    a.update(kw)
+    return lib.simple_gla_fwd(a["q"], a["k"], a["v"], a["g"], a["g_gamma"], a["scale"], a["h0"], a["o"],
+                              a["hT"], a["B"], a["T"], a["H"], a["K"], a["V"], a["C"], a["dtype"], a["ws"],
+                              a["wsb"], a["stream"])
+
+
+def test_invalid_calls_are_rejected_on_the_host(lib):
+    assert _fwd(lib, g=FAKE, g_gamma=FAKE) == L.SGLA_ERR_INVALID_ARGUMENT   # both gates
+    assert _fwd(lib, C=48) == L.SGLA_ERR_INVALID_ARGUMENT                    # not a power of two
+    assert _fwd(lib, C=256) == L.SGLA_ERR_UNSUPPORTED
+    assert _fwd(lib, K=520) == L.SGLA_ERR_UNSUPPORTED
+    assert _fwd(lib, V=60) == L.SGLA_ERR_UNSUPPORTED
+    assert _fwd(lib, q=None) == L.SGLA_ERR_INVALID_ARGUMENT
+    assert _fwd(lib, q=FAKE + 2) == L.SGLA_ERR_INVALID_ARGUMENT             # misaligned
+    assert _fwd(lib, H=0) == L.SGLA_ERR_INVALID_ARGUMENT
+    assert _fwd(lib, B=-1) == L.SGLA_ERR_INVALID_ARGUMENT
+    assert _fwd(lib, dtype=7) == L.SGLA_ERR_INVALID_ARGUMENT
+    assert _fwd(lib, ws=None) == L.SGLA_ERR_WORKSPACE
+    assert _fwd(lib, wsb=16) == L.SGLA_ERR_WORKSPACE
+    assert _fwd(lib, ws=FAKE + 16) == L.SGLA_ERR_INVALID_ARGUMENT           # workspace not 256-aligned
+    r = lib.simple_gla_fwd_varlen(FAKE, FAKE, FAKE, None, None, 1.0, None, 2, 100, None, FAKE, None,
+                                  2, 64, 64, 64, L.SGLA_BF16, FAKE, 1 << 30, None)
+    assert r == L.SGLA_ERR_INVALID_ARGUMENT                                  # cu_seqlens missing
+    r = lib.simple_gla_fwd_varlen(FAKE, FAKE, FAKE, None, None, 1.0, FAKE, 0, 100, None, FAKE, None,
+                                  2, 64, 64, 64, L.SGLA_BF16, FAKE, 1 << 30, None)
+    assert r == L.SGLA_ERR_INVALID_ARGUMENT                                  # N == 0
+    d = lib.simple_gla_decode_step
+    assert d(FAKE, FAKE, FAKE, FAKE, FAKE, 1.0, FAKE, FAKE, 4, 2, 64, 64, 0, None) == L.SGLA_ERR_INVALID_ARGUMENT
+    assert d(FAKE, FAKE, FAKE, None, None, 1.0, FAKE, FAKE, 4, 2, 64, 66, 0, None) == L.SGLA_ERR_UNSUPPORTED
+    assert d(FAKE, FAKE, FAKE, None, None, 1.0, None, FAKE, 4, 2, 64, 64, 0, None) == L.SGLA_ERR_INVALID_ARGUMENT
+
+
+def test_binding_refuses_cpu_tensors():
+    import gated_linear_attention_local_b200 as sg
+    x = torch.zeros(1, 8, 1, 16)
+    with pytest.raises(TypeError):
+        sg.simple_gla_fwd(x, x, x)
+    with pytest.raises(TypeError):
+        sg.simple_gla_decode_step(x[0], x[0], x[0], torch.zeros(1, 8, 16, 16))
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(L, "library_path", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(L, "_lib", None)
+    with pytest.raises(ImportError):
+        L.lib()

@@ -1,0 +1,259 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs, element by element.
+
+Small cases span several chunks and segments plus ragged tails and the edge cases
+of the method (empty and one-token sequences, gate 0 and gate 1, chunk sizes
+16..128, scales and gate normalisers of the article's test matrix, section 5).
+Full-size workloads run in the same launch configuration the bench times and are
+checked on sampled heads / sequences the oracle computes one by one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import gated_linear_attention_local_b200 as sg
+from gated_linear_attention_local_b200.workloads import make_workload, random_inputs
+from parity_utils import TOL, assert_close, host, oracle_fwd, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+
+
+def run_dense(inp, scale=None, final=True, chunk=64):
+    o, ht = sg.simple_gla_fwd(to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"]), g=to_dev(inp["g"]),
+                              g_gamma=to_dev(inp["g_gamma"]), scale=scale, initial_state=to_dev(inp["h0"]),
+                              output_final_state=final, chunk_size=chunk)
+    torch.cuda.synchronize()
+    return host(o), host(ht)
+
+
+def run_varlen(inp, cu, scale=None, final=True, chunk=64):
+    o, ht = sg.simple_gla_fwd_varlen(to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"]), to_dev(cu),
+                                     g=to_dev(inp["g"]), g_gamma=to_dev(inp["g_gamma"]), scale=scale,
+                                     initial_state=to_dev(inp["h0"]), output_final_state=final,
+                                     chunk_size=chunk)
+    torch.cuda.synchronize()
+    return host(o), host(ht)
+
+
+def check(inp, gpu, ref, dtype, what):
+    tol = TOL[dtype]
+    assert_close(gpu[0], ref[0], tol, what + " o")
+    if ref[1] is not None:
+        assert_close(gpu[1], ref[1], tol, what + " final_state")
+
+
+# ----------------------------------------------------------------------------- small dense
+
+DENSE_CASES = [
+    # (B, T, H, K, V, dtype, gate, normalizer, h0, chunk, scale)
+    (1, 256, 2, 64, 64, torch.float32, "g", 1.0, False, 64, 0.125),
+    (2, 300, 3, 64, 64, torch.float32, "g", 1.0, True, 64, None),
+    (1, 1, 2, 64, 32, torch.float32, "g", 1.0, True, 64, None),
+    (1, 17, 1, 32, 64, torch.float32, "gamma", 1.0, True, 16, 1.0),
+    (2, 100, 2, 128, 128, torch.bfloat16, "g", 1.0, True, 64, None),
+    (1, 513, 2, 128, 128, torch.bfloat16, "g", 0.1, True, 64, 0.1),
+    (1, 200, 2, 128, 128, torch.bfloat16, "g", 10.0, False, 64, 1.0),
+    (1, 333, 4, 64, 128, torch.bfloat16, "gamma", 1.0, True, 64, None),
+    (1, 130, 2, 128, 64, torch.bfloat16, "none", 1.0, True, 64, None),
+    (1, 90, 2, 64, 64, torch.bfloat16, "zero", 1.0, False, 32, None),
+    (1, 77, 2, 64, 64, torch.float32, "neg_inf", 1.0, True, 64, 1.0),
+    (1, 250, 2, 40, 24, torch.float32, "g", 1.0, True, 128, None),
+    (2, 129, 2, 256, 256, torch.bfloat16, "g", 1.0, True, 64, None),
+    (1, 200, 1, 512, 512, torch.bfloat16, "g", 1.0, True, 64, None),
+]
+
+
+@pytest.mark.parametrize("case", DENSE_CASES, ids=lambda c: f"B{c[0]}T{c[1]}H{c[2]}K{c[3]}V{c[4]}-"
+                         f"{str(c[5])[6:]}-{c[6]}{c[7]}-h0{int(c[8])}-C{c[9]}-s{c[10]}")
+def test_dense_small(case):
+    B, T, H, K, V, dt, gate, norm, h0, chunk, scale = case
+    inp = random_inputs(B, T, H, K, V, dt, gate=gate, normalizer=norm, h0=h0, seed=11)
+    check(inp, run_dense(inp, scale, True, chunk), oracle_fwd(inp, scale), dt, "dense")
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64, 128])
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+def test_chunk_size_only_changes_rounding(chunk, dt):
+    inp = random_inputs(1, 301, 2, 64, 64, dt, gate="g", h0=True, seed=5)
+    check(inp, run_dense(inp, None, True, chunk), oracle_fwd(inp), dt, f"chunk {chunk}")
+
+
+def test_empty_sequence_dense_returns_initial_state():
+    inp = random_inputs(2, 0, 2, 64, 64, torch.bfloat16, gate="g", h0=True, seed=3)
+    o, ht = run_dense(inp)
+    assert o.shape == (2, 0, 2, 64)
+    np.testing.assert_array_equal(ht, inp["h0"].numpy())
+
+
+# ----------------------------------------------------------------------------- varlen
+
+VARLEN_CASES = [
+    ([0, 15, 100, 300, 1200, 2000], torch.bfloat16, "g", True, 64),
+    ([0, 15, 100, 300, 1200, 2000], torch.float32, "g", True, 32),
+    ([0, 0, 5, 5, 70, 200, 201], torch.bfloat16, "g", True, 64),
+    ([0, 64, 128, 129], torch.bfloat16, "gamma", True, 64),
+    ([0, 1000], torch.float32, "none", False, 16),
+]
+
+
+@pytest.mark.parametrize("case", VARLEN_CASES, ids=lambda c: f"n{len(c[0]) - 1}-{str(c[1])[6:]}-{c[2]}-C{c[4]}")
+def test_varlen(case):
+    cu_list, dt, gate, h0, chunk = case
+    cu = torch.tensor(cu_list, dtype=torch.int64)
+    inp = random_inputs(1, cu_list[-1], 3, 64, 128, dt, gate=gate, h0=h0, seed=7, cu_seqlens=cu)
+    check(inp, run_varlen(inp, cu, None, True, chunk), oracle_fwd(inp, cu=cu), dt, "varlen")
+
+
+def test_varlen_equals_separate_calls():
+    cu = torch.tensor([0, 40, 300, 301, 700], dtype=torch.int64)
+    inp = random_inputs(1, 700, 2, 64, 64, torch.bfloat16, gate="g", h0=True, seed=9, cu_seqlens=cu)
+    o, ht = run_varlen(inp, cu)
+    for n in range(4):
+        a, b = int(cu[n]), int(cu[n + 1])
+        part = dict(q=inp["q"][:, a:b], k=inp["k"][:, a:b], v=inp["v"][:, a:b], g=inp["g"][:, a:b],
+                    g_gamma=None, h0=inp["h0"][n:n + 1].contiguous())
+        on, hn = run_dense({k_: (v_.contiguous() if v_ is not None else None) for k_, v_ in part.items()})
+        assert_close(o[:, a:b], on, 1e-5, f"seq {n} o")
+        assert_close(ht[n:n + 1], hn, 1e-5, f"seq {n} state")
+
+
+def test_bad_cu_seqlens_is_reported_on_the_device():
+    cu = torch.tensor([0, 50, 40, 100], dtype=torch.int64)  # decreasing
+    inp = random_inputs(1, 100, 2, 64, 64, torch.bfloat16, gate="g", seed=1)
+    q, k, v, g = (to_dev(inp[x]) for x in ("q", "k", "v", "g"))
+    nbytes = sg.varlen_workspace_size(3, 100, 2, 64, 64)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    o, _ = sg.simple_gla_fwd_varlen(q, k, v, cu.cuda(), g=g, workspace=ws)
+    assert sg.workspace_status(ws) == 1
+    # a good call on the same workspace clears the status
+    good = torch.tensor([0, 50, 60, 100], dtype=torch.int64, device="cuda")
+    sg.simple_gla_fwd_varlen(q, k, v, good, g=g, workspace=ws)
+    assert sg.workspace_status(ws) == 0
+
+
+def test_initial_state_count_must_match():
+    cu = torch.tensor([0, 10, 20], dtype=torch.int64, device="cuda")
+    x = torch.zeros(1, 20, 2, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        sg.simple_gla_fwd_varlen(x, x, x, cu, initial_state=torch.zeros(3, 2, 64, 64, device="cuda"))
+    with pytest.raises(ValueError):
+        sg.simple_gla_fwd_varlen(torch.zeros(2, 10, 2, 64, dtype=torch.bfloat16, device="cuda"),
+                                 x[:, :10].expand(2, -1, -1, -1).contiguous(),
+                                 x[:, :10].expand(2, -1, -1, -1).contiguous(), cu)
+
+
+def test_split_and_carry_matches_one_call():
+    inp = random_inputs(1, 400, 2, 128, 128, torch.bfloat16, gate="g", h0=True, seed=13)
+    o, ht = run_dense(inp)
+    t1 = 150
+    first = {k_: (v_[:, :t1].contiguous() if k_ in ("q", "k", "v", "g") else v_) for k_, v_ in inp.items()}
+    o1, h1 = run_dense(first)
+    second = {k_: (v_[:, t1:].contiguous() if k_ in ("q", "k", "v", "g") else v_) for k_, v_ in inp.items()}
+    second["h0"] = torch.from_numpy(h1)
+    o2, h2 = run_dense(second)
+    assert_close(np.concatenate([o1, o2], axis=1), o, 2e-2, "split o")
+    assert_close(h2, ht, 2e-2, "split state")
+
+
+# ----------------------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("dt,gate", [(torch.bfloat16, "g"), (torch.float32, "g"), (torch.bfloat16, "gamma"),
+                                     (torch.float32, "none")])
+def test_decode_steps_match_oracle(dt, gate):
+    import oracle
+    N, H, K, V, steps = 5, 3, 64, 128, 20
+    inp = random_inputs(N, steps, H, K, V, dt, gate=gate, h0=True, seed=21)
+    state = to_dev(inp["h0"]).clone()
+    ref_state = inp["h0"].double().numpy().copy()
+    for t in range(steps):
+        q, k, v = (to_dev(inp[x][:, t].contiguous()) for x in ("q", "k", "v"))
+        g = to_dev(inp["g"][:, t].contiguous()) if inp["g"] is not None else None
+        o = sg.simple_gla_decode_step(q, k, v, state, g=g, g_gamma=to_dev(inp["g_gamma"]))
+        ro = oracle.simple_gla_decode_step(inp["q"][:, t], inp["k"][:, t], inp["v"][:, t], ref_state,
+                                           g=None if inp["g"] is None else inp["g"][:, t],
+                                           g_gamma=inp["g_gamma"])
+        assert_close(host(o), ro, TOL[dt], f"step {t} o")
+    assert_close(host(state), ref_state, TOL[dt], "state")
+
+
+def test_decode_equals_forward_on_gpu():
+    inp = random_inputs(3, 64, 2, 128, 128, torch.bfloat16, gate="g", h0=True, seed=4)
+    o_fwd, ht = run_dense(inp)
+    state = to_dev(inp["h0"]).clone()
+    for t in range(64):
+        o = sg.simple_gla_decode_step(*(to_dev(inp[x][:, t].contiguous()) for x in ("q", "k", "v")), state,
+                                      g=to_dev(inp["g"][:, t].contiguous()))
+        assert_close(host(o), o_fwd[:, t], 2e-2, f"step {t}")
+    assert_close(host(state), ht, 2e-2, "state")
+
+
+# ----------------------------------------------------------------------------- full-size workloads
+
+def _heads(inp, hs):
+    out = {}
+    for key in ("q", "k", "v", "g"):
+        out[key] = None if inp[key] is None else inp[key][:, :, hs].contiguous()
+    out["g_gamma"] = None if inp["g_gamma"] is None else inp["g_gamma"][hs].contiguous()
+    out["h0"] = None if inp["h0"] is None else inp["h0"][:, hs].contiguous()
+    return out
+
+
+def _full_size(name, heads, batches=None):
+    w = make_workload(name)
+    if w["kind"] == "varlen":
+        o, ht = run_varlen(w, w["cu_seqlens"], w["scale"], w["output_final_state"], w["chunk_size"])
+    else:
+        o, ht = run_dense(w, w["scale"], w["output_final_state"], w["chunk_size"])
+    sub = _heads(w, heads)
+    if batches is not None:
+        sub = {k_: (None if v_ is None else (v_[batches].contiguous() if k_ != "g_gamma" else v_))
+               for k_, v_ in sub.items()}
+        o, ht = o[batches], (None if ht is None else ht[batches])
+    ro, rht = oracle_fwd(sub, w["scale"], w["output_final_state"], w["cu_seqlens"])
+    assert_close(o[:, :, heads], ro, 2e-2, f"{name} o")
+    if w["output_final_state"]:
+        assert_close(ht[:, heads], rht, 2e-2, f"{name} final_state")
+
+
+def test_workload_tiny_fp32_full():
+    w = make_workload("tiny_fp32")
+    o, ht = run_dense(w, w["scale"], True, 64)
+    ro, rht = oracle_fwd(w, w["scale"])
+    assert_close(o, ro, 1e-4, "o")
+    assert_close(ht, rht, 1e-4, "final_state")
+
+
+def test_workload_dense_prefill_sampled():
+    _full_size("dense_prefill", heads=[0, 3], batches=[0, 3])
+
+
+def test_workload_varlen_prefill_sampled():
+    _full_size("varlen_prefill", heads=[0, 15])
+
+
+def test_workload_long_gamma_sampled():
+    _full_size("long_gamma", heads=[0, 31])
+
+
+def test_workload_decode_sampled():
+    import oracle
+    w = make_workload("decode")
+    state = w["state"].cuda()
+    sel_n, sel_h = [0, 77, 255], [0, 31]
+    ref_state = w["state"][sel_n][:, sel_h].double().numpy().copy()
+    for t in range(w["steps"]):
+        o = sg.simple_gla_decode_step(w["q"][t].cuda(), w["k"][t].cuda(), w["v"][t].cuda(), state,
+                                      g=w["g"][t].cuda())
+        sub = lambda x: x[t][sel_n][:, sel_h]
+        ro = oracle.simple_gla_decode_step(sub(w["q"]), sub(w["k"]), sub(w["v"]), ref_state, g=sub(w["g"]))
+        assert_close(host(o)[sel_n][:, sel_h], ro, 2e-2, f"step {t}")
+    assert_close(host(state)[sel_n][:, sel_h], ref_state, 2e-2, "state")
