@@ -1,0 +1,522 @@
+#!/usr/bin/env python
+"""Benchmark of the Simple GLA forward (and decode step) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
+
+One JSON line on rank 0.  A "step" is one pass of the whole forward hot path --
+plan, chunk cumsum, segment states, carry, fused output walk -- over one batch of
+the named workload (default: dense_prefill, B=4 T=2048 H=4 K=V=512 bf16), with
+inputs resident in HBM.  Each step is timed with CUDA events on the launching
+stream; L2 is flushed (256 MiB write) between steps, outside the events.  The
+other workloads are measured the same way and reported under "secondary".
+
+Multi-GPU (torchrun, one process per GPU): every (sequence, head) is independent,
+so each rank runs its own batch of the workload with no collective on the data
+path (weak scaling); the timed region is bracketed by a barrier and a device
+synchronize, and the step time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only reference this method has:
+the pages ship no implementation) on this machine's host cores, on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Simple GLA fwd tokens/s & % roofline; decode-step state GB/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------- counts
+
+def algorithmic_counts(w):
+    """Compulsory bytes and causal FLOPs of one forward (or one decode step).
+
+    FLOPs per head = 4*T*K*V + T*(C+1)*(K+V): the state update and q.h_prev
+    (2*T*K*V each) plus the causal half of the intra-chunk q k^T and P v.
+    Bytes: q, k, v, g (or g_gamma), o, initial and final state, each moved once."""
+    if w["kind"] == "decode":
+        N, H, K, V = w["N"], w["H"], w["K"], w["V"]
+        e = 2  # bf16 operands
+        state = 2 * N * H * K * V * 4
+        io = N * H * (2 * K + 2 * V) * e + N * H * 4
+        flops = N * H * 4 * K * V
+        return dict(bytes=state + io, flops=flops, tokens=N)
+    H, K, V, C = w["H"], w["K"], w["V"], w["chunk_size"]
+    tokens = w["B"] * w["T"] if w["kind"] == "dense" else w["T"]
+    e = w["q"].element_size()
+    b = tokens * H * (2 * K + 2 * V) * e
+    b += tokens * H * 4 if w["g"] is not None else (H * 4 if w["g_gamma"] is not None else 0)
+    states = w["N"] * H * K * V * 4
+    if w["h0"] is not None:
+        b += states
+    if w["output_final_state"]:
+        b += states
+    flops = H * (4 * tokens * K * V + tokens * (C + 1) * (K + V))
+    return dict(bytes=b, flops=flops, tokens=tokens)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_tflops_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def roofline(w, counts, kernel_ms, peaks, traffic=None):
+    """Roofline object for the dominant kernel of this workload.  The fused output
+    walk (or the decode kernel) moves all compulsory bytes of the call."""
+    t_bytes = counts["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_flops = counts["flops"] / (peaks["bf16_tflops"] * 1e12)
+    if w["kind"] != "decode" and w.get("dtype_name") == "fp32":
+        t_flops = 0.0  # FFMA path: never tensor-bound; report HBM
+    if t_flops > t_bytes:
+        ach = counts["flops"] / (kernel_ms * 1e-3) / 1e12
+        return dict(bound="tensor", achieved=round(ach, 3), peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                    frac=round(ach / peaks["bf16_tflops"], 4), traffic=traffic,
+                    peak_source=peaks["source"])
+    ach = counts["bytes"] / (kernel_ms * 1e-3) / 1e9
+    return dict(bound="hbm", achieved=round(ach, 1), peak=peaks["hbm_gbs"], unit="GB/s",
+                frac=round(ach / peaks["hbm_gbs"], 4), traffic=traffic, peak_source=peaks["source"])
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.lines = []
+        sel = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            pass
+        self.cmd = ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                    "-lms", "100"]
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, pw, reasons = [], None, [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+                pw.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=[], samples=0)
+        # samples under load: power above the midpoint of the observed range
+        lo, hi = min(pw), max(pw)
+        loaded = [s for s, p in zip(sm, pw) if p >= lo + 0.5 * (hi - lo)] or sm
+        return dict(sm_mhz=statistics.median(loaded), sm_max_mhz=mx, reasons=sorted(reasons),
+                    samples=len(sm), power_w_max=hi)
+
+
+# ----------------------------------------------------------------------------- running
+
+def dev_inputs(w, device):
+    keys = ("q", "k", "v", "g", "g_gamma", "h0", "cu_seqlens", "state")
+    return {k: (w[k].to(device) if w.get(k) is not None else None) for k in keys}
+
+
+def make_step(w, d, sg, ws):
+    if w["kind"] == "decode":
+        S = w["steps"]
+        state0 = d["state"].clone()
+        o = torch.empty(w["N"], w["H"], w["V"], dtype=d["q"].dtype, device=d["q"].device)
+
+        def reset():
+            d["state"].copy_(state0)
+
+        def step():
+            for t in range(S):
+                sg.simple_gla_decode_step(d["q"][t], d["k"][t], d["v"][t], d["state"], g=d["g"][t],
+                                          scale=w["scale"], out=o)
+        return step, reset
+    if w["kind"] == "varlen":
+        def step():
+            sg.simple_gla_fwd_varlen(d["q"], d["k"], d["v"], d["cu_seqlens"], g=d["g"], g_gamma=d["g_gamma"],
+                                     scale=w["scale"], initial_state=d["h0"],
+                                     output_final_state=w["output_final_state"], chunk_size=w["chunk_size"],
+                                     workspace=ws)
+    else:
+        def step():
+            sg.simple_gla_fwd(d["q"], d["k"], d["v"], g=d["g"], g_gamma=d["g_gamma"], scale=w["scale"],
+                              initial_state=d["h0"], output_final_state=w["output_final_state"],
+                              chunk_size=w["chunk_size"], workspace=ws)
+    return step, (lambda: None)
+
+
+def workspace_for(w, sg, device):
+    if w["kind"] == "decode":
+        return None
+    dt = w["q"].dtype
+    if w["kind"] == "varlen":
+        n = sg.varlen_workspace_size(w["N"], w["T"], w["H"], w["K"], w["V"], w["chunk_size"], dt)
+    else:
+        n = sg.fwd_workspace_size(w["B"], w["T"], w["H"], w["K"], w["V"], w["chunk_size"], dt)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def time_steps(step, reset, steps, warmup, flush, dist_on, profile=True):
+    from gated_linear_attention_local_b200 import _lib
+    for _ in range(warmup):
+        reset()
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    n0 = _lib.kernel_launch_count()
+    if profile:
+        _lib.profile_begin()
+    for i in range(steps):
+        reset()
+        flush.zero_()
+        evs[i][0].record()
+        step()
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    prof = _lib.profile_end() if profile else {}
+    launches = _lib.kernel_launch_count() - n0
+    if dist_on:
+        torch.distributed.barrier()
+    per_step = [a.elapsed_time(b) for a, b in evs]
+    return per_step, prof, launches
+
+
+def dominant(prof):
+    if not prof:
+        return None, 0, 0.0
+    name = max(prof, key=lambda k: prof[k][1])
+    n, ms = prof[name]
+    return name, n, ms
+
+
+def e2e_measure(w, sg, device, steps, warmup):
+    """Same metric through the public API with inputs in pinned HOST memory: every
+    step copies the inputs host->device, runs the call and reads the result back."""
+    keys = [k for k in ("q", "k", "v", "g", "h0", "cu_seqlens") if w.get(k) is not None]
+    if w["kind"] == "decode":
+        keys = ["q", "k", "v", "g", "state"]
+    hostin = {k: w[k].pin_memory() for k in keys}
+    h2d = sum(t.numel() * t.element_size() for t in hostin.values())
+    g_gamma = w["g_gamma"].to(device) if w.get("g_gamma") is not None else None
+    ws = workspace_for(w, sg, device)
+    if w["kind"] == "decode":
+        out_host = torch.empty(w["steps"], w["N"], w["H"], w["V"], dtype=w["q"].dtype).pin_memory()
+        st_host = torch.empty_like(w["state"]).pin_memory()
+        d2h = out_host.numel() * out_host.element_size() + st_host.numel() * 4
+    else:
+        tokens_shape = (w["B"], w["T"]) if w["kind"] == "dense" else (w["T"],)
+        out_host = torch.empty(*tokens_shape, w["H"], w["V"], dtype=w["q"].dtype).pin_memory()
+        st_host = torch.empty(w["N"], w["H"], w["K"], w["V"]).pin_memory() if w["output_final_state"] else None
+        d2h = out_host.numel() * out_host.element_size() + (st_host.numel() * 4 if st_host is not None else 0)
+
+    def one():
+        d = {k: v.to(device, non_blocking=True) for k, v in hostin.items()}
+        if w["kind"] == "decode":
+            for t in range(w["steps"]):
+                o = sg.simple_gla_decode_step(d["q"][t], d["k"][t], d["v"][t], d["state"], g=d["g"][t],
+                                              scale=w["scale"])
+                out_host[t].copy_(o, non_blocking=True)
+            st_host.copy_(d["state"], non_blocking=True)
+            return
+        if w["kind"] == "varlen":
+            o, ht = sg.simple_gla_fwd_varlen(d["q"][0], d["k"][0], d["v"][0], d["cu_seqlens"], g=d["g"][0],
+                                             g_gamma=g_gamma, scale=w["scale"], initial_state=d.get("h0"),
+                                             output_final_state=w["output_final_state"],
+                                             chunk_size=w["chunk_size"], workspace=ws)
+        else:
+            o, ht = sg.simple_gla_fwd(d["q"], d["k"], d["v"], g=d.get("g"), g_gamma=g_gamma, scale=w["scale"],
+                                      initial_state=d.get("h0"), output_final_state=w["output_final_state"],
+                                      chunk_size=w["chunk_size"], workspace=ws)
+        out_host.copy_(o, non_blocking=True)
+        if st_host is not None:
+            st_host.copy_(ht, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps, h2d, d2h
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+
+def oracle_sample(w, budget_s=12.0):
+    """Time the fp64 oracle on a bounded sample of the workload: all heads and
+    sequences, a prefix of the tokens (decode: a subset of the sequences), sized
+    from a short calibration run to take about budget_s seconds."""
+    import oracle
+    threads = oracle.default_threads()
+    if w["kind"] == "decode":
+        def run(nseq):
+            st = w["state"][:nseq].double().numpy().copy()
+            t0 = time.perf_counter()
+            for t in range(w["steps"]):
+                oracle.simple_gla_decode_step(w["q"][t, :nseq], w["k"][t, :nseq], w["v"][t, :nseq], st,
+                                              g=w["g"][t, :nseq], scale=w["scale"], threads=threads)
+            return time.perf_counter() - t0
+        cal = run(4)
+        nseq = int(max(4, min(w["N"], 4 * budget_s / max(cal, 1e-6))))
+        dt = run(nseq)
+        # unit: state GB/s over the sampled sequences, all steps
+        gb = w["steps"] * 2 * nseq * w["H"] * w["K"] * w["V"] * 4 / 1e9
+        return dict(value=gb / dt, unit="GB/s", cores=threads, kind="oracle",
+                    sample=f"{nseq} of {w['N']} sequences x {w['steps']} steps, all heads ({dt:.1f} s)")
+
+    def sub(tn):
+        d = {}
+        if w["kind"] == "varlen":
+            cu = w["cu_seqlens"]
+            lens = torch.clamp(cu[1:] - cu[:-1], max=tn)
+            idx = torch.cat([torch.arange(int(cu[n]), int(cu[n]) + int(lens[n])) for n in range(w["N"])])
+            for k in ("q", "k", "v", "g"):
+                d[k] = None if w[k] is None else w[k][:, idx]
+            d["cu"] = torch.cat([torch.zeros(1, dtype=torch.int64), torch.cumsum(lens, 0)])
+            return d, int(lens.sum())
+        for k in ("q", "k", "v", "g"):
+            d[k] = None if w[k] is None else w[k][:, :tn]
+        d["cu"] = None
+        return d, w["B"] * min(tn, w["T"])
+
+    def run(tn):
+        d, ntok = sub(tn)
+        t0 = time.perf_counter()
+        oracle.simple_gla_fwd(d["q"], d["k"], d["v"], g=d["g"], g_gamma=w["g_gamma"], scale=w["scale"],
+                              initial_state=w["h0"], output_final_state=w["output_final_state"],
+                              cu_seqlens=d["cu"], threads=threads)
+        return time.perf_counter() - t0, ntok
+    cal_t, cal_tok = run(32)
+    per_tok = cal_t / max(cal_tok, 1)
+    max_t = w["T"] if w["kind"] == "dense" else int((w["cu_seqlens"][1:] - w["cu_seqlens"][:-1]).max())
+    full_tokens = w["B"] * w["T"] if w["kind"] == "dense" else w["T"]
+    tn = int(min(max_t, max(32, 32 * budget_s / max(cal_t, 1e-6))))
+    dt, ntok = run(tn)
+    return dict(value=ntok / dt, unit="tokens/s", cores=threads, kind="oracle",
+                sample=f"first {tn} tokens of every sequence ({ntok} of {full_tokens} tokens), all heads, "
+                       f"fp64 naive recurrence ({dt:.1f} s)")
+
+
+# ----------------------------------------------------------------------------- main
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="dense_prefill")
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the other workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args(argv)
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reference_arm(args, world, rank):
+    from gated_linear_attention_local_b200.workloads import make_workload
+    if rank != 0:
+        return None
+    w = make_workload(args.workload, seed=args.seed)
+    budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, budget_s=budget / 4)
+    vals = [oracle_sample(w, budget_s=budget) for _ in range(args.steps)]
+    v = statistics.median(x["value"] for x in vals)
+    unit = vals[0]["unit"]
+    line = dict(metric=METRIC, value=v, unit=unit, n_gpus=world, steps=args.steps, warmup=args.warmup,
+                ms_per_step=None, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
+                data="synthetic (seeded)", impl="reference",
+                config=dict(workload=args.workload, **_config_of(w)),
+                cpu_baseline=dict(value=v, unit=unit, cores=vals[0]["cores"], kind="oracle",
+                                  sample=vals[0]["sample"]),
+                e2e=dict(value=v, unit=unit, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    return line
+
+
+def _config_of(w):
+    if w["kind"] == "decode":
+        return dict(N=w["N"], steps_per_call=w["steps"], H=w["H"], K=w["K"], V=w["V"], state="fp32")
+    c = dict(H=w["H"], K=w["K"], V=w["V"], chunk_size=w["chunk_size"],
+             gate="g" if w["g"] is not None else ("g_gamma" if w["g_gamma"] is not None else "none"))
+    if w["kind"] == "varlen":
+        c.update(N=w["N"], T_total=w["T"], seqlens=[int(x) for x in (w["cu_seqlens"][1:] - w["cu_seqlens"][:-1])])
+    else:
+        c.update(B=w["B"], T=w["T"])
+    return c
+
+
+def measure_workload(name, args, device, world, rank, peaks, steps, warmup, flush, want_e2e, want_cpu):
+    import gated_linear_attention_local_b200 as sg
+    from gated_linear_attention_local_b200.workloads import make_workload
+    w = make_workload(name, seed=args.seed + 1000 * rank)
+    w["dtype_name"] = "fp32" if w["q"].dtype == torch.float32 else "bf16"
+    d = dev_inputs(w, device)
+    ws = workspace_for(w, sg, device)
+    step, reset = make_step(w, d, sg, ws)
+    with ClockSampler(device) as clk:
+        per_step, prof, launches = time_steps(step, reset, steps, warmup, flush, world > 1)
+    total_ms = max_over_ranks(sum(per_step), world, device)
+    ms = total_ms / steps
+    counts = algorithmic_counts(w)
+    kname, kn, kms = dominant(prof)
+    if w["kind"] == "decode":
+        value = world * counts["bytes"] * w["steps"] / (ms * 1e-3) / 1e9
+        unit = "GB/s"
+    else:
+        value = world * counts["tokens"] / (ms * 1e-3)
+        unit = "tokens/s"
+    kernel_ms = kms / max(kn, 1)
+    res = dict(value=value, unit=unit, ms_per_step=ms,
+               ms_p10=sorted(per_step)[len(per_step) // 10], ms_p90=sorted(per_step)[(9 * len(per_step)) // 10],
+               tflops=counts["flops"] * (w["steps"] if w["kind"] == "decode" else 1) / (ms * 1e-3) / 1e12,
+               gbs=counts["bytes"] * (w["steps"] if w["kind"] == "decode" else 1) / (ms * 1e-3) / 1e9,
+               roofline=roofline(w, counts, kernel_ms, peaks) if kname else None,
+               dominant_kernel=dict(name=kname, launches=kn, avg_ms=kernel_ms,
+                                    share=(kms / sum(v[1] for v in prof.values())) if prof else None),
+               kernels={k: dict(launches=v[0], total_ms=round(v[1], 4)) for k, v in prof.items()},
+               gpu_launches=launches, clocks=clk.summary(), config=dict(workload=name, **_config_of(w)),
+               dtype=w["dtype_name"])
+    # whole-call roofline fraction (all kernels, launches included)
+    t_roof = max(counts["bytes"] / (peaks["hbm_gbs"] * 1e9), counts["flops"] / (peaks["bf16_tflops"] * 1e12))
+    res["call_roofline_frac"] = t_roof * (w["steps"] if w["kind"] == "decode" else 1) / (ms * 1e-3)
+    if want_e2e:
+        e_ms, h2d, d2h = e2e_measure(w, sg, device, max(3, steps // 5), 2)
+        e_ms = max_over_ranks(e_ms, world, device)
+        ev = world * (counts["tokens"] / (e_ms * 1e-3) if w["kind"] != "decode"
+                      else counts["bytes"] * w["steps"] / (e_ms * 1e-3) / 1e9)
+        res["e2e"] = dict(value=ev, unit=unit, h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e_ms)
+    if want_cpu and rank == 0 and world == 1:
+        res["cpu_baseline"] = oracle_sample(w)
+    del d, ws
+    return res
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        line = reference_arm(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return 0
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    peaks = load_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    main_res = measure_workload(args.workload, args, device, world, rank, peaks, args.steps, args.warmup, flush,
+                                want_e2e=True, want_cpu=not args.no_cpu_baseline)
+    secondary = {}
+    if not args.no_secondary:
+        from gated_linear_attention_local_b200.workloads import WORKLOADS
+        for name in WORKLOADS:
+            if name == args.workload:
+                continue
+            r = measure_workload(name, args, device, world, rank, peaks, max(5, min(args.steps, 20)),
+                                 max(3, args.warmup), flush, want_e2e=False, want_cpu=False)
+            secondary[name] = {k: r[k] for k in ("value", "unit", "ms_per_step", "tflops", "gbs", "roofline",
+                                                  "call_roofline_frac", "dominant_kernel", "gpu_launches",
+                                                  "clocks", "config")}
+            torch.cuda.empty_cache()
+    if rank == 0:
+        line = dict(metric=METRIC, value=main_res["value"], unit=main_res["unit"], n_gpus=world,
+                    steps=args.steps, warmup=args.warmup, ms_per_step=main_res["ms_per_step"],
+                    higher_is_better=True, scaling="weak", vs_baseline=None, dtype=main_res["dtype"],
+                    data="synthetic: seeded N(0,1) / logsigmoid(N(0,1)) inputs shaped like the pages' workloads",
+                    config=dict(main_res["config"], parallelism=f"dp{world} (independent batches, no collective)",
+                                l2="flushed between steps (256 MiB write outside the per-step events)"),
+                    roofline=main_res["roofline"], call_roofline_frac=main_res["call_roofline_frac"],
+                    cpu_baseline=main_res.get("cpu_baseline"), e2e=main_res["e2e"],
+                    gpu_launches=main_res["gpu_launches"], clocks=main_res["clocks"],
+                    kernels=main_res["kernels"], dominant_kernel=main_res["dominant_kernel"],
+                    ms_p10=main_res["ms_p10"], ms_p90=main_res["ms_p90"], tflops=main_res["tflops"],
+                    gbs=main_res["gbs"], secondary=secondary)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
