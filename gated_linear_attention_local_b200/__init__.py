@@ -30,7 +30,7 @@ import torch
 from ._lib import (SGLA_BF16, SGLA_FP32, SGLA_OK, SglaError, lib, library_path,  # noqa: F401
                    raise_for_status)
 
-__all__ = ["simple_gla_fwd", "simple_gla_fwd_varlen", "simple_gla_decode_step", "chunk_simple_gla",
+__all__ = ["simple_gla_fwd", "simple_gla_fwd_noalloc", "simple_gla_fwd_varlen", "simple_gla_decode_step", "chunk_simple_gla",
            "fwd_workspace_size", "varlen_workspace_size", "workspace_status", "library_path",
            "SglaError"]
 
@@ -117,6 +117,29 @@ def simple_gla_fwd(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None
                               ctypes.c_float(_scale(scale)), _ptr(initial_state), _ptr(o), _ptr(ht),
                               B, T, H, K, V, chunk_size, dt, _ptr(ws), ws.numel(), _stream())
     raise_for_status(st, "simple_gla_fwd")
+    return o, ht
+
+
+def simple_gla_fwd_noalloc(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
+                           output_final_state=False, chunk_size=64):
+    """simple_gla_fwd using the library's built-in 16 MiB scratch instead of a
+    workspace, for callers that must not allocate device memory.  Outputs are
+    still allocated here (a caller that cannot allocate calls the C entry point
+    with its own output buffers).  Calls that may overlap on the GPU race on the
+    shared scratch."""
+    _common_checks(q, k, v, g, g_gamma, initial_state)
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q,k must be [B,T,H,K] and v [B,T,H,V]")
+    B, T, H, K = q.shape
+    V = v.shape[3]
+    if initial_state is not None and tuple(initial_state.shape) != (B, H, K, V):
+        raise ValueError(f"initial_state must be [B,H,K,V] = {(B, H, K, V)}")
+    o = torch.empty((B, T, H, V), dtype=q.dtype, device=q.device)
+    ht = torch.empty((B, H, K, V), dtype=torch.float32, device=q.device) if output_final_state else None
+    st = lib().simple_gla_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma),
+                                      ctypes.c_float(_scale(scale)), _ptr(initial_state), _ptr(o), _ptr(ht),
+                                      B, T, H, K, V, chunk_size, _DTYPES[q.dtype], _stream())
+    raise_for_status(st, "simple_gla_fwd_noalloc")
     return o, ht
 
 

@@ -33,6 +33,8 @@ _SIG = {
                                              ctypes.c_size_t),
     "simple_gla_fwd": ([_P, _P, _P, _P, _P, _F, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int,
                         ctypes.c_int, _P, ctypes.c_size_t, _P], ctypes.c_int),
+    "simple_gla_fwd_noalloc": ([_P, _P, _P, _P, _P, _F, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int,
+                                ctypes.c_int, _P], ctypes.c_int),
     "simple_gla_fwd_varlen": ([_P, _P, _P, _P, _P, _F, _P, _I64, _I64, _P, _P, _P, _I64, _I64, _I64,
                                ctypes.c_int, ctypes.c_int, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "simple_gla_decode_step": ([_P, _P, _P, _P, _P, _F, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_int, _P],

@@ -175,6 +175,26 @@ SGLA_API sgla_status simple_gla_decode_step(const void *q, const void *k, const 
                                    int64_t V, sgla_dtype dtype, void *stream);
 
 /*
+ * simple_gla_fwd without a workspace argument, for callers that may not allocate
+ * device memory (for example a plugin inside a runtime that owns the GPU memory
+ * pool, or a loop that must never pay for an allocation).  The article has no
+ * counterpart: this is a convenience of this library.
+ *
+ * Arguments and results are exactly those of simple_gla_fwd; the scratch comes
+ * from a 16 MiB array inside the library (one per GPU that loads it, held until
+ * the process exits).  Sizes whose simple_gla_fwd_workspace_size() exceeds
+ * 16 MiB return SGLA_ERR_WORKSPACE.  All calls on a device share that array, so
+ * calls that may run at the same time on the GPU race; order them.  The first
+ * call on each device resolves the array's device address (with that device
+ * current) and should come before any stream capture.  Allocates nothing.
+ */
+SGLA_API sgla_status simple_gla_fwd_noalloc(const void *q, const void *k, const void *v,
+                                            const float *g, const float *g_gamma, float scale,
+                                            const float *initial_state, void *o, float *final_state,
+                                            int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                                            int chunk_size, sgla_dtype dtype, void *stream);
+
+/*
  * Read the device-side status word of the last forward call that used
  * `workspace` (SGLA_DEVICE_OK or SGLA_DEVICE_*).  Synchronises `stream`.
  * Returns SGLA_OK and fills *device_status, or an error status.
