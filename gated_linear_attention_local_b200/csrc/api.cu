@@ -105,15 +105,41 @@ Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t 
     if (N < (varlen ? 1 : 0) || T < 0) return p;
     const int64_t tokens = varlen ? T : N * T;
     if (tokens >= kMaxTokens || N >= kMaxTokens) { p.why = SGLA_ERR_UNSUPPORTED; return p; }
-    p.C = C;
     p.tc = tc_path_supports(dtype == SGLA_BF16, (int)K, (int)V, C);
-    const int64_t chunks_est = varlen ? (T + C - 1) / C : N * ((T + C - 1) / C);
-    // Segment length: long enough to keep state round trips rare, short enough that
-    // (segments x heads x V tiles) still fills the 148 SMs a few times over.
-    const int64_t vtiles = p.tc ? tc_path_vtiles((int)K, (int)V) : (V + 31) / 32;
-    const int64_t target_ctas = p.tc ? tc_path_target_ctas() : 4 * 148;
-    int64_t L = std::max<int64_t>(1, (chunks_est * H * vtiles) / target_ctas);
-    if (!varlen) L = std::min<int64_t>(L, std::max<int64_t>(1, (T + C - 1) / C));
+    p.C = p.tc ? tc_path_step() : C;  // the tensor-core kernels step 128 tokens at a time
+    C = p.C;
+    int64_t L;
+    if (p.tc) {
+        // One CTA per (segment, head, V tile), one CTA per SM, each walking its
+        // segment's steps in order; segments other than the last of a sequence also
+        // cost a state pass (about a third of a walk step per step).  Every segment
+        // pays a fixed cost of about two steps (set-up, state in / out, carry).  Pick
+        // the number of segments per sequence that minimises waves x (steps + 2) for
+        // both kernels, with at least 4 steps per segment.
+        const int64_t nt = varlen ? std::max<int64_t>(1, (T / std::max<int64_t>(N, 1) + C - 1) / C)
+                                  : std::max<int64_t>(1, (T + C - 1) / C);
+        const int64_t units = std::max<int64_t>(1, N * H * tc_path_vtiles((int)K, (int)V));
+        double best = 1e300;
+        L = nt;
+        const int64_t min_l = std::min<int64_t>(nt, 4);
+        for (int64_t ns = 1; ns <= std::min<int64_t>(nt, 512); ++ns) {
+            const int64_t l = (nt + ns - 1) / ns, ns_eff = (nt + l - 1) / l;
+            if (l < min_l) break;
+            const double waves_walk = (double)((units * ns_eff + 147) / 148);
+            const double waves_state = (double)((units * (ns_eff - 1) + 147) / 148);
+            const double cost = (waves_walk + 0.35 * waves_state) * (double)(l + 2);
+            if (cost < best - 1e-9) {
+                best = cost;
+                L = l;
+            }
+        }
+    } else {
+        // Segment length: long enough to keep state round trips rare, short enough that
+        // (segments x heads x V tiles) still fills the 148 SMs a few times over.
+        const int64_t chunks_est = varlen ? (T + C - 1) / C : N * ((T + C - 1) / C);
+        L = std::max<int64_t>(1, (chunks_est * H * ((V + 31) / 32)) / (4 * 148));
+        if (!varlen) L = std::min<int64_t>(L, std::max<int64_t>(1, (T + C - 1) / C));
+    }
     L = std::min<int64_t>(L, 1 << 20);
     p.L = (int)L;
     if (varlen) {
@@ -185,6 +211,7 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
     lay.chunk_off = varlen ? reinterpret_cast<int *>(ws + p.off_chunk_off) : nullptr;
     lay.seg_off = varlen ? reinterpret_cast<int *>(ws + p.off_seg_off) : nullptr;
     lay.status = reinterpret_cast<int *>(ws);
+    a.dev_status = reinterpret_cast<int *>(ws);
     lay.T = T; lay.N = (int)N; lay.H = (int)H; lay.C = p.C; lay.L = p.L;
     lay.NT = p.NT; lay.NS = p.NS;
     lay.max_chunks = (int)p.max_chunks; lay.max_segs = (int)p.max_segs;

@@ -35,6 +35,7 @@ enum GateMode : int { kGateNone = 0, kGatePerToken = 1, kGatePerHead = 2 };
 // Device status word at the head of the workspace.
 constexpr int kDevOk = 0;
 constexpr int kDevBadCuSeqlens = 1;
+constexpr int kDevTimeout = 2;  // a bounded wait inside a kernel gave up
 
 template <typename T>
 __device__ __forceinline__ float to_f32(T x);

@@ -22,6 +22,7 @@ struct FwdArgs {
     float *gcum;     // [tokens, H] chunk-local cumsum of g in log2 units (per-token gates)
     float *seg_dec;  // [max_segs, H] log2 total decay of each segment
     float *seg_state;// [max_segs, H, K, V] segment states (local end state, then entering state)
+    int *dev_status; // writable status word (bounded device waits record time-outs here)
     SeqLayout lay;
 };
 

@@ -62,18 +62,43 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete, giving up after a bounded
-// number of polls (each try_wait itself blocks for a short, hardware-chosen time).
-// On give-up (or when another thread already gave up) sets *abort and returns false.
-constexpr uint32_t kMaxPolls = 1u << 22;
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
 
+// Every wait on an mbarrier is bounded in wall time (2 s of %globaltimer; a
+// healthy wait inside these kernels lasts microseconds).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Wait for the phase with the given parity to complete.  Gives up when the time
+// limit passes (then sets *abort) or when another thread of the CTA has already
+// given up (*abort set); returns false in both cases.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
-    for (uint32_t i = 0; i < kMaxPolls; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t start = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 255u && *abort) return false;
+        if ((i & 63u) == 0) {
+            if (*abort) return false;
+            if (globaltimer_ns() - start > kWaitLimitNs) {
+                *abort = 1;
+                return false;
+            }
+        }
     }
-    *abort = 1;
-    return false;
+}
+
+// Bounded wait that ignores the abort flag: used to let in-flight copies and MMAs
+// retire before a CTA that gave up frees its resources.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return;
+    const uint64_t start = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return;
+        if ((i & 63u) == 0 && globaltimer_ns() - start > kWaitLimitNs) return;
+    }
 }
 
 // ---------------------------------------------------------------- TMA

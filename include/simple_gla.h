@@ -77,6 +77,7 @@ typedef enum { SGLA_BF16 = 0, SGLA_FP32 = 1 } sgla_dtype;
 /* Device-side status words, as returned by sgla_workspace_status(). */
 #define SGLA_DEVICE_OK 0
 #define SGLA_DEVICE_BAD_CU_SEQLENS 1 /* cu_seqlens[0] != 0, decreasing, or cu[N] != T_total */
+#define SGLA_DEVICE_TIMEOUT 2        /* a bounded wait inside a kernel gave up; outputs are invalid */
 
 /* Library version: major*10000 + minor*100 + patch. */
 SGLA_API int sgla_version(void);

@@ -257,3 +257,55 @@ def test_workload_decode_sampled():
         ro = oracle.simple_gla_decode_step(sub(w["q"]), sub(w["k"]), sub(w["v"]), ref_state, g=sub(w["g"]))
         assert_close(host(o)[sel_n][:, sel_h], ro, 2e-2, f"step {t}")
     assert_close(host(state)[sel_n][:, sel_h], ref_state, 2e-2, "state")
+
+
+# ----------------------------------------------------------------------------- tensor-core path
+
+TC_CASES = [
+    # (B, T, H, V, gate, h0, chunk)   K = 128, bf16
+    (1, 1, 1, 64, "g", True, 64),
+    (1, 127, 2, 128, "g", True, 64),
+    (1, 128, 2, 128, "gamma", False, 128),
+    (2, 129, 2, 192, "g", True, 64),
+    (1, 300, 3, 512, "g", True, 64),
+    (1, 5000, 1, 64, "g", True, 64),        # many segments: state pass + carry
+    (1, 5000, 1, 128, "gamma", True, 128),
+    (2, 1000, 2, 128, "none", True, 64),
+    (1, 700, 2, 64, "zero", False, 64),
+    (1, 1030, 2, 128, "neg_inf", True, 64),
+]
+
+
+def _ran(kernel_prefix, fn):
+    from gated_linear_attention_local_b200 import _lib
+    _lib.profile_begin()
+    out = fn()
+    torch.cuda.synchronize()
+    prof = _lib.profile_end()
+    assert any(k.startswith(kernel_prefix) for k in prof), f"{kernel_prefix} did not run: {sorted(prof)}"
+    return out
+
+
+@pytest.mark.parametrize("case", TC_CASES, ids=lambda c: f"B{c[0]}T{c[1]}H{c[2]}V{c[3]}-{c[4]}-h0{int(c[5])}-C{c[6]}")
+def test_tensor_core_dense(case):
+    B, T, H, V, gate, h0, chunk = case
+    inp = random_inputs(B, T, H, 128, V, torch.bfloat16, gate=gate, h0=h0, seed=31)
+    gpu = _ran("chunk_output_tc", lambda: run_dense(inp, None, True, chunk))
+    check(inp, gpu, oracle_fwd(inp), torch.bfloat16, "tc dense")
+
+
+@pytest.mark.parametrize("cu_list", [[0, 15, 100, 300, 1200, 2000], [0, 0, 129, 129, 2500, 2501, 6000]])
+def test_tensor_core_varlen(cu_list):
+    cu = torch.tensor(cu_list, dtype=torch.int64)
+    inp = random_inputs(1, cu_list[-1], 4, 128, 128, torch.bfloat16, gate="g", h0=True, seed=41, cu_seqlens=cu)
+    gpu = _ran("chunk_output_tc", lambda: run_varlen(inp, cu))
+    check(inp, gpu, oracle_fwd(inp, cu=cu), torch.bfloat16, "tc varlen")
+
+
+def test_tensor_core_workspace_status_clean():
+    inp = random_inputs(1, 3000, 2, 128, 128, torch.bfloat16, gate="g", h0=True, seed=2)
+    d = {k_: (v_.cuda() if v_ is not None else None) for k_, v_ in inp.items()}
+    ws = torch.empty(sg.fwd_workspace_size(1, 3000, 2, 128, 128), dtype=torch.uint8, device="cuda")
+    sg.simple_gla_fwd(d["q"], d["k"], d["v"], g=d["g"], initial_state=d["h0"], output_final_state=True,
+                      workspace=ws)
+    assert sg.workspace_status(ws) == 0
