@@ -82,7 +82,7 @@ struct Plan {
     int C = 0, L = 1, NT = 0, NS = 0;
     int64_t max_chunks = 0, max_segs = 0;
     bool multi_seg = false;    // some sequence may have more than one segment
-    size_t off_chunk_off = 0, off_seg_off = 0, off_gcum = 0, off_seg_dec = 0, off_seg_state = 0;
+    size_t off_chunk_off = 0, off_seg_off = 0, off_gcum = 0, off_gpos = 0, off_seg_dec = 0, off_seg_state = 0;
     size_t bytes = 0;
 };
 
@@ -164,6 +164,8 @@ Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t 
     if (per_token_gate) {
         p.off_gcum = off;
         off = align_up(off + sizeof(float) * (size_t)tokens * H, 256);
+        p.off_gpos = off;
+        off = align_up(off + sizeof(int) * (size_t)p.max_chunks * H, 256);
     }
     if (p.multi_seg) {
         p.off_seg_dec = off;
@@ -204,6 +206,7 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
     a.gate_mode = g ? kGatePerToken : (g_gamma ? kGatePerHead : kGateNone);
     a.bf16 = dtype == SGLA_BF16;
     a.gcum = per_token ? reinterpret_cast<float *>(ws + p.off_gcum) : nullptr;
+    a.gpos = per_token ? reinterpret_cast<int *>(ws + p.off_gpos) : nullptr;
     a.seg_dec = p.multi_seg ? reinterpret_cast<float *>(ws + p.off_seg_dec) : nullptr;
     a.seg_state = p.multi_seg ? reinterpret_cast<float *>(ws + p.off_seg_state) : nullptr;
     SeqLayout &lay = a.lay;
@@ -224,7 +227,7 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
         SGLA_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), st), "status reset");
     }
     if (N == 0) return SGLA_OK;
-    if (per_token && tokens > 0) SGLA_LAUNCH("chunk_cumsum", launch_chunk_cumsum(g, a.gcum, lay, st));
+    if (per_token && tokens > 0) SGLA_LAUNCH("chunk_cumsum", launch_chunk_cumsum(g, a.gcum, a.gpos, lay, st));
     if (p.multi_seg && p.max_segs > 0) {
         if (p.tc) SGLA_LAUNCH("segment_state_tc", tc_launch_segment_state(a, st));
         else SGLA_LAUNCH("segment_state_simt", launch_segment_state_simt(a, st));

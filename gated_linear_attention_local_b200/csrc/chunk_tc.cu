@@ -34,8 +34,8 @@
 //    a running suffix sum folded into the row weights of V; the product then simply
 //    accumulates in TMEM with no per-step state rescaling.
 //
-// Roles inside a CTA: warps 0-3 "epilogue" (thread i owns row / TMEM lane i),
-// warp 4 TMA producer (one thread), warp 5 MMA issuer (one thread).  Every wait on
+// Roles inside a CTA: epilogue warpgroups (thread i owns row / TMEM lane i), one
+// TMA producer thread, one MMA issuer thread.  Every wait on
 // an mbarrier is bounded; a wait that gives up marks the CTA aborted, the CTA
 // drains its in-flight copies and MMAs, frees its TMEM, skips its global writes and
 // records SGLA_DEVICE_TIMEOUT in the workspace status word.
@@ -45,6 +45,25 @@
 
 #include "tc_path.h"
 #include "tc_ptx.cuh"
+
+// Device tracing (off unless built with -DSGLA_DEVICE_TRACE): per-CTA cycle counters
+// of where each role of the walk kernel spends its time, read back with
+// sgla_device_trace_read().  The default build compiles every hook to nothing.
+#ifdef SGLA_DEVICE_TRACE
+__device__ unsigned long long g_sgla_trace[65536][32];
+extern "C" __attribute__((visibility("default"))) int sgla_device_trace_read(unsigned long long *dst, int n) {
+    return (int)cudaMemcpyFromSymbol(dst, g_sgla_trace, sizeof(unsigned long long) * 32 * n);
+}
+#define TR_DECL(v) unsigned long long v = 0
+#define TR_T0(v) const unsigned long long v = clock64()
+#define TR_ACC(acc, v) acc += clock64() - v
+#define TR_STORE(idx, val) g_sgla_trace[(blockIdx.y * gridDim.x + blockIdx.x) & 65535][idx] = (val)
+#else
+#define TR_DECL(v)
+#define TR_T0(v)
+#define TR_ACC(acc, v)
+#define TR_STORE(idx, val)
+#endif
 
 namespace sgla {
 
@@ -60,22 +79,21 @@ constexpr int kThreads = 192;
 
 // ---------------------------------------------------------------- walk kernel smem
 namespace ws {
-constexpr uint32_t Q = 0;                    // per stage: Q (2 regions), K (2), V (1)
-constexpr uint32_t K = 2 * kRegion;
-constexpr uint32_t V = 4 * kRegion;
-constexpr uint32_t STAGE = 5 * kRegion;
-constexpr uint32_t VW = 2 * STAGE;           // weighted V (1 region)
-constexpr uint32_t P = VW + kRegion;         // P (2 regions)
-constexpr uint32_t HB = P + 2 * kRegion;     // bf16 state copy, MN-major (128 k rows x 64 v)
-constexpr uint32_t GS = HB + kRegion;        // gates, 2 x 128 floats
-constexpr uint32_t BARS = GS + 2 * 128 * 4;  // 16 mbarriers
-constexpr uint32_t MISC = BARS + 16 * 8;     // tmem address, abort flag
+constexpr uint32_t QK = 0;                   // Q/K ring, 2 stages: Q (2 regions), K (2 regions)
+constexpr uint32_t QK_STAGE = 4 * kRegion;
+constexpr uint32_t VR = 2 * QK_STAGE;        // V ring, 2 stages of 1 region
+constexpr uint32_t VW = VR + 2 * kRegion;    // weighted V (1 region)
+constexpr uint32_t HB = VW + kRegion;        // bf16 state copy, MN-major (128 k rows x 64 v)
+constexpr uint32_t GS = HB + kRegion;        // gates, column factors, decay table: 3 x 128 floats
+constexpr uint32_t BARS = GS + 3 * 128 * 4;  // 24 mbarriers
+constexpr uint32_t MISC = BARS + 24 * 8;     // tmem address, abort flag
 constexpr uint32_t TOTAL = MISC + 16;
 }  // namespace ws
 constexpr size_t kWalkSmem = ws::TOTAL + 1024;  // + alignment slack
 
-// TMEM columns of the walk kernel
-constexpr uint32_t kColS = 0, kColO1 = 128, kColO2 = 256, kColH = 320, kWalkCols = 512;
+// TMEM columns of the walk kernel: S x2 (128 each; the bf16 P of a step overwrites
+// the first 64 columns of its S buffer), O1 x2 (64 each), O2, H
+constexpr uint32_t kColS = 0, kColO1 = 256, kColO2 = 384, kColH = 448, kWalkCols = 512;
 
 // ---------------------------------------------------------------- state kernel smem
 constexpr int kStateStages = 3;
@@ -102,21 +120,27 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 // Scale the 128-byte row `row` of a swizzled bf16 region by w (the swizzle only
 // permutes 16-byte chunks inside a row, so a whole-row operation ignores it).
+// Thread `row` visits the row's chunks starting at chunk row%8, so the 8 threads of
+// a quarter-warp touch 8 different 16-byte bank groups (rows are 128 B apart, so a
+// common starting chunk would put every thread of the warp on the same 4 banks).
 __device__ __forceinline__ void scale_row(const unsigned char *src, unsigned char *dst, int row, float w) {
     const uint4 *s = reinterpret_cast<const uint4 *>(src + row * 128);
     uint4 *d = reinterpret_cast<uint4 *>(dst + row * 128);
+    uint4 x[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        uint4 x = s[c];
-        uint32_t *xs = reinterpret_cast<uint32_t *>(&x);
+    for (int cc = 0; cc < 8; ++cc) x[cc] = s[(cc + row) & 7];  // every load issued before any store
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+        uint32_t *xs = reinterpret_cast<uint32_t *>(&x[cc]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&xs[e]);
             float2 f = __bfloat1622float2(b);
             xs[e] = pack_bf16(f.x * w, f.y * w);
         }
-        d[c] = x;
     }
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) d[(cc + row) & 7] = x[cc];
 }
 
 // Store 32 fp32 values as bf16 into row `row`, columns [c0, c0+32) (c0 % 32 == 0,
@@ -154,19 +178,27 @@ __device__ __forceinline__ void record_timeout(const FwdArgs &a) {
 // =============================================================================
 // walk kernel (fused output)
 // =============================================================================
-__global__ void __launch_bounds__(kThreads, 1)
+// Warp roles: 0-7 WG_A (P = masked S, then the output rows), 8-11 WG_B (weighted V
+// and the state pass: Hb and the in-place rescale of H, initial / final state),
+// 12 TMA producer, 13 MMA issuer.  S and O1 are double-buffered in TMEM and the MMA
+// issuer runs one step ahead (O1, H and S of step t+1 are issued before P V of
+// step t), so the tensor core keeps working while WG_A masks the previous S.
+constexpr int kWalkThreads = 448;
+
+__global__ void __launch_bounds__(kWalkThreads, 1)
 tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, FwdArgs a) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = align1024(smem_raw);
     const SeqLayout &lay = a.lay;
     if (device_failed(lay)) return;
+    const int VT = a.V / kBV;
+    const int u = blockIdx.x / VT;           // V tiles of one (segment, head) are adjacent
+    const int v0 = (blockIdx.x % VT) * kBV;  // in the launch order, so Q/K are shared in L2
     int n, s;
-    if (!locate_segment(lay, blockIdx.x, n, s)) return;
-    const int u = blockIdx.x;
+    if (!locate_segment(lay, u, n, s)) return;
     const int nseg = seq_segments(lay, n);
     const int h = blockIdx.y, H = a.H, V = a.V;
-    const int v0 = blockIdx.z * kBV;
     int64_t t0, t1;
     seq_span(lay, n, t0, t1);
     const int nt = (int)((t1 - t0 + kStep - 1) / kStep);
@@ -175,28 +207,36 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     const bool last_seg = (s == nseg - 1);
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ws::BARS);
-    uint64_t *full = bars + 0;     // [2] TMA -> consumers
-    uint64_t *empty = bars + 2;    // [2] MMA -> producer
-    uint64_t *b_smma = bars + 4;   // S, O1, H products of a step done
-    uint64_t *b_pv = bars + 5;     // P V product of a step done
-    uint64_t *b_p = bars + 6;      // P written (128 arrivals)
-    uint64_t *b_hb = bars + 7;     // Hb written and H rescaled (128 arrivals)
-    uint64_t *b_vw = bars + 8;     // weighted V written (128 arrivals)
-    uint64_t *b_drain = bars + 9;  // all MMAs retired
+    uint64_t *full_qk = bars + 0;   // [2] Q/K of a step landed
+    uint64_t *empty_qk = bars + 2;  // [2] Q/K stage free (its last reader, K^T Vw, retired)
+    uint64_t *full_v = bars + 4;    // [2] V of a step landed
+    uint64_t *empty_v = bars + 6;   // [2] V stage free (P V retired)
+    uint64_t *b_s = bars + 8;       // [2] S product done, per S buffer
+    uint64_t *b_oh = bars + 10;     // O1 and H products of a step done (Hb, Vw free again)
+    uint64_t *b_pv = bars + 11;     // P V product of a step done
+    uint64_t *b_p = bars + 12;      // P written (WG_A, 256 arrivals)
+    uint64_t *b_hb = bars + 13;     // Hb written and H rescaled (WG_B, 128 arrivals)
+    uint64_t *b_vw = bars + 14;     // weighted V written (WG_B, 128 arrivals)
+    uint64_t *b_ofree = bars + 15;  // O1 / O2 of a step read out (WG_A, 256 arrivals)
+    uint64_t *b_drain = bars + 16;  // all MMAs retired
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + ws::MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + ws::MISC + 8);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(&full[0], 1);
-        mbar_init(&full[1], 1);
-        mbar_init(&empty[0], 1);
-        mbar_init(&empty[1], 1);
-        mbar_init(b_smma, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&full_qk[b], 1);
+            mbar_init(&empty_qk[b], 1);
+            mbar_init(&full_v[b], 1);
+            mbar_init(&empty_v[b], 1);
+            mbar_init(&b_s[b], 1);
+        }
+        mbar_init(b_oh, 1);
         mbar_init(b_pv, 1);
-        mbar_init(b_p, 128);
+        mbar_init(b_p, 256);
         mbar_init(b_hb, 128);
         mbar_init(b_vw, 128);
+        mbar_init(b_ofree, 256);
         mbar_init(b_drain, 1);
         *abort_flag = 0;
         mbar_fence_init();
@@ -210,8 +250,19 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    auto gate_at = [&](int t, int pos) -> float {  // G~ of position pos of local step t
+        const StepSpan sp = step_span(t0, t1, cb + t);
+        return (pos < sp.len) ? chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + pos, pos, h, H) : 0.f;
+    };
+    auto last_gate = [&](int t) -> float {
+        const StepSpan sp = step_span(t0, t1, cb + t);
+        return chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + sp.len - 1, sp.len - 1, h, H);
+    };
+
+    if (warp == 12) {
         // ------------------------------------------------------------ TMA producer
+        // Q/K of step t reuse the stage of step t-2 once its K^T Vw retired; V of step t
+        // reuses the stage of step t-2 once its P V retired (later), so Q/K go first.
         if (lane == 0) {
             prefetch_tmap(&tq);
             prefetch_tmap(&tk);
@@ -219,92 +270,265 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             int issued = 0;
             for (int t = 0; t < nsteps; ++t) {
                 const int st = t & 1;
-                if (t >= 2 && !mbar_wait(&empty[st], ((t >> 1) - 1) & 1, abort_flag)) break;
                 const int tok = (int)(t0 + (int64_t)(cb + t) * kStep);
-                unsigned char *base = sm + st * ws::STAGE;
-                mbar_arrive_expect_tx(&full[st], 5 * kRegion);
-                tma_load_3d(base + ws::Q, &tq, &full[st], 0, h, tok);
-                tma_load_3d(base + ws::Q + kRegion, &tq, &full[st], 64, h, tok);
-                tma_load_3d(base + ws::K, &tk, &full[st], 0, h, tok);
-                tma_load_3d(base + ws::K + kRegion, &tk, &full[st], 64, h, tok);
-                tma_load_3d(base + ws::V, &tv, &full[st], v0, h, tok);
-                issued = t + 1;
+                if (t >= 2 && !mbar_wait(&empty_qk[st], ((t >> 1) - 1) & 1, abort_flag)) break;
+                unsigned char *qk = sm + ws::QK + st * ws::QK_STAGE;
+                mbar_arrive_expect_tx(&full_qk[st], 4 * kRegion);
+                tma_load_3d(qk, &tq, &full_qk[st], 0, h, tok);
+                tma_load_3d(qk + kRegion, &tq, &full_qk[st], 64, h, tok);
+                tma_load_3d(qk + 2 * kRegion, &tk, &full_qk[st], 0, h, tok);
+                tma_load_3d(qk + 3 * kRegion, &tk, &full_qk[st], 64, h, tok);
+                issued = 2 * t + 1;
+                if (t >= 2 && !mbar_wait(&empty_v[st], ((t >> 1) - 1) & 1, abort_flag)) break;
+                mbar_arrive_expect_tx(&full_v[st], kRegion);
+                tma_load_3d(sm + ws::VR + st * kRegion, &tv, &full_v[st], v0, h, tok);
+                issued = 2 * t + 2;
             }
-            if (*abort_flag)  // let every copy still in flight land before the CTA exits
-                for (int t = max(0, issued - 2); t < issued; ++t) mbar_drain(&full[t & 1], (t >> 1) & 1);
+            if (*abort_flag) {  // let every copy still in flight land before the CTA exits
+                for (int c = max(0, issued - 4); c < issued; ++c) {
+                    const int t = c >> 1;
+                    mbar_drain((c & 1) ? &full_v[t & 1] : &full_qk[t & 1], (t >> 1) & 1);
+                }
+            }
         }
-    } else if (warp == 5) {
+    } else if (warp == 13) {
         // ------------------------------------------------------------ MMA issuer
+        // Issue order per iteration t: S(t+1), O1(t+1), P V(t), H(t+1).  S and O1 of the
+        // next step run while WG_A masks S(t); the V tile of step t+1 (whose stage only
+        // frees when P V(t-1) retires) gets until after P V(t) to land.
         if (lane == 0) {
             const uint32_t idS = idesc_bf16_f32(128, 128, false, false);
             const uint32_t idO = idesc_bf16_f32(128, kBV, false, true);
             const uint32_t idH = idesc_bf16_f32(128, kBV, true, true);
             const uint32_t sbase = smem_u32(sm);
-            for (int t = 0; t < nsteps; ++t) {
-                const int st = t & 1;
-                const uint32_t ph = t & 1;
-                if (!mbar_wait(&full[st], (t >> 1) & 1, abort_flag)) break;
-                if (!mbar_wait(b_hb, ph, abort_flag)) break;
-                if (!mbar_wait(b_vw, ph, abort_flag)) break;
+            auto qk_at = [&](int t) { return sbase + ws::QK + (t & 1) * ws::QK_STAGE; };
+            TR_DECL(m_wqk); TR_DECL(m_whb); TR_DECL(m_wof); TR_DECL(m_wvw); TR_DECL(m_wp); TR_DECL(m_wv);
+            TR_DECL(m_is); TR_DECL(m_io); TR_DECL(m_ih); TR_DECL(m_ipv);
+            TR_T0(m_start);
+            auto do_S = [&](int t) -> bool {  // S = Q K^T (both K-major)
+                { TR_T0(x0); if (!mbar_wait(&full_qk[t & 1], (t >> 1) & 1, abort_flag)) return false; TR_ACC(m_wqk, x0); }
+                TR_T0(x1);
                 tc_fence_after();
-                const uint32_t q = sbase + st * ws::STAGE + ws::Q;
-                const uint32_t k = sbase + st * ws::STAGE + ws::K;
-                const uint32_t v = sbase + st * ws::STAGE + ws::V;
-                // S = Q K^T  (both K-major; K steps of 16 inside 64-wide regions)
+                const uint32_t q = qk_at(t), k = q + 2 * kRegion, sd = tmem + kColS + (t & 1) * 128;
 #pragma unroll
                 for (int kk = 0; kk < kHeadK / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
-                    mma_bf16(tmem + kColS, sdesc_sw128(q + off, 16, 1024), sdesc_sw128(k + off, 16, 1024), idS,
-                             kk > 0);
+                    mma_bf16(sd, sdesc_sw128(q + off, 16, 1024), sdesc_sw128(k + off, 16, 1024), idS, kk > 0);
                 }
-                // O1 = Q Hb  (Hb MN-major: 16 k rows per K step)
-                const uint32_t o1 = tmem + kColO1 + (t & 1) * kBV;
+                mma_commit(&b_s[t & 1]);
+                TR_ACC(m_is, x1);
+                return true;
+            };
+            auto do_O1 = [&](int t) -> bool {  // O1 = Q Hb (Hb MN-major: 16 k rows per K step)
+                { TR_T0(x0); if (!mbar_wait(b_hb, t & 1, abort_flag)) return false; TR_ACC(m_whb, x0); }
+                { TR_T0(x0); if (t >= 2 && !mbar_wait(b_ofree, t & 1, abort_flag)) return false; TR_ACC(m_wof, x0); }
+                TR_T0(x1);
+                tc_fence_after();
+                const uint32_t q = qk_at(t), o1 = tmem + kColO1 + (t & 1) * kBV;
 #pragma unroll
                 for (int kk = 0; kk < kHeadK / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
                     mma_bf16(o1, sdesc_sw128(q + off, 16, 1024),
                              sdesc_sw128(sbase + ws::HB + kk * 2048, 1024, 1024), idO, kk > 0);
                 }
-                // H += K^T Vw  (A = K read MN-major: two 64-wide k groups LBO apart)
+                TR_ACC(m_io, x1);
+                return true;
+            };
+            auto do_H = [&](int t) -> bool {  // H += K^T Vw (A = K read MN-major: two k groups LBO apart)
+                { TR_T0(x0); if (!mbar_wait(b_vw, t & 1, abort_flag)) return false; TR_ACC(m_wvw, x0); }
+                TR_T0(x1);
+                tc_fence_after();
+                const uint32_t k = qk_at(t) + 2 * kRegion;
 #pragma unroll
                 for (int jj = 0; jj < kStep / 16; ++jj)
                     mma_bf16(tmem + kColH, sdesc_sw128(k + jj * 2048, kRegion, 1024),
                              sdesc_sw128(sbase + ws::VW + jj * 2048, 1024, 1024), idH, 1);
-                mma_commit(b_smma);
-                if (!mbar_wait(b_p, ph, abort_flag)) break;
+                mma_commit(b_oh);             // WG_B may rewrite Hb, Vw and H
+                mma_commit(&empty_qk[t & 1]); // Q/K stage free
+                TR_ACC(m_ih, x1);
+                return true;
+            };
+            auto do_PV = [&](int t) -> bool {  // O2 = P V (P from TMEM, V MN-major)
+                { TR_T0(x0); if (!mbar_wait(b_p, t & 1, abort_flag)) return false; TR_ACC(m_wp, x0); }
+                { TR_T0(x0); if (!mbar_wait(&full_v[t & 1], (t >> 1) & 1, abort_flag)) return false; TR_ACC(m_wv, x0); }
+                TR_T0(x1);
                 tc_fence_after();
-                // O2 = P V  (P K-major, V MN-major)
+                const uint32_t v = sbase + ws::VR + (t & 1) * kRegion;
+                const uint32_t pt = tmem + kColS + (t & 1) * 128;
 #pragma unroll
-                for (int jj = 0; jj < kStep / 16; ++jj) {
-                    const uint32_t off = (jj >> 2) * kRegion + (jj & 3) * 32;
-                    mma_bf16(tmem + kColO2, sdesc_sw128(sbase + ws::P + off, 16, 1024),
-                             sdesc_sw128(v + jj * 2048, 1024, 1024), idO, jj > 0);
-                }
+                for (int jj = 0; jj < kStep / 16; ++jj)
+                    mma_bf16_tmem_a(tmem + kColO2, pt + jj * 8, sdesc_sw128(v + jj * 2048, 1024, 1024), idO, jj > 0);
                 mma_commit(b_pv);
-                mma_commit(&empty[st]);
+                mma_commit(&empty_v[t & 1]);
+                TR_ACC(m_ipv, x1);
+                return true;
+            };
+            if (nsteps > 0 && do_S(0) && do_O1(0) && do_H(0)) {
+                for (int t = 0; t < nsteps; ++t) {
+                    const bool more = t + 1 < nsteps;
+                    if (more && !(do_S(t + 1) && do_O1(t + 1))) break;
+                    if (!do_PV(t)) break;
+                    if (more && !do_H(t + 1)) break;
+                }
             }
             mma_commit(b_drain);
             mbar_drain(b_drain, 0);
+            TR_STORE(0, clock64() - m_start); TR_STORE(1, nsteps);
+            TR_STORE(2, m_wqk); TR_STORE(3, m_whb); TR_STORE(4, m_wof); TR_STORE(5, m_wvw); TR_STORE(6, m_wp);
+            TR_STORE(7, m_wv); TR_STORE(8, m_is); TR_STORE(9, m_io); TR_STORE(10, m_ih); TR_STORE(11, m_ipv);
         }
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ WG_A: P and output
+        // Eight warps, two per TMEM sub-partition: warp w owns rows 32(w%4).. and half
+        // w/4 of the work -- S tiles {0,1} or {2,3} of its rows, output columns 0-31 or
+        // 32-63.  P_ij = 2^(G~_i - G~_j) S_ij for j <= i.  For the 32-column tiles strictly
+        // below the diagonal the decay factors as 2^(G~_i - G~_r) * 2^(G~_r - G~_j) with r
+        // the tile's last column: one exp2 per row and tile plus a per-column table f
+        // (both factors <= 1 because G~ does not increase when the log gates are <= 0).
+        // The diagonal tile, and every tile of a step that holds a positive log gate, use
+        // the direct 2^(G~_i - G~_j).  Tiles above the diagonal are zero.
+        const int quarter = warp & 3, half = warp >> 2;
+        const int i = quarter * 32 + lane;  // row of S / O
+        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+        float *gs = reinterpret_cast<float *>(sm + ws::GS);          // [128] gates of the step
+        float *fs = gs + 128;                                         // [128] column factors
+        float *tab = gs + 256;                                        // [128] 2^(d gamma)
+        const bool per_token = a.gate_mode == kGatePerToken;
+        if (!per_token && half == 0) {
+            const float gam = (a.gate_mode == kGatePerHead) ? fmaxf(a.g_gamma[h], kMinLogGate) * kRcpLn2 : 0.f;
+            tab[i] = exp2f((float)i * gam);
+        }
+        const bool gamma_pos = a.gate_mode == kGatePerHead && a.g_gamma[h] > 0.f;
+        const int64_t chunk0 = (lay.cu ? (int64_t)lay.chunk_off[n] : (int64_t)n * lay.NT) + cb;
+        // gate, column factor and "holds a positive gate" flag of local step t for this row
+        auto load_step = [&](int t, float &g_out, float &f_out, bool &pos_out) {
+            const StepSpan sp = step_span(t0, t1, cb + t);
+            g_out = (i < sp.len) ? chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + i, i, h, H) : 0.f;
+            const int r = min((i | 31), sp.len - 1);
+            const float gr = chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + r, r, h, H);
+            f_out = (i < sp.len) ? fast_exp2(fminf(gr - g_out, 0.f)) : 0.f;
+            pos_out = per_token ? (a.gpos[(chunk0 + t) * H + h] != 0) : gamma_pos;
+        };
+        float gi, fi;
+        bool pos;
+        load_step(0, gi, fi, pos);
+        if (half == 0) {
+            gs[i] = gi;
+            fs[i] = fi;
+        }
+        named_sync(1, 256);
+        TR_DECL(a_ws); TR_DECL(a_p); TR_DECL(a_s1); TR_DECL(a_wpv); TR_DECL(a_out); TR_DECL(a_s2);
+        for (int t = 0; t < nsteps; ++t) {
+            const StepSpan sp = step_span(t0, t1, cb + t);
+            float gnext = 0.f, fnext = 0.f;
+            bool posnext = false;
+            if (t + 1 < nsteps) load_step(t + 1, gnext, fnext, posnext);  // in flight during the step
+
+            { TR_T0(x0); mbar_wait(&b_s[t & 1], (t >> 1) & 1, abort_flag); TR_ACC(a_ws, x0); }
+            TR_T0(xp);
+            tc_fence_after();
+            const uint32_t srow = trow + kColS + (t & 1) * 128;
+            // this half's two S tiles -> P (bf16 pairs).  P tile c is written to columns
+            // 16c.. of the same S buffer once both halves have read their S tiles.
+            uint32_t pk[2][16];
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * half + cc;
+                float x[32];
+                if (c < quarter && !pos) {
+                    tmem_ld32(srow + 32 * c, x);
+                    const float gr = gs[min(32 * c + 31, sp.len - 1)];
+                    const float rfac = fast_exp2(fminf(gi - gr, 0.f));
+                    tmem_wait_ld();
+                    const float4 *f4 = reinterpret_cast<const float4 *>(fs + 32 * c);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float4 f = f4[e];
+                        x[4 * e + 0] = (rfac * x[4 * e + 0]) * f.x;
+                        x[4 * e + 1] = (rfac * x[4 * e + 1]) * f.y;
+                        x[4 * e + 2] = (rfac * x[4 * e + 2]) * f.z;
+                        x[4 * e + 3] = (rfac * x[4 * e + 3]) * f.w;
+                    }
+                } else if (c <= quarter) {
+                    tmem_ld32(srow + 32 * c, x);
+                    tmem_wait_ld();
+                    if (!per_token) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int j = 32 * c + e;
+                            x[e] = (j <= i && j < sp.len) ? tab[i - j] * x[e] : 0.f;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int j = 32 * c + e;
+                            x[e] = (j <= i && j < sp.len) ? fast_exp2(gi - gs[j]) * x[e] : 0.f;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[e] = 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < 16; ++e) pk[cc][e] = pack_bf16(x[2 * e], x[2 * e + 1]);
+            }
+            named_sync(1, 256);  // both halves have read their S tiles
+            tmem_st16(srow + 32 * half, pk[0]);
+            tmem_st16(srow + 32 * half + 16, pk[1]);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(b_p);
+            TR_ACC(a_p, xp);
+            { TR_T0(x0); named_sync(1, 256); TR_ACC(a_s1, x0); }  // every row is done with this step's gates and factors
+            if (half == 0) {
+                gs[i] = gnext;
+                fs[i] = fnext;
+            }
+
+            // o = scale (2^G~_i O1 + O2), row i, columns 32*half ..
+            { TR_T0(x0); mbar_wait(b_pv, t & 1, abort_flag); TR_ACC(a_wpv, x0); }
+            TR_T0(xo);
+            tc_fence_after();
+            const float ei = a.scale * fast_exp2(gi);
+            __nv_bfloat16 *orow =
+                static_cast<__nv_bfloat16 *>(a.o) + ((sp.ta + i) * H + h) * (int64_t)V + v0 + 32 * half;
+            {
+                float ox[32], oy[32];
+                tmem_ld32(trow + kColO1 + (t & 1) * kBV + 32 * half, ox);
+                tmem_ld32(trow + kColO2 + 32 * half, oy);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) ox[e] = fmaf(ei, ox[e], a.scale * oy[e]);
+                if (i < sp.len && !*abort_flag) {
+                    uint4 *d = reinterpret_cast<uint4 *>(orow);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        d[q] = make_uint4(pack_bf16(ox[8 * q], ox[8 * q + 1]), pack_bf16(ox[8 * q + 2], ox[8 * q + 3]),
+                                          pack_bf16(ox[8 * q + 4], ox[8 * q + 5]), pack_bf16(ox[8 * q + 6], ox[8 * q + 7]));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(b_ofree);
+            TR_ACC(a_out, xo);
+            { TR_T0(x0); named_sync(1, 256); TR_ACC(a_s2, x0); }  // next step's gates and factors are in place
+            gi = gnext;
+            pos = posnext;
+        }
+        if (threadIdx.x == 96) { TR_STORE(12, a_ws); TR_STORE(13, a_p); TR_STORE(14, a_s1); TR_STORE(15, a_wpv); TR_STORE(16, a_out); TR_STORE(17, a_s2); }
     } else {
-        // ------------------------------------------------------------ epilogue (rows)
-        const int i = threadIdx.x;  // row of S / O, row k of H, token i of V
-        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-        float *gs = reinterpret_cast<float *>(sm + ws::GS);
+        // ------------------------------------------------------------ WG_B: V weights and state
+        const int i = threadIdx.x - 256;  // token i of V; row k of H
+        const uint32_t trow = tmem + ((uint32_t)((warp - 8) * 32) << 16);
         unsigned char *hb = sm + ws::HB;
         const int64_t KV = (int64_t)kHeadK * V;
-
-        auto step_last_gate = [&](int t) -> float {
-            const StepSpan sp = step_span(t0, t1, cb + t);
-            return chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + sp.len - 1, sp.len - 1, h, H);
-        };
+        float gi = gate_at(0, i), glast = last_gate(0);
 
         // state entering the segment -> Hb (bf16) and TMEM (times the first step's decay)
         {
             const float *src = nullptr;
             if (s == 0) src = a.h0 ? a.h0 + ((int64_t)n * H + h) * KV : nullptr;
             else src = a.seg_state + ((int64_t)(u - 1) * H + h) * KV;
-            const float gam = exp2f(step_last_gate(0));
+            const float gam = exp2f(glast);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 float x[32];
@@ -330,55 +554,38 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             mbar_arrive(b_hb);
         }
 
+        TR_DECL(b_wv); TR_DECL(b_sv); TR_DECL(b_woh); TR_DECL(b_hp);
         for (int t = 0; t < nsteps; ++t) {
             const StepSpan sp = step_span(t0, t1, cb + t);
-            const float gi = (i < sp.len) ? chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + i, i, h, H) : 0.f;
-            float *g = gs + (t & 1) * 128;
-            g[i] = gi;
-            named_sync(1, 128);
-            const float glast = g[sp.len - 1];
-
+            const bool more = t + 1 < nsteps;
+            const float gnext = more ? gate_at(t + 1, i) : 0.f;  // in flight during the step
+            const float glnext = more ? last_gate(t + 1) : 0.f;
             // weighted V rows: Vw_j = 2^(G~_last - G~_j) v_j (0 past the end of the sequence)
-            mbar_wait(&full[t & 1], (t >> 1) & 1, abort_flag);
-            {
-                const float w = (i < sp.len) ? fast_exp2(glast - gi) : 0.f;
-                scale_row(sm + (t & 1) * ws::STAGE + ws::V, sm + ws::VW, i, w);
-            }
+            { TR_T0(x0); mbar_wait(&full_v[t & 1], (t >> 1) & 1, abort_flag); TR_ACC(b_wv, x0); }
+            TR_T0(xv);
+            scale_row(sm + ws::VR + (t & 1) * kRegion, sm + ws::VW, i, (i < sp.len) ? fast_exp2(glast - gi) : 0.f);
             fence_proxy_async_smem();
             mbar_arrive(b_vw);
-
-            // P = decay-masked S, row i
-            mbar_wait(b_smma, t & 1, abort_flag);
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float x[32];
-                tmem_ld32(trow + kColS + 32 * c, x);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int j = 32 * c + e;
-                    x[e] = (j <= i && j < sp.len) ? fast_exp2(gi - g[j]) * x[e] : 0.f;
-                }
-                store_row32_bf16(sm + ws::P + (c >> 1) * kRegion, i, 32 * (c & 1), x);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(b_p);
+            TR_ACC(b_sv, xv);
 
             // state: Hb <- bf16(H_{t+1}); H <- 2^G~_last(t+1) H_{t+1}; or the final state
-            if (t + 1 < nsteps) {
-                const float gam = exp2f(step_last_gate(t + 1));
+            { TR_T0(x0); mbar_wait(b_oh, t & 1, abort_flag); TR_ACC(b_woh, x0); }
+            TR_T0(xh);
+            tc_fence_after();
+            if (more) {
+                const float gam = exp2f(glnext);
+                float x[2][32];
+                tmem_ld32(trow + kColH, x[0]);
+                tmem_ld32(trow + kColH + 32, x[1]);
+                tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
-                    float x[32];
-                    tmem_ld32(trow + kColH + 32 * c, x);
-                    tmem_wait_ld();
-                    store_row32_bf16(hb, i, 32 * c, x);
+                    store_row32_bf16(hb, i, 32 * c, x[c]);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] *= gam;
-                    tmem_st32(trow + kColH + 32 * c, x);
+                    for (int e = 0; e < 32; ++e) x[c][e] *= gam;
                 }
+                tmem_st32(trow + kColH, x[0]);
+                tmem_st32(trow + kColH + 32, x[1]);
                 tmem_wait_st();
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -397,30 +604,11 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     }
                 }
             }
-
-            // o = scale (2^G~_i O1 + O2), row i
-            mbar_wait(b_pv, t & 1, abort_flag);
-            tc_fence_after();
-            const float ei = a.scale * fast_exp2(gi);
-            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(a.o) + ((sp.ta + i) * H + h) * (int64_t)V + v0;
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                float x[32], y[32];
-                tmem_ld32(trow + kColO1 + (t & 1) * kBV + 32 * c, x);
-                tmem_ld32(trow + kColO2 + 32 * c, y);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = fmaf(ei, x[e], a.scale * y[e]);
-                if (i < sp.len && !*abort_flag) {
-                    uint4 *d = reinterpret_cast<uint4 *>(orow + 32 * c);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        d[q] = make_uint4(pack_bf16(x[8 * q], x[8 * q + 1]), pack_bf16(x[8 * q + 2], x[8 * q + 3]),
-                                          pack_bf16(x[8 * q + 4], x[8 * q + 5]), pack_bf16(x[8 * q + 6], x[8 * q + 7]));
-                }
-            }
-            tc_fence_before();
+            TR_ACC(b_hp, xh);
+            gi = gnext;
+            glast = glnext;
         }
+        if (i == 0) { TR_STORE(18, b_wv); TR_STORE(19, b_sv); TR_STORE(20, b_woh); TR_STORE(21, b_hp); }
     }
 
     tc_fence_before();
@@ -439,13 +627,14 @@ tc_segment_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_con
     unsigned char *sm = align1024(smem_raw);
     const SeqLayout &lay = a.lay;
     if (device_failed(lay)) return;
+    const int VT = a.V / kBV;
+    const int u = blockIdx.x / VT;
+    const int v0 = (blockIdx.x % VT) * kBV;
     int n, s;
-    if (!locate_segment(lay, blockIdx.x, n, s)) return;
+    if (!locate_segment(lay, u, n, s)) return;
     const int nseg = seq_segments(lay, n);
     if (s == nseg - 1) return;
-    const int u = blockIdx.x;
     const int h = blockIdx.y, H = a.H, V = a.V;
-    const int v0 = blockIdx.z * kBV;
     int64_t t0, t1;
     seq_span(lay, n, t0, t1);
     const int nt = (int)((t1 - t0 + kStep - 1) / kStep);
@@ -550,7 +739,7 @@ tc_segment_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_con
                 for (int e = 0; e < 8; ++e) d4[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
             }
         }
-        if (i == 0 && blockIdx.z == 0 && !*abort_flag) a.seg_dec[(int64_t)u * H + h] = lsuf;
+        if (i == 0 && v0 == 0 && !*abort_flag) a.seg_dec[(int64_t)u * H + h] = lsuf;
     }
 
     tc_fence_before();
@@ -615,7 +804,7 @@ cudaError_t tc_launch_segment_state(const FwdArgs &a, cudaStream_t st) {
     if ((e = cudaFuncSetAttribute(tc_segment_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kStateSmem)) != cudaSuccess)
         return e;
-    dim3 grid(a.lay.max_segs, a.H, a.V / kBV);
+    dim3 grid(a.lay.max_segs * (a.V / kBV), a.H);
     tc_segment_state_kernel<<<grid, kThreads, kStateSmem, st>>>(tk, tv, a);
     return cudaGetLastError();
 }
@@ -631,8 +820,8 @@ cudaError_t tc_launch_chunk_output(const FwdArgs &a, cudaStream_t st) {
     if ((e = cudaFuncSetAttribute(tc_walk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWalkSmem)) !=
         cudaSuccess)
         return e;
-    dim3 grid(a.lay.max_segs, a.H, a.V / kBV);
-    tc_walk_kernel<<<grid, kThreads, kWalkSmem, st>>>(tq, tk, tv, a);
+    dim3 grid(a.lay.max_segs * (a.V / kBV), a.H);
+    tc_walk_kernel<<<grid, kWalkThreads, kWalkSmem, st>>>(tq, tk, tv, a);
     return cudaGetLastError();
 }
 

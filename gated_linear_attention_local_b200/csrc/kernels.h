@@ -20,6 +20,7 @@ struct FwdArgs {
     bool bf16;
     // workspace carve-up
     float *gcum;     // [tokens, H] chunk-local cumsum of g in log2 units (per-token gates)
+    int *gpos;       // [chunks, H] 1 if the chunk holds a positive log gate (per-token gates)
     float *seg_dec;  // [max_segs, H] log2 total decay of each segment
     float *seg_state;// [max_segs, H, K, V] segment states (local end state, then entering state)
     int *dev_status; // writable status word (bounded device waits record time-outs here)
@@ -31,7 +32,7 @@ cudaError_t launch_varlen_plan(const int64_t *cu, int N, int64_t T_total, int C,
                                int *chunk_off, int *seg_off, int *status, cudaStream_t st);
 
 // Chunk-local inclusive cumsum of g times 1/ln2 (warp-shuffle scan).
-cudaError_t launch_chunk_cumsum(const float *g, float *gcum, const SeqLayout &lay, cudaStream_t st);
+cudaError_t launch_chunk_cumsum(const float *g, float *gcum, int *gpos, const SeqLayout &lay, cudaStream_t st);
 
 // Scalar-decay carry across segments (also writes final states of empty sequences).
 cudaError_t launch_segment_carry(const FwdArgs &a, bool need_carry, cudaStream_t st);

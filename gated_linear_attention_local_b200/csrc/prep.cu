@@ -93,7 +93,8 @@ cudaError_t launch_varlen_plan(const int64_t *cu, int N, int64_t T_total, int C,
 constexpr int kCumsumMaxC = 128;
 
 __global__ void __launch_bounds__(256)
-chunk_cumsum_kernel(const float *__restrict__ g, float *__restrict__ gcum, SeqLayout lay) {
+chunk_cumsum_kernel(const float *__restrict__ g, float *__restrict__ gcum, int *__restrict__ gpos,
+                    SeqLayout lay) {
     __shared__ float tile[kCumsumMaxC][33];
     if (device_failed(lay)) return;
     int n, c;
@@ -115,14 +116,19 @@ chunk_cumsum_kernel(const float *__restrict__ g, float *__restrict__ gcum, SeqLa
     for (int j = warp; j < hw; j += 8) {
         float vals[kCumsumMaxC / 32];
         float run = 0.f;
+        bool positive = false;
 #pragma unroll
         for (int r = 0; r < kCumsumMaxC / 32; ++r) {
             if (r < R) {
                 const int i = lane * R + r;
-                run += (i < len) ? tile[i][j] : 0.f;
+                const float x = (i < len) ? tile[i][j] : 0.f;
+                positive |= x > 0.f;
+                run += x;
                 vals[r] = run;
             }
         }
+        positive = __any_sync(0xffffffffu, positive);
+        if (gpos && lane == 0) gpos[(int64_t)blockIdx.x * H + h0 + j] = positive ? 1 : 0;
         float incl = run;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -143,10 +149,10 @@ chunk_cumsum_kernel(const float *__restrict__ g, float *__restrict__ gcum, SeqLa
     }
 }
 
-cudaError_t launch_chunk_cumsum(const float *g, float *gcum, const SeqLayout &lay, cudaStream_t st) {
+cudaError_t launch_chunk_cumsum(const float *g, float *gcum, int *gpos, const SeqLayout &lay, cudaStream_t st) {
     if (lay.max_chunks == 0) return cudaSuccess;
     dim3 grid(lay.max_chunks, (lay.H + 31) / 32);
-    chunk_cumsum_kernel<<<grid, 256, 0, st>>>(g, gcum, lay);
+    chunk_cumsum_kernel<<<grid, 256, 0, st>>>(g, gcum, gpos, lay);
     return cudaGetLastError();
 }
 

@@ -56,7 +56,9 @@ def random_inputs(B, T, H, K, V, dtype=torch.bfloat16, gate="g", normalizer=1.0,
     """Generic seeded inputs (tests use this for edge cases).
 
     gate: "g" -> g = logsigmoid(N(0,1)) / normalizer [B,T,H]; "gamma" -> retnet_gammas(H);
-          "none" -> no gate; "zero" -> g = 0; "neg_inf" -> g = -inf (gate 0).
+          "none" -> no gate; "zero" -> g = 0; "neg_inf" -> g = -inf (gate 0);
+          "mixed" -> g = 0.3 N(0,1) (log gates of both signs: a gate above 1 is outside the
+          method's forget-gate range, but the operator is still defined).
     With cu_seqlens, B must be 1 and initial states number len(cu_seqlens) - 1.
     Returns a dict of CPU tensors: q,k,v (dtype), g / g_gamma (fp32 or None), h0 (fp32 or None).
     """
@@ -73,6 +75,8 @@ def random_inputs(B, T, H, K, V, dtype=torch.bfloat16, gate="g", normalizer=1.0,
         g = torch.zeros(B, T, H)
     elif gate == "neg_inf":
         g = torch.full((B, T, H), float("-inf"))
+    elif gate == "mixed":
+        g = 0.3 * torch.randn(B, T, H, generator=gen)
     N = (len(cu_seqlens) - 1) if cu_seqlens is not None else B
     s0 = (torch.randn(N, H, K, V, generator=gen) * h0_std) if h0 else None
     return dict(q=q, k=k, v=v, g=g, g_gamma=g_gamma, h0=s0)

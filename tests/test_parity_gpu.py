@@ -273,6 +273,7 @@ TC_CASES = [
     (2, 1000, 2, 128, "none", True, 64),
     (1, 700, 2, 64, "zero", False, 64),
     (1, 1030, 2, 128, "neg_inf", True, 64),
+    (1, 900, 2, 128, "mixed", True, 64),    # positive log gates: exact-decay fallback
 ]
 
 
