@@ -13,21 +13,26 @@
 // through a bf16 copy of the intermediate state -- the same sums, regrouped,
 // which the article's chunk-size tests treat as a rounding-only change.
 //
-// Kernels (one CTA per (segment, head, 64-wide V tile), 1 CTA per SM):
+// Head dims K = 128, 256 and 512 are handled (q/k stream through shared memory one
+// 128-wide k slice at a time); the V tile of a CTA is 64 wide for K = 128 and 32
+// wide otherwise (64-byte swizzled tiles) so the K x BV fp32 state fits in TMEM.
+//
+// Kernels (one CTA per (segment, head, V tile), 1 CTA per SM):
 //  * tc_walk_kernel  -- the fused output: walks the segment's steps in order,
 //      S  = Q K^T                      -> TMEM  (128 x 128 fp32)
 //      O1 = Q Hb                       -> TMEM  (Hb: bf16 copy of the state)
 //      H += K^T Vw  (Vw = rows of V scaled by 2^(G~_last - G~_j))  -> TMEM, fp32
-//      P  = mask(S) (2^(G~_i - G~_j) for j <= i, 0 above) -> smem bf16
+//      P  = mask(S) (2^(G~_i - G~_j) for j <= i, 0 above) -> TMEM bf16 (A of P V)
 //      O2 = P V                        -> TMEM
 //      o  = scale (2^G~_i O1 + O2)     -> HBM (bf16)
 //    The fp32 state H lives in TMEM for the whole segment.  Before the K^T Vw
 //    product of a step accumulates into it, the epilogue multiplies it in place by
 //    the step's total decay 2^G~_last (tcgen05.ld / st) while writing the bf16 copy
 //    Hb for that step's Q Hb -- so the carry h <- 2^G~_last h + sum_j ... happens
-//    on chip with one fp32 read/write of the K x 64 tile per step.
-//    (MN-major operands that are a single 64-wide group -- Hb, Vw, V -- carry an
-//    unused leading byte offset; it is set to 1024 so no address can leave the tile.)
+//    on chip with one fp32 read/write of the K x BV tile per step.
+//    (MN-major operands that are a single group -- Hb, Vw, V -- carry an unused
+//    leading byte offset; it is set to the 8-row stride so no address can leave the
+//    tile.)
 //  * tc_segment_state_kernel -- the state pass for segments that are not the last
 //    of their sequence: the local end state sum_j 2^(Gseg_end - Gseg_j) k_j v_j^T.
 //    It walks the segment BACKWARDS so the decay from a token to the segment end is
@@ -72,42 +77,36 @@ using namespace tc;
 namespace {
 
 constexpr int kStep = 128;                // tokens per step (MMA M)
-constexpr int kHeadK = 128;               // K (q/k head dim) handled by this path
-constexpr int kBV = 64;                   // V tile of one CTA
-constexpr uint32_t kRegion = 128 * 128;   // [128 rows x 64 bf16] swizzled region, bytes
-constexpr int kThreads = 192;
+constexpr uint32_t kRegion = 128 * 128;   // [128 rows x 64 bf16] 128-byte-swizzled region, bytes
 
-// ---------------------------------------------------------------- walk kernel smem
-namespace ws {
-constexpr uint32_t QK = 0;                   // Q/K ring, 2 stages: Q (2 regions), K (2 regions)
-constexpr uint32_t QK_STAGE = 4 * kRegion;
-constexpr uint32_t VR = 2 * QK_STAGE;        // V ring, 2 stages of 1 region
-constexpr uint32_t VW = VR + 2 * kRegion;    // weighted V (1 region)
-constexpr uint32_t HB = VW + kRegion;        // bf16 state copy, MN-major (128 k rows x 64 v)
-constexpr uint32_t GS = HB + kRegion;        // gates, column factors, decay table: 3 x 128 floats
-constexpr uint32_t BARS = GS + 3 * 128 * 4;  // 24 mbarriers
-constexpr uint32_t MISC = BARS + 24 * 8;     // tmem address, abort flag
-constexpr uint32_t TOTAL = MISC + 16;
-}  // namespace ws
-constexpr size_t kWalkSmem = ws::TOTAL + 1024;  // + alignment slack
+// Swizzle of a tile made of `ROWB`-byte rows (ROWB = 128: 64 bf16 per row, the
+// 128-byte swizzle; ROWB = 64: 32 bf16 per row, the 64-byte swizzle).  The 16-byte
+// chunk c of row r is stored at chunk position phys(r, c) of that row.
+template <int ROWB>
+struct Sw;
+template <>
+struct Sw<128> {
+    static constexpr uint32_t layout = 2;  // descriptor swizzle field
+    static __device__ __forceinline__ int phys(int r, int c) { return (c ^ (r & 7)) & 7; }
+};
+template <>
+struct Sw<64> {
+    static constexpr uint32_t layout = 4;
+    static __device__ __forceinline__ int phys(int r, int c) { return (c ^ ((r >> 1) & 3)) & 3; }
+};
 
-// TMEM columns of the walk kernel: S x2 (128 each; the bf16 P of a step overwrites
-// the first 64 columns of its S buffer), O1 x2 (64 each), O2, H
-constexpr uint32_t kColS = 0, kColO1 = 256, kColO2 = 384, kColH = 448, kWalkCols = 512;
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;  // version (sm_100)
+    d |= (uint64_t)layout << 61;
+    return d;
+}
 
-// ---------------------------------------------------------------- state kernel smem
-constexpr int kStateStages = 3;
-namespace ss {
-constexpr uint32_t K = 0;                    // per stage: K (2 regions), V (1), Vw (1)
-constexpr uint32_t V = 2 * kRegion;
-constexpr uint32_t VW = 3 * kRegion;
-constexpr uint32_t STAGE = 4 * kRegion;
-constexpr uint32_t BARS = kStateStages * STAGE;
-constexpr uint32_t MISC = BARS + 16 * 8;
-constexpr uint32_t TOTAL = MISC + 16;
-}  // namespace ss
-constexpr size_t kStateSmem = ss::TOTAL + 1024;
-constexpr uint32_t kStateCols = 64;
+// K-major 128-byte-swizzled operand (Q, K as the B of Q K^T): 8-row atoms 1024 B apart.
+__device__ __forceinline__ uint64_t kdesc(uint32_t saddr) { return sdesc(saddr, 16, 1024, 2); }
 
 __device__ __forceinline__ unsigned char *align1024(unsigned char *p) {
     return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -118,19 +117,21 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Scale the 128-byte row `row` of a swizzled bf16 region by w (the swizzle only
-// permutes 16-byte chunks inside a row, so a whole-row operation ignores it).
-// Thread `row` visits the row's chunks starting at chunk row%8, so the 8 threads of
-// a quarter-warp touch 8 different 16-byte bank groups (rows are 128 B apart, so a
-// common starting chunk would put every thread of the warp on the same 4 banks).
+// Scale row `row` (ROWB bytes of bf16) of a swizzled tile by w.  The swizzle only
+// permutes 16-byte chunks inside a row, so a whole-row operation ignores it.  Thread
+// `row` starts at chunk row % chunks so the threads of a quarter-warp hit different
+// bank groups, and every load is issued before any store (src and dst may alias as
+// far as the compiler knows).
+template <int ROWB>
 __device__ __forceinline__ void scale_row(const unsigned char *src, unsigned char *dst, int row, float w) {
-    const uint4 *s = reinterpret_cast<const uint4 *>(src + row * 128);
-    uint4 *d = reinterpret_cast<uint4 *>(dst + row * 128);
-    uint4 x[8];
+    constexpr int NC = ROWB / 16;
+    const uint4 *s = reinterpret_cast<const uint4 *>(src + row * ROWB);
+    uint4 *d = reinterpret_cast<uint4 *>(dst + row * ROWB);
+    uint4 x[NC];
 #pragma unroll
-    for (int cc = 0; cc < 8; ++cc) x[cc] = s[(cc + row) & 7];  // every load issued before any store
+    for (int cc = 0; cc < NC; ++cc) x[cc] = s[(cc + row) % NC];
 #pragma unroll
-    for (int cc = 0; cc < 8; ++cc) {
+    for (int cc = 0; cc < NC; ++cc) {
         uint32_t *xs = reinterpret_cast<uint32_t *>(&x[cc]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -140,21 +141,21 @@ __device__ __forceinline__ void scale_row(const unsigned char *src, unsigned cha
         }
     }
 #pragma unroll
-    for (int cc = 0; cc < 8; ++cc) d[(cc + row) & 7] = x[cc];
+    for (int cc = 0; cc < NC; ++cc) d[(cc + row) % NC] = x[cc];
 }
 
-// Store 32 fp32 values as bf16 into row `row`, columns [c0, c0+32) (c0 % 32 == 0,
-// c0 + 32 <= 64) of a swizzled region.
-__device__ __forceinline__ void store_row32_bf16(unsigned char *region, int row, int c0, const float (&v)[32]) {
+// Store 32 fp32 values as bf16 into row `row`, logical columns [c0, c0 + 32), of a
+// tile of ROWB-byte rows.
+template <int ROWB>
+__device__ __forceinline__ void store_row32_bf16(unsigned char *tile, int row, int c0, const float (&v)[32]) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        const int chunk = (c0 >> 3) + q;
         uint4 x;
         x.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
         x.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
         x.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
         x.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
-        *reinterpret_cast<uint4 *>(region + row * 128 + (((chunk ^ (row & 7)) & 7) << 4)) = x;
+        *reinterpret_cast<uint4 *>(tile + row * ROWB + (Sw<ROWB>::phys(row, (c0 >> 3) + q) << 4)) = x;
     }
 }
 
@@ -170,31 +171,60 @@ __device__ __forceinline__ StepSpan step_span(int64_t t0, int64_t t1, int step) 
     return s;
 }
 
-__device__ __forceinline__ void record_timeout(const FwdArgs &a) {
-    atomicCAS(a.dev_status, kDevOk, kDevTimeout);
-}
-
+__device__ __forceinline__ void record_timeout(const FwdArgs &a) { atomicCAS(a.dev_status, kDevOk, kDevTimeout); }
 
 // =============================================================================
-// walk kernel (fused output)
+// walk kernel (fused output), templated on the head dim K = 128 KS and the V tile BV
 // =============================================================================
 // Warp roles: 0-7 WG_A (P = masked S, then the output rows), 8-11 WG_B (weighted V
 // and the state pass: Hb and the in-place rescale of H, initial / final state),
 // 12 TMA producer, 13 MMA issuer.  S and O1 are double-buffered in TMEM and the MMA
-// issuer runs one step ahead (O1, H and S of step t+1 are issued before P V of
-// step t), so the tensor core keeps working while WG_A masks the previous S.
+// issuer runs one step ahead, so the tensor core keeps working while WG_A masks
+// the previous S.  Q and K stream through a 2-stage ring one 128-wide k slice at a
+// time; V has its own ring.
 constexpr int kWalkThreads = 448;
 
+template <int KS, int BV>
+struct WalkCfg {
+    static constexpr int HK = 128 * KS;              // q/k head dim
+    static constexpr int VROWB = 2 * BV;             // bytes per row of V, Vw, Hb
+    static constexpr uint32_t VTILE = 128 * VROWB;   // V or Vw tile (128 tokens)
+    static constexpr uint32_t HBB = HK * VROWB;      // Hb: HK rows (k) of BV values
+    static constexpr int NV = (KS == 1) ? 2 : 3;     // V ring stages
+    static constexpr uint32_t VLAYOUT = Sw<VROWB>::layout;
+    static constexpr uint32_t VSBO = 8 * VROWB;      // 8-row group stride of V, Vw, Hb
+    static constexpr uint32_t VKSTEP = 16 * VROWB;   // 16 rows: one MMA K step
+    // shared memory (offsets from a 1024-aligned base)
+    static constexpr uint32_t QK = 0;                // Q/K ring: Q slice (2 regions), K slice (2 regions)
+    static constexpr uint32_t QK_STAGE = 4 * kRegion;
+    static constexpr uint32_t VR = 2 * QK_STAGE;     // V ring
+    static constexpr uint32_t VW = VR + NV * VTILE;  // weighted V
+    static constexpr uint32_t HB = VW + VTILE;       // bf16 state copy, MN-major (rows k)
+    static constexpr uint32_t GS = HB + HBB;         // gates, column factors, decay table
+    static constexpr uint32_t BARS = GS + 3 * 128 * 4;
+    static constexpr uint32_t MISC = BARS + 32 * 8;  // tmem address, abort flag
+    static constexpr uint32_t TOTAL = MISC + 16;
+    static constexpr size_t SMEM = TOTAL + 1024;     // + alignment slack
+    // tensor memory columns: S x2 (the bf16 P of a step overwrites the first 64
+    // columns of its S buffer), O1 x2, O2, H (KS blocks of BV)
+    static constexpr uint32_t COL_S = 0, COL_O1 = 256, COL_O2 = 256 + 2 * BV, COL_H = 256 + 3 * BV;
+    static constexpr uint32_t COLS = 512;
+    static_assert(COL_H + KS * BV <= COLS, "TMEM budget");
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+template <int KS, int BV>
 __global__ void __launch_bounds__(kWalkThreads, 1)
 tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, FwdArgs a) {
+    using C = WalkCfg<KS, BV>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = align1024(smem_raw);
     const SeqLayout &lay = a.lay;
     if (device_failed(lay)) return;
-    const int VT = a.V / kBV;
+    const int VT = a.V / BV;
     const int u = blockIdx.x / VT;           // V tiles of one (segment, head) are adjacent
-    const int v0 = (blockIdx.x % VT) * kBV;  // in the launch order, so Q/K are shared in L2
+    const int v0 = (blockIdx.x % VT) * BV;   // in the launch order, so Q/K are shared in L2
     int n, s;
     if (!locate_segment(lay, u, n, s)) return;
     const int nseg = seq_segments(lay, n);
@@ -206,30 +236,32 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     const int nsteps = min(cb + lay.L, nt) - cb;
     const bool last_seg = (s == nseg - 1);
 
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ws::BARS);
-    uint64_t *full_qk = bars + 0;   // [2] Q/K of a step landed
-    uint64_t *empty_qk = bars + 2;  // [2] Q/K stage free (its last reader, K^T Vw, retired)
-    uint64_t *full_v = bars + 4;    // [2] V of a step landed
-    uint64_t *empty_v = bars + 6;   // [2] V stage free (P V retired)
-    uint64_t *b_s = bars + 8;       // [2] S product done, per S buffer
-    uint64_t *b_oh = bars + 10;     // O1 and H products of a step done (Hb, Vw free again)
-    uint64_t *b_pv = bars + 11;     // P V product of a step done
-    uint64_t *b_p = bars + 12;      // P written (WG_A, 256 arrivals)
-    uint64_t *b_hb = bars + 13;     // Hb written and H rescaled (WG_B, 128 arrivals)
-    uint64_t *b_vw = bars + 14;     // weighted V written (WG_B, 128 arrivals)
-    uint64_t *b_ofree = bars + 15;  // O1 / O2 of a step read out (WG_A, 256 arrivals)
-    uint64_t *b_drain = bars + 16;  // all MMAs retired
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + ws::MISC);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + ws::MISC + 8);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::BARS);
+    uint64_t *full_qk = bars + 0;   // [2] Q/K slice landed
+    uint64_t *empty_qk = bars + 2;  // [2] Q/K slice stage free (its last reader retired)
+    uint64_t *full_v = bars + 4;    // [NV] V of a step landed
+    uint64_t *empty_v = bars + 7;   // [NV] V stage free (P V retired)
+    uint64_t *b_s = bars + 10;      // [2] S product done, per S buffer
+    uint64_t *b_oh = bars + 12;     // O1 and H products of a step done (Hb, Vw free again)
+    uint64_t *b_pv = bars + 13;     // P V product of a step done
+    uint64_t *b_p = bars + 14;      // P written (WG_A, 256 arrivals)
+    uint64_t *b_hb = bars + 15;     // Hb written and H rescaled (WG_B, 128 arrivals)
+    uint64_t *b_vw = bars + 16;     // weighted V written (WG_B, 128 arrivals)
+    uint64_t *b_ofree = bars + 17;  // O1 / O2 of a step read out (WG_A, 256 arrivals)
+    uint64_t *b_drain = bars + 18;  // all MMAs retired
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + C::MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + C::MISC + 8);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int b = 0; b < 2; ++b) {
             mbar_init(&full_qk[b], 1);
             mbar_init(&empty_qk[b], 1);
+            mbar_init(&b_s[b], 1);
+        }
+        for (int b = 0; b < C::NV; ++b) {
             mbar_init(&full_v[b], 1);
             mbar_init(&empty_v[b], 1);
-            mbar_init(&b_s[b], 1);
         }
         mbar_init(b_oh, 1);
         mbar_init(b_pv, 1);
@@ -242,7 +274,7 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         mbar_fence_init();
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, kWalkCols);
+        tmem_alloc(tmem_slot, C::COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -261,138 +293,187 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
 
     if (warp == 12) {
         // ------------------------------------------------------------ TMA producer
-        // Q/K of step t reuse the stage of step t-2 once its K^T Vw retired; V of step t
-        // reuses the stage of step t-2 once its P V retired (later), so Q/K go first.
+        // K = 128: Q/K of step t reuse the stage of step t-2 once its K^T Vw retired,
+        // V of step t the stage of step t-2 once its P V retired (later): Q/K first.
+        // K > 128: V of step t goes first (its 3-stage ring frees early) so the slices
+        // of step t, which wait on the MMAs of earlier slices, never hold it back.
         if (lane == 0) {
             prefetch_tmap(&tq);
             prefetch_tmap(&tk);
             prefetch_tmap(&tv);
-            int issued = 0;
-            for (int t = 0; t < nsteps; ++t) {
-                const int st = t & 1;
-                const int tok = (int)(t0 + (int64_t)(cb + t) * kStep);
-                if (t >= 2 && !mbar_wait(&empty_qk[st], ((t >> 1) - 1) & 1, abort_flag)) break;
-                unsigned char *qk = sm + ws::QK + st * ws::QK_STAGE;
+            int qi = 0, vi = 0;  // slices / V tiles issued
+            auto load_v = [&](int t, int tok) -> bool {
+                const int st = t % C::NV;
+                if (t >= C::NV && !mbar_wait(&empty_v[st], ((t / C::NV) - 1) & 1, abort_flag)) return false;
+                mbar_arrive_expect_tx(&full_v[st], C::VTILE);
+                tma_load_3d(sm + C::VR + st * C::VTILE, &tv, &full_v[st], v0, h, tok);
+                vi = t + 1;
+                return true;
+            };
+            auto load_qk = [&](int q, int sl, int tok) -> bool {
+                const int st = q & 1;
+                if (q >= 2 && !mbar_wait(&empty_qk[st], ((q >> 1) - 1) & 1, abort_flag)) return false;
+                unsigned char *qk = sm + C::QK + st * C::QK_STAGE;
                 mbar_arrive_expect_tx(&full_qk[st], 4 * kRegion);
-                tma_load_3d(qk, &tq, &full_qk[st], 0, h, tok);
-                tma_load_3d(qk + kRegion, &tq, &full_qk[st], 64, h, tok);
-                tma_load_3d(qk + 2 * kRegion, &tk, &full_qk[st], 0, h, tok);
-                tma_load_3d(qk + 3 * kRegion, &tk, &full_qk[st], 64, h, tok);
-                issued = 2 * t + 1;
-                if (t >= 2 && !mbar_wait(&empty_v[st], ((t >> 1) - 1) & 1, abort_flag)) break;
-                mbar_arrive_expect_tx(&full_v[st], kRegion);
-                tma_load_3d(sm + ws::VR + st * kRegion, &tv, &full_v[st], v0, h, tok);
-                issued = 2 * t + 2;
+                tma_load_3d(qk, &tq, &full_qk[st], 128 * sl, h, tok);
+                tma_load_3d(qk + kRegion, &tq, &full_qk[st], 128 * sl + 64, h, tok);
+                tma_load_3d(qk + 2 * kRegion, &tk, &full_qk[st], 128 * sl, h, tok);
+                tma_load_3d(qk + 3 * kRegion, &tk, &full_qk[st], 128 * sl + 64, h, tok);
+                qi = q + 1;
+                return true;
+            };
+            for (int t = 0; t < nsteps; ++t) {
+                const int tok = (int)(t0 + (int64_t)(cb + t) * kStep);
+                if (KS > 1 && !load_v(t, tok)) break;
+                bool ok = true;
+                for (int sl = 0; sl < KS && ok; ++sl) ok = load_qk(t * KS + sl, sl, tok);
+                if (!ok) break;
+                if (KS == 1 && !load_v(t, tok)) break;
             }
             if (*abort_flag) {  // let every copy still in flight land before the CTA exits
-                for (int c = max(0, issued - 4); c < issued; ++c) {
-                    const int t = c >> 1;
-                    mbar_drain((c & 1) ? &full_v[t & 1] : &full_qk[t & 1], (t >> 1) & 1);
-                }
+                for (int q = max(0, qi - 2); q < qi; ++q) mbar_drain(&full_qk[q & 1], (q >> 1) & 1);
+                for (int t = max(0, vi - C::NV); t < vi; ++t) mbar_drain(&full_v[t % C::NV], (t / C::NV) & 1);
             }
         }
     } else if (warp == 13) {
         // ------------------------------------------------------------ MMA issuer
-        // Issue order per iteration t: S(t+1), O1(t+1), P V(t), H(t+1).  S and O1 of the
-        // next step run while WG_A masks S(t); the V tile of step t+1 (whose stage only
-        // frees when P V(t-1) retires) gets until after P V(t) to land.
         if (lane == 0) {
             const uint32_t idS = idesc_bf16_f32(128, 128, false, false);
-            const uint32_t idO = idesc_bf16_f32(128, kBV, false, true);
-            const uint32_t idH = idesc_bf16_f32(128, kBV, true, true);
+            const uint32_t idO = idesc_bf16_f32(128, BV, false, true);
+            const uint32_t idH = idesc_bf16_f32(128, BV, true, true);
             const uint32_t sbase = smem_u32(sm);
-            auto qk_at = [&](int t) { return sbase + ws::QK + (t & 1) * ws::QK_STAGE; };
-            TR_DECL(m_wqk); TR_DECL(m_whb); TR_DECL(m_wof); TR_DECL(m_wvw); TR_DECL(m_wp); TR_DECL(m_wv);
-            TR_DECL(m_is); TR_DECL(m_io); TR_DECL(m_ih); TR_DECL(m_ipv);
-            TR_T0(m_start);
-            auto do_S = [&](int t) -> bool {  // S = Q K^T (both K-major)
-                { TR_T0(x0); if (!mbar_wait(&full_qk[t & 1], (t >> 1) & 1, abort_flag)) return false; TR_ACC(m_wqk, x0); }
-                TR_T0(x1);
-                tc_fence_after();
-                const uint32_t q = qk_at(t), k = q + 2 * kRegion, sd = tmem + kColS + (t & 1) * 128;
+            auto vdesc = [&](uint32_t addr) { return sdesc(addr, C::VSBO, C::VSBO, C::VLAYOUT); };
+            auto qk_at = [&](int q) { return sbase + C::QK + (q & 1) * C::QK_STAGE; };
+            // S (+)= Q_s K_s^T   (both K-major; K steps of 16 inside 64-wide regions)
+            auto mma_S = [&](uint32_t q, uint32_t d, bool acc) {
 #pragma unroll
-                for (int kk = 0; kk < kHeadK / 16; ++kk) {
+                for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
-                    mma_bf16(sd, sdesc_sw128(q + off, 16, 1024), sdesc_sw128(k + off, 16, 1024), idS, kk > 0);
+                    mma_bf16(d, kdesc(q + off), kdesc(q + 2 * kRegion + off), idS, (acc || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(&b_s[t & 1]);
-                TR_ACC(m_is, x1);
+            };
+            // O1 (+)= Q_s Hb_s   (Hb MN-major, rows k: slice s holds rows 128 s ..)
+            auto mma_O1 = [&](uint32_t q, int sl, uint32_t d, bool acc) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
+                    mma_bf16(d, kdesc(q + off), vdesc(sbase + C::HB + (uint32_t)(sl * 128 + kk * 16) * C::VROWB), idO,
+                             (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+            // H_s += K_s^T Vw   (A = K read MN-major: two 64-wide k groups kRegion apart)
+            auto mma_H = [&](uint32_t q, int sl) {
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+                    mma_bf16(tmem + C::COL_H + sl * BV, sdesc(q + 2 * kRegion + jj * 2048, kRegion, 1024, 2),
+                             vdesc(sbase + C::VW + jj * C::VKSTEP), idH, 1);
+            };
+            auto wait_hb_of = [&](int t) -> bool {
+                if (!mbar_wait(b_hb, t & 1, abort_flag)) return false;
+                if (t >= 2 && !mbar_wait(b_ofree, t & 1, abort_flag)) return false;  // O1 buffer t&1 read out
+                tc_fence_after();
                 return true;
             };
-            auto do_O1 = [&](int t) -> bool {  // O1 = Q Hb (Hb MN-major: 16 k rows per K step)
-                { TR_T0(x0); if (!mbar_wait(b_hb, t & 1, abort_flag)) return false; TR_ACC(m_whb, x0); }
-                { TR_T0(x0); if (t >= 2 && !mbar_wait(b_ofree, t & 1, abort_flag)) return false; TR_ACC(m_wof, x0); }
-                TR_T0(x1);
+            auto wait_vw = [&](int t) -> bool {
+                if (!mbar_wait(b_vw, t & 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t q = qk_at(t), o1 = tmem + kColO1 + (t & 1) * kBV;
-#pragma unroll
-                for (int kk = 0; kk < kHeadK / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
-                    mma_bf16(o1, sdesc_sw128(q + off, 16, 1024),
-                             sdesc_sw128(sbase + ws::HB + kk * 2048, 1024, 1024), idO, kk > 0);
-                }
-                TR_ACC(m_io, x1);
                 return true;
             };
-            auto do_H = [&](int t) -> bool {  // H += K^T Vw (A = K read MN-major: two k groups LBO apart)
-                { TR_T0(x0); if (!mbar_wait(b_vw, t & 1, abort_flag)) return false; TR_ACC(m_wvw, x0); }
-                TR_T0(x1);
+            auto wait_qk = [&](int q) -> bool {
+                if (!mbar_wait(&full_qk[q & 1], (q >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t k = qk_at(t) + 2 * kRegion;
-#pragma unroll
-                for (int jj = 0; jj < kStep / 16; ++jj)
-                    mma_bf16(tmem + kColH, sdesc_sw128(k + jj * 2048, kRegion, 1024),
-                             sdesc_sw128(sbase + ws::VW + jj * 2048, 1024, 1024), idH, 1);
-                mma_commit(b_oh);             // WG_B may rewrite Hb, Vw and H
-                mma_commit(&empty_qk[t & 1]); // Q/K stage free
-                TR_ACC(m_ih, x1);
                 return true;
             };
             auto do_PV = [&](int t) -> bool {  // O2 = P V (P from TMEM, V MN-major)
-                { TR_T0(x0); if (!mbar_wait(b_p, t & 1, abort_flag)) return false; TR_ACC(m_wp, x0); }
-                { TR_T0(x0); if (!mbar_wait(&full_v[t & 1], (t >> 1) & 1, abort_flag)) return false; TR_ACC(m_wv, x0); }
-                TR_T0(x1);
+                if (!mbar_wait(b_p, t & 1, abort_flag)) return false;
+                if (!mbar_wait(&full_v[t % C::NV], (t / C::NV) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t v = sbase + ws::VR + (t & 1) * kRegion;
-                const uint32_t pt = tmem + kColS + (t & 1) * 128;
+                const uint32_t v = sbase + C::VR + (t % C::NV) * C::VTILE;
+                const uint32_t pt = tmem + C::COL_S + (t & 1) * 128;
 #pragma unroll
                 for (int jj = 0; jj < kStep / 16; ++jj)
-                    mma_bf16_tmem_a(tmem + kColO2, pt + jj * 8, sdesc_sw128(v + jj * 2048, 1024, 1024), idO, jj > 0);
+                    mma_bf16_tmem_a(tmem + C::COL_O2, pt + jj * 8, vdesc(v + jj * C::VKSTEP), idO, jj > 0);
                 mma_commit(b_pv);
-                mma_commit(&empty_v[t & 1]);
-                TR_ACC(m_ipv, x1);
+                mma_commit(&empty_v[t % C::NV]);
                 return true;
             };
-            if (nsteps > 0 && do_S(0) && do_O1(0) && do_H(0)) {
-                for (int t = 0; t < nsteps; ++t) {
-                    const bool more = t + 1 < nsteps;
-                    if (more && !(do_S(t + 1) && do_O1(t + 1))) break;
-                    if (!do_PV(t)) break;
-                    if (more && !do_H(t + 1)) break;
+            const uint32_t o1_of[2] = {tmem + C::COL_O1, tmem + C::COL_O1 + BV};
+            const uint32_t s_of[2] = {tmem + C::COL_S, tmem + C::COL_S + 128};
+            if constexpr (KS == 1) {
+                // order per iteration t: S(t+1), O1(t+1), P V(t), H(t+1)
+                auto do_S = [&](int t) -> bool {
+                    if (!wait_qk(t)) return false;
+                    mma_S(qk_at(t), s_of[t & 1], false);
+                    mma_commit(&b_s[t & 1]);
+                    return true;
+                };
+                auto do_O1 = [&](int t) -> bool {
+                    if (!wait_hb_of(t)) return false;
+                    mma_O1(qk_at(t), 0, o1_of[t & 1], false);
+                    return true;
+                };
+                auto do_H = [&](int t) -> bool {
+                    if (!wait_vw(t)) return false;
+                    mma_H(qk_at(t), 0);
+                    mma_commit(b_oh);              // WG_B may rewrite Hb, Vw and H
+                    mma_commit(&empty_qk[t & 1]);  // Q/K stage free
+                    return true;
+                };
+                if (nsteps > 0 && do_S(0) && do_O1(0) && do_H(0)) {
+                    for (int t = 0; t < nsteps; ++t) {
+                        const bool more = t + 1 < nsteps;
+                        if (more && !(do_S(t + 1) && do_O1(t + 1))) break;
+                        if (!do_PV(t)) break;
+                        if (more && !do_H(t + 1)) break;
+                    }
+                }
+            } else {
+                // per step: for each k slice S, O1 and H of that slice, then P V of the
+                // previous step
+                auto do_front = [&](int t) -> bool {
+                    for (int sl = 0; sl < KS; ++sl) {
+                        const int q = t * KS + sl;
+                        if (!wait_qk(q)) return false;
+                        const uint32_t qa = qk_at(q);
+                        mma_S(qa, s_of[t & 1], sl > 0);
+                        if (sl == KS - 1) mma_commit(&b_s[t & 1]);
+                        if (sl == 0 && !wait_hb_of(t)) return false;
+                        mma_O1(qa, sl, o1_of[t & 1], sl > 0);
+                        if (sl == 0 && !wait_vw(t)) return false;
+                        mma_H(qa, sl);
+                        mma_commit(&empty_qk[q & 1]);
+                    }
+                    mma_commit(b_oh);
+                    return true;
+                };
+                if (nsteps > 0 && do_front(0)) {
+                    for (int t = 0; t < nsteps; ++t) {
+                        if (t + 1 < nsteps && !do_front(t + 1)) break;
+                        if (!do_PV(t)) break;
+                    }
                 }
             }
             mma_commit(b_drain);
             mbar_drain(b_drain, 0);
-            TR_STORE(0, clock64() - m_start); TR_STORE(1, nsteps);
-            TR_STORE(2, m_wqk); TR_STORE(3, m_whb); TR_STORE(4, m_wof); TR_STORE(5, m_wvw); TR_STORE(6, m_wp);
-            TR_STORE(7, m_wv); TR_STORE(8, m_is); TR_STORE(9, m_io); TR_STORE(10, m_ih); TR_STORE(11, m_ipv);
         }
     } else if (warp < 8) {
         // ------------------------------------------------------------ WG_A: P and output
         // Eight warps, two per TMEM sub-partition: warp w owns rows 32(w%4).. and half
-        // w/4 of the work -- S tiles {0,1} or {2,3} of its rows, output columns 0-31 or
-        // 32-63.  P_ij = 2^(G~_i - G~_j) S_ij for j <= i.  For the 32-column tiles strictly
-        // below the diagonal the decay factors as 2^(G~_i - G~_r) * 2^(G~_r - G~_j) with r
-        // the tile's last column: one exp2 per row and tile plus a per-column table f
-        // (both factors <= 1 because G~ does not increase when the log gates are <= 0).
-        // The diagonal tile, and every tile of a step that holds a positive log gate, use
-        // the direct 2^(G~_i - G~_j).  Tiles above the diagonal are zero.
+        // w/4 of the work -- S tiles {0,1} or {2,3} of its rows, output columns of one
+        // half of the V tile.  P_ij = 2^(G~_i - G~_j) S_ij for j <= i.  For the
+        // 32-column tiles strictly below the diagonal the decay factors as
+        // 2^(G~_i - G~_r) * 2^(G~_r - G~_j) with r the tile's last column: one exp2 per
+        // row and tile plus a per-column table f (both factors <= 1 because G~ does not
+        // increase when the log gates are <= 0).  The diagonal tile, and every tile of
+        // a step that holds a positive log gate, use the direct 2^(G~_i - G~_j).  Tiles
+        // above the diagonal are zero.
+        constexpr int OW = BV / 2;  // output columns per half
         const int quarter = warp & 3, half = warp >> 2;
         const int i = quarter * 32 + lane;  // row of S / O
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
-        float *gs = reinterpret_cast<float *>(sm + ws::GS);          // [128] gates of the step
-        float *fs = gs + 128;                                         // [128] column factors
-        float *tab = gs + 256;                                        // [128] 2^(d gamma)
+        float *gs = reinterpret_cast<float *>(sm + C::GS);  // [128] gates of the step
+        float *fs = gs + 128;                                // [128] column factors
+        float *tab = gs + 256;                               // [128] 2^(d gamma)
         const bool per_token = a.gate_mode == kGatePerToken;
         if (!per_token && half == 0) {
             const float gam = (a.gate_mode == kGatePerHead) ? fmaxf(a.g_gamma[h], kMinLogGate) * kRcpLn2 : 0.f;
@@ -417,7 +498,7 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             fs[i] = fi;
         }
         named_sync(1, 256);
-        TR_DECL(a_ws); TR_DECL(a_p); TR_DECL(a_s1); TR_DECL(a_wpv); TR_DECL(a_out); TR_DECL(a_s2);
+        TR_DECL(a_ws); TR_DECL(a_p); TR_DECL(a_wpv); TR_DECL(a_out);
         for (int t = 0; t < nsteps; ++t) {
             const StepSpan sp = step_span(t0, t1, cb + t);
             float gnext = 0.f, fnext = 0.f;
@@ -427,7 +508,7 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             { TR_T0(x0); mbar_wait(&b_s[t & 1], (t >> 1) & 1, abort_flag); TR_ACC(a_ws, x0); }
             TR_T0(xp);
             tc_fence_after();
-            const uint32_t srow = trow + kColS + (t & 1) * 128;
+            const uint32_t srow = trow + C::COL_S + (t & 1) * 128;
             // this half's two S tiles -> P (bf16 pairs).  P tile c is written to columns
             // 16c.. of the same S buffer once both halves have read their S tiles.
             uint32_t pk[2][16];
@@ -479,30 +560,35 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             tc_fence_before();
             mbar_arrive(b_p);
             TR_ACC(a_p, xp);
-            { TR_T0(x0); named_sync(1, 256); TR_ACC(a_s1, x0); }  // every row is done with this step's gates and factors
+            named_sync(1, 256);  // every row is done with this step's gates and factors
             if (half == 0) {
                 gs[i] = gnext;
                 fs[i] = fnext;
             }
 
-            // o = scale (2^G~_i O1 + O2), row i, columns 32*half ..
+            // o = scale (2^G~_i O1 + O2), row i, columns [OW half, OW (half + 1)) of the tile
             { TR_T0(x0); mbar_wait(b_pv, t & 1, abort_flag); TR_ACC(a_wpv, x0); }
             TR_T0(xo);
             tc_fence_after();
             const float ei = a.scale * fast_exp2(gi);
             __nv_bfloat16 *orow =
-                static_cast<__nv_bfloat16 *>(a.o) + ((sp.ta + i) * H + h) * (int64_t)V + v0 + 32 * half;
+                static_cast<__nv_bfloat16 *>(a.o) + ((sp.ta + i) * H + h) * (int64_t)V + v0 + OW * half;
             {
-                float ox[32], oy[32];
-                tmem_ld32(trow + kColO1 + (t & 1) * kBV + 32 * half, ox);
-                tmem_ld32(trow + kColO2 + 32 * half, oy);
+                float ox[OW], oy[OW];
+                if constexpr (OW == 32) {
+                    tmem_ld32(trow + C::COL_O1 + (t & 1) * BV + OW * half, ox);
+                    tmem_ld32(trow + C::COL_O2 + OW * half, oy);
+                } else {
+                    tmem_ld16f(trow + C::COL_O1 + (t & 1) * BV + OW * half, ox);
+                    tmem_ld16f(trow + C::COL_O2 + OW * half, oy);
+                }
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) ox[e] = fmaf(ei, ox[e], a.scale * oy[e]);
+                for (int e = 0; e < OW; ++e) ox[e] = fmaf(ei, ox[e], a.scale * oy[e]);
                 if (i < sp.len && !*abort_flag) {
                     uint4 *d = reinterpret_cast<uint4 *>(orow);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
+                    for (int q = 0; q < OW / 8; ++q)
                         d[q] = make_uint4(pack_bf16(ox[8 * q], ox[8 * q + 1]), pack_bf16(ox[8 * q + 2], ox[8 * q + 3]),
                                           pack_bf16(ox[8 * q + 4], ox[8 * q + 5]), pack_bf16(ox[8 * q + 6], ox[8 * q + 7]));
                 }
@@ -510,18 +596,45 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             tc_fence_before();
             mbar_arrive(b_ofree);
             TR_ACC(a_out, xo);
-            { TR_T0(x0); named_sync(1, 256); TR_ACC(a_s2, x0); }  // next step's gates and factors are in place
+            named_sync(1, 256);  // next step's gates and factors are in place
             gi = gnext;
             pos = posnext;
         }
-        if (threadIdx.x == 96) { TR_STORE(12, a_ws); TR_STORE(13, a_p); TR_STORE(14, a_s1); TR_STORE(15, a_wpv); TR_STORE(16, a_out); TR_STORE(17, a_s2); }
+        if (threadIdx.x == 96) { TR_STORE(12, a_ws); TR_STORE(13, a_p); TR_STORE(15, a_wpv); TR_STORE(16, a_out); TR_STORE(1, nsteps); }
     } else {
         // ------------------------------------------------------------ WG_B: V weights and state
-        const int i = threadIdx.x - 256;  // token i of V; row k of H
+        const int i = threadIdx.x - 256;  // token i of V; row 128 b + i of H, block b
         const uint32_t trow = tmem + ((uint32_t)((warp - 8) * 32) << 16);
-        unsigned char *hb = sm + ws::HB;
-        const int64_t KV = (int64_t)kHeadK * V;
+        unsigned char *hb = sm + C::HB;
+        const int64_t KV = (int64_t)C::HK * V;
         float gi = gate_at(0, i), glast = last_gate(0);
+
+        // moves BV fp32 values between a state row in TMEM block b and registers
+        auto h_ld = [&](int b, float (&x)[BV]) {
+            if constexpr (BV == 64) {
+                float (&x0)[32] = *reinterpret_cast<float(*)[32]>(&x[0]);
+                float (&x1)[32] = *reinterpret_cast<float(*)[32]>(&x[32]);
+                tmem_ld32(trow + C::COL_H + b * BV, x0);
+                tmem_ld32(trow + C::COL_H + b * BV + 32, x1);
+            } else {
+                tmem_ld32(trow + C::COL_H + b * BV, x);
+            }
+        };
+        auto h_st = [&](int b, const float (&x)[BV]) {
+            if constexpr (BV == 64) {
+                const float (&x0)[32] = *reinterpret_cast<const float(*)[32]>(&x[0]);
+                const float (&x1)[32] = *reinterpret_cast<const float(*)[32]>(&x[32]);
+                tmem_st32(trow + C::COL_H + b * BV, x0);
+                tmem_st32(trow + C::COL_H + b * BV + 32, x1);
+            } else {
+                tmem_st32(trow + C::COL_H + b * BV, x);
+            }
+        };
+        auto hb_row = [&](int b, const float (&x)[BV]) {  // bf16 copy of state row 128 b + i
+#pragma unroll
+            for (int c = 0; c < BV / 32; ++c)
+                store_row32_bf16<C::VROWB>(hb, 128 * b + i, 32 * c, *reinterpret_cast<const float(*)[32]>(&x[32 * c]));
+        };
 
         // state entering the segment -> Hb (bf16) and TMEM (times the first step's decay)
         {
@@ -529,24 +642,24 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             if (s == 0) src = a.h0 ? a.h0 + ((int64_t)n * H + h) * KV : nullptr;
             else src = a.seg_state + ((int64_t)(u - 1) * H + h) * KV;
             const float gam = exp2f(glast);
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                float x[32];
+#pragma unroll 1
+            for (int b = 0; b < KS; ++b) {
+                float x[BV];
                 if (src) {
-                    const float4 *p4 = reinterpret_cast<const float4 *>(src + (int64_t)i * V + v0 + 32 * c);
+                    const float4 *p4 = reinterpret_cast<const float4 *>(src + (int64_t)(128 * b + i) * V + v0);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
+                    for (int e = 0; e < BV / 4; ++e) {
                         const float4 f = p4[e];
                         x[4 * e] = f.x; x[4 * e + 1] = f.y; x[4 * e + 2] = f.z; x[4 * e + 3] = f.w;
                     }
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] = 0.f;
+                    for (int e = 0; e < BV; ++e) x[e] = 0.f;
                 }
-                store_row32_bf16(hb, i, 32 * c, x);
+                hb_row(b, x);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] *= gam;
-                tmem_st32(trow + kColH + 32 * c, x);
+                for (int e = 0; e < BV; ++e) x[e] *= gam;
+                h_st(b, x);
             }
             tmem_wait_st();
             fence_proxy_async_smem();
@@ -554,16 +667,17 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             mbar_arrive(b_hb);
         }
 
-        TR_DECL(b_wv); TR_DECL(b_sv); TR_DECL(b_woh); TR_DECL(b_hp);
+        TR_DECL(b_sv); TR_DECL(b_woh); TR_DECL(b_hp);
         for (int t = 0; t < nsteps; ++t) {
             const StepSpan sp = step_span(t0, t1, cb + t);
             const bool more = t + 1 < nsteps;
             const float gnext = more ? gate_at(t + 1, i) : 0.f;  // in flight during the step
             const float glnext = more ? last_gate(t + 1) : 0.f;
             // weighted V rows: Vw_j = 2^(G~_last - G~_j) v_j (0 past the end of the sequence)
-            { TR_T0(x0); mbar_wait(&full_v[t & 1], (t >> 1) & 1, abort_flag); TR_ACC(b_wv, x0); }
+            mbar_wait(&full_v[t % C::NV], (t / C::NV) & 1, abort_flag);
             TR_T0(xv);
-            scale_row(sm + ws::VR + (t & 1) * kRegion, sm + ws::VW, i, (i < sp.len) ? fast_exp2(glast - gi) : 0.f);
+            scale_row<C::VROWB>(sm + C::VR + (t % C::NV) * C::VTILE, sm + C::VW, i,
+                                (i < sp.len) ? fast_exp2(glast - gi) : 0.f);
             fence_proxy_async_smem();
             mbar_arrive(b_vw);
             TR_ACC(b_sv, xv);
@@ -574,33 +688,31 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             tc_fence_after();
             if (more) {
                 const float gam = exp2f(glnext);
-                float x[2][32];
-                tmem_ld32(trow + kColH, x[0]);
-                tmem_ld32(trow + kColH + 32, x[1]);
-                tmem_wait_ld();
+#pragma unroll 1
+                for (int b = 0; b < KS; ++b) {
+                    float x[BV];
+                    h_ld(b, x);
+                    tmem_wait_ld();
+                    hb_row(b, x);
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    store_row32_bf16(hb, i, 32 * c, x[c]);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) x[c][e] *= gam;
+                    for (int e = 0; e < BV; ++e) x[e] *= gam;
+                    h_st(b, x);
                 }
-                tmem_st32(trow + kColH, x[0]);
-                tmem_st32(trow + kColH + 32, x[1]);
                 tmem_wait_st();
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(b_hb);
             } else if (last_seg && a.hT) {
-                float *dst = a.hT + ((int64_t)n * H + h) * KV + (int64_t)i * V + v0;
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    float x[32];
-                    tmem_ld32(trow + kColH + 32 * c, x);
+#pragma unroll 1
+                for (int b = 0; b < KS; ++b) {
+                    float x[BV];
+                    h_ld(b, x);
                     tmem_wait_ld();
                     if (!*abort_flag) {
-                        float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * c);
+                        float4 *d4 = reinterpret_cast<float4 *>(a.hT + ((int64_t)n * H + h) * KV +
+                                                                (int64_t)(128 * b + i) * V + v0);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) d4[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+                        for (int e = 0; e < BV / 4; ++e) d4[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
                     }
                 }
             }
@@ -608,28 +720,48 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             gi = gnext;
             glast = glnext;
         }
-        if (i == 0) { TR_STORE(18, b_wv); TR_STORE(19, b_sv); TR_STORE(20, b_woh); TR_STORE(21, b_hp); }
+        if (i == 0) { TR_STORE(19, b_sv); TR_STORE(20, b_woh); TR_STORE(21, b_hp); }
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, kWalkCols);
+    if (warp == 0) tmem_dealloc(tmem, C::COLS);
     if (threadIdx.x == 0 && *abort_flag) record_timeout(a);
 }
 
 // =============================================================================
 // segment state kernel: local end state of a non-final segment, walked backwards
 // =============================================================================
-__global__ void __launch_bounds__(kThreads, 1)
+// One CTA per (segment, head, 128-row k block, 64-wide V tile): the state rows of
+// one k block are independent of the others, so any K = 128 KB splits into KB
+// problems of this one shape.
+constexpr int kStateThreads = 192;
+constexpr int kStateStages = 3;
+constexpr int kStateBV = 64;
+namespace ss {
+constexpr uint32_t K = 0;                    // per stage: K (2 regions), V (1), Vw (1)
+constexpr uint32_t V = 2 * kRegion;
+constexpr uint32_t VW = 3 * kRegion;
+constexpr uint32_t STAGE = 4 * kRegion;
+constexpr uint32_t BARS = kStateStages * STAGE;
+constexpr uint32_t MISC = BARS + 16 * 8;
+constexpr uint32_t TOTAL = MISC + 16;
+}  // namespace ss
+constexpr size_t kStateSmem = ss::TOTAL + 1024;
+constexpr uint32_t kStateCols = 64;
+
+__global__ void __launch_bounds__(kStateThreads, 1)
 tc_segment_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, FwdArgs a) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = align1024(smem_raw);
     const SeqLayout &lay = a.lay;
     if (device_failed(lay)) return;
-    const int VT = a.V / kBV;
-    const int u = blockIdx.x / VT;
-    const int v0 = (blockIdx.x % VT) * kBV;
+    const int VT = a.V / kStateBV, KB = a.K / 128;
+    const int u = blockIdx.x / (VT * KB);
+    const int rem = blockIdx.x % (VT * KB);
+    const int kb = rem / VT;
+    const int v0 = (rem % VT) * kStateBV;
     int n, s;
     if (!locate_segment(lay, u, n, s)) return;
     const int nseg = seq_segments(lay, n);
@@ -642,9 +774,9 @@ tc_segment_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_con
     const int nsteps = min(cb + lay.L, nt) - cb;
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ss::BARS);
-    uint64_t *full = bars;                      // [3]
-    uint64_t *empty = bars + kStateStages;      // [3]
-    uint64_t *vwready = bars + 2 * kStateStages;// [3], 128 arrivals
+    uint64_t *full = bars;                        // [3]
+    uint64_t *empty = bars + kStateStages;        // [3]
+    uint64_t *vwready = bars + 2 * kStateStages;  // [3], 128 arrivals
     uint64_t *b_done = bars + 3 * kStateStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + ss::MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + ss::MISC + 8);
@@ -680,8 +812,8 @@ tc_segment_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_con
                 const int tok = (int)(t0 + (int64_t)(cb + nsteps - 1 - r) * kStep);
                 unsigned char *base = sm + st * ss::STAGE;
                 mbar_arrive_expect_tx(&full[st], 3 * kRegion);
-                tma_load_3d(base + ss::K, &tk, &full[st], 0, h, tok);
-                tma_load_3d(base + ss::K + kRegion, &tk, &full[st], 64, h, tok);
+                tma_load_3d(base + ss::K, &tk, &full[st], 128 * kb, h, tok);
+                tma_load_3d(base + ss::K + kRegion, &tk, &full[st], 128 * kb + 64, h, tok);
                 tma_load_3d(base + ss::V, &tv, &full[st], v0, h, tok);
                 issued = r + 1;
             }
@@ -691,7 +823,7 @@ tc_segment_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_con
         }
     } else if (warp == 5) {
         if (lane == 0) {
-            const uint32_t idH = idesc_bf16_f32(128, kBV, true, true);
+            const uint32_t idH = idesc_bf16_f32(128, kStateBV, true, true);
             const uint32_t sbase = smem_u32(sm);
             for (int r = 0; r < nsteps; ++r) {
                 const int st = r % kStateStages;
@@ -703,8 +835,8 @@ tc_segment_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_con
                 const uint32_t vw = sbase + st * ss::STAGE + ss::VW;
 #pragma unroll
                 for (int jj = 0; jj < kStep / 16; ++jj)
-                    mma_bf16(tmem, sdesc_sw128(k + jj * 2048, kRegion, 1024), sdesc_sw128(vw + jj * 2048, 1024, 1024),
-                             idH, (r > 0 || jj > 0) ? 1u : 0u);
+                    mma_bf16(tmem, sdesc(k + jj * 2048, kRegion, 1024, 2), sdesc(vw + jj * 2048, 1024, 1024, 2), idH,
+                             (r > 0 || jj > 0) ? 1u : 0u);
                 mma_commit(&empty[st]);
             }
             mma_commit(b_done);
@@ -720,26 +852,27 @@ tc_segment_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_con
             const float glast = chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + sp.len - 1, sp.len - 1, h, H);
             mbar_wait(&full[st], (r / kStateStages) & 1, abort_flag);
             const float w = (i < sp.len) ? fast_exp2(lsuf + (glast - gi)) : 0.f;
-            scale_row(sm + st * ss::STAGE + ss::V, sm + st * ss::STAGE + ss::VW, i, w);
+            scale_row<128>(sm + st * ss::STAGE + ss::V, sm + st * ss::STAGE + ss::VW, i, w);
             fence_proxy_async_smem();
             mbar_arrive(&vwready[st]);
             lsuf += glast;
         }
         mbar_wait(b_done, 0, abort_flag);
         tc_fence_after();
-        float *dst = a.seg_state + (((int64_t)u * H + h) * kHeadK + i) * V + v0;
+        float *dst = a.seg_state + (((int64_t)u * H + h) * a.K + 128 * kb + i) * V + v0;
+        float x[2][32];
+        tmem_ld32(trow, x[0]);
+        tmem_ld32(trow + 32, x[1]);
+        tmem_wait_ld();
+        if (!*abort_flag) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            float x[32];
-            tmem_ld32(trow + 32 * c, x);
-            tmem_wait_ld();
-            if (!*abort_flag) {
+            for (int c = 0; c < 2; ++c) {
                 float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * c);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) d4[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+                for (int e = 0; e < 8; ++e) d4[e] = make_float4(x[c][4 * e], x[c][4 * e + 1], x[c][4 * e + 2], x[c][4 * e + 3]);
             }
         }
-        if (i == 0 && v0 == 0 && !*abort_flag) a.seg_dec[(int64_t)u * H + h] = lsuf;
+        if (i == 0 && v0 == 0 && kb == 0 && !*abort_flag) a.seg_dec[(int64_t)u * H + h] = lsuf;
     }
 
     tc_fence_before();
@@ -769,60 +902,76 @@ cudaError_t get_encoder() {
     return g_encode ? cudaSuccess : cudaErrorNotSupported;
 }
 
-// 3-D map over a [tokens, H, D] bf16 tensor with a [128 tokens x 1 head x 64] box,
-// 128-byte swizzle (rows of 64 bf16 = 128 B).
-cudaError_t make_map(CUtensorMap *m, const void *ptr, int64_t tokens, int H, int D) {
+// 3-D map over a [tokens, H, D] bf16 tensor with a [128 tokens x 1 head x box]
+// box; box = 64 (128-byte rows, 128-byte swizzle) or 32 (64-byte rows, 64-byte swizzle).
+cudaError_t make_map(CUtensorMap *m, const void *ptr, int64_t tokens, int H, int D, int box) {
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)tokens};
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-    cuuint32_t box[3] = {64, 1, (cuuint32_t)kStep};
+    cuuint32_t boxd[3] = {(cuuint32_t)box, 1, (cuuint32_t)kStep};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUtensorMapSwizzle sw = (box == 64) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, boxd, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 int64_t total_tokens(const FwdArgs &a) { return a.lay.cu ? a.lay.T : (int64_t)a.lay.N * a.lay.T; }
 
+int walk_bv(int K) { return K == 128 ? 64 : 32; }
+
+template <int KS, int BV>
+cudaError_t launch_walk(const FwdArgs &a, cudaStream_t st) {
+    using C = WalkCfg<KS, BV>;
+    CUtensorMap tq, tk, tv;
+    const int64_t tok = total_tokens(a);
+    cudaError_t e;
+    if ((e = make_map(&tq, a.q, tok, a.H, a.K, 64)) != cudaSuccess) return e;
+    if ((e = make_map(&tk, a.k, tok, a.H, a.K, 64)) != cudaSuccess) return e;
+    if ((e = make_map(&tv, a.v, tok, a.H, a.V, BV)) != cudaSuccess) return e;
+    auto kern = tc_walk_kernel<KS, BV>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM)) != cudaSuccess)
+        return e;
+    dim3 grid(a.lay.max_segs * (a.V / BV), a.H);
+    kern<<<grid, kWalkThreads, C::SMEM, st>>>(tq, tk, tv, a);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 bool tc_path_supports(bool bf16, int K, int V, int C) {
-    return bf16 && K == kHeadK && V % kBV == 0 && V >= kBV && V <= 512 && (C == 64 || C == 128);
+    return bf16 && (K == 128 || K == 256 || K == 512) && V % 64 == 0 && V >= 64 && V <= 512 &&
+           (C == 64 || C == 128);
 }
 
 int tc_path_step() { return kStep; }
 
-int tc_path_vtiles(int, int V) { return V / kBV; }
+int tc_path_vtiles(int K, int V) { return V / walk_bv(K); }
 
 cudaError_t tc_launch_segment_state(const FwdArgs &a, cudaStream_t st) {
     cudaError_t e = get_encoder();
     if (e != cudaSuccess) return e;
     CUtensorMap tk, tv;
     const int64_t tok = total_tokens(a);
-    if ((e = make_map(&tk, a.k, tok, a.H, a.K)) != cudaSuccess) return e;
-    if ((e = make_map(&tv, a.v, tok, a.H, a.V)) != cudaSuccess) return e;
+    if ((e = make_map(&tk, a.k, tok, a.H, a.K, 64)) != cudaSuccess) return e;
+    if ((e = make_map(&tv, a.v, tok, a.H, a.V, 64)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(tc_segment_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kStateSmem)) != cudaSuccess)
         return e;
-    dim3 grid(a.lay.max_segs * (a.V / kBV), a.H);
-    tc_segment_state_kernel<<<grid, kThreads, kStateSmem, st>>>(tk, tv, a);
+    dim3 grid(a.lay.max_segs * (a.V / kStateBV) * (a.K / 128), a.H);
+    tc_segment_state_kernel<<<grid, kStateThreads, kStateSmem, st>>>(tk, tv, a);
     return cudaGetLastError();
 }
 
 cudaError_t tc_launch_chunk_output(const FwdArgs &a, cudaStream_t st) {
     cudaError_t e = get_encoder();
     if (e != cudaSuccess) return e;
-    CUtensorMap tq, tk, tv;
-    const int64_t tok = total_tokens(a);
-    if ((e = make_map(&tq, a.q, tok, a.H, a.K)) != cudaSuccess) return e;
-    if ((e = make_map(&tk, a.k, tok, a.H, a.K)) != cudaSuccess) return e;
-    if ((e = make_map(&tv, a.v, tok, a.H, a.V)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(tc_walk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWalkSmem)) !=
-        cudaSuccess)
-        return e;
-    dim3 grid(a.lay.max_segs * (a.V / kBV), a.H);
-    tc_walk_kernel<<<grid, kWalkThreads, kWalkSmem, st>>>(tq, tk, tv, a);
-    return cudaGetLastError();
+    switch (a.K) {
+        case 128: return launch_walk<1, 64>(a, st);
+        case 256: return launch_walk<2, 32>(a, st);
+        case 512: return launch_walk<4, 32>(a, st);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace sgla

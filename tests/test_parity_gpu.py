@@ -310,3 +310,28 @@ def test_tensor_core_workspace_status_clean():
     sg.simple_gla_fwd(d["q"], d["k"], d["v"], g=d["g"], initial_state=d["h0"], output_final_state=True,
                       workspace=ws)
     assert sg.workspace_status(ws) == 0
+
+
+WIDE_K_CASES = [
+    # (B, T, H, K, V, gate, h0)   bf16, tensor-core path with K > 128 (V tile 32)
+    (2, 129, 2, 256, 256, "g", True),
+    (1, 300, 1, 512, 512, "g", True),
+    (1, 3000, 1, 512, 64, "g", True),     # many segments: k-block state pass + carry
+    (1, 2500, 2, 256, 128, "gamma", True),
+    (2, 700, 1, 512, 128, "mixed", False),
+]
+
+
+@pytest.mark.parametrize("case", WIDE_K_CASES, ids=lambda c: f"B{c[0]}T{c[1]}H{c[2]}K{c[3]}V{c[4]}-{c[5]}-h0{int(c[6])}")
+def test_tensor_core_wide_k(case):
+    B, T, H, K, V, gate, h0 = case
+    inp = random_inputs(B, T, H, K, V, torch.bfloat16, gate=gate, h0=h0, seed=51)
+    gpu = _ran("chunk_output_tc", lambda: run_dense(inp))
+    check(inp, gpu, oracle_fwd(inp), torch.bfloat16, "tc wide-k")
+
+
+def test_tensor_core_wide_k_varlen():
+    cu = torch.tensor([0, 100, 1600, 1601, 2900], dtype=torch.int64)
+    inp = random_inputs(1, 2900, 2, 512, 128, torch.bfloat16, gate="g", h0=True, seed=52, cu_seqlens=cu)
+    gpu = _ran("chunk_output_tc", lambda: run_varlen(inp, cu))
+    check(inp, gpu, oracle_fwd(inp, cu=cu), torch.bfloat16, "tc wide-k varlen")
