@@ -81,6 +81,31 @@ def load_peaks():
         return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+def sources_hash():
+    """sha256[:16] of the CUDA sources, to tell whether a stored ncu capture still
+    describes the kernels that run."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "gated_linear_attention_local_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def captured_traffic(workload, kernel):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu capture
+    (profiles/traffic.json), or None when there is none or the sources changed since."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[workload][kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    if rec.get("sources_sha256_16") != sources_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def roofline(w, counts, kernel_ms, peaks, traffic=None):
     """Roofline object for the dominant kernel of this workload.  The fused output
     walk (or the decode kernel) moves all compulsory bytes of the call."""
@@ -447,7 +472,7 @@ def measure_workload(name, args, device, world, rank, peaks, steps, warmup, flus
                ms_p10=sorted(per_step)[len(per_step) // 10], ms_p90=sorted(per_step)[(9 * len(per_step)) // 10],
                tflops=counts["flops"] * (w["steps"] if w["kind"] == "decode" else 1) / (ms * 1e-3) / 1e12,
                gbs=counts["bytes"] * (w["steps"] if w["kind"] == "decode" else 1) / (ms * 1e-3) / 1e9,
-               roofline=roofline(w, counts, kernel_ms, peaks) if kname else None,
+               roofline=roofline(w, counts, kernel_ms, peaks, captured_traffic(name, kname)) if kname else None,
                dominant_kernel=dict(name=kname, launches=kn, avg_ms=kernel_ms,
                                     share=(kms / sum(v[1] for v in prof.values())) if prof else None),
                kernels={k: dict(launches=v[0], total_ms=round(v[1], 4)) for k, v in prof.items()},
