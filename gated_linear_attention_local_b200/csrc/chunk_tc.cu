@@ -190,7 +190,7 @@ struct WalkCfg {
     static constexpr int VROWB = 2 * BV;             // bytes per row of V, Vw, Hb
     static constexpr uint32_t VTILE = 128 * VROWB;   // V or Vw tile (128 tokens)
     static constexpr uint32_t HBB = HK * VROWB;      // Hb: HK rows (k) of BV values
-    static constexpr int NV = (KS == 1) ? 2 : 3;     // V ring stages
+    static constexpr int NV = 3;                     // V ring stages
     static constexpr uint32_t VLAYOUT = Sw<VROWB>::layout;
     static constexpr uint32_t VSBO = 8 * VROWB;      // 8-row group stride of V, Vw, Hb
     static constexpr uint32_t VKSTEP = 16 * VROWB;   // 16 rows: one MMA K step
@@ -198,8 +198,8 @@ struct WalkCfg {
     static constexpr uint32_t QK = 0;                // Q/K ring: Q slice (2 regions), K slice (2 regions)
     static constexpr uint32_t QK_STAGE = 4 * kRegion;
     static constexpr uint32_t VR = 2 * QK_STAGE;     // V ring
-    static constexpr uint32_t VW = VR + NV * VTILE;  // weighted V
-    static constexpr uint32_t HB = VW + VTILE;       // bf16 state copy, MN-major (rows k)
+    static constexpr uint32_t VW = VR + NV * VTILE;  // weighted V, 2 buffers (steps alternate)
+    static constexpr uint32_t HB = VW + 2 * VTILE;   // bf16 state copy, MN-major (rows k)
     static constexpr uint32_t GS = HB + HBB;         // gates, column factors, decay table
     static constexpr uint32_t BARS = GS + 3 * 128 * 4;
     static constexpr uint32_t MISC = BARS + 32 * 8;  // tmem address, abort flag
@@ -246,9 +246,9 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     uint64_t *b_pv = bars + 13;     // P V product of a step done
     uint64_t *b_p = bars + 14;      // P written (WG_A, 256 arrivals)
     uint64_t *b_hb = bars + 15;     // Hb written and H rescaled (WG_B, 128 arrivals)
-    uint64_t *b_vw = bars + 16;     // weighted V written (WG_B, 128 arrivals)
-    uint64_t *b_ofree = bars + 17;  // O1 / O2 of a step read out (WG_A, 256 arrivals)
-    uint64_t *b_drain = bars + 18;  // all MMAs retired
+    uint64_t *b_vw = bars + 16;     // [2] weighted V written, per Vw buffer (WG_B, 128 arrivals)
+    uint64_t *b_ofree = bars + 18;  // [2] O1 buffer (and O2) of a step read out (WG_A, 256 arrivals)
+    uint64_t *b_drain = bars + 20;  // all MMAs retired
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + C::MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + C::MISC + 8);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -267,8 +267,10 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         mbar_init(b_pv, 1);
         mbar_init(b_p, 256);
         mbar_init(b_hb, 128);
-        mbar_init(b_vw, 128);
-        mbar_init(b_ofree, 256);
+        mbar_init(&b_vw[0], 128);
+        mbar_init(&b_vw[1], 128);
+        mbar_init(&b_ofree[0], 256);
+        mbar_init(&b_ofree[1], 256);
         mbar_init(b_drain, 1);
         *abort_flag = 0;
         mbar_fence_init();
@@ -293,10 +295,9 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
 
     if (warp == 12) {
         // ------------------------------------------------------------ TMA producer
-        // K = 128: Q/K of step t reuse the stage of step t-2 once its K^T Vw retired,
-        // V of step t the stage of step t-2 once its P V retired (later): Q/K first.
-        // K > 128: V of step t goes first (its 3-stage ring frees early) so the slices
-        // of step t, which wait on the MMAs of earlier slices, never hold it back.
+        // V of step t goes first: its 3-stage ring frees when P V of step t-3 retires,
+        // long before the Q/K slices of step t (which wait on the MMAs of the slices
+        // two back) free up, so V never waits behind them.
         if (lane == 0) {
             prefetch_tmap(&tq);
             prefetch_tmap(&tk);
@@ -324,11 +325,10 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             };
             for (int t = 0; t < nsteps; ++t) {
                 const int tok = (int)(t0 + (int64_t)(cb + t) * kStep);
-                if (KS > 1 && !load_v(t, tok)) break;
+                if (!load_v(t, tok)) break;
                 bool ok = true;
                 for (int sl = 0; sl < KS && ok; ++sl) ok = load_qk(t * KS + sl, sl, tok);
                 if (!ok) break;
-                if (KS == 1 && !load_v(t, tok)) break;
             }
             if (*abort_flag) {  // let every copy still in flight land before the CTA exits
                 for (int q = max(0, qi - 2); q < qi; ++q) mbar_drain(&full_qk[q & 1], (q >> 1) & 1);
@@ -344,50 +344,64 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             const uint32_t sbase = smem_u32(sm);
             auto vdesc = [&](uint32_t addr) { return sdesc(addr, C::VSBO, C::VSBO, C::VLAYOUT); };
             auto qk_at = [&](int q) { return sbase + C::QK + (q & 1) * C::QK_STAGE; };
-            // S (+)= Q_s K_s^T   (both K-major; K steps of 16 inside 64-wide regions)
-            auto mma_S = [&](uint32_t q, uint32_t d, bool acc) {
+            const uint32_t o1_of[2] = {tmem + C::COL_O1, tmem + C::COL_O1 + BV};
+            const uint32_t s_of[2] = {tmem + C::COL_S, tmem + C::COL_S + 128};
+            // Consecutive MMAs into one accumulator are latency-bound (~200 cycles each
+            // whatever their width), so the independent products are interleaved: the
+            // S, O1 and H MMAs of the next step go round-robin one k step at a time, and
+            // the P V MMAs of the current step are slotted in between as soon as WG_A has
+            // written P.  The issuer polls every input without blocking.
+            // S, O1 and H of one k slice, interleaved
+            auto issue_slice = [&](int t, int sl) {
+                const int q = t * KS + sl;
+                const uint32_t qa = qk_at(q), ka = qa + 2 * kRegion;
+                const uint32_t vw = sbase + C::VW + (t & 1) * C::VTILE;
+                const uint32_t sd = s_of[t & 1], od = o1_of[t & 1], hd = tmem + C::COL_H + sl * BV;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
-                    mma_bf16(d, kdesc(q + off), kdesc(q + 2 * kRegion + off), idS, (acc || kk > 0) ? 1u : 0u);
+                    const uint32_t acc = (sl > 0 || kk > 0) ? 1u : 0u;
+                    mma_bf16(sd, kdesc(qa + off), kdesc(ka + off), idS, acc);
+                    mma_bf16(od, kdesc(qa + off), vdesc(sbase + C::HB + (uint32_t)(sl * 128 + kk * 16) * C::VROWB),
+                             idO, acc);
+                    mma_bf16(hd, sdesc(ka + kk * 2048, kRegion, 1024, 2), vdesc(vw + kk * C::VKSTEP), idH, 1);
                 }
+                mma_commit(&empty_qk[q & 1]);  // Q/K slice stage free once these retire
             };
-            // O1 (+)= Q_s Hb_s   (Hb MN-major, rows k: slice s holds rows 128 s ..)
-            auto mma_O1 = [&](uint32_t q, int sl, uint32_t d, bool acc) {
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
-                    mma_bf16(d, kdesc(q + off), vdesc(sbase + C::HB + (uint32_t)(sl * 128 + kk * 16) * C::VROWB), idO,
-                             (acc || kk > 0) ? 1u : 0u);
+            // inputs of step t's group (state pass, weighted V, O1 buffer, slice sl)
+            auto group_ready = [&](int t, int sl) -> bool {
+                if (!mbar_test(&full_qk[(t * KS + sl) & 1], ((t * KS + sl) >> 1) & 1)) return false;
+                if (sl > 0) return true;
+                return mbar_test(b_hb, t & 1) && mbar_test(&b_vw[t & 1], (t >> 1) & 1) &&
+                       (t < 2 || mbar_test(&b_ofree[t & 1], ((t >> 1) - 1) & 1));
+            };
+            bool ok = nsteps > 0;
+            // poll until `ready` holds; false on time-out or abort
+            auto poll = [&](auto &&ready) -> bool {
+                const uint64_t start = globaltimer_ns();
+                while (!ready()) {
+                    if (*abort_flag) return false;
+                    if (globaltimer_ns() - start > kWaitLimitNs) {
+                        *abort_flag = 1;
+                        return false;
+                    }
+                    __nanosleep(32);
                 }
-            };
-            // H_s += K_s^T Vw   (A = K read MN-major: two 64-wide k groups kRegion apart)
-            auto mma_H = [&](uint32_t q, int sl) {
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj)
-                    mma_bf16(tmem + C::COL_H + sl * BV, sdesc(q + 2 * kRegion + jj * 2048, kRegion, 1024, 2),
-                             vdesc(sbase + C::VW + jj * C::VKSTEP), idH, 1);
-            };
-            auto wait_hb_of = [&](int t) -> bool {
-                if (!mbar_wait(b_hb, t & 1, abort_flag)) return false;
-                if (t >= 2 && !mbar_wait(b_ofree, t & 1, abort_flag)) return false;  // O1 buffer t&1 read out
-                tc_fence_after();
                 return true;
             };
-            auto wait_vw = [&](int t) -> bool {
-                if (!mbar_wait(b_vw, t & 1, abort_flag)) return false;
-                tc_fence_after();
-                return true;
-            };
-            auto wait_qk = [&](int q) -> bool {
-                if (!mbar_wait(&full_qk[q & 1], (q >> 1) & 1, abort_flag)) return false;
-                tc_fence_after();
-                return true;
-            };
-            auto do_PV = [&](int t) -> bool {  // O2 = P V (P from TMEM, V MN-major)
-                if (!mbar_wait(b_p, t & 1, abort_flag)) return false;
-                if (!mbar_wait(&full_v[t % C::NV], (t / C::NV) & 1, abort_flag)) return false;
-                tc_fence_after();
+            // prologue: the group of step 0
+            for (int sl = 0; ok && sl < KS; ++sl) {
+                ok = poll([&] { return group_ready(0, sl); });
+                if (ok) {
+                    tc_fence_after();
+                    issue_slice(0, sl);
+                }
+            }
+            if (ok) {
+                mma_commit(&b_s[0]);
+                mma_commit(b_oh);
+            }
+            auto issue_PV = [&](int t) {
                 const uint32_t v = sbase + C::VR + (t % C::NV) * C::VTILE;
                 const uint32_t pt = tmem + C::COL_S + (t & 1) * 128;
 #pragma unroll
@@ -395,61 +409,33 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     mma_bf16_tmem_a(tmem + C::COL_O2, pt + jj * 8, vdesc(v + jj * C::VKSTEP), idO, jj > 0);
                 mma_commit(b_pv);
                 mma_commit(&empty_v[t % C::NV]);
-                return true;
             };
-            const uint32_t o1_of[2] = {tmem + C::COL_O1, tmem + C::COL_O1 + BV};
-            const uint32_t s_of[2] = {tmem + C::COL_S, tmem + C::COL_S + 128};
-            if constexpr (KS == 1) {
-                // order per iteration t: S(t+1), O1(t+1), P V(t), H(t+1)
-                auto do_S = [&](int t) -> bool {
-                    if (!wait_qk(t)) return false;
-                    mma_S(qk_at(t), s_of[t & 1], false);
-                    mma_commit(&b_s[t & 1]);
-                    return true;
-                };
-                auto do_O1 = [&](int t) -> bool {
-                    if (!wait_hb_of(t)) return false;
-                    mma_O1(qk_at(t), 0, o1_of[t & 1], false);
-                    return true;
-                };
-                auto do_H = [&](int t) -> bool {
-                    if (!wait_vw(t)) return false;
-                    mma_H(qk_at(t), 0);
-                    mma_commit(b_oh);              // WG_B may rewrite Hb, Vw and H
-                    mma_commit(&empty_qk[t & 1]);  // Q/K stage free
-                    return true;
-                };
-                if (nsteps > 0 && do_S(0) && do_O1(0) && do_H(0)) {
-                    for (int t = 0; t < nsteps; ++t) {
-                        const bool more = t + 1 < nsteps;
-                        if (more && !(do_S(t + 1) && do_O1(t + 1))) break;
-                        if (!do_PV(t)) break;
-                        if (more && !do_H(t + 1)) break;
+            for (int t = 0; ok && t < nsteps; ++t) {
+                const int tn = t + 1;
+                const bool more = tn < nsteps;
+                bool pv = false;
+                int sl = more ? 0 : KS;
+                const uint64_t start = globaltimer_ns();
+                while (!pv || sl < KS) {
+                    bool progress = false;
+                    if (!pv && mbar_test(b_p, t & 1) && mbar_test(&full_v[t % C::NV], (t / C::NV) & 1)) {
+                        tc_fence_after();
+                        issue_PV(t);
+                        pv = progress = true;
                     }
-                }
-            } else {
-                // per step: for each k slice S, O1 and H of that slice, then P V of the
-                // previous step
-                auto do_front = [&](int t) -> bool {
-                    for (int sl = 0; sl < KS; ++sl) {
-                        const int q = t * KS + sl;
-                        if (!wait_qk(q)) return false;
-                        const uint32_t qa = qk_at(q);
-                        mma_S(qa, s_of[t & 1], sl > 0);
-                        if (sl == KS - 1) mma_commit(&b_s[t & 1]);
-                        if (sl == 0 && !wait_hb_of(t)) return false;
-                        mma_O1(qa, sl, o1_of[t & 1], sl > 0);
-                        if (sl == 0 && !wait_vw(t)) return false;
-                        mma_H(qa, sl);
-                        mma_commit(&empty_qk[q & 1]);
+                    if (sl < KS && group_ready(tn, sl)) {
+                        tc_fence_after();
+                        issue_slice(tn, sl);
+                        if (++sl == KS) {
+                            mma_commit(&b_s[tn & 1]);
+                            mma_commit(b_oh);
+                        }
+                        progress = true;
                     }
-                    mma_commit(b_oh);
-                    return true;
-                };
-                if (nsteps > 0 && do_front(0)) {
-                    for (int t = 0; t < nsteps; ++t) {
-                        if (t + 1 < nsteps && !do_front(t + 1)) break;
-                        if (!do_PV(t)) break;
+                    if (!progress) {
+                        if (*abort_flag) { ok = false; break; }
+                        if (globaltimer_ns() - start > kWaitLimitNs) { *abort_flag = 1; ok = false; break; }
+                        __nanosleep(32);
                     }
                 }
             }
@@ -482,28 +468,33 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         const bool gamma_pos = a.gate_mode == kGatePerHead && a.g_gamma[h] > 0.f;
         const int64_t chunk0 = (lay.cu ? (int64_t)lay.chunk_off[n] : (int64_t)n * lay.NT) + cb;
         // gate, column factor and "holds a positive gate" flag of local step t for this row
-        auto load_step = [&](int t, float &g_out, float &f_out, bool &pos_out) {
+        // gate, reference gate of its 32-column tile and "holds a positive gate" flag of
+        // local step t for this row; issued a step ahead, consumed after the P pass
+        auto load_step = [&](int t, float &g_out, float &gr_out, bool &pos_out) {
             const StepSpan sp = step_span(t0, t1, cb + t);
             g_out = (i < sp.len) ? chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + i, i, h, H) : 0.f;
             const int r = min((i | 31), sp.len - 1);
-            const float gr = chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + r, r, h, H);
-            f_out = (i < sp.len) ? fast_exp2(fminf(gr - g_out, 0.f)) : 0.f;
+            gr_out = chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + r, r, h, H);
             pos_out = per_token ? (a.gpos[(chunk0 + t) * H + h] != 0) : gamma_pos;
         };
-        float gi, fi;
+        auto factor = [&](int t, float g, float gr) -> float {
+            return (i < step_span(t0, t1, cb + t).len) ? fast_exp2(fminf(gr - g, 0.f)) : 0.f;
+        };
+        float gi, gri;
         bool pos;
-        load_step(0, gi, fi, pos);
+        load_step(0, gi, gri, pos);
         if (half == 0) {
             gs[i] = gi;
-            fs[i] = fi;
+            fs[i] = factor(0, gi, gri);
         }
         named_sync(1, 256);
         TR_DECL(a_ws); TR_DECL(a_p); TR_DECL(a_wpv); TR_DECL(a_out);
         for (int t = 0; t < nsteps; ++t) {
             const StepSpan sp = step_span(t0, t1, cb + t);
-            float gnext = 0.f, fnext = 0.f;
+            float gnext = 0.f, grnext = 0.f;
             bool posnext = false;
-            if (t + 1 < nsteps) load_step(t + 1, gnext, fnext, posnext);  // in flight during the step
+            if (t + 1 < nsteps) load_step(t + 1, gnext, grnext, posnext);  // in flight during the step
+            const float fnext = (t + 1 < nsteps) ? factor(t + 1, gnext, grnext) : 0.f;
 
             { TR_T0(x0); mbar_wait(&b_s[t & 1], (t >> 1) & 1, abort_flag); TR_ACC(a_ws, x0); }
             TR_T0(xp);
@@ -594,7 +585,7 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 }
             }
             tc_fence_before();
-            mbar_arrive(b_ofree);
+            mbar_arrive(&b_ofree[t & 1]);
             TR_ACC(a_out, xo);
             named_sync(1, 256);  // next step's gates and factors are in place
             gi = gnext;
@@ -603,11 +594,13 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         if (threadIdx.x == 96) { TR_STORE(12, a_ws); TR_STORE(13, a_p); TR_STORE(15, a_wpv); TR_STORE(16, a_out); TR_STORE(1, nsteps); }
     } else {
         // ------------------------------------------------------------ WG_B: V weights and state
+        // The weighted V of step t+2 is prepared right after the state pass of step t
+        // (Vw is double-buffered), so only the state pass sits on the step-to-step
+        // chain; gates are loaded two steps before they are used.
         const int i = threadIdx.x - 256;  // token i of V; row 128 b + i of H, block b
         const uint32_t trow = tmem + ((uint32_t)((warp - 8) * 32) << 16);
         unsigned char *hb = sm + C::HB;
         const int64_t KV = (int64_t)C::HK * V;
-        float gi = gate_at(0, i), glast = last_gate(0);
 
         // moves BV fp32 values between a state row in TMEM block b and registers
         auto h_ld = [&](int b, float (&x)[BV]) {
@@ -635,13 +628,25 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             for (int c = 0; c < BV / 32; ++c)
                 store_row32_bf16<C::VROWB>(hb, 128 * b + i, 32 * c, *reinterpret_cast<const float(*)[32]>(&x[32 * c]));
         };
+        // weighted V rows of step k: Vw_j = 2^(G~_last - G~_j) v_j (0 past the sequence end)
+        auto weigh_v = [&](int k, float gk, float lk) {
+            const StepSpan sp = step_span(t0, t1, cb + k);
+            mbar_wait(&full_v[k % C::NV], (k / C::NV) & 1, abort_flag);
+            scale_row<C::VROWB>(sm + C::VR + (k % C::NV) * C::VTILE, sm + C::VW + (k & 1) * C::VTILE, i,
+                                (i < sp.len) ? fast_exp2(lk - gk) : 0.f);
+            fence_proxy_async_smem();
+            mbar_arrive(&b_vw[k & 1]);
+        };
+        auto gate_or0 = [&](int k) { return k < nsteps ? gate_at(k, i) : 0.f; };
+        auto last_or0 = [&](int k) { return k < nsteps ? last_gate(k) : 0.f; };
 
+        const float g0 = gate_or0(0), l0 = last_or0(0), g1 = gate_or0(1), l1 = last_or0(1);
         // state entering the segment -> Hb (bf16) and TMEM (times the first step's decay)
         {
             const float *src = nullptr;
             if (s == 0) src = a.h0 ? a.h0 + ((int64_t)n * H + h) * KV : nullptr;
             else src = a.seg_state + ((int64_t)(u - 1) * H + h) * KV;
-            const float gam = exp2f(glast);
+            const float gam = exp2f(l0);
 #pragma unroll 1
             for (int b = 0; b < KS; ++b) {
                 float x[BV];
@@ -666,28 +671,21 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             tc_fence_before();
             mbar_arrive(b_hb);
         }
+        if (nsteps > 0) weigh_v(0, g0, l0);
+        if (nsteps > 1) weigh_v(1, g1, l1);
 
+        float lnext = l1;                             // G~_last of step t+1 (rescale of the state pass)
+        float g2 = gate_or0(2), l2 = last_or0(2);     // gates of step t+2 (its weighted V)
         TR_DECL(b_sv); TR_DECL(b_woh); TR_DECL(b_hp);
         for (int t = 0; t < nsteps; ++t) {
-            const StepSpan sp = step_span(t0, t1, cb + t);
-            const bool more = t + 1 < nsteps;
-            const float gnext = more ? gate_at(t + 1, i) : 0.f;  // in flight during the step
-            const float glnext = more ? last_gate(t + 1) : 0.f;
-            // weighted V rows: Vw_j = 2^(G~_last - G~_j) v_j (0 past the end of the sequence)
-            mbar_wait(&full_v[t % C::NV], (t / C::NV) & 1, abort_flag);
-            TR_T0(xv);
-            scale_row<C::VROWB>(sm + C::VR + (t % C::NV) * C::VTILE, sm + C::VW, i,
-                                (i < sp.len) ? fast_exp2(glast - gi) : 0.f);
-            fence_proxy_async_smem();
-            mbar_arrive(b_vw);
-            TR_ACC(b_sv, xv);
+            const float g3 = gate_or0(t + 3), l3 = last_or0(t + 3);  // in flight for the next step
 
             // state: Hb <- bf16(H_{t+1}); H <- 2^G~_last(t+1) H_{t+1}; or the final state
             { TR_T0(x0); mbar_wait(b_oh, t & 1, abort_flag); TR_ACC(b_woh, x0); }
             TR_T0(xh);
             tc_fence_after();
-            if (more) {
-                const float gam = exp2f(glnext);
+            if (t + 1 < nsteps) {
+                const float gam = exp2f(lnext);
 #pragma unroll 1
                 for (int b = 0; b < KS; ++b) {
                     float x[BV];
@@ -717,8 +715,13 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 }
             }
             TR_ACC(b_hp, xh);
-            gi = gnext;
-            glast = glnext;
+            // weighted V of step t+2 into the buffer step t just released
+            TR_T0(xv);
+            if (t + 2 < nsteps) weigh_v(t + 2, g2, l2);
+            TR_ACC(b_sv, xv);
+            lnext = l2;
+            g2 = g3;
+            l2 = l3;
         }
         if (i == 0) { TR_STORE(19, b_sv); TR_STORE(20, b_woh); TR_STORE(21, b_hp); }
     }
