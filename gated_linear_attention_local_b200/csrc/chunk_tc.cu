@@ -344,19 +344,18 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             const uint32_t sbase = smem_u32(sm);
             auto vdesc = [&](uint32_t addr) { return sdesc(addr, C::VSBO, C::VSBO, C::VLAYOUT); };
             auto qk_at = [&](int q) { return sbase + C::QK + (q & 1) * C::QK_STAGE; };
-            const uint32_t o1_of[2] = {tmem + C::COL_O1, tmem + C::COL_O1 + BV};
-            const uint32_t s_of[2] = {tmem + C::COL_S, tmem + C::COL_S + 128};
             // Consecutive MMAs into one accumulator are latency-bound (~200 cycles each
-            // whatever their width), so the independent products are interleaved: the
-            // S, O1 and H MMAs of the next step go round-robin one k step at a time, and
-            // the P V MMAs of the current step are slotted in between as soon as WG_A has
-            // written P.  The issuer polls every input without blocking.
+            // whatever their width), so the three independent products of a step -- S,
+            // O1 and H -- go round-robin one k step at a time, a 128-wide k slice per
+            // call.  P V of the current step (its own chain) is issued as soon as WG_A
+            // has written P; the issuer polls both without blocking.
             // S, O1 and H of one k slice, interleaved
             auto issue_slice = [&](int t, int sl) {
                 const int q = t * KS + sl;
                 const uint32_t qa = qk_at(q), ka = qa + 2 * kRegion;
                 const uint32_t vw = sbase + C::VW + (t & 1) * C::VTILE;
-                const uint32_t sd = s_of[t & 1], od = o1_of[t & 1], hd = tmem + C::COL_H + sl * BV;
+                const uint32_t sd = tmem + C::COL_S + (t & 1) * 128, od = tmem + C::COL_O1 + (t & 1) * BV;
+                const uint32_t hd = tmem + C::COL_H + sl * BV;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
@@ -466,8 +465,8 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             tab[i] = exp2f((float)i * gam);
         }
         const bool gamma_pos = a.gate_mode == kGatePerHead && a.g_gamma[h] > 0.f;
+        const bool o32 = (reinterpret_cast<uintptr_t>(a.o) & 31) == 0;  // 32-byte row segments
         const int64_t chunk0 = (lay.cu ? (int64_t)lay.chunk_off[n] : (int64_t)n * lay.NT) + cb;
-        // gate, column factor and "holds a positive gate" flag of local step t for this row
         // gate, reference gate of its 32-column tile and "holds a positive gate" flag of
         // local step t for this row; issued a step ahead, consumed after the P pass
         auto load_step = [&](int t, float &g_out, float &gr_out, bool &pos_out) {
@@ -487,14 +486,22 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             gs[i] = gi;
             fs[i] = factor(0, gi, gri);
         }
+        float g1 = 0.f, gr1 = 0.f;  // loads of step t+1, issued a step before their use
+        bool pos1 = false;
+        if (nsteps > 1) load_step(1, g1, gr1, pos1);
         named_sync(1, 256);
         TR_DECL(a_ws); TR_DECL(a_p); TR_DECL(a_wpv); TR_DECL(a_out);
         for (int t = 0; t < nsteps; ++t) {
             const StepSpan sp = step_span(t0, t1, cb + t);
-            float gnext = 0.f, grnext = 0.f;
-            bool posnext = false;
-            if (t + 1 < nsteps) load_step(t + 1, gnext, grnext, posnext);  // in flight during the step
-            const float fnext = (t + 1 < nsteps) ? factor(t + 1, gnext, grnext) : 0.f;
+            float g2 = 0.f, gr2 = 0.f;
+            bool pos2 = false;
+            if (t + 2 < nsteps) load_step(t + 2, g2, gr2, pos2);  // in flight for two steps
+            const float gnext = g1;
+            const bool posnext = pos1;
+            const float fnext = (t + 1 < nsteps) ? factor(t + 1, g1, gr1) : 0.f;
+            g1 = g2;
+            gr1 = gr2;
+            pos1 = pos2;
 
             { TR_T0(x0); mbar_wait(&b_s[t & 1], (t >> 1) & 1, abort_flag); TR_ACC(a_ws, x0); }
             TR_T0(xp);
@@ -574,18 +581,24 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     tmem_ld16f(trow + C::COL_O2 + OW * half, oy);
                 }
                 tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&b_ofree[t & 1]);  // O1 and O2 of this step are in registers
+                uint32_t w[OW / 2];
 #pragma unroll
-                for (int e = 0; e < OW; ++e) ox[e] = fmaf(ei, ox[e], a.scale * oy[e]);
+                for (int e = 0; e < OW / 2; ++e)
+                    w[e] = pack_bf16(fmaf(ei, ox[2 * e], a.scale * oy[2 * e]), fmaf(ei, ox[2 * e + 1], a.scale * oy[2 * e + 1]));
                 if (i < sp.len && !*abort_flag) {
-                    uint4 *d = reinterpret_cast<uint4 *>(orow);
+                    if (o32) {  // one 32-byte store per 16 values
 #pragma unroll
-                    for (int q = 0; q < OW / 8; ++q)
-                        d[q] = make_uint4(pack_bf16(ox[8 * q], ox[8 * q + 1]), pack_bf16(ox[8 * q + 2], ox[8 * q + 3]),
-                                          pack_bf16(ox[8 * q + 4], ox[8 * q + 5]), pack_bf16(ox[8 * q + 6], ox[8 * q + 7]));
+                        for (int q = 0; q < OW / 16; ++q)
+                            st_global_v8(orow + 16 * q, *reinterpret_cast<const uint32_t(*)[8]>(&w[8 * q]));
+                    } else {
+                        uint4 *d = reinterpret_cast<uint4 *>(orow);
+#pragma unroll
+                        for (int q = 0; q < OW / 8; ++q) d[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                    }
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&b_ofree[t & 1]);
             TR_ACC(a_out, xo);
             named_sync(1, 256);  // next step's gates and factors are in place
             gi = gnext;
@@ -602,31 +615,12 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         unsigned char *hb = sm + C::HB;
         const int64_t KV = (int64_t)C::HK * V;
 
-        // moves BV fp32 values between a state row in TMEM block b and registers
-        auto h_ld = [&](int b, float (&x)[BV]) {
-            if constexpr (BV == 64) {
-                float (&x0)[32] = *reinterpret_cast<float(*)[32]>(&x[0]);
-                float (&x1)[32] = *reinterpret_cast<float(*)[32]>(&x[32]);
-                tmem_ld32(trow + C::COL_H + b * BV, x0);
-                tmem_ld32(trow + C::COL_H + b * BV + 32, x1);
-            } else {
-                tmem_ld32(trow + C::COL_H + b * BV, x);
-            }
-        };
-        auto h_st = [&](int b, const float (&x)[BV]) {
-            if constexpr (BV == 64) {
-                const float (&x0)[32] = *reinterpret_cast<const float(*)[32]>(&x[0]);
-                const float (&x1)[32] = *reinterpret_cast<const float(*)[32]>(&x[32]);
-                tmem_st32(trow + C::COL_H + b * BV, x0);
-                tmem_st32(trow + C::COL_H + b * BV + 32, x1);
-            } else {
-                tmem_st32(trow + C::COL_H + b * BV, x);
-            }
-        };
-        auto hb_row = [&](int b, const float (&x)[BV]) {  // bf16 copy of state row 128 b + i
-#pragma unroll
-            for (int c = 0; c < BV / 32; ++c)
-                store_row32_bf16<C::VROWB>(hb, 128 * b + i, 32 * c, *reinterpret_cast<const float(*)[32]>(&x[32 * c]));
+        // A state row (row 128 b + i of H, BV columns) is handled in 32-column pieces:
+        // piece p of block b lives at TMEM column COL_H + b BV + 32 p.
+        constexpr int NP = BV / 32;
+        auto h_col = [&](int b, int pc) { return trow + C::COL_H + b * BV + 32 * pc; };
+        auto hb_piece = [&](int b, int pc, const float (&x)[32]) {  // bf16 copy into Hb
+            store_row32_bf16<C::VROWB>(hb, 128 * b + i, 32 * pc, x);
         };
         // weighted V rows of step k: Vw_j = 2^(G~_last - G~_j) v_j (0 past the sequence end)
         auto weigh_v = [&](int k, float gk, float lk) {
@@ -649,22 +643,26 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             const float gam = exp2f(l0);
 #pragma unroll 1
             for (int b = 0; b < KS; ++b) {
-                float x[BV];
-                if (src) {
-                    const float4 *p4 = reinterpret_cast<const float4 *>(src + (int64_t)(128 * b + i) * V + v0);
+#pragma unroll 1
+                for (int pc = 0; pc < NP; ++pc) {
+                    float x[32];
+                    if (src) {
+                        const float4 *p4 =
+                            reinterpret_cast<const float4 *>(src + (int64_t)(128 * b + i) * V + v0 + 32 * pc);
 #pragma unroll
-                    for (int e = 0; e < BV / 4; ++e) {
-                        const float4 f = p4[e];
-                        x[4 * e] = f.x; x[4 * e + 1] = f.y; x[4 * e + 2] = f.z; x[4 * e + 3] = f.w;
+                        for (int e = 0; e < 8; ++e) {
+                            const float4 f = p4[e];
+                            x[4 * e] = f.x; x[4 * e + 1] = f.y; x[4 * e + 2] = f.z; x[4 * e + 3] = f.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) x[e] = 0.f;
                     }
-                } else {
+                    hb_piece(b, pc, x);
 #pragma unroll
-                    for (int e = 0; e < BV; ++e) x[e] = 0.f;
+                    for (int e = 0; e < 32; ++e) x[e] *= gam;
+                    tmem_st32(h_col(b, pc), x);
                 }
-                hb_row(b, x);
-#pragma unroll
-                for (int e = 0; e < BV; ++e) x[e] *= gam;
-                h_st(b, x);
             }
             tmem_wait_st();
             fence_proxy_async_smem();
@@ -688,13 +686,16 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 const float gam = exp2f(lnext);
 #pragma unroll 1
                 for (int b = 0; b < KS; ++b) {
-                    float x[BV];
-                    h_ld(b, x);
-                    tmem_wait_ld();
-                    hb_row(b, x);
 #pragma unroll
-                    for (int e = 0; e < BV; ++e) x[e] *= gam;
-                    h_st(b, x);
+                    for (int pc = 0; pc < NP; ++pc) {
+                        float x[32];
+                        tmem_ld32(h_col(b, pc), x);
+                        tmem_wait_ld();
+                        hb_piece(b, pc, x);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) x[e] *= gam;
+                        tmem_st32(h_col(b, pc), x);
+                    }
                 }
                 tmem_wait_st();
                 fence_proxy_async_smem();
@@ -703,14 +704,18 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             } else if (last_seg && a.hT) {
 #pragma unroll 1
                 for (int b = 0; b < KS; ++b) {
-                    float x[BV];
-                    h_ld(b, x);
-                    tmem_wait_ld();
-                    if (!*abort_flag) {
-                        float4 *d4 = reinterpret_cast<float4 *>(a.hT + ((int64_t)n * H + h) * KV +
-                                                                (int64_t)(128 * b + i) * V + v0);
+#pragma unroll 1
+                    for (int pc = 0; pc < NP; ++pc) {
+                        float x[32];
+                        tmem_ld32(h_col(b, pc), x);
+                        tmem_wait_ld();
+                        if (!*abort_flag) {
+                            float4 *d4 = reinterpret_cast<float4 *>(a.hT + ((int64_t)n * H + h) * KV +
+                                                                    (int64_t)(128 * b + i) * V + v0 + 32 * pc);
 #pragma unroll
-                        for (int e = 0; e < BV / 4; ++e) d4[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+                            for (int e = 0; e < 8; ++e)
+                                d4[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+                        }
                     }
                 }
             }
