@@ -455,8 +455,24 @@ def measure_workload(name, args, device, world, rank, peaks, steps, warmup, flus
     d = dev_inputs(w, device)
     ws = workspace_for(w, sg, device)
     step, reset = make_step(w, d, sg, ws)
+    timing = "eager launches"
     with ClockSampler(device) as clk:
         per_step, prof, launches = time_steps(step, reset, steps, warmup, flush, world > 1)
+        if w["kind"] == "decode":
+            # the 64 consecutive decode steps of a call are timed as one CUDA graph; the
+            # eager pass above supplies the per-kernel times
+            from gated_linear_attention_local_b200 import _lib
+            graph = torch.cuda.CUDAGraph()
+            reset()
+            torch.cuda.synchronize()
+            n0 = _lib.kernel_launch_count()
+            with torch.cuda.graph(graph):
+                step()
+            per_graph = _lib.kernel_launch_count() - n0
+            per_step, _, _ = time_steps(graph.replay, reset, steps, warmup, flush, world > 1, profile=False)
+            launches = per_graph * steps
+            timing = f"one CUDA graph of {per_graph} decode-step launches per call"
+            del graph
     total_ms = max_over_ranks(sum(per_step), world, device)
     ms = total_ms / steps
     counts = algorithmic_counts(w)
@@ -476,7 +492,7 @@ def measure_workload(name, args, device, world, rank, peaks, steps, warmup, flus
                dominant_kernel=dict(name=kname, launches=kn, avg_ms=kernel_ms,
                                     share=(kms / sum(v[1] for v in prof.values())) if prof else None),
                kernels={k: dict(launches=v[0], total_ms=round(v[1], 4)) for k, v in prof.items()},
-               gpu_launches=launches, clocks=clk.summary(), config=dict(workload=name, **_config_of(w)),
+               gpu_launches=launches, clocks=clk.summary(), config=dict(workload=name, timing=timing, **_config_of(w)),
                dtype=w["dtype_name"])
     # whole-call roofline fraction (all kernels, launches included)
     t_roof = max(counts["bytes"] / (peaks["hbm_gbs"] * 1e9), counts["flops"] / (peaks["bf16_tflops"] * 1e12))
