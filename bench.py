@@ -66,6 +66,8 @@ def algorithmic_counts(w):
     if w["output_final_state"]:
         b += states
     flops = H * (4 * tokens * K * V + tokens * (C + 1) * (K + V))
+    if w.get("entry") == "recurrent":  # token-serial: state update and read-out per token
+        flops = H * tokens * 4 * K * V
     return dict(bytes=b, flops=flops, tokens=tokens)
 
 
@@ -106,9 +108,20 @@ def captured_traffic(workload, kernel):
     return rec.get("dram_bytes_per_launch")
 
 
+# FP32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 flops (FMA) x 1965 MHz max SM clock
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def roofline(w, counts, kernel_ms, peaks, traffic=None):
     """Roofline object for the dominant kernel of this workload.  The fused output
-    walk (or the decode kernel) moves all compulsory bytes of the call."""
+    walk (or the decode kernel) moves all compulsory bytes of the call.  The
+    token-serial recurrence runs on the FP32 CUDA cores (two FMAs and a multiply per
+    state element and token), so its bound is the ALU peak."""
+    if w.get("entry") == "recurrent":
+        ach = counts["flops"] / (kernel_ms * 1e-3) / 1e12
+        return dict(bound="alu", achieved=round(ach, 3), peak=round(FP32_ALU_TFLOPS, 1), unit="TFLOP/s",
+                    frac=round(ach / FP32_ALU_TFLOPS, 4), traffic=traffic,
+                    peak_source="derived: 148 SMs x 128 FP32 lanes x 2 x 1965 MHz")
     t_bytes = counts["bytes"] / (peaks["hbm_gbs"] * 1e9)
     t_flops = counts["flops"] / (peaks["bf16_tflops"] * 1e12)
     if w["kind"] != "decode" and w.get("dtype_name") == "fp32":
@@ -208,6 +221,11 @@ def make_step(w, d, sg, ws):
                 sg.simple_gla_decode_step(d["q"][t], d["k"][t], d["v"][t], d["state"], g=d["g"][t],
                                           scale=w["scale"], out=o)
         return step, reset
+    if w.get("entry") == "recurrent":
+        def step():
+            sg.simple_gla_fused_recurrent(d["q"], d["k"], d["v"], g=d["g"], g_gamma=d["g_gamma"], scale=w["scale"],
+                                          initial_state=d["h0"], output_final_state=w["output_final_state"])
+        return step, (lambda: None)
     if w["kind"] == "varlen":
         def step():
             sg.simple_gla_fwd_varlen(d["q"], d["k"], d["v"], d["cu_seqlens"], g=d["g"], g_gamma=d["g_gamma"],
@@ -223,7 +241,7 @@ def make_step(w, d, sg, ws):
 
 
 def workspace_for(w, sg, device):
-    if w["kind"] == "decode":
+    if w["kind"] == "decode" or w.get("entry") == "recurrent":
         return None
     dt = w["q"].dtype
     if w["kind"] == "varlen":
@@ -303,6 +321,10 @@ def e2e_measure(w, sg, device, steps, warmup):
                                              g_gamma=g_gamma, scale=w["scale"], initial_state=d.get("h0"),
                                              output_final_state=w["output_final_state"],
                                              chunk_size=w["chunk_size"], workspace=ws)
+        elif w.get("entry") == "recurrent":
+            o, ht = sg.simple_gla_fused_recurrent(d["q"], d["k"], d["v"], g=d.get("g"), g_gamma=g_gamma,
+                                                  scale=w["scale"], initial_state=d.get("h0"),
+                                                  output_final_state=w["output_final_state"])
         else:
             o, ht = sg.simple_gla_fwd(d["q"], d["k"], d["v"], g=d.get("g"), g_gamma=g_gamma, scale=w["scale"],
                                       initial_state=d.get("h0"), output_final_state=w["output_final_state"],
@@ -438,6 +460,9 @@ def reference_arm(args, world, rank):
 def _config_of(w):
     if w["kind"] == "decode":
         return dict(N=w["N"], steps_per_call=w["steps"], H=w["H"], K=w["K"], V=w["V"], state="fp32")
+    if w.get("entry") == "recurrent":
+        return dict(entry="simple_gla_fused_recurrent", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
+                    gate="g" if w["g"] is not None else "none", initial_state=w["h0"] is not None)
     c = dict(H=w["H"], K=w["K"], V=w["V"], chunk_size=w["chunk_size"],
              gate="g" if w["g"] is not None else ("g_gamma" if w["g_gamma"] is not None else "none"))
     if w["kind"] == "varlen":

@@ -17,8 +17,13 @@ Public functions (same names as the C entry points):
   simple_gla_fwd(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
                  output_final_state=False, chunk_size=64) -> (o, final_state|None)
   simple_gla_fwd_varlen(q, k, v, cu_seqlens, g=None, ...) -> (o, final_state|None)
-  simple_gla_decode_step(q, k, v, state, g=None, g_gamma=None, scale=None) -> o
+  simple_gla_decode_step(q, k, v, state, g=None, g_gamma=None, scale=None,
+                         state_v_first=False) -> o
+  simple_gla_fused_recurrent(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
+                             output_final_state=False, cu_seqlens=None,
+                             state_v_first=False) -> (o, final_state|None)
   chunk_simple_gla(...)  -- the article's entry-point name; dispatches on cu_seqlens.
+  fused_recurrent_simple_gla(...) -- the article's name for simple_gla_fused_recurrent.
 """
 from __future__ import annotations
 
@@ -31,6 +36,7 @@ from ._lib import (SGLA_BF16, SGLA_FP32, SGLA_OK, SglaError, lib, library_path, 
                    raise_for_status)
 
 __all__ = ["simple_gla_fwd", "simple_gla_fwd_noalloc", "simple_gla_fwd_varlen", "simple_gla_decode_step", "chunk_simple_gla",
+           "simple_gla_fused_recurrent", "fused_recurrent_simple_gla",
            "fwd_workspace_size", "varlen_workspace_size", "workspace_status", "library_path",
            "SglaError"]
 
@@ -197,28 +203,98 @@ def chunk_simple_gla(q, k, v, g=None, g_gamma=None, scale=None, initial_state=No
                                  output_final_state, chunk_size)
 
 
-def simple_gla_decode_step(q, k, v, state, g=None, g_gamma=None, scale=None, out=None):
+def simple_gla_decode_step(q, k, v, state, g=None, g_gamma=None, scale=None, out=None, state_v_first=False):
     """One recurrent step.  q,k [N,H,K]; v [N,H,V]; g [N,H] fp32 or g_gamma [H];
-    state [N,H,K,V] fp32 updated in place.  Returns o [N,H,V]."""
+    state [N,H,K,V] fp32 ([N,H,V,K] with state_v_first) updated in place.  Returns
+    o [N,H,V].  The [V,K] layout runs as a one-token simple_gla_fused_recurrent."""
     _common_checks(q, k, v, g, g_gamma, None)
     _check_cuda("state", state, torch.float32, 4)
     if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
         raise ValueError("q,k must be [N,H,K] and v [N,H,V]")
     N, H, K = q.shape
     V = v.shape[2]
-    if tuple(state.shape) != (N, H, K, V):
-        raise ValueError(f"state must be [N,H,K,V] = {(N, H, K, V)}")
+    want = (N, H, V, K) if state_v_first else (N, H, K, V)
+    if tuple(state.shape) != want:
+        raise ValueError(f"state must be {'[N,H,V,K]' if state_v_first else '[N,H,K,V]'} = {want}")
     if g is not None and tuple(g.shape) != (N, H):
         raise ValueError("g must be [N,H]")
     if g_gamma is not None and tuple(g_gamma.shape) != (H,):
         raise ValueError("g_gamma must be [H]")
     o = out if out is not None else torch.empty((N, H, V), dtype=q.dtype, device=q.device)
     _check_cuda("out", o, q.dtype, 3)
+    if state_v_first:
+        st = lib().simple_gla_fused_recurrent(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma),
+                                              ctypes.c_float(_scale(scale)), _ptr(state), _ptr(o), _ptr(state),
+                                              None, N, 1, H, K, V, 1, _DTYPES[q.dtype], None, _stream())
+        raise_for_status(st, "simple_gla_fused_recurrent")
+        return o
     st = lib().simple_gla_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma),
                                       ctypes.c_float(_scale(scale)), _ptr(state), _ptr(o), N, H, K, V,
                                       _DTYPES[q.dtype], _stream())
     raise_for_status(st, "simple_gla_decode_step")
     return o
+
+
+def simple_gla_fused_recurrent(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
+                               output_final_state=False, cu_seqlens=None, state_v_first=False,
+                               device_status=None):
+    """Token-serial recurrence with the state held on chip for the whole sequence.
+
+    Dense: q,k [B,T,H,K], v [B,T,H,V], g [B,T,H].  Packed (cu_seqlens int64 [N+1] on
+    the device): q,k [1,T,H,K] or [T,H,K] and likewise v, g.  initial_state /
+    final_state [N,H,K,V] fp32, [N,H,V,K] with state_v_first.  device_status: optional
+    int32 CUDA tensor of one element that receives the cu_seqlens check.
+    Returns (o shaped like v, final_state|None)."""
+    _common_checks(q, k, v, g, g_gamma, None)
+    _check_cuda("initial_state", initial_state, torch.float32, 4)
+    squeeze = False
+    if cu_seqlens is not None:
+        _check_cuda("cu_seqlens", cu_seqlens, torch.int64, 1)
+        if q.dim() == 4:
+            if q.shape[0] != 1:
+                raise ValueError("with cu_seqlens the batch dimension must be 1")
+            squeeze = True
+            q, k, v = q[0], k[0], v[0]
+            g = g[0] if g is not None else None
+        if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+            raise ValueError("q,k must be [T,H,K] and v [T,H,V] with cu_seqlens")
+        N = cu_seqlens.numel() - 1
+        if N < 1:
+            raise ValueError("cu_seqlens needs at least two entries")
+        T, H, K = q.shape
+        V = v.shape[2]
+        if g is not None and tuple(g.shape) != (T, H):
+            raise ValueError(f"g must be [T,H] = {(T, H)}")
+    else:
+        if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+            raise ValueError("q,k must be [B,T,H,K] and v [B,T,H,V]")
+        N, T, H, K = q.shape
+        V = v.shape[3]
+        if g is not None and tuple(g.shape) != (N, T, H):
+            raise ValueError(f"g must be [B,T,H] = {(N, T, H)}")
+    if g_gamma is not None and tuple(g_gamma.shape) != (H,):
+        raise ValueError(f"g_gamma must be [H] = ({H},)")
+    sshape = (N, H, V, K) if state_v_first else (N, H, K, V)
+    if initial_state is not None and tuple(initial_state.shape) != sshape:
+        raise ValueError(f"initial_state must be {sshape}")
+    if device_status is not None:
+        _check_cuda("device_status", device_status, torch.int32)
+    o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    ht = torch.empty(sshape, dtype=torch.float32, device=q.device) if output_final_state else None
+    st = lib().simple_gla_fused_recurrent(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma),
+                                          ctypes.c_float(_scale(scale)), _ptr(initial_state), _ptr(o), _ptr(ht),
+                                          _ptr(cu_seqlens), N, T, H, K, V, 1 if state_v_first else 0,
+                                          _DTYPES[q.dtype], _ptr(device_status), _stream())
+    raise_for_status(st, "simple_gla_fused_recurrent")
+    return (o.unsqueeze(0) if squeeze else o), ht
+
+
+def fused_recurrent_simple_gla(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
+                               output_final_state=False, cu_seqlens=None, state_v_first=False):
+    """The article's name (section 2) for simple_gla_fused_recurrent."""
+    return simple_gla_fused_recurrent(q, k, v, g=g, g_gamma=g_gamma, scale=scale, initial_state=initial_state,
+                                      output_final_state=output_final_state, cu_seqlens=cu_seqlens,
+                                      state_v_first=state_v_first)
 
 
 def workspace_status(workspace) -> int:

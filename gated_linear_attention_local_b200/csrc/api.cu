@@ -314,6 +314,40 @@ sgla_status simple_gla_decode_step(const void *q, const void *k, const void *v, 
     return SGLA_OK;
 }
 
+sgla_status simple_gla_fused_recurrent(const void *q, const void *k, const void *v, const float *g,
+                                       const float *g_gamma, float scale, const float *initial_state, void *o,
+                                       float *final_state, const int64_t *cu_seqlens, int64_t N, int64_t T,
+                                       int64_t H, int64_t K, int64_t V, int state_v_first, sgla_dtype dtype,
+                                       int *device_status, void *stream) {
+    if (g && g_gamma) return SGLA_ERR_INVALID_ARGUMENT;
+    if (N < 0 || T < 0 || H < 1 || K < 1 || V < 1) return SGLA_ERR_INVALID_ARGUMENT;
+    if (cu_seqlens && N < 1) return SGLA_ERR_INVALID_ARGUMENT;
+    if (dtype != SGLA_BF16 && dtype != SGLA_FP32) return SGLA_ERR_INVALID_ARGUMENT;
+    const int epc = dtype == SGLA_BF16 ? 8 : 4;  // elements per 16-byte copy
+    if (K > (dtype == SGLA_BF16 ? 512 : 256) || V > 4096 || K % epc || V % epc) return SGLA_ERR_UNSUPPORTED;
+    const int64_t tokens = cu_seqlens ? T : N * T;
+    if (tokens >= kMaxTokens || N * H >= kMaxTokens) return SGLA_ERR_UNSUPPORTED;
+    if (tokens > 0 && (!q || !k || !v || !o)) return SGLA_ERR_INVALID_ARGUMENT;
+    for (const void *p : {q, k, v})
+        if (!aligned(p, 16)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!aligned(o, dtype == SGLA_BF16 ? 2 : 4)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!aligned(initial_state, 16) || !aligned(final_state, 16)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!aligned(g, 4) || !aligned(g_gamma, 4) || !aligned(cu_seqlens, 8) || !aligned(device_status, 4))
+        return SGLA_ERR_INVALID_ARGUMENT;
+    if (!(scale > 0.f) || isnan(scale) || isinf(scale)) scale = 1.0f / sqrtf((float)K);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (device_status) SGLA_CUDA(cudaMemsetAsync(device_status, 0, sizeof(int), st), "status reset");
+    if (N == 0) return SGLA_OK;
+    RecArgs a{};
+    a.q = q; a.k = k; a.v = v; a.g = g; a.g_gamma = g_gamma; a.scale = scale;
+    a.h0 = initial_state; a.o = o; a.hT = final_state; a.cu = cu_seqlens;
+    a.N = N; a.T_dense = cu_seqlens ? 0 : T; a.T_total = tokens;
+    a.H = (int)H; a.K = (int)K; a.V = (int)V;
+    a.state_v_first = state_v_first != 0; a.bf16 = dtype == SGLA_BF16; a.status = device_status;
+    SGLA_LAUNCH("fused_recurrent", launch_fused_recurrent(a, st));
+    return SGLA_OK;
+}
+
 sgla_status sgla_workspace_status(const void *workspace, int *device_status, void *stream) {
     if (!workspace || !device_status) return SGLA_ERR_INVALID_ARGUMENT;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -41,6 +41,22 @@ cudaError_t launch_segment_carry(const FwdArgs &a, bool need_carry, cudaStream_t
 cudaError_t launch_segment_state_simt(const FwdArgs &a, cudaStream_t st);
 cudaError_t launch_chunk_output_simt(const FwdArgs &a, cudaStream_t st);
 
+// Token-serial recurrence over whole sequences (state in registers, [K,V] or [V,K]).
+struct RecArgs {
+    const void *q, *k, *v;
+    const float *g, *g_gamma;
+    float scale;
+    const float *h0;
+    void *o;
+    float *hT;
+    const int64_t *cu;  // packed sequences, or NULL: N sequences of T_dense tokens
+    int64_t N, T_dense, T_total;
+    int H, K, V;
+    bool state_v_first, bf16;
+    int *status;        // optional device word: SGLA_DEVICE_BAD_CU_SEQLENS
+};
+cudaError_t launch_fused_recurrent(const RecArgs &a, cudaStream_t st);
+
 // Recurrent decode step.
 cudaError_t launch_decode_step(const void *q, const void *k, const void *v, const float *g,
                                const float *g_gamma, float scale, float *state, void *o,

@@ -21,6 +21,9 @@ test matrix with gate normalisers 0.1/1/10, scales 0.1/1 and the packed lengths
                 no per-token gate, no states
   decode        256 sequences x 64 single-token steps, H=32 K=V=128, bf16, g per step,
                 state 0.1*N(0,1) fp32 updated in place
+  recurrent_prefill  the inference routing case of section 4 (at most 64 tokens go to
+                the fused recurrence): 256 sequences x 64 tokens, H=32 K=V=128, bf16,
+                g, initial state 0.1*N(0,1), final state -- simple_gla_fused_recurrent
 """
 from __future__ import annotations
 
@@ -42,6 +45,9 @@ WORKLOADS = {
                        chunk_size=64),
     "decode": dict(kind="decode", N=256, steps=64, H=32, K=128, V=128, dtype=torch.bfloat16, gate="g",
                    scale=None),
+    "recurrent_prefill": dict(kind="dense", entry="recurrent", B=256, T=64, H=32, K=128, V=128,
+                              dtype=torch.bfloat16, gate="g", h0=True, final_state=True, scale=None,
+                              chunk_size=64),
 }
 
 
@@ -113,6 +119,6 @@ def make_workload(name: str, seed: int = 0):
     g_gamma = retnet_gammas(H) if w["gate"] == "gamma" else None
     N = (len(cu) - 1) if cu is not None else B
     h0 = torch.randn(N, H, K, V, generator=gen) * 0.1 if w["h0"] else None
-    return dict(name=name, kind=w["kind"], q=q, k=k, v=v, g=g, g_gamma=g_gamma, h0=h0, cu_seqlens=cu,
-                scale=w["scale"], output_final_state=w["final_state"], chunk_size=w["chunk_size"],
-                B=B, T=T, N=N, H=H, K=K, V=V)
+    return dict(name=name, kind=w["kind"], entry=w.get("entry", "chunk"), q=q, k=k, v=v, g=g, g_gamma=g_gamma,
+                h0=h0, cu_seqlens=cu, scale=w["scale"], output_final_state=w["final_state"],
+                chunk_size=w["chunk_size"], B=B, T=T, N=N, H=H, K=K, V=V)

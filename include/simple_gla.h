@@ -159,6 +159,38 @@ SGLA_API sgla_status simple_gla_fwd_varlen(const void *q, const void *k, const v
                                   void *stream);
 
 /*
+ * Token-serial recurrence over whole sequences (fused_recurrent_simple_gla, article
+ * section 2; section 4: the layer sends inference calls of at most 64 tokens here):
+ *   S <- exp(a_t) S + k_t v_t^T ;  o_t = scale * S^T q_t  (post-update state)
+ * for every token t of every sequence, starting from initial_state (or zeros), with
+ * a_t = g[t,h], or g_gamma[h], or 0.  The state is read once and written once per
+ * call, so this is the cheap path for short sequences; its result equals that of
+ * simple_gla_fwd(_varlen) up to rounding.
+ *
+ *   cu_seqlens == NULL: N sequences of T tokens; q, k [N,T,H,K], v, o [N,T,H,V].
+ *   cu_seqlens != NULL: DEVICE pointer to N+1 int64 (N >= 1); sequence n covers
+ *       tokens cu_seqlens[n] .. cu_seqlens[n+1]-1 of T packed tokens; q, k [T,H,K],
+ *       v, o [T,H,V].  A sequence whose bounds are not 0 <= start <= end <= T is
+ *       skipped (none of its outputs or final state are written) and *device_status,
+ *       when given, is set to SGLA_DEVICE_BAD_CU_SEQLENS.
+ *   g [tokens,H] or g_gamma [H] (fp32, not both) or neither; scale as simple_gla_fwd.
+ *   initial_state, final_state: fp32, NULL or [N,H,K,V] -- [N,H,V,K] when
+ *       state_v_first != 0 (the transposed layout of article section 2), 16-byte
+ *       aligned.  They may be the same buffer (in-place update: the T = 1 case is a
+ *       decode step on a [V,K] state).
+ *   device_status: optional DEVICE int, reset to SGLA_DEVICE_OK by this call.
+ * Supported sizes: K and V multiples of 8 (bf16) or 4 (fp32); 1 <= K <= 512 (bf16) or
+ * 256 (fp32); V <= 4096.  q, k, v 16-byte aligned, o aligned to its element size.
+ * No workspace.
+ */
+SGLA_API sgla_status simple_gla_fused_recurrent(const void *q, const void *k, const void *v,
+                                       const float *g, const float *g_gamma, float scale,
+                                       const float *initial_state, void *o, float *final_state,
+                                       const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H,
+                                       int64_t K, int64_t V, int state_v_first, sgla_dtype dtype,
+                                       int *device_status, void *stream);
+
+/*
  * One recurrent decode step for N independent sequences (the single-token case of
  * fused_recurrent_simple_gla, article sections 2 and 4):
  *   state <- exp(a) * state + k v^T ;  o = scale * state^T q   (post-update state)

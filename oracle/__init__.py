@@ -83,10 +83,17 @@ def default_threads() -> int:
 
 
 def simple_gla_fwd(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
-                   output_final_state=False, cu_seqlens=None, threads=None, lib_path=None):
+                   output_final_state=False, cu_seqlens=None, threads=None, lib_path=None,
+                   state_v_first=False):
     """fp64 naive recurrence.  q,k [B,T,H,K]; v [B,T,H,V]; g [B,T,H]; g_gamma [H];
-    initial_state [N,H,K,V].  Returns (o [B,T,H,V] float64, final_state or None)."""
+    initial_state [N,H,K,V] -- [N,H,V,K] with state_v_first, the transposed state
+    layout of section 2 of the article (the final state is returned in the same
+    layout).  Returns (o [B,T,H,V] float64, final_state or None)."""
     q, k, v, g, g_gamma, h0 = map(_f64, (q, k, v, g, g_gamma, initial_state))
+    if state_v_first and h0 is not None:
+        if h0.ndim != 4:
+            raise ValueError("initial_state must have 4 dimensions")
+        h0 = np.ascontiguousarray(h0.transpose(0, 1, 3, 2))
     if g is not None and g_gamma is not None:
         raise ValueError("only one of g and g_gamma may be given")
     if q.ndim != 4 or k.shape != q.shape or v.shape[:3] != q.shape[:3]:
@@ -120,6 +127,8 @@ def simple_gla_fwd(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None
                                  int(threads or default_threads()))
     if rc != 0:
         raise RuntimeError(f"sgla_oracle_fwd failed with code {rc}")
+    if state_v_first and hT is not None:
+        hT = np.ascontiguousarray(hT.transpose(0, 1, 3, 2))
     return o, hT
 
 

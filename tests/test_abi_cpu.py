@@ -102,6 +102,26 @@ def test_invalid_calls_are_rejected_on_the_host(lib):
     assert d(FAKE, FAKE, FAKE, None, None, 1.0, None, FAKE, 4, 2, 64, 64, 0, None) == L.SGLA_ERR_INVALID_ARGUMENT
 
 
+def test_fused_recurrent_validation_on_the_host(lib):
+    f = lib.simple_gla_fused_recurrent
+
+    def call(q=FAKE, g=None, gg=None, h0=None, hT=None, cu=None, N=4, T=8, H=2, K=64, V=64, vf=0,
+             dt=L.SGLA_BF16, status=None):
+        return f(q, FAKE, FAKE, g, gg, 1.0, h0, FAKE, hT, cu, N, T, H, K, V, vf, dt, status, None)
+
+    assert call(g=FAKE, gg=FAKE) == L.SGLA_ERR_INVALID_ARGUMENT       # both gates
+    assert call(K=520) == L.SGLA_ERR_UNSUPPORTED                      # K above 512
+    assert call(K=264, dt=L.SGLA_FP32) == L.SGLA_ERR_UNSUPPORTED      # fp32 K above 256
+    assert call(V=68) == L.SGLA_ERR_UNSUPPORTED                       # bf16 V not a multiple of 8
+    assert call(K=60) == L.SGLA_ERR_UNSUPPORTED                       # bf16 K not a multiple of 8
+    assert call(q=FAKE + 8) == L.SGLA_ERR_INVALID_ARGUMENT            # q not 16-byte aligned
+    assert call(h0=FAKE + 8) == L.SGLA_ERR_INVALID_ARGUMENT           # state not 16-byte aligned
+    assert call(cu=FAKE, N=0) == L.SGLA_ERR_INVALID_ARGUMENT          # packed with no sequence
+    assert call(q=None) == L.SGLA_ERR_INVALID_ARGUMENT                # tokens but no q
+    assert call(dt=7) == L.SGLA_ERR_INVALID_ARGUMENT                  # unknown dtype
+    assert call(N=0) == L.SGLA_OK                                     # nothing to do, nothing launched
+
+
 def test_binding_refuses_cpu_tensors():
     import gated_linear_attention_local_b200 as sg
     x = torch.zeros(1, 8, 1, 16)

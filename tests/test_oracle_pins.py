@@ -105,11 +105,13 @@ def pin_golden(lib_path=None):
         k = np.array(c["k"]).reshape(1, T, 1, K)
         v = np.array(c["v"]).reshape(1, T, 1, V)
         g = np.log(np.array(c["gate"])).reshape(1, T, 1)
-        h0 = None if c["h0"] is None else np.array(c["h0"]).reshape(1, 1, K, V)
+        vf = bool(c.get("state_v_first", False))
+        sshape = (V, K) if vf else (K, V)
+        h0 = None if c["h0"] is None else np.array(c["h0"]).reshape(1, 1, *sshape)
         o, hT = oracle.simple_gla_fwd(q, k, v, g=g, scale=c["scale"], initial_state=h0,
-                                      output_final_state=True, lib_path=lib_path)
+                                      output_final_state=True, state_v_first=vf, lib_path=lib_path)
         _close(o.reshape(T, V), np.array(c["o"]), 1e-13)
-        _close(hT.reshape(K, V), np.array(c["hT"]), 1e-13)
+        _close(hT.reshape(*sshape), np.array(c["hT"]), 1e-13)
 
 
 def pin_brute_force_dense(lib_path=None):
