@@ -22,6 +22,7 @@ Public functions (same names as the C entry points):
   simple_gla_fused_recurrent(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
                              output_final_state=False, cu_seqlens=None,
                              state_v_first=False) -> (o, final_state|None)
+  simple_gla_chunk(q, k, v, ..., cu_seqlens=None, chunk_size=64, state_v_first=False)
   chunk_simple_gla(...)  -- the article's entry-point name; dispatches on cu_seqlens.
   fused_recurrent_simple_gla(...) -- the article's name for simple_gla_fused_recurrent.
 """
@@ -36,7 +37,7 @@ from ._lib import (SGLA_BF16, SGLA_FP32, SGLA_OK, SglaError, lib, library_path, 
                    raise_for_status)
 
 __all__ = ["simple_gla_fwd", "simple_gla_fwd_noalloc", "simple_gla_fwd_varlen", "simple_gla_decode_step", "chunk_simple_gla",
-           "simple_gla_fused_recurrent", "fused_recurrent_simple_gla",
+           "simple_gla_fused_recurrent", "fused_recurrent_simple_gla", "simple_gla_chunk",
            "fwd_workspace_size", "varlen_workspace_size", "workspace_status", "library_path",
            "SglaError"]
 
@@ -194,9 +195,68 @@ def simple_gla_fwd_varlen(q, k, v, cu_seqlens, g=None, g_gamma=None, scale=None,
     return (o.unsqueeze(0) if squeeze else o), ht
 
 
+def simple_gla_chunk(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None, output_final_state=False,
+                     cu_seqlens=None, chunk_size=64, state_v_first=False, workspace=None):
+    """Chunked forward with every option in one call: dense q,k [B,T,H,K] (or packed
+    [1,T,H,K] / [T,H,K] with cu_seqlens), states [N,H,K,V] or, with state_v_first,
+    [N,H,V,K].  Returns (o shaped like v, final_state|None)."""
+    _common_checks(q, k, v, g, g_gamma, None)
+    _check_cuda("initial_state", initial_state, torch.float32, 4)
+    squeeze = False
+    if cu_seqlens is not None:
+        _check_cuda("cu_seqlens", cu_seqlens, torch.int64, 1)
+        if q.dim() == 4:
+            if q.shape[0] != 1:
+                raise ValueError("with cu_seqlens the batch size must be 1 (flatten the batch first)")
+            squeeze = True
+            q, k, v = q[0], k[0], v[0]
+            g = g[0] if g is not None else None
+        if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+            raise ValueError("q,k must be [T,H,K] and v [T,H,V] with cu_seqlens")
+        N = cu_seqlens.shape[0] - 1
+        if N < 1:
+            raise ValueError("cu_seqlens must hold at least two entries")
+        T, H, K = q.shape
+        V = v.shape[2]
+        if g is not None and tuple(g.shape) != (T, H):
+            raise ValueError("g must be [T,H] (or [1,T,H])")
+        if initial_state is not None and initial_state.shape[0] != N:
+            raise ValueError(f"the number of initial states must equal len(cu_seqlens) - 1 = {N}, "
+                             f"got {initial_state.shape[0]}")
+    else:
+        if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+            raise ValueError("q,k must be [B,T,H,K] and v [B,T,H,V]")
+        N, T, H, K = q.shape
+        V = v.shape[3]
+        if g is not None and tuple(g.shape) != (N, T, H):
+            raise ValueError(f"g must be [B,T,H] = {(N, T, H)}")
+    if g_gamma is not None and tuple(g_gamma.shape) != (H,):
+        raise ValueError("g_gamma must be [H]")
+    sshape = (N, H, V, K) if state_v_first else (N, H, K, V)
+    if initial_state is not None and tuple(initial_state.shape) != sshape:
+        raise ValueError(f"initial_state must be {sshape}")
+    dt = _DTYPES[q.dtype]
+    vf = 1 if state_v_first else 0
+    o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    ht = torch.empty(sshape, dtype=torch.float32, device=q.device) if output_final_state else None
+    nbytes = int(lib().simple_gla_chunk_workspace_size(_ptr(cu_seqlens), N, T, H, K, V, chunk_size, vf, dt))
+    if nbytes == 0:
+        raise_for_status(_size_status(K, V, chunk_size), "simple_gla_chunk")
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().simple_gla_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma), ctypes.c_float(_scale(scale)),
+                                _ptr(initial_state), _ptr(o), _ptr(ht), _ptr(cu_seqlens), N, T, H, K, V, chunk_size,
+                                vf, dt, _ptr(ws), ws.numel(), _stream())
+    raise_for_status(st, "simple_gla_chunk")
+    return (o.unsqueeze(0) if squeeze else o), ht
+
+
 def chunk_simple_gla(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
-                     output_final_state=False, cu_seqlens=None, chunk_size=64):
-    """The article's entry-point name (section 2): dense, or packed when cu_seqlens is given."""
+                     output_final_state=False, cu_seqlens=None, chunk_size=64, state_v_first=False):
+    """The article's entry-point name (section 2): dense, or packed when cu_seqlens is
+    given; state_v_first selects the [N,H,V,K] state layout."""
+    if state_v_first:
+        return simple_gla_chunk(q, k, v, g, g_gamma, scale, initial_state, output_final_state, cu_seqlens,
+                                chunk_size, state_v_first=True)
     if cu_seqlens is None:
         return simple_gla_fwd(q, k, v, g, g_gamma, scale, initial_state, output_final_state, chunk_size)
     return simple_gla_fwd_varlen(q, k, v, cu_seqlens, g, g_gamma, scale, initial_state,

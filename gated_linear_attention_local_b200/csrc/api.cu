@@ -83,6 +83,7 @@ struct Plan {
     int64_t max_chunks = 0, max_segs = 0;
     bool multi_seg = false;    // some sequence may have more than one segment
     size_t off_chunk_off = 0, off_seg_off = 0, off_gcum = 0, off_gpos = 0, off_seg_dec = 0, off_seg_state = 0;
+    size_t off_state_in = 0, off_state_out = 0;  // [K,V] copies of [V,K] states (state_v_first)
     size_t bytes = 0;
 };
 
@@ -97,7 +98,7 @@ sgla_status check_sizes(int64_t H, int64_t K, int64_t V, int chunk_size) {
 
 // varlen: N sequences, T = total tokens; dense: N = B, T = tokens per sequence.
 Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V, int C,
-               sgla_dtype dtype, bool per_token_gate) {
+               sgla_dtype dtype, bool per_token_gate, bool state_v_first = false) {
     Plan p;
     sgla_status st = check_sizes(H, K, V, C);
     if (st != SGLA_OK) { p.why = st; return p; }
@@ -173,6 +174,12 @@ Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t 
         p.off_seg_state = off;
         off = align_up(off + sizeof(float) * (size_t)p.max_segs * H * K * V, 256);
     }
+    if (state_v_first) {
+        p.off_state_in = off;
+        off = align_up(off + sizeof(float) * (size_t)N * H * K * V, 256);
+        p.off_state_out = off;
+        off = align_up(off + sizeof(float) * (size_t)N * H * K * V, 256);
+    }
     p.bytes = off;
     p.valid = true;
     return p;
@@ -182,7 +189,7 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
                         const float *g_gamma, float scale, const int64_t *cu, int64_t N, int64_t T,
                         const float *h0, void *o, float *hT, int64_t H, int64_t K, int64_t V,
                         int chunk_size, sgla_dtype dtype, void *workspace, size_t workspace_bytes,
-                        void *stream) {
+                        void *stream, bool state_v_first = false) {
     if (g && g_gamma) return SGLA_ERR_INVALID_ARGUMENT;
     const int64_t tokens = varlen ? T : N * T;
     if (tokens > 0 && (!q || !k || !v || !o)) return SGLA_ERR_INVALID_ARGUMENT;
@@ -191,7 +198,7 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
         if (!aligned(p, 16)) return SGLA_ERR_INVALID_ARGUMENT;
     if (!aligned(g, 4) || !aligned(g_gamma, 4) || !aligned(cu, 8)) return SGLA_ERR_INVALID_ARGUMENT;
     const bool per_token = g != nullptr;
-    Plan p = make_plan(varlen, N, T, H, K, V, chunk_size, dtype, per_token);
+    Plan p = make_plan(varlen, N, T, H, K, V, chunk_size, dtype, per_token, state_v_first);
     if (!p.valid) return p.why;
     if (!workspace || workspace_bytes < p.bytes) return SGLA_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return SGLA_ERR_INVALID_ARGUMENT;
@@ -202,6 +209,10 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
     FwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.g = g; a.g_gamma = g_gamma; a.scale = scale;
     a.h0 = h0; a.o = o; a.hT = hT;
+    if (state_v_first) {  // the passes work on [K,V] copies in the workspace
+        if (h0) a.h0 = reinterpret_cast<float *>(ws + p.off_state_in);
+        if (hT) a.hT = reinterpret_cast<float *>(ws + p.off_state_out);
+    }
     a.H = (int)H; a.K = (int)K; a.V = (int)V;
     a.gate_mode = g ? kGatePerToken : (g_gamma ? kGatePerHead : kGateNone);
     a.bf16 = dtype == SGLA_BF16;
@@ -227,6 +238,8 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
         SGLA_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), st), "status reset");
     }
     if (N == 0) return SGLA_OK;
+    if (state_v_first && h0)
+        SGLA_LAUNCH("state_transpose", launch_state_transpose(h0, const_cast<float *>(a.h0), N * H, (int)V, (int)K, st));
     if (per_token && tokens > 0) SGLA_LAUNCH("chunk_cumsum", launch_chunk_cumsum(g, a.gcum, a.gpos, lay, st));
     if (p.multi_seg && p.max_segs > 0) {
         if (p.tc) SGLA_LAUNCH("segment_state_tc", tc_launch_segment_state(a, st));
@@ -238,6 +251,8 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
         if (p.tc) SGLA_LAUNCH("chunk_output_tc", tc_launch_chunk_output(a, st));
         else SGLA_LAUNCH("chunk_output_simt", launch_chunk_output_simt(a, st));
     }
+    if (state_v_first && hT)
+        SGLA_LAUNCH("state_transpose", launch_state_transpose(a.hT, hT, N * H, (int)K, (int)V, st));
     return SGLA_OK;
 }
 
@@ -292,6 +307,23 @@ sgla_status simple_gla_fwd_varlen(const void *q, const void *k, const void *v, c
     if (N < 1 || T_total < 0) return SGLA_ERR_INVALID_ARGUMENT;
     return run_forward(true, q, k, v, g, g_gamma, scale, cu_seqlens, N, T_total, initial_state, o,
                        final_state, H, K, V, chunk_size, dtype, workspace, workspace_bytes, stream);
+}
+
+size_t simple_gla_chunk_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H, int64_t K,
+                                       int64_t V, int chunk_size, int state_v_first, sgla_dtype dtype) {
+    Plan p = make_plan(cu_seqlens != nullptr, N, T, H, K, V, chunk_size, dtype, true, state_v_first != 0);
+    return p.valid ? p.bytes : 0;
+}
+
+sgla_status simple_gla_chunk(const void *q, const void *k, const void *v, const float *g, const float *g_gamma,
+                             float scale, const float *initial_state, void *o, float *final_state,
+                             const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V,
+                             int chunk_size, int state_v_first, sgla_dtype dtype, void *workspace,
+                             size_t workspace_bytes, void *stream) {
+    const bool varlen = cu_seqlens != nullptr;
+    if (N < (varlen ? 1 : 0) || T < 0) return SGLA_ERR_INVALID_ARGUMENT;
+    return run_forward(varlen, q, k, v, g, g_gamma, scale, cu_seqlens, N, T, initial_state, o, final_state,
+                       H, K, V, chunk_size, dtype, workspace, workspace_bytes, stream, state_v_first != 0);
 }
 
 sgla_status simple_gla_decode_step(const void *q, const void *k, const void *v, const float *g,

@@ -41,6 +41,9 @@ cudaError_t launch_segment_carry(const FwdArgs &a, bool need_carry, cudaStream_t
 cudaError_t launch_segment_state_simt(const FwdArgs &a, cudaStream_t st);
 cudaError_t launch_chunk_output_simt(const FwdArgs &a, cudaStream_t st);
 
+// src [mats][R][C] -> dst [mats][C][R] (fp32), for the [V,K] state layout.
+cudaError_t launch_state_transpose(const float *src, float *dst, int64_t mats, int R, int C, cudaStream_t st);
+
 // Token-serial recurrence over whole sequences (state in registers, [K,V] or [V,K]).
 struct RecArgs {
     const void *q, *k, *v;

@@ -202,4 +202,37 @@ cudaError_t launch_segment_carry(const FwdArgs &a, bool need_carry, cudaStream_t
     return cudaGetLastError();
 }
 
+// Batched matrix transpose for the [V,K] state layout (state_v_first, "Simple GLA in
+// flash-linear-attention" section 2): src [mats][R][C] -> dst [mats][C][R], fp32, one
+// 32 x 32 tile per CTA through a padded shared-memory tile (coalesced both ways).
+__global__ void __launch_bounds__(256) state_transpose_kernel(const float *__restrict__ src, float *__restrict__ dst,
+                                                              int R, int C, int tiles_r, int tiles_c) {
+    __shared__ float tile[32][33];
+    const int64_t b = blockIdx.x;
+    const int64_t mat = b / ((int64_t)tiles_r * tiles_c);
+    const int rem = (int)(b - mat * tiles_r * tiles_c);
+    const int r0 = (rem / tiles_c) * 32, c0 = (rem % tiles_c) * 32;
+    const float *s = src + mat * (int64_t)R * C;
+    float *d = dst + mat * (int64_t)R * C;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+    for (int i = ty; i < 32; i += 8) {
+        const int r = r0 + i, c = c0 + tx;
+        if (r < R && c < C) tile[i][tx] = s[(int64_t)r * C + c];
+    }
+    __syncthreads();
+    for (int i = ty; i < 32; i += 8) {
+        const int c = c0 + i, r = r0 + tx;
+        if (r < R && c < C) d[(int64_t)c * R + r] = tile[tx][i];
+    }
+}
+
+cudaError_t launch_state_transpose(const float *src, float *dst, int64_t mats, int R, int C, cudaStream_t st) {
+    const int tr = (R + 31) / 32, tc = (C + 31) / 32;
+    const int64_t blocks = mats * tr * tc;
+    if (blocks == 0) return cudaSuccess;
+    if (blocks >= ((int64_t)1 << 31)) return cudaErrorInvalidValue;
+    state_transpose_kernel<<<(unsigned)blocks, 256, 0, st>>>(src, dst, R, C, tr, tc);
+    return cudaGetLastError();
+}
+
 }  // namespace sgla

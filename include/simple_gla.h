@@ -191,6 +191,28 @@ SGLA_API sgla_status simple_gla_fused_recurrent(const void *q, const void *k, co
                                        int *device_status, void *stream);
 
 /*
+ * The chunked forward with every option of chunk_simple_gla (article section 2) in
+ * one call: dense (cu_seqlens == NULL: N sequences of T tokens, q [N,T,H,K]) or
+ * packed (cu_seqlens != NULL: N sequences in T tokens, exactly as
+ * simple_gla_fwd_varlen), and the state layout: state_v_first != 0 stores
+ * initial_state / final_state as [N,H,V,K], the transpose of [N,H,K,V] (section 2).
+ * Other arguments, sizes and errors as simple_gla_fwd / simple_gla_fwd_varlen.  The
+ * workspace must hold simple_gla_chunk_workspace_size() bytes for the same
+ * arguments (a [V,K] layout adds two state-sized buffers: the state passes run on
+ * [K,V] copies, transposed on the way in and out).  The size query only tests
+ * cu_seqlens against NULL (it is never read on the host) and returns 0 for
+ * unsupported sizes.
+ */
+SGLA_API size_t simple_gla_chunk_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H,
+                                                int64_t K, int64_t V, int chunk_size, int state_v_first,
+                                                sgla_dtype dtype);
+SGLA_API sgla_status simple_gla_chunk(const void *q, const void *k, const void *v, const float *g,
+                             const float *g_gamma, float scale, const float *initial_state, void *o,
+                             float *final_state, const int64_t *cu_seqlens, int64_t N, int64_t T,
+                             int64_t H, int64_t K, int64_t V, int chunk_size, int state_v_first,
+                             sgla_dtype dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * One recurrent decode step for N independent sequences (the single-token case of
  * fused_recurrent_simple_gla, article sections 2 and 4):
  *   state <- exp(a) * state + k v^T ;  o = scale * state^T q   (post-update state)

@@ -102,6 +102,14 @@ def test_invalid_calls_are_rejected_on_the_host(lib):
     assert d(FAKE, FAKE, FAKE, None, None, 1.0, None, FAKE, 4, 2, 64, 64, 0, None) == L.SGLA_ERR_INVALID_ARGUMENT
 
 
+def test_chunk_workspace_grows_with_the_vk_layout(lib):
+    kv = lib.simple_gla_chunk_workspace_size(None, 4, 2048, 4, 128, 128, 64, 0, L.SGLA_BF16)
+    vk = lib.simple_gla_chunk_workspace_size(None, 4, 2048, 4, 128, 128, 64, 1, L.SGLA_BF16)
+    assert kv == lib.simple_gla_fwd_workspace_size(4, 2048, 4, 128, 128, 64, L.SGLA_BF16)
+    assert vk >= kv + 2 * 4 * 4 * 128 * 128 * 4  # two [K,V] state copies
+    assert lib.simple_gla_chunk_workspace_size(None, 4, 2048, 4, 128, 130, 64, 1, L.SGLA_BF16) == 0
+
+
 def test_fused_recurrent_validation_on_the_host(lib):
     f = lib.simple_gla_fused_recurrent
 

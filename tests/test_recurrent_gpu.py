@@ -158,3 +158,45 @@ def test_fused_recurrent_inference_shape():
                                        output_final_state=True)
         assert_close(o[n:n + 1], ro, TOL[torch.bfloat16], f"o seq {n}")
         assert_close(ht[n:n + 1], rh, TOL[torch.bfloat16], f"final_state seq {n}")
+
+
+CHUNK_VF = [
+    # (B, T, H, K, V, dtype, gate, h0, chunk) -- tensor-core and SIMT paths, empty
+    (2, 300, 2, 128, 128, torch.bfloat16, "g", True, 64),
+    (1, 520, 2, 256, 64, torch.bfloat16, "gamma", True, 64),
+    (2, 150, 3, 64, 32, torch.float32, "g", True, 32),
+    (2, 0, 2, 64, 64, torch.float32, "g", True, 64),
+]
+
+
+@pytest.mark.parametrize("case", CHUNK_VF, ids=[f"B{c[0]}T{c[1]}K{c[3]}V{c[4]}-{str(c[5])[6:]}-C{c[8]}"
+                                                 for c in CHUNK_VF])
+def test_chunk_state_v_first_dense(case):
+    B, T, H, K, V, dt, gate, h0, chunk = case
+    inp = random_inputs(B, T, H, K, V, dtype=dt, gate=gate, h0=h0, seed=41)
+    s0 = _vk(inp["h0"])
+    o, ht = sg.chunk_simple_gla(to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"]), g=to_dev(inp["g"]),
+                                g_gamma=to_dev(inp["g_gamma"]), initial_state=to_dev(s0), output_final_state=True,
+                                chunk_size=chunk, state_v_first=True)
+    torch.cuda.synchronize()
+    ro, rh = oracle.simple_gla_fwd(inp["q"], inp["k"], inp["v"], g=inp["g"], g_gamma=inp["g_gamma"],
+                                   initial_state=s0, output_final_state=True, state_v_first=True)
+    assert tuple(ht.shape) == (B, H, V, K)
+    assert_close(host(o), ro, TOL[dt], "o")
+    assert_close(host(ht), rh, TOL[dt], "final_state")
+
+
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float32])
+def test_chunk_state_v_first_varlen(dt):
+    cu = torch.tensor([0, 15, 15, 100, 300, 1200, 2000], dtype=torch.int64)
+    T, H, K, V = 2000, 2, 128, 128
+    inp = random_inputs(1, T, H, K, V, dtype=dt, gate="g", h0=True, seed=43, cu_seqlens=cu)
+    s0 = _vk(inp["h0"])
+    o, ht = sg.chunk_simple_gla(to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"]), g=to_dev(inp["g"]),
+                                initial_state=to_dev(s0), output_final_state=True, cu_seqlens=to_dev(cu),
+                                state_v_first=True)
+    torch.cuda.synchronize()
+    ro, rh = oracle.simple_gla_fwd(inp["q"], inp["k"], inp["v"], g=inp["g"], initial_state=s0,
+                                   output_final_state=True, cu_seqlens=cu, state_v_first=True)
+    assert_close(host(o), ro, TOL[dt], "o")
+    assert_close(host(ht), rh, TOL[dt], "final_state")
