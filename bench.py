@@ -252,6 +252,10 @@ def workspace_for(w, sg, device):
 
 
 def time_steps(step, reset, steps, warmup, flush, dist_on, profile=True):
+    """Time `steps` steps with CUDA events on the launching stream (L2 flushed before
+    each, outside the events).  The timed steps run without the library's per-kernel
+    event recording; when `profile` is set, a separate pass of min(steps, 5) steps
+    afterwards records the per-kernel times."""
     from gated_linear_attention_local_b200 import _lib
     for _ in range(warmup):
         reset()
@@ -262,8 +266,6 @@ def time_steps(step, reset, steps, warmup, flush, dist_on, profile=True):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     n0 = _lib.kernel_launch_count()
-    if profile:
-        _lib.profile_begin()
     for i in range(steps):
         reset()
         flush.zero_()
@@ -271,11 +273,19 @@ def time_steps(step, reset, steps, warmup, flush, dist_on, profile=True):
         step()
         evs[i][1].record()
     torch.cuda.synchronize()
-    prof = _lib.profile_end() if profile else {}
     launches = _lib.kernel_launch_count() - n0
     if dist_on:
         torch.distributed.barrier()
     per_step = [a.elapsed_time(b) for a, b in evs]
+    prof = {}
+    if profile:
+        _lib.profile_begin()
+        for _ in range(min(steps, 5)):
+            reset()
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+        prof = _lib.profile_end()
     return per_step, prof, launches
 
 

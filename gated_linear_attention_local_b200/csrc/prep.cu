@@ -105,10 +105,19 @@ chunk_cumsum_kernel(const float *__restrict__ g, float *__restrict__ gcum, int *
     const int len = (int)min64(lay.C, t1 - ta);
     const int H = lay.H, h0 = blockIdx.y * 32;
     const int hw = min(32, H - h0);
-    // coalesced load: each row of 32 heads is contiguous
-    for (int e = threadIdx.x; e < len * 32; e += blockDim.x) {
-        const int i = e >> 5, j = e & 31;
-        tile[i][j] = (j < hw) ? fmaxf(g[(ta + i) * H + h0 + j], kMinLogGate) : 0.f;
+    // coalesced load: each row of 32 heads is contiguous; all loads of a thread are
+    // issued before any is used (one memory latency per block, not one per element)
+    constexpr int kPer = kCumsumMaxC * 32 / 256;
+    float gv[kPer];
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+        const int e = threadIdx.x + r * 256, i = e >> 5, j = e & 31;
+        gv[r] = (i < len && j < hw) ? g[(ta + i) * H + h0 + j] : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+        const int e = threadIdx.x + r * 256, i = e >> 5, j = e & 31;
+        if (i < len) tile[i][j] = (j < hw) ? fmaxf(gv[r], kMinLogGate) : 0.f;
     }
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -182,16 +191,27 @@ segment_carry_kernel(FwdArgs a, bool need_carry) {
     if (!need_carry || nseg == 1) return;
     const int first = seq_first_segment(lay, n);
     float4 S = a.h0 ? *reinterpret_cast<const float4 *>(a.h0 + sidx) : make_float4(0.f, 0.f, 0.f, 0.f);
+    // the loads of segment s+1 are in flight while segment s is combined
+    auto slot_of = [&](int s) {
+        return reinterpret_cast<float4 *>(a.seg_state + ((int64_t)(first + s) * a.H + h) * KV + e);
+    };
+    float4 d = *slot_of(0);
+    float lg = a.seg_dec[(int64_t)first * a.H + h];
     for (int s = 0; s + 1 < nseg; ++s) {
-        const int64_t u = first + s;
-        float4 *slot = reinterpret_cast<float4 *>(a.seg_state + (u * a.H + h) * KV + e);
-        const float4 d = *slot;
-        const float dec = exp2f(a.seg_dec[u * a.H + h]);
+        float4 dn = d;
+        float lgn = lg;
+        if (s + 2 < nseg) {
+            dn = *slot_of(s + 1);
+            lgn = a.seg_dec[(int64_t)(first + s + 1) * a.H + h];
+        }
+        const float dec = exp2f(lg);
         S.x = fmaf(dec, S.x, d.x);
         S.y = fmaf(dec, S.y, d.y);
         S.z = fmaf(dec, S.z, d.z);
         S.w = fmaf(dec, S.w, d.w);
-        *slot = S;
+        *slot_of(s) = S;
+        d = dn;
+        lg = lgn;
     }
 }
 
