@@ -46,6 +46,7 @@ _SIG = {
     "simple_gla_fused_recurrent": ([_P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64,
                                     ctypes.c_int, ctypes.c_int, _P, _P], ctypes.c_int),
     "sgla_workspace_status": ([_P, ctypes.POINTER(ctypes.c_int), _P], ctypes.c_int),
+    "sgla_selftest_wait_timeout": ([_P, _P], ctypes.c_int),
     "sgla_kernel_launch_count": ([], ctypes.c_uint64),
     "sgla_profile_begin": ([], ctypes.c_int),
     "sgla_profile_end": ([ctypes.c_char_p, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double),

@@ -390,6 +390,13 @@ sgla_status sgla_workspace_status(const void *workspace, int *device_status, voi
     return SGLA_OK;
 }
 
+sgla_status sgla_selftest_wait_timeout(int *device_status, void *stream) {
+    if (!device_status || !aligned(device_status, 4)) return SGLA_ERR_INVALID_ARGUMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    SGLA_LAUNCH("selftest_wait_timeout", launch_wait_timeout_selftest(device_status, st));
+    return SGLA_OK;
+}
+
 uint64_t sgla_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 sgla_status sgla_profile_begin(void) {

@@ -60,6 +60,10 @@ struct RecArgs {
 };
 cudaError_t launch_fused_recurrent(const RecArgs &a, cudaStream_t st);
 
+// Self-test: one CTA waits on an mbarrier phase nothing completes; writes
+// SGLA_DEVICE_TIMEOUT to *status once the bounded wait has given up.
+cudaError_t launch_wait_timeout_selftest(int *status, cudaStream_t st);
+
 // Recurrent decode step.
 cudaError_t launch_decode_step(const void *q, const void *k, const void *v, const float *g,
                                const float *g_gamma, float scale, float *state, void *o,

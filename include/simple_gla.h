@@ -257,6 +257,18 @@ SGLA_API sgla_status simple_gla_fwd_noalloc(const void *q, const void *k, const 
 SGLA_API sgla_status sgla_workspace_status(const void *workspace, int *device_status, void *stream);
 
 /*
+ * Self-test of the library's failure detection (no counterpart on the pages).  Every
+ * wait of the tensor-core pipelines on an mbarrier is bounded: after 2 s of wall time
+ * the waiting thread gives up, raises its CTA's abort flag (on which the CTA's other
+ * waits give up too) and the call's status word reads SGLA_DEVICE_TIMEOUT.  This
+ * launches one CTA that waits on a phase nothing completes and writes, to the DEVICE
+ * int *device_status, SGLA_DEVICE_TIMEOUT if both of its waiting threads gave up as
+ * designed (SGLA_DEVICE_OK otherwise).  Takes about 2 s; faults and traps nothing,
+ * and the context stays usable.
+ */
+SGLA_API sgla_status sgla_selftest_wait_timeout(int *device_status, void *stream);
+
+/*
  * Tracing aids (no counterpart in the article; they observe, never change, the
  * computation).
  *

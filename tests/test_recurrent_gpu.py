@@ -40,6 +40,11 @@ DENSE = [
     (2, 33, 2, 20, 8, torch.float32, "g", 10.0, True, False, 1.0),
     (1, 64, 2, 64, 64, torch.float32, "g", 0.1, True, True, None),
     (2, 0, 2, 64, 64, torch.float32, "g", 1.0, True, True, None),
+    # gate 0 and log gates of both signs: the blocks whose cumulative decay leaves the
+    # range where it can be factored out take the exact per-token update
+    (2, 40, 2, 64, 64, torch.float32, "neg_inf", 1.0, True, False, None),
+    (2, 40, 2, 64, 64, torch.float32, "mixed", 1.0, True, False, None),
+    (2, 40, 2, 64, 64, torch.float32, "g", 0.05, True, False, None),
 ]
 
 
@@ -200,3 +205,28 @@ def test_chunk_state_v_first_varlen(dt):
                                    output_final_state=True, cu_seqlens=cu, state_v_first=True)
     assert_close(host(o), ro, TOL[dt], "o")
     assert_close(host(ht), rh, TOL[dt], "final_state")
+
+
+def test_bounded_wait_gives_up_and_the_context_survives():
+    """Failure detection without a GPU fault: a CTA waits on an mbarrier phase that
+    nothing completes; the bounded wait gives up after its 2 s limit, raises the CTA's
+    abort flag (the second waiter gives up through it) and reports the time-out in a
+    status word the host reads.  The context then runs a forward normally."""
+    import ctypes
+    import time
+    from gated_linear_attention_local_b200 import _lib
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    st = _lib.lib().sgla_selftest_wait_timeout(ctypes.c_void_p(status.data_ptr()),
+                                               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert st == _lib.SGLA_OK
+    assert int(status.item()) == 2  # SGLA_DEVICE_TIMEOUT
+    assert 1.5 < dt < 30.0, dt
+    inp = random_inputs(1, 256, 2, 128, 128, dtype=torch.bfloat16, gate="g", seed=1)
+    o, _ = sg.simple_gla_fwd(to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"]), g=to_dev(inp["g"]))
+    torch.cuda.synchronize()
+    ro, _ = oracle.simple_gla_fwd(inp["q"], inp["k"], inp["v"], g=inp["g"])
+    assert_close(host(o), ro, TOL[torch.bfloat16], "o after the time-out")
