@@ -221,6 +221,12 @@ def make_step(w, d, sg, ws):
                 sg.simple_gla_decode_step(d["q"][t], d["k"][t], d["v"][t], d["state"], g=d["g"][t],
                                           scale=w["scale"], out=o)
         return step, reset
+    if w.get("entry") == "normalized":
+        def step():
+            sg.simple_gla_normalized(d["q"], d["k"], d["v"], g=d["g"], g_gamma=d["g_gamma"], initial_state=d["h0"],
+                                     output_final_state=w["output_final_state"], chunk_size=w["chunk_size"],
+                                     workspace=ws)
+        return step, (lambda: None)
     if w.get("entry") == "recurrent":
         def step():
             sg.simple_gla_fused_recurrent(d["q"], d["k"], d["v"], g=d["g"], g_gamma=d["g_gamma"], scale=w["scale"],
@@ -244,6 +250,10 @@ def workspace_for(w, sg, device):
     if w["kind"] == "decode" or w.get("entry") == "recurrent":
         return None
     dt = w["q"].dtype
+    if w.get("entry") == "normalized":
+        n = sg.lib().simple_gla_normalized_workspace_size(None, w["B"], w["T"], w["H"], w["K"], w["V"],
+                                                          w["chunk_size"], sg._DTYPES[dt])
+        return torch.empty(max(int(n), 256), dtype=torch.uint8, device=device)
     if w["kind"] == "varlen":
         n = sg.varlen_workspace_size(w["N"], w["T"], w["H"], w["K"], w["V"], w["chunk_size"], dt)
     else:
@@ -314,7 +324,8 @@ def e2e_measure(w, sg, device, steps, warmup):
     else:
         tokens_shape = (w["B"], w["T"]) if w["kind"] == "dense" else (w["T"],)
         out_host = torch.empty(*tokens_shape, w["H"], w["V"], dtype=w["q"].dtype).pin_memory()
-        st_host = torch.empty(w["N"], w["H"], w["K"], w["V"]).pin_memory() if w["output_final_state"] else None
+        sv = w["V"] + 1 if w.get("entry") == "normalized" else w["V"]
+        st_host = torch.empty(w["N"], w["H"], w["K"], sv).pin_memory() if w["output_final_state"] else None
         d2h = out_host.numel() * out_host.element_size() + (st_host.numel() * 4 if st_host is not None else 0)
 
     def one():
@@ -330,6 +341,10 @@ def e2e_measure(w, sg, device, steps, warmup):
             o, ht = sg.simple_gla_fwd_varlen(d["q"][0], d["k"][0], d["v"][0], d["cu_seqlens"], g=d["g"][0],
                                              g_gamma=g_gamma, scale=w["scale"], initial_state=d.get("h0"),
                                              output_final_state=w["output_final_state"],
+                                             chunk_size=w["chunk_size"], workspace=ws)
+        elif w.get("entry") == "normalized":
+            o, ht = sg.simple_gla_normalized(d["q"], d["k"], d["v"], g=d.get("g"), g_gamma=g_gamma,
+                                             initial_state=d.get("h0"), output_final_state=w["output_final_state"],
                                              chunk_size=w["chunk_size"], workspace=ws)
         elif w.get("entry") == "recurrent":
             o, ht = sg.simple_gla_fused_recurrent(d["q"], d["k"], d["v"], g=d.get("g"), g_gamma=g_gamma,
@@ -397,9 +412,14 @@ def oracle_sample(w, budget_s=12.0):
     def run(tn):
         d, ntok = sub(tn)
         t0 = time.perf_counter()
-        oracle.simple_gla_fwd(d["q"], d["k"], d["v"], g=d["g"], g_gamma=w["g_gamma"], scale=w["scale"],
-                              initial_state=w["h0"], output_final_state=w["output_final_state"],
-                              cu_seqlens=d["cu"], threads=threads)
+        if w.get("entry") == "normalized":
+            oracle.simple_gla_normalized(d["q"], d["k"], d["v"], g=d["g"], g_gamma=w["g_gamma"],
+                                         initial_state=w["h0"], output_final_state=w["output_final_state"],
+                                         cu_seqlens=d["cu"], threads=threads)
+        else:
+            oracle.simple_gla_fwd(d["q"], d["k"], d["v"], g=d["g"], g_gamma=w["g_gamma"], scale=w["scale"],
+                                  initial_state=w["h0"], output_final_state=w["output_final_state"],
+                                  cu_seqlens=d["cu"], threads=threads)
         return time.perf_counter() - t0, ntok
     cal_t, cal_tok = run(32)
     per_tok = cal_t / max(cal_tok, 1)
@@ -470,6 +490,9 @@ def reference_arm(args, world, rank):
 def _config_of(w):
     if w["kind"] == "decode":
         return dict(N=w["N"], steps_per_call=w["steps"], H=w["H"], K=w["K"], V=w["V"], state="fp32")
+    if w.get("entry") == "normalized":
+        return dict(entry="simple_gla_normalized", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
+                    gate="g" if w["g"] is not None else "none", feature_map="|x|+0.1", scale=1.0)
     if w.get("entry") == "recurrent":
         return dict(entry="simple_gla_fused_recurrent", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
                     gate="g" if w["g"] is not None else "none", initial_state=w["h0"] is not None)

@@ -23,6 +23,8 @@ Public functions (same names as the C entry points):
                              output_final_state=False, cu_seqlens=None,
                              state_v_first=False) -> (o, final_state|None)
   simple_gla_chunk(q, k, v, ..., cu_seqlens=None, chunk_size=64, state_v_first=False)
+  simple_gla_normalized(q, k, v, ...) / simple_gla_normalized_decode_step(...) -- the
+      normalised variant through the augmented value (states [.., K, V+1])
   chunk_simple_gla(...)  -- the article's entry-point name; dispatches on cu_seqlens.
   fused_recurrent_simple_gla(...) -- the article's name for simple_gla_fused_recurrent.
 """
@@ -38,6 +40,7 @@ from ._lib import (SGLA_BF16, SGLA_FP32, SGLA_OK, SglaError, lib, library_path, 
 
 __all__ = ["simple_gla_fwd", "simple_gla_fwd_noalloc", "simple_gla_fwd_varlen", "simple_gla_decode_step", "chunk_simple_gla",
            "simple_gla_fused_recurrent", "fused_recurrent_simple_gla", "simple_gla_chunk",
+           "simple_gla_normalized", "simple_gla_normalized_decode_step", "normalized_decode_state_width",
            "fwd_workspace_size", "varlen_workspace_size", "workspace_status", "library_path",
            "SglaError"]
 
@@ -347,6 +350,77 @@ def simple_gla_fused_recurrent(q, k, v, g=None, g_gamma=None, scale=None, initia
                                           _DTYPES[q.dtype], _ptr(device_status), _stream())
     raise_for_status(st, "simple_gla_fused_recurrent")
     return (o.unsqueeze(0) if squeeze else o), ht
+
+
+def simple_gla_normalized(q, k, v, g=None, g_gamma=None, initial_state=None, output_final_state=False,
+                          cu_seqlens=None, chunk_size=64, workspace=None):
+    """Normalised variant (augmented value, scale 1): o = (q^T S) / (q^T z).  Shapes as
+    simple_gla_chunk; states are the augmented [N,H,K,V+1] (last column z).
+    Returns (o shaped like v, final_state|None)."""
+    _common_checks(q, k, v, g, g_gamma, None)
+    _check_cuda("initial_state", initial_state, torch.float32, 4)
+    squeeze = False
+    if cu_seqlens is not None:
+        _check_cuda("cu_seqlens", cu_seqlens, torch.int64, 1)
+        if q.dim() == 4:
+            if q.shape[0] != 1:
+                raise ValueError("with cu_seqlens the batch size must be 1 (flatten the batch first)")
+            squeeze = True
+            q, k, v = q[0], k[0], v[0]
+            g = g[0] if g is not None else None
+        if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+            raise ValueError("q,k must be [T,H,K] and v [T,H,V] with cu_seqlens")
+        N = cu_seqlens.shape[0] - 1
+        T, H, K = q.shape
+        V = v.shape[2]
+    else:
+        if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+            raise ValueError("q,k must be [B,T,H,K] and v [B,T,H,V]")
+        N, T, H, K = q.shape
+        V = v.shape[3]
+    sshape = (N, H, K, V + 1)
+    if initial_state is not None and tuple(initial_state.shape) != sshape:
+        raise ValueError(f"initial_state must be the augmented state {sshape}")
+    dt = _DTYPES[q.dtype]
+    o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    ht = torch.empty(sshape, dtype=torch.float32, device=q.device) if output_final_state else None
+    nbytes = int(lib().simple_gla_normalized_workspace_size(_ptr(cu_seqlens), N, T, H, K, V, chunk_size, dt))
+    if nbytes == 0:
+        raise_for_status(_size_status(K, V + 1, chunk_size), "simple_gla_normalized")
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().simple_gla_normalized(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma), _ptr(initial_state), _ptr(o),
+                                     _ptr(ht), _ptr(cu_seqlens), N, T, H, K, V, chunk_size, dt, _ptr(ws), ws.numel(),
+                                     _stream())
+    raise_for_status(st, "simple_gla_normalized")
+    return (o.unsqueeze(0) if squeeze else o), ht
+
+
+def normalized_decode_state_width(V: int) -> int:
+    """Columns of the augmented decode state: V + 1 rounded up to a multiple of 4."""
+    return (V + 1 + 3) // 4 * 4
+
+
+def simple_gla_normalized_decode_step(q, k, v, state, g=None, g_gamma=None, out=None, workspace=None):
+    """One token of the normalised variant, in place on the augmented state
+    [N,H,K,normalized_decode_state_width(V)] fp32 (column V is z, later ones stay 0)."""
+    _common_checks(q, k, v, g, g_gamma, None)
+    _check_cuda("state", state, torch.float32, 4)
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+        raise ValueError("q,k must be [N,H,K] and v [N,H,V]")
+    N, H, K = q.shape
+    V = v.shape[2]
+    want = (N, H, K, normalized_decode_state_width(V))
+    if tuple(state.shape) != want:
+        raise ValueError(f"state must be {want}")
+    dt = _DTYPES[q.dtype]
+    o = out if out is not None else torch.empty((N, H, V), dtype=q.dtype, device=q.device)
+    _check_cuda("out", o, q.dtype, 3)
+    nbytes = int(lib().simple_gla_normalized_decode_workspace_size(N, H, V, dt))
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().simple_gla_normalized_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma), _ptr(state),
+                                                 _ptr(o), N, H, K, V, dt, _ptr(ws), ws.numel(), _stream())
+    raise_for_status(st, "simple_gla_normalized_decode_step")
+    return o
 
 
 def fused_recurrent_simple_gla(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,

@@ -256,6 +256,43 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
     return SGLA_OK;
 }
 
+// Normalised variant: the augmented value [v, 1] is padded to the width the forward
+// kernels take (multiples of 64 on the tensor-core path, of 8 on the SIMT path).
+struct NormLayout {
+    bool valid = false;
+    sgla_status why = SGLA_ERR_INVALID_ARGUMENT;
+    int Vp = 0;
+    Plan inner;
+    size_t off_va = 0, off_oa = 0, off_h0 = 0, off_hT = 0, bytes = 0;
+};
+
+NormLayout norm_layout(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V, int chunk_size,
+                       sgla_dtype dtype) {
+    NormLayout L;
+    if (V < 1 || V >= 512 || H < 1 || K < 1) { L.why = V >= 512 ? SGLA_ERR_UNSUPPORTED : SGLA_ERR_INVALID_ARGUMENT; return L; }
+    const int64_t v64 = (V + 1 + 63) / 64 * 64;
+    L.Vp = (dtype == SGLA_BF16 && K <= 512 && tc_path_supports(true, (int)K, (int)v64, chunk_size))
+               ? (int)v64 : (int)((V + 1 + 7) / 8 * 8);
+    L.inner = make_plan(varlen, N, T, H, K, L.Vp, chunk_size, dtype, true);
+    if (!L.inner.valid) { L.why = L.inner.why; return L; }
+    const int64_t tokens = varlen ? T : N * T;
+    const size_t es = dtype == SGLA_BF16 ? 2 : 4;
+    size_t off = align_up(L.inner.bytes, 256);
+    L.off_va = off;
+    off = align_up(off + es * (size_t)tokens * H * L.Vp, 256);
+    L.off_oa = off;
+    off = align_up(off + es * (size_t)tokens * H * L.Vp, 256);
+    L.off_h0 = off;
+    off = align_up(off + sizeof(float) * (size_t)N * H * K * L.Vp, 256);
+    L.off_hT = off;
+    off = align_up(off + sizeof(float) * (size_t)N * H * K * L.Vp, 256);
+    L.bytes = off;
+    L.valid = true;
+    return L;
+}
+
+int norm_decode_width(int64_t V) { return (int)((V + 1 + 3) / 4 * 4); }
+
 }  // namespace
 
 extern "C" {
@@ -387,6 +424,77 @@ sgla_status sgla_workspace_status(const void *workspace, int *device_status, voi
     SGLA_CUDA(cudaMemcpyAsync(&host, workspace, sizeof(int), cudaMemcpyDeviceToHost, st), "status read");
     SGLA_CUDA(cudaStreamSynchronize(st), "status sync");
     *device_status = host;
+    return SGLA_OK;
+}
+
+size_t simple_gla_normalized_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H, int64_t K,
+                                            int64_t V, int chunk_size, sgla_dtype dtype) {
+    NormLayout L = norm_layout(cu_seqlens != nullptr, N, T, H, K, V, chunk_size, dtype);
+    return L.valid ? L.bytes : 0;
+}
+
+sgla_status simple_gla_normalized(const void *q, const void *k, const void *v, const float *g, const float *g_gamma,
+                                  const float *initial_state, void *o, float *final_state,
+                                  const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V,
+                                  int chunk_size, sgla_dtype dtype, void *workspace, size_t workspace_bytes,
+                                  void *stream) {
+    const bool varlen = cu_seqlens != nullptr;
+    if (N < (varlen ? 1 : 0) || T < 0) return SGLA_ERR_INVALID_ARGUMENT;
+    if (dtype != SGLA_BF16 && dtype != SGLA_FP32) return SGLA_ERR_INVALID_ARGUMENT;
+    NormLayout L = norm_layout(varlen, N, T, H, K, V, chunk_size, dtype);
+    if (!L.valid) return L.why;
+    if (!workspace || workspace_bytes < L.bytes) return SGLA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return SGLA_ERR_INVALID_ARGUMENT;
+    const int64_t tokens = varlen ? T : N * T;
+    if (tokens > 0 && (!v || !o)) return SGLA_ERR_INVALID_ARGUMENT;
+    const size_t es = dtype == SGLA_BF16 ? 2 : 4;
+    if (!aligned(v, es) || !aligned(o, es) || !aligned(initial_state, 4) || !aligned(final_state, 4))
+        return SGLA_ERR_INVALID_ARGUMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+    void *va = ws + L.off_va, *oa = ws + L.off_oa;
+    float *h0p = initial_state ? reinterpret_cast<float *>(ws + L.off_h0) : nullptr;
+    float *hTp = final_state ? reinterpret_cast<float *>(ws + L.off_hT) : nullptr;
+    const bool bf16 = dtype == SGLA_BF16;
+    SGLA_LAUNCH("augment_v", launch_augment_v(v, va, tokens * H, (int)V, L.Vp, bf16, st));
+    if (h0p) SGLA_LAUNCH("state_repack", launch_state_repack(initial_state, h0p, N * H * K, (int)V + 1, L.Vp, st));
+    const sgla_status r = run_forward(varlen, q, k, va, g, g_gamma, 1.0f, cu_seqlens, N, T, h0p, oa, hTp, H, K, L.Vp,
+                                      chunk_size, dtype, workspace, L.inner.bytes, stream);
+    if (r != SGLA_OK) return r;
+    SGLA_LAUNCH("normalize", launch_normalize(oa, o, tokens * H, (int)V, L.Vp, bf16, st));
+    if (hTp) SGLA_LAUNCH("state_repack", launch_state_repack(hTp, final_state, N * H * K, L.Vp, (int)V + 1, st));
+    return SGLA_OK;
+}
+
+size_t simple_gla_normalized_decode_workspace_size(int64_t N, int64_t H, int64_t V, sgla_dtype dtype) {
+    if (N < 0 || H < 1 || V < 1 || (dtype != SGLA_BF16 && dtype != SGLA_FP32)) return 0;
+    const size_t es = dtype == SGLA_BF16 ? 2 : 4;
+    return 2 * align_up(es * (size_t)N * H * norm_decode_width(V), 256);
+}
+
+sgla_status simple_gla_normalized_decode_step(const void *q, const void *k, const void *v, const float *g,
+                                              const float *g_gamma, float *state, void *o, int64_t N, int64_t H,
+                                              int64_t K, int64_t V, sgla_dtype dtype, void *workspace,
+                                              size_t workspace_bytes, void *stream) {
+    if (N < 0 || H < 1 || K < 1 || V < 1) return SGLA_ERR_INVALID_ARGUMENT;
+    if (dtype != SGLA_BF16 && dtype != SGLA_FP32) return SGLA_ERR_INVALID_ARGUMENT;
+    const int Vs = norm_decode_width(V);
+    if (K > 1024 || Vs > 512) return SGLA_ERR_UNSUPPORTED;
+    const size_t need = simple_gla_normalized_decode_workspace_size(N, H, V, dtype);
+    if (!workspace || workspace_bytes < need) return SGLA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (N == 0) return SGLA_OK;
+    if (!v || !o) return SGLA_ERR_INVALID_ARGUMENT;
+    const size_t es = dtype == SGLA_BF16 ? 2 : 4;
+    if (!aligned(v, es) || !aligned(o, es)) return SGLA_ERR_INVALID_ARGUMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+    void *va = ws, *oa = ws + need / 2;
+    const bool bf16 = dtype == SGLA_BF16;
+    SGLA_LAUNCH("augment_v", launch_augment_v(v, va, N * H, (int)V, Vs, bf16, st));
+    const sgla_status r = simple_gla_decode_step(q, k, va, g, g_gamma, 1.0f, state, oa, N, H, K, Vs, dtype, stream);
+    if (r != SGLA_OK) return r;
+    SGLA_LAUNCH("normalize", launch_normalize(oa, o, N * H, (int)V, Vs, bf16, st));
     return SGLA_OK;
 }
 

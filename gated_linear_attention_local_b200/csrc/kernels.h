@@ -60,6 +60,13 @@ struct RecArgs {
 };
 cudaError_t launch_fused_recurrent(const RecArgs &a, cudaStream_t st);
 
+// Normalised variant through the augmented value: widen v with a ones column (zero
+// padding up to Vp), repack [rows][Vin] states to [rows][Vout], divide by the last
+// column.
+cudaError_t launch_augment_v(const void *v, void *va, int64_t rows, int V, int Vp, bool bf16, cudaStream_t st);
+cudaError_t launch_state_repack(const float *src, float *dst, int64_t rows, int Vin, int Vout, cudaStream_t st);
+cudaError_t launch_normalize(const void *oa, void *o, int64_t rows, int V, int Vp, bool bf16, cudaStream_t st);
+
 // Self-test: one CTA waits on an mbarrier phase nothing completes; writes
 // SGLA_DEVICE_TIMEOUT to *status once the bounded wait has given up.
 cudaError_t launch_wait_timeout_selftest(int *status, cudaStream_t st);

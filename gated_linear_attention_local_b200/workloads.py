@@ -21,6 +21,9 @@ test matrix with gate normalisers 0.1/1/10, scales 0.1/1 and the packed lengths
                 no per-token gate, no states
   decode        256 sequences x 64 single-token steps, H=32 K=V=128, bf16, g per step,
                 state 0.1*N(0,1) fp32 updated in place
+  normalized_prefill  relinear's normalised variant at its measured scale (B=8, T=512,
+                d=2048 as H=16 heads of K=V=128): bf16, g, feature-mapped q, k = |N(0,1)| + 0.1,
+                scale 1 -- simple_gla_normalized
   recurrent_prefill  the inference routing case of section 4 (at most 64 tokens go to
                 the fused recurrence): 256 sequences x 64 tokens, H=32 K=V=128, bf16,
                 g, initial state 0.1*N(0,1), final state -- simple_gla_fused_recurrent
@@ -45,6 +48,9 @@ WORKLOADS = {
                        chunk_size=64),
     "decode": dict(kind="decode", N=256, steps=64, H=32, K=128, V=128, dtype=torch.bfloat16, gate="g",
                    scale=None),
+    "normalized_prefill": dict(kind="dense", entry="normalized", B=8, T=512, H=16, K=128, V=128,
+                               dtype=torch.bfloat16, gate="g", h0=False, final_state=True, scale=1.0,
+                               chunk_size=64, feature_map="abs"),
     "recurrent_prefill": dict(kind="dense", entry="recurrent", B=256, T=64, H=32, K=128, V=128,
                               dtype=torch.bfloat16, gate="g", h0=True, final_state=True, scale=None,
                               chunk_size=64),
@@ -112,8 +118,11 @@ def make_workload(name: str, seed: int = 0):
     else:
         B, T = w["B"], w["T"]
     std = 1.0 / math.sqrt(K) if w.get("qkv_std") == "rsqrt_k" else 1.0
-    q = (torch.randn(B, T, H, K, generator=gen) * std).to(dt)
-    k = (torch.randn(B, T, H, K, generator=gen) * std).to(dt)
+    q = torch.randn(B, T, H, K, generator=gen) * std
+    k = torch.randn(B, T, H, K, generator=gen) * std
+    if w.get("feature_map") == "abs":  # positive feature maps: q.z > 0 for the normalised variant
+        q, k = q.abs() + 0.1, k.abs() + 0.1
+    q, k = q.to(dt), k.to(dt)
     v = (torch.randn(B, T, H, V, generator=gen) * std).to(dt)
     g = F.logsigmoid(torch.randn(B, T, H, generator=gen)) if w["gate"] == "g" else None
     g_gamma = retnet_gammas(H) if w["gate"] == "gamma" else None

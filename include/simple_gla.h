@@ -257,6 +257,43 @@ SGLA_API sgla_status simple_gla_fwd_noalloc(const void *q, const void *k, const 
 SGLA_API sgla_status sgla_workspace_status(const void *workspace, int *device_status, void *stream);
 
 /*
+ * Normalised gated linear attention through the augmented value ("relinear -- convert
+ * pretrained transformers to linear/hybrid-attention models", fla-org kernel
+ * integration): o_t = (q_t^T S_t) / (q_t^T z_t) with the normaliser state
+ * z_t = exp(a_t) z_{t-1} + k_t and scale 1.  A column of ones appended to v turns the
+ * state into [K, V+1] whose last column is z, so one pass gives numerator and
+ * denominator.  q and k are expected to be feature-mapped so that q_t^T z_t > 0 (a
+ * zero denominator gives inf / NaN, as the definition does).
+ *
+ * simple_gla_normalized: the chunked forward of that operator, dense
+ *   (cu_seqlens == NULL, N sequences of T tokens) or packed (as simple_gla_fwd_varlen).
+ *   q, k [tokens,H,K], v, o [tokens,H,V] in dtype; g / g_gamma as simple_gla_fwd;
+ *   initial_state / final_state fp32 [N,H,K,V+1] (the augmented state: columns 0..V-1
+ *   are S, column V is z), NULL for zeros / not written.  1 <= V <= 511; K and the
+ *   other sizes as simple_gla_fwd.  The workspace (simple_gla_normalized_workspace_size,
+ *   256-byte aligned) holds the widened v and output and the padded states besides
+ *   the forward's own workspace, whose status word (sgla_workspace_status) it shares.
+ *
+ * simple_gla_normalized_decode_step: one token of the same operator for N sequences,
+ *   in place on the augmented state [N,H,K,W] fp32 with W = V+1 rounded up to a
+ *   multiple of 4 (columns past V stay 0).  Workspace:
+ *   simple_gla_normalized_decode_workspace_size(N, H, V, dtype) bytes.
+ */
+SGLA_API size_t simple_gla_normalized_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H,
+                                                     int64_t K, int64_t V, int chunk_size, sgla_dtype dtype);
+SGLA_API sgla_status simple_gla_normalized(const void *q, const void *k, const void *v, const float *g,
+                                  const float *g_gamma, const float *initial_state, void *o,
+                                  float *final_state, const int64_t *cu_seqlens, int64_t N, int64_t T,
+                                  int64_t H, int64_t K, int64_t V, int chunk_size, sgla_dtype dtype,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+SGLA_API size_t simple_gla_normalized_decode_workspace_size(int64_t N, int64_t H, int64_t V, sgla_dtype dtype);
+SGLA_API sgla_status simple_gla_normalized_decode_step(const void *q, const void *k, const void *v,
+                                              const float *g, const float *g_gamma, float *state,
+                                              void *o, int64_t N, int64_t H, int64_t K, int64_t V,
+                                              sgla_dtype dtype, void *workspace, size_t workspace_bytes,
+                                              void *stream);
+
+/*
  * Self-test of the library's failure detection (no counterpart on the pages).  Every
  * wait of the tensor-core pipelines on an mbarrier is bounded: after 2 s of wall time
  * the waiting thread gives up, raises its CTA's abort flag (on which the CTA's other

@@ -155,3 +155,19 @@ def simple_gla_decode_step(q, k, v, state, g=None, g_gamma=None, scale=None, thr
     if rc != 0:
         raise RuntimeError(f"sgla_oracle_decode_step failed with code {rc}")
     return o
+
+
+def simple_gla_normalized(q, k, v, g=None, g_gamma=None, initial_state=None, output_final_state=False,
+                          cu_seqlens=None, threads=None, lib_path=None):
+    """Normalised variant, as "relinear" runs it through fla's kernel (fla-org kernel
+    integration): append a column of ones to v, run the recurrence with scale 1 --
+    the state's last column is then the normaliser z and the last output column is
+    q.z -- and divide the other output columns by it.  initial_state and the final
+    state are the augmented [N,H,K,V+1].  Returns (o [B,T,H,V] float64, final_state)."""
+    v = _f64(v)
+    ones = np.ones(v.shape[:-1] + (1,), dtype=np.float64)
+    o_aug, hT = simple_gla_fwd(q, k, np.concatenate([v, ones], axis=-1), g=g, g_gamma=g_gamma, scale=1.0,
+                               initial_state=initial_state, output_final_state=output_final_state,
+                               cu_seqlens=cu_seqlens, threads=threads, lib_path=lib_path)
+    with np.errstate(divide="ignore", invalid="ignore"):  # a zero q.z gives inf / NaN, as defined
+        return o_aug[..., :-1] / o_aug[..., -1:], hT

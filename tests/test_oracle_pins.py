@@ -105,6 +105,11 @@ def pin_golden(lib_path=None):
         k = np.array(c["k"]).reshape(1, T, 1, K)
         v = np.array(c["v"]).reshape(1, T, 1, V)
         g = np.log(np.array(c["gate"])).reshape(1, T, 1)
+        if c.get("normalized"):
+            o, hT = oracle.simple_gla_normalized(q, k, v, g=g, output_final_state=True, lib_path=lib_path)
+            _close(o.reshape(T, V), np.array(c["o"]), 1e-13)
+            _close(hT.reshape(K, V + 1), np.array(c["hT"]), 1e-13)
+            continue
         vf = bool(c.get("state_v_first", False))
         sshape = (V, K) if vf else (K, V)
         h0 = None if c["h0"] is None else np.array(c["h0"]).reshape(1, 1, *sshape)
@@ -233,6 +238,38 @@ def pin_decode_equals_forward(lib_path=None):
     _close(state, h2)
 
 
+def pin_normalized_brute_force(lib_path=None):
+    """The normalised variant against its definition written out for positive
+    (feature-mapped) q, k: o_i = sum_j D_ij (q_i.k_j) v_j / sum_j D_ij (q_i.k_j), with
+    the initial state's S and z entering both sums through the decay from the start."""
+    rng = np.random.default_rng(11)
+    B, T, H, K, V = 2, 23, 2, 3, 4
+    q = np.abs(rng.standard_normal((B, T, H, K))) + 0.1
+    k = np.abs(rng.standard_normal((B, T, H, K))) + 0.1
+    v = rng.standard_normal((B, T, H, V))
+    g = _logsigmoid(rng.standard_normal((B, T, H)))
+    s0 = np.abs(rng.standard_normal((B, H, K, V + 1)))
+    o, hT = oracle.simple_gla_normalized(q, k, v, g=g, initial_state=s0, output_final_state=True,
+                                         lib_path=lib_path)
+    for b in range(B):
+        for h in range(H):
+            a = g[b, :, h]
+            for i in range(T):
+                num = np.zeros(V)
+                den = 0.0
+                for j in range(i + 1):
+                    w = math.exp(math.fsum(a[j + 1:i + 1])) * float(q[b, i, h] @ k[b, j, h])
+                    num += w * v[b, j, h]
+                    den += w
+                lead = math.exp(math.fsum(a[:i + 1]))
+                num += lead * (q[b, i, h] @ s0[b, h, :, :V])
+                den += lead * float(q[b, i, h] @ s0[b, h, :, V])
+                _close(o[b, i, h], num / den)
+            zT = sum(math.exp(math.fsum(a[j + 1:])) * k[b, j, h] for j in range(T)) + \
+                math.exp(math.fsum(a)) * s0[b, h, :, V]
+            _close(hT[b, h, :, V], zT)
+
+
 def pin_linearity(lib_path=None):
     rng = np.random.default_rng(8)
     q, k, v, g, _, _ = _inputs(rng, 1, 30, 2, 3, 4, h0=False)
@@ -248,7 +285,7 @@ def pin_linearity(lib_path=None):
 
 PINS = [pin_golden, pin_brute_force_dense, pin_brute_force_varlen, pin_closed_form_no_decay,
         pin_special_cases, pin_split_invariant, pin_varlen_equals_separate,
-        pin_decode_equals_forward, pin_linearity]
+        pin_decode_equals_forward, pin_linearity, pin_normalized_brute_force]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
