@@ -59,14 +59,14 @@ def algorithmic_counts(w):
     tokens = w["B"] * w["T"] if w["kind"] == "dense" else w["T"]
     e = w["q"].element_size()
     b = tokens * H * (2 * K + 2 * V) * e
-    b += tokens * H * 4 if w["g"] is not None else (H * 4 if w["g_gamma"] is not None else 0)
+    b += w["g"].numel() * 4 if w["g"] is not None else (H * 4 if w["g_gamma"] is not None else 0)
     states = w["N"] * H * K * V * 4
     if w["h0"] is not None:
         b += states
     if w["output_final_state"]:
         b += states
     flops = H * (4 * tokens * K * V + tokens * (C + 1) * (K + V))
-    if w.get("entry") == "recurrent":  # token-serial: state update and read-out per token
+    if w.get("entry") in ("recurrent", "gla"):  # token-serial: state update and read-out per token
         flops = H * tokens * 4 * K * V
     return dict(bytes=b, flops=flops, tokens=tokens)
 
@@ -117,7 +117,7 @@ def roofline(w, counts, kernel_ms, peaks, traffic=None):
     walk (or the decode kernel) moves all compulsory bytes of the call.  The
     token-serial recurrence runs on the FP32 CUDA cores (two FMAs and a multiply per
     state element and token), so its bound is the ALU peak."""
-    if w.get("entry") == "recurrent":
+    if w.get("entry") in ("recurrent", "gla"):
         ach = counts["flops"] / (kernel_ms * 1e-3) / 1e12
         return dict(bound="alu", achieved=round(ach, 3), peak=round(FP32_ALU_TFLOPS, 1), unit="TFLOP/s",
                     frac=round(ach / FP32_ALU_TFLOPS, 4), traffic=traffic,
@@ -227,6 +227,11 @@ def make_step(w, d, sg, ws):
                                      output_final_state=w["output_final_state"], chunk_size=w["chunk_size"],
                                      workspace=ws)
         return step, (lambda: None)
+    if w.get("entry") == "gla":
+        def step():
+            sg.gla_fused_recurrent(d["q"], d["k"], d["v"], d["g"], scale=w["scale"], initial_state=d["h0"],
+                                   output_final_state=w["output_final_state"])
+        return step, (lambda: None)
     if w.get("entry") == "recurrent":
         def step():
             sg.simple_gla_fused_recurrent(d["q"], d["k"], d["v"], g=d["g"], g_gamma=d["g_gamma"], scale=w["scale"],
@@ -247,7 +252,7 @@ def make_step(w, d, sg, ws):
 
 
 def workspace_for(w, sg, device):
-    if w["kind"] == "decode" or w.get("entry") == "recurrent":
+    if w["kind"] == "decode" or w.get("entry") in ("recurrent", "gla"):
         return None
     dt = w["q"].dtype
     if w.get("entry") == "normalized":
@@ -346,6 +351,9 @@ def e2e_measure(w, sg, device, steps, warmup):
             o, ht = sg.simple_gla_normalized(d["q"], d["k"], d["v"], g=d.get("g"), g_gamma=g_gamma,
                                              initial_state=d.get("h0"), output_final_state=w["output_final_state"],
                                              chunk_size=w["chunk_size"], workspace=ws)
+        elif w.get("entry") == "gla":
+            o, ht = sg.gla_fused_recurrent(d["q"], d["k"], d["v"], d["g"], scale=w["scale"], initial_state=d.get("h0"),
+                                           output_final_state=w["output_final_state"])
         elif w.get("entry") == "recurrent":
             o, ht = sg.simple_gla_fused_recurrent(d["q"], d["k"], d["v"], g=d.get("g"), g_gamma=g_gamma,
                                                   scale=w["scale"], initial_state=d.get("h0"),
@@ -412,7 +420,10 @@ def oracle_sample(w, budget_s=12.0):
     def run(tn):
         d, ntok = sub(tn)
         t0 = time.perf_counter()
-        if w.get("entry") == "normalized":
+        if w.get("entry") == "gla":
+            oracle.gla_fwd(d["q"], d["k"], d["v"], d["g"], scale=w["scale"], initial_state=w["h0"],
+                           output_final_state=w["output_final_state"], threads=threads)
+        elif w.get("entry") == "normalized":
             oracle.simple_gla_normalized(d["q"], d["k"], d["v"], g=d["g"], g_gamma=w["g_gamma"],
                                          initial_state=w["h0"], output_final_state=w["output_final_state"],
                                          cu_seqlens=d["cu"], threads=threads)
@@ -493,6 +504,9 @@ def _config_of(w):
     if w.get("entry") == "normalized":
         return dict(entry="simple_gla_normalized", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
                     gate="g" if w["g"] is not None else "none", feature_map="|x|+0.1", scale=1.0)
+    if w.get("entry") == "gla":
+        return dict(entry="gla_fused_recurrent", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
+                    gate="gk [B,T,H,K] = logsigmoid(N(0,1))/16", initial_state=True)
     if w.get("entry") == "recurrent":
         return dict(entry="simple_gla_fused_recurrent", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
                     gate="g" if w["g"] is not None else "none", initial_state=w["h0"] is not None)

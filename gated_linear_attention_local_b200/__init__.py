@@ -25,6 +25,7 @@ Public functions (same names as the C entry points):
   simple_gla_chunk(q, k, v, ..., cu_seqlens=None, chunk_size=64, state_v_first=False)
   simple_gla_normalized(q, k, v, ...) / simple_gla_normalized_decode_step(...) -- the
       normalised variant through the augmented value (states [.., K, V+1])
+  gla_fused_recurrent(q, k, v, gk, ...) -- GLA with a gate vector over the key dimension
   chunk_simple_gla(...)  -- the article's entry-point name; dispatches on cu_seqlens.
   fused_recurrent_simple_gla(...) -- the article's name for simple_gla_fused_recurrent.
 """
@@ -41,6 +42,7 @@ from ._lib import (SGLA_BF16, SGLA_FP32, SGLA_OK, SglaError, lib, library_path, 
 __all__ = ["simple_gla_fwd", "simple_gla_fwd_noalloc", "simple_gla_fwd_varlen", "simple_gla_decode_step", "chunk_simple_gla",
            "simple_gla_fused_recurrent", "fused_recurrent_simple_gla", "simple_gla_chunk",
            "simple_gla_normalized", "simple_gla_normalized_decode_step", "normalized_decode_state_width",
+           "gla_fused_recurrent",
            "fwd_workspace_size", "varlen_workspace_size", "workspace_status", "library_path",
            "SglaError"]
 
@@ -421,6 +423,45 @@ def simple_gla_normalized_decode_step(q, k, v, state, g=None, g_gamma=None, out=
                                                  _ptr(o), N, H, K, V, dt, _ptr(ws), ws.numel(), _stream())
     raise_for_status(st, "simple_gla_normalized_decode_step")
     return o
+
+
+def gla_fused_recurrent(q, k, v, gk, scale=None, initial_state=None, output_final_state=False, cu_seqlens=None,
+                        state_v_first=False, device_status=None):
+    """GLA (gate vector over the key dimension), token-serial: gk fp32 log gates shaped
+    like q.  Other arguments and shapes as simple_gla_fused_recurrent."""
+    _common_checks(q, k, v, None, None, None)
+    _check_cuda("gk", gk, torch.float32)
+    _check_cuda("initial_state", initial_state, torch.float32, 4)
+    if tuple(gk.shape) != tuple(q.shape):
+        raise ValueError(f"gk must be shaped like q {tuple(q.shape)}, got {tuple(gk.shape)}")
+    squeeze = False
+    if cu_seqlens is not None:
+        _check_cuda("cu_seqlens", cu_seqlens, torch.int64, 1)
+        if q.dim() == 4:
+            if q.shape[0] != 1:
+                raise ValueError("with cu_seqlens the batch dimension must be 1")
+            squeeze = True
+            q, k, v, gk = q[0], k[0], v[0], gk[0]
+        N = cu_seqlens.numel() - 1
+        T, H, K = q.shape
+        V = v.shape[2]
+    else:
+        if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+            raise ValueError("q,k must be [B,T,H,K] and v [B,T,H,V]")
+        N, T, H, K = q.shape
+        V = v.shape[3]
+    sshape = (N, H, V, K) if state_v_first else (N, H, K, V)
+    if initial_state is not None and tuple(initial_state.shape) != sshape:
+        raise ValueError(f"initial_state must be {sshape}")
+    if device_status is not None:
+        _check_cuda("device_status", device_status, torch.int32)
+    o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    ht = torch.empty(sshape, dtype=torch.float32, device=q.device) if output_final_state else None
+    st = lib().gla_fused_recurrent(_ptr(q), _ptr(k), _ptr(v), _ptr(gk), ctypes.c_float(_scale(scale)),
+                                   _ptr(initial_state), _ptr(o), _ptr(ht), _ptr(cu_seqlens), N, T, H, K, V,
+                                   1 if state_v_first else 0, _DTYPES[q.dtype], _ptr(device_status), _stream())
+    raise_for_status(st, "gla_fused_recurrent")
+    return (o.unsqueeze(0) if squeeze else o), ht
 
 
 def fused_recurrent_simple_gla(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,

@@ -53,6 +53,8 @@ _SIG = {
     "simple_gla_normalized_decode_workspace_size": ([_I64, _I64, _I64, ctypes.c_int], ctypes.c_size_t),
     "simple_gla_normalized_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_int, _P,
                                            ctypes.c_size_t, _P], ctypes.c_int),
+    "gla_fused_recurrent": ([_P, _P, _P, _P, _F, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int,
+                             ctypes.c_int, _P, _P], ctypes.c_int),
     "sgla_selftest_wait_timeout": ([_P, _P], ctypes.c_int),
     "sgla_kernel_launch_count": ([], ctypes.c_uint64),
     "sgla_profile_begin": ([], ctypes.c_int),

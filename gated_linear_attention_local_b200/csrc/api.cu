@@ -383,12 +383,16 @@ sgla_status simple_gla_decode_step(const void *q, const void *k, const void *v, 
     return SGLA_OK;
 }
 
-sgla_status simple_gla_fused_recurrent(const void *q, const void *k, const void *v, const float *g,
-                                       const float *g_gamma, float scale, const float *initial_state, void *o,
-                                       float *final_state, const int64_t *cu_seqlens, int64_t N, int64_t T,
-                                       int64_t H, int64_t K, int64_t V, int state_v_first, sgla_dtype dtype,
-                                       int *device_status, void *stream) {
-    if (g && g_gamma) return SGLA_ERR_INVALID_ARGUMENT;
+}  // extern "C"
+
+namespace {
+sgla_status fused_recurrent_impl(const void *q, const void *k, const void *v, const float *g, const float *gk,
+                                 const float *g_gamma, float scale, const float *initial_state, void *o,
+                                 float *final_state, const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H,
+                                 int64_t K, int64_t V, int state_v_first, sgla_dtype dtype, int *device_status,
+                                 void *stream) {
+    if ((g != nullptr) + (g_gamma != nullptr) + (gk != nullptr) > 1) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!aligned(gk, 16)) return SGLA_ERR_INVALID_ARGUMENT;
     if (N < 0 || T < 0 || H < 1 || K < 1 || V < 1) return SGLA_ERR_INVALID_ARGUMENT;
     if (cu_seqlens && N < 1) return SGLA_ERR_INVALID_ARGUMENT;
     if (dtype != SGLA_BF16 && dtype != SGLA_FP32) return SGLA_ERR_INVALID_ARGUMENT;
@@ -411,10 +415,32 @@ sgla_status simple_gla_fused_recurrent(const void *q, const void *k, const void 
     a.q = q; a.k = k; a.v = v; a.g = g; a.g_gamma = g_gamma; a.scale = scale;
     a.h0 = initial_state; a.o = o; a.hT = final_state; a.cu = cu_seqlens;
     a.N = N; a.T_dense = cu_seqlens ? 0 : T; a.T_total = tokens;
-    a.H = (int)H; a.K = (int)K; a.V = (int)V;
+    a.H = (int)H; a.K = (int)K; a.V = (int)V; a.gk = gk;
     a.state_v_first = state_v_first != 0; a.bf16 = dtype == SGLA_BF16; a.status = device_status;
-    SGLA_LAUNCH("fused_recurrent", launch_fused_recurrent(a, st));
+    if (gk) SGLA_LAUNCH("gla_fused_recurrent", launch_fused_recurrent(a, st));
+    else SGLA_LAUNCH("fused_recurrent", launch_fused_recurrent(a, st));
     return SGLA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+sgla_status simple_gla_fused_recurrent(const void *q, const void *k, const void *v, const float *g,
+                                       const float *g_gamma, float scale, const float *initial_state, void *o,
+                                       float *final_state, const int64_t *cu_seqlens, int64_t N, int64_t T,
+                                       int64_t H, int64_t K, int64_t V, int state_v_first, sgla_dtype dtype,
+                                       int *device_status, void *stream) {
+    return fused_recurrent_impl(q, k, v, g, nullptr, g_gamma, scale, initial_state, o, final_state, cu_seqlens, N,
+                                T, H, K, V, state_v_first, dtype, device_status, stream);
+}
+
+sgla_status gla_fused_recurrent(const void *q, const void *k, const void *v, const float *gk, float scale,
+                                const float *initial_state, void *o, float *final_state,
+                                const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V,
+                                int state_v_first, sgla_dtype dtype, int *device_status, void *stream) {
+    if (!gk && (cu_seqlens ? T : N * T) > 0) return SGLA_ERR_INVALID_ARGUMENT;
+    return fused_recurrent_impl(q, k, v, nullptr, gk, nullptr, scale, initial_state, o, final_state, cu_seqlens, N,
+                                T, H, K, V, state_v_first, dtype, device_status, stream);
 }
 
 sgla_status sgla_workspace_status(const void *workspace, int *device_status, void *stream) {

@@ -48,6 +48,7 @@ cudaError_t launch_state_transpose(const float *src, float *dst, int64_t mats, i
 struct RecArgs {
     const void *q, *k, *v;
     const float *g, *g_gamma;
+    const float *gk;    // GLA: [tokens, H, K] log gates over the key dimension, or NULL
     float scale;
     const float *h0;
     void *o;

@@ -29,18 +29,24 @@ constexpr int kRecMaxWarps = 16;  // K <= 512
 
 // shared memory of one CTA: two raw (input dtype) token buffers, the fp32 copy of the
 // current block, and the per-warp partial read-outs
+// (with a gate vector over the key dimension, GLA, each buffer also holds the
+// block's [kRecTB][kpad] fp32 log gates and the fp32 copy their decays)
 struct RecSmem {
     int kpad, warps, es;
+    bool gvec;
     __host__ __device__ size_t raw_q() const { return 0; }
     __host__ __device__ size_t raw_k() const { return (size_t)kRecTB * kpad * es; }
     __host__ __device__ size_t raw_v() const { return 2 * (size_t)kRecTB * kpad * es; }
     __host__ __device__ size_t raw_g() const { return raw_v() + (size_t)kRecTB * kRecCols * es; }
-    __host__ __device__ size_t raw_bytes() const { return raw_g() + kRecTB * 4; }
+    __host__ __device__ size_t raw_gk() const { return raw_g() + kRecTB * 4; }  // 16-byte aligned
+    __host__ __device__ size_t raw_bytes() const { return raw_gk() + (gvec ? (size_t)kRecTB * kpad * 4 : 0); }
     __host__ __device__ size_t raw(int b) const { return (size_t)b * ((raw_bytes() + 15) / 16 * 16); }
-    __host__ __device__ size_t f32() const { return raw(2); }  // qs, ks [kRecTB][kpad], vs [kRecTB][64], ds [kRecTB]
-    __host__ __device__ size_t red() const {
+    // qs, ks [kRecTB][kpad], vs [kRecTB][64], ds [kRecTB], then (GLA) dks [kRecTB][kpad]
+    __host__ __device__ size_t f32() const { return raw(2); }
+    __host__ __device__ size_t f32_dk() const {
         return f32() + 4 * ((size_t)2 * kRecTB * kpad + (size_t)kRecTB * kRecCols + kRecTB);
     }
+    __host__ __device__ size_t red() const { return f32_dk() + (gvec ? 4 * (size_t)kRecTB * kpad : 0); }
     __host__ __device__ size_t bytes() const { return red() + 4 * (size_t)kRecTB * warps * kRecCols; }
 };
 
@@ -57,21 +63,23 @@ __device__ __forceinline__ void cp_async4(void *dst, const void *src, int src_by
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_one_pending() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
-template <typename T, bool VFIRST>
+template <typename T, bool VFIRST, bool GVEC>
 __global__ void __launch_bounds__(32 * kRecMaxWarps)
 fused_recurrent_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                       const float *__restrict__ g, const float *__restrict__ g_gamma, float scale,
+                       const float *__restrict__ g, const float *__restrict__ gk, const float *__restrict__ g_gamma,
+                       float scale,
                        const float *h0, T *__restrict__ o, float *hT, const int64_t *__restrict__ cu,
                        int64_t T_dense, int64_t T_total, int H, int K, int V, int *status) {
     extern __shared__ float4 rec_smem4[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(rec_smem4);
     const int nthr = blockDim.x, nwarps = nthr >> 5;
-    const RecSmem L{nwarps * 32, nwarps, (int)sizeof(T)};
+    const RecSmem L{nwarps * 32, nwarps, (int)sizeof(T), GVEC};
     const int kpad = L.kpad;
     float *qs = reinterpret_cast<float *>(smem + L.f32());  // [kRecTB][kpad]
     float *ks = qs + kRecTB * kpad;                          // [kRecTB][kpad]
     float *vs = ks + kRecTB * kpad;                          // [kRecTB][kRecCols]
     float *ds = vs + kRecTB * kRecCols;                      // [kRecTB] decays
+    float *dks = reinterpret_cast<float *>(smem + L.f32_dk());  // [kRecTB][kpad] per-row decays (GLA)
     float *red = reinterpret_cast<float *>(smem + L.red());  // [kRecTB][nwarps][kRecCols]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t n = blockIdx.x / H;
@@ -119,6 +127,15 @@ fused_recurrent_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
             const bool ok = tid < nt;
             cp_async4(base + L.raw_g() + 4 * tid, g + (ok ? (tb + tid) * H + h : 0), ok ? 4 : 0);
         }
+        if constexpr (GVEC) {  // log gates of every key row, 4 per 16-byte copy
+            const int gch = kpad / 4;
+            for (int e = tid; e < kRecTB * gch; e += nthr) {
+                const int t = e / gch, c = (e - t * gch) * 4;
+                const bool ok = t < nt && c < K;
+                const int64_t off = ok ? ((tb + t) * H + h) * (int64_t)K + c : 0;
+                cp_async16(base + L.raw_gk() + ((size_t)t * kpad + c) * 4, gk + off, ok ? 16 : 0);
+            }
+        }
     };
 
     float sa[32], sb[32];  // state rows r0 .. r0+31, columns ca and cb
@@ -162,6 +179,10 @@ fused_recurrent_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
                 ks[e] = to_f32(rk[e]);
             }
             for (int e = tid; e < kRecTB * kRecCols; e += nthr) vs[e] = to_f32(rv[e]);
+            if constexpr (GVEC) {
+                const float *rgk = reinterpret_cast<const float *>(base + L.raw_gk());
+                for (int e = tid; e < kRecTB * kpad; e += nthr) dks[e] = expf(rgk[e]);
+            }
             if (tid < kRecTB) {
                 const float a = g ? reinterpret_cast<const float *>(base + L.raw_g())[tid]
                                   : (g_gamma ? g_gamma[h] : 0.f);
@@ -176,16 +197,22 @@ fused_recurrent_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
             const float2 vv = *reinterpret_cast<const float2 *>(vs + t * kRecCols + ca);
             const float4 *k4 = reinterpret_cast<const float4 *>(ks + t * kpad + r0);
             const float4 *q4 = reinterpret_cast<const float4 *>(qs + t * kpad + r0);
+            const float4 *d4 = reinterpret_cast<const float4 *>(dks + t * kpad + r0);
             float pa = 0.f, pb = 0.f;
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const float4 kk = k4[m], qq = q4[m];
                 const float kj[4] = {kk.x, kk.y, kk.z, kk.w}, qj[4] = {qq.x, qq.y, qq.z, qq.w};
+                float dj[4] = {d, d, d, d};
+                if constexpr (GVEC) {
+                    const float4 dd = d4[m];
+                    dj[0] = dd.x; dj[1] = dd.y; dj[2] = dd.z; dj[3] = dd.w;
+                }
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int j = 4 * m + e;
-                    sa[j] = fmaf(d, sa[j], kj[e] * vv.x);
-                    sb[j] = fmaf(d, sb[j], kj[e] * vv.y);
+                    sa[j] = fmaf(dj[e], sa[j], kj[e] * vv.x);
+                    sb[j] = fmaf(dj[e], sb[j], kj[e] * vv.y);
                     pa = fmaf(qj[e], sa[j], pa);
                     pb = fmaf(qj[e], sb[j], pb);
                 }
@@ -228,12 +255,14 @@ template <typename T>
 cudaError_t launch_rec_typed(const RecArgs &a, cudaStream_t st) {
     const dim3 grid((unsigned)(a.N * a.H), (unsigned)((a.V + kRecCols - 1) / kRecCols));
     const int warps = (a.K + 31) / 32;
-    const size_t smem = RecSmem{32 * warps, warps, (int)sizeof(T)}.bytes();
-    auto kern = a.state_v_first ? fused_recurrent_kernel<T, true> : fused_recurrent_kernel<T, false>;
+    const bool gvec = a.gk != nullptr;
+    const size_t smem = RecSmem{32 * warps, warps, (int)sizeof(T), gvec}.bytes();
+    auto kern = gvec ? (a.state_v_first ? fused_recurrent_kernel<T, true, true> : fused_recurrent_kernel<T, false, true>)
+                     : (a.state_v_first ? fused_recurrent_kernel<T, true, false> : fused_recurrent_kernel<T, false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 32 * warps, smem, st>>>((const T *)a.q, (const T *)a.k, (const T *)a.v, a.g, a.g_gamma, a.scale,
-                                         a.h0, (T *)a.o, a.hT, a.cu, a.T_dense, a.T_total, a.H, a.K, a.V,
+    kern<<<grid, 32 * warps, smem, st>>>((const T *)a.q, (const T *)a.k, (const T *)a.v, a.g, a.gk, a.g_gamma,
+                                         a.scale, a.h0, (T *)a.o, a.hT, a.cu, a.T_dense, a.T_total, a.H, a.K, a.V,
                                          a.status);
     return cudaGetLastError();
 }

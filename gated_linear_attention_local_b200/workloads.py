@@ -24,6 +24,8 @@ test matrix with gate normalisers 0.1/1/10, scales 0.1/1 and the packed lengths
   normalized_prefill  relinear's normalised variant at its measured scale (B=8, T=512,
                 d=2048 as H=16 heads of K=V=128): bf16, g, feature-mapped q, k = |N(0,1)| + 0.1,
                 scale 1 -- simple_gla_normalized
+  gla_recurrent  GLA with a gate vector over the key dimension, token-serial, at the
+                recurrent_prefill size: gk = logsigmoid(N(0,1)) / 16 per key -- gla_fused_recurrent
   recurrent_prefill  the inference routing case of section 4 (at most 64 tokens go to
                 the fused recurrence): 256 sequences x 64 tokens, H=32 K=V=128, bf16,
                 g, initial state 0.1*N(0,1), final state -- simple_gla_fused_recurrent
@@ -51,6 +53,8 @@ WORKLOADS = {
     "normalized_prefill": dict(kind="dense", entry="normalized", B=8, T=512, H=16, K=128, V=128,
                                dtype=torch.bfloat16, gate="g", h0=False, final_state=True, scale=1.0,
                                chunk_size=64, feature_map="abs"),
+    "gla_recurrent": dict(kind="dense", entry="gla", B=256, T=64, H=32, K=128, V=128, dtype=torch.bfloat16,
+                          gate="gk", h0=True, final_state=True, scale=None, chunk_size=64),
     "recurrent_prefill": dict(kind="dense", entry="recurrent", B=256, T=64, H=32, K=128, V=128,
                               dtype=torch.bfloat16, gate="g", h0=True, final_state=True, scale=None,
                               chunk_size=64),
@@ -125,6 +129,8 @@ def make_workload(name: str, seed: int = 0):
     q, k = q.to(dt), k.to(dt)
     v = (torch.randn(B, T, H, V, generator=gen) * std).to(dt)
     g = F.logsigmoid(torch.randn(B, T, H, generator=gen)) if w["gate"] == "g" else None
+    if w["gate"] == "gk":  # GLA: one log gate per key, gate logit normaliser 16 (section 4)
+        g = F.logsigmoid(torch.randn(B, T, H, K, generator=gen)) / 16.0
     g_gamma = retnet_gammas(H) if w["gate"] == "gamma" else None
     N = (len(cu) - 1) if cu is not None else B
     h0 = torch.randn(N, H, K, V, generator=gen) * 0.1 if w["h0"] else None

@@ -257,6 +257,22 @@ SGLA_API sgla_status simple_gla_fwd_noalloc(const void *q, const void *k, const 
 SGLA_API sgla_status sgla_workspace_status(const void *workspace, int *device_status, void *stream);
 
 /*
+ * GLA with a gate vector over the key dimension (the general form; "relinear --
+ * convert pretrained transformers to linear/hybrid-attention models", fla-org kernel
+ * integration, gate-shape item: the head-wise scalar gate of Simple GLA is its
+ * special case): row i of the state decays by its own factor,
+ *   S_t[i][:] <- exp(gk[t,h,i]) S_{t-1}[i][:] + k_t[i] v_t ;  o_t = scale * S_t^T q_t,
+ * computed token by token with the state on chip (the token-serial form; arguments,
+ * layouts, sizes and errors as simple_gla_fused_recurrent, with gk fp32 [tokens,H,K],
+ * 16-byte aligned, in place of g / g_gamma).
+ */
+SGLA_API sgla_status gla_fused_recurrent(const void *q, const void *k, const void *v, const float *gk, float scale,
+                                const float *initial_state, void *o, float *final_state,
+                                const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H, int64_t K,
+                                int64_t V, int state_v_first, sgla_dtype dtype, int *device_status,
+                                void *stream);
+
+/*
  * Normalised gated linear attention through the augmented value ("relinear -- convert
  * pretrained transformers to linear/hybrid-attention models", fla-org kernel
  * integration): o_t = (q_t^T S_t) / (q_t^T z_t) with the normaliser state

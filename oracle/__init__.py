@@ -58,6 +58,9 @@ def _load(lib_path=None):
         lib.sgla_oracle_decode_step.argtypes = [P, P, P, P, P, ctypes.c_double, P, P,
                                                 I64, I64, I64, I64, ctypes.c_int]
         lib.sgla_oracle_decode_step.restype = ctypes.c_int
+        lib.sgla_oracle_gla_fwd.argtypes = [P, P, P, P, ctypes.c_double, P, P, P,
+                                            P, I64, I64, I64, I64, I64, I64, ctypes.c_int]
+        lib.sgla_oracle_gla_fwd.restype = ctypes.c_int
         _libs[path] = lib
     return _libs[path]
 
@@ -171,3 +174,36 @@ def simple_gla_normalized(q, k, v, g=None, g_gamma=None, initial_state=None, out
                                cu_seqlens=cu_seqlens, threads=threads, lib_path=lib_path)
     with np.errstate(divide="ignore", invalid="ignore"):  # a zero q.z gives inf / NaN, as defined
         return o_aug[..., :-1] / o_aug[..., -1:], hT
+
+
+def gla_fwd(q, k, v, gk, scale=None, initial_state=None, output_final_state=False, cu_seqlens=None,
+            threads=None, lib_path=None):
+    """fp64 recurrence of GLA with a gate vector over the key dimension (row i of the
+    state decays by exp(gk_t[i])).  q,k,gk [B,T,H,K]; v [B,T,H,V]; initial_state
+    [N,H,K,V].  Returns (o [B,T,H,V] float64, final_state or None)."""
+    q, k, v, gk, h0 = map(_f64, (q, k, v, gk, initial_state))
+    if q.ndim != 4 or k.shape != q.shape or gk.shape != q.shape or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q,k,gk must be [B,T,H,K] and v [B,T,H,V]")
+    B, T, H, K = q.shape
+    V = v.shape[3]
+    cu = None
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int64))
+        if B != 1:
+            raise ValueError("with cu_seqlens the batch size must be 1")
+        N = cu.shape[0] - 1
+    else:
+        N = B
+    if h0 is not None and h0.shape != (N, H, K, V):
+        raise ValueError(f"initial_state must be [{N},{H},{K},{V}]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(K)
+    o = np.zeros((B, T, H, V), dtype=np.float64)
+    hT = np.zeros((N, H, K, V), dtype=np.float64) if output_final_state else None
+    rc = _load(lib_path).sgla_oracle_gla_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(gk), float(scale), _ptr(h0),
+                                             _ptr(o), _ptr(hT), _ptr(cu), N, B, T, H, K, V,
+                                             int(threads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"sgla_oracle_gla_fwd failed with code {rc}")
+    return o, hT

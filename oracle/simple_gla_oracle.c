@@ -181,3 +181,87 @@ int sgla_oracle_decode_step(const double *q, const double *k, const double *v,
     }
     return err;
 }
+
+/*
+ * GLA with a gate vector over the key dimension (the general form of which the
+ * scalar head-wise gate above is the special case: "relinear -- convert pretrained
+ * transformers to linear/hybrid-attention models", fla-org kernel integration, gate
+ * shape item; "Simple GLA in flash-linear-attention", section 1, contrasts it with
+ * the head-wise gate).  Row i of the state decays by its own factor:
+ *   S_t[i][j] = exp(gk_t[i]) S_{t-1}[i][j] + k_t[i] v_t[j],   o_t = scale * S_t^T q_t.
+ * gk is [tokens, H, K] (log space); everything else as sgla_oracle_fwd.  Token by
+ * token in fp64, no chunking.
+ */
+static void gla_one_head(const double *q, const double *k, const double *v, const double *gk,
+                         double scale, const double *h0, double *o, double *hT,
+                         int64_t t_begin, int64_t t_end, int64_t h, int64_t H,
+                         int64_t K, int64_t V, double *S)
+{
+    if (h0)
+        memcpy(S, h0, (size_t)(K * V) * sizeof(double));
+    else
+        memset(S, 0, (size_t)(K * V) * sizeof(double));
+    for (int64_t t = t_begin; t < t_end; ++t) {
+        const double *qt = q + (t * H + h) * K;
+        const double *kt = k + (t * H + h) * K;
+        const double *vt = v + (t * H + h) * V;
+        const double *gt = gk + (t * H + h) * K;
+        for (int64_t i = 0; i < K; ++i) {
+            const double row_decay = exp(gt[i]);
+            for (int64_t j = 0; j < V; ++j)
+                S[i * V + j] = row_decay * S[i * V + j] + kt[i] * vt[j];
+        }
+        double *ot = o + (t * H + h) * V;
+        for (int64_t j = 0; j < V; ++j) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < K; ++i)
+                acc += qt[i] * S[i * V + j];
+            ot[j] = scale * acc;
+        }
+    }
+    if (hT)
+        memcpy(hT, S, (size_t)(K * V) * sizeof(double));
+}
+
+int sgla_oracle_gla_fwd(const double *q, const double *k, const double *v, const double *gk,
+                        double scale, const double *h0, double *o, double *hT,
+                        const int64_t *cu_seqlens, int64_t N,
+                        int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                        int nthreads)
+{
+    if (!gk)
+        return -1;
+    if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0)
+        return -2;
+    if (cu_seqlens) {
+        if (B != 1 || N < 1 || cu_seqlens[0] != 0 || cu_seqlens[N] != T)
+            return -3;
+        for (int64_t n = 0; n < N; ++n)
+            if (cu_seqlens[n + 1] < cu_seqlens[n])
+                return -4;
+    } else {
+        N = B;
+    }
+    const int64_t units = N * H;
+    int err = 0;
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+    for (int64_t u = 0; u < units; ++u) {
+        const int64_t n = u / H, h = u % H;
+        const int64_t t0 = cu_seqlens ? cu_seqlens[n] : n * T;
+        const int64_t t1 = cu_seqlens ? cu_seqlens[n + 1] : (n + 1) * T;
+        double *S = (double *)malloc((size_t)(K * V) * sizeof(double));
+        if (!S) {
+            err = -5;
+            continue;
+        }
+        const size_t state_off = (size_t)((n * H + h) * K * V);
+        gla_one_head(q, k, v, gk, scale, h0 ? h0 + state_off : NULL, o, hT ? hT + state_off : NULL,
+                     t0, t1, h, H, K, V, S);
+        free(S);
+    }
+    return err;
+}

@@ -99,6 +99,17 @@ def pin_golden(lib_path=None):
     with open(os.path.join(HERE, "golden", "worked_examples.json")) as f:
         cases = json.load(f)["cases"]
     for c in cases:
+        if c.get("gla"):
+            T, K = np.array(c["q"]).shape
+            V = np.array(c["v"]).shape[1]
+            gk = np.log(np.array(c["gate_vec"])).reshape(1, T, 1, K)
+            h0 = np.array(c["h0"]).reshape(1, 1, K, V)
+            o, hT = oracle.gla_fwd(np.array(c["q"]).reshape(1, T, 1, K), np.array(c["k"]).reshape(1, T, 1, K),
+                                   np.array(c["v"]).reshape(1, T, 1, V), gk, scale=c["scale"], initial_state=h0,
+                                   output_final_state=True, lib_path=lib_path)
+            _close(o.reshape(T, V), np.array(c["o"]), 1e-13)
+            _close(hT.reshape(K, V), np.array(c["hT"]), 1e-13)
+            continue
         T, K = np.array(c["q"]).shape
         V = np.array(c["v"]).shape[1]
         q = np.array(c["q"]).reshape(1, T, 1, K)
@@ -270,6 +281,57 @@ def pin_normalized_brute_force(lib_path=None):
             _close(hT[b, h, :, V], zT)
 
 
+def _gla_brute_force_head(q, k, v, gk, scale, h0):
+    """Parallel form of the vector-gate recurrence for one (sequence, head):
+    o_t = scale sum_{j<=t} sum_i q_t[i] k_j[i] exp(sum_{l=j+1..t} gk_l[i]) v_j
+          + scale sum_i q_t[i] exp(sum_{l<=t} gk_l[i]) h0[i]."""
+    T, K = q.shape
+    V = v.shape[1]
+    o = np.zeros((T, V))
+    for t in range(T):
+        for j in range(t + 1):
+            dec = np.array([math.exp(math.fsum(gk[j + 1:t + 1, i])) for i in range(K)])
+            o[t] += scale * float(np.sum(q[t] * k[j] * dec)) * v[j]
+        if h0 is not None:
+            lead = np.array([math.exp(math.fsum(gk[:t + 1, i])) for i in range(K)])
+            o[t] += scale * (q[t] * lead) @ h0
+    ST = np.zeros((K, V))
+    for j in range(T):
+        dec = np.array([math.exp(math.fsum(gk[j + 1:, i])) for i in range(K)])
+        ST += np.outer(dec * k[j], v[j])
+    if h0 is not None:
+        ST += np.array([math.exp(math.fsum(gk[:, i])) for i in range(K)])[:, None] * h0
+    return o, ST
+
+
+def pin_gla_brute_force(lib_path=None):
+    rng = np.random.default_rng(13)
+    for B, T, H, K, V, h0 in [(2, 17, 2, 3, 4, True), (1, 23, 1, 4, 2, False)]:
+        q = rng.standard_normal((B, T, H, K))
+        k = rng.standard_normal((B, T, H, K))
+        v = rng.standard_normal((B, T, H, V))
+        gk = _logsigmoid(rng.standard_normal((B, T, H, K)))
+        s0 = 0.5 * rng.standard_normal((B, H, K, V)) if h0 else None
+        o, hT = oracle.gla_fwd(q, k, v, gk, scale=0.7, initial_state=s0, output_final_state=True, lib_path=lib_path)
+        for b in range(B):
+            for h in range(H):
+                ob, hb = _gla_brute_force_head(q[b, :, h], k[b, :, h], v[b, :, h], gk[b, :, h], 0.7,
+                                               None if s0 is None else s0[b, h])
+                _close(o[b, :, h], ob)
+                _close(hT[b, h], hb)
+
+
+def pin_gla_reduces_to_simple_gla(lib_path=None):
+    """A gate vector with all K entries equal is the head-wise gate of Simple GLA."""
+    rng = np.random.default_rng(17)
+    q, k, v, g, _, s0 = _inputs(rng, 2, 29, 3, 4, 5, "g", 1.0, True)
+    gk = np.repeat(g[..., None], 4, axis=-1)
+    o1, h1 = oracle.gla_fwd(q, k, v, gk, initial_state=s0, output_final_state=True, lib_path=lib_path)
+    o2, h2 = oracle.simple_gla_fwd(q, k, v, g=g, initial_state=s0, output_final_state=True, lib_path=lib_path)
+    _close(o1, o2)
+    _close(h1, h2)
+
+
 def pin_linearity(lib_path=None):
     rng = np.random.default_rng(8)
     q, k, v, g, _, _ = _inputs(rng, 1, 30, 2, 3, 4, h0=False)
@@ -285,7 +347,8 @@ def pin_linearity(lib_path=None):
 
 PINS = [pin_golden, pin_brute_force_dense, pin_brute_force_varlen, pin_closed_form_no_decay,
         pin_special_cases, pin_split_invariant, pin_varlen_equals_separate,
-        pin_decode_equals_forward, pin_linearity, pin_normalized_brute_force]
+        pin_decode_equals_forward, pin_linearity, pin_normalized_brute_force, pin_gla_brute_force,
+        pin_gla_reduces_to_simple_gla]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -305,6 +368,9 @@ MUTATIONS = {
     "last_token_dropped": ("for (int64_t t = t_begin; t < t_end; ++t)",
                            "for (int64_t t = t_begin; t + 1 < t_end; ++t)"),
     "gamma_of_head_zero": ("a = g_gamma[h];", "a = g_gamma[0];"),
+    "gla_gate_of_key_zero": ("const double row_decay = exp(gt[i]);", "const double row_decay = exp(gt[0]);"),
+    "gla_outer_product_transposed": ("row_decay * S[i * V + j] + kt[i] * vt[j]",
+                                     "row_decay * S[i * V + j] + kt[j % K] * vt[i % V]"),
 }
 
 
