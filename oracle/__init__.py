@@ -61,6 +61,9 @@ def _load(lib_path=None):
         lib.sgla_oracle_gla_fwd.argtypes = [P, P, P, P, ctypes.c_double, P, P, P,
                                             P, I64, I64, I64, I64, I64, I64, ctypes.c_int]
         lib.sgla_oracle_gla_fwd.restype = ctypes.c_int
+        lib.sgla_oracle_bwd.argtypes = [P, P, P, P, P, ctypes.c_double, P, P, P, P, P, P, P, P, P,
+                                        P, I64, I64, I64, I64, I64, I64]
+        lib.sgla_oracle_bwd.restype = ctypes.c_int
         _libs[path] = lib
     return _libs[path]
 
@@ -207,3 +210,33 @@ def gla_fwd(q, k, v, gk, scale=None, initial_state=None, output_final_state=Fals
     if rc != 0:
         raise RuntimeError(f"sgla_oracle_gla_fwd failed with code {rc}")
     return o, hT
+
+
+def simple_gla_bwd(q, k, v, do, g=None, g_gamma=None, scale=None, initial_state=None, dht=None, cu_seqlens=None,
+                   lib_path=None):
+    """fp64 reverse-mode of the recurrence (section 3's gradients).  do [B,T,H,V]; dht
+    [N,H,K,V] or None.  Returns dict(dq, dk, dv, dg [B,T,H] or None, dg_gamma [H] or
+    None, dh0 [N,H,K,V] or None -- dh0 only when initial_state is given)."""
+    q, k, v, do, g, g_gamma, h0, dht = map(_f64, (q, k, v, do, g, g_gamma, initial_state, dht))
+    B, T, H, K = q.shape
+    V = v.shape[3]
+    cu = None
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int64))
+        N = cu.shape[0] - 1
+    else:
+        N = B
+    if scale is None:
+        scale = 1.0 / math.sqrt(K)
+    out = dict(dq=np.zeros((B, T, H, K)), dk=np.zeros((B, T, H, K)), dv=np.zeros((B, T, H, V)),
+               dg=np.zeros((B, T, H)) if g is not None else None,
+               dg_gamma=np.zeros(H) if g_gamma is not None else None,
+               dh0=np.zeros((N, H, K, V)) if h0 is not None else None)
+    rc = _load(lib_path).sgla_oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma), float(scale), _ptr(h0),
+                                         _ptr(do), _ptr(dht), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                                         _ptr(out["dg"]), _ptr(out["dg_gamma"]), _ptr(out["dh0"]), _ptr(cu),
+                                         N, B, T, H, K, V)
+    if rc != 0:
+        raise RuntimeError(f"sgla_oracle_bwd failed with code {rc}")
+    return out

@@ -265,3 +265,128 @@ int sgla_oracle_gla_fwd(const double *q, const double *k, const double *v, const
     }
     return err;
 }
+
+/*
+ * Backward of the Simple GLA recurrence (reverse-mode of the loop in
+ * recur_one_head, fp64, one (sequence, head) at a time; "Simple GLA in
+ * flash-linear-attention", section 3, lists the gradients dq, dk, dv, dg and dh0).
+ * Given do (gradient of o) and dhT (gradient of the final state, or NULL):
+ *   dS_t  = scale q_t do_t^T + a_{t+1} dS_{t+1}   (dS_{T-1} also receives dhT)
+ *   dq_t  = scale S_t do_t        dk_t = dS_t v_t        dv_t = dS_t^T k_t
+ *   da_t  = <dS_t, S_{t-1}>       dg_t = a_t da_t  (a_t = exp(g_t))
+ *   dh0   = a_0 dS_0
+ * dg is [tokens, H] for per-token gates, dg_gamma [H] (summed over tokens and
+ * sequences) for a per-head gate; either may be NULL.  All states S_t are kept
+ * (T*K*V doubles per sequence and head): meant for small test sizes.
+ */
+static int bwd_one_head(const double *q, const double *k, const double *v, const double *g,
+                        const double *g_gamma, int gate_mode, double scale, const double *h0,
+                        const double *dout, const double *dhT, double *dq, double *dk, double *dv,
+                        double *dg, double *dgg_h, double *dh0, int64_t t_begin, int64_t t_end,
+                        int64_t h, int64_t H, int64_t K, int64_t V)
+{
+    const int64_t L = t_end - t_begin, KV = K * V;
+    double *S = (double *)calloc((size_t)((L + 1) * KV), sizeof(double));  /* S[0] = h0, S[t+1] = S_t */
+    double *G = (double *)calloc((size_t)KV, sizeof(double));
+    double *a = (double *)calloc((size_t)(L + 1), sizeof(double));
+    if (!S || !G || !a) {
+        free(S); free(G); free(a);
+        return -5;
+    }
+    if (h0)
+        memcpy(S, h0, (size_t)KV * sizeof(double));
+    for (int64_t l = 0; l < L; ++l) {
+        const int64_t t = t_begin + l;
+        double gl = 0.0;
+        if (gate_mode == GATE_PER_TOKEN)
+            gl = g[t * H + h];
+        else if (gate_mode == GATE_PER_HEAD)
+            gl = g_gamma[h];
+        a[l] = exp(gl);
+        const double *kt = k + (t * H + h) * K, *vt = v + (t * H + h) * V;
+        for (int64_t i = 0; i < K; ++i)
+            for (int64_t j = 0; j < V; ++j)
+                S[(l + 1) * KV + i * V + j] = a[l] * S[l * KV + i * V + j] + kt[i] * vt[j];
+    }
+    if (dhT)
+        memcpy(G, dhT, (size_t)KV * sizeof(double));
+    for (int64_t l = L - 1; l >= 0; --l) {
+        const int64_t t = t_begin + l;
+        const double *qt = q + (t * H + h) * K, *kt = k + (t * H + h) * K, *vt = v + (t * H + h) * V;
+        const double *dot = dout + (t * H + h) * V;
+        /* G becomes dS_t: the later tokens' share, decayed by a_{t+1}, plus this token's read-out */
+        if (l + 1 < L)
+            for (int64_t e = 0; e < KV; ++e)
+                G[e] *= a[l + 1];
+        for (int64_t i = 0; i < K; ++i)
+            for (int64_t j = 0; j < V; ++j)
+                G[i * V + j] += scale * qt[i] * dot[j];
+        const double *St = S + (l + 1) * KV, *Sp = S + l * KV;
+        for (int64_t i = 0; i < K; ++i) {
+            double accq = 0.0, acck = 0.0;
+            for (int64_t j = 0; j < V; ++j) {
+                accq += St[i * V + j] * dot[j];
+                acck += G[i * V + j] * vt[j];
+            }
+            dq[(t * H + h) * K + i] = scale * accq;
+            dk[(t * H + h) * K + i] = acck;
+        }
+        for (int64_t j = 0; j < V; ++j) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < K; ++i)
+                acc += G[i * V + j] * kt[i];
+            dv[(t * H + h) * V + j] = acc;
+        }
+        double da = 0.0;
+        for (int64_t e = 0; e < KV; ++e)
+            da += G[e] * Sp[e];
+        if (dg && gate_mode == GATE_PER_TOKEN)
+            dg[t * H + h] = a[l] * da;
+        if (dgg_h && gate_mode == GATE_PER_HEAD)
+            *dgg_h += a[l] * da;
+    }
+    if (dh0) {
+        const double a0 = L > 0 ? a[0] : 1.0;
+        for (int64_t e = 0; e < KV; ++e)
+            dh0[e] = a0 * G[e];
+    }
+    free(S); free(G); free(a);
+    return 0;
+}
+
+int sgla_oracle_bwd(const double *q, const double *k, const double *v, const double *g,
+                    const double *g_gamma, double scale, const double *h0, const double *dout,
+                    const double *dhT, double *dq, double *dk, double *dv, double *dg,
+                    double *dg_gamma, double *dh0, const int64_t *cu_seqlens, int64_t N,
+                    int64_t B, int64_t T, int64_t H, int64_t K, int64_t V)
+{
+    const int gate_mode = gate_mode_of(g, g_gamma);
+    if (gate_mode < 0)
+        return -1;
+    if (B < 0 || T < 0 || H <= 0 || K <= 0 || V <= 0)
+        return -2;
+    if (cu_seqlens) {
+        if (B != 1 || N < 1 || cu_seqlens[0] != 0 || cu_seqlens[N] != T)
+            return -3;
+        for (int64_t n = 0; n < N; ++n)
+            if (cu_seqlens[n + 1] < cu_seqlens[n])
+                return -4;
+    } else {
+        N = B;
+    }
+    if (dg_gamma)
+        for (int64_t h = 0; h < H; ++h)
+            dg_gamma[h] = 0.0;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t h = 0; h < H; ++h) {
+            const int64_t t0 = cu_seqlens ? cu_seqlens[n] : n * T;
+            const int64_t t1 = cu_seqlens ? cu_seqlens[n + 1] : (n + 1) * T;
+            const size_t so = (size_t)((n * H + h) * K * V);
+            const int rc = bwd_one_head(q, k, v, g, g_gamma, gate_mode, scale, h0 ? h0 + so : NULL, dout,
+                                        dhT ? dhT + so : NULL, dq, dk, dv, dg, dg_gamma ? dg_gamma + h : NULL,
+                                        dh0 ? dh0 + so : NULL, t0, t1, h, H, K, V);
+            if (rc)
+                return rc;
+        }
+    return 0;
+}

@@ -332,6 +332,49 @@ def pin_gla_reduces_to_simple_gla(lib_path=None):
     _close(h1, h2)
 
 
+def _fd_grad(f, x, eps=1e-6):
+    """Central finite differences of the scalar f at every element of x (in place)."""
+    gr = np.zeros_like(x)
+    it = np.nditer(x, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        old = x[i]
+        x[i] = old + eps
+        fp = f()
+        x[i] = old - eps
+        fm = f()
+        x[i] = old
+        gr[i] = (fp - fm) / (2 * eps)
+    return gr
+
+
+def pin_backward_finite_differences(lib_path=None):
+    """The reverse-mode backward against central finite differences of the forward
+    for L = sum(o * do) + sum(hT * dhT), every input, per-token and per-head gates,
+    dense and packed."""
+    rng = np.random.default_rng(19)
+    for gate, cu in (("g", None), ("gamma", None), ("g", np.array([0, 2, 2, 7]))):
+        B, T, H, K, V = (1, 7, 2, 3, 2) if cu is not None else (2, 5, 2, 3, 2)
+        q, k, v, g, gg, s0 = _inputs(rng, B, T, H, K, V, gate, 1.0, True)
+        N = len(cu) - 1 if cu is not None else B
+        s0 = 0.5 * rng.standard_normal((N, H, K, V))
+        do = rng.standard_normal((B, T, H, V))
+        dht = rng.standard_normal((N, H, K, V))
+
+        def loss():
+            o, hT = oracle.simple_gla_fwd(q, k, v, g=g, g_gamma=gg, scale=0.8, initial_state=s0,
+                                          output_final_state=True, cu_seqlens=cu, lib_path=lib_path)
+            return float(np.sum(o * do) + np.sum(hT * dht))
+        grads = oracle.simple_gla_bwd(q, k, v, do, g=g, g_gamma=gg, scale=0.8, initial_state=s0, dht=dht,
+                                      cu_seqlens=cu, lib_path=lib_path)
+        for name, x in (("dq", q), ("dk", k), ("dv", v), ("dh0", s0)):
+            _close(grads[name], _fd_grad(loss, x), 1e-6)
+        if g is not None:
+            _close(grads["dg"], _fd_grad(loss, g), 1e-6)
+        else:
+            _close(grads["dg_gamma"], _fd_grad(loss, gg), 1e-6)
+
+
 def pin_linearity(lib_path=None):
     rng = np.random.default_rng(8)
     q, k, v, g, _, _ = _inputs(rng, 1, 30, 2, 3, 4, h0=False)
@@ -348,7 +391,7 @@ def pin_linearity(lib_path=None):
 PINS = [pin_golden, pin_brute_force_dense, pin_brute_force_varlen, pin_closed_form_no_decay,
         pin_special_cases, pin_split_invariant, pin_varlen_equals_separate,
         pin_decode_equals_forward, pin_linearity, pin_normalized_brute_force, pin_gla_brute_force,
-        pin_gla_reduces_to_simple_gla]
+        pin_gla_reduces_to_simple_gla, pin_backward_finite_differences]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -369,6 +412,8 @@ MUTATIONS = {
                            "for (int64_t t = t_begin; t + 1 < t_end; ++t)"),
     "gamma_of_head_zero": ("a = g_gamma[h];", "a = g_gamma[0];"),
     "gla_gate_of_key_zero": ("const double row_decay = exp(gt[i]);", "const double row_decay = exp(gt[0]);"),
+    "bwd_decay_of_current_token": ("                G[e] *= a[l + 1];", "                G[e] *= a[l];"),
+    "bwd_dv_uses_query": ("                acc += G[i * V + j] * kt[i];", "                acc += G[i * V + j] * qt[i];"),
     "gla_outer_product_transposed": ("row_decay * S[i * V + j] + kt[i] * vt[j]",
                                      "row_decay * S[i * V + j] + kt[j % K] * vt[i % V]"),
 }
