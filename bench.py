@@ -68,6 +68,13 @@ def algorithmic_counts(w):
     flops = H * (4 * tokens * K * V + tokens * (C + 1) * (K + V))
     if w.get("entry") in ("recurrent", "gla"):  # token-serial: state update and read-out per token
         flops = H * tokens * 4 * K * V
+    if w.get("entry") == "recurrent_bwd":
+        # read do; write dq, dk, dv, dg; read dht, write dh0.  FLOPs per token and head:
+        # forward sweep 4KV (state update, dq), reverse sweep 6KV (dS update, dk, dv)
+        b += tokens * H * (V + 2 * K + V) * e + w["g"].numel() * 4 + 2 * states
+        kernel = {"recurrent_bwd_forward_sweep": H * tokens * 4 * K * V,
+                  "recurrent_bwd_reverse_sweep": H * tokens * 6 * K * V}
+        return dict(bytes=b, flops=sum(kernel.values()), tokens=tokens, kernel_flops=kernel)
     return dict(bytes=b, flops=flops, tokens=tokens)
 
 
@@ -112,13 +119,14 @@ def captured_traffic(workload, kernel):
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
-def roofline(w, counts, kernel_ms, peaks, traffic=None):
+def roofline(w, counts, kernel_ms, peaks, traffic=None, kernel=None):
     """Roofline object for the dominant kernel of this workload.  The fused output
     walk (or the decode kernel) moves all compulsory bytes of the call.  The
     token-serial recurrence runs on the FP32 CUDA cores (two FMAs and a multiply per
     state element and token), so its bound is the ALU peak."""
-    if w.get("entry") in ("recurrent", "gla"):
-        ach = counts["flops"] / (kernel_ms * 1e-3) / 1e12
+    if w.get("entry") in ("recurrent", "gla", "recurrent_bwd"):
+        flops = counts.get("kernel_flops", {}).get(kernel, counts["flops"])
+        ach = flops / (kernel_ms * 1e-3) / 1e12
         return dict(bound="alu", achieved=round(ach, 3), peak=round(FP32_ALU_TFLOPS, 1), unit="TFLOP/s",
                     frac=round(ach / FP32_ALU_TFLOPS, 4), traffic=traffic,
                     peak_source="derived: 148 SMs x 128 FP32 lanes x 2 x 1965 MHz")
@@ -203,7 +211,7 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- running
 
 def dev_inputs(w, device):
-    keys = ("q", "k", "v", "g", "g_gamma", "h0", "cu_seqlens", "state")
+    keys = ("q", "k", "v", "g", "g_gamma", "h0", "cu_seqlens", "state", "do", "dht")
     return {k: (w[k].to(device) if w.get(k) is not None else None) for k in keys}
 
 
@@ -232,6 +240,11 @@ def make_step(w, d, sg, ws):
             sg.gla_fused_recurrent(d["q"], d["k"], d["v"], d["g"], scale=w["scale"], initial_state=d["h0"],
                                    output_final_state=w["output_final_state"])
         return step, (lambda: None)
+    if w.get("entry") == "recurrent_bwd":
+        def step():
+            sg.simple_gla_fused_recurrent_bwd(d["q"], d["k"], d["v"], d["do"], g=d["g"], g_gamma=d["g_gamma"],
+                                              scale=w["scale"], initial_state=d["h0"], dht=d["dht"], workspace=ws)
+        return step, (lambda: None)
     if w.get("entry") == "recurrent":
         def step():
             sg.simple_gla_fused_recurrent(d["q"], d["k"], d["v"], g=d["g"], g_gamma=d["g_gamma"], scale=w["scale"],
@@ -255,6 +268,9 @@ def workspace_for(w, sg, device):
     if w["kind"] == "decode" or w.get("entry") in ("recurrent", "gla"):
         return None
     dt = w["q"].dtype
+    if w.get("entry") == "recurrent_bwd":
+        n = sg.lib().simple_gla_fused_recurrent_bwd_workspace_size(None, w["B"], w["T"], w["H"], w["K"])
+        return torch.empty(max(int(n), 256), dtype=torch.uint8, device=device)
     if w.get("entry") == "normalized":
         n = sg.lib().simple_gla_normalized_workspace_size(None, w["B"], w["T"], w["H"], w["K"], w["V"],
                                                           w["chunk_size"], sg._DTYPES[dt])
@@ -315,7 +331,7 @@ def dominant(prof):
 def e2e_measure(w, sg, device, steps, warmup):
     """Same metric through the public API with inputs in pinned HOST memory: every
     step copies the inputs host->device, runs the call and reads the result back."""
-    keys = [k for k in ("q", "k", "v", "g", "h0", "cu_seqlens") if w.get(k) is not None]
+    keys = [k for k in ("q", "k", "v", "g", "h0", "cu_seqlens", "do", "dht") if w.get(k) is not None]
     if w["kind"] == "decode":
         keys = ["q", "k", "v", "g", "state"]
     hostin = {k: w[k].pin_memory() for k in keys}
@@ -326,6 +342,10 @@ def e2e_measure(w, sg, device, steps, warmup):
         out_host = torch.empty(w["steps"], w["N"], w["H"], w["V"], dtype=w["q"].dtype).pin_memory()
         st_host = torch.empty_like(w["state"]).pin_memory()
         d2h = out_host.numel() * out_host.element_size() + st_host.numel() * 4
+    elif w.get("entry") == "recurrent_bwd":
+        grads_host = {n: torch.empty_like(w[s]).pin_memory() for n, s in (("dq", "q"), ("dk", "k"), ("dv", "v"),
+                                                                          ("dg", "g"), ("dh0", "h0"))}
+        d2h = sum(t.numel() * t.element_size() for t in grads_host.values())
     else:
         tokens_shape = (w["B"], w["T"]) if w["kind"] == "dense" else (w["T"],)
         out_host = torch.empty(*tokens_shape, w["H"], w["V"], dtype=w["q"].dtype).pin_memory()
@@ -341,6 +361,13 @@ def e2e_measure(w, sg, device, steps, warmup):
                                               scale=w["scale"])
                 out_host[t].copy_(o, non_blocking=True)
             st_host.copy_(d["state"], non_blocking=True)
+            return
+        if w.get("entry") == "recurrent_bwd":
+            r = sg.simple_gla_fused_recurrent_bwd(d["q"], d["k"], d["v"], d["do"], g=d["g"], g_gamma=g_gamma,
+                                                  scale=w["scale"], initial_state=d["h0"], dht=d["dht"],
+                                                  workspace=ws)
+            for n, t in grads_host.items():
+                t.copy_(r[n], non_blocking=True)
             return
         if w["kind"] == "varlen":
             o, ht = sg.simple_gla_fwd_varlen(d["q"][0], d["k"][0], d["v"][0], d["cu_seqlens"], g=d["g"][0],
@@ -420,7 +447,10 @@ def oracle_sample(w, budget_s=12.0):
     def run(tn):
         d, ntok = sub(tn)
         t0 = time.perf_counter()
-        if w.get("entry") == "gla":
+        if w.get("entry") == "recurrent_bwd":
+            oracle.simple_gla_bwd(d["q"], d["k"], d["v"], w["do"][:, :tn], g=d["g"], g_gamma=w["g_gamma"],
+                                  scale=w["scale"], initial_state=w["h0"], dht=w["dht"])
+        elif w.get("entry") == "gla":
             oracle.gla_fwd(d["q"], d["k"], d["v"], d["g"], scale=w["scale"], initial_state=w["h0"],
                            output_final_state=w["output_final_state"], threads=threads)
         elif w.get("entry") == "normalized":
@@ -438,9 +468,11 @@ def oracle_sample(w, budget_s=12.0):
     full_tokens = w["B"] * w["T"] if w["kind"] == "dense" else w["T"]
     tn = int(min(max_t, max(32, 32 * budget_s / max(cal_t, 1e-6))))
     dt, ntok = run(tn)
-    return dict(value=ntok / dt, unit="tokens/s", cores=threads, kind="oracle",
-                sample=f"first {tn} tokens of every sequence ({ntok} of {full_tokens} tokens), all heads, "
-                       f"fp64 naive recurrence ({dt:.1f} s)")
+    what = "fp64 reverse-mode of the naive recurrence" if w.get("entry") == "recurrent_bwd" else \
+        "fp64 naive recurrence"
+    return dict(value=ntok / dt, unit="tokens/s", cores=1 if w.get("entry") == "recurrent_bwd" else threads,
+                kind="oracle", sample=f"first {tn} tokens of every sequence ({ntok} of {full_tokens} tokens), "
+                                      f"all heads, {what} ({dt:.1f} s)")
 
 
 # ----------------------------------------------------------------------------- main
@@ -507,6 +539,9 @@ def _config_of(w):
     if w.get("entry") == "gla":
         return dict(entry="gla_fused_recurrent", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
                     gate="gk [B,T,H,K] = logsigmoid(N(0,1))/16", initial_state=True)
+    if w.get("entry") == "recurrent_bwd":
+        return dict(entry="simple_gla_fused_recurrent_bwd", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
+                    gate="g" if w["g"] is not None else "none", initial_state=True, dht=True)
     if w.get("entry") == "recurrent":
         return dict(entry="simple_gla_fused_recurrent", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
                     gate="g" if w["g"] is not None else "none", initial_state=w["h0"] is not None)
@@ -560,7 +595,7 @@ def measure_workload(name, args, device, world, rank, peaks, steps, warmup, flus
                ms_p10=sorted(per_step)[len(per_step) // 10], ms_p90=sorted(per_step)[(9 * len(per_step)) // 10],
                tflops=counts["flops"] * (w["steps"] if w["kind"] == "decode" else 1) / (ms * 1e-3) / 1e12,
                gbs=counts["bytes"] * (w["steps"] if w["kind"] == "decode" else 1) / (ms * 1e-3) / 1e9,
-               roofline=roofline(w, counts, kernel_ms, peaks, captured_traffic(name, kname)) if kname else None,
+               roofline=roofline(w, counts, kernel_ms, peaks, captured_traffic(name, kname), kname) if kname else None,
                dominant_kernel=dict(name=kname, launches=kn, avg_ms=kernel_ms,
                                     share=(kms / sum(v[1] for v in prof.values())) if prof else None),
                kernels={k: dict(launches=v[0], total_ms=round(v[1], 4)) for k, v in prof.items()},

@@ -443,6 +443,61 @@ sgla_status gla_fused_recurrent(const void *q, const void *k, const void *v, con
                                 T, H, K, V, state_v_first, dtype, device_status, stream);
 }
 
+size_t simple_gla_fused_recurrent_bwd_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H,
+                                                     int64_t K) {
+    if (N < 0 || T < 0 || H < 1 || K < 1) return 0;
+    const int64_t tokens = cu_seqlens ? T : N * T;
+    return 2 * align_up(sizeof(float) * (size_t)tokens * H * K, 256) + align_up(sizeof(float) * (size_t)N * H, 256);
+}
+
+sgla_status simple_gla_fused_recurrent_bwd(const void *q, const void *k, const void *v, const float *g,
+                                           const float *g_gamma, float scale, const float *initial_state,
+                                           const void *dout, const float *dht, void *dq, void *dk, void *dv,
+                                           float *dg, float *dg_gamma, float *dh0, const int64_t *cu_seqlens,
+                                           int64_t N, int64_t T, int64_t H, int64_t K, int64_t V, sgla_dtype dtype,
+                                           void *workspace, size_t workspace_bytes, void *stream) {
+    if (g && g_gamma) return SGLA_ERR_INVALID_ARGUMENT;
+    if (N < 0 || T < 0 || H < 1 || K < 1 || V < 1) return SGLA_ERR_INVALID_ARGUMENT;
+    if (cu_seqlens && N < 1) return SGLA_ERR_INVALID_ARGUMENT;
+    if (dtype != SGLA_BF16 && dtype != SGLA_FP32) return SGLA_ERR_INVALID_ARGUMENT;
+    if (K > 512 || V > 4096) return SGLA_ERR_UNSUPPORTED;
+    if (dg && !g) return SGLA_ERR_INVALID_ARGUMENT;
+    if (dg_gamma && !g_gamma) return SGLA_ERR_INVALID_ARGUMENT;
+    if (dh0 && !initial_state) return SGLA_ERR_INVALID_ARGUMENT;
+    const int64_t tokens = cu_seqlens ? T : N * T;
+    if (tokens >= kMaxTokens || N * H >= kMaxTokens) return SGLA_ERR_UNSUPPORTED;
+    if (tokens > 0 && (!q || !k || !v || !dout || !dq || !dk || !dv)) return SGLA_ERR_INVALID_ARGUMENT;
+    const size_t es = dtype == SGLA_BF16 ? 2 : 4;
+    for (const void *p : {q, k, v, dout, (const void *)dq, (const void *)dk, (const void *)dv})
+        if (!aligned(p, es)) return SGLA_ERR_INVALID_ARGUMENT;
+    for (const void *p : {(const void *)g, (const void *)g_gamma, (const void *)initial_state, (const void *)dht,
+                          (const void *)dg, (const void *)dg_gamma, (const void *)dh0})
+        if (!aligned(p, 4)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!aligned(cu_seqlens, 8)) return SGLA_ERR_INVALID_ARGUMENT;
+    const size_t need = simple_gla_fused_recurrent_bwd_workspace_size(cu_seqlens, N, T, H, K);
+    if (!workspace || workspace_bytes < need) return SGLA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!(scale > 0.f) || isnan(scale) || isinf(scale)) scale = 1.0f / sqrtf((float)K);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    SGLA_CUDA(cudaMemsetAsync(workspace, 0, need, st), "backward workspace reset");
+    if (dg_gamma) SGLA_CUDA(cudaMemsetAsync(dg_gamma, 0, sizeof(float) * H, st), "dg_gamma reset");
+    if (N == 0) return SGLA_OK;
+    char *ws = static_cast<char *>(workspace);
+    const size_t acc = align_up(sizeof(float) * (size_t)tokens * H * K, 256);
+    RecBwdArgs a{};
+    a.q = q; a.k = k; a.v = v; a.dout = dout; a.g = g; a.g_gamma = g_gamma; a.scale = scale;
+    a.h0 = initial_state; a.dhT = dht;
+    a.dqf = reinterpret_cast<float *>(ws); a.dkf = reinterpret_cast<float *>(ws + acc);
+    a.ddot = reinterpret_cast<float *>(ws + 2 * acc);
+    a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dg_gamma = dg_gamma; a.dh0 = dh0; a.cu = cu_seqlens;
+    a.N = N; a.T_dense = cu_seqlens ? 0 : T; a.T_total = tokens;
+    a.H = (int)H; a.K = (int)K; a.V = (int)V; a.bf16 = dtype == SGLA_BF16;
+    SGLA_LAUNCH("recurrent_bwd_forward_sweep", launch_rec_bwd(a, 0, st));
+    SGLA_LAUNCH("recurrent_bwd_reverse_sweep", launch_rec_bwd(a, 1, st));
+    SGLA_LAUNCH("recurrent_bwd_finalize", launch_rec_bwd(a, 2, st));
+    return SGLA_OK;
+}
+
 sgla_status sgla_workspace_status(const void *workspace, int *device_status, void *stream) {
     if (!workspace || !device_status) return SGLA_ERR_INVALID_ARGUMENT;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

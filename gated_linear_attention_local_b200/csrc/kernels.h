@@ -61,6 +61,26 @@ struct RecArgs {
 };
 cudaError_t launch_fused_recurrent(const RecArgs &a, cudaStream_t st);
 
+// Backward of the token-serial recurrence: dq, dk, dv, dg, dg_gamma, dh0 from do and dhT.
+struct RecBwdArgs {
+    const void *q, *k, *v, *dout;
+    const float *g, *g_gamma;
+    float scale;
+    const float *h0, *dhT;
+    float *dqf, *dkf;   // [tokens, H, K] fp32 accumulators, zeroed by the caller
+    float *ddot;        // [N, H] <dhT, hT>, zeroed by the caller (used when dhT)
+    void *dq, *dk, *dv;
+    float *dg;          // [tokens, H] or NULL
+    float *dg_gamma;    // [H], zeroed by the caller, or NULL
+    float *dh0;         // [N, H, K, V] or NULL
+    const int64_t *cu;
+    int64_t N, T_dense, T_total;
+    int H, K, V;
+    bool bf16;
+};
+// part 0: forward sweep (dq, <dhT, hT>); 1: reverse sweep (dv, dk, dh0); 2: finalize (casts, dg)
+cudaError_t launch_rec_bwd(const RecBwdArgs &a, int part, cudaStream_t st);
+
 // Normalised variant through the augmented value: widen v with a ones column (zero
 // padding up to Vp), repack [rows][Vin] states to [rows][Vout], divide by the last
 // column.

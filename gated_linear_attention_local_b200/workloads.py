@@ -26,6 +26,10 @@ test matrix with gate normalisers 0.1/1/10, scales 0.1/1 and the packed lengths
                 scale 1 -- simple_gla_normalized
   gla_recurrent  GLA with a gate vector over the key dimension, token-serial, at the
                 recurrent_prefill size: gk = logsigmoid(N(0,1)) / 16 per key -- gla_fused_recurrent
+  recurrent_bwd  gradients of the token-serial recurrence at relinear's training scale
+                (B=8, T=512, H=16, K=V=128, bf16, g, initial state, output gradient do ~
+                N(0,1) and final-state gradient dht ~ 0.1 N(0,1)) --
+                simple_gla_fused_recurrent_bwd
   recurrent_prefill  the inference routing case of section 4 (at most 64 tokens go to
                 the fused recurrence): 256 sequences x 64 tokens, H=32 K=V=128, bf16,
                 g, initial state 0.1*N(0,1), final state -- simple_gla_fused_recurrent
@@ -55,6 +59,8 @@ WORKLOADS = {
                                chunk_size=64, feature_map="abs"),
     "gla_recurrent": dict(kind="dense", entry="gla", B=256, T=64, H=32, K=128, V=128, dtype=torch.bfloat16,
                           gate="gk", h0=True, final_state=True, scale=None, chunk_size=64),
+    "recurrent_bwd": dict(kind="dense", entry="recurrent_bwd", B=8, T=512, H=16, K=128, V=128,
+                          dtype=torch.bfloat16, gate="g", h0=True, final_state=False, scale=None, chunk_size=64),
     "recurrent_prefill": dict(kind="dense", entry="recurrent", B=256, T=64, H=32, K=128, V=128,
                               dtype=torch.bfloat16, gate="g", h0=True, final_state=True, scale=None,
                               chunk_size=64),
@@ -98,6 +104,15 @@ def random_inputs(B, T, H, K, V, dtype=torch.bfloat16, gate="g", normalizer=1.0,
     return dict(q=q, k=k, v=v, g=g, g_gamma=g_gamma, h0=s0)
 
 
+def random_cotangents(v_shape, N, H, K, V, dtype=torch.bfloat16, dht=True, seed=0, dht_std=0.1):
+    """Seeded output gradients for the backward: do shaped like v (dtype) and dht
+    [N,H,K,V] fp32 (or None).  CPU tensors."""
+    gen = torch.Generator(device="cpu").manual_seed(seed)
+    do = torch.randn(*v_shape, generator=gen).to(dtype)
+    dh = (torch.randn(N, H, K, V, generator=gen) * dht_std) if dht else None
+    return do, dh
+
+
 def make_workload(name: str, seed: int = 0):
     """Inputs of a named workload as CPU tensors plus its call options."""
     w = WORKLOADS[name]
@@ -134,6 +149,9 @@ def make_workload(name: str, seed: int = 0):
     g_gamma = retnet_gammas(H) if w["gate"] == "gamma" else None
     N = (len(cu) - 1) if cu is not None else B
     h0 = torch.randn(N, H, K, V, generator=gen) * 0.1 if w["h0"] else None
+    do = dht = None
+    if w.get("entry") == "recurrent_bwd":
+        do, dht = random_cotangents(v.shape, N, H, K, V, dtype=dt, seed=seed + 1)
     return dict(name=name, kind=w["kind"], entry=w.get("entry", "chunk"), q=q, k=k, v=v, g=g, g_gamma=g_gamma,
                 h0=h0, cu_seqlens=cu, scale=w["scale"], output_final_state=w["final_state"],
-                chunk_size=w["chunk_size"], B=B, T=T, N=N, H=H, K=K, V=V)
+                chunk_size=w["chunk_size"], B=B, T=T, N=N, H=H, K=K, V=V, do=do, dht=dht)

@@ -191,6 +191,38 @@ SGLA_API sgla_status simple_gla_fused_recurrent(const void *q, const void *k, co
                                        int *device_status, void *stream);
 
 /*
+ * Gradients of the token-serial recurrence above (article section 3: the training
+ * path differentiates the operator with fp32 states and recovers the gate gradient
+ * by a reverse cumulative sum; section 5: dq, dk, dv, dg and dh0 are checked).  For
+ * the loss L = sum_t <o_t, do_t> + sum_n <final_state_n, dht_n>, with o and
+ * final_state those of simple_gla_fused_recurrent on the same inputs (state_v_first
+ * = 0):
+ *   dq [tokens,H,K], dk [tokens,H,K], dv [tokens,H,V]  dtype, always written;
+ *   dg [tokens,H] fp32 = dL/dg (only with g; NULL to skip);
+ *   dg_gamma [H] fp32 = dL/dg_gamma, summed over every token of every sequence (only
+ *       with g_gamma; NULL to skip);
+ *   dh0 [N,H,K,V] fp32 = dL/d initial_state (only with initial_state; NULL to skip).
+ * Inputs: q, k, v, g, g_gamma, scale, initial_state, cu_seqlens, N, T, H, K, V, dtype
+ * as simple_gla_fused_recurrent; dout [tokens,H,V] dtype; dht [N,H,K,V] fp32 or NULL
+ * (zero).  A packed sequence whose bounds are not 0 <= start <= end <= T is skipped
+ * (its gradients are not written); tokens outside every sequence are not written.
+ * Supported sizes: 1 <= K <= 512, 1 <= V <= 4096; pointers aligned to their element
+ * size.  workspace: at least simple_gla_fused_recurrent_bwd_workspace_size() bytes,
+ * 256-byte aligned (fp32 accumulators for dq and dk and one scalar per sequence and
+ * head; zeroed by the call).  The state trajectory is recomputed, not stored.
+ */
+SGLA_API size_t simple_gla_fused_recurrent_bwd_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T,
+                                                              int64_t H, int64_t K);
+SGLA_API sgla_status simple_gla_fused_recurrent_bwd(const void *q, const void *k, const void *v,
+                                                    const float *g, const float *g_gamma, float scale,
+                                                    const float *initial_state, const void *dout,
+                                                    const float *dht, void *dq, void *dk, void *dv,
+                                                    float *dg, float *dg_gamma, float *dh0,
+                                                    const int64_t *cu_seqlens, int64_t N, int64_t T,
+                                                    int64_t H, int64_t K, int64_t V, sgla_dtype dtype,
+                                                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * The chunked forward with every option of chunk_simple_gla (article section 2) in
  * one call: dense (cu_seqlens == NULL: N sequences of T tokens, q [N,T,H,K]) or
  * packed (cu_seqlens != NULL: N sequences in T tokens, exactly as

@@ -130,6 +130,32 @@ def test_fused_recurrent_validation_on_the_host(lib):
     assert call(N=0) == L.SGLA_OK                                     # nothing to do, nothing launched
 
 
+def test_fused_recurrent_bwd_validation_on_the_host(lib):
+    f = lib.simple_gla_fused_recurrent_bwd
+    ws_need = lib.simple_gla_fused_recurrent_bwd_workspace_size(None, 4, 8, 2, 64)
+    assert ws_need >= 2 * 4 * 8 * 2 * 64 * 4 + 4 * 2 * 4   # fp32 dq, dk and one scalar per (sequence, head)
+    assert lib.simple_gla_fused_recurrent_bwd_workspace_size(None, 4, 8, 0, 64) == 0
+
+    def call(q=FAKE, g=None, gg=None, h0=None, dht=None, dg=None, dgg=None, dh0=None, cu=None, N=4, T=8, H=2,
+             K=64, V=64, dt=L.SGLA_BF16, ws=FAKE, nws=None):
+        return f(q, FAKE, FAKE, g, gg, 1.0, h0, FAKE, dht, FAKE, FAKE, FAKE, dg, dgg, dh0, cu, N, T, H, K, V, dt, ws,
+                 ws_need if nws is None else nws, None)
+
+    assert call(g=FAKE, gg=FAKE) == L.SGLA_ERR_INVALID_ARGUMENT       # both gates
+    assert call(K=520) == L.SGLA_ERR_UNSUPPORTED                      # K above 512
+    assert call(V=4100) == L.SGLA_ERR_UNSUPPORTED                     # V above 4096
+    assert call(dg=FAKE) == L.SGLA_ERR_INVALID_ARGUMENT               # dg without g
+    assert call(g=FAKE, dgg=FAKE) == L.SGLA_ERR_INVALID_ARGUMENT      # dg_gamma without g_gamma
+    assert call(dh0=FAKE) == L.SGLA_ERR_INVALID_ARGUMENT              # dh0 without an initial state
+    assert call(q=FAKE + 1) == L.SGLA_ERR_INVALID_ARGUMENT            # q not aligned to its element
+    assert call(q=None) == L.SGLA_ERR_INVALID_ARGUMENT                # tokens but no q
+    assert call(cu=FAKE, N=0) == L.SGLA_ERR_INVALID_ARGUMENT          # packed with no sequence
+    assert call(nws=ws_need - 4) == L.SGLA_ERR_WORKSPACE              # workspace too small
+    assert call(ws=None) == L.SGLA_ERR_WORKSPACE                      # no workspace
+    assert call(ws=FAKE + 16) == L.SGLA_ERR_INVALID_ARGUMENT          # workspace not 256-byte aligned
+    assert call(dt=7) == L.SGLA_ERR_INVALID_ARGUMENT                  # unknown dtype
+
+
 def test_binding_refuses_cpu_tensors():
     import gated_linear_attention_local_b200 as sg
     x = torch.zeros(1, 8, 1, 16)
