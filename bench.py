@@ -22,6 +22,7 @@ sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import functools
 import json
 import math
 import os
@@ -68,13 +69,19 @@ def algorithmic_counts(w):
     flops = H * (4 * tokens * K * V + tokens * (C + 1) * (K + V))
     if w.get("entry") in ("recurrent", "gla"):  # token-serial: state update and read-out per token
         flops = H * tokens * 4 * K * V
-    if w.get("entry") == "recurrent_bwd":
-        # read do; write dq, dk, dv, dg; read dht, write dh0.  FLOPs per token and head:
-        # forward sweep 4KV (state update, dq), reverse sweep 6KV (dS update, dk, dv)
+    if w.get("entry") in ("recurrent_bwd", "chunk_bwd"):
+        fwd = dict(bytes=b, flops=flops)  # one forward call with these operands (K == V)
+        # read do; write dq, dk, dv, dg; read dht, write dh0
         b += tokens * H * (V + 2 * K + V) * e + w["g"].numel() * 4 + 2 * states
-        kernel = {"recurrent_bwd_forward_sweep": H * tokens * 4 * K * V,
-                  "recurrent_bwd_reverse_sweep": H * tokens * 6 * K * V}
-        return dict(bytes=b, flops=sum(kernel.values()), tokens=tokens, kernel_flops=kernel)
+        if w["entry"] == "chunk_bwd":
+            # three chunked forward calls (dv, dk, dq); the output walk of each moves
+            # that call's compulsory bytes
+            return dict(bytes=b, flops=3 * flops, tokens=tokens, kernel={"chunk_output_tc": fwd})
+        # token-serial FLOPs per token and head: forward sweep 4KV (state update, dq),
+        # reverse sweep 6KV (dS update, dk, dv)
+        kernel = {"recurrent_bwd_forward_sweep": dict(bytes=b, flops=H * tokens * 4 * K * V),
+                  "recurrent_bwd_reverse_sweep": dict(bytes=b, flops=H * tokens * 6 * K * V)}
+        return dict(bytes=b, flops=H * tokens * 10 * K * V, tokens=tokens, kernel=kernel)
     return dict(bytes=b, flops=flops, tokens=tokens)
 
 
@@ -124,22 +131,22 @@ def roofline(w, counts, kernel_ms, peaks, traffic=None, kernel=None):
     walk (or the decode kernel) moves all compulsory bytes of the call.  The
     token-serial recurrence runs on the FP32 CUDA cores (two FMAs and a multiply per
     state element and token), so its bound is the ALU peak."""
+    kc = counts.get("kernel", {}).get(kernel, counts)  # per-launch counts of that kernel
     if w.get("entry") in ("recurrent", "gla", "recurrent_bwd"):
-        flops = counts.get("kernel_flops", {}).get(kernel, counts["flops"])
-        ach = flops / (kernel_ms * 1e-3) / 1e12
+        ach = kc["flops"] / (kernel_ms * 1e-3) / 1e12
         return dict(bound="alu", achieved=round(ach, 3), peak=round(FP32_ALU_TFLOPS, 1), unit="TFLOP/s",
                     frac=round(ach / FP32_ALU_TFLOPS, 4), traffic=traffic,
                     peak_source="derived: 148 SMs x 128 FP32 lanes x 2 x 1965 MHz")
-    t_bytes = counts["bytes"] / (peaks["hbm_gbs"] * 1e9)
-    t_flops = counts["flops"] / (peaks["bf16_tflops"] * 1e12)
+    t_bytes = kc["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_flops = kc["flops"] / (peaks["bf16_tflops"] * 1e12)
     if w["kind"] != "decode" and w.get("dtype_name") == "fp32":
         t_flops = 0.0  # FFMA path: never tensor-bound; report HBM
     if t_flops > t_bytes:
-        ach = counts["flops"] / (kernel_ms * 1e-3) / 1e12
+        ach = kc["flops"] / (kernel_ms * 1e-3) / 1e12
         return dict(bound="tensor", achieved=round(ach, 3), peak=peaks["bf16_tflops"], unit="TFLOP/s",
                     frac=round(ach / peaks["bf16_tflops"], 4), traffic=traffic,
                     peak_source=peaks["source"])
-    ach = counts["bytes"] / (kernel_ms * 1e-3) / 1e9
+    ach = kc["bytes"] / (kernel_ms * 1e-3) / 1e9
     return dict(bound="hbm", achieved=round(ach, 1), peak=peaks["hbm_gbs"], unit="GB/s",
                 frac=round(ach / peaks["hbm_gbs"], 4), traffic=traffic, peak_source=peaks["source"])
 
@@ -240,10 +247,13 @@ def make_step(w, d, sg, ws):
             sg.gla_fused_recurrent(d["q"], d["k"], d["v"], d["g"], scale=w["scale"], initial_state=d["h0"],
                                    output_final_state=w["output_final_state"])
         return step, (lambda: None)
-    if w.get("entry") == "recurrent_bwd":
+    if w.get("entry") in ("recurrent_bwd", "chunk_bwd"):
+        fn = sg.simple_gla_fused_recurrent_bwd if w["entry"] == "recurrent_bwd" else \
+            functools.partial(sg.simple_gla_chunk_bwd, chunk_size=w["chunk_size"])
+
         def step():
-            sg.simple_gla_fused_recurrent_bwd(d["q"], d["k"], d["v"], d["do"], g=d["g"], g_gamma=d["g_gamma"],
-                                              scale=w["scale"], initial_state=d["h0"], dht=d["dht"], workspace=ws)
+            fn(d["q"], d["k"], d["v"], d["do"], g=d["g"], g_gamma=d["g_gamma"], scale=w["scale"],
+               initial_state=d["h0"], dht=d["dht"], workspace=ws)
         return step, (lambda: None)
     if w.get("entry") == "recurrent":
         def step():
@@ -270,6 +280,10 @@ def workspace_for(w, sg, device):
     dt = w["q"].dtype
     if w.get("entry") == "recurrent_bwd":
         n = sg.lib().simple_gla_fused_recurrent_bwd_workspace_size(None, w["B"], w["T"], w["H"], w["K"])
+        return torch.empty(max(int(n), 256), dtype=torch.uint8, device=device)
+    if w.get("entry") == "chunk_bwd":
+        n = sg.lib().simple_gla_chunk_bwd_workspace_size(None, w["B"], w["T"], w["H"], w["K"], w["V"],
+                                                         w["chunk_size"], sg._DTYPES[dt])
         return torch.empty(max(int(n), 256), dtype=torch.uint8, device=device)
     if w.get("entry") == "normalized":
         n = sg.lib().simple_gla_normalized_workspace_size(None, w["B"], w["T"], w["H"], w["K"], w["V"],
@@ -342,7 +356,7 @@ def e2e_measure(w, sg, device, steps, warmup):
         out_host = torch.empty(w["steps"], w["N"], w["H"], w["V"], dtype=w["q"].dtype).pin_memory()
         st_host = torch.empty_like(w["state"]).pin_memory()
         d2h = out_host.numel() * out_host.element_size() + st_host.numel() * 4
-    elif w.get("entry") == "recurrent_bwd":
+    elif w.get("entry") in ("recurrent_bwd", "chunk_bwd"):
         grads_host = {n: torch.empty_like(w[s]).pin_memory() for n, s in (("dq", "q"), ("dk", "k"), ("dv", "v"),
                                                                           ("dg", "g"), ("dh0", "h0"))}
         d2h = sum(t.numel() * t.element_size() for t in grads_host.values())
@@ -362,10 +376,11 @@ def e2e_measure(w, sg, device, steps, warmup):
                 out_host[t].copy_(o, non_blocking=True)
             st_host.copy_(d["state"], non_blocking=True)
             return
-        if w.get("entry") == "recurrent_bwd":
-            r = sg.simple_gla_fused_recurrent_bwd(d["q"], d["k"], d["v"], d["do"], g=d["g"], g_gamma=g_gamma,
-                                                  scale=w["scale"], initial_state=d["h0"], dht=d["dht"],
-                                                  workspace=ws)
+        if w.get("entry") in ("recurrent_bwd", "chunk_bwd"):
+            fn = sg.simple_gla_fused_recurrent_bwd if w["entry"] == "recurrent_bwd" else \
+                functools.partial(sg.simple_gla_chunk_bwd, chunk_size=w["chunk_size"])
+            r = fn(d["q"], d["k"], d["v"], d["do"], g=d["g"], g_gamma=g_gamma, scale=w["scale"],
+                   initial_state=d["h0"], dht=d["dht"], workspace=ws)
             for n, t in grads_host.items():
                 t.copy_(r[n], non_blocking=True)
             return
@@ -447,7 +462,7 @@ def oracle_sample(w, budget_s=12.0):
     def run(tn):
         d, ntok = sub(tn)
         t0 = time.perf_counter()
-        if w.get("entry") == "recurrent_bwd":
+        if w.get("entry") in ("recurrent_bwd", "chunk_bwd"):
             oracle.simple_gla_bwd(d["q"], d["k"], d["v"], w["do"][:, :tn], g=d["g"], g_gamma=w["g_gamma"],
                                   scale=w["scale"], initial_state=w["h0"], dht=w["dht"])
         elif w.get("entry") == "gla":
@@ -468,9 +483,9 @@ def oracle_sample(w, budget_s=12.0):
     full_tokens = w["B"] * w["T"] if w["kind"] == "dense" else w["T"]
     tn = int(min(max_t, max(32, 32 * budget_s / max(cal_t, 1e-6))))
     dt, ntok = run(tn)
-    what = "fp64 reverse-mode of the naive recurrence" if w.get("entry") == "recurrent_bwd" else \
-        "fp64 naive recurrence"
-    return dict(value=ntok / dt, unit="tokens/s", cores=1 if w.get("entry") == "recurrent_bwd" else threads,
+    bwd = w.get("entry") in ("recurrent_bwd", "chunk_bwd")
+    what = "fp64 reverse-mode of the naive recurrence" if bwd else "fp64 naive recurrence"
+    return dict(value=ntok / dt, unit="tokens/s", cores=1 if bwd else threads,
                 kind="oracle", sample=f"first {tn} tokens of every sequence ({ntok} of {full_tokens} tokens), "
                                       f"all heads, {what} ({dt:.1f} s)")
 
@@ -539,6 +554,9 @@ def _config_of(w):
     if w.get("entry") == "gla":
         return dict(entry="gla_fused_recurrent", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
                     gate="gk [B,T,H,K] = logsigmoid(N(0,1))/16", initial_state=True)
+    if w.get("entry") == "chunk_bwd":
+        return dict(entry="simple_gla_chunk_bwd", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
+                    chunk_size=w["chunk_size"], gate="g", initial_state=True, dht=True)
     if w.get("entry") == "recurrent_bwd":
         return dict(entry="simple_gla_fused_recurrent_bwd", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
                     gate="g" if w["g"] is not None else "none", initial_state=True, dht=True)

@@ -42,7 +42,7 @@ from ._lib import (SGLA_BF16, SGLA_FP32, SGLA_OK, SglaError, lib, library_path, 
 __all__ = ["simple_gla_fwd", "simple_gla_fwd_noalloc", "simple_gla_fwd_varlen", "simple_gla_decode_step", "chunk_simple_gla",
            "simple_gla_fused_recurrent", "fused_recurrent_simple_gla", "simple_gla_chunk",
            "simple_gla_normalized", "simple_gla_normalized_decode_step", "normalized_decode_state_width",
-           "gla_fused_recurrent", "simple_gla_fused_recurrent_bwd",
+           "gla_fused_recurrent", "simple_gla_fused_recurrent_bwd", "simple_gla_chunk_bwd",
            "fwd_workspace_size", "varlen_workspace_size", "workspace_status", "library_path",
            "SglaError"]
 
@@ -354,13 +354,9 @@ def simple_gla_fused_recurrent(q, k, v, g=None, g_gamma=None, scale=None, initia
     return (o.unsqueeze(0) if squeeze else o), ht
 
 
-def simple_gla_fused_recurrent_bwd(q, k, v, do, g=None, g_gamma=None, scale=None, initial_state=None, dht=None,
-                                   cu_seqlens=None, workspace=None):
-    """Gradients of simple_gla_fused_recurrent (state_v_first off) for the loss
-    sum(o * do) + sum(final_state * dht).  Shapes as the forward; do like v; dht like
-    the final state or None.  Returns dict(dq, dk, dv, dg, dg_gamma, dh0): dq, dk, dv
-    in the dtype and shape of q, k, v; dg like g (None without g); dg_gamma [H] (None
-    without g_gamma); dh0 like initial_state (None without it)."""
+def _bwd_prepare(q, k, v, do, g, g_gamma, initial_state, dht, cu_seqlens):
+    """Checks shared by the two backward entry points; returns (N, T, H, K, V) and the
+    output tensors."""
     _common_checks(q, k, v, g, g_gamma, initial_state)
     _check_cuda("do", do, q.dtype)
     _check_cuda("dht", dht, torch.float32, 4)
@@ -392,20 +388,48 @@ def simple_gla_fused_recurrent_bwd(q, k, v, do, g=None, g_gamma=None, scale=None
     for name, t in (("initial_state", initial_state), ("dht", dht)):
         if t is not None and tuple(t.shape) != (N, H, K, V):
             raise ValueError(f"{name} must be {(N, H, K, V)}")
-    dq = torch.empty_like(q)
-    dk = torch.empty_like(k)
-    dv = torch.empty_like(v)
-    dg = torch.zeros_like(g) if g is not None else None
-    dg_gamma = torch.empty_like(g_gamma) if g_gamma is not None else None
-    dh0 = torch.empty_like(initial_state) if initial_state is not None else None
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               dg=torch.zeros_like(g) if g is not None else None,
+               dg_gamma=torch.empty_like(g_gamma) if g_gamma is not None else None,
+               dh0=torch.empty_like(initial_state) if initial_state is not None else None)
+    return (N, T, H, K, V), out
+
+
+def simple_gla_fused_recurrent_bwd(q, k, v, do, g=None, g_gamma=None, scale=None, initial_state=None, dht=None,
+                                   cu_seqlens=None, workspace=None):
+    """Gradients of simple_gla_fused_recurrent (state_v_first off) for the loss
+    sum(o * do) + sum(final_state * dht).  Shapes as the forward; do like v; dht like
+    the final state or None.  Returns dict(dq, dk, dv, dg, dg_gamma, dh0): dq, dk, dv
+    in the dtype and shape of q, k, v; dg like g (None without g); dg_gamma [H] (None
+    without g_gamma); dh0 like initial_state (None without it)."""
+    (N, T, H, K, V), out = _bwd_prepare(q, k, v, do, g, g_gamma, initial_state, dht, cu_seqlens)
     nbytes = int(lib().simple_gla_fused_recurrent_bwd_workspace_size(_ptr(cu_seqlens), N, T, H, K))
     ws = _workspace(nbytes, q.device, workspace)
     st = lib().simple_gla_fused_recurrent_bwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma), ctypes.c_float(_scale(scale)), _ptr(initial_state),
-        _ptr(do), _ptr(dht), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dg_gamma), _ptr(dh0), _ptr(cu_seqlens),
-        N, T, H, K, V, _DTYPES[q.dtype], _ptr(ws), ws.numel(), _stream())
+        _ptr(do), _ptr(dht), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dg_gamma"]),
+        _ptr(out["dh0"]), _ptr(cu_seqlens), N, T, H, K, V, _DTYPES[q.dtype], _ptr(ws), ws.numel(), _stream())
     raise_for_status(st, "simple_gla_fused_recurrent_bwd")
-    return dict(dq=dq, dk=dk, dv=dv, dg=dg, dg_gamma=dg_gamma, dh0=dh0)
+    return out
+
+
+def simple_gla_chunk_bwd(q, k, v, do, g=None, g_gamma=None, scale=None, initial_state=None, dht=None,
+                         cu_seqlens=None, chunk_size=64, workspace=None):
+    """Gradients of simple_gla_chunk (state_v_first off) on the tensor-core path, for
+    the loss sum(o * do) + sum(final_state * dht).  Arguments and result as
+    simple_gla_fused_recurrent_bwd, plus chunk_size."""
+    (N, T, H, K, V), out = _bwd_prepare(q, k, v, do, g, g_gamma, initial_state, dht, cu_seqlens)
+    dt = _DTYPES[q.dtype]
+    nbytes = int(lib().simple_gla_chunk_bwd_workspace_size(_ptr(cu_seqlens), N, T, H, K, V, chunk_size, dt))
+    if nbytes == 0:
+        raise_for_status(_size_status(K, V, chunk_size), "simple_gla_chunk_bwd")
+    ws = _workspace(nbytes, q.device, workspace)
+    st = lib().simple_gla_chunk_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma), ctypes.c_float(_scale(scale)), _ptr(initial_state),
+        _ptr(do), _ptr(dht), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dg_gamma"]),
+        _ptr(out["dh0"]), _ptr(cu_seqlens), N, T, H, K, V, chunk_size, dt, _ptr(ws), ws.numel(), _stream())
+    raise_for_status(st, "simple_gla_chunk_bwd")
+    return out
 
 
 def simple_gla_normalized(q, k, v, g=None, g_gamma=None, initial_state=None, output_final_state=False,

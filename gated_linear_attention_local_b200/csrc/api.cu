@@ -293,6 +293,45 @@ NormLayout norm_layout(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, 
 
 int norm_decode_width(int64_t V) { return (int)((V + 1 + 3) / 4 * 4); }
 
+// Chunked backward: three forward calls share the inner workspace (at offset 0, so
+// that its status word is the one sgla_workspace_status reads), followed by the
+// time-reversed operands, the reversed dk / dv, q.dq - k.dk per row and five states
+// (dhT / scale in both layouts, h0 transposed, and the final states of calls A and C).
+struct BwdLayout {
+    bool valid = false;
+    sgla_status why = SGLA_ERR_INVALID_ARGUMENT;
+    size_t inner = 0, off_qr = 0, off_kr = 0, off_vr = 0, off_dor = 0, off_gr = 0, off_dkr = 0, off_dvr = 0,
+           off_x = 0, off_s0 = 0, off_s0T = 0, off_h0T = 0, off_xf = 0, off_hT = 0, bytes = 0;
+};
+
+BwdLayout bwd_layout(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V, int C, sgla_dtype dtype) {
+    BwdLayout L;
+    const Plan a = make_plan(varlen, N, T, H, K, V, C, dtype, true, false);
+    const Plan b = make_plan(varlen, N, T, H, V, K, C, dtype, true, false);
+    if (!a.valid || !b.valid) { L.why = !a.valid ? a.why : b.why; return L; }
+    L.inner = std::max(a.bytes, b.bytes);  // call C needs no more than call B
+    const int64_t rows = (varlen ? T : N * T) * H;
+    const size_t es = dtype == SGLA_BF16 ? 2 : 4, st = sizeof(float) * (size_t)N * H * K * V;
+    size_t off = align_up(L.inner, 256);
+    auto take = [&](size_t &o, size_t n) { o = off; off = align_up(off + n, 256); };
+    take(L.off_qr, es * rows * K);
+    take(L.off_kr, es * rows * K);
+    take(L.off_vr, es * rows * V);
+    take(L.off_dor, es * rows * V);
+    take(L.off_gr, sizeof(float) * rows);
+    take(L.off_dkr, es * rows * K);
+    take(L.off_dvr, es * rows * V);
+    take(L.off_x, sizeof(float) * rows);
+    take(L.off_s0, st);
+    take(L.off_s0T, st);
+    take(L.off_h0T, st);
+    take(L.off_xf, st);
+    take(L.off_hT, st);
+    L.bytes = off;
+    L.valid = true;
+    return L;
+}
+
 }  // namespace
 
 extern "C" {
@@ -441,6 +480,81 @@ sgla_status gla_fused_recurrent(const void *q, const void *k, const void *v, con
     if (!gk && (cu_seqlens ? T : N * T) > 0) return SGLA_ERR_INVALID_ARGUMENT;
     return fused_recurrent_impl(q, k, v, nullptr, gk, nullptr, scale, initial_state, o, final_state, cu_seqlens, N,
                                 T, H, K, V, state_v_first, dtype, device_status, stream);
+}
+
+size_t simple_gla_chunk_bwd_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H, int64_t K,
+                                           int64_t V, int chunk_size, sgla_dtype dtype) {
+    const BwdLayout L = bwd_layout(cu_seqlens != nullptr, N, T, H, K, V, chunk_size, dtype);
+    return L.valid ? L.bytes : 0;
+}
+
+sgla_status simple_gla_chunk_bwd(const void *q, const void *k, const void *v, const float *g, const float *g_gamma,
+                                 float scale, const float *initial_state, const void *dout, const float *dht,
+                                 void *dq, void *dk, void *dv, float *dg, float *dg_gamma, float *dh0,
+                                 const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V,
+                                 int chunk_size, sgla_dtype dtype, void *workspace, size_t workspace_bytes,
+                                 void *stream) {
+    const bool varlen = cu_seqlens != nullptr;
+    if (g && g_gamma) return SGLA_ERR_INVALID_ARGUMENT;
+    if (N < (varlen ? 1 : 0) || T < 0) return SGLA_ERR_INVALID_ARGUMENT;
+    if (dtype != SGLA_BF16 && dtype != SGLA_FP32) return SGLA_ERR_INVALID_ARGUMENT;
+    if ((dg && !g) || (dg_gamma && !g_gamma) || (dh0 && !initial_state)) return SGLA_ERR_INVALID_ARGUMENT;
+    const BwdLayout L = bwd_layout(varlen, N, T, H, K, V, chunk_size, dtype);
+    if (!L.valid) return L.why;
+    const int64_t tokens = varlen ? T : N * T;
+    if (tokens > 0 && (!q || !k || !v || !dout || !dq || !dk || !dv)) return SGLA_ERR_INVALID_ARGUMENT;
+    for (const void *p : {q, k, v, dout, (const void *)dq, (const void *)dk, (const void *)dv,
+                          (const void *)initial_state, (const void *)dht, (const void *)dh0})
+        if (!aligned(p, 16)) return SGLA_ERR_INVALID_ARGUMENT;
+    for (const void *p : {(const void *)g, (const void *)g_gamma, (const void *)dg, (const void *)dg_gamma})
+        if (!aligned(p, 4)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!aligned(cu_seqlens, 8)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!workspace || workspace_bytes < L.bytes) return SGLA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!(scale > 0.f) || isnan(scale) || isinf(scale)) scale = 1.0f / sqrtf((float)K);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dg_gamma) SGLA_CUDA(cudaMemsetAsync(dg_gamma, 0, sizeof(float) * H, st), "dg_gamma reset");
+    if (N == 0) return SGLA_OK;
+    char *ws = static_cast<char *>(workspace);
+    const bool gate = g || g_gamma, want_dg = dg || dg_gamma;
+    BwdRowArgs r{};
+    r.q = q; r.k = k; r.v = v; r.dout = dout; r.g = g; r.g_gamma = g_gamma;
+    r.qr = ws + L.off_qr; r.kr = ws + L.off_kr; r.vr = ws + L.off_vr; r.dor = ws + L.off_dor;
+    r.gr = gate ? reinterpret_cast<float *>(ws + L.off_gr) : nullptr;
+    r.dkr = ws + L.off_dkr; r.dvr = ws + L.off_dvr; r.dq = dq; r.dk = dk; r.dv = dv;
+    r.x = want_dg ? reinterpret_cast<float *>(ws + L.off_x) : nullptr;
+    r.dhT = dht;
+    r.xf = dh0 ? reinterpret_cast<float *>(ws + L.off_xf) : nullptr;
+    r.scale = scale; r.dg = dg; r.dg_gamma = dg_gamma; r.dh0 = dh0; r.cu = cu_seqlens;
+    r.N = (int)N; r.T_dense = varlen ? 0 : T; r.T_total = tokens; r.H = (int)H; r.K = (int)K; r.V = (int)V;
+    r.bf16 = dtype == SGLA_BF16;
+    float *s0 = dht ? reinterpret_cast<float *>(ws + L.off_s0) : nullptr;
+    float *s0T = dht ? reinterpret_cast<float *>(ws + L.off_s0T) : nullptr;
+    float *h0T = initial_state ? reinterpret_cast<float *>(ws + L.off_h0T) : nullptr;
+    void *dkr = ws + L.off_dkr, *dvr = ws + L.off_dvr;
+    float *xf = dh0 ? reinterpret_cast<float *>(ws + L.off_xf) : nullptr;
+    float *hTT = (dht && want_dg) ? reinterpret_cast<float *>(ws + L.off_hT) : nullptr;
+    r.s0T = hTT ? s0T : nullptr;
+    r.hT = hTT;
+    SGLA_LAUNCH("bwd_reverse_inputs", launch_bwd_reverse_inputs(r, st));
+    SGLA_LAUNCH("bwd_state_prep", launch_bwd_state_prep(dht, initial_state, 1.0f / scale, s0, s0T, h0T, N * H,
+                                                        (int)K, (int)V, st));
+    sgla_status rs;
+    // call A: dv on the reversed sequence, state [K,V] = dS / scale
+    rs = run_forward(varlen, r.kr, r.qr, r.dor, r.gr, nullptr, scale, cu_seqlens, N, T, s0, dvr, xf, H, K, V,
+                     chunk_size, dtype, workspace, L.inner, stream, false);
+    if (rs != SGLA_OK) return rs;
+    // call B: dk on the reversed sequence, state [V,K] = (dS / scale)^T
+    rs = run_forward(varlen, r.vr, r.dor, r.qr, r.gr, nullptr, scale, cu_seqlens, N, T, s0T, dkr, nullptr, H, V,
+                     K, chunk_size, dtype, workspace, L.inner, stream, false);
+    if (rs != SGLA_OK) return rs;
+    // call C: dq in token order, state [V,K] = S^T
+    rs = run_forward(varlen, dout, v, k, g, g_gamma, scale, cu_seqlens, N, T, h0T, dq, hTT, H, V, K, chunk_size,
+                     dtype, workspace, L.inner, stream, false);
+    if (rs != SGLA_OK) return rs;
+    SGLA_LAUNCH("bwd_unreverse", launch_bwd_unreverse(r, st));
+    if (want_dg || dh0) SGLA_LAUNCH("bwd_gate_scan", launch_bwd_gate_scan(r, st));
+    return SGLA_OK;
 }
 
 size_t simple_gla_fused_recurrent_bwd_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H,

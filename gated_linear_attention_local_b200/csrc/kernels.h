@@ -78,6 +78,32 @@ struct RecBwdArgs {
     int H, K, V;
     bool bf16;
 };
+// Row movers and the gate-gradient scan of the chunked backward (chunk_bwd.cu).
+struct BwdRowArgs {
+    const void *q, *k, *v, *dout;  // token order, [tokens,H,K] / [tokens,H,V]
+    const float *g, *g_gamma;
+    void *qr, *kr, *vr, *dor;      // time-reversed copies per sequence
+    float *gr;                     // [tokens,H] gates shifted by one token, reversed (or NULL)
+    const void *dkr, *dvr;         // reversed dk, dv from the forward calls
+    const void *dq;                // dq in token order
+    void *dk, *dv;                 // outputs in token order
+    float *x;                      // [tokens,H] q.dq - k.dk (or NULL)
+    const float *dhT, *xf;         // [N,H,K,V]: output-state gradient, final state of call A
+    const float *s0T, *hT;         // [N,H,V,K]: dhT^T / scale, final state of call C (S_T^T)
+    float scale;
+    float *dg, *dg_gamma, *dh0;
+    const int64_t *cu;
+    int N;
+    int64_t T_dense, T_total;
+    int H, K, V;
+    bool bf16;
+};
+cudaError_t launch_bwd_reverse_inputs(const BwdRowArgs &a, cudaStream_t st);
+cudaError_t launch_bwd_unreverse(const BwdRowArgs &a, cudaStream_t st);
+cudaError_t launch_bwd_gate_scan(const BwdRowArgs &a, cudaStream_t st);
+cudaError_t launch_bwd_state_prep(const float *dhT, const float *h0, float inv_scale, float *s0, float *s0T,
+                                  float *h0T, int64_t mats, int K, int V, cudaStream_t st);
+
 // part 0: forward sweep (dq, <dhT, hT>); 1: reverse sweep (dv, dk, dh0); 2: finalize (casts, dg)
 cudaError_t launch_rec_bwd(const RecBwdArgs &a, int part, cudaStream_t st);
 

@@ -30,6 +30,8 @@ test matrix with gate normalisers 0.1/1/10, scales 0.1/1 and the packed lengths
                 (B=8, T=512, H=16, K=V=128, bf16, g, initial state, output gradient do ~
                 N(0,1) and final-state gradient dht ~ 0.1 N(0,1)) --
                 simple_gla_fused_recurrent_bwd
+  chunk_bwd     the same gradients through the chunked tensor-core path at the same
+                size -- simple_gla_chunk_bwd
   recurrent_prefill  the inference routing case of section 4 (at most 64 tokens go to
                 the fused recurrence): 256 sequences x 64 tokens, H=32 K=V=128, bf16,
                 g, initial state 0.1*N(0,1), final state -- simple_gla_fused_recurrent
@@ -61,6 +63,8 @@ WORKLOADS = {
                           gate="gk", h0=True, final_state=True, scale=None, chunk_size=64),
     "recurrent_bwd": dict(kind="dense", entry="recurrent_bwd", B=8, T=512, H=16, K=128, V=128,
                           dtype=torch.bfloat16, gate="g", h0=True, final_state=False, scale=None, chunk_size=64),
+    "chunk_bwd": dict(kind="dense", entry="chunk_bwd", B=8, T=512, H=16, K=128, V=128, dtype=torch.bfloat16,
+                      gate="g", h0=True, final_state=False, scale=None, chunk_size=64),
     "recurrent_prefill": dict(kind="dense", entry="recurrent", B=256, T=64, H=32, K=128, V=128,
                               dtype=torch.bfloat16, gate="g", h0=True, final_state=True, scale=None,
                               chunk_size=64),
@@ -150,7 +154,7 @@ def make_workload(name: str, seed: int = 0):
     N = (len(cu) - 1) if cu is not None else B
     h0 = torch.randn(N, H, K, V, generator=gen) * 0.1 if w["h0"] else None
     do = dht = None
-    if w.get("entry") == "recurrent_bwd":
+    if w.get("entry") in ("recurrent_bwd", "chunk_bwd"):
         do, dht = random_cotangents(v.shape, N, H, K, V, dtype=dt, seed=seed + 1)
     return dict(name=name, kind=w["kind"], entry=w.get("entry", "chunk"), q=q, k=k, v=v, g=g, g_gamma=g_gamma,
                 h0=h0, cu_seqlens=cu, scale=w["scale"], output_final_state=w["final_state"],

@@ -223,6 +223,34 @@ SGLA_API sgla_status simple_gla_fused_recurrent_bwd(const void *q, const void *k
                                                     void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Gradients of the chunked forward (simple_gla_chunk with state_v_first = 0) on the
+ * tensor cores: the article's section 3 backward -- a reverse state pass and
+ * output-style passes with fp32 states, and dg by a reverse cumulative sum.  The
+ * gradient recurrence dS_t = exp(g_{t+1}) dS_{t+1} + scale q_t do_t^T is the forward
+ * recurrence run on the time-reversed sequence, so dv, dk and dq each come from one
+ * call of the chunked forward with other operands (dv: query k, key q, value do;
+ * dk: query v, key do, value q, both on the reversed tokens with the gates shifted by
+ * one; dq: query do, key v, value k in token order), plus three row kernels.
+ *
+ * Outputs, loss, inputs and the packed / dense conventions are those of
+ * simple_gla_fused_recurrent_bwd; chunk_size as simple_gla_chunk.  Sizes as the
+ * chunked forward with K and V exchanged as well (both multiples of 8, at most 512);
+ * q, k, v, dout, dq, dk, dv, initial_state, dht and dh0 16-byte aligned.  workspace:
+ * at least simple_gla_chunk_bwd_workspace_size() bytes, 256-byte aligned, contents
+ * on entry irrelevant; sgla_workspace_status() on it reports a bad cu_seqlens as for
+ * the forward (no gradient of a bad sequence is written).
+ */
+SGLA_API size_t simple_gla_chunk_bwd_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H,
+                                                    int64_t K, int64_t V, int chunk_size, sgla_dtype dtype);
+SGLA_API sgla_status simple_gla_chunk_bwd(const void *q, const void *k, const void *v, const float *g,
+                                          const float *g_gamma, float scale, const float *initial_state,
+                                          const void *dout, const float *dht, void *dq, void *dk, void *dv,
+                                          float *dg, float *dg_gamma, float *dh0, const int64_t *cu_seqlens,
+                                          int64_t N, int64_t T, int64_t H, int64_t K, int64_t V, int chunk_size,
+                                          sgla_dtype dtype, void *workspace, size_t workspace_bytes,
+                                          void *stream);
+
+/*
  * The chunked forward with every option of chunk_simple_gla (article section 2) in
  * one call: dense (cu_seqlens == NULL: N sequences of T tokens, q [N,T,H,K]) or
  * packed (cu_seqlens != NULL: N sequences in T tokens, exactly as

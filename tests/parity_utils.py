@@ -44,3 +44,32 @@ def oracle_fwd(inp, scale=None, final=True, cu=None):
     return oracle.simple_gla_fwd(inp["q"], inp["k"], inp["v"], g=inp.get("g"), g_gamma=inp.get("g_gamma"),
                                  scale=scale, initial_state=inp.get("h0"), output_final_state=final,
                                  cu_seqlens=cu)
+
+
+def dg_scale(inp, ref):
+    """Magnitude of the terms the gate gradient is assembled from: dg_t sums
+    q_i . dq_i - k_i . dk_i over the tokens from t on (a reverse cumulative sum), so
+    its rounding error is relative to those terms, not to dg itself -- which is
+    exactly 0 when every gate is 0."""
+    q = np.asarray(inp["q"].double().numpy())
+    k = np.asarray(inp["k"].double().numpy())
+    terms = np.abs((q * ref["dq"]).sum(-1)) + np.abs((k * ref["dk"]).sum(-1))
+    return float(terms.max()) if terms.size else 0.0
+
+
+def compare_grads(gpu, ref, tol, inp):
+    """Every gradient of the backward within tol: dq, dk, dv, dh0 normalised by their
+    largest oracle magnitude; dg and dg_gamma by the larger of that and dg_scale
+    (times the token count for dg_gamma, a sum over tokens)."""
+    for name in ("dq", "dk", "dv", "dg", "dg_gamma", "dh0"):
+        if ref[name] is None:
+            assert gpu[name] is None, name
+            continue
+        x, y = host(gpu[name]), ref[name]
+        if name in ("dg", "dg_gamma") and y.size:
+            floor = dg_scale(inp, ref) * (inp["q"].shape[0] * inp["q"].shape[1] if name == "dg_gamma" else 1)
+            assert np.all(np.isfinite(x)), name
+            err = float(np.max(np.abs(x - y)))
+            assert err <= tol * max(float(np.max(np.abs(y))), floor), f"{name}: max error {err:.3e}"
+        else:
+            assert_close(x, y, tol, name)

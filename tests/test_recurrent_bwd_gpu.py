@@ -15,7 +15,7 @@ import torch
 import gated_linear_attention_local_b200 as sg
 import oracle
 from gated_linear_attention_local_b200.workloads import random_cotangents, random_inputs
-from parity_utils import TOL, assert_close, host, to_dev
+from parity_utils import TOL, assert_close, compare_grads, host, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -36,32 +36,6 @@ def _run(inp, do, dht, scale=None, cu=None):
     ref = oracle.simple_gla_bwd(inp["q"], inp["k"], inp["v"], do, g=inp["g"], g_gamma=inp["g_gamma"], scale=scale,
                                 initial_state=inp["h0"], dht=dht, cu_seqlens=cu)
     return gpu, ref
-
-
-def _dg_scale(inp, ref):
-    """Magnitude of the terms the gate gradient is assembled from: dg_t sums
-    q_i . dq_i - k_i . dk_i over the tokens from t on (the reverse cumulative sum of
-    the article's section 3), so its rounding error is relative to those terms, not to
-    dg itself -- which is exactly 0 when every gate is 0."""
-    q = np.asarray(inp["q"].double().numpy())
-    k = np.asarray(inp["k"].double().numpy())
-    terms = np.abs((q * ref["dq"]).sum(-1)) + np.abs((k * ref["dk"]).sum(-1))
-    return float(terms.max()) if terms.size else 0.0
-
-
-def _compare(gpu, ref, tol, inp):
-    for name in ("dq", "dk", "dv", "dg", "dg_gamma", "dh0"):
-        if ref[name] is None:
-            assert gpu[name] is None, name
-            continue
-        x, y = host(gpu[name]), ref[name]
-        if name in ("dg", "dg_gamma") and y.size:
-            floor = _dg_scale(inp, ref) * (inp["q"].shape[0] * inp["q"].shape[1] if name == "dg_gamma" else 1)
-            assert np.all(np.isfinite(x)), name
-            err = float(np.max(np.abs(x - y)))
-            assert err <= tol * max(float(np.max(np.abs(y))), floor), f"{name}: max error {err:.3e}"
-        else:
-            assert_close(x, y, tol, name)
 
 
 DENSE = [
@@ -86,7 +60,7 @@ def test_fused_recurrent_bwd_dense(case):
     inp = random_inputs(N, T, H, K, V, dtype=dt, gate=gate, normalizer=norm, h0=h0, seed=23)
     do, dh = random_cotangents(inp["v"].shape, N, H, K, V, dtype=dt, dht=dht, seed=24)
     gpu, ref = _run(inp, do, dh, scale=scale)
-    _compare(gpu, ref, TOL[dt], inp)
+    compare_grads(gpu, ref, TOL[dt], inp)
 
 
 @pytest.mark.parametrize("gate", ["g", "gamma"])
@@ -99,7 +73,7 @@ def test_fused_recurrent_bwd_varlen(dt, gate):
     inp = random_inputs(1, T, H, K, V, dtype=dt, gate=gate, h0=True, seed=31, cu_seqlens=cu)
     do, dh = random_cotangents(inp["v"].shape, len(cu) - 1, H, K, V, dtype=dt, seed=32)
     gpu, ref = _run(inp, do, dh, cu=cu)
-    _compare(gpu, ref, TOL[dt], inp)
+    compare_grads(gpu, ref, TOL[dt], inp)
 
 
 def test_fused_recurrent_bwd_bad_cu_seqlens():
