@@ -189,7 +189,7 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
                         const float *g_gamma, float scale, const int64_t *cu, int64_t N, int64_t T,
                         const float *h0, void *o, float *hT, int64_t H, int64_t K, int64_t V,
                         int chunk_size, sgla_dtype dtype, void *workspace, size_t workspace_bytes,
-                        void *stream, bool state_v_first = false) {
+                        void *stream, bool state_v_first = false, bool out_f32 = false) {
     if (g && g_gamma) return SGLA_ERR_INVALID_ARGUMENT;
     const int64_t tokens = varlen ? T : N * T;
     if (tokens > 0 && (!q || !k || !v || !o)) return SGLA_ERR_INVALID_ARGUMENT;
@@ -216,6 +216,7 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
     a.H = (int)H; a.K = (int)K; a.V = (int)V;
     a.gate_mode = g ? kGatePerToken : (g_gamma ? kGatePerHead : kGateNone);
     a.bf16 = dtype == SGLA_BF16;
+    a.o_f32 = out_f32;
     a.gcum = per_token ? reinterpret_cast<float *>(ws + p.off_gcum) : nullptr;
     a.gpos = per_token ? reinterpret_cast<int *>(ws + p.off_gpos) : nullptr;
     a.seg_dec = p.multi_seg ? reinterpret_cast<float *>(ws + p.off_seg_dec) : nullptr;
@@ -295,13 +296,14 @@ int norm_decode_width(int64_t V) { return (int)((V + 1 + 3) / 4 * 4); }
 
 // Chunked backward: three forward calls share the inner workspace (at offset 0, so
 // that its status word is the one sgla_workspace_status reads), followed by the
-// time-reversed operands, the reversed dk / dv, q.dq - k.dk per row and five states
+// time-reversed operands, dk (fp32, reversed), dq (fp32), dv (reversed), q.dq - k.dk
+// per row and five states
 // (dhT / scale in both layouts, h0 transposed, and the final states of calls A and C).
 struct BwdLayout {
     bool valid = false;
     sgla_status why = SGLA_ERR_INVALID_ARGUMENT;
-    size_t inner = 0, off_qr = 0, off_kr = 0, off_vr = 0, off_dor = 0, off_gr = 0, off_dkr = 0, off_dvr = 0,
-           off_x = 0, off_s0 = 0, off_s0T = 0, off_h0T = 0, off_xf = 0, off_hT = 0, bytes = 0;
+    size_t inner = 0, off_qr = 0, off_kr = 0, off_vr = 0, off_dor = 0, off_gr = 0, off_dkf = 0, off_dqf = 0,
+           off_dvr = 0, off_x = 0, off_s0 = 0, off_s0T = 0, off_h0T = 0, off_xf = 0, off_hT = 0, bytes = 0;
 };
 
 BwdLayout bwd_layout(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V, int C, sgla_dtype dtype) {
@@ -319,7 +321,8 @@ BwdLayout bwd_layout(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, in
     take(L.off_vr, es * rows * V);
     take(L.off_dor, es * rows * V);
     take(L.off_gr, sizeof(float) * rows);
-    take(L.off_dkr, es * rows * K);
+    take(L.off_dkf, sizeof(float) * rows * K);
+    take(L.off_dqf, sizeof(float) * rows * K);
     take(L.off_dvr, es * rows * V);
     take(L.off_x, sizeof(float) * rows);
     take(L.off_s0, st);
@@ -521,7 +524,8 @@ sgla_status simple_gla_chunk_bwd(const void *q, const void *k, const void *v, co
     r.q = q; r.k = k; r.v = v; r.dout = dout; r.g = g; r.g_gamma = g_gamma;
     r.qr = ws + L.off_qr; r.kr = ws + L.off_kr; r.vr = ws + L.off_vr; r.dor = ws + L.off_dor;
     r.gr = gate ? reinterpret_cast<float *>(ws + L.off_gr) : nullptr;
-    r.dkr = ws + L.off_dkr; r.dvr = ws + L.off_dvr; r.dq = dq; r.dk = dk; r.dv = dv;
+    r.dkf = reinterpret_cast<float *>(ws + L.off_dkf); r.dqf = reinterpret_cast<float *>(ws + L.off_dqf);
+    r.dvr = ws + L.off_dvr; r.dq = dq; r.dk = dk; r.dv = dv;
     r.x = want_dg ? reinterpret_cast<float *>(ws + L.off_x) : nullptr;
     r.dhT = dht;
     r.xf = dh0 ? reinterpret_cast<float *>(ws + L.off_xf) : nullptr;
@@ -531,7 +535,7 @@ sgla_status simple_gla_chunk_bwd(const void *q, const void *k, const void *v, co
     float *s0 = dht ? reinterpret_cast<float *>(ws + L.off_s0) : nullptr;
     float *s0T = dht ? reinterpret_cast<float *>(ws + L.off_s0T) : nullptr;
     float *h0T = initial_state ? reinterpret_cast<float *>(ws + L.off_h0T) : nullptr;
-    void *dkr = ws + L.off_dkr, *dvr = ws + L.off_dvr;
+    void *dkf = ws + L.off_dkf, *dqf = ws + L.off_dqf, *dvr = ws + L.off_dvr;
     float *xf = dh0 ? reinterpret_cast<float *>(ws + L.off_xf) : nullptr;
     float *hTT = (dht && want_dg) ? reinterpret_cast<float *>(ws + L.off_hT) : nullptr;
     r.s0T = hTT ? s0T : nullptr;
@@ -544,13 +548,13 @@ sgla_status simple_gla_chunk_bwd(const void *q, const void *k, const void *v, co
     rs = run_forward(varlen, r.kr, r.qr, r.dor, r.gr, nullptr, scale, cu_seqlens, N, T, s0, dvr, xf, H, K, V,
                      chunk_size, dtype, workspace, L.inner, stream, false);
     if (rs != SGLA_OK) return rs;
-    // call B: dk on the reversed sequence, state [V,K] = (dS / scale)^T
-    rs = run_forward(varlen, r.vr, r.dor, r.qr, r.gr, nullptr, scale, cu_seqlens, N, T, s0T, dkr, nullptr, H, V,
-                     K, chunk_size, dtype, workspace, L.inner, stream, false);
+    // call B: dk (fp32) on the reversed sequence, state [V,K] = (dS / scale)^T
+    rs = run_forward(varlen, r.vr, r.dor, r.qr, r.gr, nullptr, scale, cu_seqlens, N, T, s0T, dkf, nullptr, H, V,
+                     K, chunk_size, dtype, workspace, L.inner, stream, false, true);
     if (rs != SGLA_OK) return rs;
-    // call C: dq in token order, state [V,K] = S^T
-    rs = run_forward(varlen, dout, v, k, g, g_gamma, scale, cu_seqlens, N, T, h0T, dq, hTT, H, V, K, chunk_size,
-                     dtype, workspace, L.inner, stream, false);
+    // call C: dq (fp32) in token order, state [V,K] = S^T
+    rs = run_forward(varlen, dout, v, k, g, g_gamma, scale, cu_seqlens, N, T, h0T, dqf, hTT, H, V, K, chunk_size,
+                     dtype, workspace, L.inner, stream, false, true);
     if (rs != SGLA_OK) return rs;
     SGLA_LAUNCH("bwd_unreverse", launch_bwd_unreverse(r, st));
     if (want_dg || dh0) SGLA_LAUNCH("bwd_gate_scan", launch_bwd_gate_scan(r, st));

@@ -72,27 +72,6 @@ __host__ __device__ __forceinline__ int group_lanes(int pieces) {
     return pieces <= 4 ? 4 : pieces <= 8 ? 8 : pieces <= 16 ? 16 : 32;
 }
 
-// sum over the 16-byte pieces a and b of a[i] * b[i] as T
-template <typename T>
-__device__ __forceinline__ float dot16(const uint4 &a, const uint4 &b);
-template <>
-__device__ __forceinline__ float dot16<float>(const uint4 &a, const uint4 &b) {
-    return __uint_as_float(a.x) * __uint_as_float(b.x) + __uint_as_float(a.y) * __uint_as_float(b.y) +
-           __uint_as_float(a.z) * __uint_as_float(b.z) + __uint_as_float(a.w) * __uint_as_float(b.w);
-}
-template <>
-__device__ __forceinline__ float dot16<__nv_bfloat16>(const uint4 &a, const uint4 &b) {
-    const __nv_bfloat162 *x = reinterpret_cast<const __nv_bfloat162 *>(&a);
-    const __nv_bfloat162 *y = reinterpret_cast<const __nv_bfloat162 *>(&b);
-    float acc = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 u = __bfloat1622float2(x[i]), w = __bfloat1622float2(y[i]);
-        acc = fmaf(u.x, w.x, fmaf(u.y, w.y, acc));
-    }
-    return acc;
-}
-
 // Group of G lanes per (token, head) row: q, k, v, do to their mirrored position in
 // the sequence, and the shifted gate g'[mirror] = g[t+1] (0 at the last token).
 template <typename T>
@@ -128,22 +107,60 @@ bwd_reverse_inputs_kernel(const T *__restrict__ q, const T *__restrict__ k, cons
     }
 }
 
-// Group of G lanes per (token, head) row: dk, dv back to token order, and
-// x = q.dq - k.dk (from the same loads).
+// A piece of 16 bytes of T as fp32 values, and back
+template <typename T>
+struct Piece;
+template <>
+struct Piece<float> {
+    static constexpr int n = 4;
+    __device__ static void unpack(const uint4 &p, float *f) {
+        f[0] = __uint_as_float(p.x); f[1] = __uint_as_float(p.y); f[2] = __uint_as_float(p.z); f[3] = __uint_as_float(p.w);
+    }
+    __device__ static uint4 pack(const float *f) {
+        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3]));
+    }
+};
+template <>
+struct Piece<__nv_bfloat16> {
+    static constexpr int n = 8;
+    __device__ static void unpack(const uint4 &p, float *f) {
+        const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&p);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 u = __bfloat1622float2(b[i]);
+            f[2 * i] = u.x;
+            f[2 * i + 1] = u.y;
+        }
+    }
+    __device__ static uint4 pack(const float *f) {
+        uint4 p;
+        __nv_bfloat162 *b = reinterpret_cast<__nv_bfloat162 *>(&p);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) b[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+        return p;
+    }
+};
+
+// Group of G lanes per (token, head) row: dk (fp32, reversed) and dq (fp32) to the
+// operand dtype in token order, dv back to token order, and x = q.dq - k.dk from the
+// fp32 values.
 template <typename T>
 __global__ void __launch_bounds__(256)
-bwd_unreverse_kernel(const T *__restrict__ dkr, const T *__restrict__ dvr, const T *__restrict__ q,
-                     const T *__restrict__ k, const T *__restrict__ dq, T *__restrict__ dk, T *__restrict__ dv,
-                     float *__restrict__ x, const int64_t *__restrict__ cu, int N, int64_t T_dense, int64_t T_total,
-                     int H, int K, int V) {
-    const int pk = K * (int)sizeof(T) / 16, pv = V * (int)sizeof(T) / 16;
+bwd_unreverse_kernel(const float *__restrict__ dkf, const T *__restrict__ dvr, const T *__restrict__ q,
+                     const T *__restrict__ k, const float *__restrict__ dqf, T *__restrict__ dq, T *__restrict__ dk,
+                     T *__restrict__ dv, float *__restrict__ x, const int64_t *__restrict__ cu, int N,
+                     int64_t T_dense, int64_t T_total, int H, int K, int V) {
+    using P = Piece<T>;
+    const int pk = K / P::n, pv = V / P::n;  // 16-byte pieces of T per row
     const int G = group_lanes(max(pk, pv));
     const int lane = threadIdx.x & 31, j = lane & (G - 1);
     const int64_t groups = (int64_t)gridDim.x * (blockDim.x / G);
-    const uint4 *dkr4 = reinterpret_cast<const uint4 *>(dkr), *dvr4 = reinterpret_cast<const uint4 *>(dvr);
+    const uint4 *dvr4 = reinterpret_cast<const uint4 *>(dvr);
     const uint4 *q4 = reinterpret_cast<const uint4 *>(q), *k4 = reinterpret_cast<const uint4 *>(k);
-    const uint4 *dq4 = reinterpret_cast<const uint4 *>(dq);
-    uint4 *dk4 = reinterpret_cast<uint4 *>(dk), *dv4 = reinterpret_cast<uint4 *>(dv);
+    const float4 *dkf4 = reinterpret_cast<const float4 *>(dkf), *dqf4 = reinterpret_cast<const float4 *>(dqf);
+    uint4 *dq4 = reinterpret_cast<uint4 *>(dq), *dk4 = reinterpret_cast<uint4 *>(dk);
+    uint4 *dv4 = reinterpret_cast<uint4 *>(dv);
+    constexpr int F4 = P::n / 4;  // float4s per piece
     // every lane of a group runs the same rows, so the group reductions below see
     // only lanes of their own row; groups never straddle warps
     for (int64_t row0 = blockIdx.x * (int64_t)(blockDim.x / G); row0 < T_total * H; row0 += groups) {
@@ -160,12 +177,24 @@ bwd_unreverse_kernel(const T *__restrict__ dkr, const T *__restrict__ dvr, const
         float acc = 0.f;
         if (live) {
             for (int i = j; i < max(pk, pv); i += G) {
-                uint4 a, b, c, d, e;
-                if (i < pk) { a = dkr4[mrow * pk + i]; if (x) { b = q4[row * pk + i]; c = dq4[row * pk + i]; d = k4[row * pk + i]; } }
+                uint4 e;
                 if (i < pv) e = dvr4[mrow * pv + i];
                 if (i < pk) {
-                    dk4[row * pk + i] = a;
-                    if (x) acc += dot16<T>(b, c) - dot16<T>(d, a);
+                    float fk[P::n], fq[P::n], xq[P::n], xk[P::n];
+#pragma unroll
+                    for (int u = 0; u < F4; ++u) {
+                        const float4 a4 = dkf4[(mrow * pk + i) * F4 + u], b4 = dqf4[(row * pk + i) * F4 + u];
+                        fk[4 * u] = a4.x; fk[4 * u + 1] = a4.y; fk[4 * u + 2] = a4.z; fk[4 * u + 3] = a4.w;
+                        fq[4 * u] = b4.x; fq[4 * u + 1] = b4.y; fq[4 * u + 2] = b4.z; fq[4 * u + 3] = b4.w;
+                    }
+                    if (x) {
+                        P::unpack(q4[row * pk + i], xq);
+                        P::unpack(k4[row * pk + i], xk);
+#pragma unroll
+                        for (int u = 0; u < P::n; ++u) acc = fmaf(xq[u], fq[u], fmaf(-xk[u], fk[u], acc));
+                    }
+                    dk4[row * pk + i] = P::pack(fk);
+                    dq4[row * pk + i] = P::pack(fq);
                 }
                 if (i < pv) dv4[row * pv + i] = e;
             }
@@ -332,13 +361,14 @@ cudaError_t launch_bwd_unreverse(const BwdRowArgs &a, cudaStream_t st) {
     const unsigned grid = rows_grid(a.T_total * a.H, a.K, a.V, a.bf16 ? 2 : 4);
     if (a.bf16) {
         using T = __nv_bfloat16;
-        bwd_unreverse_kernel<T><<<grid, 256, 0, st>>>((const T *)a.dkr, (const T *)a.dvr, (const T *)a.q,
-                                                     (const T *)a.k, (const T *)a.dq, (T *)a.dk, (T *)a.dv, a.x,
-                                                     a.cu, a.N, a.T_dense, a.T_total, a.H, a.K, a.V);
+        bwd_unreverse_kernel<T><<<grid, 256, 0, st>>>(a.dkf, (const T *)a.dvr, (const T *)a.q, (const T *)a.k,
+                                                     a.dqf, (T *)a.dq, (T *)a.dk, (T *)a.dv, a.x, a.cu, a.N,
+                                                     a.T_dense, a.T_total, a.H, a.K, a.V);
     } else {
-        bwd_unreverse_kernel<float><<<grid, 256, 0, st>>>(
-            (const float *)a.dkr, (const float *)a.dvr, (const float *)a.q, (const float *)a.k, (const float *)a.dq,
-            (float *)a.dk, (float *)a.dv, a.x, a.cu, a.N, a.T_dense, a.T_total, a.H, a.K, a.V);
+        bwd_unreverse_kernel<float><<<grid, 256, 0, st>>>(a.dkf, (const float *)a.dvr, (const float *)a.q,
+                                                         (const float *)a.k, a.dqf, (float *)a.dq, (float *)a.dk,
+                                                         (float *)a.dv, a.x, a.cu, a.N, a.T_dense, a.T_total, a.H,
+                                                         a.K, a.V);
     }
     return cudaGetLastError();
 }

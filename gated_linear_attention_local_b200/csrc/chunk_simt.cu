@@ -235,7 +235,9 @@ chunk_output_simt_kernel(FwdArgs a) {
             if (i < len && j < vw) {
                 float acc = exp2f(gs[i]) * accO[r];
                 for (int x = 0; x <= i; ++x) acc = fmaf(Ps[i * (C + 1) + x], vs[x * (kBV + 1) + j], acc);
-                op[((ta + i) * H + h) * V + v0 + j] = from_f32<T>(a.scale * acc);
+                const int64_t oe = ((ta + i) * H + h) * V + v0 + j;
+                if (a.o_f32) static_cast<float *>(a.o)[oe] = a.scale * acc;
+                else op[oe] = from_f32<T>(a.scale * acc);
             }
         }
     }

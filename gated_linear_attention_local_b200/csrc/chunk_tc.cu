@@ -583,6 +583,18 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&b_ofree[t & 1]);  // O1 and O2 of this step are in registers
+                if (a.o_f32) {  // fp32 output rows (16-byte aligned: V is a multiple of 64 here)
+                    if (i < sp.len && !*abort_flag) {
+                        float4 *d = reinterpret_cast<float4 *>(static_cast<float *>(a.o) +
+                                                               ((sp.ta + i) * H + h) * (int64_t)V + v0 + OW * half);
+#pragma unroll
+                        for (int q = 0; q < OW / 4; ++q)
+                            d[q] = make_float4(fmaf(ei, ox[4 * q], a.scale * oy[4 * q]),
+                                               fmaf(ei, ox[4 * q + 1], a.scale * oy[4 * q + 1]),
+                                               fmaf(ei, ox[4 * q + 2], a.scale * oy[4 * q + 2]),
+                                               fmaf(ei, ox[4 * q + 3], a.scale * oy[4 * q + 3]));
+                    }
+                } else {
                 uint32_t w[OW / 2];
 #pragma unroll
                 for (int e = 0; e < OW / 2; ++e)
@@ -597,6 +609,7 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
 #pragma unroll
                         for (int q = 0; q < OW / 8; ++q) d[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
                     }
+                }
                 }
             }
             TR_ACC(a_out, xo);

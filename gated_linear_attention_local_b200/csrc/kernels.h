@@ -18,6 +18,7 @@ struct FwdArgs {
     int H, K, V;
     int gate_mode;
     bool bf16;
+    bool o_f32;      // o is written as fp32 whatever the operand dtype (the backward's dq, dk)
     // workspace carve-up
     float *gcum;     // [tokens, H] chunk-local cumsum of g in log2 units (per-token gates)
     int *gpos;       // [chunks, H] 1 if the chunk holds a positive log gate (per-token gates)
@@ -84,9 +85,10 @@ struct BwdRowArgs {
     const float *g, *g_gamma;
     void *qr, *kr, *vr, *dor;      // time-reversed copies per sequence
     float *gr;                     // [tokens,H] gates shifted by one token, reversed (or NULL)
-    const void *dkr, *dvr;         // reversed dk, dv from the forward calls
-    const void *dq;                // dq in token order
-    void *dk, *dv;                 // outputs in token order
+    const float *dkf;              // dk from the forward call, fp32, reversed
+    const void *dvr;               // dv from the forward call, reversed
+    const float *dqf;              // dq from the forward call, fp32, token order
+    void *dq, *dk, *dv;            // outputs in token order
     float *x;                      // [tokens,H] q.dq - k.dk (or NULL)
     const float *dhT, *xf;         // [N,H,K,V]: output-state gradient, final state of call A
     const float *s0T, *hT;         // [N,H,V,K]: dhT^T / scale, final state of call C (S_T^T)
