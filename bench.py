@@ -67,7 +67,7 @@ def algorithmic_counts(w):
     if w["output_final_state"]:
         b += states
     flops = H * (4 * tokens * K * V + tokens * (C + 1) * (K + V))
-    if w.get("entry") in ("recurrent", "gla"):  # token-serial: state update and read-out per token
+    if w.get("entry") in ("recurrent", "gla", "gla_chunk"):  # state update and read-out per token
         flops = H * tokens * 4 * K * V
     if w.get("entry") in ("recurrent_bwd", "chunk_bwd"):
         fwd = dict(bytes=b, flops=flops)  # one forward call with these operands (K == V)
@@ -132,7 +132,7 @@ def roofline(w, counts, kernel_ms, peaks, traffic=None, kernel=None):
     token-serial recurrence runs on the FP32 CUDA cores (two FMAs and a multiply per
     state element and token), so its bound is the ALU peak."""
     kc = counts.get("kernel", {}).get(kernel, counts)  # per-launch counts of that kernel
-    if w.get("entry") in ("recurrent", "gla", "recurrent_bwd"):
+    if w.get("entry") in ("recurrent", "gla", "gla_chunk", "recurrent_bwd"):
         ach = kc["flops"] / (kernel_ms * 1e-3) / 1e12
         return dict(bound="alu", achieved=round(ach, 3), peak=round(FP32_ALU_TFLOPS, 1), unit="TFLOP/s",
                     frac=round(ach / FP32_ALU_TFLOPS, 4), traffic=traffic,
@@ -242,6 +242,11 @@ def make_step(w, d, sg, ws):
                                      output_final_state=w["output_final_state"], chunk_size=w["chunk_size"],
                                      workspace=ws)
         return step, (lambda: None)
+    if w.get("entry") == "gla_chunk":
+        def step():
+            sg.gla_chunk(d["q"], d["k"], d["v"], d["g"], scale=w["scale"], initial_state=d["h0"],
+                         output_final_state=w["output_final_state"], workspace=ws)
+        return step, (lambda: None)
     if w.get("entry") == "gla":
         def step():
             sg.gla_fused_recurrent(d["q"], d["k"], d["v"], d["g"], scale=w["scale"], initial_state=d["h0"],
@@ -280,6 +285,9 @@ def workspace_for(w, sg, device):
     dt = w["q"].dtype
     if w.get("entry") == "recurrent_bwd":
         n = sg.lib().simple_gla_fused_recurrent_bwd_workspace_size(None, w["B"], w["T"], w["H"], w["K"])
+        return torch.empty(max(int(n), 256), dtype=torch.uint8, device=device)
+    if w.get("entry") == "gla_chunk":
+        n = sg.lib().gla_chunk_workspace_size(None, w["B"], w["T"], w["H"], w["K"], w["V"], sg._DTYPES[dt])
         return torch.empty(max(int(n), 256), dtype=torch.uint8, device=device)
     if w.get("entry") == "chunk_bwd":
         n = sg.lib().simple_gla_chunk_bwd_workspace_size(None, w["B"], w["T"], w["H"], w["K"], w["V"],
@@ -393,6 +401,9 @@ def e2e_measure(w, sg, device, steps, warmup):
             o, ht = sg.simple_gla_normalized(d["q"], d["k"], d["v"], g=d.get("g"), g_gamma=g_gamma,
                                              initial_state=d.get("h0"), output_final_state=w["output_final_state"],
                                              chunk_size=w["chunk_size"], workspace=ws)
+        elif w.get("entry") == "gla_chunk":
+            o, ht = sg.gla_chunk(d["q"], d["k"], d["v"], d["g"], scale=w["scale"], initial_state=d.get("h0"),
+                                 output_final_state=w["output_final_state"], workspace=ws)
         elif w.get("entry") == "gla":
             o, ht = sg.gla_fused_recurrent(d["q"], d["k"], d["v"], d["g"], scale=w["scale"], initial_state=d.get("h0"),
                                            output_final_state=w["output_final_state"])
@@ -465,7 +476,7 @@ def oracle_sample(w, budget_s=12.0):
         if w.get("entry") in ("recurrent_bwd", "chunk_bwd"):
             oracle.simple_gla_bwd(d["q"], d["k"], d["v"], w["do"][:, :tn], g=d["g"], g_gamma=w["g_gamma"],
                                   scale=w["scale"], initial_state=w["h0"], dht=w["dht"])
-        elif w.get("entry") == "gla":
+        elif w.get("entry") in ("gla", "gla_chunk"):
             oracle.gla_fwd(d["q"], d["k"], d["v"], d["g"], scale=w["scale"], initial_state=w["h0"],
                            output_final_state=w["output_final_state"], threads=threads)
         elif w.get("entry") == "normalized":
@@ -551,6 +562,9 @@ def _config_of(w):
     if w.get("entry") == "normalized":
         return dict(entry="simple_gla_normalized", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
                     gate="g" if w["g"] is not None else "none", feature_map="|x|+0.1", scale=1.0)
+    if w.get("entry") == "gla_chunk":
+        return dict(entry="gla_chunk", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"], chunk=32, sub_chunk=16,
+                    gate="gk [B,T,H,K] = logsigmoid(N(0,1))/16", initial_state=True)
     if w.get("entry") == "gla":
         return dict(entry="gla_fused_recurrent", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
                     gate="gk [B,T,H,K] = logsigmoid(N(0,1))/16", initial_state=True)

@@ -42,7 +42,7 @@ from ._lib import (SGLA_BF16, SGLA_FP32, SGLA_OK, SglaError, lib, library_path, 
 __all__ = ["simple_gla_fwd", "simple_gla_fwd_noalloc", "simple_gla_fwd_varlen", "simple_gla_decode_step", "chunk_simple_gla",
            "simple_gla_fused_recurrent", "fused_recurrent_simple_gla", "simple_gla_chunk",
            "simple_gla_normalized", "simple_gla_normalized_decode_step", "normalized_decode_state_width",
-           "gla_fused_recurrent", "simple_gla_fused_recurrent_bwd", "simple_gla_chunk_bwd",
+           "gla_fused_recurrent", "simple_gla_fused_recurrent_bwd", "simple_gla_chunk_bwd", "gla_chunk",
            "fwd_workspace_size", "varlen_workspace_size", "workspace_status", "library_path",
            "SglaError"]
 
@@ -540,6 +540,45 @@ def gla_fused_recurrent(q, k, v, gk, scale=None, initial_state=None, output_fina
                                    1 if state_v_first else 0, _DTYPES[q.dtype], _ptr(device_status), _stream())
     raise_for_status(st, "gla_fused_recurrent")
     return (o.unsqueeze(0) if squeeze else o), ht
+
+
+def gla_chunk(q, k, v, gk, scale=None, initial_state=None, output_final_state=False, cu_seqlens=None,
+              workspace=None):
+    """GLA (gate vector over the key dimension) in the chunked form: gk fp32 log gates
+    shaped like q.  Dense q,k [B,T,H,K], v [B,T,H,V]; packed (cu_seqlens) [1,T,...] or
+    [T,...].  States [N,H,K,V] fp32.  Returns (o shaped like v, final_state|None)."""
+    _common_checks(q, k, v, None, None, initial_state)
+    _check_cuda("gk", gk, torch.float32)
+    if tuple(gk.shape) != tuple(q.shape):
+        raise ValueError(f"gk must be shaped like q {tuple(q.shape)}, got {tuple(gk.shape)}")
+    if cu_seqlens is not None:
+        _check_cuda("cu_seqlens", cu_seqlens, torch.int64, 1)
+        if q.dim() == 4 and q.shape[0] != 1:
+            raise ValueError("with cu_seqlens the batch dimension must be 1")
+        N = cu_seqlens.numel() - 1
+        if N < 1:
+            raise ValueError("cu_seqlens needs at least two entries")
+        T, H, K = q.shape[-3:]
+    else:
+        if q.dim() != 4:
+            raise ValueError("q must be [B,T,H,K]")
+        N, T, H, K = q.shape
+    V = v.shape[-1]
+    if k.shape != q.shape or v.shape[:-1] != q.shape[:-1]:
+        raise ValueError("k must match q, and v must match q except in the last dimension")
+    if initial_state is not None and tuple(initial_state.shape) != (N, H, K, V):
+        raise ValueError(f"initial_state must be {(N, H, K, V)}")
+    dt = _DTYPES[q.dtype]
+    nbytes = int(lib().gla_chunk_workspace_size(_ptr(cu_seqlens), N, T, H, K, V, dt))
+    if nbytes == 0:
+        raise SglaError(2, "gla_chunk: unsupported sizes (K <= 256, V <= 4096)")
+    ws = _workspace(nbytes, q.device, workspace)
+    o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    ht = torch.empty((N, H, K, V), dtype=torch.float32, device=q.device) if output_final_state else None
+    st = lib().gla_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(gk), ctypes.c_float(_scale(scale)), _ptr(initial_state),
+                         _ptr(o), _ptr(ht), _ptr(cu_seqlens), N, T, H, K, V, dt, _ptr(ws), ws.numel(), _stream())
+    raise_for_status(st, "gla_chunk")
+    return o, ht
 
 
 def fused_recurrent_simple_gla(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,

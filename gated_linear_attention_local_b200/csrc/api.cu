@@ -294,6 +294,47 @@ NormLayout norm_layout(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, 
 
 int norm_decode_width(int64_t V) { return (int)((V + 1 + 3) / 4 * 4); }
 
+// Chunked GLA: status word, varlen prefix sums, q~, k~, A and the row decays.
+struct GlaLayout {
+    bool valid = false;
+    sgla_status why = SGLA_ERR_INVALID_ARGUMENT;
+    int C = 0, NT = 0;
+    int64_t max_chunks = 0;
+    size_t off_chunk = 0, off_seg = 0, off_qt = 0, off_kt = 0, off_A = 0, off_gl = 0, bytes = 0;
+};
+
+GlaLayout gla_layout(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V, sgla_dtype dtype) {
+    GlaLayout L;
+    if (N < (varlen ? 1 : 0) || T < 0 || H < 1 || K < 1 || V < 1) return L;
+    if (dtype != SGLA_BF16 && dtype != SGLA_FP32) return L;
+    const int epc = dtype == SGLA_BF16 ? 8 : 4;  // elements per 16-byte piece
+    if (K > 256 || V > 4096 || H > 65535 || K % epc || V % epc) { L.why = SGLA_ERR_UNSUPPORTED; return L; }
+    const int64_t tokens = varlen ? T : N * T;
+    if (tokens >= kMaxTokens || N * H >= kMaxTokens) { L.why = SGLA_ERR_UNSUPPORTED; return L; }
+    L.C = gla_chunk_size((int)K);
+    if (varlen) {
+        L.max_chunks = T / L.C + N;
+    } else {
+        L.NT = (int)((T + L.C - 1) / L.C);
+        L.max_chunks = N * L.NT;
+    }
+    if (L.max_chunks >= kMaxTokens) { L.why = SGLA_ERR_UNSUPPORTED; return L; }
+    const size_t es = dtype == SGLA_BF16 ? 2 : 4;
+    size_t off = 256;
+    auto take = [&](size_t &o, size_t n) { o = off; off = align_up(off + n, 256); };
+    if (varlen) {
+        take(L.off_chunk, sizeof(int) * (size_t)(N + 1));
+        take(L.off_seg, sizeof(int) * (size_t)(N + 1));
+    }
+    take(L.off_qt, es * (size_t)tokens * H * K);
+    take(L.off_kt, es * (size_t)tokens * H * K);
+    take(L.off_A, es * (size_t)L.max_chunks * H * L.C * L.C);
+    take(L.off_gl, sizeof(float) * (size_t)L.max_chunks * H * K);
+    L.bytes = off;
+    L.valid = true;
+    return L;
+}
+
 // Chunked backward: three forward calls share the inner workspace (at offset 0, so
 // that its status word is the one sgla_workspace_status reads), followed by the
 // time-reversed operands, dk (fp32, reversed), dq (fp32), dv (reversed), q.dq - k.dk
@@ -483,6 +524,58 @@ sgla_status gla_fused_recurrent(const void *q, const void *k, const void *v, con
     if (!gk && (cu_seqlens ? T : N * T) > 0) return SGLA_ERR_INVALID_ARGUMENT;
     return fused_recurrent_impl(q, k, v, nullptr, gk, nullptr, scale, initial_state, o, final_state, cu_seqlens, N,
                                 T, H, K, V, state_v_first, dtype, device_status, stream);
+}
+
+size_t gla_chunk_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V,
+                                sgla_dtype dtype) {
+    const GlaLayout L = gla_layout(cu_seqlens != nullptr, N, T, H, K, V, dtype);
+    return L.valid ? L.bytes : 0;
+}
+
+sgla_status gla_chunk(const void *q, const void *k, const void *v, const float *gk, float scale,
+                      const float *initial_state, void *o, float *final_state, const int64_t *cu_seqlens, int64_t N,
+                      int64_t T, int64_t H, int64_t K, int64_t V, sgla_dtype dtype, void *workspace,
+                      size_t workspace_bytes, void *stream) {
+    const bool varlen = cu_seqlens != nullptr;
+    const GlaLayout L = gla_layout(varlen, N, T, H, K, V, dtype);
+    if (!L.valid) return L.why;
+    const int64_t tokens = varlen ? T : N * T;
+    if (tokens > 0 && (!q || !k || !v || !gk || !o)) return SGLA_ERR_INVALID_ARGUMENT;
+    const size_t es = dtype == SGLA_BF16 ? 2 : 4;
+    for (const void *p : {q, k, v, (const void *)gk})
+        if (!aligned(p, 16)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!aligned(o, es)) return SGLA_ERR_INVALID_ARGUMENT;
+    for (const void *p : {(const void *)initial_state, (const void *)final_state})
+        if (!aligned(p, 4)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!aligned(cu_seqlens, 8)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!workspace || workspace_bytes < L.bytes) return SGLA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!(scale > 0.f) || isnan(scale) || isinf(scale)) scale = 1.0f / sqrtf((float)K);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+    GlaArgs a{};
+    a.q = q; a.k = k; a.v = v; a.gk = gk; a.scale = scale; a.h0 = initial_state; a.o = o; a.hT = final_state;
+    a.qt = ws + L.off_qt; a.kt = ws + L.off_kt; a.A = ws + L.off_A;
+    a.gl = reinterpret_cast<float *>(ws + L.off_gl);
+    a.H = (int)H; a.K = (int)K; a.V = (int)V; a.bf16 = dtype == SGLA_BF16;
+    SeqLayout &lay = a.lay;
+    lay.cu = cu_seqlens;
+    lay.chunk_off = varlen ? reinterpret_cast<int *>(ws + L.off_chunk) : nullptr;
+    lay.seg_off = varlen ? reinterpret_cast<int *>(ws + L.off_seg) : nullptr;
+    lay.status = reinterpret_cast<int *>(ws);
+    lay.T = T; lay.N = (int)N; lay.H = (int)H; lay.C = L.C; lay.L = 1; lay.NT = L.NT; lay.NS = L.NT;
+    lay.max_chunks = (int)L.max_chunks; lay.max_segs = (int)L.max_chunks;
+    if (varlen) {
+        SGLA_LAUNCH("varlen_plan", launch_varlen_plan(cu_seqlens, (int)N, T, L.C, 1, const_cast<int *>(lay.chunk_off),
+                                                      const_cast<int *>(lay.seg_off), reinterpret_cast<int *>(ws),
+                                                      st));
+    } else {
+        SGLA_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), st), "status reset");
+    }
+    if (N == 0) return SGLA_OK;
+    if (tokens > 0) SGLA_LAUNCH("gla_chunk_prep", launch_gla_chunk_prep(a, st));
+    SGLA_LAUNCH("gla_chunk_walk", launch_gla_chunk_walk(a, st));
+    return SGLA_OK;
 }
 
 size_t simple_gla_chunk_bwd_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H, int64_t K,

@@ -79,6 +79,25 @@ struct RecBwdArgs {
     int H, K, V;
     bool bf16;
 };
+// Chunked GLA with a gate vector over K (gla_chunk.cu).
+struct GlaArgs {
+    const void *q, *k, *v;
+    const float *gk;      // [tokens, H, K] log gates
+    float scale;
+    const float *h0;      // [N, H, K, V] or NULL
+    void *o;
+    float *hT;            // [N, H, K, V] or NULL
+    void *qt, *kt;        // [tokens, H, K] q * 2^G, k * 2^(G_last - G) (workspace, operand dtype)
+    void *A;              // [chunks, H, C, C] intra-chunk scores (workspace, operand dtype)
+    float *gl;            // [chunks, H, K] row decays 2^G_last (workspace)
+    SeqLayout lay;        // C = chunk size, L = 1
+    int H, K, V;
+    bool bf16;
+};
+int gla_chunk_size(int K);
+cudaError_t launch_gla_chunk_prep(const GlaArgs &a, cudaStream_t st);
+cudaError_t launch_gla_chunk_walk(const GlaArgs &a, cudaStream_t st);
+
 // Row movers and the gate-gradient scan of the chunked backward (chunk_bwd.cu).
 struct BwdRowArgs {
     const void *q, *k, *v, *dout;  // token order, [tokens,H,K] / [tokens,H,V]

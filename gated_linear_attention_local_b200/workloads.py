@@ -32,6 +32,9 @@ test matrix with gate normalisers 0.1/1/10, scales 0.1/1 and the packed lengths
                 simple_gla_fused_recurrent_bwd
   chunk_bwd     the same gradients through the chunked tensor-core path at the same
                 size -- simple_gla_chunk_bwd
+  gla_chunk_prefill  GLA (gate vector over K) in the chunked form at relinear's training
+                scale: B=8, T=512, H=16, K=V=128, bf16, gk = logsigmoid(N(0,1)) / 16 per key,
+                initial and final state -- gla_chunk
   recurrent_prefill  the inference routing case of section 4 (at most 64 tokens go to
                 the fused recurrence): 256 sequences x 64 tokens, H=32 K=V=128, bf16,
                 g, initial state 0.1*N(0,1), final state -- simple_gla_fused_recurrent
@@ -65,6 +68,8 @@ WORKLOADS = {
                           dtype=torch.bfloat16, gate="g", h0=True, final_state=False, scale=None, chunk_size=64),
     "chunk_bwd": dict(kind="dense", entry="chunk_bwd", B=8, T=512, H=16, K=128, V=128, dtype=torch.bfloat16,
                       gate="g", h0=True, final_state=False, scale=None, chunk_size=64),
+    "gla_chunk_prefill": dict(kind="dense", entry="gla_chunk", B=8, T=512, H=16, K=128, V=128,
+                              dtype=torch.bfloat16, gate="gk", h0=True, final_state=True, scale=None, chunk_size=32),
     "recurrent_prefill": dict(kind="dense", entry="recurrent", B=256, T=64, H=32, K=128, V=128,
                               dtype=torch.bfloat16, gate="g", h0=True, final_state=True, scale=None,
                               chunk_size=64),

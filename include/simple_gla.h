@@ -333,6 +333,35 @@ SGLA_API sgla_status gla_fused_recurrent(const void *q, const void *k, const voi
                                 void *stream);
 
 /*
+ * GLA with a gate vector over K in the chunked form ("relinear", fla-org kernel
+ * integration: GLA's gate is [B,T,H,K] and its kernels are a vector chunk-local
+ * cumsum, an intra-chunk score matrix built from 16-token sub-chunks, and the output
+ * from the inter-chunk state; [FLA-SG] sections 3 and 6 on the per-key decay).  The
+ * same operator as gla_fused_recurrent:
+ *   S_t = diag(exp(gk_t)) S_{t-1} + k_t v_t^T ;  o_t = scale * S_t^T q_t
+ * computed chunk by chunk (32 tokens, two 16-token sub-chunks): a prep kernel
+ * forms, for every chunk in parallel, the per-key cumulative gates, q * 2^G,
+ * k * 2^(G_last - G), the row decays and the intra-chunk scores (exact inside each
+ * 16-token sub-chunk, through the sub-chunk boundary between sub-chunks); a walk
+ * kernel carries the K x 64 state in registers from chunk to chunk.
+ *   q, k [tokens,H,K], v, o [tokens,H,V] dtype; gk [tokens,H,K] fp32 log gates;
+ *   dense (cu_seqlens == NULL: N sequences of T tokens) or packed (cu_seqlens: DEVICE
+ *   [N+1], N >= 1, T packed tokens; a bad cu_seqlens writes nothing and is reported by
+ *   sgla_workspace_status(workspace)); initial_state / final_state [N,H,K,V] fp32 or
+ *   NULL; scale as simple_gla_fwd.
+ * Supported sizes: 1 <= K <= 256, 1 <= V <= 4096, K and V multiples of 8 (bf16) or 4
+ * (fp32); q, k, v, gk 16-byte aligned, o and the states aligned to their element.
+ * workspace: gla_chunk_workspace_size() bytes, 256-byte aligned.
+ */
+SGLA_API size_t gla_chunk_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H, int64_t K,
+                                         int64_t V, sgla_dtype dtype);
+SGLA_API sgla_status gla_chunk(const void *q, const void *k, const void *v, const float *gk, float scale,
+                               const float *initial_state, void *o, float *final_state,
+                               const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H, int64_t K,
+                               int64_t V, sgla_dtype dtype, void *workspace, size_t workspace_bytes,
+                               void *stream);
+
+/*
  * Normalised gated linear attention through the augmented value ("relinear -- convert
  * pretrained transformers to linear/hybrid-attention models", fla-org kernel
  * integration): o_t = (q_t^T S_t) / (q_t^T z_t) with the normaliser state

@@ -156,6 +156,28 @@ def test_fused_recurrent_bwd_validation_on_the_host(lib):
     assert call(dt=7) == L.SGLA_ERR_INVALID_ARGUMENT                  # unknown dtype
 
 
+def test_gla_chunk_validation_on_the_host(lib):
+    f = lib.gla_chunk
+    need = lib.gla_chunk_workspace_size(None, 4, 64, 2, 64, 64, L.SGLA_BF16)
+    # q~, k~ (bf16) and the 32 x 32 score blocks of 2 chunks per sequence, plus row decays
+    assert need >= 2 * 4 * 64 * 2 * 64 * 2 + 8 * 2 * 32 * 32 * 2 + 8 * 2 * 64 * 4
+    assert lib.gla_chunk_workspace_size(None, 4, 64, 2, 264, 64, L.SGLA_BF16) == 0   # K above 256
+    assert lib.gla_chunk_workspace_size(None, 4, 64, 2, 60, 64, L.SGLA_BF16) == 0    # bf16 K not a multiple of 8
+
+    def call(q=FAKE, gk=FAKE, cu=None, N=4, T=64, K=64, V=64, dt=L.SGLA_BF16, ws=FAKE, nws=None):
+        return f(q, FAKE, FAKE, gk, 1.0, None, FAKE, None, cu, N, T, 2, K, V, dt, ws, need if nws is None else nws,
+                 None)
+
+    assert call(K=264) == L.SGLA_ERR_UNSUPPORTED
+    assert call(V=68) == L.SGLA_ERR_UNSUPPORTED                       # bf16 V not a multiple of 8
+    assert call(q=FAKE + 8) == L.SGLA_ERR_INVALID_ARGUMENT            # q not 16-byte aligned
+    assert call(gk=None) == L.SGLA_ERR_INVALID_ARGUMENT               # tokens but no gate
+    assert call(cu=FAKE, N=0) == L.SGLA_ERR_INVALID_ARGUMENT          # packed with no sequence
+    assert call(nws=need - 1) == L.SGLA_ERR_WORKSPACE
+    assert call(ws=FAKE + 16) == L.SGLA_ERR_INVALID_ARGUMENT          # workspace not 256-byte aligned
+    assert call(dt=7) == L.SGLA_ERR_INVALID_ARGUMENT
+
+
 def test_binding_refuses_cpu_tensors():
     import gated_linear_attention_local_b200 as sg
     x = torch.zeros(1, 8, 1, 16)
