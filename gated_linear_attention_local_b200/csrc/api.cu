@@ -311,7 +311,7 @@ GlaLayout gla_layout(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, in
     if (K > 256 || V > 4096 || H > 65535 || K % epc || V % epc) { L.why = SGLA_ERR_UNSUPPORTED; return L; }
     const int64_t tokens = varlen ? T : N * T;
     if (tokens >= kMaxTokens || N * H >= kMaxTokens) { L.why = SGLA_ERR_UNSUPPORTED; return L; }
-    L.C = gla_chunk_size((int)K);
+    L.C = gla_chunk_size(dtype == SGLA_BF16, (int)K, (int)V);
     if (varlen) {
         L.max_chunks = T / L.C + N;
     } else {
@@ -573,8 +573,17 @@ sgla_status gla_chunk(const void *q, const void *k, const void *v, const float *
         SGLA_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), st), "status reset");
     }
     if (N == 0) return SGLA_OK;
-    if (tokens > 0) SGLA_LAUNCH("gla_chunk_prep", launch_gla_chunk_prep(a, st));
-    SGLA_LAUNCH("gla_chunk_walk", launch_gla_chunk_walk(a, st));
+    if (tokens == 0) {  // every sequence is empty: the final state is the initial one
+        const size_t sb = sizeof(float) * (size_t)N * H * K * V;
+        if (final_state && initial_state)
+            SGLA_CUDA(cudaMemcpyAsync(final_state, initial_state, sb, cudaMemcpyDeviceToDevice, st), "final state");
+        else if (final_state)
+            SGLA_CUDA(cudaMemsetAsync(final_state, 0, sb, st), "final state");
+        return SGLA_OK;
+    }
+    SGLA_LAUNCH("gla_chunk_prep", launch_gla_chunk_prep(a, st));
+    if (gla_chunk_tc(a.bf16, a.K, a.V)) SGLA_LAUNCH("gla_chunk_walk_tc", launch_gla_chunk_walk_tc(a, st));
+    else SGLA_LAUNCH("gla_chunk_walk", launch_gla_chunk_walk(a, st));
     return SGLA_OK;
 }
 

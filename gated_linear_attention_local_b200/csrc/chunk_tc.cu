@@ -967,6 +967,12 @@ bool tc_path_supports(bool bf16, int K, int V, int C) {
 
 int tc_path_step() { return kStep; }
 
+cudaError_t tc_make_map(CUtensorMap *m, const void *ptr, int64_t tokens, int H, int D, int box) {
+    cudaError_t e = get_encoder();
+    if (e != cudaSuccess) return e;
+    return make_map(m, ptr, tokens, H, D, box);
+}
+
 int tc_path_vtiles(int K, int V) { return V / walk_bv(K); }
 
 cudaError_t tc_launch_segment_state(const FwdArgs &a, cudaStream_t st) {

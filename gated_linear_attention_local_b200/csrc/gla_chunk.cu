@@ -24,14 +24,15 @@
 // tile)) walks the chunks of its sequence in order with the K x 64 state in
 // registers: o from q~ h + A v, then h' from the decays and k~^T v.
 #include "kernels.h"
+#include "tc_ptx.cuh"
 
 namespace sgla {
 
 namespace {
 
 constexpr int kGlaSub = 16;      // sub-chunk (tokens)
-constexpr int kGlaC = 32;        // chunk (tokens): two sub-chunks
-constexpr int kGlaKS = 128;      // key columns per pass of the prep kernel
+constexpr int kGlaC = 32;        // chunk of the CUDA-core walk (tokens): two sub-chunks
+constexpr int kGlaCTc = 128;     // chunk of the tensor-core walk: eight sub-chunks, one MMA M
 constexpr int kGlaThreads = 256;
 constexpr int kGlaBV = 64;       // V tile of the walk
 
@@ -44,6 +45,9 @@ struct Vec<float> {
     __device__ static void load(const float *p, float *f) {
         const float4 v = *reinterpret_cast<const float4 *>(p);
         f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+    }
+    __device__ static void store(float *p, const float *f) {
+        *reinterpret_cast<float4 *>(p) = make_float4(f[0], f[1], f[2], f[3]);
     }
 };
 template <>
@@ -59,19 +63,54 @@ struct Vec<__nv_bfloat16> {
             f[2 * i + 1] = u.y;
         }
     }
+    __device__ static void store(__nv_bfloat16 *p, const float *f) {
+        uint4 v;
+        __nv_bfloat162 *b = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) b[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+        *reinterpret_cast<uint4 *>(p) = v;
+    }
 };
 
+// Shared-memory plan of the prep kernel for chunk C and key pass KS (floats).
+template <int C, int KS>
 struct PrepSmem {
-    static constexpr int LD = kGlaKS + 1;
-    static constexpr size_t floats = 4 * (size_t)kGlaC * LD + (size_t)kGlaC * (kGlaC + 1);
+    static constexpr int NSUB = C / kGlaSub;
+    static constexpr int NOFF = 8 * NSUB * (NSUB - 1);  // columns of all off-diagonal block rows
+    static constexpr int LG = KS + 1;                   // G, QH rows
+    static constexpr int LP = 2 * (KS + 1);             // QG, KG rows (float2 pairs)
+    static constexpr int LKT = NOFF + 4;                // KT rows (x)
+    static constexpr int LK0 = C + 4;                   // K0T rows (x)
+    static constexpr size_t G = 0;
+    static constexpr size_t QG = G + (size_t)C * LG;
+    static constexpr size_t KG = QG + (size_t)C * LP;
+    static constexpr size_t QH = KG + (size_t)C * LP;
+    static constexpr size_t KT = (QH + (size_t)C * LG + 3) / 4 * 4;
+    static constexpr size_t K0T = KT + (size_t)KS * LKT;
+    static constexpr size_t DD = K0T + (size_t)KS * LK0;
+    static constexpr size_t floats = DD + (size_t)NSUB * NSUB * KS;
 };
 
-// One CTA per (chunk, head).  Key columns go in passes of kGlaKS; A accumulates over
-// the passes in shared memory.
-template <typename T>
+// One CTA per (chunk, head); key columns in passes of KS.  Per pass: stage q, k and
+// the log gates; cumulative sums down each column (TPC threads per column); q~, k~
+// and the row decays out; then the scores.  Diagonal 16 x 16 blocks: their lower
+// triangles, one entry per thread slot, each term with the exact exp2 of its gate
+// difference.  Blocks left of the diagonal (block row I, columns j < 16 I): through
+// the boundary b(I) = 16 I - 1, A_ij = sum_x qh_ix kh^(I)_jx with qh_i = q_i 2^{G_i -
+// G_b(I)} and kh^(I)_j = k_j 2^{G_e(J) - G_j} 2^{G_b(I) - G_e(J)} (e(J) the last token
+// of j's block J: both factors <= 1, the second one per (I, J, x) only); each thread
+// slot owns a 2 x 4 tile of one block row.  Sums live in registers across passes.  A
+// is stored [chunk][i][head][j], a [chunks * C, H, C] tensor whose rows are token
+// positions (a TMA box of C rows is one block).
+template <typename T, int C, int KS>
 __global__ void __launch_bounds__(kGlaThreads)
 gla_chunk_prep_kernel(GlaArgs a) {
-    constexpr int C = kGlaC, LD = PrepSmem::LD, NSUB = C / kGlaSub, VN = Vec<T>::n;
+    using P = PrepSmem<C, KS>;
+    constexpr int NSUB = P::NSUB, VN = Vec<T>::n;
+    constexpr int NDIAG = NSUB * (kGlaSub * (kGlaSub + 1) / 2), DSLOTS = (NDIAG + kGlaThreads - 1) / kGlaThreads;
+    constexpr int NTILE = 16 * NSUB * (NSUB - 1), TSLOTS = (NTILE + kGlaThreads - 1) / kGlaThreads;
+    constexpr int TPC = kGlaThreads / KS, RPT = C / TPC;  // cumsum: threads per column, rows per thread
+    static_assert(kGlaThreads % KS == 0 && C % TPC == 0 && TPC <= 32, "cumsum split");
     const SeqLayout &lay = a.lay;
     if (device_failed(lay)) return;
     int n, c;
@@ -83,26 +122,70 @@ gla_chunk_prep_kernel(GlaArgs a) {
     const int len = (int)min64(C, t1 - ta);
     const int64_t u = blockIdx.x;  // global chunk index
 
-    extern __shared__ float gsm[];
-    float *G = gsm;              // [C][LD] cumulative log2 gates
-    float *Q = G + C * LD;       // [C][LD] q, then q * 2^{G_i - G_b(I)}
-    float *Kr = Q + C * LD;      // [C][LD] k
-    float *Kh = Kr + C * LD;     // [C][LD] k * 2^{G_b(I) - G_j}
-    float *A = Kh + C * LD;      // [C][C+1]
+    extern __shared__ float4 psm4[];
+    float *sm = reinterpret_cast<float *>(psm4);
+    float *G = sm + P::G;
+    float2 *QG = reinterpret_cast<float2 *>(sm + P::QG);
+    float2 *KG = reinterpret_cast<float2 *>(sm + P::KG);
+    float *QH = sm + P::QH;
+    float *KT = sm + P::KT;
+    float *K0T = sm + P::K0T;
+    float *DD = sm + P::DD;
     const T *qp = static_cast<const T *>(a.q);
     const T *kp = static_cast<const T *>(a.k);
     T *qt = static_cast<T *>(a.qt);
     T *kt = static_cast<T *>(a.kt);
     const int tid = threadIdx.x;
 
-    for (int e = tid; e < C * (C + 1); e += kGlaThreads) A[e] = 0.f;
+    // slots: diagonal entries (lower triangles) and 2 x 4 tiles left of the diagonal
+    int di[DSLOTS], dj[DSLOTS], ti[TSLOTS], tcol[TSLOTS], tko[TSLOTS];
+    bool dv[DSLOTS], tv[TSLOTS];
+#pragma unroll
+    for (int d = 0; d < DSLOTS; ++d) {
+        const int L = tid + kGlaThreads * d;
+        const int m = L / 136, r = L % 136;
+        int il = 0;
+        while ((il + 1) * (il + 2) / 2 <= r) ++il;
+        di[d] = m * kGlaSub + il;
+        dj[d] = m * kGlaSub + (r - il * (il + 1) / 2);
+        dv[d] = L < NDIAG && di[d] < len;
+    }
+#pragma unroll
+    for (int q = 0; q < TSLOTS; ++q) {
+        const int L = tid + kGlaThreads * q;
+        int I = 1, base = 0;
+        while (I < NSUB - 1 && L >= base + 32 * I) base += 32 * I++;
+        const int idx = L - base;
+        ti[q] = I * kGlaSub + 2 * (idx / (4 * I));
+        tcol[q] = 4 * (idx % (4 * I));
+        tko[q] = 8 * I * (I - 1) + tcol[q];  // column of the tile in KT
+        tv[q] = L < NTILE && ti[q] < len;
+    }
+    // columns of KT this thread fills: block row I, key row j of block J
+    constexpr int KSLOTS = (P::NOFF + kGlaThreads - 1) / kGlaThreads;
+    int kc[KSLOTS], kj[KSLOTS], kd[KSLOTS];
+#pragma unroll
+    for (int m = 0; m < KSLOTS; ++m) {
+        const int col = tid + kGlaThreads * m;
+        int I = 1;
+        while (8 * (I + 1) * I <= col && I < NSUB - 1) ++I;
+        kc[m] = col;
+        kj[m] = col - 8 * I * (I - 1);
+        kd[m] = I * NSUB + kj[m] / kGlaSub;  // (I, J) row of DD
+    }
+    float dacc[DSLOTS], oacc[TSLOTS][8];
+#pragma unroll
+    for (int d = 0; d < DSLOTS; ++d) dacc[d] = 0.f;
+#pragma unroll
+    for (int q = 0; q < TSLOTS; ++q)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) oacc[q][e] = 0.f;
 
-    for (int k0 = 0; k0 < K; k0 += kGlaKS) {
-        const int kw = min(kGlaKS, K - k0);
+    for (int k0 = 0; k0 < K; k0 += KS) {
+        const int kw = min(KS, K - k0);
         __syncthreads();  // the previous pass is done with every buffer
-        // rows of q, k (16-byte pieces) and of the gates (float4), all loads first
-        for (int e = tid; e < C * (kGlaKS / VN); e += kGlaThreads) {
-            const int i = e / (kGlaKS / VN), x = (e % (kGlaKS / VN)) * VN;
+        for (int e = tid; e < C * (KS / VN); e += kGlaThreads) {
+            const int i = e / (KS / VN), x = (e % (KS / VN)) * VN;
             float qv[VN], kv[VN], gv[VN];
             const bool ok = i < len && x < kw;
             const int64_t off = ((ta + i) * H + h) * (int64_t)K + k0 + x;
@@ -114,73 +197,109 @@ gla_chunk_prep_kernel(GlaArgs a) {
             }
 #pragma unroll
             for (int y = 0; y < VN; ++y) {
-                G[i * LD + x + y] = ok ? fmaxf(gv[y], kMinLogGate) * kRcpLn2 : 0.f;
-                Q[i * LD + x + y] = ok ? qv[y] : 0.f;
-                Kr[i * LD + x + y] = ok ? kv[y] : 0.f;
+                G[i * P::LG + x + y] = ok ? fmaxf(gv[y], kMinLogGate) * kRcpLn2 : 0.f;
+                QG[i * (KS + 1) + x + y].x = ok ? qv[y] : 0.f;
+                KG[i * (KS + 1) + x + y].x = ok ? kv[y] : 0.f;
             }
         }
         __syncthreads();
-        // chunk-local inclusive cumsum down each column (padding rows add 0)
-        for (int x = tid; x < kGlaKS; x += kGlaThreads) {
-            float acc = 0.f;
-#pragma unroll 8
-            for (int i = 0; i < C; ++i) {
-                acc += G[i * LD + x];
-                G[i * LD + x] = acc;
+        {   // cumsum: column x = tid / TPC, rows [RPT s, RPT s + RPT) for s = tid % TPC
+            const int x = tid / TPC, sg = tid % TPC;
+            float part = 0.f;
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) part += G[(sg * RPT + r) * P::LG + x];
+            float incl = part;
+#pragma unroll
+            for (int o = 1; o < TPC; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, o, TPC);
+                if (sg >= o) incl += y;
+            }
+            float run = incl - part;
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) {
+                run += G[(sg * RPT + r) * P::LG + x];
+                G[(sg * RPT + r) * P::LG + x] = run;
             }
         }
         __syncthreads();
-        // q~, k~ and the row decays of this pass
-        for (int e = tid; e < C * kGlaKS; e += kGlaThreads) {
-            const int i = e / kGlaKS, x = e - i * kGlaKS;
-            if (i < len && x < kw) {
-                const int64_t off = ((ta + i) * H + h) * (int64_t)K + k0 + x;
-                const float gi = G[i * LD + x], gl = G[(C - 1) * LD + x];
-                qt[off] = from_f32<T>(Q[i * LD + x] * exp2f(gi));
-                kt[off] = from_f32<T>(Kr[i * LD + x] * exp2f(gl - gi));
+        // one 16-byte piece (VN keys) of one row per step: q~, k~ out as whole pieces
+        for (int e = tid; e < C * (KS / VN); e += kGlaThreads) {
+            const int i = e / (KS / VN), x0 = (e % (KS / VN)) * VN, I = i / kGlaSub;
+            const int b = I * kGlaSub - 1, ee = I * kGlaSub + kGlaSub - 1;
+            float fq[VN], fk[VN];
+#pragma unroll
+            for (int y = 0; y < VN; ++y) {
+                const int x = x0 + y;
+                const float gi = G[i * P::LG + x], gl = G[(C - 1) * P::LG + x];
+                const float qv = QG[i * (KS + 1) + x].x, kv = KG[i * (KS + 1) + x].x;
+                QG[i * (KS + 1) + x].y = gi;
+                KG[i * (KS + 1) + x].y = gi;
+                fq[y] = qv * tc::fast_exp2(gi);
+                fk[y] = kv * tc::fast_exp2(gl - gi);
+                if (I > 0) QH[i * P::LG + x] = qv * tc::fast_exp2(gi - G[b * P::LG + x]);
+                K0T[x * P::LK0 + i] = kv * tc::fast_exp2(G[ee * P::LG + x] - gi);
             }
+            if (i < len && x0 < kw) {
+                const int64_t off = ((ta + i) * H + h) * (int64_t)K + k0 + x0;
+                Vec<T>::store(qt + off, fq);
+                Vec<T>::store(kt + off, fk);
+            }
+        }
+        for (int e = tid; e < NSUB * NSUB * KS; e += kGlaThreads) {
+            const int I = e / (NSUB * KS), J = (e / KS) % NSUB, x = e % KS;
+            if (J < I) DD[e] = tc::fast_exp2(G[(I * kGlaSub - 1) * P::LG + x] - G[(J * kGlaSub + kGlaSub - 1) * P::LG + x]);
         }
         for (int x = tid; x < kw; x += kGlaThreads)
-            a.gl[(u * H + h) * (int64_t)K + k0 + x] = exp2f(G[(C - 1) * LD + x]);
-        // diagonal sub-chunks, term by term
-        for (int e = tid; e < NSUB * kGlaSub * kGlaSub; e += kGlaThreads) {
-            const int I = e / (kGlaSub * kGlaSub), r = e - I * kGlaSub * kGlaSub;
-            const int i = I * kGlaSub + r / kGlaSub, j = I * kGlaSub + r % kGlaSub;
-            if (j > i || i >= len) continue;
-            float acc = 0.f;
-            for (int x = 0; x < kw; ++x)
-                acc = fmaf(Q[i * LD + x] * Kr[j * LD + x], exp2f(G[i * LD + x] - G[j * LD + x]), acc);
-            A[i * (C + 1) + j] += acc;
+            a.gl[(u * H + h) * (int64_t)K + k0 + x] = tc::fast_exp2(G[(C - 1) * P::LG + x]);
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < KSLOTS; ++m) {  // kh^(I) for every block row, fixed columns per thread
+            if (kc[m] < P::NOFF)
+                for (int x = 0; x < KS; ++x)
+                    KT[x * P::LKT + kc[m]] = K0T[x * P::LK0 + kj[m]] * DD[kd[m] * KS + x];
         }
-        __syncthreads();  // diagonal blocks have read the raw q
-        // q rows of sub-chunks I >= 1 relative to the boundary b(I) = 16 I - 1
-        for (int e = tid; e < (C - kGlaSub) * kGlaKS; e += kGlaThreads) {
-            const int i = kGlaSub + e / kGlaKS, x = e % kGlaKS;
-            const int b = (i / kGlaSub) * kGlaSub - 1;
-            Q[i * LD + x] *= exp2f(G[i * LD + x] - G[b * LD + x]);
-        }
-        for (int I = 1; I < NSUB; ++I) {
-            const int s = I * kGlaSub, b = s - 1;
-            __syncthreads();  // Q is rescaled; the previous block is done with Kh
-            for (int e = tid; e < s * kGlaKS; e += kGlaThreads) {
-                const int j = e / kGlaKS, x = e - j * kGlaKS;
-                Kh[j * LD + x] = Kr[j * LD + x] * exp2f(G[b * LD + x] - G[j * LD + x]);
+        __syncthreads();
+        for (int x = 0; x < kw; ++x) {
+#pragma unroll
+            for (int d = 0; d < DSLOTS; ++d) {
+                if (dv[d]) {
+                    const float2 qg = QG[di[d] * (KS + 1) + x], kg = KG[dj[d] * (KS + 1) + x];
+                    dacc[d] = fmaf(qg.x * kg.x, tc::fast_exp2(qg.y - kg.y), dacc[d]);
+                }
             }
-            __syncthreads();
-            for (int e = tid; e < kGlaSub * s; e += kGlaThreads) {
-                const int i = s + e / s, j = e % s;
-                if (i >= len) continue;
-                float acc = 0.f;
-                for (int x = 0; x < kw; ++x) acc = fmaf(Q[i * LD + x], Kh[j * LD + x], acc);
-                A[i * (C + 1) + j] += acc;
+#pragma unroll
+            for (int q = 0; q < TSLOTS; ++q) {
+                if (tv[q]) {
+                    const float q0 = QH[ti[q] * P::LG + x], q1 = QH[(ti[q] + 1) * P::LG + x];
+                    const float4 k4 = *reinterpret_cast<const float4 *>(KT + x * P::LKT + tko[q]);
+                    oacc[q][0] = fmaf(q0, k4.x, oacc[q][0]);
+                    oacc[q][1] = fmaf(q0, k4.y, oacc[q][1]);
+                    oacc[q][2] = fmaf(q0, k4.z, oacc[q][2]);
+                    oacc[q][3] = fmaf(q0, k4.w, oacc[q][3]);
+                    oacc[q][4] = fmaf(q1, k4.x, oacc[q][4]);
+                    oacc[q][5] = fmaf(q1, k4.y, oacc[q][5]);
+                    oacc[q][6] = fmaf(q1, k4.z, oacc[q][6]);
+                    oacc[q][7] = fmaf(q1, k4.w, oacc[q][7]);
+                }
             }
         }
     }
-    __syncthreads();
-    T *Ap = static_cast<T *>(a.A) + (u * H + h) * (int64_t)C * C;
+    // A: the slots' sums (rows past the sequence end as 0), and 0 above the diagonal
+    T *Ap = static_cast<T *>(a.A);
+    auto put = [&](int i, int j, float v) {
+        Ap[((u * C + i) * H + h) * (int64_t)C + j] = from_f32<T>(i < len ? v : 0.f);
+    };
+#pragma unroll
+    for (int d = 0; d < DSLOTS; ++d)
+        if (tid + kGlaThreads * d < NDIAG) put(di[d], dj[d], dacc[d]);
+#pragma unroll
+    for (int q = 0; q < TSLOTS; ++q)
+        if (tid + kGlaThreads * q < NTILE)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) put(ti[q] + e / 4, tcol[q] + e % 4, oacc[q][e]);
     for (int e = tid; e < C * C; e += kGlaThreads) {
         const int i = e / C, j = e - i * C;
-        Ap[e] = from_f32<T>((j <= i && i < len) ? A[i * (C + 1) + j] : 0.f);
+        if (j > i) Ap[((u * C + i) * H + h) * (int64_t)C + j] = from_f32<T>(0.f);
     }
 }
 
@@ -262,11 +381,10 @@ gla_chunk_walk_kernel(GlaArgs a) {
                     kS[i * S::LDK + x + y] = ok ? kv[y] : 0.f;
                 }
             }
-            const T *Ac = At + (u * H + h) * (int64_t)C * C;
             for (int e = tid; e < C * C / VN; e += kGlaThreads) {
                 const int i = e / (C / VN), j = (e % (C / VN)) * VN;
                 float av[VN];
-                Vec<T>::load(Ac + i * C + j, av);
+                Vec<T>::load(At + ((u * C + i) * H + h) * (int64_t)C + j, av);
 #pragma unroll
                 for (int y = 0; y < VN; ++y) aS[i * S::LDA + j + y] = av[y];
             }
@@ -365,10 +483,10 @@ gla_chunk_walk_kernel(GlaArgs a) {
     }
 }
 
-template <typename T>
+template <typename T, int C, int KS>
 cudaError_t launch_prep_t(const GlaArgs &a, cudaStream_t st) {
-    const size_t smem = sizeof(float) * PrepSmem::floats;
-    auto kern = gla_chunk_prep_kernel<T>;
+    const size_t smem = sizeof(float) * PrepSmem<C, KS>::floats;
+    auto kern = gla_chunk_prep_kernel<T, C, KS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<dim3((unsigned)a.lay.max_chunks, (unsigned)a.H), kGlaThreads, smem, st>>>(a);
@@ -387,12 +505,15 @@ cudaError_t launch_walk_t(const GlaArgs &a, cudaStream_t st) {
 
 }  // namespace
 
-int gla_chunk_size(int) { return kGlaC; }
+bool gla_chunk_tc(bool bf16, int K, int V) { return bf16 && K == 128 && V % 64 == 0 && V >= 64; }
+
+int gla_chunk_size(bool bf16, int K, int V) { return gla_chunk_tc(bf16, K, V) ? kGlaCTc : kGlaC; }
 
 cudaError_t launch_gla_chunk_prep(const GlaArgs &a, cudaStream_t st) {
     if (a.lay.max_chunks == 0) return cudaSuccess;
+    if (a.lay.C == kGlaCTc && a.bf16) return launch_prep_t<__nv_bfloat16, kGlaCTc, 16>(a, st);
     if (a.lay.C != kGlaC) return cudaErrorInvalidValue;
-    return a.bf16 ? launch_prep_t<__nv_bfloat16>(a, st) : launch_prep_t<float>(a, st);
+    return a.bf16 ? launch_prep_t<__nv_bfloat16, kGlaC, 64>(a, st) : launch_prep_t<float, kGlaC, 64>(a, st);
 }
 
 cudaError_t launch_gla_chunk_walk(const GlaArgs &a, cudaStream_t st) {

@@ -88,15 +88,17 @@ struct GlaArgs {
     void *o;
     float *hT;            // [N, H, K, V] or NULL
     void *qt, *kt;        // [tokens, H, K] q * 2^G, k * 2^(G_last - G) (workspace, operand dtype)
-    void *A;              // [chunks, H, C, C] intra-chunk scores (workspace, operand dtype)
+    void *A;              // [chunks, C, H, C] intra-chunk scores (workspace, operand dtype)
     float *gl;            // [chunks, H, K] row decays 2^G_last (workspace)
     SeqLayout lay;        // C = chunk size, L = 1
     int H, K, V;
     bool bf16;
 };
-int gla_chunk_size(int K);
+bool gla_chunk_tc(bool bf16, int K, int V);           // tensor-core walk covers these sizes
+int gla_chunk_size(bool bf16, int K, int V);         // chunk (tokens) of the path taken
 cudaError_t launch_gla_chunk_prep(const GlaArgs &a, cudaStream_t st);
 cudaError_t launch_gla_chunk_walk(const GlaArgs &a, cudaStream_t st);
+cudaError_t launch_gla_chunk_walk_tc(const GlaArgs &a, cudaStream_t st);
 
 // Row movers and the gate-gradient scan of the chunked backward (chunk_bwd.cu).
 struct BwdRowArgs {

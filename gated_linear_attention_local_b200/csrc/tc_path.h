@@ -1,6 +1,8 @@
 // Tensor-core (tcgen05 / TMEM / TMA) chunk path for bf16 operands.
 #pragma once
 
+#include <cuda.h>
+
 #include "kernels.h"
 
 namespace sgla {
@@ -13,6 +15,9 @@ int tc_path_vtiles(int K, int V);
 int tc_path_step();
 
 cudaError_t tc_launch_segment_state(const FwdArgs &a, cudaStream_t st);
+// 3-D TMA map over a [tokens, H, D] bf16 tensor, box [128 tokens x 1 head x box],
+// box = 64 (128-byte swizzle) or 32 (64-byte swizzle).
+cudaError_t tc_make_map(CUtensorMap *m, const void *ptr, int64_t tokens, int H, int D, int box);
 cudaError_t tc_launch_chunk_output(const FwdArgs &a, cudaStream_t st);
 
 }  // namespace sgla

@@ -53,6 +53,12 @@ CASES = [
     (2, 90, 2, 64, 64, torch.float32, True, "zero"),
     (2, 0, 2, 64, 64, torch.float32, True, "weak"),
     (3, 1, 2, 128, 64, torch.bfloat16, True, "weak"),
+    # tensor-core walk (bf16, K = 128, V a multiple of 64): several 128-token chunks,
+    # a ragged last one, three V tiles, strong and zero gates, no initial state
+    (2, 300, 2, 128, 192, torch.bfloat16, True, "strong"),
+    (1, 1000, 2, 128, 64, torch.bfloat16, False, "weak"),
+    (2, 129, 1, 128, 128, torch.bfloat16, True, "zero"),
+    (2, 0, 2, 128, 64, torch.bfloat16, True, "weak"),
 ]
 
 
@@ -70,10 +76,10 @@ def test_gla_chunk_dense(case):
     assert_close(host(ht), rh, TOL[dt], "final_state")
 
 
-@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float32])
-def test_gla_chunk_varlen(dt):
+@pytest.mark.parametrize("dt,K", [(torch.bfloat16, 64), (torch.float32, 64), (torch.bfloat16, 128)])
+def test_gla_chunk_varlen(dt, K):
     cu = torch.tensor([0, 15, 15, 100, 300, 1200], dtype=torch.int64)
-    T, H, K, V = 1200, 2, 64, 64
+    T, H, V = 1200, 2, 64
     inp = random_inputs(1, T, H, K, V, dtype=dt, gate="none", h0=True, seed=93, cu_seqlens=cu)
     gk = _gk((1, T, H, K), 94, "strong")
     o, ht = sg.gla_chunk(to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"]), gk.cuda(),
@@ -112,3 +118,18 @@ def test_gla_chunk_workload_sampled():
         assert_close(host(ht[n:n + 1]), rh, TOL[torch.bfloat16], f"final_state[{n}]")
     assert_close(host(o), host(o2), TOL[torch.bfloat16], "o vs token-serial")
     assert_close(host(ht), host(ht2), TOL[torch.bfloat16], "final_state vs token-serial")
+
+
+def test_gla_chunk_takes_the_tensor_core_walk():
+    """bf16 with K = 128 and V a multiple of 64 runs the tcgen05 walk; other shapes the
+    CUDA-core one."""
+    from gated_linear_attention_local_b200 import _lib
+    for K, V, dt, want in ((128, 128, torch.bfloat16, "gla_chunk_walk_tc"), (64, 64, torch.bfloat16, "gla_chunk_walk"),
+                           (128, 128, torch.float32, "gla_chunk_walk")):
+        inp = random_inputs(1, 200, 2, K, V, dtype=dt, gate="none", seed=97)
+        gk = _gk((1, 200, 2, K), 98)
+        _lib.profile_begin()
+        sg.gla_chunk(to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"]), gk.cuda())
+        torch.cuda.synchronize()
+        names = set(_lib.profile_end())
+        assert want in names and ({"gla_chunk_walk", "gla_chunk_walk_tc"} - {want}).isdisjoint(names), names
