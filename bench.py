@@ -97,13 +97,35 @@ def load_peaks():
         return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
-def sources_hash():
-    """sha256[:16] of the CUDA sources, to tell whether a stored ncu capture still
-    describes the kernels that run."""
+# The source files each timed kernel is built from (its own file plus the shared
+# headers), so that a stored ncu capture stays valid while unrelated files change.
+_CSRC_COMMON = ["common.cuh", "kernels.h"]
+KERNEL_SOURCES = {
+    "chunk_output_tc": ["chunk_tc.cu", "tc_ptx.cuh", "tc_path.h"],
+    "segment_state_tc": ["chunk_tc.cu", "tc_ptx.cuh", "tc_path.h"],
+    "decode_step": ["decode.cu"],
+    "fused_recurrent": ["recurrent.cu"],
+    "gla_fused_recurrent": ["recurrent.cu"],
+    "recurrent_bwd_reverse_sweep": ["recurrent_bwd.cu"],
+    "recurrent_bwd_forward_sweep": ["recurrent_bwd.cu"],
+    "gla_chunk_prep": ["gla_chunk.cu", "tc_ptx.cuh"],
+    "gla_chunk_walk_tc": ["gla_chunk_tc.cu", "tc_ptx.cuh", "tc_path.h"],
+}
+
+
+def sources_hash(kernel=None):
+    """sha256[:16] of the CUDA sources a kernel is built from (all of csrc/ when the
+    kernel is not listed), to tell whether a stored ncu capture still describes the
+    kernel that runs."""
     import glob
     import hashlib
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "gated_linear_attention_local_b200", "csrc", "*"))):
+    csrc = os.path.join(ROOT, "gated_linear_attention_local_b200", "csrc")
+    if kernel in KERNEL_SOURCES:
+        paths = [os.path.join(csrc, f) for f in sorted(set(KERNEL_SOURCES[kernel] + _CSRC_COMMON))]
+    else:
+        paths = sorted(glob.glob(os.path.join(csrc, "*")))
+    for p in paths:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -111,13 +133,14 @@ def sources_hash():
 
 def captured_traffic(workload, kernel):
     """DRAM bytes per launch of `kernel` on `workload` from the committed ncu capture
-    (profiles/traffic.json), or None when there is none or the sources changed since."""
+    (profiles/traffic.json), or None when there is none or the kernel's sources
+    changed since."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)[workload][kernel]
     except (OSError, KeyError, ValueError):
         return None
-    if rec.get("sources_sha256_16") != sources_hash():
+    if rec.get("sources_sha256_16") != sources_hash(kernel):
         return None
     return rec.get("dram_bytes_per_launch")
 
