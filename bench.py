@@ -69,6 +69,14 @@ def algorithmic_counts(w):
     flops = H * (4 * tokens * K * V + tokens * (C + 1) * (K + V))
     if w.get("entry") in ("recurrent", "gla", "gla_chunk"):  # state update and read-out per token
         flops = H * tokens * 4 * K * V
+    if w.get("entry") == "gla_chunk":
+        # prep (CUDA cores): the causal half of the intra-chunk q k^T with per-key decays,
+        # 128-token chunks; walk (tensor cores): q~ h, A v and the state update
+        Cg = 128
+        prep = dict(bytes=b, flops=H * tokens * (Cg + 1) * K)
+        walk = dict(bytes=b, flops=H * tokens * (4 * K * V + (Cg + 1) * V))
+        return dict(bytes=b, flops=prep["flops"] + walk["flops"], tokens=tokens,
+                    kernel={"gla_chunk_prep": prep, "gla_chunk_walk_tc": walk})
     if w.get("entry") in ("recurrent_bwd", "chunk_bwd"):
         fwd = dict(bytes=b, flops=flops)  # one forward call with these operands (K == V)
         # read do; write dq, dk, dv, dg; read dht, write dh0
@@ -109,6 +117,7 @@ KERNEL_SOURCES = {
     "recurrent_bwd_reverse_sweep": ["recurrent_bwd.cu"],
     "recurrent_bwd_forward_sweep": ["recurrent_bwd.cu"],
     "gla_chunk_prep": ["gla_chunk.cu", "tc_ptx.cuh"],
+    "bwd_reverse_inputs": ["chunk_bwd.cu"],
     "gla_chunk_walk_tc": ["gla_chunk_tc.cu", "tc_ptx.cuh", "tc_path.h"],
 }
 
