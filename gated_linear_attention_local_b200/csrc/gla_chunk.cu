@@ -139,7 +139,6 @@ gla_chunk_prep_kernel(GlaArgs a) {
 
     // slots: diagonal entries (lower triangles) and 2 x 4 tiles left of the diagonal
     int di[DSLOTS], dj[DSLOTS], ti[TSLOTS], tcol[TSLOTS], tko[TSLOTS];
-    bool dv[DSLOTS], tv[TSLOTS];
 #pragma unroll
     for (int d = 0; d < DSLOTS; ++d) {
         const int L = tid + kGlaThreads * d;
@@ -148,7 +147,6 @@ gla_chunk_prep_kernel(GlaArgs a) {
         while ((il + 1) * (il + 2) / 2 <= r) ++il;
         di[d] = m * kGlaSub + il;
         dj[d] = m * kGlaSub + (r - il * (il + 1) / 2);
-        dv[d] = L < NDIAG && di[d] < len;
     }
 #pragma unroll
     for (int q = 0; q < TSLOTS; ++q) {
@@ -159,7 +157,19 @@ gla_chunk_prep_kernel(GlaArgs a) {
         ti[q] = I * kGlaSub + 2 * (idx / (4 * I));
         tcol[q] = 4 * (idx % (4 * I));
         tko[q] = 8 * I * (I - 1) + tcol[q];  // column of the tile in KT
-        tv[q] = L < NTILE && ti[q] < len;
+    }
+    int dq_off[DSLOTS], dk_off[DSLOTS], tq_off[TSLOTS];
+#pragma unroll
+    for (int d = 0; d < DSLOTS; ++d) {
+        const bool in = tid + kGlaThreads * d < NDIAG;
+        dq_off[d] = in ? di[d] * (KS + 1) : 0;
+        dk_off[d] = in ? dj[d] * (KS + 1) : 0;
+    }
+#pragma unroll
+    for (int q = 0; q < TSLOTS; ++q) {
+        const bool in = tid + kGlaThreads * q < NTILE;
+        tq_off[q] = in ? ti[q] * P::LG : kGlaSub * P::LG;
+        if (!in) tko[q] = 0;
     }
     // columns of KT this thread fills: block row I, key row j of block J
     constexpr int KSLOTS = (P::NOFF + kGlaThreads - 1) / kGlaThreads;
@@ -259,28 +269,27 @@ gla_chunk_prep_kernel(GlaArgs a) {
                     KT[x * P::LKT + kc[m]] = K0T[x * P::LK0 + kj[m]] * DD[kd[m] * KS + x];
         }
         __syncthreads();
+        // slots past the end of the block lists read row 0 (their sums are never
+        // written); rows past the sequence end hold q = k = 0 and add nothing
+#pragma unroll 1
         for (int x = 0; x < kw; ++x) {
 #pragma unroll
             for (int d = 0; d < DSLOTS; ++d) {
-                if (dv[d]) {
-                    const float2 qg = QG[di[d] * (KS + 1) + x], kg = KG[dj[d] * (KS + 1) + x];
-                    dacc[d] = fmaf(qg.x * kg.x, tc::fast_exp2(qg.y - kg.y), dacc[d]);
-                }
+                const float2 qg = QG[dq_off[d] + x], kg = KG[dk_off[d] + x];
+                dacc[d] = fmaf(qg.x * kg.x, tc::fast_exp2(qg.y - kg.y), dacc[d]);
             }
 #pragma unroll
             for (int q = 0; q < TSLOTS; ++q) {
-                if (tv[q]) {
-                    const float q0 = QH[ti[q] * P::LG + x], q1 = QH[(ti[q] + 1) * P::LG + x];
-                    const float4 k4 = *reinterpret_cast<const float4 *>(KT + x * P::LKT + tko[q]);
-                    oacc[q][0] = fmaf(q0, k4.x, oacc[q][0]);
-                    oacc[q][1] = fmaf(q0, k4.y, oacc[q][1]);
-                    oacc[q][2] = fmaf(q0, k4.z, oacc[q][2]);
-                    oacc[q][3] = fmaf(q0, k4.w, oacc[q][3]);
-                    oacc[q][4] = fmaf(q1, k4.x, oacc[q][4]);
-                    oacc[q][5] = fmaf(q1, k4.y, oacc[q][5]);
-                    oacc[q][6] = fmaf(q1, k4.z, oacc[q][6]);
-                    oacc[q][7] = fmaf(q1, k4.w, oacc[q][7]);
-                }
+                const float q0 = QH[tq_off[q] + x], q1 = QH[tq_off[q] + P::LG + x];
+                const float4 k4 = *reinterpret_cast<const float4 *>(KT + x * P::LKT + tko[q]);
+                oacc[q][0] = fmaf(q0, k4.x, oacc[q][0]);
+                oacc[q][1] = fmaf(q0, k4.y, oacc[q][1]);
+                oacc[q][2] = fmaf(q0, k4.z, oacc[q][2]);
+                oacc[q][3] = fmaf(q0, k4.w, oacc[q][3]);
+                oacc[q][4] = fmaf(q1, k4.x, oacc[q][4]);
+                oacc[q][5] = fmaf(q1, k4.y, oacc[q][5]);
+                oacc[q][6] = fmaf(q1, k4.z, oacc[q][6]);
+                oacc[q][7] = fmaf(q1, k4.w, oacc[q][7]);
             }
         }
     }
