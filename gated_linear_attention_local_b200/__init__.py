@@ -354,7 +354,7 @@ def simple_gla_fused_recurrent(q, k, v, g=None, g_gamma=None, scale=None, initia
     return (o.unsqueeze(0) if squeeze else o), ht
 
 
-def _bwd_prepare(q, k, v, do, g, g_gamma, initial_state, dht, cu_seqlens):
+def _bwd_prepare(q, k, v, do, g, g_gamma, initial_state, dht, cu_seqlens, state_v_first=False):
     """Checks shared by the two backward entry points; returns (N, T, H, K, V) and the
     output tensors."""
     _common_checks(q, k, v, g, g_gamma, initial_state)
@@ -385,9 +385,10 @@ def _bwd_prepare(q, k, v, do, g, g_gamma, initial_state, dht, cu_seqlens):
         raise ValueError("k must match q, and v must match q except in the last dimension")
     if g_gamma is not None and tuple(g_gamma.shape) != (H,):
         raise ValueError(f"g_gamma must be [H] = ({H},)")
+    sshape = (N, H, V, K) if state_v_first else (N, H, K, V)
     for name, t in (("initial_state", initial_state), ("dht", dht)):
-        if t is not None and tuple(t.shape) != (N, H, K, V):
-            raise ValueError(f"{name} must be {(N, H, K, V)}")
+        if t is not None and tuple(t.shape) != sshape:
+            raise ValueError(f"{name} must be {sshape}")
     out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
                dg=torch.zeros_like(g) if g is not None else None,
                dg_gamma=torch.empty_like(g_gamma) if g_gamma is not None else None,
@@ -396,29 +397,31 @@ def _bwd_prepare(q, k, v, do, g, g_gamma, initial_state, dht, cu_seqlens):
 
 
 def simple_gla_fused_recurrent_bwd(q, k, v, do, g=None, g_gamma=None, scale=None, initial_state=None, dht=None,
-                                   cu_seqlens=None, workspace=None):
-    """Gradients of simple_gla_fused_recurrent (state_v_first off) for the loss
+                                   cu_seqlens=None, state_v_first=False, workspace=None):
+    """Gradients of simple_gla_fused_recurrent for the loss
     sum(o * do) + sum(final_state * dht).  Shapes as the forward; do like v; dht like
     the final state or None.  Returns dict(dq, dk, dv, dg, dg_gamma, dh0): dq, dk, dv
     in the dtype and shape of q, k, v; dg like g (None without g); dg_gamma [H] (None
-    without g_gamma); dh0 like initial_state (None without it)."""
-    (N, T, H, K, V), out = _bwd_prepare(q, k, v, do, g, g_gamma, initial_state, dht, cu_seqlens)
+    without g_gamma); dh0 like initial_state (None without it).  state_v_first: the
+    states and their gradients are [N,H,V,K]."""
+    (N, T, H, K, V), out = _bwd_prepare(q, k, v, do, g, g_gamma, initial_state, dht, cu_seqlens, state_v_first)
     nbytes = int(lib().simple_gla_fused_recurrent_bwd_workspace_size(_ptr(cu_seqlens), N, T, H, K))
     ws = _workspace(nbytes, q.device, workspace)
     st = lib().simple_gla_fused_recurrent_bwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma), ctypes.c_float(_scale(scale)), _ptr(initial_state),
         _ptr(do), _ptr(dht), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dg_gamma"]),
-        _ptr(out["dh0"]), _ptr(cu_seqlens), N, T, H, K, V, _DTYPES[q.dtype], _ptr(ws), ws.numel(), _stream())
+        _ptr(out["dh0"]), _ptr(cu_seqlens), N, T, H, K, V, 1 if state_v_first else 0, _DTYPES[q.dtype], _ptr(ws),
+        ws.numel(), _stream())
     raise_for_status(st, "simple_gla_fused_recurrent_bwd")
     return out
 
 
 def simple_gla_chunk_bwd(q, k, v, do, g=None, g_gamma=None, scale=None, initial_state=None, dht=None,
-                         cu_seqlens=None, chunk_size=64, workspace=None):
-    """Gradients of simple_gla_chunk (state_v_first off) on the tensor-core path, for
+                         cu_seqlens=None, chunk_size=64, state_v_first=False, workspace=None):
+    """Gradients of simple_gla_chunk on the tensor-core path, for
     the loss sum(o * do) + sum(final_state * dht).  Arguments and result as
     simple_gla_fused_recurrent_bwd, plus chunk_size."""
-    (N, T, H, K, V), out = _bwd_prepare(q, k, v, do, g, g_gamma, initial_state, dht, cu_seqlens)
+    (N, T, H, K, V), out = _bwd_prepare(q, k, v, do, g, g_gamma, initial_state, dht, cu_seqlens, state_v_first)
     dt = _DTYPES[q.dtype]
     nbytes = int(lib().simple_gla_chunk_bwd_workspace_size(_ptr(cu_seqlens), N, T, H, K, V, chunk_size, dt))
     if nbytes == 0:
@@ -427,7 +430,8 @@ def simple_gla_chunk_bwd(q, k, v, do, g=None, g_gamma=None, scale=None, initial_
     st = lib().simple_gla_chunk_bwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma), ctypes.c_float(_scale(scale)), _ptr(initial_state),
         _ptr(do), _ptr(dht), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dg_gamma"]),
-        _ptr(out["dh0"]), _ptr(cu_seqlens), N, T, H, K, V, chunk_size, dt, _ptr(ws), ws.numel(), _stream())
+        _ptr(out["dh0"]), _ptr(cu_seqlens), N, T, H, K, V, chunk_size, 1 if state_v_first else 0, dt, _ptr(ws),
+        ws.numel(), _stream())
     raise_for_status(st, "simple_gla_chunk_bwd")
     return out
 

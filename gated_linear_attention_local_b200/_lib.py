@@ -47,11 +47,12 @@ _SIG = {
                                     ctypes.c_int, ctypes.c_int, _P, _P], ctypes.c_int),
     "simple_gla_fused_recurrent_bwd_workspace_size": ([_P, _I64, _I64, _I64, _I64], ctypes.c_size_t),
     "simple_gla_fused_recurrent_bwd": ([_P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64,
-                                        _I64, _I64, _I64, ctypes.c_int, _P, ctypes.c_size_t, _P], ctypes.c_int),
+                                        _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, _P, ctypes.c_size_t, _P],
+                                       ctypes.c_int),
     "simple_gla_chunk_bwd_workspace_size": ([_P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int],
                                             ctypes.c_size_t),
     "simple_gla_chunk_bwd": ([_P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64,
-                              _I64, ctypes.c_int, ctypes.c_int, _P, ctypes.c_size_t, _P], ctypes.c_int),
+                              _I64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "gla_chunk_workspace_size": ([_P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int], ctypes.c_size_t),
     "gla_chunk": ([_P, _P, _P, _P, _F, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int, _P,
                    ctypes.c_size_t, _P], ctypes.c_int),

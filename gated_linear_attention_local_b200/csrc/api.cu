@@ -597,8 +597,8 @@ sgla_status simple_gla_chunk_bwd(const void *q, const void *k, const void *v, co
                                  float scale, const float *initial_state, const void *dout, const float *dht,
                                  void *dq, void *dk, void *dv, float *dg, float *dg_gamma, float *dh0,
                                  const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V,
-                                 int chunk_size, sgla_dtype dtype, void *workspace, size_t workspace_bytes,
-                                 void *stream) {
+                                 int chunk_size, int state_v_first, sgla_dtype dtype, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
     const bool varlen = cu_seqlens != nullptr;
     if (g && g_gamma) return SGLA_ERR_INVALID_ARGUMENT;
     if (N < (varlen ? 1 : 0) || T < 0) return SGLA_ERR_INVALID_ARGUMENT;
@@ -643,8 +643,16 @@ sgla_status simple_gla_chunk_bwd(const void *q, const void *k, const void *v, co
     r.s0T = hTT ? s0T : nullptr;
     r.hT = hTT;
     SGLA_LAUNCH("bwd_reverse_inputs", launch_bwd_reverse_inputs(r, st));
-    SGLA_LAUNCH("bwd_state_prep", launch_bwd_state_prep(dht, initial_state, 1.0f / scale, s0, s0T, h0T, N * H,
-                                                        (int)K, (int)V, st));
+    if (state_v_first) {
+        // states arrive [V,K]: dhT / scale is s0T as given and s0 its transpose; the
+        // initial state is already the [V,K] state of the dq call
+        SGLA_LAUNCH("bwd_state_prep", launch_bwd_state_prep(dht, nullptr, 1.0f / scale, s0T, s0, nullptr, N * H,
+                                                            (int)V, (int)K, st));
+        h0T = const_cast<float *>(initial_state);
+    } else {
+        SGLA_LAUNCH("bwd_state_prep", launch_bwd_state_prep(dht, initial_state, 1.0f / scale, s0, s0T, h0T, N * H,
+                                                            (int)K, (int)V, st));
+    }
     sgla_status rs;
     // call A: dv on the reversed sequence, state [K,V] = dS / scale
     rs = run_forward(varlen, r.kr, r.qr, r.dor, r.gr, nullptr, scale, cu_seqlens, N, T, s0, dvr, xf, H, K, V,
@@ -659,7 +667,12 @@ sgla_status simple_gla_chunk_bwd(const void *q, const void *k, const void *v, co
                      dtype, workspace, L.inner, stream, false, true);
     if (rs != SGLA_OK) return rs;
     SGLA_LAUNCH("bwd_unreverse", launch_bwd_unreverse(r, st));
+    // dh0 in [V,K]: the scan writes it [K,V] into the s0 buffer (no longer read), then
+    // a transpose puts it in place
+    if (state_v_first && dh0) r.dh0 = reinterpret_cast<float *>(ws + L.off_s0);
     if (want_dg || dh0) SGLA_LAUNCH("bwd_gate_scan", launch_bwd_gate_scan(r, st));
+    if (state_v_first && dh0)
+        SGLA_LAUNCH("state_transpose", launch_state_transpose(r.dh0, dh0, N * H, (int)K, (int)V, st));
     return SGLA_OK;
 }
 
@@ -674,8 +687,9 @@ sgla_status simple_gla_fused_recurrent_bwd(const void *q, const void *k, const v
                                            const float *g_gamma, float scale, const float *initial_state,
                                            const void *dout, const float *dht, void *dq, void *dk, void *dv,
                                            float *dg, float *dg_gamma, float *dh0, const int64_t *cu_seqlens,
-                                           int64_t N, int64_t T, int64_t H, int64_t K, int64_t V, sgla_dtype dtype,
-                                           void *workspace, size_t workspace_bytes, void *stream) {
+                                           int64_t N, int64_t T, int64_t H, int64_t K, int64_t V,
+                                           int state_v_first, sgla_dtype dtype, void *workspace,
+                                           size_t workspace_bytes, void *stream) {
     if (g && g_gamma) return SGLA_ERR_INVALID_ARGUMENT;
     if (N < 0 || T < 0 || H < 1 || K < 1 || V < 1) return SGLA_ERR_INVALID_ARGUMENT;
     if (cu_seqlens && N < 1) return SGLA_ERR_INVALID_ARGUMENT;
@@ -711,7 +725,7 @@ sgla_status simple_gla_fused_recurrent_bwd(const void *q, const void *k, const v
     a.ddot = reinterpret_cast<float *>(ws + 2 * acc);
     a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dg_gamma = dg_gamma; a.dh0 = dh0; a.cu = cu_seqlens;
     a.N = N; a.T_dense = cu_seqlens ? 0 : T; a.T_total = tokens;
-    a.H = (int)H; a.K = (int)K; a.V = (int)V; a.bf16 = dtype == SGLA_BF16;
+    a.H = (int)H; a.K = (int)K; a.V = (int)V; a.bf16 = dtype == SGLA_BF16; a.vfirst = state_v_first != 0;
     SGLA_LAUNCH("recurrent_bwd_forward_sweep", launch_rec_bwd(a, 0, st));
     SGLA_LAUNCH("recurrent_bwd_reverse_sweep", launch_rec_bwd(a, 1, st));
     SGLA_LAUNCH("recurrent_bwd_finalize", launch_rec_bwd(a, 2, st));

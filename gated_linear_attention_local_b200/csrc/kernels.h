@@ -78,6 +78,7 @@ struct RecBwdArgs {
     int64_t N, T_dense, T_total;
     int H, K, V;
     bool bf16;
+    bool vfirst;        // h0, dhT, dh0 stored [N, H, V, K] (state_v_first)
 };
 // Chunked GLA with a gate vector over K (gla_chunk.cu).
 struct GlaArgs {

@@ -41,6 +41,12 @@ __device__ __forceinline__ float reduce_scatter32(float (&p)[32], int lane) {
     return p[0];
 }
 
+// Offset of element (row r of K, column c of V) of one state: [K,V] layout, or the
+// transposed [V,K] one (state_v_first).
+__device__ __forceinline__ int64_t st_off(int r, int c, int K, int V, bool vfirst) {
+    return vfirst ? (int64_t)c * K + r : (int64_t)r * V + c;
+}
+
 struct SeqSpan {
     int64_t bos, eos;
     bool ok;
@@ -73,7 +79,7 @@ rec_bwd_forward_kernel(const T *__restrict__ k, const T *__restrict__ v, const T
                        const float *__restrict__ g, const float *__restrict__ g_gamma, float scale,
                        const float *__restrict__ h0, const float *__restrict__ dhT, float *__restrict__ dqf,
                        float *__restrict__ ddot, const int64_t *__restrict__ cu, int64_t T_dense, int64_t T_total,
-                       int H, int K, int V) {
+                       int H, int K, int V, bool vfirst) {
     extern __shared__ float4 bsm4[];
     float *sm = reinterpret_cast<float *>(bsm4);
     const int nthr = blockDim.x, nwarps = nthr >> 5, kpad = nwarps * 32;
@@ -95,8 +101,8 @@ rec_bwd_forward_kernel(const T *__restrict__ k, const T *__restrict__ v, const T
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         const int r = r0 + j;
-        sa[j] = (h0 && r < K && has_a) ? h0[sbase + (int64_t)r * V + c0 + ca] : 0.f;
-        sb[j] = (h0 && r < K && has_b) ? h0[sbase + (int64_t)r * V + c0 + cb] : 0.f;
+        sa[j] = (h0 && r < K && has_a) ? h0[sbase + st_off(r, c0 + ca, K, V, vfirst)] : 0.f;
+        sb[j] = (h0 && r < K && has_b) ? h0[sbase + st_off(r, c0 + cb, K, V, vfirst)] : 0.f;
     }
     for (int64_t tb = sp.bos; tb < sp.eos; tb += kBTB) {
         const int nt = (int)min64(kBTB, sp.eos - tb);
@@ -135,8 +141,8 @@ rec_bwd_forward_kernel(const T *__restrict__ k, const T *__restrict__ v, const T
         for (int j = 0; j < 32; ++j) {
             const int r = r0 + j;
             if (r < K) {
-                if (has_a) acc = fmaf(dhT[sbase + (int64_t)r * V + c0 + ca], sa[j], acc);
-                if (has_b) acc = fmaf(dhT[sbase + (int64_t)r * V + c0 + cb], sb[j], acc);
+                if (has_a) acc = fmaf(dhT[sbase + st_off(r, c0 + ca, K, V, vfirst)], sa[j], acc);
+                if (has_b) acc = fmaf(dhT[sbase + st_off(r, c0 + cb, K, V, vfirst)], sb[j], acc);
             }
         }
 #pragma unroll
@@ -158,7 +164,7 @@ rec_bwd_reverse_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
                        const T *__restrict__ dout, const float *__restrict__ g, const float *__restrict__ g_gamma,
                        float scale, const float *__restrict__ dhT, float *__restrict__ dkf, T *__restrict__ dv,
                        float *__restrict__ dh0, const int64_t *__restrict__ cu, int64_t T_dense, int64_t T_total,
-                       int H, int K, int V) {
+                       int H, int K, int V, bool vfirst) {
     extern __shared__ float4 bsm4[];
     float *sm = reinterpret_cast<float *>(bsm4);
     const int nthr = blockDim.x, nwarps = nthr >> 5, kpad = nwarps * 32;
@@ -181,8 +187,8 @@ rec_bwd_reverse_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         const int r = r0 + j;
-        xa[j] = (dhT && r < K && has_a) ? dhT[sbase + (int64_t)r * V + c0 + ca] : 0.f;
-        xb[j] = (dhT && r < K && has_b) ? dhT[sbase + (int64_t)r * V + c0 + cb] : 0.f;
+        xa[j] = (dhT && r < K && has_a) ? dhT[sbase + st_off(r, c0 + ca, K, V, vfirst)] : 0.f;
+        xb[j] = (dhT && r < K && has_b) ? dhT[sbase + st_off(r, c0 + cb, K, V, vfirst)] : 0.f;
     }
     // blocks from the end: block tokens [tb, tb + nt), processed from tb + nt - 1 down
     for (int64_t te = sp.eos; te > sp.bos; te -= kBTB) {
@@ -242,8 +248,8 @@ rec_bwd_reverse_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
         for (int j = 0; j < 32; ++j) {
             const int r = r0 + j;
             if (r < K) {
-                if (has_a) dh0[sbase + (int64_t)r * V + c0 + ca] = a0 * xa[j];
-                if (has_b) dh0[sbase + (int64_t)r * V + c0 + cb] = a0 * xb[j];
+                if (has_a) dh0[sbase + st_off(r, c0 + ca, K, V, vfirst)] = a0 * xa[j];
+                if (has_b) dh0[sbase + st_off(r, c0 + cb, K, V, vfirst)] = a0 * xb[j];
             }
         }
     }
@@ -340,7 +346,7 @@ cudaError_t rec_bwd_part(const RecBwdArgs &a, int part, cudaStream_t st) {
             return e;
         rec_bwd_forward_kernel<T><<<grid, 32 * warps, sm, st>>>(
             (const T *)a.k, (const T *)a.v, (const T *)a.dout, a.g, a.g_gamma, a.scale, a.h0, a.dhT, a.dqf, a.ddot,
-            a.cu, a.T_dense, a.T_total, a.H, a.K, a.V);
+            a.cu, a.T_dense, a.T_total, a.H, a.K, a.V, a.vfirst);
     } else if (part == 1) {
         const size_t sm = sizeof(float) * (2 * (size_t)kBTB * kpad + 2 * (size_t)kBTB * kBCols + kBTB +
                                            (size_t)kBTB * warps * kBCols);
@@ -349,7 +355,7 @@ cudaError_t rec_bwd_part(const RecBwdArgs &a, int part, cudaStream_t st) {
             return e;
         rec_bwd_reverse_kernel<T><<<grid, 32 * warps, sm, st>>>(
             (const T *)a.q, (const T *)a.k, (const T *)a.v, (const T *)a.dout, a.g, a.g_gamma, a.scale, a.dhT,
-            a.dkf, (T *)a.dv, a.dh0, a.cu, a.T_dense, a.T_total, a.H, a.K, a.V);
+            a.dkf, (T *)a.dv, a.dh0, a.cu, a.T_dense, a.T_total, a.H, a.K, a.V, a.vfirst);
     } else {
         rec_bwd_finalize_kernel<T><<<(unsigned)(a.N * a.H), 256, 0, st>>>(
             (const T *)a.q, (const T *)a.k, a.dqf, a.dkf, a.dhT ? a.ddot : nullptr, (T *)a.dq, (T *)a.dk, a.dg,

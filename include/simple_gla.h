@@ -204,7 +204,9 @@ SGLA_API sgla_status simple_gla_fused_recurrent(const void *q, const void *k, co
  *   dh0 [N,H,K,V] fp32 = dL/d initial_state (only with initial_state; NULL to skip).
  * Inputs: q, k, v, g, g_gamma, scale, initial_state, cu_seqlens, N, T, H, K, V, dtype
  * as simple_gla_fused_recurrent; dout [tokens,H,V] dtype; dht [N,H,K,V] fp32 or NULL
- * (zero).  A packed sequence whose bounds are not 0 <= start <= end <= T is skipped
+ * (zero).  state_v_first != 0 stores initial_state, dht and dh0 as [N,H,V,K] (the
+ * transposed layout of article section 2, whose section 5 checks the gradients of
+ * both layouts against each other).  A packed sequence whose bounds are not 0 <= start <= end <= T is skipped
  * (its gradients are not written); tokens outside every sequence are not written.
  * Supported sizes: 1 <= K <= 512, 1 <= V <= 4096; pointers aligned to their element
  * size.  workspace: at least simple_gla_fused_recurrent_bwd_workspace_size() bytes,
@@ -219,8 +221,9 @@ SGLA_API sgla_status simple_gla_fused_recurrent_bwd(const void *q, const void *k
                                                     const float *dht, void *dq, void *dk, void *dv,
                                                     float *dg, float *dg_gamma, float *dh0,
                                                     const int64_t *cu_seqlens, int64_t N, int64_t T,
-                                                    int64_t H, int64_t K, int64_t V, sgla_dtype dtype,
-                                                    void *workspace, size_t workspace_bytes, void *stream);
+                                                    int64_t H, int64_t K, int64_t V, int state_v_first,
+                                                    sgla_dtype dtype, void *workspace, size_t workspace_bytes,
+                                                    void *stream);
 
 /*
  * Gradients of the chunked forward (simple_gla_chunk with state_v_first = 0) on the
@@ -233,7 +236,8 @@ SGLA_API sgla_status simple_gla_fused_recurrent_bwd(const void *q, const void *k
  * one; dq: query do, key v, value k in token order), plus three row kernels.
  *
  * Outputs, loss, inputs and the packed / dense conventions are those of
- * simple_gla_fused_recurrent_bwd; chunk_size as simple_gla_chunk.  Sizes as the
+ * simple_gla_fused_recurrent_bwd (state_v_first included); chunk_size as
+ * simple_gla_chunk.  Sizes as the
  * chunked forward with K and V exchanged as well (both multiples of 8, at most 512);
  * q, k, v, dout, dq, dk, dv, initial_state, dht and dh0 16-byte aligned.  workspace:
  * at least simple_gla_chunk_bwd_workspace_size() bytes, 256-byte aligned, contents
@@ -247,8 +251,8 @@ SGLA_API sgla_status simple_gla_chunk_bwd(const void *q, const void *k, const vo
                                           const void *dout, const float *dht, void *dq, void *dk, void *dv,
                                           float *dg, float *dg_gamma, float *dh0, const int64_t *cu_seqlens,
                                           int64_t N, int64_t T, int64_t H, int64_t K, int64_t V, int chunk_size,
-                                          sgla_dtype dtype, void *workspace, size_t workspace_bytes,
-                                          void *stream);
+                                          int state_v_first, sgla_dtype dtype, void *workspace,
+                                          size_t workspace_bytes, void *stream);
 
 /*
  * The chunked forward with every option of chunk_simple_gla (article section 2) in

@@ -138,7 +138,7 @@ def test_fused_recurrent_bwd_validation_on_the_host(lib):
 
     def call(q=FAKE, g=None, gg=None, h0=None, dht=None, dg=None, dgg=None, dh0=None, cu=None, N=4, T=8, H=2,
              K=64, V=64, dt=L.SGLA_BF16, ws=FAKE, nws=None):
-        return f(q, FAKE, FAKE, g, gg, 1.0, h0, FAKE, dht, FAKE, FAKE, FAKE, dg, dgg, dh0, cu, N, T, H, K, V, dt, ws,
+        return f(q, FAKE, FAKE, g, gg, 1.0, h0, FAKE, dht, FAKE, FAKE, FAKE, dg, dgg, dh0, cu, N, T, H, K, V, 0, dt, ws,
                  ws_need if nws is None else nws, None)
 
     assert call(g=FAKE, gg=FAKE) == L.SGLA_ERR_INVALID_ARGUMENT       # both gates

@@ -116,3 +116,22 @@ def test_chunk_bwd_training_batch_sampled():
     for name in ("dq", "dk", "dv", "dh0"):
         a, b = host(gpu[name]), host(rec[name])
         assert abs(a - b).max() <= 2e-2 * abs(b).max(), name
+
+
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float32])
+def test_simple_gla_chunk_bwd_state_v_first(dt):
+    """States and their gradients in the [V,K] layout (the article's section 2
+    state_v_first; section 5 checks both layouts' gradients against each other): the
+    oracle runs on the transposed [K,V] states and its dh0 is transposed back."""
+    N, T, H, K, V = 2, 150, 2, 128, 64
+    inp = random_inputs(N, T, H, K, V, dtype=dt, gate="g", h0=True, seed=71)
+    do, dh = random_cotangents(inp["v"].shape, N, H, K, V, dtype=dt, seed=72)
+    h0_vk, dh_vk = inp["h0"].transpose(-1, -2).contiguous(), dh.transpose(-1, -2).contiguous()
+    dev = {k: to_dev(v) for k, v in inp.items()}
+    gpu = sg.simple_gla_chunk_bwd(dev["q"], dev["k"], dev["v"], to_dev(do), g=dev["g"], initial_state=to_dev(h0_vk),
+             dht=to_dev(dh_vk), state_v_first=True)
+    torch.cuda.synchronize()
+    assert tuple(gpu["dh0"].shape) == (N, H, V, K)
+    gpu["dh0"] = gpu["dh0"].transpose(-1, -2)
+    ref = oracle.simple_gla_bwd(inp["q"], inp["k"], inp["v"], do, g=inp["g"], initial_state=inp["h0"], dht=dh)
+    compare_grads(gpu, ref, TOL[dt], inp)
