@@ -11,6 +11,8 @@
 // One CTA per (sequence, head, 64-wide V tile), 192 threads: warps 0-3 own TMEM lanes
 // 0-127 (output row i and state row k = i), warp 4 lane 0 issues the TMA copies,
 // warp 5 lane 0 the MMAs.  TMEM: O in columns 0-63, H (fp32, 128 x 64) in 64-127.
+// Per step the state product is issued first and the output products behind it, so
+// the threads' state pass for the next step overlaps this step's output products.
 // Every wait is bounded; a CTA that gives up drains its copies and products, frees
 // its TMEM and records a time-out in the workspace status word.
 #include <cudaTypedefs.h>
@@ -34,8 +36,8 @@ constexpr uint32_t K = 2 * kReg;
 constexpr uint32_t V = 4 * kReg;
 constexpr uint32_t STAGE = 5 * kReg;
 constexpr uint32_t A = 2 * STAGE;       // scores (2 regions), one buffer
-constexpr uint32_t HB = A + 2 * kReg;   // bf16 state, 128 rows (k) x 64 (v), MN-major
-constexpr uint32_t BARS = HB + kReg;
+constexpr uint32_t HB = A + 2 * kReg;   // 2 x bf16 state, 128 rows (k) x 64 (v), MN-major
+constexpr uint32_t BARS = HB + 2 * kReg;
 constexpr uint32_t MISC = BARS + 16 * 8;
 constexpr uint32_t TOTAL = MISC + 16;
 }  // namespace gt
@@ -168,15 +170,24 @@ gla_tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
             const uint32_t idH = idesc_bf16_f32(128, 64, true, true);
             const uint32_t sbase = smem_u32(sm);
             const uint32_t tO = tmem, tH = tmem + 64;
+            // The state product of a step goes first: the next step waits only on it (and
+            // on the threads' state pass), while the output products of this step run
+            // behind it and overlap that pass.  Hb is double-buffered by step parity.
             for (int t = 0; t < nsteps; ++t) {
                 const int st = t & 1;
                 if (!mbar_wait(&full[st], (t >> 1) & 1, abort_flag)) break;
-                if (!mbar_wait(full_a, t & 1, abort_flag)) break;
                 if (!mbar_wait(b_hb, t & 1, abort_flag)) break;
-                if (t >= 1 && !mbar_wait(o_free, (t - 1) & 1, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t q = sbase + st * gt::STAGE + gt::Q, k = sbase + st * gt::STAGE + gt::K;
-                const uint32_t v = sbase + st * gt::STAGE + gt::V, s = sbase + gt::A, hb = sbase + gt::HB;
+                const uint32_t v = sbase + st * gt::STAGE + gt::V, s = sbase + gt::A;
+                const uint32_t hb = sbase + gt::HB + st * kReg;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tH, desc(k + kk * 2048, kReg, 1024), mnmaj(v + kk * 2048), idH, 1u);
+                mma_commit(h_ready);
+                if (!mbar_wait(full_a, t & 1, abort_flag)) break;
+                if (t >= 1 && !mbar_wait(o_free, (t - 1) & 1, abort_flag)) break;
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * kReg + (kk & 3) * 32;
@@ -188,10 +199,6 @@ gla_tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                     mma_bf16(tO, kmaj(s + off), mnmaj(v + kk * 2048), idO, 1u);
                 }
                 mma_commit(o_ready);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tH, desc(k + kk * 2048, kReg, 1024), mnmaj(v + kk * 2048), idH, 1u);
-                mma_commit(h_ready);
                 mma_commit(&empty[st]);
             }
             mma_commit(b_done);
@@ -247,6 +254,43 @@ gla_tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
         for (int t = 0; ok && t < nsteps; ++t) {
             const int64_t ta = t0 + (int64_t)t * kTcStep;
             const int len = (int)min64(kTcStep, t1 - ta);
+            // state: Hb of the next step <- bf16(H); H <- decay of the next chunk; or the
+            // final state.  Hb[(t+1) & 1] was last read by the products of step t-1,
+            // which retired before this thread read step t-1's output.
+            if (!mbar_wait(h_ready, t & 1, abort_flag)) break;
+            tc_fence_after();
+            if (t + 1 < nsteps) {
+                const float d = decay(t + 1);
+                unsigned char *hbn = hb + ((t + 1) & 1) * kReg;
+#pragma unroll 1
+                for (int pc = 0; pc < 2; ++pc) {
+                    float x[32];
+                    tmem_ld32(trow + 64 + 32 * pc, x);
+                    tmem_wait_ld();
+                    store_row32(hbn, i, 32 * pc, x);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[e] *= d;
+                    tmem_st32(trow + 64 + 32 * pc, x);
+                }
+                tmem_wait_st();
+                ok = zero_tail(t + 1);
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(b_hb);
+            } else if (a.hT) {
+#pragma unroll 1
+                for (int pc = 0; pc < 2; ++pc) {
+                    float x[32];
+                    tmem_ld32(trow + 64 + 32 * pc, x);
+                    tmem_wait_ld();
+                    if (!*abort_flag) {
+                        float4 *d4 = reinterpret_cast<float4 *>(a.hT + sbase + 32 * pc);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            d4[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+                    }
+                }
+            }
             // output rows
             if (!mbar_wait(o_ready, t & 1, abort_flag)) break;
             tc_fence_after();
@@ -271,40 +315,6 @@ gla_tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
                                           pack2(a.scale * o1[8 * q + 2], a.scale * o1[8 * q + 3]),
                                           pack2(a.scale * o1[8 * q + 4], a.scale * o1[8 * q + 5]),
                                           pack2(a.scale * o1[8 * q + 6], a.scale * o1[8 * q + 7]));
-            }
-            // state: Hb <- bf16(H); H <- decay of the next chunk; or the final state
-            if (!mbar_wait(h_ready, t & 1, abort_flag)) break;
-            tc_fence_after();
-            if (t + 1 < nsteps) {
-                const float d = decay(t + 1);
-#pragma unroll 1
-                for (int pc = 0; pc < 2; ++pc) {
-                    float x[32];
-                    tmem_ld32(trow + 64 + 32 * pc, x);
-                    tmem_wait_ld();
-                    store_row32(hb, i, 32 * pc, x);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] *= d;
-                    tmem_st32(trow + 64 + 32 * pc, x);
-                }
-                tmem_wait_st();
-                ok = zero_tail(t + 1);
-                fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive(b_hb);
-            } else if (a.hT) {
-#pragma unroll 1
-                for (int pc = 0; pc < 2; ++pc) {
-                    float x[32];
-                    tmem_ld32(trow + 64 + 32 * pc, x);
-                    tmem_wait_ld();
-                    if (!*abort_flag) {
-                        float4 *d4 = reinterpret_cast<float4 *>(a.hT + sbase + 32 * pc);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            d4[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
-                    }
-                }
             }
         }
         if (nsteps == 0 && a.hT) {  // empty sequence: the final state is the initial one
