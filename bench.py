@@ -595,7 +595,9 @@ def _config_of(w):
         return dict(entry="simple_gla_normalized", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
                     gate="g" if w["g"] is not None else "none", feature_map="|x|+0.1", scale=1.0)
     if w.get("entry") == "gla_chunk":
-        return dict(entry="gla_chunk", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"], chunk=32, sub_chunk=16,
+        tc = w["q"].dtype == torch.bfloat16 and w["K"] == 128 and w["V"] % 64 == 0
+        return dict(entry="gla_chunk", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"], chunk=128 if tc else 32,
+                    sub_chunk=16, walk="tcgen05" if tc else "CUDA cores",
                     gate="gk [B,T,H,K] = logsigmoid(N(0,1))/16", initial_state=True)
     if w.get("entry") == "gla":
         return dict(entry="gla_fused_recurrent", B=w["B"], T=w["T"], H=w["H"], K=w["K"], V=w["V"],
