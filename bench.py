@@ -85,10 +85,9 @@ def algorithmic_counts(w):
             # three chunked forward calls (dv, dk, dq); the output walk of each moves
             # that call's compulsory bytes
             return dict(bytes=b, flops=3 * flops, tokens=tokens, kernel={"chunk_output_tc": fwd})
-        # token-serial FLOPs per token and head: forward sweep 4KV (state update, dq),
-        # reverse sweep 6KV (dS update, dk, dv)
-        kernel = {"recurrent_bwd_forward_sweep": dict(bytes=b, flops=H * tokens * 4 * K * V),
-                  "recurrent_bwd_reverse_sweep": dict(bytes=b, flops=H * tokens * 6 * K * V)}
+        # token-serial FLOPs per token and head: forward sweep 4KV (state update, dq)
+        # and reverse sweep 6KV (dS update, dk, dv), one launch
+        kernel = {"recurrent_bwd_sweeps": dict(bytes=b, flops=H * tokens * 10 * K * V)}
         return dict(bytes=b, flops=H * tokens * 10 * K * V, tokens=tokens, kernel=kernel)
     return dict(bytes=b, flops=flops, tokens=tokens)
 
@@ -114,8 +113,8 @@ KERNEL_SOURCES = {
     "decode_step": ["decode.cu"],
     "fused_recurrent": ["recurrent.cu"],
     "gla_fused_recurrent": ["recurrent.cu"],
-    "recurrent_bwd_reverse_sweep": ["recurrent_bwd.cu"],
-    "recurrent_bwd_forward_sweep": ["recurrent_bwd.cu"],
+    "recurrent_bwd_sweeps": ["recurrent_bwd.cu"],
+    "recurrent_bwd_rows": ["recurrent_bwd.cu"],
     "gla_chunk_prep": ["gla_chunk.cu", "tc_ptx.cuh"],
     "bwd_reverse_inputs": ["chunk_bwd.cu"],
     "gla_chunk_walk_tc": ["gla_chunk_tc.cu", "tc_ptx.cuh", "tc_path.h"],

@@ -680,7 +680,8 @@ size_t simple_gla_fused_recurrent_bwd_workspace_size(const int64_t *cu_seqlens, 
                                                      int64_t K) {
     if (N < 0 || T < 0 || H < 1 || K < 1) return 0;
     const int64_t tokens = cu_seqlens ? T : N * T;
-    return 2 * align_up(sizeof(float) * (size_t)tokens * H * K, 256) + align_up(sizeof(float) * (size_t)N * H, 256);
+    return 2 * align_up(sizeof(float) * (size_t)tokens * H * K, 256) + align_up(sizeof(float) * (size_t)N * H, 256) +
+           align_up(sizeof(float) * (size_t)tokens * H, 256);
 }
 
 sgla_status simple_gla_fused_recurrent_bwd(const void *q, const void *k, const void *v, const float *g,
@@ -723,12 +724,13 @@ sgla_status simple_gla_fused_recurrent_bwd(const void *q, const void *k, const v
     a.h0 = initial_state; a.dhT = dht;
     a.dqf = reinterpret_cast<float *>(ws); a.dkf = reinterpret_cast<float *>(ws + acc);
     a.ddot = reinterpret_cast<float *>(ws + 2 * acc);
+    a.x = reinterpret_cast<float *>(ws + 2 * acc + align_up(sizeof(float) * (size_t)N * H, 256));
     a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dg_gamma = dg_gamma; a.dh0 = dh0; a.cu = cu_seqlens;
     a.N = N; a.T_dense = cu_seqlens ? 0 : T; a.T_total = tokens;
     a.H = (int)H; a.K = (int)K; a.V = (int)V; a.bf16 = dtype == SGLA_BF16; a.vfirst = state_v_first != 0;
-    SGLA_LAUNCH("recurrent_bwd_forward_sweep", launch_rec_bwd(a, 0, st));
-    SGLA_LAUNCH("recurrent_bwd_reverse_sweep", launch_rec_bwd(a, 1, st));
-    SGLA_LAUNCH("recurrent_bwd_finalize", launch_rec_bwd(a, 2, st));
+    SGLA_LAUNCH("recurrent_bwd_sweeps", launch_rec_bwd(a, 0, st));
+    SGLA_LAUNCH("recurrent_bwd_rows", launch_rec_bwd(a, 1, st));
+    SGLA_LAUNCH("recurrent_bwd_scan", launch_rec_bwd(a, 2, st));
     return SGLA_OK;
 }
 

@@ -70,6 +70,7 @@ struct RecBwdArgs {
     const float *h0, *dhT;
     float *dqf, *dkf;   // [tokens, H, K] fp32 accumulators, zeroed by the caller
     float *ddot;        // [N, H] <dhT, hT>, zeroed by the caller (used when dhT)
+    float *x;           // [tokens, H] q . dq - k . dk (workspace)
     void *dq, *dk, *dv;
     float *dg;          // [tokens, H] or NULL
     float *dg_gamma;    // [H], zeroed by the caller, or NULL
@@ -128,7 +129,8 @@ cudaError_t launch_bwd_gate_scan(const BwdRowArgs &a, cudaStream_t st);
 cudaError_t launch_bwd_state_prep(const float *dhT, const float *h0, float inv_scale, float *s0, float *s0T,
                                   float *h0T, int64_t mats, int K, int V, cudaStream_t st);
 
-// part 0: forward sweep (dq, <dhT, hT>); 1: reverse sweep (dv, dk, dh0); 2: finalize (casts, dg)
+// part 0: both sweeps in one launch (dq, <dhT, hT>; dv, dk, dh0); 1: row pass (casts,
+// q . dq - k . dk); 2: reverse scan for dg
 cudaError_t launch_rec_bwd(const RecBwdArgs &a, int part, cudaStream_t st);
 
 // Normalised variant through the augmented value: widen v with a ones column (zero

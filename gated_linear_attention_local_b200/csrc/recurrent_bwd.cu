@@ -8,15 +8,19 @@
 //   dS_t = scale q_t do_t^T + a_{t+1} dS_{t+1}   (the last token also receives dhT)
 //   dk_t = dS_t v_t,   dv_t = dS_t^T k_t,   dh0 = a_first dS_first
 //   dg_t = sum_{i >= t} (q_i . dq_i - k_i . dk_i) + <dhT, S_T>   (S_T = final state)
-// Three kernels:
-//   forward sweep: S in registers token by token, dq partials per V tile (added
+// Three launches:
+//   the sweeps (one grid, half its CTAs each):
+//     forward sweep: S in registers token by token, dq partials per V tile (added
 //       across the V tiles with atomics into an fp32 buffer), <dhT, S_T> per head;
-//   reverse sweep: dS in registers from the last token back, dv complete per V tile,
-//       dk partials (atomics), dh0;
-//   finalize: dq, dk to the operand dtype and dg by a reverse scan per sequence.
+//     reverse sweep: dS in registers from the last token back, dv complete per V
+//       tile, dk partials (atomics), dh0;
+//   finalize: a row pass (dq, dk to the operand dtype and q . dq - k . dk per row)
+//     and a reverse scan per sequence for dg.
 // The thread layout of both sweeps is the one of the forward recurrence: one CTA per
 // (sequence, head, 64-column V tile), warp w holds rows 32w .. 32w+31, lane l columns
 // 2l, 2l+1; tokens are staged in blocks of 8 in shared memory as fp32.
+#include <algorithm>
+
 #include "kernels.h"
 
 namespace sgla {
@@ -74,8 +78,7 @@ __device__ __forceinline__ float gate_at(const float *g, const float *g_gamma, i
 
 // ---------------------------------------------------------------- forward sweep
 template <typename T>
-__global__ void __launch_bounds__(512)
-rec_bwd_forward_kernel(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ dout,
+__device__ __forceinline__ void rec_bwd_forward_body(const T *__restrict__ k, const T *__restrict__ v, const T *__restrict__ dout,
                        const float *__restrict__ g, const float *__restrict__ g_gamma, float scale,
                        const float *__restrict__ h0, const float *__restrict__ dhT, float *__restrict__ dqf,
                        float *__restrict__ ddot, const int64_t *__restrict__ cu, int64_t T_dense, int64_t T_total,
@@ -159,8 +162,7 @@ rec_bwd_forward_kernel(const T *__restrict__ k, const T *__restrict__ v, const T
 
 // ---------------------------------------------------------------- reverse sweep
 template <typename T>
-__global__ void __launch_bounds__(512)
-rec_bwd_reverse_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+__device__ __forceinline__ void rec_bwd_reverse_body(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                        const T *__restrict__ dout, const float *__restrict__ g, const float *__restrict__ g_gamma,
                        float scale, const float *__restrict__ dhT, float *__restrict__ dkf, T *__restrict__ dv,
                        float *__restrict__ dh0, const int64_t *__restrict__ cu, int64_t T_dense, int64_t T_total,
@@ -255,18 +257,71 @@ rec_bwd_reverse_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
     }
 }
 
+// The two sweeps are independent (each reads only the inputs), so one launch runs
+// both: blockIdx.z = 0 the forward sweep, 1 the reverse sweep -- twice the CTAs in
+// flight for the same grid of (sequence, head, V tile).
+template <typename T>
+__global__ void __launch_bounds__(512)
+rec_bwd_sweeps_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                      const T *__restrict__ dout, const float *__restrict__ g, const float *__restrict__ g_gamma,
+                      float scale, const float *__restrict__ h0, const float *__restrict__ dhT,
+                      float *__restrict__ dqf, float *__restrict__ ddot, float *__restrict__ dkf, T *__restrict__ dv,
+                      float *__restrict__ dh0, const int64_t *__restrict__ cu, int64_t T_dense, int64_t T_total,
+                      int H, int K, int V, bool vfirst) {
+    if (blockIdx.z == 0)
+        rec_bwd_forward_body<T>(k, v, dout, g, g_gamma, scale, h0, dhT, dqf, ddot, cu, T_dense, T_total, H, K, V,
+                                vfirst);
+    else
+        rec_bwd_reverse_body<T>(q, k, v, dout, g, g_gamma, scale, dhT, dkf, dv, dh0, cu, T_dense, T_total, H, K, V,
+                                vfirst);
+}
+
 // ---------------------------------------------------------------- finalize
-// One CTA of 256 threads per (sequence, head): dq and dk to the operand dtype, and
-// dg_t = sum_{i >= t} (q_i . dq_i - k_i . dk_i) (+ <dhT, S_T>) by a reverse scan in
-// chunks of 256 tokens (a warp per token for the dot products); dg_gamma sums dg over
-// tokens and sequences.
+// Rows: a warp per (token, head) row casts dq and dk to the operand dtype and forms
+// x = q . dq - k . dk from the fp32 sums; rows outside every well-formed sequence are
+// left alone.  Scan: one CTA of 256 threads per (sequence, head) turns x into
+// dg_t = sum_{i >= t} x_i (+ <dhT, S_T>) by a reverse scan in chunks of 256 tokens;
+// dg_gamma sums dg over tokens and sequences.
+__device__ __forceinline__ bool token_in_sequence(int64_t t, const int64_t *cu, int64_t N, int64_t T_total) {
+    if (!cu) return true;
+    int64_t lo = 0, hi = N - 1;
+    while (lo < hi) {  // last sequence whose start is <= t
+        const int64_t mid = (lo + hi + 1) >> 1;
+        if (cu[mid] <= t) lo = mid;
+        else hi = mid - 1;
+    }
+    const int64_t bos = cu[lo], eos = cu[lo + 1];
+    return bos >= 0 && bos <= t && t < eos && eos <= T_total;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256)
-rec_bwd_finalize_kernel(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ dqf,
-                        const float *__restrict__ dkf, const float *__restrict__ ddot, T *__restrict__ dq,
-                        T *__restrict__ dk, float *__restrict__ dg, float *__restrict__ dg_gamma,
-                        const int64_t *__restrict__ cu, int64_t T_dense, int64_t T_total, int H, int K) {
-    __shared__ float xs[256];
+rec_bwd_rows_kernel(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ dqf,
+                    const float *__restrict__ dkf, T *__restrict__ dq, T *__restrict__ dk, float *__restrict__ x,
+                    const int64_t *__restrict__ cu, int64_t N, int64_t T_total, int H, int K) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t row = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); row < T_total * H;
+         row += warps) {
+        if (!token_in_sequence(row / H, cu, N, T_total)) continue;
+        const int64_t off = row * K;
+        float acc = 0.f;
+        for (int r = lane; r < K; r += 32) {
+            const float a = dqf[off + r], b = dkf[off + r];
+            acc = fmaf(to_f32(q[off + r]), a, fmaf(-to_f32(k[off + r]), b, acc));
+            dq[off + r] = from_f32<T>(a);
+            dk[off + r] = from_f32<T>(b);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (x && lane == 0) x[row] = acc;
+    }
+}
+
+__global__ void __launch_bounds__(256)
+rec_bwd_scan_kernel(const float *__restrict__ x, const float *__restrict__ ddot, float *__restrict__ dg,
+                    float *__restrict__ dg_gamma, const int64_t *__restrict__ cu, int64_t T_dense, int64_t T_total,
+                    int H) {
     __shared__ float wtot[8];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t n = blockIdx.x / H;
@@ -274,31 +329,12 @@ rec_bwd_finalize_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
     const SeqSpan sp = span_of(cu, n, T_dense, T_total);
     if (!sp.ok) return;
     const int64_t len = sp.eos - sp.bos;
-    for (int64_t e = tid; e < len * K; e += 256) {
-        const int64_t t = sp.bos + e / K;
-        const int64_t off = (t * H + h) * (int64_t)K + (int)(e % K);
-        dq[off] = from_f32<T>(dqf[off]);
-        dk[off] = from_f32<T>(dkf[off]);
-    }
-    if (!dg && !dg_gamma) return;  // no gate: nothing to differentiate
     float carry = (ddot && len > 0) ? ddot[n * H + h] : 0.f;
     float total = 0.f;
     for (int64_t base = 0; base < len; base += 256) {
-        for (int i = 32 * warp; i < 32 * warp + 32; ++i) {
-            const int64_t t = sp.eos - 1 - base - i;  // reversed index base + i
-            float x = 0.f;
-            if (t >= sp.bos) {
-                const int64_t off = (t * H + h) * (int64_t)K;
-                for (int r = lane; r < K; r += 32)
-                    x = fmaf(to_f32(q[off + r]), dqf[off + r], fmaf(-to_f32(k[off + r]), dkf[off + r], x));
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-            }
-            if (lane == 0) xs[i] = x;
-        }
-        __syncthreads();
+        const int64_t t = sp.eos - 1 - base - tid;  // reversed index base + tid
+        float s = t >= sp.bos ? x[t * H + h] : 0.f;
         // inclusive scan over the reversed index within the chunk
-        float s = xs[tid];
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const float y = __shfl_up_sync(0xffffffffu, s, off);
@@ -311,8 +347,7 @@ rec_bwd_finalize_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
             if (w < warp) before += wtot[w];
             chunk += wtot[w];
         }
-        __syncthreads();  // wtot and xs are rewritten by the next chunk
-        const int64_t t = sp.eos - 1 - base - tid;
+        __syncthreads();  // wtot is rewritten by the next chunk
         const float val = carry + before + s;
         if (t >= sp.bos) {
             if (dg) dg[t * H + h] = val;
@@ -337,29 +372,31 @@ namespace {
 template <typename T>
 cudaError_t rec_bwd_part(const RecBwdArgs &a, int part, cudaStream_t st) {
     const int warps = (a.K + 31) / 32, kpad = 32 * warps;
-    const dim3 grid((unsigned)(a.N * a.H), (unsigned)((a.V + kBCols - 1) / kBCols));
     cudaError_t e;
-    if (part == 0) {
-        const size_t sm = sizeof(float) * ((size_t)kBTB * kpad + 2 * (size_t)kBTB * kBCols + kBTB + warps);
-        if ((e = cudaFuncSetAttribute(rec_bwd_forward_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (part == 0) {  // both sweeps in one launch
+        const size_t smf = sizeof(float) * ((size_t)kBTB * kpad + 2 * (size_t)kBTB * kBCols + kBTB + warps);
+        const size_t smr = sizeof(float) * (2 * (size_t)kBTB * kpad + 2 * (size_t)kBTB * kBCols + kBTB +
+                                            (size_t)kBTB * warps * kBCols);
+        const size_t sm = smf > smr ? smf : smr;
+        if ((e = cudaFuncSetAttribute(rec_bwd_sweeps_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)sm)) != cudaSuccess)
             return e;
-        rec_bwd_forward_kernel<T><<<grid, 32 * warps, sm, st>>>(
-            (const T *)a.k, (const T *)a.v, (const T *)a.dout, a.g, a.g_gamma, a.scale, a.h0, a.dhT, a.dqf, a.ddot,
-            a.cu, a.T_dense, a.T_total, a.H, a.K, a.V, a.vfirst);
+        const dim3 grid((unsigned)(a.N * a.H), (unsigned)((a.V + kBCols - 1) / kBCols), 2);
+        rec_bwd_sweeps_kernel<T><<<grid, 32 * warps, sm, st>>>(
+            (const T *)a.q, (const T *)a.k, (const T *)a.v, (const T *)a.dout, a.g, a.g_gamma, a.scale, a.h0, a.dhT,
+            a.dqf, a.ddot, a.dkf, (T *)a.dv, a.dh0, a.cu, a.T_dense, a.T_total, a.H, a.K, a.V, a.vfirst);
     } else if (part == 1) {
-        const size_t sm = sizeof(float) * (2 * (size_t)kBTB * kpad + 2 * (size_t)kBTB * kBCols + kBTB +
-                                           (size_t)kBTB * warps * kBCols);
-        if ((e = cudaFuncSetAttribute(rec_bwd_reverse_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)sm)) != cudaSuccess)
-            return e;
-        rec_bwd_reverse_kernel<T><<<grid, 32 * warps, sm, st>>>(
-            (const T *)a.q, (const T *)a.k, (const T *)a.v, (const T *)a.dout, a.g, a.g_gamma, a.scale, a.dhT,
-            a.dkf, (T *)a.dv, a.dh0, a.cu, a.T_dense, a.T_total, a.H, a.K, a.V, a.vfirst);
+        const int64_t rows = a.T_total * a.H;
+        if (rows > 0) {
+            const unsigned grid = (unsigned)std::min<int64_t>((rows + 7) / 8, 148 * 16);
+            rec_bwd_rows_kernel<T><<<grid, 256, 0, st>>>((const T *)a.q, (const T *)a.k, a.dqf, a.dkf, (T *)a.dq,
+                                                        (T *)a.dk, (a.dg || a.dg_gamma) ? a.x : nullptr, a.cu, a.N,
+                                                        a.T_total, a.H, a.K);
+        }
     } else {
-        rec_bwd_finalize_kernel<T><<<(unsigned)(a.N * a.H), 256, 0, st>>>(
-            (const T *)a.q, (const T *)a.k, a.dqf, a.dkf, a.dhT ? a.ddot : nullptr, (T *)a.dq, (T *)a.dk, a.dg,
-            a.dg_gamma, a.cu, a.T_dense, a.T_total, a.H, a.K);
+        if (a.dg || a.dg_gamma)
+            rec_bwd_scan_kernel<<<(unsigned)(a.N * a.H), 256, 0, st>>>(a.x, a.dhT ? a.ddot : nullptr, a.dg,
+                                                                      a.dg_gamma, a.cu, a.T_dense, a.T_total, a.H);
     }
     return cudaGetLastError();
 }

@@ -210,8 +210,8 @@ SGLA_API sgla_status simple_gla_fused_recurrent(const void *q, const void *k, co
  * (its gradients are not written); tokens outside every sequence are not written.
  * Supported sizes: 1 <= K <= 512, 1 <= V <= 4096; pointers aligned to their element
  * size.  workspace: at least simple_gla_fused_recurrent_bwd_workspace_size() bytes,
- * 256-byte aligned (fp32 accumulators for dq and dk and one scalar per sequence and
- * head; zeroed by the call).  The state trajectory is recomputed, not stored.
+ * 256-byte aligned (fp32 accumulators for dq and dk, one scalar per sequence and
+ * head, one per token and head; zeroed by the call).  The state trajectory is recomputed, not stored.
  */
 SGLA_API size_t simple_gla_fused_recurrent_bwd_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T,
                                                               int64_t H, int64_t K);
