@@ -26,7 +26,10 @@ Public functions (same names as the C entry points):
   simple_gla_normalized(q, k, v, ...) / simple_gla_normalized_decode_step(...) -- the
       normalised variant through the augmented value (states [.., K, V+1])
   gla_fused_recurrent(q, k, v, gk, ...) -- GLA with a gate vector over the key dimension
-  chunk_simple_gla(...)  -- the article's entry-point name; dispatches on cu_seqlens.
+  chunk_simple_gla(...)  -- the article's entry-point name; dispatches on cu_seqlens, and
+      is differentiable (ChunkSimpleGLAFunction) when an input requires gradients.
+  simple_gla_chunk_bwd(...), simple_gla_fused_recurrent_bwd(...) -- the gradients.
+  gla_chunk(q, k, v, gk, ...) -- GLA with a vector gate, chunked form.
   fused_recurrent_simple_gla(...) -- the article's name for simple_gla_fused_recurrent.
 """
 from __future__ import annotations
@@ -42,7 +45,7 @@ from ._lib import (SGLA_BF16, SGLA_FP32, SGLA_OK, SglaError, lib, library_path, 
 __all__ = ["simple_gla_fwd", "simple_gla_fwd_noalloc", "simple_gla_fwd_varlen", "simple_gla_decode_step", "chunk_simple_gla",
            "simple_gla_fused_recurrent", "fused_recurrent_simple_gla", "simple_gla_chunk",
            "simple_gla_normalized", "simple_gla_normalized_decode_step", "normalized_decode_state_width",
-           "gla_fused_recurrent", "simple_gla_fused_recurrent_bwd", "simple_gla_chunk_bwd", "gla_chunk",
+           "gla_fused_recurrent", "simple_gla_fused_recurrent_bwd", "simple_gla_chunk_bwd", "gla_chunk", "ChunkSimpleGLAFunction",
            "fwd_workspace_size", "varlen_workspace_size", "workspace_status", "library_path",
            "SglaError"]
 
@@ -255,10 +258,41 @@ def simple_gla_chunk(q, k, v, g=None, g_gamma=None, scale=None, initial_state=No
     return (o.unsqueeze(0) if squeeze else o), ht
 
 
+class ChunkSimpleGLAFunction(torch.autograd.Function):
+    """Differentiable chunked forward (the article's section 3: the training path is
+    an autograd function whose backward recovers dq, dk, dv, dg and dh0).  Forward:
+    simple_gla_chunk; backward: simple_gla_chunk_bwd on the saved inputs (the state
+    trajectory is recomputed, not stored).  Argument marshalling only."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, g, g_gamma, initial_state, scale, output_final_state, cu_seqlens, chunk_size,
+                state_v_first):
+        o, ht = simple_gla_chunk(q, k, v, g, g_gamma, scale, initial_state, output_final_state, cu_seqlens,
+                                 chunk_size, state_v_first)
+        ctx.save_for_backward(q, k, v, g, g_gamma, initial_state, cu_seqlens)
+        ctx.opts = (scale, chunk_size, state_v_first)
+        return o, ht
+
+    @staticmethod
+    def backward(ctx, do, dht):
+        q, k, v, g, g_gamma, h0, cu = ctx.saved_tensors
+        scale, chunk_size, vf = ctx.opts
+        r = simple_gla_chunk_bwd(q, k, v, do.contiguous(), g=g, g_gamma=g_gamma, scale=scale, initial_state=h0,
+                                 dht=None if dht is None else dht.contiguous(), cu_seqlens=cu,
+                                 chunk_size=chunk_size, state_v_first=vf)
+        return r["dq"], r["dk"], r["dv"], r["dg"], r["dg_gamma"], r["dh0"], None, None, None, None, None
+
+
 def chunk_simple_gla(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
                      output_final_state=False, cu_seqlens=None, chunk_size=64, state_v_first=False):
     """The article's entry-point name (section 2): dense, or packed when cu_seqlens is
-    given; state_v_first selects the [N,H,V,K] state layout."""
+    given; state_v_first selects the [N,H,V,K] state layout.  When gradients are
+    enabled and an input requires them, the call is differentiable (backward through
+    simple_gla_chunk_bwd)."""
+    if torch.is_grad_enabled() and any(t is not None and t.requires_grad
+                                       for t in (q, k, v, g, g_gamma, initial_state)):
+        return ChunkSimpleGLAFunction.apply(q, k, v, g, g_gamma, initial_state, scale, output_final_state,
+                                            cu_seqlens, chunk_size, state_v_first)
     if state_v_first:
         return simple_gla_chunk(q, k, v, g, g_gamma, scale, initial_state, output_final_state, cu_seqlens,
                                 chunk_size, state_v_first=True)

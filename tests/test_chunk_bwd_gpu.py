@@ -135,3 +135,31 @@ def test_simple_gla_chunk_bwd_state_v_first(dt):
     gpu["dh0"] = gpu["dh0"].transpose(-1, -2)
     ref = oracle.simple_gla_bwd(inp["q"], inp["k"], inp["v"], do, g=inp["g"], initial_state=inp["h0"], dht=dh)
     compare_grads(gpu, ref, TOL[dt], inp)
+
+
+@pytest.mark.parametrize("packed", [False, True])
+def test_chunk_simple_gla_is_differentiable(packed):
+    """chunk_simple_gla with inputs that require gradients: loss.backward() fills
+    q.grad .. initial_state.grad with the oracle's reverse-mode gradients."""
+    dt = torch.bfloat16
+    if packed:
+        cu = torch.tensor([0, 100, 100, 300], dtype=torch.int64)
+        T, H, K, V = 300, 2, 128, 128
+        inp = random_inputs(1, T, H, K, V, dtype=dt, gate="g", h0=True, seed=81, cu_seqlens=cu)
+        N = 3
+    else:
+        cu = None
+        N, T, H, K, V = 2, 200, 2, 128, 64
+        inp = random_inputs(N, T, H, K, V, dtype=dt, gate="g", h0=True, seed=81)
+    do, dh = random_cotangents(inp["v"].shape, N, H, K, V, dtype=dt, seed=82)
+    leaves = {n: to_dev(inp[n]).requires_grad_(True) for n in ("q", "k", "v", "g", "h0")}
+    o, ht = sg.chunk_simple_gla(leaves["q"], leaves["k"], leaves["v"], g=leaves["g"], initial_state=leaves["h0"],
+                                output_final_state=True, cu_seqlens=to_dev(cu))
+    loss = (o.float() * to_dev(do).float()).sum() + (ht * to_dev(dh)).sum()
+    loss.backward()
+    torch.cuda.synchronize()
+    ref = oracle.simple_gla_bwd(inp["q"], inp["k"], inp["v"], do, g=inp["g"], initial_state=inp["h0"], dht=dh,
+                                cu_seqlens=cu)
+    got = dict(dq=leaves["q"].grad, dk=leaves["k"].grad, dv=leaves["v"].grad, dg=leaves["g"].grad,
+               dg_gamma=None, dh0=leaves["h0"].grad)
+    compare_grads(got, ref, TOL[dt], inp)
