@@ -185,6 +185,20 @@ def test_binding_refuses_cpu_tensors():
         sg.simple_gla_fwd(x, x, x)
     with pytest.raises(TypeError):
         sg.simple_gla_decode_step(x[0], x[0], x[0], torch.zeros(1, 8, 16, 16))
+    # every other entry point: no CPU path, the call fails before reaching the library
+    calls = [
+        lambda: sg.simple_gla_chunk(x, x, x),
+        lambda: sg.simple_gla_fused_recurrent(x, x, x),
+        lambda: sg.simple_gla_normalized(x, x, x),
+        lambda: sg.gla_fused_recurrent(x, x, x, x),
+        lambda: sg.gla_chunk(x, x, x, x),
+        lambda: sg.simple_gla_chunk_bwd(x, x, x, x),
+        lambda: sg.simple_gla_fused_recurrent_bwd(x, x, x, x),
+        lambda: sg.chunk_simple_gla(x.clone().requires_grad_(True), x, x),
+    ]
+    for call in calls:
+        with pytest.raises(TypeError):
+            call()
 
 
 def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
