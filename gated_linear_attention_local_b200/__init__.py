@@ -46,6 +46,7 @@ __all__ = ["simple_gla_fwd", "simple_gla_fwd_noalloc", "simple_gla_fwd_varlen", 
            "simple_gla_fused_recurrent", "fused_recurrent_simple_gla", "simple_gla_chunk",
            "simple_gla_normalized", "simple_gla_normalized_decode_step", "normalized_decode_state_width",
            "gla_fused_recurrent", "simple_gla_fused_recurrent_bwd", "simple_gla_chunk_bwd", "gla_chunk", "ChunkSimpleGLAFunction",
+           "simple_gla_log_decay_total", "simple_gla_state_carry",
            "fwd_workspace_size", "varlen_workspace_size", "workspace_status", "library_path",
            "SglaError"]
 
@@ -617,6 +618,40 @@ def gla_chunk(q, k, v, gk, scale=None, initial_state=None, output_final_state=Fa
                          _ptr(o), _ptr(ht), _ptr(cu_seqlens), N, T, H, K, V, dt, _ptr(ws), ws.numel(), _stream())
     raise_for_status(st, "gla_chunk")
     return o, ht
+
+
+def simple_gla_log_decay_total(g=None, g_gamma=None, T=None, H=None):
+    """Total log decay per head of one slice: sum over its tokens of g [T,H] (or
+    [1,T,H]), or T * g_gamma, or 0.  Returns a fp32 [H] CUDA tensor."""
+    _check_cuda("g", g, torch.float32)
+    _check_cuda("g_gamma", g_gamma, torch.float32, 1)
+    if g is not None:
+        T, H = g.shape[-2], g.shape[-1]
+        dev = g.device
+    elif g_gamma is not None:
+        H = g_gamma.shape[0]
+        dev = g_gamma.device
+    else:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    out = torch.empty(H, dtype=torch.float32, device=dev)
+    st = lib().simple_gla_log_decay_total(_ptr(g), _ptr(g_gamma), int(T or 0), int(H), _ptr(out), _stream())
+    raise_for_status(st, "simple_gla_log_decay_total")
+    return out
+
+
+def simple_gla_state_carry(log_decay, states, initial_state=None, rank=0):
+    """State entering rank `rank`'s slice: the fold of the summaries of ranks
+    0 .. rank-1 (log_decay [G,H], states [G,H,K,V] fp32) onto initial_state [H,K,V]
+    (None = 0).  Returns a fp32 [H,K,V] CUDA tensor."""
+    _check_cuda("log_decay", log_decay, torch.float32, 2)
+    _check_cuda("states", states, torch.float32, 4)
+    _check_cuda("initial_state", initial_state, torch.float32, 3)
+    G, H, K, V = states.shape
+    out = torch.empty((H, K, V), dtype=torch.float32, device=states.device)
+    st = lib().simple_gla_state_carry(_ptr(log_decay), _ptr(states), _ptr(initial_state), _ptr(out), int(rank), H, K,
+                                      V, _stream())
+    raise_for_status(st, "simple_gla_state_carry")
+    return out
 
 
 def fused_recurrent_simple_gla(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,

@@ -56,6 +56,8 @@ _SIG = {
     "gla_chunk_workspace_size": ([_P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int], ctypes.c_size_t),
     "gla_chunk": ([_P, _P, _P, _P, _F, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int, _P,
                    ctypes.c_size_t, _P], ctypes.c_int),
+    "simple_gla_log_decay_total": ([_P, _P, _I64, _I64, _P, _P], ctypes.c_int),
+    "simple_gla_state_carry": ([_P, _P, _P, _P, ctypes.c_int, _I64, _I64, _I64, _P], ctypes.c_int),
     "sgla_workspace_status": ([_P, ctypes.POINTER(ctypes.c_int), _P], ctypes.c_int),
     "simple_gla_normalized_workspace_size": ([_P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int],
                                              ctypes.c_size_t),

@@ -314,6 +314,28 @@ SGLA_API sgla_status simple_gla_fwd_noalloc(const void *q, const void *k, const 
                                             int chunk_size, sgla_dtype dtype, void *stream);
 
 /*
+ * Exchange step of one long sequence split along time across G ranks (each rank holds
+ * a contiguous slice).  The carry between slices is associative because the gate is
+ * one scalar per head (article section 3: the inter-chunk propagation is only a
+ * scalar multiplication of S): with rank r's summary (D_r = total log decay of its
+ * slice per head, S_r = its end state from a zero state), the state entering rank
+ * r's slice is  h_r = exp(D_{r-1}) h_{r-1} + S_{r-1},  h_0 = the initial state.
+ *
+ * simple_gla_log_decay_total: out[h] = sum_t g[t, h] over the T tokens of a slice
+ *   (g [T,H] fp32), or T * g_gamma[h], or 0 with neither.  DEVICE pointers.
+ * simple_gla_state_carry: state_in [H,K,V] = the fold of the summaries of ranks
+ *   0 .. rank-1 (log_decay [G,H], states [G,H,K,V], gathered from every rank) onto
+ *   initial_state [H,K,V] (NULL = 0).  DEVICE pointers, fp32.
+ * Both enqueue one kernel on `stream`; invalid arguments return
+ * SGLA_ERR_INVALID_ARGUMENT without launching.
+ */
+SGLA_API sgla_status simple_gla_log_decay_total(const float *g, const float *g_gamma, int64_t T, int64_t H,
+                                                float *out, void *stream);
+SGLA_API sgla_status simple_gla_state_carry(const float *log_decay, const float *states,
+                                            const float *initial_state, float *state_in, int rank,
+                                            int64_t H, int64_t K, int64_t V, void *stream);
+
+/*
  * Read the device-side status word of the last forward call that used
  * `workspace` (SGLA_DEVICE_OK or SGLA_DEVICE_*).  Synchronises `stream`.
  * Returns SGLA_OK and fills *device_status, or an error status.
