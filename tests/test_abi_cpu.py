@@ -35,6 +35,16 @@ def test_header_declares_the_three_entry_points():
         assert n in names
 
 
+def test_header_is_plain_c(tmp_path):
+    """The boundary is a C ABI: the header compiles as C (no C++ or torch types)."""
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "simple_gla.h"\nint main(void) { return 0; }\n')
+    r = subprocess.run(["gcc", "-fsyntax-only", "-std=c11", "-Wall", "-Wextra", "-Werror", "-I",
+                        os.path.join(ROOT, "include"), "-I", "/usr/local/cuda/include", str(src)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
 def test_library_exports_every_declared_symbol(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", L.library_path], capture_output=True, text=True,
                          check=True).stdout
