@@ -42,6 +42,8 @@ def _oracle_ops():
     def log_decay_total(g, g_gamma, T_r, H_):
         if g is not None:
             return g[0].double().sum(0)
+        if g_gamma is not None:
+            return T_r * g_gamma.double()
         return torch.zeros(H_, dtype=torch.float64)
 
     def state_carry(d_all, s_all, h0, rank):
@@ -55,32 +57,34 @@ def _oracle_ops():
 
 def _slices(inp):
     bounds = np.cumsum([0] + LENS)
-    return [{k_: (v_[:, bounds[r]:bounds[r + 1]] if k_ in ("q", "k", "v", "g") else v_) for k_, v_ in inp.items()}
+    return [{k_: (v_[:, bounds[r]:bounds[r + 1]] if k_ in ("q", "k", "v", "g") and v_ is not None else v_)
+             for k_, v_ in inp.items()}
             for r in range(len(LENS))]
 
 
-def _worker(rank, world, port, out):
+def _worker(rank, world, port, out, gate, h0):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     from gated_linear_attention_local_b200.seqsplit import chunk_simple_gla_seq_split
-    inp = random_inputs(1, T, H, K, V, dtype=torch.float32, gate="g", h0=True, seed=7)
+    inp = random_inputs(1, T, H, K, V, dtype=torch.float32, gate=gate, h0=h0, seed=7)
     sl = _slices(inp)[rank]
-    o, ht = chunk_simple_gla_seq_split(sl["q"], sl["k"], sl["v"], g=sl["g"], initial_state=inp["h0"],
-                                       output_final_state=True, ops=_oracle_ops())
+    o, ht = chunk_simple_gla_seq_split(sl["q"], sl["k"], sl["v"], g=sl["g"], g_gamma=inp["g_gamma"],
+                                       initial_state=inp["h0"], output_final_state=True, ops=_oracle_ops())
     out[rank] = (o.numpy(), ht.numpy())
     dist.barrier()
     dist.destroy_process_group()
 
 
-def test_seq_split_orchestration_on_cpu_ranks():
+@pytest.mark.parametrize("gate,h0", [("g", True), ("gamma", False)])
+def test_seq_split_orchestration_on_cpu_ranks(gate, h0):
     import oracle
     world = len(LENS)
     mgr = mp.Manager()
     out = mgr.dict()
-    mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
-    inp = random_inputs(1, T, H, K, V, dtype=torch.float32, gate="g", h0=True, seed=7)
-    ro, rh = oracle.simple_gla_fwd(inp["q"], inp["k"], inp["v"], g=inp["g"], initial_state=inp["h0"],
-                                   output_final_state=True)
+    mp.start_processes(_worker, args=(world, _free_port(), out, gate, h0), nprocs=world, start_method="spawn")
+    inp = random_inputs(1, T, H, K, V, dtype=torch.float32, gate=gate, h0=h0, seed=7)
+    ro, rh = oracle.simple_gla_fwd(inp["q"], inp["k"], inp["v"], g=inp["g"], g_gamma=inp["g_gamma"],
+                                   initial_state=inp["h0"], output_final_state=True)
     bounds = np.cumsum([0] + LENS)
     for r in range(world):
         o, ht = out[r]
