@@ -38,7 +38,7 @@ def _worker(rank, world, port, out):
 
 def test_two_rank_timing_and_sharding():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
     assert sorted(out.keys()) == [0, 1]

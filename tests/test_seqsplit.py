@@ -79,7 +79,7 @@ def _worker(rank, world, port, out, gate, h0):
 def test_seq_split_orchestration_on_cpu_ranks(gate, h0):
     import oracle
     world = len(LENS)
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.start_processes(_worker, args=(world, _free_port(), out, gate, h0), nprocs=world, start_method="spawn")
     inp = random_inputs(1, T, H, K, V, dtype=torch.float32, gate=gate, h0=h0, seed=7)
