@@ -35,6 +35,7 @@ Public functions (same names as the C entry points):
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 
 import torch
@@ -59,6 +60,28 @@ def _ptr(t):
 
 def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _on_tensor_device(fn):
+    """Run ``fn`` with the CUDA device of its tensor arguments current.  The library
+    launches on the calling thread's current device and on that device's current
+    stream, so a call whose tensors live on another device than the current one
+    switches to theirs first; tensors on two different devices are an error (the
+    kernels read only memory local to the device they run on)."""
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        dev = None
+        for t in (*args, *kwargs.values()):
+            if isinstance(t, torch.Tensor) and t.is_cuda:
+                if dev is None:
+                    dev = t.device
+                elif t.device != dev:
+                    raise ValueError(f"{fn.__name__}: tensors on {dev} and {t.device}; all must be on one device")
+        if dev is None or dev.index == torch.cuda.current_device():
+            return fn(*args, **kwargs)
+        with torch.cuda.device(dev):
+            return fn(*args, **kwargs)
+    return wrapper
 
 
 def _check_cuda(name, t, dtype=None, ndim=None):
@@ -107,6 +130,7 @@ def _common_checks(q, k, v, g, g_gamma, initial_state):
     _check_cuda("initial_state", initial_state, torch.float32, 4)
 
 
+@_on_tensor_device
 def simple_gla_fwd(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
                    output_final_state=False, chunk_size=64, workspace=None):
     """Dense chunked forward.  q,k [B,T,H,K]; v [B,T,H,V]; g [B,T,H] fp32 log gates or
@@ -136,6 +160,7 @@ def simple_gla_fwd(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None
     return o, ht
 
 
+@_on_tensor_device
 def simple_gla_fwd_noalloc(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
                            output_final_state=False, chunk_size=64):
     """simple_gla_fwd using the library's built-in 16 MiB scratch instead of a
@@ -159,6 +184,7 @@ def simple_gla_fwd_noalloc(q, k, v, g=None, g_gamma=None, scale=None, initial_st
     return o, ht
 
 
+@_on_tensor_device
 def simple_gla_fwd_varlen(q, k, v, cu_seqlens, g=None, g_gamma=None, scale=None, initial_state=None,
                           output_final_state=False, chunk_size=64, workspace=None):
     """Packed variable-length forward.  q,k [1,T,H,K] or [T,H,K]; v likewise with V;
@@ -204,6 +230,7 @@ def simple_gla_fwd_varlen(q, k, v, cu_seqlens, g=None, g_gamma=None, scale=None,
     return (o.unsqueeze(0) if squeeze else o), ht
 
 
+@_on_tensor_device
 def simple_gla_chunk(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None, output_final_state=False,
                      cu_seqlens=None, chunk_size=64, state_v_first=False, workspace=None):
     """Chunked forward with every option in one call: dense q,k [B,T,H,K] (or packed
@@ -284,6 +311,7 @@ class ChunkSimpleGLAFunction(torch.autograd.Function):
         return r["dq"], r["dk"], r["dv"], r["dg"], r["dg_gamma"], r["dh0"], None, None, None, None, None
 
 
+@_on_tensor_device
 def chunk_simple_gla(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
                      output_final_state=False, cu_seqlens=None, chunk_size=64, state_v_first=False):
     """The article's entry-point name (section 2): dense, or packed when cu_seqlens is
@@ -303,6 +331,7 @@ def chunk_simple_gla(q, k, v, g=None, g_gamma=None, scale=None, initial_state=No
                                  output_final_state, chunk_size)
 
 
+@_on_tensor_device
 def simple_gla_decode_step(q, k, v, state, g=None, g_gamma=None, scale=None, out=None, state_v_first=False):
     """One recurrent step.  q,k [N,H,K]; v [N,H,V]; g [N,H] fp32 or g_gamma [H];
     state [N,H,K,V] fp32 ([N,H,V,K] with state_v_first) updated in place.  Returns
@@ -335,6 +364,7 @@ def simple_gla_decode_step(q, k, v, state, g=None, g_gamma=None, scale=None, out
     return o
 
 
+@_on_tensor_device
 def simple_gla_fused_recurrent(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
                                output_final_state=False, cu_seqlens=None, state_v_first=False,
                                device_status=None):
@@ -431,6 +461,7 @@ def _bwd_prepare(q, k, v, do, g, g_gamma, initial_state, dht, cu_seqlens, state_
     return (N, T, H, K, V), out
 
 
+@_on_tensor_device
 def simple_gla_fused_recurrent_bwd(q, k, v, do, g=None, g_gamma=None, scale=None, initial_state=None, dht=None,
                                    cu_seqlens=None, state_v_first=False, workspace=None):
     """Gradients of simple_gla_fused_recurrent for the loss
@@ -451,6 +482,7 @@ def simple_gla_fused_recurrent_bwd(q, k, v, do, g=None, g_gamma=None, scale=None
     return out
 
 
+@_on_tensor_device
 def simple_gla_chunk_bwd(q, k, v, do, g=None, g_gamma=None, scale=None, initial_state=None, dht=None,
                          cu_seqlens=None, chunk_size=64, state_v_first=False, workspace=None):
     """Gradients of simple_gla_chunk on the tensor-core path, for
@@ -471,6 +503,7 @@ def simple_gla_chunk_bwd(q, k, v, do, g=None, g_gamma=None, scale=None, initial_
     return out
 
 
+@_on_tensor_device
 def simple_gla_normalized(q, k, v, g=None, g_gamma=None, initial_state=None, output_final_state=False,
                           cu_seqlens=None, chunk_size=64, workspace=None):
     """Normalised variant (augmented value, scale 1): o = (q^T S) / (q^T z).  Shapes as
@@ -519,6 +552,7 @@ def normalized_decode_state_width(V: int) -> int:
     return (V + 1 + 3) // 4 * 4
 
 
+@_on_tensor_device
 def simple_gla_normalized_decode_step(q, k, v, state, g=None, g_gamma=None, out=None, workspace=None):
     """One token of the normalised variant, in place on the augmented state
     [N,H,K,normalized_decode_state_width(V)] fp32 (column V is z, later ones stay 0)."""
@@ -542,6 +576,7 @@ def simple_gla_normalized_decode_step(q, k, v, state, g=None, g_gamma=None, out=
     return o
 
 
+@_on_tensor_device
 def gla_fused_recurrent(q, k, v, gk, scale=None, initial_state=None, output_final_state=False, cu_seqlens=None,
                         state_v_first=False, device_status=None):
     """GLA (gate vector over the key dimension), token-serial: gk fp32 log gates shaped
@@ -581,6 +616,7 @@ def gla_fused_recurrent(q, k, v, gk, scale=None, initial_state=None, output_fina
     return (o.unsqueeze(0) if squeeze else o), ht
 
 
+@_on_tensor_device
 def gla_chunk(q, k, v, gk, scale=None, initial_state=None, output_final_state=False, cu_seqlens=None,
               workspace=None):
     """GLA (gate vector over the key dimension) in the chunked form: gk fp32 log gates
@@ -620,6 +656,7 @@ def gla_chunk(q, k, v, gk, scale=None, initial_state=None, output_final_state=Fa
     return o, ht
 
 
+@_on_tensor_device
 def simple_gla_log_decay_total(g=None, g_gamma=None, T=None, H=None):
     """Total log decay per head of one slice: sum over its tokens of g [T,H] (or
     [1,T,H]), or T * g_gamma, or 0.  Returns a fp32 [H] CUDA tensor."""
@@ -639,6 +676,7 @@ def simple_gla_log_decay_total(g=None, g_gamma=None, T=None, H=None):
     return out
 
 
+@_on_tensor_device
 def simple_gla_state_carry(log_decay, states, initial_state=None, rank=0):
     """State entering rank `rank`'s slice: the fold of the summaries of ranks
     0 .. rank-1 (log_decay [G,H], states [G,H,K,V] fp32) onto initial_state [H,K,V]
@@ -662,6 +700,7 @@ def fused_recurrent_simple_gla(q, k, v, g=None, g_gamma=None, scale=None, initia
                                       state_v_first=state_v_first)
 
 
+@_on_tensor_device
 def workspace_status(workspace) -> int:
     """Device status word of the last forward that used ``workspace`` (synchronises)."""
     out = ctypes.c_int(-1)

@@ -216,3 +216,39 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(L, "_lib", None)
     with pytest.raises(ImportError):
         L.lib()
+
+
+class _OnDevice(torch.Tensor):
+    """A CPU tensor that reports itself as living on a given CUDA device (only the
+    binding's device check looks at it; nothing reaches the library)."""
+
+    @property
+    def is_cuda(self):
+        return True
+
+    @property
+    def device(self):
+        return self._dev
+
+
+def _on(dev, *shape):
+    t = torch.Tensor._make_subclass(_OnDevice, torch.zeros(*shape))
+    t._dev = torch.device(dev)
+    return t
+
+
+def test_binding_refuses_tensors_on_two_devices():
+    import gated_linear_attention_local_b200 as sg
+    q0 = _on("cuda:0", 1, 8, 2, 16)
+    g1 = _on("cuda:1", 1, 8, 2)
+    calls = [
+        lambda: sg.simple_gla_fwd(q0, q0, q0, g=g1),
+        lambda: sg.chunk_simple_gla(q0, q0, q0, g=g1),
+        lambda: sg.simple_gla_decode_step(*[_on("cuda:0", 8, 2, 16)] * 3, _on("cuda:1", 8, 2, 16, 16)),
+        lambda: sg.simple_gla_chunk_bwd(q0, q0, q0, q0, g=g1),
+        lambda: sg.gla_chunk(q0, q0, q0, _on("cuda:1", 1, 8, 2, 16)),
+        lambda: sg.simple_gla_state_carry(_on("cuda:0", 2, 2), _on("cuda:1", 2, 2, 16, 16)),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="one device"):
+            call()

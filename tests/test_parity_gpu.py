@@ -335,3 +335,16 @@ def test_tensor_core_wide_k_varlen():
     inp = random_inputs(1, 2900, 2, 512, 128, torch.bfloat16, gate="g", h0=True, seed=52, cu_seqlens=cu)
     gpu = _ran("chunk_output_tc", lambda: run_varlen(inp, cu))
     check(inp, gpu, oracle_fwd(inp, cu=cu), torch.bfloat16, "tc wide-k varlen")
+
+
+@pytest.mark.skipif(torch.cuda.device_count() < 2, reason="needs a second CUDA device")
+def test_call_runs_on_the_device_of_its_tensors():
+    inp = random_inputs(2, 300, 2, 128, 128, torch.bfloat16, gate="g", h0=True, seed=53)
+    dev = torch.device("cuda", 1)
+    d = {k_: (v_.to(dev) if v_ is not None else None) for k_, v_ in inp.items()}
+    with torch.cuda.device(0):
+        o, ht = sg.chunk_simple_gla(d["q"], d["k"], d["v"], g=d["g"], initial_state=d["h0"],
+                                    output_final_state=True)
+        assert o.device == dev and ht.device == dev
+        torch.cuda.synchronize(dev)
+    check(inp, (host(o), host(ht)), oracle_fwd(inp), torch.bfloat16, "second device")
