@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "kernels.h"
+#include "launch_status.h"
 #include "simple_gla.h"
 #include "tc_path.h"
 
@@ -377,6 +378,18 @@ BwdLayout bwd_layout(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, in
 }
 
 }  // namespace
+
+namespace sgla {
+
+sgla_status launch_status(cudaError_t e, const char *where) {
+    if (e != cudaSuccess) return cuda_fail(e, where);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return SGLA_OK;
+}
+
+sgla_status cuda_failure(cudaError_t e, const char *where) { return cuda_fail(e, where); }
+
+}  // namespace sgla
 
 extern "C" {
 

@@ -22,6 +22,7 @@
 //     before any stream capture begins.
 #include <mutex>
 
+#include "launch_status.h"
 #include "simple_gla.h"
 
 namespace {
@@ -39,11 +40,15 @@ std::mutex g_scratch_mutex;
 // resolved here once per device and cached.
 sgla_status static_scratch(void **out) {
     int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SGLA_ERR_CUDA;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return sgla::cuda_failure(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return sgla::cuda_failure(cudaErrorInvalidDevice, "cudaGetDevice");
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
     if (g_scratch_addr[dev] == nullptr) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return SGLA_ERR_CUDA;
+        const cudaError_t es = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (es != cudaSuccess) return sgla::cuda_failure(es, "cudaGetSymbolAddress");
+        if (p == nullptr) return sgla::cuda_failure(cudaErrorInvalidSymbol, "cudaGetSymbolAddress");
         g_scratch_addr[dev] = p;
     }
     *out = g_scratch_addr[dev];

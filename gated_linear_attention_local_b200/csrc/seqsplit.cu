@@ -17,6 +17,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "launch_status.h"
 #include "simple_gla.h"
 
 namespace sgla {
@@ -65,7 +66,7 @@ sgla_status simple_gla_log_decay_total(const float *g, const float *g_gamma, int
     const int warps = 8;
     sgla::log_decay_total_kernel<<<(unsigned)((H + warps - 1) / warps), 32 * warps, 0, st>>>(g, g_gamma, T, (int)H,
                                                                                              out);
-    return cudaGetLastError() == cudaSuccess ? SGLA_OK : SGLA_ERR_CUDA;
+    return sgla::launch_status(cudaGetLastError(), "log_decay_total");
 }
 
 sgla_status simple_gla_state_carry(const float *log_decay, const float *states, const float *initial_state,
@@ -76,7 +77,7 @@ sgla_status simple_gla_state_carry(const float *log_decay, const float *states, 
     const int64_t total = H * K * V;
     const unsigned grid = (unsigned)std::min<int64_t>((total + 255) / 256, 148 * 8);
     sgla::state_carry_kernel<<<grid, 256, 0, st>>>(log_decay, states, initial_state, state_in, rank, (int)H, K * V);
-    return cudaGetLastError() == cudaSuccess ? SGLA_OK : SGLA_ERR_CUDA;
+    return sgla::launch_status(cudaGetLastError(), "state_carry");
 }
 
 }  // extern "C"

@@ -43,8 +43,12 @@
  *     available from sgla_last_cuda_error().  Problems only visible on the device
  *     (a malformed cu_seqlens) are recorded in the workspace and read back with
  *     sgla_workspace_status(); the kernels then write no outputs.
- *   - Not thread-safe with respect to sgla_last_cuda_error() only; everything else
- *     is reentrant.
+ *   - Thread safety: the compute entry points are reentrant (all state lives in
+ *     the caller's buffers).  sgla_last_cuda_error() reports the last failure of
+ *     the calling thread.  Two things are shared by the whole process: the
+ *     launch-recording of sgla_profile_begin / sgla_profile_end (not thread-safe)
+ *     and the fixed scratch of simple_gla_fwd_noalloc (calls that may overlap on
+ *     the GPU race on it).
  */
 #ifndef SIMPLE_GLA_H
 #define SIMPLE_GLA_H

@@ -119,7 +119,9 @@ def test_seq_split_kernels_on_one_gpu(gate):
         h_r = sg.simple_gla_state_carry(d_all, s_all, dev["h0"][0], r)
         o, _ = sg.chunk_simple_gla(s["q"], s["k"], s["v"], g=s["g"], g_gamma=s["g_gamma"], initial_state=h_r[None])
         outs.append(o)
+    n0 = sg.lib().sgla_kernel_launch_count()
     final = sg.simple_gla_state_carry(d_all, s_all, dev["h0"][0], len(lens))
+    assert sg.lib().sgla_kernel_launch_count() == n0 + 1  # the carry is one counted launch
     torch.cuda.synchronize()
     ro, rh = oracle.simple_gla_fwd(inp["q"], inp["k"], inp["v"], g=inp["g"], g_gamma=inp["g_gamma"],
                                    initial_state=inp["h0"], output_final_state=True)
