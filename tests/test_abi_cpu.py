@@ -74,6 +74,20 @@ def test_workspace_sizes(lib):
     assert vs(0, 100, 16, 128, 128, 64, L.SGLA_BF16) == 0
 
 
+
+def test_size_limits_on_the_host(lib):
+    """The largest accepted sizes are accepted and one past them is refused as
+    unsupported, before anything is launched (grid y/z bound for H, int32 token
+    indices inside the kernels)."""
+    ws = lib.simple_gla_fwd_workspace_size
+    assert ws(1, 64, 65535, 64, 64, 64, L.SGLA_BF16) > 0
+    assert ws(1, 64, 65536, 64, 64, 64, L.SGLA_BF16) == 0
+    assert ws(1, 2**31 - 1, 1, 64, 64, 64, L.SGLA_BF16) > 0
+    assert ws(2, 2**30, 1, 64, 64, 64, L.SGLA_BF16) == 0          # B x T = 2^31 tokens
+    assert ws(1, 64, 1, 512, 512, 64, L.SGLA_BF16) > 0
+    assert ws(1, 64, 1, 8, 8, 16, L.SGLA_FP32) > 0                 # smallest head dims, smallest chunk
+    assert lib.simple_gla_fwd_varlen_workspace_size(2, 2**31, 1, 64, 64, 64, L.SGLA_BF16) == 0
+
 FAKE = 1 << 20  # an aligned non-NULL address: every call below must return before using it
 
 
@@ -95,6 +109,8 @@ def test_invalid_calls_are_rejected_on_the_host(lib):
     assert _fwd(lib, q=None) == L.SGLA_ERR_INVALID_ARGUMENT
     assert _fwd(lib, q=FAKE + 2) == L.SGLA_ERR_INVALID_ARGUMENT             # misaligned
     assert _fwd(lib, H=0) == L.SGLA_ERR_INVALID_ARGUMENT
+    assert _fwd(lib, H=65536) == L.SGLA_ERR_UNSUPPORTED
+    assert _fwd(lib, B=2, T=2**30) == L.SGLA_ERR_UNSUPPORTED               # 2^31 tokens
     assert _fwd(lib, B=-1) == L.SGLA_ERR_INVALID_ARGUMENT
     assert _fwd(lib, dtype=7) == L.SGLA_ERR_INVALID_ARGUMENT
     assert _fwd(lib, ws=None) == L.SGLA_ERR_WORKSPACE
