@@ -481,8 +481,9 @@ def oracle_sample(w, budget_s=12.0):
         cal = run(4)
         nseq = int(max(4, min(w["N"], 4 * budget_s / max(cal, 1e-6))))
         dt = run(nseq)
-        # unit: state GB/s over the sampled sequences, all steps
-        gb = w["steps"] * 2 * nseq * w["H"] * w["K"] * w["V"] * 4 / 1e9
+        # unit: GB/s over the sampled sequences, all steps, counting the bytes of a
+        # step as the native arm does (state read + write and the step's q, k, v, g, o)
+        gb = w["steps"] * algorithmic_counts(w)["bytes"] * nseq / w["N"] / 1e9
         return dict(value=gb / dt, unit="GB/s", cores=threads, kind="oracle",
                     sample=f"{nseq} of {w['N']} sequences x {w['steps']} steps, all heads ({dt:.1f} s)")
 
@@ -577,8 +578,14 @@ def reference_arm(args, world, rank):
     vals = [oracle_sample(w, budget_s=budget) for _ in range(args.steps)]
     v = statistics.median(x["value"] for x in vals)
     unit = vals[0]["unit"]
+    # the time one whole step of the workload takes at the sampled rate
+    counts = algorithmic_counts(w)
+    if unit == "GB/s":
+        ms = w["steps"] * counts["bytes"] / (v * 1e9) * 1e3
+    else:
+        ms = counts["tokens"] / v * 1e3
     line = dict(metric=METRIC, value=v, unit=unit, n_gpus=world, steps=args.steps, warmup=args.warmup,
-                ms_per_step=None, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
+                ms_per_step=ms, ms_per_step_basis="a whole step at the sampled rate", higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
                 data="synthetic (seeded)", impl="reference",
                 config=dict(workload=args.workload, **_config_of(w)),
                 cpu_baseline=dict(value=v, unit=unit, cores=vals[0]["cores"], kind="oracle",

@@ -61,3 +61,6 @@ def test_reference_arm_prints_the_contract_line():
         assert key in line, key
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    # per-step time: the whole tiny step (B*T tokens) at the sampled rate
+    w = make_workload("tiny_fp32")
+    assert math.isclose(line["ms_per_step"], w["B"] * w["T"] / line["value"] * 1e3, rel_tol=1e-9)
