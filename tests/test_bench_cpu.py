@@ -64,3 +64,19 @@ def test_reference_arm_prints_the_contract_line():
     # per-step time: the whole tiny step (B*T tokens) at the sampled rate
     w = make_workload("tiny_fp32")
     assert math.isclose(line["ms_per_step"], w["B"] * w["T"] / line["value"] * 1e3, rel_tol=1e-9)
+
+
+def test_reference_arm_under_torchrun_prints_one_line_from_rank_0():
+    import socket
+    with socket.socket() as s_:
+        s_.bind(("127.0.0.1", 0))
+        port = s_.getsockname()[1]
+    out = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                          "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+                          "--impl", "reference", "--gpus", "2", "--workload", "tiny_fp32", "--steps", "1",
+                          "--warmup", "1"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
