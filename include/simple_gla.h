@@ -369,11 +369,14 @@ SGLA_API sgla_status gla_fused_recurrent(const void *q, const void *k, const voi
  * from the inter-chunk state; [FLA-SG] sections 3 and 6 on the per-key decay).  The
  * same operator as gla_fused_recurrent:
  *   S_t = diag(exp(gk_t)) S_{t-1} + k_t v_t^T ;  o_t = scale * S_t^T q_t
- * computed chunk by chunk (32 tokens, two 16-token sub-chunks): a prep kernel
- * forms, for every chunk in parallel, the per-key cumulative gates, q * 2^G,
- * k * 2^(G_last - G), the row decays and the intra-chunk scores (exact inside each
- * 16-token sub-chunk, through the sub-chunk boundary between sub-chunks); a walk
- * kernel carries the K x 64 state in registers from chunk to chunk.
+ * computed chunk by chunk in 16-token sub-chunks: a prep kernel forms, for every
+ * chunk in parallel, the per-key cumulative gates, q * 2^G, k * 2^(G_last - G), the
+ * row decays and the intra-chunk scores (exact inside each sub-chunk, through the
+ * sub-chunk boundary between sub-chunks); a walk kernel carries the state from
+ * chunk to chunk.  bf16 with K = 128 and V a multiple of 64: 128-token chunks and a
+ * tensor-core walk (tcgen05, the fp32 K x 64 state tile in tensor memory);
+ * otherwise 32-token chunks and a CUDA-core walk (the K x 64 state tile in
+ * registers).
  *   q, k [tokens,H,K], v, o [tokens,H,V] dtype; gk [tokens,H,K] fp32 log gates;
  *   dense (cu_seqlens == NULL: N sequences of T tokens) or packed (cu_seqlens: DEVICE
  *   [N+1], N >= 1, T packed tokens; a bad cu_seqlens writes nothing and is reported by
