@@ -89,8 +89,8 @@ SGLA_API int sgla_version(void);
 /* Human-readable name of a status code (static storage; never NULL). */
 SGLA_API const char *sgla_status_string(int status);
 
-/* Message of the last CUDA error seen by this library in the calling process
- * (static storage; "" if none). */
+/* Message of the last CUDA error this library saw in the calling thread
+ * (thread-local storage, valid until that thread's next failing call; "" if none). */
 SGLA_API const char *sgla_last_cuda_error(void);
 
 /*
@@ -130,8 +130,9 @@ SGLA_API size_t simple_gla_fwd_varlen_workspace_size(int64_t N, int64_t T_total,
  *   workspace      device scratch of at least simple_gla_fwd_workspace_size() bytes,
  *                  256-byte aligned; its contents on entry do not matter.
  *   stream         cudaStream_t
- * Supported sizes: 1 <= K, V <= 512, both multiples of 8; H >= 1; B, T >= 0
- * (B*T == 0 writes only final_state = initial_state).
+ * Supported sizes: 1 <= K, V <= 512, both multiples of 8; 1 <= H <= 65535; B, T >= 0
+ * with B*T < 2^31 (B*T == 0 writes only final_state = initial_state).  Larger sizes
+ * -> SGLA_ERR_UNSUPPORTED.
  */
 SGLA_API sgla_status simple_gla_fwd(const void *q, const void *k, const void *v,
                            const float *g, const float *g_gamma, float scale,
