@@ -290,7 +290,7 @@ SGLA_API sgla_status simple_gla_chunk(const void *q, const void *k, const void *
  *   q, k   [N,H,K] dtype;  v, o [N,H,V] dtype;  g [N,H] fp32 or NULL;
  *   g_gamma [H] fp32 or NULL (not both);  scale as simple_gla_fwd;
  *   state  [N,H,K,V] fp32, read and updated IN PLACE.
- * Supported sizes: 1 <= K <= 1024, 1 <= V <= 512 with V a multiple of 4.
+ * Supported sizes: 1 <= K <= 1024, 1 <= V <= 512 with V a multiple of 4, N*H < 2^31.
  * No workspace.
  */
 SGLA_API sgla_status simple_gla_decode_step(const void *q, const void *k, const void *v,
