@@ -5,7 +5,8 @@ xxqk.cn article) defines, per head and token, S_t = exp(g_t) S_{t-1} + k_t v_t^T
 and o_t = scale q_t^T S_t (section 1), with the layout, g/g_gamma and varlen
 conventions of section 2.  The pages print no numeric example, so the pins are:
 
-* hand-derived worked examples (tests/golden/worked_examples.json);
+* hand-derived worked examples (tests/golden/worked_examples.json), forward and
+  gradients;
 * brute force of the parallel form: the explicit decay-masked attention matrix
   D_ij = exp(sum_{l=j+1..i} g_l) (j <= i, diagonal included), built by explicit
   summation, O(T^3) -- the view behind parallel_simple_gla / test_parallel in
@@ -95,10 +96,33 @@ def _close(x, y, rtol=RTOL):
 # ----------------------------------------------------------------------------- pins
 
 
+def _golden_bwd(c, lib_path):
+    """A hand-derived gradient example: every gradient of the loss
+    sum_t <o_t, do_t> + <S_T, dht> against the values worked out in its note."""
+    T, K = np.array(c["q"]).shape
+    V = np.array(c["v"]).shape[1]
+    arr = lambda key, *shape: np.array(c[key], dtype=np.float64).reshape(*shape)  # noqa: E731
+    g = np.log(arr("gate", 1, T, 1)) if "gate" in c else None
+    g_gamma = np.log(np.array([c["gamma"]])) if "gamma" in c else None
+    r = oracle.simple_gla_bwd(arr("q", 1, T, 1, K), arr("k", 1, T, 1, K), arr("v", 1, T, 1, V),
+                              arr("do", 1, T, 1, V), g=g, g_gamma=g_gamma, scale=c["scale"],
+                              initial_state=arr("h0", 1, 1, K, V), dht=arr("dht", 1, 1, K, V), lib_path=lib_path)
+    _close(r["dq"].reshape(T, K), arr("dq", T, K), 1e-12)
+    _close(r["dk"].reshape(T, K), arr("dk", T, K), 1e-12)
+    _close(r["dv"].reshape(T, V), arr("dv", T, V), 1e-12)
+    _close(r["dh0"].reshape(K, V), arr("dh0", K, V), 1e-12)
+    if "dg" in c:
+        _close(r["dg"].reshape(T), arr("dg", T), 1e-12)
+    else:
+        _close(r["dg_gamma"].reshape(1), np.array([c["dg_gamma"]]), 1e-12)
+
 def pin_golden(lib_path=None):
     with open(os.path.join(HERE, "golden", "worked_examples.json")) as f:
         cases = json.load(f)["cases"]
     for c in cases:
+        if c.get("bwd"):
+            _golden_bwd(c, lib_path)
+            continue
         if c.get("gla"):
             T, K = np.array(c["q"]).shape
             V = np.array(c["v"]).shape[1]
