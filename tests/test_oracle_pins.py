@@ -17,6 +17,10 @@ conventions of section 2.  The pages print no numeric example, so the pins are:
   separate per-sequence calls, decode == forward, linearity, default scale;
 * planted mistakes: plausible bugs are planted in a copy of the oracle source and
   each must fail at least one of the pins above.
+
+The brute-force forms (Simple GLA and GLA) and the finite-difference check of the
+backward also run over many small random shapes (hypothesis, derandomised),
+T = 0 and one-element head dims included.
 """
 import json
 import math
@@ -462,3 +466,74 @@ def test_planted_mistake_is_caught(name, tmp_path):
         except (AssertionError, RuntimeError):
             failed.append(pin.__name__)
     assert failed, f"planted mistake {name} passed every pin"
+
+
+# ----------------------------------------------------------------------------- randomised shapes
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=60, deadline=None, derandomize=True)
+@given(B=st.integers(1, 2), T=st.integers(0, 20), H=st.integers(1, 3), K=st.integers(1, 5), V=st.integers(1, 5),
+       gate=st.sampled_from(["g", "gamma", "none"]), h0=st.booleans(),
+       scale=st.sampled_from([None, 0.25, 1.0]), seed=st.integers(0, 2**16))
+def test_oracle_equals_brute_force_on_random_shapes(B, T, H, K, V, gate, h0, scale, seed, oracle_lib):
+    """The brute-force parallel form against the oracle over many small shapes,
+    including T = 0 and one-element head dims."""
+    rng = np.random.default_rng(seed)
+    q, k, v, g, gg, s0 = _inputs(rng, B, T, H, K, V, gate, 1.0, h0)
+    o, hT = oracle.simple_gla_fwd(q, k, v, g=g, g_gamma=gg, scale=scale, initial_state=s0,
+                                  output_final_state=True, lib_path=oracle_lib)
+    ob, hb = _brute_force(q, k, v, g, gg, scale, s0)
+    _close(o, ob)
+    _close(hT, hb)
+
+
+@settings(max_examples=25, deadline=None, derandomize=True)
+@given(B=st.integers(1, 2), T=st.integers(1, 6), H=st.integers(1, 2), K=st.integers(1, 3), V=st.integers(1, 3),
+       gate=st.sampled_from(["g", "gamma"]), h0=st.booleans(), with_dht=st.booleans(), seed=st.integers(0, 2**16))
+def test_oracle_backward_equals_finite_differences_on_random_shapes(B, T, H, K, V, gate, h0, with_dht, seed,
+                                                                    oracle_lib):
+    """Reverse mode against central finite differences of the forward over many
+    small shapes, with and without an initial state and an output-state gradient."""
+    rng = np.random.default_rng(seed)
+    q, k, v, g, gg, s0 = _inputs(rng, B, T, H, K, V, gate, 1.0, h0)
+    do = rng.standard_normal((B, T, H, V))
+    dht = rng.standard_normal((B, H, K, V)) if with_dht else None
+
+    def loss():
+        o, hT = oracle.simple_gla_fwd(q, k, v, g=g, g_gamma=gg, scale=0.7, initial_state=s0,
+                                      output_final_state=True, lib_path=oracle_lib)
+        return float(np.sum(o * do) + (np.sum(hT * dht) if dht is not None else 0.0))
+    r = oracle.simple_gla_bwd(q, k, v, do, g=g, g_gamma=gg, scale=0.7, initial_state=s0, dht=dht,
+                              lib_path=oracle_lib)
+    for name, x in (("dq", q), ("dk", k), ("dv", v)):
+        _close(r[name], _fd_grad(loss, x), 1e-6)
+    if s0 is not None:
+        _close(r["dh0"], _fd_grad(loss, s0), 1e-6)
+    else:
+        assert r["dh0"] is None
+    if g is not None:
+        _close(r["dg"], _fd_grad(loss, g), 1e-6)
+    else:
+        _close(r["dg_gamma"], _fd_grad(loss, gg), 1e-6)
+
+
+@settings(max_examples=40, deadline=None, derandomize=True)
+@given(B=st.integers(1, 2), T=st.integers(0, 16), H=st.integers(1, 2), K=st.integers(1, 5), V=st.integers(1, 4),
+       h0=st.booleans(), seed=st.integers(0, 2**16))
+def test_gla_oracle_equals_brute_force_on_random_shapes(B, T, H, K, V, h0, seed, oracle_lib):
+    """GLA's per-key-decay parallel form against the oracle over many small shapes."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, T, H, K))
+    k = rng.standard_normal((B, T, H, K))
+    v = rng.standard_normal((B, T, H, V))
+    gk = _logsigmoid(rng.standard_normal((B, T, H, K)))
+    s0 = 0.5 * rng.standard_normal((B, H, K, V)) if h0 else None
+    o, hT = oracle.gla_fwd(q, k, v, gk, scale=0.6, initial_state=s0, output_final_state=True, lib_path=oracle_lib)
+    for b in range(B):
+        for h in range(H):
+            ob, hb = _gla_brute_force_head(q[b, :, h], k[b, :, h], v[b, :, h], gk[b, :, h], 0.6,
+                                           None if s0 is None else s0[b, h])
+            _close(o[b, :, h], ob)
+            _close(hT[b, h], hb)
