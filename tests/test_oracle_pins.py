@@ -537,3 +537,21 @@ def test_gla_oracle_equals_brute_force_on_random_shapes(B, T, H, K, V, h0, seed,
                                            None if s0 is None else s0[b, h])
             _close(o[b, :, h], ob)
             _close(hT[b, h], hb)
+
+
+@settings(max_examples=40, deadline=None, derandomize=True)
+@given(lens=st.lists(st.integers(0, 9), min_size=1, max_size=4), H=st.integers(1, 2), K=st.integers(1, 4),
+       V=st.integers(1, 4), gate=st.sampled_from(["g", "gamma", "none"]), h0=st.booleans(),
+       seed=st.integers(0, 2**16))
+def test_varlen_oracle_equals_brute_force_on_random_lengths(lens, H, K, V, gate, h0, seed, oracle_lib):
+    """Packed sequences of random lengths (empty ones included) against the parallel
+    form of each sequence on its own span."""
+    rng = np.random.default_rng(seed)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    q, k, v, g, gg, _ = _inputs(rng, 1, int(cu[-1]), H, K, V, gate, 1.0, False)
+    s0 = 0.5 * rng.standard_normal((len(lens), H, K, V)) if h0 else None
+    o, hT = oracle.simple_gla_fwd(q, k, v, g=g, g_gamma=gg, initial_state=s0, output_final_state=True,
+                                  cu_seqlens=cu, lib_path=oracle_lib)
+    ob, hb = _brute_force(q, k, v, g, gg, None, s0, cu)
+    _close(o, ob)
+    _close(hT, hb)
