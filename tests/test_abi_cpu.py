@@ -268,3 +268,13 @@ def test_binding_refuses_tensors_on_two_devices():
     for call in calls:
         with pytest.raises(ValueError, match="one device"):
             call()
+
+
+def test_every_compute_entry_point_has_a_binding_of_the_same_name():
+    import gated_linear_attention_local_b200 as sg
+    text = open(HEADER).read()
+    names = re.findall(r"SGLA_API\s+sgla_status\s+(\w+)\s*\(", text)
+    compute = [n for n in names if not n.startswith("sgla_")]
+    assert {"simple_gla_fwd", "simple_gla_fwd_varlen", "simple_gla_decode_step"} <= set(compute)
+    missing = [n for n in compute if not callable(getattr(sg, n, None))]
+    assert not missing, missing
