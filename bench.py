@@ -5,10 +5,13 @@
 
 One JSON line on rank 0.  A "step" is one pass of the whole forward hot path --
 plan, chunk cumsum, segment states, carry, fused output walk -- over one batch of
-the named workload (default: dense_prefill, B=4 T=2048 H=4 K=V=512 bf16), with
-inputs resident in HBM.  Each step is timed with CUDA events on the launching
-stream; L2 is flushed (256 MiB write) between steps, outside the events.  The
-other workloads are measured the same way and reported under "secondary".
+the named workload (default: long_gamma, B=1 T=65536 H=32 K=V=128 bf16 with a
+per-head decay -- the largest single-GPU workload), with inputs resident in HBM.
+Each step is timed with CUDA events on the launching stream; L2 is flushed
+(256 MiB write) between steps, outside the events; the step time reported is the
+median over the timed steps (p10 and p90 beside it).  The other workloads are
+measured the same way and reported, in compact form, under "secondary" (last key
+of the line; the dense, packed and decode workloads are its last entries).
 
 Multi-GPU (torchrun, one process per GPU): every (sequence, head) is independent,
 so each rank runs its own batch of the workload with no collective on the data
@@ -373,6 +376,17 @@ def time_steps(step, reset, steps, warmup, flush, dist_on, profile=True):
     return per_step, prof, launches
 
 
+def percentile(xs, p):
+    """p-th percentile of xs (linear interpolation between order statistics)."""
+    ys = sorted(xs)
+    if not ys:
+        return float("nan")
+    x = (len(ys) - 1) * p / 100.0
+    lo = int(math.floor(x))
+    hi = min(lo + 1, len(ys) - 1)
+    return ys[lo] + (ys[hi] - ys[lo]) * (x - lo)
+
+
 def dominant(prof):
     if not prof:
         return None, 0, 0.0
@@ -382,92 +396,122 @@ def dominant(prof):
 
 
 def e2e_measure(w, sg, device, steps, warmup):
-    """Same metric through the public API with inputs in pinned HOST memory: every
-    step copies the inputs host->device, runs the call and reads the result back."""
-    keys = [k for k in ("q", "k", "v", "g", "h0", "cu_seqlens", "do", "dht") if w.get(k) is not None]
+    """Same metric through the public API with inputs in pinned HOST memory.  Every
+    step uploads its inputs host->device, runs the call and reads its results back
+    into pinned host memory.  Steps are pipelined over three streams (upload,
+    compute, read-back) with two device input buffers, so the upload of step i+1 and
+    the read-back of step i-1 overlap the compute of step i (each PCIe direction has
+    its own copy engine).  The time is taken with events from before the first
+    upload to after the last read-back.  Returns (ms per step, h2d bytes per step,
+    d2h bytes per step)."""
+    keys = [k for k in ("q", "k", "v", "g", "g_gamma", "h0", "cu_seqlens", "do", "dht") if w.get(k) is not None]
     if w["kind"] == "decode":
         keys = ["q", "k", "v", "g", "state"]
     hostin = {k: w[k].pin_memory() for k in keys}
     h2d = sum(t.numel() * t.element_size() for t in hostin.values())
-    g_gamma = w["g_gamma"].to(device) if w.get("g_gamma") is not None else None
+    bufs = [{k: torch.empty(t.shape, dtype=t.dtype, device=device) for k, t in hostin.items()} for _ in range(2)]
     ws = workspace_for(w, sg, device)
-    if w["kind"] == "decode":
-        out_host = torch.empty(w["steps"], w["N"], w["H"], w["V"], dtype=w["q"].dtype).pin_memory()
-        st_host = torch.empty_like(w["state"]).pin_memory()
-        d2h = out_host.numel() * out_host.element_size() + st_host.numel() * 4
-    elif w.get("entry") in ("recurrent_bwd", "chunk_bwd"):
-        grads_host = {n: torch.empty_like(w[s]).pin_memory() for n, s in (("dq", "q"), ("dk", "k"), ("dv", "v"),
-                                                                          ("dg", "g"), ("dh0", "h0"))}
-        d2h = sum(t.numel() * t.element_size() for t in grads_host.values())
-    else:
-        tokens_shape = (w["B"], w["T"]) if w["kind"] == "dense" else (w["T"],)
-        out_host = torch.empty(*tokens_shape, w["H"], w["V"], dtype=w["q"].dtype).pin_memory()
-        sv = w["V"] + 1 if w.get("entry") == "normalized" else w["V"]
-        st_host = torch.empty(w["N"], w["H"], w["K"], sv).pin_memory() if w["output_final_state"] else None
-        d2h = out_host.numel() * out_host.element_size() + (st_host.numel() * 4 if st_host is not None else 0)
+    host_out = {}
 
-    def one():
-        d = {k: v.to(device, non_blocking=True) for k, v in hostin.items()}
+    def call(d):
+        """One public-API call on the current (compute) stream; returns the device
+        tensors to read back, by name."""
         if w["kind"] == "decode":
+            outs = {}
             for t in range(w["steps"]):
-                o = sg.simple_gla_decode_step(d["q"][t], d["k"][t], d["v"][t], d["state"], g=d["g"][t],
-                                              scale=w["scale"])
-                out_host[t].copy_(o, non_blocking=True)
-            st_host.copy_(d["state"], non_blocking=True)
-            return
+                outs[f"o{t}"] = sg.simple_gla_decode_step(d["q"][t], d["k"][t], d["v"][t], d["state"], g=d["g"][t],
+                                                          scale=w["scale"])
+            outs["state"] = d["state"]
+            return outs
         if w.get("entry") in ("recurrent_bwd", "chunk_bwd"):
             fn = sg.simple_gla_fused_recurrent_bwd if w["entry"] == "recurrent_bwd" else \
                 functools.partial(sg.simple_gla_chunk_bwd, chunk_size=w["chunk_size"])
-            r = fn(d["q"], d["k"], d["v"], d["do"], g=d["g"], g_gamma=g_gamma, scale=w["scale"],
-                   initial_state=d["h0"], dht=d["dht"], workspace=ws)
-            for n, t in grads_host.items():
-                t.copy_(r[n], non_blocking=True)
-            return
+            r = fn(d["q"], d["k"], d["v"], d["do"], g=d.get("g"), g_gamma=d.get("g_gamma"), scale=w["scale"],
+                   initial_state=d.get("h0"), dht=d.get("dht"), workspace=ws)
+            return {n: r[n] for n in ("dq", "dk", "dv", "dg", "dh0") if r.get(n) is not None}
         if w["kind"] == "varlen":
             o, ht = sg.simple_gla_fwd_varlen(d["q"][0], d["k"][0], d["v"][0], d["cu_seqlens"], g=d["g"][0],
-                                             g_gamma=g_gamma, scale=w["scale"], initial_state=d.get("h0"),
+                                             g_gamma=d.get("g_gamma"), scale=w["scale"], initial_state=d.get("h0"),
                                              output_final_state=w["output_final_state"],
                                              chunk_size=w["chunk_size"], workspace=ws)
         elif w.get("entry") == "normalized":
-            o, ht = sg.simple_gla_normalized(d["q"], d["k"], d["v"], g=d.get("g"), g_gamma=g_gamma,
+            o, ht = sg.simple_gla_normalized(d["q"], d["k"], d["v"], g=d.get("g"), g_gamma=d.get("g_gamma"),
                                              initial_state=d.get("h0"), output_final_state=w["output_final_state"],
                                              chunk_size=w["chunk_size"], workspace=ws)
         elif w.get("entry") == "gla_chunk":
             o, ht = sg.gla_chunk(d["q"], d["k"], d["v"], d["g"], scale=w["scale"], initial_state=d.get("h0"),
                                  output_final_state=w["output_final_state"], workspace=ws)
         elif w.get("entry") == "gla":
-            o, ht = sg.gla_fused_recurrent(d["q"], d["k"], d["v"], d["g"], scale=w["scale"], initial_state=d.get("h0"),
-                                           output_final_state=w["output_final_state"])
+            o, ht = sg.gla_fused_recurrent(d["q"], d["k"], d["v"], d["g"], scale=w["scale"],
+                                           initial_state=d.get("h0"), output_final_state=w["output_final_state"])
         elif w.get("entry") == "recurrent":
-            o, ht = sg.simple_gla_fused_recurrent(d["q"], d["k"], d["v"], g=d.get("g"), g_gamma=g_gamma,
+            o, ht = sg.simple_gla_fused_recurrent(d["q"], d["k"], d["v"], g=d.get("g"), g_gamma=d.get("g_gamma"),
                                                   scale=w["scale"], initial_state=d.get("h0"),
                                                   output_final_state=w["output_final_state"])
         else:
-            o, ht = sg.simple_gla_fwd(d["q"], d["k"], d["v"], g=d.get("g"), g_gamma=g_gamma, scale=w["scale"],
-                                      initial_state=d.get("h0"), output_final_state=w["output_final_state"],
-                                      chunk_size=w["chunk_size"], workspace=ws)
-        out_host.copy_(o, non_blocking=True)
-        if st_host is not None:
-            st_host.copy_(ht, non_blocking=True)
+            o, ht = sg.simple_gla_fwd(d["q"], d["k"], d["v"], g=d.get("g"), g_gamma=d.get("g_gamma"),
+                                      scale=w["scale"], initial_state=d.get("h0"),
+                                      output_final_state=w["output_final_state"], chunk_size=w["chunk_size"],
+                                      workspace=ws)
+        outs = {"o": o}
+        if ht is not None:
+            outs["final_state"] = ht
+        return outs
 
-    for _ in range(warmup):
-        one()
-    torch.cuda.synchronize()
+    comp = torch.cuda.current_stream(device)
+    s_up, s_down = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b uploaded
+    ev_used = [torch.cuda.Event() for _ in range(2)]  # the call reading buffer b has been enqueued after
+    used = [False, False]
+
+    def one(i):
+        b = i % 2
+        d = bufs[b]
+        with torch.cuda.stream(s_up):
+            if used[b]:
+                s_up.wait_event(ev_used[b])
+            for k, t in hostin.items():
+                d[k].copy_(t, non_blocking=True)
+            ev_in[b].record(s_up)
+        comp.wait_event(ev_in[b])
+        outs = call(d)
+        ev_used[b].record(comp)
+        used[b] = True
+        s_down.wait_event(ev_used[b])
+        with torch.cuda.stream(s_down):
+            for n, t in outs.items():
+                if n not in host_out:
+                    host_out[n] = torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                host_out[n].copy_(t, non_blocking=True)
+                t.record_stream(s_down)
+
+    for i in range(warmup):
+        one(i)
+    torch.cuda.synchronize(device)
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
-        one()
-    b.record()
-    torch.cuda.synchronize()
+    a.record(comp)
+    s_up.wait_event(a)
+    s_down.wait_event(a)
+    for i in range(steps):
+        one(i)
+    done = torch.cuda.Event()
+    done.record(s_down)
+    comp.wait_event(done)
+    b.record(comp)
+    torch.cuda.synchronize(device)
     return a.elapsed_time(b) / steps, h2d, d2h
 
 
 # ----------------------------------------------------------------------------- CPU oracle leg
 
-def oracle_sample(w, budget_s=12.0):
+def oracle_sample(w, budget_s=4.0, repeats=3):
     """Time the fp64 oracle on a bounded sample of the workload: all heads and
     sequences, a prefix of the tokens (decode: a subset of the sequences), sized
-    from a short calibration run to take about budget_s seconds."""
+    from a short calibration run to take about budget_s seconds per run; the rate
+    is the median of `repeats` runs of that sample.  Both bench arms (the native
+    arm's cpu_baseline leg and --impl reference) time the oracle through this one
+    function, so their figures differ only by run-to-run noise of the host."""
     import oracle
     threads = oracle.default_threads()
     if w["kind"] == "decode":
@@ -480,12 +524,13 @@ def oracle_sample(w, budget_s=12.0):
             return time.perf_counter() - t0
         cal = run(4)
         nseq = int(max(4, min(w["N"], 4 * budget_s / max(cal, 1e-6))))
-        dt = run(nseq)
+        dt = statistics.median(run(nseq) for _ in range(repeats))
         # unit: GB/s over the sampled sequences, all steps, counting the bytes of a
         # step as the native arm does (state read + write and the step's q, k, v, g, o)
         gb = w["steps"] * algorithmic_counts(w)["bytes"] * nseq / w["N"] / 1e9
         return dict(value=gb / dt, unit="GB/s", cores=threads, kind="oracle",
-                    sample=f"{nseq} of {w['N']} sequences x {w['steps']} steps, all heads ({dt:.1f} s)")
+                    sample=f"{nseq} of {w['N']} sequences x {w['steps']} steps, all heads "
+                           f"(median of {repeats} runs of {dt:.1f} s)")
 
     def sub(tn):
         d = {}
@@ -525,12 +570,13 @@ def oracle_sample(w, budget_s=12.0):
     max_t = w["T"] if w["kind"] == "dense" else int((w["cu_seqlens"][1:] - w["cu_seqlens"][:-1]).max())
     full_tokens = w["B"] * w["T"] if w["kind"] == "dense" else w["T"]
     tn = int(min(max_t, max(32, 32 * budget_s / max(cal_t, 1e-6))))
-    dt, ntok = run(tn)
+    runs = [run(tn) for _ in range(repeats)]
+    dt, ntok = statistics.median(r[0] for r in runs), runs[0][1]
     bwd = w.get("entry") in ("recurrent_bwd", "chunk_bwd")
     what = "fp64 reverse-mode of the naive recurrence" if bwd else "fp64 naive recurrence"
     return dict(value=ntok / dt, unit="tokens/s", cores=1 if bwd else threads,
                 kind="oracle", sample=f"first {tn} tokens of every sequence ({ntok} of {full_tokens} tokens), "
-                                      f"all heads, {what} ({dt:.1f} s)")
+                                      f"all heads, {what} (median of {repeats} runs of {dt:.1f} s)")
 
 
 # ----------------------------------------------------------------------------- main
@@ -540,7 +586,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="dense_prefill")
+    ap.add_argument("--workload", default="long_gamma")
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-secondary", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -572,10 +618,10 @@ def reference_arm(args, world, rank):
     if rank != 0:
         return None
     w = make_workload(args.workload, seed=args.seed)
-    budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    budget = max(2.0, min(4.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_sample(w, budget_s=budget / 4)
-    vals = [oracle_sample(w, budget_s=budget) for _ in range(args.steps)]
+        oracle_sample(w, budget_s=budget / 4, repeats=1)
+    vals = [oracle_sample(w, budget_s=budget, repeats=1) for _ in range(args.steps)]
     v = statistics.median(x["value"] for x in vals)
     unit = vals[0]["unit"]
     # the time one whole step of the workload takes at the sampled rate
@@ -652,8 +698,10 @@ def measure_workload(name, args, device, world, rank, peaks, steps, warmup, flus
             launches = per_graph * steps
             timing = f"one CUDA graph of {per_graph} decode-step launches per call"
             del graph
-    total_ms = max_over_ranks(sum(per_step), world, device)
-    ms = total_ms / steps
+    # median step (p10, p90 beside it); multi-GPU: the max over ranks of each
+    ms = max_over_ranks(percentile(per_step, 50), world, device)
+    ms_p10 = max_over_ranks(percentile(per_step, 10), world, device)
+    ms_p90 = max_over_ranks(percentile(per_step, 90), world, device)
     counts = algorithmic_counts(w)
     kname, kn, kms = dominant(prof)
     if w["kind"] == "decode":
@@ -663,8 +711,8 @@ def measure_workload(name, args, device, world, rank, peaks, steps, warmup, flus
         value = world * counts["tokens"] / (ms * 1e-3)
         unit = "tokens/s"
     kernel_ms = kms / max(kn, 1)
-    res = dict(value=value, unit=unit, ms_per_step=ms,
-               ms_p10=sorted(per_step)[len(per_step) // 10], ms_p90=sorted(per_step)[(9 * len(per_step)) // 10],
+    res = dict(value=value, unit=unit, ms_per_step=ms, ms_p10=ms_p10, ms_p90=ms_p90,
+               ms_mean=max_over_ranks(sum(per_step) / len(per_step), world, device),
                tflops=counts["flops"] * (w["steps"] if w["kind"] == "decode" else 1) / (ms * 1e-3) / 1e12,
                gbs=counts["bytes"] * (w["steps"] if w["kind"] == "decode" else 1) / (ms * 1e-3) / 1e9,
                roofline=roofline(w, counts, kernel_ms, peaks, captured_traffic(name, kname), kname) if kname else None,
@@ -688,6 +736,29 @@ def measure_workload(name, args, device, world, rank, peaks, steps, warmup, flus
     return res
 
 
+# Secondary workloads in the order they are printed: the rows built on the hot path
+# first, the hot-path workloads last (a reader of the end of the line sees them).
+_SECONDARY_LAST = ("tiny_fp32", "dense_prefill", "varlen_prefill", "long_gamma", "decode")
+
+
+def secondary_order(headline):
+    from gated_linear_attention_local_b200.workloads import WORKLOADS
+    first = [n for n in WORKLOADS if n not in _SECONDARY_LAST]
+    return [n for n in first + list(_SECONDARY_LAST) if n != headline]
+
+
+def compact(r):
+    """The figures of a secondary workload, without its per-kernel breakdown."""
+    rf = r.get("roofline") or {}
+    dk = r.get("dominant_kernel") or {}
+    rnd = lambda x, n=4: None if x is None else round(x, n)
+    return dict(value=float(f"{r['value']:.5g}"), unit=r["unit"], ms=rnd(r["ms_per_step"]),
+                p10=rnd(r["ms_p10"]), p90=rnd(r["ms_p90"]), bound=rf.get("bound"), frac=rf.get("frac"),
+                call_frac=rnd(r["call_roofline_frac"]), kernel=dk.get("name"), kernel_ms=rnd(dk.get("avg_ms")),
+                launches=r["gpu_launches"], reasons=(r.get("clocks") or {}).get("reasons"),
+                sm_mhz=(r.get("clocks") or {}).get("sm_mhz"))
+
+
 def main(argv=None):
     args = parse_args(argv)
     world, rank, local = dist_setup(args)
@@ -708,19 +779,16 @@ def main(argv=None):
                                 want_e2e=True, want_cpu=not args.no_cpu_baseline)
     secondary = {}
     if not args.no_secondary:
-        from gated_linear_attention_local_b200.workloads import WORKLOADS
-        for name in WORKLOADS:
-            if name == args.workload:
-                continue
+        for name in secondary_order(args.workload):
             r = measure_workload(name, args, device, world, rank, peaks, max(5, min(args.steps, 20)),
                                  max(3, args.warmup), flush, want_e2e=False, want_cpu=False)
-            secondary[name] = {k: r[k] for k in ("value", "unit", "ms_per_step", "tflops", "gbs", "roofline",
-                                                  "call_roofline_frac", "dominant_kernel", "gpu_launches",
-                                                  "clocks", "config")}
+            secondary[name] = compact(r)
             torch.cuda.empty_cache()
     if rank == 0:
         line = dict(metric=METRIC, value=main_res["value"], unit=main_res["unit"], n_gpus=world,
                     steps=args.steps, warmup=args.warmup, ms_per_step=main_res["ms_per_step"],
+                    ms_per_step_stat="median over the timed steps", ms_p10=main_res["ms_p10"],
+                    ms_p90=main_res["ms_p90"], ms_mean=main_res["ms_mean"],
                     higher_is_better=True, scaling="weak", vs_baseline=None, dtype=main_res["dtype"],
                     data="synthetic: seeded N(0,1) / logsigmoid(N(0,1)) inputs shaped like the pages' workloads",
                     config=dict(main_res["config"], parallelism=f"dp{world} (independent batches, no collective)",
@@ -729,8 +797,7 @@ def main(argv=None):
                     cpu_baseline=main_res.get("cpu_baseline"), e2e=main_res["e2e"],
                     gpu_launches=main_res["gpu_launches"], clocks=main_res["clocks"],
                     kernels=main_res["kernels"], dominant_kernel=main_res["dominant_kernel"],
-                    ms_p10=main_res["ms_p10"], ms_p90=main_res["ms_p90"], tflops=main_res["tflops"],
-                    gbs=main_res["gbs"], secondary=secondary)
+                    tflops=main_res["tflops"], gbs=main_res["gbs"], secondary=secondary)
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()

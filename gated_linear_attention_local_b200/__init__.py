@@ -48,7 +48,7 @@ __all__ = ["simple_gla_fwd", "simple_gla_fwd_noalloc", "simple_gla_fwd_varlen", 
            "simple_gla_normalized", "simple_gla_normalized_decode_step", "normalized_decode_state_width",
            "gla_fused_recurrent", "simple_gla_fused_recurrent_bwd", "simple_gla_chunk_bwd", "gla_chunk", "ChunkSimpleGLAFunction",
            "simple_gla_log_decay_total", "simple_gla_state_carry",
-           "fwd_workspace_size", "varlen_workspace_size", "workspace_status", "library_path",
+           "fwd_workspace_size", "varlen_workspace_size", "workspace_status", "noalloc_status", "library_path",
            "SglaError"]
 
 _DTYPES = {torch.bfloat16: SGLA_BF16, torch.float32: SGLA_FP32}
@@ -130,11 +130,10 @@ def _common_checks(q, k, v, g, g_gamma, initial_state):
     _check_cuda("initial_state", initial_state, torch.float32, 4)
 
 
-@_on_tensor_device
-def simple_gla_fwd(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
-                   output_final_state=False, chunk_size=64, workspace=None):
-    """Dense chunked forward.  q,k [B,T,H,K]; v [B,T,H,V]; g [B,T,H] fp32 log gates or
-    g_gamma [H]; initial_state [B,H,K,V] fp32.  Returns (o [B,T,H,V], final_state)."""
+def _dense_shapes(q, k, v, g, g_gamma, initial_state):
+    """Checks shared by the dense forwards; returns (B, T, H, K, V).  Every tensor the
+    kernels index by these sizes is checked against them, so no mis-shaped argument
+    reaches the device."""
     _common_checks(q, k, v, g, g_gamma, initial_state)
     if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
         raise ValueError("q,k must be [B,T,H,K] and v [B,T,H,V]")
@@ -146,6 +145,15 @@ def simple_gla_fwd(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None
         raise ValueError(f"g_gamma must be [H] = ({H},)")
     if initial_state is not None and tuple(initial_state.shape) != (B, H, K, V):
         raise ValueError(f"initial_state must be [B,H,K,V] = {(B, H, K, V)}")
+    return B, T, H, K, V
+
+
+@_on_tensor_device
+def simple_gla_fwd(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
+                   output_final_state=False, chunk_size=64, workspace=None):
+    """Dense chunked forward.  q,k [B,T,H,K]; v [B,T,H,V]; g [B,T,H] fp32 log gates or
+    g_gamma [H]; initial_state [B,H,K,V] fp32.  Returns (o [B,T,H,V], final_state)."""
+    B, T, H, K, V = _dense_shapes(q, k, v, g, g_gamma, initial_state)
     dt = _DTYPES[q.dtype]
     o = torch.empty((B, T, H, V), dtype=q.dtype, device=q.device)
     ht = torch.empty((B, H, K, V), dtype=torch.float32, device=q.device) if output_final_state else None
@@ -167,14 +175,9 @@ def simple_gla_fwd_noalloc(q, k, v, g=None, g_gamma=None, scale=None, initial_st
     workspace, for callers that must not allocate device memory.  Outputs are
     still allocated here (a caller that cannot allocate calls the C entry point
     with its own output buffers).  Calls that may overlap on the GPU race on the
-    shared scratch."""
-    _common_checks(q, k, v, g, g_gamma, initial_state)
-    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
-        raise ValueError("q,k must be [B,T,H,K] and v [B,T,H,V]")
-    B, T, H, K = q.shape
-    V = v.shape[3]
-    if initial_state is not None and tuple(initial_state.shape) != (B, H, K, V):
-        raise ValueError(f"initial_state must be [B,H,K,V] = {(B, H, K, V)}")
+    shared scratch; ``noalloc_status()`` reads the device status word the last call
+    left in it."""
+    B, T, H, K, V = _dense_shapes(q, k, v, g, g_gamma, initial_state)
     o = torch.empty((B, T, H, V), dtype=q.dtype, device=q.device)
     ht = torch.empty((B, H, K, V), dtype=torch.float32, device=q.device) if output_final_state else None
     st = lib().simple_gla_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma),
@@ -685,6 +688,12 @@ def simple_gla_state_carry(log_decay, states, initial_state=None, rank=0):
     _check_cuda("states", states, torch.float32, 4)
     _check_cuda("initial_state", initial_state, torch.float32, 3)
     G, H, K, V = states.shape
+    if tuple(log_decay.shape) != (G, H):
+        raise ValueError(f"log_decay must be [G,H] = {(G, H)}, got {tuple(log_decay.shape)}")
+    if initial_state is not None and tuple(initial_state.shape) != (H, K, V):
+        raise ValueError(f"initial_state must be [H,K,V] = {(H, K, V)}, got {tuple(initial_state.shape)}")
+    if not 0 <= int(rank) <= G:
+        raise ValueError(f"rank must be in [0, {G}], got {rank}")
     out = torch.empty((H, K, V), dtype=torch.float32, device=states.device)
     st = lib().simple_gla_state_carry(_ptr(log_decay), _ptr(states), _ptr(initial_state), _ptr(out), int(rank), H, K,
                                       V, _stream())
@@ -698,6 +707,14 @@ def fused_recurrent_simple_gla(q, k, v, g=None, g_gamma=None, scale=None, initia
     return simple_gla_fused_recurrent(q, k, v, g=g, g_gamma=g_gamma, scale=scale, initial_state=initial_state,
                                       output_final_state=output_final_state, cu_seqlens=cu_seqlens,
                                       state_v_first=state_v_first)
+
+
+def noalloc_status() -> int:
+    """Device status word the last simple_gla_fwd_noalloc call on the current device
+    left in the library's built-in scratch (synchronises the current stream)."""
+    out = ctypes.c_int(-1)
+    raise_for_status(lib().sgla_noalloc_status(ctypes.byref(out), _stream()), "sgla_noalloc_status")
+    return out.value
 
 
 @_on_tensor_device

@@ -19,7 +19,12 @@
 //     of the scratch is always written before it is read;
 //   * the first call on each device looks up the device address of the array
 //     (cudaGetSymbolAddress, with that device current); make that first call
-//     before any stream capture begins.
+//     before any stream capture begins.  The address is kept for the life of the
+//     process: after cudaDeviceReset (or anything else that destroys the device's
+//     primary context) it is stale, and the entry point must not be used again;
+//   * the forward's device status word (a time-out of a bounded device wait, for
+//     instance) sits at the head of the array, where the caller cannot name it:
+//     sgla_noalloc_status reads it back.
 #include <mutex>
 
 #include "launch_status.h"
@@ -70,4 +75,19 @@ extern "C" sgla_status simple_gla_fwd_noalloc(const void *q, const void *k, cons
     // need == 0 means invalid sizes: simple_gla_fwd reports which error.
     return simple_gla_fwd(q, k, v, g, g_gamma, scale, initial_state, o, final_state, B, T, H, K, V, chunk_size,
                           dtype, scratch, kStaticScratchBytes, stream);
+}
+
+extern "C" sgla_status sgla_noalloc_status(int *device_status, void *stream) {
+    if (!device_status) return SGLA_ERR_INVALID_ARGUMENT;
+    void *scratch = nullptr;
+    const sgla_status st = static_scratch(&scratch);
+    if (st != SGLA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int host = -1;
+    cudaError_t e = cudaMemcpyAsync(&host, scratch, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return sgla::cuda_failure(e, "noalloc status read");
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return sgla::cuda_failure(e, "noalloc status sync");
+    *device_status = host;
+    return SGLA_OK;
 }

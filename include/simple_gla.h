@@ -310,13 +310,28 @@ SGLA_API sgla_status simple_gla_decode_step(const void *q, const void *k, const 
  * 16 MiB return SGLA_ERR_WORKSPACE.  All calls on a device share that array, so
  * calls that may run at the same time on the GPU race; order them.  The first
  * call on each device resolves the array's device address (with that device
- * current) and should come before any stream capture.  Allocates nothing.
+ * current) and should come before any stream capture; the address is kept until
+ * the process exits, so after cudaDeviceReset (or any other teardown of the
+ * device's primary context) this entry point must not be called again.
+ * Allocates nothing.  The device status word of the call (SGLA_DEVICE_TIMEOUT when
+ * a bounded device wait gave up and the outputs are invalid) is in that array:
+ * read it with sgla_noalloc_status.
  */
 SGLA_API sgla_status simple_gla_fwd_noalloc(const void *q, const void *k, const void *v,
                                             const float *g, const float *g_gamma, float scale,
                                             const float *initial_state, void *o, float *final_state,
                                             int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
                                             int chunk_size, sgla_dtype dtype, void *stream);
+
+/*
+ * Device status word (SGLA_DEVICE_OK or SGLA_DEVICE_*) left by the last
+ * simple_gla_fwd_noalloc call on the current device, read from the library's
+ * built-in scratch.  Synchronises `stream`.  The article has no counterpart: it is
+ * the sgla_workspace_status of the entry point without a workspace.  Returns SGLA_OK
+ * and fills *device_status, SGLA_ERR_INVALID_ARGUMENT for a NULL pointer, or
+ * SGLA_ERR_CUDA.
+ */
+SGLA_API sgla_status sgla_noalloc_status(int *device_status, void *stream);
 
 /*
  * Exchange step of one long sequence split along time across G ranks (each rank holds

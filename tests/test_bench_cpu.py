@@ -80,3 +80,22 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank_0():
     assert len(lines) == 1
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+
+
+def test_step_time_is_the_median_with_p10_p90():
+    xs = [5.0, 1.0, 3.0, 2.0, 4.0]
+    assert bench.percentile(xs, 50) == 3.0
+    assert bench.percentile(xs, 0) == 1.0 and bench.percentile(xs, 100) == 5.0
+    assert math.isclose(bench.percentile(xs, 10), 1.4) and math.isclose(bench.percentile(xs, 90), 4.6)
+
+
+def test_secondary_workloads_end_with_the_hot_path_ones():
+    order = bench.secondary_order("long_gamma")
+    assert "long_gamma" not in order and set(order) == set(WORKLOADS) - {"long_gamma"}
+    assert order[-4:] == ["tiny_fp32", "dense_prefill", "varlen_prefill", "decode"]
+    r = dict(value=1.2345678e7, unit="tokens/s", ms_per_step=0.5, ms_p10=0.4, ms_p90=0.6,
+             roofline=dict(bound="hbm", frac=0.5), call_roofline_frac=0.4,
+             dominant_kernel=dict(name="chunk_output_tc", avg_ms=0.3), gpu_launches=10,
+             clocks=dict(reasons=[], sm_mhz=1965.0))
+    c = bench.compact(r)
+    assert c["frac"] == 0.5 and c["kernel"] == "chunk_output_tc" and len(json.dumps(c)) < 300

@@ -15,7 +15,7 @@ import torch
 import gated_linear_attention_local_b200 as sg
 import oracle
 from gated_linear_attention_local_b200.workloads import make_workload, random_cotangents, random_inputs
-from parity_utils import TOL, compare_grads, host, to_dev
+from parity_utils import TOL, compare_grads, host, oracle_bwd, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -37,8 +37,7 @@ def _gpu(inp, do, dht, scale=None, cu=None, chunk_size=64):
 
 
 def _oracle(inp, do, dht, scale=None, cu=None):
-    return oracle.simple_gla_bwd(inp["q"], inp["k"], inp["v"], do, g=inp["g"], g_gamma=inp["g_gamma"], scale=scale,
-                                 initial_state=inp["h0"], dht=dht, cu_seqlens=cu)
+    return oracle_bwd(inp, do, dht, scale=scale, cu=cu)
 
 
 DENSE = [

@@ -15,7 +15,7 @@ import torch
 import gated_linear_attention_local_b200 as sg
 import oracle
 from gated_linear_attention_local_b200.workloads import random_cotangents, random_inputs
-from parity_utils import TOL, assert_close, compare_grads, host, to_dev
+from parity_utils import TOL, assert_close, compare_grads, host, oracle_bwd, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -33,8 +33,7 @@ def _run(inp, do, dht, scale=None, cu=None):
                                             g_gamma=dev["g_gamma"], scale=scale, initial_state=dev["h0"],
                                             dht=to_dev(dht), cu_seqlens=to_dev(cu))
     torch.cuda.synchronize()
-    ref = oracle.simple_gla_bwd(inp["q"], inp["k"], inp["v"], do, g=inp["g"], g_gamma=inp["g_gamma"], scale=scale,
-                                initial_state=inp["h0"], dht=dht, cu_seqlens=cu)
+    ref = oracle_bwd(inp, do, dht, scale=scale, cu=cu)
     return gpu, ref
 
 

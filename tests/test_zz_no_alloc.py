@@ -5,8 +5,11 @@ memory (e.g. a plugin inside a runtime that owns the GPU memory pool); it draws
 its scratch from a fixed array inside the library.  Here it is called twice in a
 row through the C ABI -- with different inputs, so stale scratch from the first
 call could not hide a fault in the second -- and each result is compared with
-simple_gla_fwd on the same inputs, within the parity tolerance of the other GPU
-tests.  This file is collected last on purpose.
+simple_gla_fwd on the same inputs and with the fp64 oracle, within the parity
+tolerance of the other GPU tests; the status word it leaves in the built-in
+scratch must read clean.  The Python wrapper is checked too: without a gate and
+without a final state, and refusing mis-shaped gates before anything is launched.
+This file is collected last on purpose.
 """
 import ctypes
 
@@ -16,7 +19,7 @@ import torch
 import gated_linear_attention_local_b200 as sg
 from gated_linear_attention_local_b200 import _lib as L
 from gated_linear_attention_local_b200.workloads import random_inputs
-from parity_utils import TOL, assert_close, host
+from parity_utils import TOL, assert_close, host, oracle_fwd
 
 pytestmark = pytest.mark.gpu
 
@@ -47,8 +50,35 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         o_ws, ht_ws = sg.simple_gla_fwd(d["q"], d["k"], d["v"], g=d["g"], g_gamma=d["g_gamma"],
                                         initial_state=d["h0"], output_final_state=True)
         torch.cuda.synchronize()
+        assert sg.noalloc_status() == 0
         assert_close(host(o_na), host(o_ws), TOL[dt], "o")
         assert_close(host(ht_na), host(ht_ws), TOL[dt], "final_state")
+        ro, rht = oracle_fwd(inp)
+        assert_close(host(o_na), ro, TOL[dt], "o vs oracle")
+        assert_close(host(ht_na), rht, TOL[dt], "final_state vs oracle")
+
+
+@pytest.mark.skipif(not torch.cuda.is_available(), reason="no CUDA device")
+def test_noalloc_python_wrapper_without_gate_or_final_state():
+    inp = random_inputs(1, 200, 2, 128, 64, torch.bfloat16, gate="none", h0=False, seed=13)
+    d = {k_: (v_.cuda() if v_ is not None else None) for k_, v_ in inp.items()}
+    o, ht = sg.simple_gla_fwd_noalloc(d["q"], d["k"], d["v"], output_final_state=False)
+    assert ht is None
+    o_ws, _ = sg.simple_gla_fwd(d["q"], d["k"], d["v"])
+    torch.cuda.synchronize()
+    assert sg.noalloc_status() == 0
+    assert_close(host(o), host(o_ws), TOL[torch.bfloat16], "o")
+    ro, _ = oracle_fwd(inp, final=False)
+    assert_close(host(o), ro, TOL[torch.bfloat16], "o vs oracle")
+
+
+@pytest.mark.skipif(not torch.cuda.is_available(), reason="no CUDA device")
+def test_noalloc_python_wrapper_refuses_misshaped_gates():
+    q = torch.zeros(1, 64, 2, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        sg.simple_gla_fwd_noalloc(q, q, q, g=torch.zeros(1, 32, 2, device="cuda"))
+    with pytest.raises(ValueError):
+        sg.simple_gla_fwd_noalloc(q, q, q, g_gamma=torch.zeros(3, device="cuda"))
 
 
 @pytest.mark.skipif(not torch.cuda.is_available(), reason="no CUDA device")
