@@ -114,13 +114,23 @@ Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t 
     if (p.tc) {
         // One CTA per (segment, head, V tile), one CTA per SM, each walking its
         // segment's steps in order; segments other than the last of a sequence also
-        // cost a state pass (about a third of a walk step per step).  Every segment
-        // pays a fixed cost of about two steps (set-up, state in / out, carry).  Pick
-        // the number of segments per sequence that minimises waves x (steps + 2) for
-        // both kernels, with at least 4 steps per segment.
+        // pay a state pass that re-reads their k and v.  The time of each kernel is
+        // the larger of its step chain (waves x steps x the measured time of one
+        // step, plus a fixed cost of about two steps per segment) and its HBM bytes
+        // at the sustained bandwidth; pick the number of segments per sequence that
+        // minimises the sum, with at least 4 steps per segment.
         const int64_t nt = varlen ? std::max<int64_t>(1, (T / std::max<int64_t>(N, 1) + C - 1) / C)
                                   : std::max<int64_t>(1, (T + C - 1) / C);
-        const int64_t units = std::max<int64_t>(1, N * H * tc_path_vtiles((int)K, (int)V));
+        const int vt = tc_path_vtiles((int)K, (int)V);
+        const int64_t units = std::max<int64_t>(1, N * H * vt);
+        const int64_t state_units = std::max<int64_t>(1, N * H * (V / 64) * (K / 128));
+        // measured per-step times (us) of the walk and of the state pass on B200
+        const double t_walk = K == 128 ? (V / vt == 128 ? 3.2 : 2.6) : (K == 256 ? 3.0 : 6.0);
+        const double t_state = 0.9 * (double)(K / 128);
+        const double bw = 6.0e6;  // sustained HBM bytes per us
+        const double tok = (double)(varlen ? T : N * T);
+        const double walk_bytes = tok * (double)H * (double)(2 * K + 2 * V) * 2.0;
+        const double kv_bytes = tok * (double)H * (double)(K + V) * 2.0;
         double best = 1e300;
         L = nt;
         const int64_t min_l = std::min<int64_t>(nt, 4);
@@ -128,8 +138,14 @@ Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t 
             const int64_t l = (nt + ns - 1) / ns, ns_eff = (nt + l - 1) / l;
             if (l < min_l) break;
             const double waves_walk = (double)((units * ns_eff + 147) / 148);
-            const double waves_state = (double)((units * (ns_eff - 1) + 147) / 148);
-            const double cost = (waves_walk + 0.35 * waves_state) * (double)(l + 2);
+            const double t_w = std::max(waves_walk * (double)(l + 2) * t_walk, walk_bytes / bw);
+            double t_s = 0.0;
+            if (ns_eff > 1) {
+                const double waves_state = (double)((state_units * (ns_eff - 1) + 147) / 148);
+                t_s = std::max(waves_state * (double)(l + 1) * t_state,
+                               kv_bytes * (double)(ns_eff - 1) / (double)ns_eff / bw);
+            }
+            const double cost = t_w + t_s;
             if (cost < best - 1e-9) {
                 best = cost;
                 L = l;

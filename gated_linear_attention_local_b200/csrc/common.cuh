@@ -30,6 +30,12 @@ constexpr float kRcpLn2 = 1.4426950408889634f;
 // the substitution changes no result at fp32 resolution.
 constexpr float kMinLogGate = -80.f;
 
+// Largest decay (log2 units) across one 32-token tile of a chunk for which the
+// tensor-core walk factors the intra-chunk decay through the tile's last token
+// (factors between 2^-64 and 2^64, far inside the fp32 / bf16 range); chunks with a
+// larger span, or a positive log gate, take the exact per-element decay.
+constexpr float kMaxTileSpan = 64.f;
+
 enum GateMode : int { kGateNone = 0, kGatePerToken = 1, kGatePerHead = 2 };
 
 // Device status word at the head of the workspace.

@@ -96,6 +96,7 @@ __global__ void __launch_bounds__(256)
 chunk_cumsum_kernel(const float *__restrict__ g, float *__restrict__ gcum, int *__restrict__ gpos,
                     SeqLayout lay) {
     __shared__ float tile[kCumsumMaxC][33];
+    __shared__ int sflag[32];
     if (device_failed(lay)) return;
     int n, c;
     if (!locate_chunk(lay, blockIdx.x, n, c)) return;
@@ -137,7 +138,7 @@ chunk_cumsum_kernel(const float *__restrict__ g, float *__restrict__ gcum, int *
             }
         }
         positive = __any_sync(0xffffffffu, positive);
-        if (gpos && lane == 0) gpos[(int64_t)blockIdx.x * H + h0 + j] = positive ? 1 : 0;
+        if (lane == 0) sflag[j] = positive ? 1 : 0;
         float incl = run;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -152,6 +153,15 @@ chunk_cumsum_kernel(const float *__restrict__ g, float *__restrict__ gcum, int *
         }
     }
     __syncthreads();
+    // decay span of every 32-token tile (log2 units, first minus last cumulative gate):
+    // past kMaxTileSpan the tensor-core walk takes its exact per-element mask
+    for (int e = threadIdx.x; e < 32 * (kCumsumMaxC / 32); e += blockDim.x) {
+        const int j = e & 31, c = e >> 5;
+        if (j < hw && 32 * c < len && tile[32 * c][j] - tile[min(32 * c + 31, len - 1)][j] > kMaxTileSpan)
+            sflag[j] = 1;
+    }
+    __syncthreads();
+    if (gpos && threadIdx.x < hw) gpos[(int64_t)blockIdx.x * H + h0 + threadIdx.x] = sflag[threadIdx.x];
     for (int e = threadIdx.x; e < len * 32; e += blockDim.x) {
         const int i = e >> 5, j = e & 31;
         if (j < hw) gcum[(ta + i) * H + h0 + j] = tile[i][j];

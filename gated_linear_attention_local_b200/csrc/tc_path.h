@@ -19,5 +19,9 @@ cudaError_t tc_launch_segment_state(const FwdArgs &a, cudaStream_t st);
 // box = 64 (128-byte swizzle) or 32 (64-byte swizzle).
 cudaError_t tc_make_map(CUtensorMap *m, const void *ptr, int64_t tokens, int H, int D, int box);
 cudaError_t tc_launch_chunk_output(const FwdArgs &a, cudaStream_t st);
+// The K = 128 walk (walk_k128.cu): V tiles of 128 columns when V is a multiple of
+// 128, else 64.
+int tc_k128_bv(int V);
+cudaError_t tc_launch_walk_k128(const FwdArgs &a, cudaStream_t st);
 
 }  // namespace sgla

@@ -1,0 +1,153 @@
+// Tile helpers shared by the tcgen05 walk and state kernels: 128-token steps,
+// 128-byte / 64-byte swizzled bf16 tiles in shared memory and their tcgen05
+// descriptors, row scaling, and the step bookkeeping of a segment.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace sgla {
+namespace {
+
+using namespace tc;
+
+constexpr int kStep = 128;                // tokens per step (MMA M)
+constexpr uint32_t kRegion = 128 * 128;   // [128 rows x 64 bf16] 128-byte-swizzled region, bytes
+
+// Swizzle of a tile made of `ROWB`-byte rows (ROWB = 128: 64 bf16 per row, the
+// 128-byte swizzle; ROWB = 64: 32 bf16 per row, the 64-byte swizzle).  The 16-byte
+// chunk c of row r is stored at chunk position phys(r, c) of that row.
+template <int ROWB>
+struct Sw;
+template <>
+struct Sw<128> {
+    static constexpr uint32_t layout = 2;  // descriptor swizzle field
+    static __device__ __forceinline__ int phys(int r, int c) { return (c ^ (r & 7)) & 7; }
+};
+template <>
+struct Sw<64> {
+    static constexpr uint32_t layout = 4;
+    static __device__ __forceinline__ int phys(int r, int c) { return (c ^ ((r >> 1) & 3)) & 3; }
+};
+
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;  // version (sm_100)
+    d |= (uint64_t)layout << 61;
+    return d;
+}
+
+// K-major 128-byte-swizzled operand (Q, K as the B of Q K^T): 8-row atoms 1024 B apart.
+__device__ __forceinline__ uint64_t kdesc(uint32_t saddr) { return sdesc(saddr, 16, 1024, 2); }
+
+__device__ __forceinline__ unsigned char *align1024(unsigned char *p) {
+    return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Scale row `row` (ROWB bytes of bf16) of a swizzled tile by w.  The swizzle only
+// permutes 16-byte chunks inside a row, so a whole-row operation ignores it.  Thread
+// `row` starts at chunk row % chunks so the threads of a quarter-warp hit different
+// bank groups, and every load is issued before any store (src and dst may alias as
+// far as the compiler knows).
+template <int ROWB>
+__device__ __forceinline__ void scale_row(const unsigned char *src, unsigned char *dst, int row, float w) {
+    constexpr int NC = ROWB / 16;
+    const uint4 *s = reinterpret_cast<const uint4 *>(src + row * ROWB);
+    uint4 *d = reinterpret_cast<uint4 *>(dst + row * ROWB);
+    uint4 x[NC];
+#pragma unroll
+    for (int cc = 0; cc < NC; ++cc) x[cc] = s[(cc + row) % NC];
+#pragma unroll
+    for (int cc = 0; cc < NC; ++cc) {
+        uint32_t *xs = reinterpret_cast<uint32_t *>(&x[cc]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&xs[e]);
+            float2 f = __bfloat1622float2(b);
+            xs[e] = pack_bf16(f.x * w, f.y * w);
+        }
+    }
+#pragma unroll
+    for (int cc = 0; cc < NC; ++cc) d[(cc + row) % NC] = x[cc];
+}
+
+// Scale row `row` (128 bytes of bf16) of a tile in place by w, in packed bf16 pairs
+// (w is rounded to bf16 first).  Every load is issued before any store.
+__device__ __forceinline__ void scale_row_bf16x2(unsigned char *tile, int row, float w) {
+    uint4 *d = reinterpret_cast<uint4 *>(tile + row * 128);
+    const __nv_bfloat162 w2 = __float2bfloat162_rn(w);
+    uint4 x[8];
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) x[cc] = d[(cc + row) & 7];
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+        __nv_bfloat162 *b = reinterpret_cast<__nv_bfloat162 *>(&x[cc]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) b[e] = __hmul2(b[e], w2);
+    }
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) d[(cc + row) & 7] = x[cc];
+}
+
+// Scale row `row` (128 bytes of bf16) of a tile in place by w in packed bf16 pairs with
+// one rounding of each product: w = w_hi + w_lo (both bf16) and
+// k w = fma(k, w_hi, k w_lo), so only the term k w_lo (at most 2^-9 of the result) is
+// rounded before the final rounding.  Every load is issued before any store.
+__device__ __forceinline__ void scale_row_2term(unsigned char *tile, int row, float w) {
+    uint4 *d = reinterpret_cast<uint4 *>(tile + row * 128);
+    const __nv_bfloat162 hi = __float2bfloat162_rn(w);
+    const __nv_bfloat162 lo = __float2bfloat162_rn(w - __low2float(hi));
+    uint4 x[8];
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) x[cc] = d[(cc + row) & 7];
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+        __nv_bfloat162 *b = reinterpret_cast<__nv_bfloat162 *>(&x[cc]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) b[e] = __hfma2(b[e], hi, __hmul2(b[e], lo));
+    }
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) d[(cc + row) & 7] = x[cc];
+}
+
+// Store 32 fp32 values as bf16 into row `row`, logical columns [c0, c0 + 32), of a
+// tile of ROWB-byte rows.
+template <int ROWB>
+__device__ __forceinline__ void store_row32_bf16(unsigned char *tile, int row, int c0, const float (&v)[32]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 x;
+        x.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+        x.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+        x.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+        x.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+        *reinterpret_cast<uint4 *>(tile + row * ROWB + (Sw<ROWB>::phys(row, (c0 >> 3) + q) << 4)) = x;
+    }
+}
+
+struct StepSpan {
+    int64_t ta;  // first token of the step
+    int len;     // tokens in the step (<= 128)
+};
+
+__device__ __forceinline__ StepSpan step_span(int64_t t0, int64_t t1, int step) {
+    StepSpan s;
+    s.ta = t0 + (int64_t)step * kStep;
+    s.len = (int)min64(kStep, t1 - s.ta);
+    return s;
+}
+
+__device__ __forceinline__ void record_timeout(const FwdArgs &a) { atomicCAS(a.dev_status, kDevOk, kDevTimeout); }
+
+}  // namespace
+}  // namespace sgla
