@@ -112,7 +112,7 @@ def load_peaks():
 _CSRC_COMMON = ["common.cuh", "kernels.h"]
 KERNEL_SOURCES = {
     "chunk_output_tc": ["chunk_tc.cu", "walk_k128.cu", "tc_ptx.cuh", "tc_tiles.cuh", "tc_path.h"],
-    "segment_state_tc": ["chunk_tc.cu", "tc_ptx.cuh", "tc_tiles.cuh", "tc_path.h"],
+    "segment_state_tc": ["chunk_tc.cu", "state_k128.cu", "tc_ptx.cuh", "tc_tiles.cuh", "tc_path.h"],
     "decode_step": ["decode.cu"],
     "fused_recurrent": ["recurrent.cu"],
     "gla_fused_recurrent": ["recurrent.cu"],

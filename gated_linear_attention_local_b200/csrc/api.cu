@@ -123,11 +123,14 @@ Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t 
                                   : std::max<int64_t>(1, (T + C - 1) / C);
         const int vt = tc_path_vtiles((int)K, (int)V);
         const int64_t units = std::max<int64_t>(1, N * H * vt);
-        const int64_t state_units = std::max<int64_t>(1, N * H * (V / 64) * (K / 128));
-        // measured per-step times (us) of the walk and of the state pass on B200
-        const double t_walk = K == 128 ? (V / vt == 128 ? 3.2 : 2.6) : (K == 256 ? 3.0 : 6.0);
-        const double t_state = 0.9 * (double)(K / 128);
-        const double bw = 6.0e6;  // sustained HBM bytes per us
+        const int64_t state_units =
+            std::max<int64_t>(1, N * H * ((K == 128 && V % 128 == 0) ? V / 128 : (V / 64) * (K / 128)));
+        // measured on B200: per-step times (us) of the walk and of the state pass, and the
+        // HBM bandwidth each reaches with the whole GPU busy (bytes per us)
+        const bool k128 = K == 128 && V % 128 == 0;
+        const double t_walk = K == 128 ? (k128 ? 3.3 : 2.6) : (K == 256 ? 3.0 : 6.0);
+        const double t_state = k128 ? 1.0 : 0.9 * (double)(K / 128);
+        const double bw = 4.9e6, bw_state = k128 ? 5.7e6 : 4.6e6;
         const double tok = (double)(varlen ? T : N * T);
         const double walk_bytes = tok * (double)H * (double)(2 * K + 2 * V) * 2.0;
         const double kv_bytes = tok * (double)H * (double)(K + V) * 2.0;
@@ -143,7 +146,7 @@ Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t 
             if (ns_eff > 1) {
                 const double waves_state = (double)((state_units * (ns_eff - 1) + 147) / 148);
                 t_s = std::max(waves_state * (double)(l + 1) * t_state,
-                               kv_bytes * (double)(ns_eff - 1) / (double)ns_eff / bw);
+                               kv_bytes * (double)(ns_eff - 1) / (double)ns_eff / bw_state);
             }
             const double cost = t_w + t_s;
             if (cost < best - 1e-9) {

@@ -378,7 +378,7 @@ tc_walk_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             g_out = (i < sp.len) ? chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + i, i, h, H) : 0.f;
             const int r = min((i | 31), sp.len - 1);
             gr_out = chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + r, r, h, H);
-            pos_out = per_token ? (a.gpos[(chunk0 + t) * H + h] != 0) : gamma_pos;
+            pos_out = per_token ? (a.gpos[(chunk0 + t) * H + h] == kDecayExact) : gamma_pos;
         };
         auto factor = [&](int t, float g, float gr) -> float {
             return (i < step_span(t0, t1, cb + t).len) ? fast_exp2(fminf(gr - g, 0.f)) : 0.f;
@@ -882,6 +882,7 @@ int tc_path_vtiles(int K, int V) { return K == 128 ? V / tc_k128_bv(V) : V / wal
 cudaError_t tc_launch_segment_state(const FwdArgs &a, cudaStream_t st) {
     cudaError_t e = get_encoder();
     if (e != cudaSuccess) return e;
+    if (a.K == 128 && a.V % 128 == 0) return tc_launch_state_k128(a, st);
     CUtensorMap tk, tv;
     const int64_t tok = total_tokens(a);
     if ((e = make_map(&tk, a.k, tok, a.H, a.K, 64)) != cudaSuccess) return e;

@@ -30,11 +30,15 @@ constexpr float kRcpLn2 = 1.4426950408889634f;
 // the substitution changes no result at fp32 resolution.
 constexpr float kMinLogGate = -80.f;
 
-// Largest decay (log2 units) across one 32-token tile of a chunk for which the
-// tensor-core walk factors the intra-chunk decay through the tile's last token
-// (factors between 2^-64 and 2^64, far inside the fp32 / bf16 range); chunks with a
-// larger span, or a positive log gate, take the exact per-element decay.
+// How the tensor-core walk applies the intra-chunk decay 2^(G~_i - G~_j) of a chunk.
+// Every factor it forms stays between 2^-64 and 2^64, far inside the fp32 / bf16 range:
+//   kDecayStep  the whole chunk spans at most kMaxTileSpan (log2 units): factored
+//               through the chunk's last token;
+//   kDecayTile  every 32-token tile spans at most kMaxTileSpan: factored through each
+//               tile's last token;
+//   kDecayExact otherwise, or with a positive log gate: per element.
 constexpr float kMaxTileSpan = 64.f;
+enum DecayMode : int { kDecayStep = 0, kDecayTile = 1, kDecayExact = 2 };
 
 enum GateMode : int { kGateNone = 0, kGatePerToken = 1, kGatePerHead = 2 };
 

@@ -21,8 +21,8 @@ struct FwdArgs {
     bool o_f32;      // o is written as fp32 whatever the operand dtype (the backward's dq, dk)
     // workspace carve-up
     float *gcum;     // [tokens, H] chunk-local cumsum of g in log2 units (per-token gates)
-    int *gpos;       // [chunks, H] 1 if the chunk needs the exact per-element decay: a positive log
-                     // gate, or a 32-token tile spanning more than kMaxTileSpan (per-token gates)
+    int *gpos;       // [chunks, H] DecayMode of the chunk (per-token gates); kDecayExact also marks
+                     // a positive log gate
     float *seg_dec;  // [max_segs, H] log2 total decay of each segment
     float *seg_state;// [max_segs, H, K, V] segment states (local end state, then entering state)
     int *dev_status; // writable status word (bounded device waits record time-outs here)

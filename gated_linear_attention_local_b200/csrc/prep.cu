@@ -153,15 +153,17 @@ chunk_cumsum_kernel(const float *__restrict__ g, float *__restrict__ gcum, int *
         }
     }
     __syncthreads();
-    // decay span of every 32-token tile (log2 units, first minus last cumulative gate):
-    // past kMaxTileSpan the tensor-core walk takes its exact per-element mask
-    for (int e = threadIdx.x; e < 32 * (kCumsumMaxC / 32); e += blockDim.x) {
-        const int j = e & 31, c = e >> 5;
-        if (j < hw && 32 * c < len && tile[32 * c][j] - tile[min(32 * c + 31, len - 1)][j] > kMaxTileSpan)
-            sflag[j] = 1;
+    // decay mode of the chunk for the tensor-core walk (sflag: 1 = a positive gate):
+    // kDecayStep if the whole chunk spans at most kMaxTileSpan (log2 units, first minus
+    // last cumulative gate), kDecayTile if each 32-token tile does, else kDecayExact
+    if (gpos && threadIdx.x < hw && len > 0) {
+        const int j = threadIdx.x;
+        int mode = (tile[0][j] - tile[len - 1][j] > kMaxTileSpan) ? kDecayTile : kDecayStep;
+        for (int c = 0; 32 * c < len && c < kCumsumMaxC / 32; ++c)
+            if (tile[32 * c][j] - tile[min(32 * c + 31, len - 1)][j] > kMaxTileSpan) mode = kDecayExact;
+        if (sflag[j]) mode = kDecayExact;
+        gpos[(int64_t)blockIdx.x * H + h0 + j] = mode;
     }
-    __syncthreads();
-    if (gpos && threadIdx.x < hw) gpos[(int64_t)blockIdx.x * H + h0 + threadIdx.x] = sflag[threadIdx.x];
     for (int e = threadIdx.x; e < len * 32; e += blockDim.x) {
         const int i = e >> 5, j = e & 31;
         if (j < hw) gcum[(ta + i) * H + h0 + j] = tile[i][j];

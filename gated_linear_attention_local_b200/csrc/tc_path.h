@@ -23,5 +23,7 @@ cudaError_t tc_launch_chunk_output(const FwdArgs &a, cudaStream_t st);
 // 128, else 64.
 int tc_k128_bv(int V);
 cudaError_t tc_launch_walk_k128(const FwdArgs &a, cudaStream_t st);
+// The K = 128, V % 128 == 0 segment-state pass (state_k128.cu).
+cudaError_t tc_launch_state_k128(const FwdArgs &a, cudaStream_t st);
 
 }  // namespace sgla

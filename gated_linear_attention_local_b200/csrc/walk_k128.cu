@@ -21,9 +21,9 @@
 //                      column factor f_j (on V); S is released as soon as it has been
 //                      read, so S(t+1) runs a step ahead;
 //   WG_S  after S(t):  K~(t) rows in place in shared memory; after H(t): Hb <- bf16(H),
-//                      H <- 2^G~_last(t+1) H, or the final state;
-//   WG_O  V_f(t+1) = diag(f) V(t+1) in place once it has landed;
-//         after O1(t): row i of O times scale 2^G~_i in place; after PV(t): the row is
+//                      H <- 2^G~_last(t+1) H, or the final state; then V_f(t+1) = diag(f)
+//                      V(t+1) in place (the column factors of the mask);
+//   WG_O  after O1(t): row i of O times scale 2^G~_i in place; after PV(t): the row is
 //                      read into registers (which releases O for O1(t+1)) and
 //                      written as bf16 into the V(t) stage just consumed, from where one
 //                      TMA store per 64 columns writes the tile.
@@ -184,11 +184,13 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     const float head_l2 = (a.gate_mode == kGatePerHead) ? fmaxf(a.g_gamma[h], kMinLogGate) * kRcpLn2 : 0.f;
     // fp32 outputs (the backward's dq and dk, whose dot products with q and k are summed
     // over the sequence for the gate gradient) keep one rounding per product: exact steps
-    const bool head_exact = a.o_f32 || head_l2 > 0.f || -31.f * head_l2 > kMaxTileSpan;
-    auto step_exact = [&](int t) -> bool {
-        if (a.o_f32 || a.gate_mode != kGatePerToken) return head_exact;
+    const int head_mode = (a.o_f32 || head_l2 > 0.f || -31.f * head_l2 > kMaxTileSpan) ? kDecayExact
+                          : (-127.f * head_l2 > kMaxTileSpan)                          ? kDecayTile
+                                                                                       : kDecayStep;
+    auto step_mode = [&](int t) -> int {
+        if (a.o_f32 || a.gate_mode != kGatePerToken) return head_mode;
         const int64_t chunk = (lay.cu ? (int64_t)lay.chunk_off[n] : (int64_t)n * lay.NT) + cb + t;
-        return a.gpos[chunk * H + h] != 0;
+        return a.gpos[chunk * H + h];
     };
     auto gate_of = [&](int t, int pos) -> float {  // G~ of position pos of local step t (0 past the end)
         const StepSpan sp = step_span(t0, t1, cb + t);
@@ -278,7 +280,7 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                 }
                 mma_commit(b_o1);
                 mma_commit(&empty_q[st]);
-                // H += K~^T V
+                // H += K~^T V_f
                 if (!(ok = wait(b_k, ph1) && wait(&b_vf[st], ph2))) break;
                 tc_fence_after();
                 K128_STAMP(t, 2);
@@ -296,7 +298,7 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                     K128_STAMP(t + 1, 0);
                     issue_S(t + 1);
                 }
-                // O += P V
+                // O += P' V_f
                 if (!(ok = wait(&b_p[st], ph2) && wait(b_o1s, ph1))) break;
                 tc_fence_after();
                 K128_STAMP(t, 3);
@@ -339,14 +341,16 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         struct StepGates {
             float g;       // G~ of row i
             float gr[4];   // G~ of the last token of tile c (for R_i(c)), clipped to the step
-            bool exact;    // exact per-element decay on this step
+            float gl;      // G~ of the step's last token
+            int mode;      // DecayMode of this step
         };
         auto load_step = [&](int t, StepGates &q) {
             const StepSpan sp = step_span(t0, t1, cb + t);
             q.g = gate_of(t, i);
 #pragma unroll
             for (int c = 0; c < 4; ++c) q.gr[c] = gate_of(t, min(32 * c + 31, sp.len - 1));
-            q.exact = (per_token && !a.o_f32) ? a.gpos[(chunk0 + t) * H + h] != 0 : head_exact;
+            q.gl = last_gate(t);
+            q.mode = (per_token && !a.o_f32) ? a.gpos[(chunk0 + t) * H + h] : head_mode;
         };
         const float log2_scale = log2f(a.scale);
         StepGates cur{}, nxt{};
@@ -357,7 +361,7 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         for (int t = 0; t < nsteps; ++t) {
             const StepSpan sp = step_span(t0, t1, cb + t);
             if (t + 1 < nsteps) load_step(t + 1, nxt);  // in flight during this step
-            const bool exact = cur.exact;
+            const bool exact = cur.mode == kDecayExact;
             if (per_token && exact) {
                 const float gri = quarter == 0 ? cur.gr[0] : quarter == 1 ? cur.gr[1] : quarter == 2 ? cur.gr[2] : cur.gr[3];
                 gs[i] = cur.g;
@@ -380,7 +384,9 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                 } else {
                     K128_MASK(t, 3 * c);
                     tmem_ld32(srow + 32 * c, x);
-                    const float grc = c == 0 ? cur.gr[0] : c == 1 ? cur.gr[1] : c == 2 ? cur.gr[2] : cur.gr[3];
+                    // the reference token of the factor: the tile's last (kDecayTile) or the step's last
+                    const float grc = cur.mode == kDecayStep ? cur.gl
+                                      : c == 0 ? cur.gr[0] : c == 1 ? cur.gr[1] : c == 2 ? cur.gr[2] : cur.gr[3];
                     const float R = a.scale * fast_exp2(cur.g - grc);
                     tmem_wait_ld();
                     K128_MASK(t, 3 * c + 1);
@@ -484,17 +490,39 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         // i of V, 2^(G~_last - G~_r(i)) (factored steps), 0 past the sequence end; in
         // place once S(t) has read K(t)
         auto k_tilde = [&](int t) {
-            const int st = t & 1;
+            const int st = t & 1, mode = step_mode(t);
             mbar_wait_idle(b_s, t & 1, abort_flag);
-            const StepSpan sp = step_span(t0, t1, cb + t);
-            const float gref = step_exact(t) ? gate_of(t, i) : gate_of(t, min(i | 31, sp.len - 1));
-            const float w = (i < sp.len) ? fast_exp2(last_gate(t) - gref) : 0.f;
-            unsigned char *kt = sm + C::K0 + st * C::QT;
+            if (mode != kDecayStep) {  // kDecayStep: the whole weight is on V, K stays as loaded
+                const StepSpan sp = step_span(t0, t1, cb + t);
+                const float gref = mode == kDecayExact ? gate_of(t, i) : gate_of(t, min(i | 31, sp.len - 1));
+                const float w = (i < sp.len) ? fast_exp2(last_gate(t) - gref) : 0.f;
+                unsigned char *kt = sm + C::K0 + st * C::QT;
 #pragma unroll 1
-            for (int g = 0; g < 2; ++g) scale_row_2term(kt + g * kRegion, i, w);
-            fence_proxy_async_smem();
+                for (int g = 0; g < 2; ++g) scale_row_2term(kt + g * kRegion, i, w);
+                fence_proxy_async_smem();
+            }
             mbar_arrive(b_k);
+            if (i == 0) K128_STAMP(t, 15);
         };
+        // V_f(t): row i of V(t) times f_i = 2^(G~_r(i) - G~_i) on a factored step, 0 past
+        // the sequence end (exact steps leave V as loaded), before H(t) and P V(t)
+        auto v_factor = [&](int t) {
+            const int st = t & 1;
+            const bool landed = mbar_wait_idle(&full_v[st], (t >> 1) & 1, abort_flag);
+            const int mode = step_mode(t);
+            if (landed && mode != kDecayExact) {
+                const StepSpan sp = step_span(t0, t1, cb + t);
+                const float gref = mode == kDecayStep ? last_gate(t) : gate_of(t, min(i | 31, sp.len - 1));
+                const float f = (i < sp.len) ? fast_exp2(gref - gate_of(t, i)) : 0.f;
+                unsigned char *vt = sm + C::V0 + st * C::VT;
+#pragma unroll 1
+                for (int g = 0; g < C::NG; ++g) scale_row_2term(vt + g * kRegion, i, f);
+                fence_proxy_async_smem();
+            }
+            mbar_arrive(&b_vf[st]);
+            if (i == 0) K128_STAMP(t, 16);
+        };
+        if (nsteps > 0) v_factor(0);
         float lnext = nsteps > 1 ? last_gate(1) : 0.f;  // G~_last of step t+1
         for (int t = 0; t < nsteps; ++t) {
             const float lnext2 = (t + 2 < nsteps) ? last_gate(t + 2) : 0.f;
@@ -519,6 +547,7 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                 tc_fence_before();
                 mbar_arrive(b_hb);
                 if (i == 0) K128_STAMP(t, 10);
+                v_factor(t + 1);
             } else if (last_seg && a.hT) {
 #pragma unroll 1
                 for (int pc = 0; pc < C::NP; ++pc) {
@@ -541,29 +570,19 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         // its named barrier needs all 128 threads every step.
         const int i = threadIdx.x - 256;
         const uint32_t orow = tmem + ((uint32_t)((warp - 8) * 32) << 16) + C::COL_O;
-        // V_f(t): row i of V(t) times f_i = 2^(G~_r(i) - G~_i) on a factored step, 0 past
-        // the sequence end (exact steps leave V as loaded), before H(t) and P V(t)
-        auto v_factor = [&](int t) {
-            const int st = t & 1;
-            const bool landed = mbar_wait_idle(&full_v[st], (t >> 1) & 1, abort_flag);
-            if (landed && !step_exact(t)) {
-                const StepSpan sp = step_span(t0, t1, cb + t);
-                const float f = (i < sp.len) ? fast_exp2(gate_of(t, min(i | 31, sp.len - 1)) - gate_of(t, i)) : 0.f;
-                unsigned char *vt = sm + C::V0 + st * C::VT;
-#pragma unroll 1
-                for (int g = 0; g < C::NG; ++g) scale_row_2term(vt + g * kRegion, i, f);
-                fence_proxy_async_smem();
-            }
-            mbar_arrive(&b_vf[st]);
-        };
-        if (nsteps > 0) v_factor(0);
         float gnext = nsteps > 0 ? gate_of(0, i) : 0.f;
+        bool store_pending = false;  // thread 0: the output store of the previous step still reads its stage
         for (int t = 0; t < nsteps; ++t) {
             const StepSpan sp = step_span(t0, t1, cb + t);
             const float gi = gnext;
             gnext = (t + 1 < nsteps) ? gate_of(t + 1, i) : 0.f;
             // O1 row i times 2^G~_i, in place, before P V accumulates onto it
             mbar_wait_idle(b_o1, t & 1, abort_flag);
+            if (store_pending) {  // thread 0 (overlapped with the products since the store)
+                tma_store_wait_read();
+                mbar_arrive(&empty_v[(t - 1) & 1]);
+                store_pending = false;
+            }
             if (i == 0) K128_STAMP(t, 11);
             tc_fence_after();
             {
@@ -620,9 +639,9 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                             for (int g = 0; g < C::NG; ++g)
                                 tma_store_3d(&to, stage + g * kRegion, v0 + 64 * g, h, (int)sp.ta);
                             tma_store_commit();
-                            tma_store_wait_read();
                         }
-                        mbar_arrive(&empty_v[t & 1]);
+                        K128_STAMP(t, 17);
+                        store_pending = true;  // the stage is released once the store has read it
                     }
                 } else {
                     if (i < sp.len && live) {
@@ -652,7 +671,10 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                 }
                 if (i == 0) mbar_arrive(&empty_v[t & 1]);
             }
-            if (t + 1 < nsteps) v_factor(t + 1);
+        }
+        if (store_pending) {
+            tma_store_wait_read();
+            mbar_arrive(&empty_v[(nsteps - 1) & 1]);
         }
         if (i == 0) tma_store_wait_all();  // every output store has landed before the CTA exits
     }
