@@ -119,7 +119,9 @@ Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t 
         // step, plus a fixed cost of about two steps per segment) and its HBM bytes
         // at the sustained bandwidth; pick the number of segments per sequence that
         // minimises the sum, with at least 4 steps per segment.
-        const int64_t nt = varlen ? std::max<int64_t>(1, (T / std::max<int64_t>(N, 1) + C - 1) / C)
+        // packed batches: the lengths are on the device, so plan for a longest sequence of
+        // 1.75 x the mean, which sets the walk's critical path
+        const int64_t nt = varlen ? std::max<int64_t>(1, (7 * (T / std::max<int64_t>(N, 1)) / 4 + C - 1) / C)
                                   : std::max<int64_t>(1, (T + C - 1) / C);
         const int vt = tc_path_vtiles((int)K, (int)V);
         const int64_t units = std::max<int64_t>(1, N * H * vt);

@@ -16,13 +16,18 @@
 // (a dependent chain of products runs at the full tensor rate; what a step waits for
 // is the warpgroup passes between products, so the order gives each pass the most
 // slack), and three warpgroups:
-//   WG_P  after S(t):  the mask P'_ij = R_i S_ij (j <= i) into P[t&1], the decay of
-//                      scale 2^(G~_i - G~_j) split into a row factor R_i (here) and a
-//                      column factor f_j (on V); S is released as soon as it has been
-//                      read, so S(t+1) runs a step ahead;
-//   WG_S  after S(t):  K~(t) rows in place in shared memory; after H(t): Hb <- bf16(H),
-//                      H <- 2^G~_last(t+1) H, or the final state; then V_f(t+1) = diag(f)
-//                      V(t+1) in place (the column factors of the mask);
+//   WG_P  after S(t):  K~(t) rows in place in shared memory (kDecayStep: none, the whole
+//                      weight is on V), then the mask P'_ij = R_i S_ij (j <= i) into
+//                      P[t&1], the decay scale 2^(G~_i - G~_j) split into a row factor R_i
+//                      (here) and a
+//                      column factor f_j (on V) through a reference token r: the step's
+//                      last token when the whole step spans little decay (kDecayStep),
+//                      else the last token of each 32-token tile (kDecayTile); steps with
+//                      large spans or positive gates, and every fp32-output call, take
+//                      the exact per-element decay (kDecayExact).  S is released as soon
+//                      as it has been read, so S(t+1) runs a step ahead;
+//   WG_S  after H(t):  Hb <- bf16(H), H <- 2^G~_last(t+1) H, or the final state; then
+//                      V_f(t+1) = diag(f) V(t+1) in place;
 //   WG_O  after O1(t): row i of O times scale 2^G~_i in place; after PV(t): the row is
 //                      read into registers (which releases O for O1(t+1)) and
 //                      written as bf16 into the V(t) stage just consumed, from where one
@@ -132,7 +137,7 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     uint64_t *empty_q = bars + 6, *empty_k = bars + 8, *empty_v = bars + 10;  // [2] stage released
     uint64_t *b_s = bars + 12;      // S(t) done
     uint64_t *b_sfree = bars + 13;  // S(t) read by WG_P (128 arrivals)
-    uint64_t *b_k = bars + 14;      // K~(t) written (WG_S, 128 arrivals)
+    uint64_t *b_k = bars + 14;      // K~(t) written (WG_P, 128 arrivals)
     uint64_t *b_p = bars + 15;      // [2] P(t) written into P[t&1] (WG_P, 128 arrivals)
     uint64_t *b_pfree = bars + 17;  // [2] P V(t) done: P[t&1] free
     uint64_t *b_o1 = bars + 19;     // O1(t) done
@@ -315,8 +320,8 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
             mbar_drain(b_drain, 0);
         }
     } else if (warp < 4) {
-        // ---------------------------------------------------------------- WG_P: the mask
-        // Thread i owns row i of S (TMEM lane i).  On a factored step (every chunk whose
+        // ---------------------------------------------------------------- WG_P: K~ and the mask
+        // Thread i owns row i of S (TMEM lane i) and row i of the step's K.  On a factored step (every chunk whose
         // 32-token tiles each span at most kMaxTileSpan of decay and whose gates are
         // <= 0) the decay factors through the last token r(c) of each tile c:
         //   scale 2^(G~_i - G~_j) = R_i(c) f_j,  R_i(c) = scale 2^(G~_i - G~_r(c)),
@@ -371,6 +376,20 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
             mbar_wait_idle(b_s, t & 1, abort_flag);
             if (i == 96) K128_STAMP(t, 5);
             K128_MASK(t, 14);
+            // K~(t): row i of K(t) (read by S(t), now done) times 2^(G~_last - G~_i) on an exact
+            // step, or 2^(G~_last - G~_r(i)) on a tile-factored step (f_i is on row i of V), 0 past
+            // the sequence end; a step-factored step leaves K as loaded (the weight is on V)
+            if (cur.mode != kDecayStep) {
+                const float gref = cur.mode == kDecayExact ? cur.g
+                                   : quarter == 0 ? cur.gr[0] : quarter == 1 ? cur.gr[1] : quarter == 2 ? cur.gr[2] : cur.gr[3];
+                const float w = (i < sp.len) ? fast_exp2(cur.gl - gref) : 0.f;
+                unsigned char *kt = sm + C::K0 + (t & 1) * C::QT;
+#pragma unroll 1
+                for (int g = 0; g < 2; ++g) scale_row_2term(kt + g * kRegion, i, w);
+                fence_proxy_async_smem();
+            }
+            mbar_arrive(b_k);
+            if (i == 0) K128_STAMP(t, 15);
             if (t >= 2) mbar_wait_idle(&b_pfree[t & 1], ((t >> 1) - 1) & 1, abort_flag);  // P V(t-2) done
             tc_fence_after();
             const uint32_t pbuf = prow + (t & 1) * 64;
@@ -486,24 +505,6 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
             tc_fence_before();
             mbar_arrive(b_hb);
         }
-        // K~(t): row i of K(t) times 2^(G~_last - G~_i) (exact steps) or, with f_i on row
-        // i of V, 2^(G~_last - G~_r(i)) (factored steps), 0 past the sequence end; in
-        // place once S(t) has read K(t)
-        auto k_tilde = [&](int t) {
-            const int st = t & 1, mode = step_mode(t);
-            mbar_wait_idle(b_s, t & 1, abort_flag);
-            if (mode != kDecayStep) {  // kDecayStep: the whole weight is on V, K stays as loaded
-                const StepSpan sp = step_span(t0, t1, cb + t);
-                const float gref = mode == kDecayExact ? gate_of(t, i) : gate_of(t, min(i | 31, sp.len - 1));
-                const float w = (i < sp.len) ? fast_exp2(last_gate(t) - gref) : 0.f;
-                unsigned char *kt = sm + C::K0 + st * C::QT;
-#pragma unroll 1
-                for (int g = 0; g < 2; ++g) scale_row_2term(kt + g * kRegion, i, w);
-                fence_proxy_async_smem();
-            }
-            mbar_arrive(b_k);
-            if (i == 0) K128_STAMP(t, 15);
-        };
         // V_f(t): row i of V(t) times f_i = 2^(G~_r(i) - G~_i) on a factored step, 0 past
         // the sequence end (exact steps leave V as loaded), before H(t) and P V(t)
         auto v_factor = [&](int t) {
@@ -526,7 +527,6 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         float lnext = nsteps > 1 ? last_gate(1) : 0.f;  // G~_last of step t+1
         for (int t = 0; t < nsteps; ++t) {
             const float lnext2 = (t + 2 < nsteps) ? last_gate(t + 2) : 0.f;
-            k_tilde(t);
             if (!mbar_wait_idle(b_h, t & 1, abort_flag)) break;
             if (i == 0) K128_STAMP(t, 9);
             tc_fence_after();
