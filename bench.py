@@ -111,7 +111,7 @@ def load_peaks():
 # headers), so that a stored ncu capture stays valid while unrelated files change.
 _CSRC_COMMON = ["common.cuh", "kernels.h"]
 KERNEL_SOURCES = {
-    "chunk_output_tc": ["chunk_tc.cu", "walk_k128.cu", "tc_ptx.cuh", "tc_tiles.cuh", "tc_path.h"],
+    "chunk_output_tc": ["chunk_tc.cu", "walk_k128.cu", "walk_k512.cu", "tc_ptx.cuh", "tc_tiles.cuh", "tc_path.h"],
     "segment_state_tc": ["chunk_tc.cu", "state_k128.cu", "tc_ptx.cuh", "tc_tiles.cuh", "tc_path.h"],
     "decode_step": ["decode.cu"],
     "fused_recurrent": ["recurrent.cu"],

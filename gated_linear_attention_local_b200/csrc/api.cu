@@ -130,7 +130,7 @@ Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t 
         // measured on B200: per-step times (us) of the walk and of the state pass, and the
         // HBM bandwidth each reaches with the whole GPU busy (bytes per us)
         const bool k128 = K == 128 && V % 128 == 0;
-        const double t_walk = K == 128 ? (k128 ? 3.3 : 2.6) : (K == 256 ? 3.0 : 6.0);
+        const double t_walk = K == 128 ? (k128 ? 3.3 : 2.6) : (K == 256 ? 1.8 : 3.0);
         const double t_state = k128 ? 1.0 : 0.9 * (double)(K / 128);
         const double bw = 4.9e6, bw_state = k128 ? 5.7e6 : 4.6e6;
         const double tok = (double)(varlen ? T : N * T);

@@ -36,9 +36,13 @@ constexpr float kMinLogGate = -80.f;
 //               through the chunk's last token;
 //   kDecayTile  every 32-token tile spans at most kMaxTileSpan: factored through each
 //               tile's last token;
-//   kDecayExact otherwise, or with a positive log gate: per element.
+//   kDecayExact otherwise: per element, or (tiles below the diagonal tile) through a row
+//               factor and a column factor that are each at most 1, which holds while
+//               the cumulative gate does not rise;
+//   kDecaySigned a positive log gate in the chunk (the cumulative gate rises): per
+//               element everywhere.
 constexpr float kMaxTileSpan = 64.f;
-enum DecayMode : int { kDecayStep = 0, kDecayTile = 1, kDecayExact = 2 };
+enum DecayMode : int { kDecayStep = 0, kDecayTile = 1, kDecayExact = 2, kDecaySigned = 3 };
 
 enum GateMode : int { kGateNone = 0, kGatePerToken = 1, kGatePerHead = 2 };
 

@@ -21,7 +21,7 @@ struct FwdArgs {
     bool o_f32;      // o is written as fp32 whatever the operand dtype (the backward's dq, dk)
     // workspace carve-up
     float *gcum;     // [tokens, H] chunk-local cumsum of g in log2 units (per-token gates)
-    int *gpos;       // [chunks, H] DecayMode of the chunk (per-token gates); kDecayExact also marks
+    int *gpos;       // [chunks, H] DecayMode of the chunk (per-token gates); kDecaySigned marks
                      // a positive log gate
     float *seg_dec;  // [max_segs, H] log2 total decay of each segment
     float *seg_state;// [max_segs, H, K, V] segment states (local end state, then entering state)

@@ -155,13 +155,14 @@ chunk_cumsum_kernel(const float *__restrict__ g, float *__restrict__ gcum, int *
     __syncthreads();
     // decay mode of the chunk for the tensor-core walk (sflag: 1 = a positive gate):
     // kDecayStep if the whole chunk spans at most kMaxTileSpan (log2 units, first minus
-    // last cumulative gate), kDecayTile if each 32-token tile does, else kDecayExact
+    // last cumulative gate), kDecayTile if each 32-token tile does, else kDecayExact;
+    // kDecaySigned whenever a log gate of the chunk is positive
     if (gpos && threadIdx.x < hw && len > 0) {
         const int j = threadIdx.x;
         int mode = (tile[0][j] - tile[len - 1][j] > kMaxTileSpan) ? kDecayTile : kDecayStep;
         for (int c = 0; 32 * c < len && c < kCumsumMaxC / 32; ++c)
             if (tile[32 * c][j] - tile[min(32 * c + 31, len - 1)][j] > kMaxTileSpan) mode = kDecayExact;
-        if (sflag[j]) mode = kDecayExact;
+        if (sflag[j]) mode = kDecaySigned;
         gpos[(int64_t)blockIdx.x * H + h0 + j] = mode;
     }
     for (int e = threadIdx.x; e < len * 32; e += blockDim.x) {

@@ -25,5 +25,8 @@ int tc_k128_bv(int V);
 cudaError_t tc_launch_walk_k128(const FwdArgs &a, cudaStream_t st);
 // The K = 128, V % 128 == 0 segment-state pass (state_k128.cu).
 cudaError_t tc_launch_state_k128(const FwdArgs &a, cudaStream_t st);
+// The K = 256 / 512 walk (walk_k512.cu): V tiles of tc_k512_bv() columns.
+int tc_k512_bv();
+cudaError_t tc_launch_walk_k512(const FwdArgs &a, cudaStream_t st);
 
 }  // namespace sgla

@@ -24,7 +24,7 @@
 //                      last token when the whole step spans little decay (kDecayStep),
 //                      else the last token of each 32-token tile (kDecayTile); steps with
 //                      large spans or positive gates, and every fp32-output call, take
-//                      the exact per-element decay (kDecayExact).  S is released as soon
+//                      the exact decay (kDecayExact, kDecaySigned).  S is released as soon
 //                      as it has been read, so S(t+1) runs a step ahead;
 //   WG_S  after H(t):  Hb <- bf16(H), H <- 2^G~_last(t+1) H, or the final state; then
 //                      V_f(t+1) = diag(f) V(t+1) in place;
@@ -193,9 +193,10 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                           : (-127.f * head_l2 > kMaxTileSpan)                          ? kDecayTile
                                                                                        : kDecayStep;
     auto step_mode = [&](int t) -> int {
-        if (a.o_f32 || a.gate_mode != kGatePerToken) return head_mode;
+        if (a.gate_mode != kGatePerToken) return head_mode;
         const int64_t chunk = (lay.cu ? (int64_t)lay.chunk_off[n] : (int64_t)n * lay.NT) + cb + t;
-        return a.gpos[chunk * H + h];
+        const int m = a.gpos[chunk * H + h];
+        return a.o_f32 ? max(m, (int)kDecayExact) : m;
     };
     auto gate_of = [&](int t, int pos) -> float {  // G~ of position pos of local step t (0 past the end)
         const StepSpan sp = step_span(t0, t1, cb + t);
@@ -342,7 +343,6 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
             const float gam = (a.gate_mode == kGatePerHead) ? fmaxf(a.g_gamma[h], kMinLogGate) * kRcpLn2 : 0.f;
             gs[i] = a.scale * exp2f((float)i * gam);
         }
-        const int64_t chunk0 = (lay.cu ? (int64_t)lay.chunk_off[n] : (int64_t)n * lay.NT) + cb;
         struct StepGates {
             float g;       // G~ of row i
             float gr[4];   // G~ of the last token of tile c (for R_i(c)), clipped to the step
@@ -355,7 +355,7 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
 #pragma unroll
             for (int c = 0; c < 4; ++c) q.gr[c] = gate_of(t, min(32 * c + 31, sp.len - 1));
             q.gl = last_gate(t);
-            q.mode = (per_token && !a.o_f32) ? a.gpos[(chunk0 + t) * H + h] : head_mode;
+            q.mode = step_mode(t);
         };
         const float log2_scale = log2f(a.scale);
         StepGates cur{}, nxt{};
@@ -366,7 +366,7 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         for (int t = 0; t < nsteps; ++t) {
             const StepSpan sp = step_span(t0, t1, cb + t);
             if (t + 1 < nsteps) load_step(t + 1, nxt);  // in flight during this step
-            const bool exact = cur.mode == kDecayExact;
+            const bool exact = cur.mode >= kDecayExact;
             if (per_token && exact) {
                 const float gri = quarter == 0 ? cur.gr[0] : quarter == 1 ? cur.gr[1] : quarter == 2 ? cur.gr[2] : cur.gr[3];
                 gs[i] = cur.g;
@@ -380,7 +380,7 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
             // step, or 2^(G~_last - G~_r(i)) on a tile-factored step (f_i is on row i of V), 0 past
             // the sequence end; a step-factored step leaves K as loaded (the weight is on V)
             if (cur.mode != kDecayStep) {
-                const float gref = cur.mode == kDecayExact ? cur.g
+                const float gref = cur.mode >= kDecayExact ? cur.g
                                    : quarter == 0 ? cur.gr[0] : quarter == 1 ? cur.gr[1] : quarter == 2 ? cur.gr[2] : cur.gr[3];
                 const float w = (i < sp.len) ? fast_exp2(cur.gl - gref) : 0.f;
                 unsigned char *kt = sm + C::K0 + (t & 1) * C::QT;
@@ -431,7 +431,7 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                             const int j = 32 * c + e;
                             x[e] = (j <= i && j < sp.len) ? gs[i - j] * x[e] : 0.f;
                         }
-                    } else if (c < quarter) {
+                    } else if (c < quarter && cur.mode == kDecayExact) {
                         const float rfac = a.scale * fast_exp2(fminf(cur.g - grc, 0.f));
                         const float4 *f4 = reinterpret_cast<const float4 *>(fs + 32 * c);
 #pragma unroll
@@ -511,7 +511,7 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
             const int st = t & 1;
             const bool landed = mbar_wait_idle(&full_v[st], (t >> 1) & 1, abort_flag);
             const int mode = step_mode(t);
-            if (landed && mode != kDecayExact) {
+            if (landed && mode < kDecayExact) {
                 const StepSpan sp = step_span(t0, t1, cb + t);
                 const float gref = mode == kDecayStep ? last_gate(t) : gate_of(t, min(i | 31, sp.len - 1));
                 const float f = (i < sp.len) ? fast_exp2(gref - gate_of(t, i)) : 0.f;

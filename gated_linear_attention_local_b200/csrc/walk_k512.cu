@@ -1,0 +1,675 @@
+// Tensor-core walk (fused output) for head dims K = 256 and 512, bf16 operands, sm_100a.
+//
+// "Simple GLA in flash-linear-attention: maths and kernels" (xxqk.cn article),
+// sections 1 and 3: inside a chunk the output is the decay-masked q k^T applied to v
+// plus the read-out q h of the state entering the chunk, and the state is carried to
+// the next chunk by one scalar decay and the k^T v of the chunk.  One CTA walks one
+// segment of one head for a V tile of 64 columns, 128 tokens per step; its K x 64 fp32
+// state stays in tensor memory (K/128 blocks of 64 columns) for the whole segment.
+//
+// Q and K are too large to hold a step of them, so they stream through a ring of five
+// 32 KB units, each one 128-wide k slice s of Q or of K (Q_s, K_s), feeding three
+// products before it is released:
+//   O[t&1] += Q_s Hb_s                 (Hb_s: bf16 copy of state block s, shared memory)
+//   S      += Q_s K_s^T                (TMEM, 128 x 128 fp32)
+//   H_s    += K_s^T V_w                (V_w,j = 2^(G~_last - G~_j) v_j)
+// and once S is complete and masked,
+//   O[t&1] += P' V_f                   (P' = R_i S_ij in bf16, written over S)
+// with the decay scale 2^(G~_i - G~_j) split into a row factor R_i (the mask) and a
+// column factor f_j on V (V_f): through the step's last token (kDecayStep: V_f = V_w),
+// through each 32-token tile's last token (kDecayTile), or per element (kDecayExact,
+// kDecaySigned: large spans, positive gates, fp32 outputs; V_f = V).  K is never
+// rewritten; the per-step shared-memory writes are V_w and V_f (16 KB each) and Hb.
+//
+// Warpgroups: WG_P masks S into P' (in place over S); WG_S turns each state block into
+// its bf16 copy and applies the next step's decay to it (Hb <- bf16(H_s),
+// H_s <- 2^G~_last H_s) between the O1 products of consecutive blocks, and prepares
+// V_w and V_f; WG_O rescales the O1 rows by scale 2^G~_i and reads the output rows
+// out (O is double-buffered in tensor memory).  Warp 12 loads the Q/K units and V,
+// warp 13 issues the products (slice by slice, P V last).  Shared memory goes to ring
+// depth: one Hb block and one V_w buffer, whose passes fit between the products that
+// read them.
+//
+// Tensor memory (512 columns): S/P' [0,128), O0 [128,192), O1 [192,256), H [256,
+// 256 + 64 K/128).  Shared memory: Q/K ring 160 KB, Hb 16 KB, V ring 32 KB, V_w 16 KB.
+//
+// Every mbarrier wait is bounded; a wait that gives up marks the CTA aborted, the CTA
+// drains its in-flight copies and products, frees its tensor memory, skips its
+// global writes and records SGLA_DEVICE_TIMEOUT in the workspace status word.
+#include <cudaTypedefs.h>
+
+#include "tc_path.h"
+#include "tc_ptx.cuh"
+#include "tc_tiles.cuh"
+
+namespace sgla {
+
+using namespace tc;
+
+namespace {
+
+// Device tracing (off unless built with -DSGLA_DEVICE_TRACE): SM-clock stamps of the
+// pipeline events of CTA (0, 0), per step, for the read-out function below.
+#ifdef SGLA_DEVICE_TRACE
+__device__ unsigned long long g_k512_trace[64][32];
+#define K512_STAMP(t, ev)                                                                        \
+    do {                                                                                         \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && (t) < 64) g_k512_trace[(t)][(ev)] = clock64(); \
+    } while (0)
+#else
+#define K512_STAMP(t, ev) \
+    do {                  \
+    } while (0)
+#endif
+
+constexpr int kK512Threads = 448;  // warps 0-3 WG_P, 4-7 WG_S, 8-11 WG_O, 12 TMA loads, 13 MMA
+constexpr int kK512BV = 64;
+
+template <int KS>
+struct K512Cfg {
+    static constexpr int NU = 5;                        // Q/K ring: units of one 128-wide k slice of Q or K
+    static constexpr uint32_t UNIT = 2 * kRegion;       // [128 tokens x 128 k] as two 64-k regions
+    static constexpr uint32_t RING = 0;
+    static constexpr uint32_t HB = NU * UNIT;           // Hb: [128 k rows x 64 v] of one state block
+    static constexpr uint32_t V0 = HB + kRegion;        // V ring: 2 x [128 tokens x 64 v] (V_f in place)
+    static constexpr uint32_t VW = V0 + 2 * kRegion;    // V_w [128 tokens x 64 v]
+    static constexpr uint32_t GS = VW + kRegion;        // exact steps: [128] gates, [128] factors
+    static constexpr uint32_t BARS = GS + 2 * 128 * 4;
+    static constexpr uint32_t MISC = BARS + 32 * 8;     // tmem address, abort flag
+    static constexpr uint32_t TOTAL = MISC + 16;
+    static constexpr size_t SMEM = TOTAL + 1024;        // + alignment slack
+    static constexpr uint32_t COL_S = 0, COL_O = 128, COL_H = 256;
+    static constexpr uint32_t COLS = 512;
+    static_assert(KS == 2 || KS == 4, "K = 256 or 512");
+    static_assert(COL_H + KS * kK512BV <= COLS, "tensor memory budget");
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+template <int KS>
+__global__ void __launch_bounds__(kK512Threads, 1)
+tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                    const __grid_constant__ CUtensorMap tv, FwdArgs a) {
+    using C = K512Cfg<KS>;
+    constexpr int BV = kK512BV;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = align1024(smem_raw);
+    const SeqLayout &lay = a.lay;
+    if (device_failed(lay)) return;
+    const int VT = a.V / BV;
+    const int u = blockIdx.x / VT;            // V tiles of one (segment, head) are adjacent
+    const int v0 = (blockIdx.x % VT) * BV;
+    int n, s;
+    if (!locate_segment(lay, u, n, s)) return;
+    const int nseg = seq_segments(lay, n);
+    const int h = blockIdx.y, H = a.H, V = a.V;
+    int64_t t0, t1;
+    seq_span(lay, n, t0, t1);
+    const int nt = (int)((t1 - t0 + kStep - 1) / kStep);
+    const int cb = s * lay.L;
+    const int nsteps = min(cb + lay.L, nt) - cb;
+    const bool last_seg = (s == nseg - 1);
+
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::BARS);
+    uint64_t *full_u = bars + 0, *empty_u = bars + 5;    // [NU] ring unit landed / released
+    uint64_t *full_v = bars + 10, *empty_v = bars + 12;  // [2] V stage landed / released (P V done)
+    uint64_t *b_s = bars + 14;      // S(t) complete
+    uint64_t *b_p = bars + 15;      // P'(t) written over S (WG_P, 128 arrivals)
+    uint64_t *b_o1 = bars + 16;     // O1(t) complete
+    uint64_t *b_o1s = bars + 17;    // O1(t) rescaled (WG_O, 128 arrivals)
+    uint64_t *b_hb = bars + 18;     // Hb holds the next block and its H block is decayed (WG_S, 128 arrivals)
+    uint64_t *b_hbfree = bars + 19; // Hb read by its O1 products
+    uint64_t *b_hdone = bars + 20;  // [KS] H block s of the step complete
+    uint64_t *b_vw = bars + 24;     // V_w(t), V_f(t) ready (WG_S, 128 arrivals)
+    uint64_t *b_pv = bars + 25;     // P V(t) done
+    uint64_t *b_ofree = bars + 26;  // [2] O buffer read out (WG_O, 128 arrivals)
+    uint64_t *b_drain = bars + 28;  // every product retired
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + C::MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + C::MISC + 8);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < 14; ++b) mbar_init(&bars[b], 1);
+        mbar_init(b_s, 1);
+        mbar_init(b_p, 128);
+        mbar_init(b_o1, 1);
+        mbar_init(b_o1s, 128);
+        mbar_init(b_hb, 128);
+        mbar_init(b_hbfree, 1);
+        for (int b = 0; b < KS; ++b) mbar_init(&b_hdone[b], 1);
+        mbar_init(b_vw, 128);
+        mbar_init(b_pv, 1);
+        mbar_init(&b_ofree[0], 128);
+        mbar_init(&b_ofree[1], 128);
+        mbar_init(b_drain, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 13) {
+        tmem_alloc(tmem_slot, C::COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // decay mode of a step; fp32 outputs keep one rounding per product (exact steps)
+    const float head_l2 = (a.gate_mode == kGatePerHead) ? fmaxf(a.g_gamma[h], kMinLogGate) * kRcpLn2 : 0.f;
+    const int head_mode = (a.o_f32 || head_l2 > 0.f || -31.f * head_l2 > kMaxTileSpan) ? kDecayExact
+                          : (-127.f * head_l2 > kMaxTileSpan)                          ? kDecayTile
+                                                                                       : kDecayStep;
+    const int64_t chunk0 = (lay.cu ? (int64_t)lay.chunk_off[n] : (int64_t)n * lay.NT) + cb;
+    auto step_mode = [&](int t) -> int {
+        if (a.gate_mode != kGatePerToken) return head_mode;
+        const int m = a.gpos[(chunk0 + t) * H + h];
+        return a.o_f32 ? max(m, (int)kDecayExact) : m;
+    };
+    auto gate_of = [&](int t, int pos) -> float {  // G~ of position pos of local step t (0 past the end)
+        const StepSpan sp = step_span(t0, t1, cb + t);
+        return (pos < sp.len) ? chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + pos, pos, h, H) : 0.f;
+    };
+    auto last_gate = [&](int t) -> float {
+        const StepSpan sp = step_span(t0, t1, cb + t);
+        return chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + sp.len - 1, sp.len - 1, h, H);
+    };
+
+    if (warp == 12) {
+        // ---------------------------------------------------------------- TMA loads
+        // Unit x of the ring is the Q (x even) or K (x odd) slice sl of step t, q = x / 2 =
+        // t KS + sl, in slot x % NU.  V(t) goes out just before unit 2 t KS: its stage is
+        // freed by P V(t-2), which retires before the unit that load waits for.
+        if (lane == 0) {
+            prefetch_tmap(&tq);
+            prefetch_tmap(&tk);
+            prefetch_tmap(&tv);
+            int issued = 0, issued_v = 0;
+            const int total = nsteps * KS * 2;
+            for (int x = 0; x < total; ++x) {
+                const int q = x >> 1, t = q / KS, sl = q - t * KS, slot = x % C::NU;
+                const int tok = (int)(t0 + (int64_t)(cb + t) * kStep);
+                if (sl == 0 && (x & 1) == 0) {
+                    const int vs = t & 1;
+                    if (t >= 2 && !mbar_wait(&empty_v[vs], ((t >> 1) - 1) & 1, abort_flag)) break;
+                    K512_STAMP(t, 28);
+                    mbar_arrive_expect_tx(&full_v[vs], kRegion);
+                    tma_load_3d(sm + C::V0 + vs * kRegion, &tv, &full_v[vs], v0, h, tok);
+                    issued_v = t + 1;
+                }
+                if (x >= C::NU && !mbar_wait(&empty_u[slot], ((x / C::NU) - 1) & 1, abort_flag)) break;
+                if (sl == 0 && (x & 1) == 0) K512_STAMP(t, 27);
+                if (sl == KS - 1 && (x & 1)) K512_STAMP(t, 29);
+                const CUtensorMap *m = (x & 1) ? &tk : &tq;
+                unsigned char *dst = sm + C::RING + slot * C::UNIT;
+                mbar_arrive_expect_tx(&full_u[slot], C::UNIT);
+                tma_load_3d(dst, m, &full_u[slot], 128 * sl, h, tok);
+                tma_load_3d(dst + kRegion, m, &full_u[slot], 128 * sl + 64, h, tok);
+                issued = x + 1;
+            }
+            if (*abort_flag) {
+                for (int x = max(0, issued - C::NU); x < issued; ++x) mbar_drain(&full_u[x % C::NU], (x / C::NU) & 1);
+                for (int t = max(0, issued_v - 2); t < issued_v; ++t) mbar_drain(&full_v[t & 1], (t >> 1) & 1);
+            }
+        }
+    } else if (warp == 13) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idS = idesc_bf16_f32(128, 128, false, false);
+            const uint32_t idO = idesc_bf16_f32(128, BV, false, true);
+            const uint32_t idH = idesc_bf16_f32(128, BV, true, true);
+            const uint32_t sbase = smem_u32(sm);
+            auto mn64 = [&](uint32_t addr) { return sdesc(addr, 1024, 1024, 2); };  // one 64-column group
+            auto wait = [&](uint64_t *bar, uint32_t ph) { return mbar_wait(bar, ph, abort_flag); };
+            bool ok = true;
+            for (int t = 0; ok && t < nsteps; ++t) {
+                const uint32_t od = tmem + C::COL_O + (t & 1) * BV;
+#pragma unroll 1
+                // products of slice s: O1 += Q_s Hb_s; S += Q_s K_s^T; H_s += K_s^T V_w.  Slice 0
+                // issues O1, H, S (S holds P'(t-1) until P V(t-1) is done); the others S, O1, H,
+                // which puts S(t) complete early in the last slice (the mask overlaps the rest
+                // of the step) and leaves the state pass of the next block the time of S and H
+#pragma unroll 1
+                for (int sl = 0; sl < KS; ++sl) {
+                    const int q = t * KS + sl, use = q;
+                    const int xq = 2 * q, xk = 2 * q + 1;
+                    const int sq = xq % C::NU, sk = xk % C::NU;
+                    const uint32_t qa = sbase + C::RING + sq * C::UNIT, ka = sbase + C::RING + sk * C::UNIT;
+                    if (sl == 0) K512_STAMP(t, 0);
+                    if (!(ok = wait(&full_u[sq], (xq / C::NU) & 1))) break;
+                    K512_STAMP(t, sl == 0 ? 1 : 4 + sl);
+                    auto issue_o1 = [&]() -> bool {
+                        if (!wait(b_hb, use & 1)) return false;
+                        if (sl == 0 && t >= 2 && !wait(&b_ofree[t & 1], ((t >> 1) - 1) & 1)) return false;
+                        if (sl == 0) K512_STAMP(t, 2);
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
+                            mma_bf16(od, kdesc(qa + off), mn64(sbase + C::HB + kk * 2048), idO, (sl > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit(b_hbfree);
+                        if (sl == KS - 1) mma_commit(b_o1);
+                        return true;
+                    };
+                    auto issue_s = [&]() {
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
+                            mma_bf16(tmem + C::COL_S, kdesc(qa + off), kdesc(ka + off), idS, (sl > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        if (sl == KS - 1) mma_commit(b_s);
+                    };
+                    auto issue_h = [&]() {
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_bf16(tmem + C::COL_H + sl * BV, sdesc(ka + kk * 2048, kRegion, 1024, 2),
+                                     mn64(sbase + C::VW + kk * 2048), idH, 1u);
+                        mma_commit(&b_hdone[sl]);
+                    };
+                    if (sl == 0) {
+                        if (!(ok = issue_o1())) break;
+                        if (!(ok = wait(&full_u[sk], (xk / C::NU) & 1))) break;
+                        if (!(ok = wait(b_vw, t & 1))) break;
+                        K512_STAMP(t, 4);
+                        issue_h();
+                        if (t >= 1 && !(ok = wait(b_pv, (t - 1) & 1))) break;
+                        K512_STAMP(t, 3);
+                        issue_s();
+                        mma_commit(&empty_u[sq]);
+                    } else {
+                        if (!(ok = wait(&full_u[sk], (xk / C::NU) & 1))) break;
+                        issue_s();
+                        if (!(ok = issue_o1())) break;
+                        mma_commit(&empty_u[sq]);
+                        issue_h();
+                    }
+                    mma_commit(&empty_u[sk]);
+                }
+                if (!ok) break;
+                K512_STAMP(t, 8);
+                // O += P' V_f
+                if (!(ok = wait(b_p, t & 1))) break;
+                K512_STAMP(t, 9);
+                if (!(ok = wait(b_o1s, t & 1))) break;
+                K512_STAMP(t, 10);
+                tc_fence_after();
+                const uint32_t vf = sbase + C::V0 + (t & 1) * kRegion;
+#pragma unroll
+                for (int jj = 0; jj < kStep / 16; ++jj)
+                    mma_bf16_tmem_a(od, tmem + C::COL_S + jj * 8, mn64(vf + jj * 2048), idO, 1u);
+                mma_commit(b_pv);
+                mma_commit(&empty_v[t & 1]);
+                K512_STAMP(t, 11);
+            }
+            mma_commit(b_drain);
+            mbar_drain(b_drain, 0);
+        }
+    } else if (warp < 4) {
+        // ---------------------------------------------------------------- WG_P: the mask
+        // Thread i owns row i of S (TMEM lane i).  Factored steps: P'_ij = R_i(c) S_ij,
+        // R_i(c) = scale 2^(G~_i - G~_r) (r: the step's last token, or the last token of
+        // tile c), with the column factor on V.  kDecayExact: per element on the
+        // diagonal tile and through at-most-1 row and column factors below it (the
+        // cumulative gate does not rise); kDecaySigned: per element.  P' tile c (16
+        // packed columns at 16c) lands on S tile c/2, which this thread has already
+        // read (tensor memory rows are per thread).  Tiles above the diagonal are 0.
+        const int i = threadIdx.x, quarter = warp;
+        const uint32_t srow = tmem + ((uint32_t)(quarter * 32) << 16) + C::COL_S;
+        float *gs = reinterpret_cast<float *>(sm + C::GS);
+        float *fs = gs + 128;
+        const bool per_token = a.gate_mode == kGatePerToken;
+        if (!per_token) gs[i] = a.scale * exp2f((float)i * head_l2);  // per-head decay table
+        struct StepGates {
+            float g, gl, gr[4];
+            int mode;
+        };
+        auto load_step = [&](int t, StepGates &q) {
+            const StepSpan sp = step_span(t0, t1, cb + t);
+            q.g = gate_of(t, i);
+            q.gl = last_gate(t);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) q.gr[c] = gate_of(t, min(32 * c + 31, sp.len - 1));
+            q.mode = step_mode(t);
+        };
+        const float log2_scale = log2f(a.scale);
+        StepGates cur{}, nxt{};
+        if (nsteps > 0) load_step(0, cur);
+        named_sync(1, 128);
+        // no early exit from this loop: its named barriers need all 128 threads every
+        // step; once the CTA has given up, every wait returns at once
+        for (int t = 0; t < nsteps; ++t) {
+            const StepSpan sp = step_span(t0, t1, cb + t);
+            if (t + 1 < nsteps) load_step(t + 1, nxt);
+            const bool exact = cur.mode >= kDecayExact;
+            if (per_token && exact) {
+                const float gri = quarter == 0 ? cur.gr[0] : quarter == 1 ? cur.gr[1] : quarter == 2 ? cur.gr[2] : cur.gr[3];
+                gs[i] = cur.g;
+                fs[i] = (i < sp.len) ? fast_exp2(gri - cur.g) : 0.f;
+            }
+            named_sync(1, 128);  // this step's gates and factors in place
+            mbar_wait(b_s, t & 1, abort_flag);
+            if (i == 0) K512_STAMP(t, 12);
+            tc_fence_after();
+            const float lsc = cur.g + log2_scale;  // per element: P'_ij = 2^(lsc - G~_j) S_ij
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                float x[32];
+                if (c > quarter) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[e] = 0.f;
+                } else {
+                    tmem_ld32(srow + 32 * c, x);
+                    const float grc = cur.mode == kDecayStep ? cur.gl
+                                      : c == 0 ? cur.gr[0] : c == 1 ? cur.gr[1] : c == 2 ? cur.gr[2] : cur.gr[3];
+                    const float R = a.scale * fast_exp2(cur.g - grc);
+                    tmem_wait_ld();
+                    if (!exact) {
+                        if (c < quarter && sp.len == kStep) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) x[e] *= R;
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) {
+                                const int j = 32 * c + e;
+                                x[e] = (j <= i && j < sp.len) ? R * x[e] : 0.f;
+                            }
+                        }
+                    } else if (!per_token) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int j = 32 * c + e;
+                            x[e] = (j <= i && j < sp.len) ? gs[i - j] * x[e] : 0.f;
+                        }
+                    } else if (c < quarter && cur.mode == kDecayExact) {
+                        const float4 *f4 = reinterpret_cast<const float4 *>(fs + 32 * c);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float4 f = f4[e];
+                            x[4 * e + 0] = (R * x[4 * e + 0]) * f.x;
+                            x[4 * e + 1] = (R * x[4 * e + 1]) * f.y;
+                            x[4 * e + 2] = (R * x[4 * e + 2]) * f.z;
+                            x[4 * e + 3] = (R * x[4 * e + 3]) * f.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int j = 32 * c + e;
+                            x[e] = (j <= i && j < sp.len) ? fast_exp2(lsc - gs[j]) * x[e] : 0.f;
+                        }
+                    }
+                }
+                // P' tile c goes to columns 16c.. (S tile c/2, already read by this thread)
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
+                tmem_st16(srow + 16 * c, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(b_p);
+            if (i == 0) K512_STAMP(t, 13);
+            named_sync(1, 128);  // every row is done with this step's gates and factors
+            cur = nxt;
+        }
+    } else if (warp < 8) {
+        // ---------------------------------------------------------------- WG_S: state blocks, V_w and V_f
+        // Thread i owns row i of every 128-row state block (k = 128 s + i) and row i
+        // (token i) of the step's V.
+        const int i = threadIdx.x - 128;
+        const uint32_t hrow = tmem + ((uint32_t)((warp - 4) * 32) << 16) + C::COL_H;
+        const int64_t KV = (int64_t)a.K * V;
+        // V(t) -> V_w = w ⊙ V (own buffer) and V_f = f ⊙ V (in place), 0 past the end;
+        // each product of a bf16 pair with an fp32 weight is rounded once
+        auto v_pass = [&](int t) {
+            const int st = t & 1;
+            if (mbar_wait(&full_v[st], (t >> 1) & 1, abort_flag)) {
+                const int mode = step_mode(t);
+                const StepSpan sp = step_span(t0, t1, cb + t);
+                const float gi = gate_of(t, i);
+                const float w = (i < sp.len) ? fast_exp2(last_gate(t) - gi) : 0.f;
+                const float f = mode == kDecayStep ? w
+                                : (i < sp.len)     ? fast_exp2(gate_of(t, min(i | 31, sp.len - 1)) - gi)
+                                                   : 0.f;
+                const bool write_f = mode < kDecayExact;
+                const __nv_bfloat162 wh = __float2bfloat162_rn(w), wl = __float2bfloat162_rn(w - __low2float(wh));
+                const __nv_bfloat162 fh = __float2bfloat162_rn(f), fl = __float2bfloat162_rn(f - __low2float(fh));
+                uint4 *vrow = reinterpret_cast<uint4 *>(sm + C::V0 + st * kRegion + i * 128);
+                uint4 *wrow = reinterpret_cast<uint4 *>(sm + C::VW + i * 128);
+                // thread i starts at chunk i % 8, so a quarter-warp's 16-byte accesses fall in
+                // different bank groups (the row is scaled as a whole, the swizzle is irrelevant)
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const int cc = (c8 + i) & 7;
+                    const uint4 x = vrow[cc];
+                    uint4 xw, xf;
+                    const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&x);
+                    __nv_bfloat162 *bw = reinterpret_cast<__nv_bfloat162 *>(&xw);
+                    __nv_bfloat162 *bf = reinterpret_cast<__nv_bfloat162 *>(&xf);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        bw[e] = __hfma2(b[e], wh, __hmul2(b[e], wl));
+                        bf[e] = __hfma2(b[e], fh, __hmul2(b[e], fl));
+                    }
+                    wrow[cc] = xw;
+                    if (write_f) vrow[cc] = xf;
+                }
+                fence_proxy_async_smem();
+            }
+            mbar_arrive(b_vw);
+        };
+        // block sl of the state entering step t (x: its row i, 64 columns in two pieces)
+        // -> Hb (bf16) and H block sl (times the decay of step t)
+        auto block_out = [&](int sl, int pc, float (&x)[32], float gam) {
+            store_row32_bf16<128>(sm + C::HB, i, 32 * pc, x);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] *= gam;
+            tmem_st32(hrow + sl * BV + 32 * pc, x);
+        };
+        auto block_done = [&]() {
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(b_hb);
+        };
+        bool ok = true;
+        if (nsteps > 0) {  // step 0: the state entering the segment
+            const float *src = nullptr;
+            if (s == 0) src = a.h0 ? a.h0 + ((int64_t)n * H + h) * KV : nullptr;
+            else src = a.seg_state + ((int64_t)(u - 1) * H + h) * KV;
+            const float gam = exp2f(last_gate(0));
+#pragma unroll 1
+            for (int sl = 0; sl < KS; ++sl) {
+                if (sl >= 1 && !(ok = mbar_wait(b_hbfree, (sl - 1) & 1, abort_flag))) break;
+#pragma unroll 1
+                for (int pc = 0; pc < 2; ++pc) {
+                    float x[32];
+                    if (src) {
+                        const float4 *p4 =
+                            reinterpret_cast<const float4 *>(src + (int64_t)(128 * sl + i) * V + v0 + 32 * pc);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float4 f = p4[e];
+                            x[4 * e] = f.x; x[4 * e + 1] = f.y; x[4 * e + 2] = f.z; x[4 * e + 3] = f.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) x[e] = 0.f;
+                    }
+                    block_out(sl, pc, x, gam);
+                }
+                block_done();
+                if (sl == 0) v_pass(0);
+            }
+        }
+        // later steps: block sl once H_sl of the previous step is done and Hb has been read
+        // by the O1 products of the block before; V_w(t) once H(t-1) is done
+        for (int t = 1; ok && t < nsteps; ++t) {
+            const float gam = exp2f(last_gate(t));  // decay of step t, applied to the entering state
+#pragma unroll 1
+            for (int sl = 0; sl < KS; ++sl) {
+                const int use = t * KS + sl;
+                if (!(ok = mbar_wait(&b_hdone[sl], (t - 1) & 1, abort_flag))) break;
+                if (!(ok = mbar_wait(b_hbfree, (use - 1) & 1, abort_flag))) break;
+                if (i == 0) K512_STAMP(t, 14 + 2 * sl);
+                tc_fence_after();
+#pragma unroll 1
+                for (int pc = 0; pc < 2; ++pc) {
+                    float x[32];
+                    tmem_ld32(hrow + sl * BV + 32 * pc, x);
+                    tmem_wait_ld();
+                    block_out(sl, pc, x, gam);
+                }
+                block_done();
+                if (i == 0) K512_STAMP(t, 15 + 2 * sl);
+                if (sl == 0) {
+                    if (!(ok = mbar_wait(&b_hdone[KS - 1], (t - 1) & 1, abort_flag))) break;
+                    v_pass(t);
+                    if (i == 0) K512_STAMP(t, 22);
+                }
+            }
+        }
+        // the state after the segment's last step
+        if (last_seg && a.hT && nsteps > 0) {
+#pragma unroll 1
+            for (int sl = 0; sl < KS; ++sl) {
+                if (!mbar_wait(&b_hdone[sl], (nsteps - 1) & 1, abort_flag)) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int pc = 0; pc < 2; ++pc) {
+                    float x[32];
+                    tmem_ld32(hrow + sl * BV + 32 * pc, x);
+                    tmem_wait_ld();
+                    if (!*abort_flag) {
+                        float4 *d4 = reinterpret_cast<float4 *>(a.hT + ((int64_t)n * H + h) * KV +
+                                                                (int64_t)(128 * sl + i) * V + v0 + 32 * pc);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) d4[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+                    }
+                }
+            }
+        }
+    } else if (warp < 12) {
+        // ---------------------------------------------------------------- WG_O: output rows
+        const int i = threadIdx.x - 256;
+        const uint32_t trow = tmem + ((uint32_t)((warp - 8) * 32) << 16) + C::COL_O;
+        const bool o32 = (reinterpret_cast<uintptr_t>(a.o) & 31) == 0;  // 32-byte row segments
+        float gnext = nsteps > 0 ? gate_of(0, i) : 0.f;
+        for (int t = 0; t < nsteps; ++t) {
+            const StepSpan sp = step_span(t0, t1, cb + t);
+            const float gi = gnext;
+            gnext = (t + 1 < nsteps) ? gate_of(t + 1, i) : 0.f;
+            const uint32_t orow = trow + (t & 1) * BV;
+            // O1 row i times scale 2^G~_i, in place, before P' V_f accumulates onto it
+            if (!mbar_wait(b_o1, t & 1, abort_flag)) break;
+            if (i == 0) K512_STAMP(t, 23);
+            tc_fence_after();
+            {
+                const float e = a.scale * fast_exp2(gi);
+#pragma unroll 1
+                for (int pc = 0; pc < 2; ++pc) {
+                    float x[32];
+                    tmem_ld32(orow + 32 * pc, x);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) x[q] *= e;
+                    tmem_st32(orow + 32 * pc, x);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(b_o1s);
+            }
+            // o = O (scale is in it) after P' V_f
+            if (!mbar_wait(b_pv, t & 1, abort_flag)) break;
+            if (i == 0) K512_STAMP(t, 24);
+            tc_fence_after();
+            const bool store = i < sp.len && !*abort_flag;
+            const int64_t row = ((sp.ta + i) * H + h) * (int64_t)V + v0;
+            if (!a.o_f32) {
+                uint32_t w[32];
+#pragma unroll
+                for (int pc = 0; pc < 4; ++pc) {
+                    float x[16];
+                    tmem_ld16f(orow + 16 * pc, x);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) w[8 * pc + q] = pack_bf16(x[2 * q], x[2 * q + 1]);
+                }
+                tc_fence_before();
+                mbar_arrive(&b_ofree[t & 1]);
+                if (store) {
+                    __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.o) + row;
+                    if (o32) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            st_global_v8(og + 16 * q, *reinterpret_cast<const uint32_t(*)[8]>(&w[8 * q]));
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            reinterpret_cast<uint4 *>(og)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int pc = 0; pc < 2; ++pc) {  // fp32 rows (16-byte aligned: V is a multiple of 64)
+                    float x[32];
+                    tmem_ld32(orow + 32 * pc, x);
+                    tmem_wait_ld();
+                    if (pc == 1) {
+                        tc_fence_before();
+                        mbar_arrive(&b_ofree[t & 1]);
+                    }
+                    if (store) {
+                        float4 *d = reinterpret_cast<float4 *>(static_cast<float *>(a.o) + row + 32 * pc);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) d[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 13) tmem_dealloc(tmem, C::COLS);
+    if (threadIdx.x == 0 && *abort_flag) record_timeout(a);
+}
+
+template <int KS>
+cudaError_t launch_k512(const FwdArgs &a, cudaStream_t st) {
+    using C = K512Cfg<KS>;
+    CUtensorMap tq, tk, tv;
+    const int64_t tok = a.lay.cu ? a.lay.T : (int64_t)a.lay.N * a.lay.T;
+    cudaError_t e;
+    if ((e = tc_make_map(&tq, a.q, tok, a.H, a.K, 64)) != cudaSuccess) return e;
+    if ((e = tc_make_map(&tk, a.k, tok, a.H, a.K, 64)) != cudaSuccess) return e;
+    if ((e = tc_make_map(&tv, a.v, tok, a.H, a.V, 64)) != cudaSuccess) return e;
+    auto kern = tc_walk_k512_kernel<KS>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM)) != cudaSuccess)
+        return e;
+    dim3 grid(a.lay.max_segs * (a.V / kK512BV), a.H);
+    kern<<<grid, kK512Threads, C::SMEM, st>>>(tq, tk, tv, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+#ifdef SGLA_DEVICE_TRACE
+extern "C" __attribute__((visibility("default"))) int sgla_k512_trace_read(unsigned long long *dst) {
+    return (int)cudaMemcpyFromSymbol(dst, g_k512_trace, sizeof(g_k512_trace));
+}
+#endif
+
+int tc_k512_bv() { return kK512BV; }
+
+cudaError_t tc_launch_walk_k512(const FwdArgs &a, cudaStream_t st) {
+    if (a.V % kK512BV != 0) return cudaErrorInvalidValue;
+    switch (a.K) {
+        case 256: return launch_k512<2>(a, st);
+        case 512: return launch_k512<4>(a, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace sgla

@@ -274,6 +274,8 @@ TC_CASES = [
     (1, 700, 2, 64, "zero", False, 64),
     (1, 1030, 2, 128, "neg_inf", True, 64),
     (1, 900, 2, 128, "mixed", True, 64),    # positive log gates: exact-decay fallback
+    (1, 256, 2, 128, "mixed", False, 128),  # positive log gates over a span short enough that
+                                            # the intra-chunk terms dominate the error measure
 ]
 
 
@@ -313,12 +315,14 @@ def test_tensor_core_workspace_status_clean():
 
 
 WIDE_K_CASES = [
-    # (B, T, H, K, V, gate, h0)   bf16, tensor-core path with K > 128 (V tile 32)
+    # (B, T, H, K, V, gate, h0)   bf16, tensor-core path with K > 128 (V tile 64)
     (2, 129, 2, 256, 256, "g", True),
     (1, 300, 1, 512, 512, "g", True),
     (1, 3000, 1, 512, 64, "g", True),     # many segments: k-block state pass + carry
     (1, 2500, 2, 256, 128, "gamma", True),
     (2, 700, 1, 512, 128, "mixed", False),
+    (1, 256, 2, 256, 64, "mixed", False),
+    (1, 200, 1, 512, 64, "mixed", False),
 ]
 
 
