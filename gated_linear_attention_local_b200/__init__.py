@@ -47,7 +47,7 @@ __all__ = ["simple_gla_fwd", "simple_gla_fwd_noalloc", "simple_gla_fwd_varlen", 
            "simple_gla_fused_recurrent", "fused_recurrent_simple_gla", "simple_gla_chunk",
            "simple_gla_normalized", "simple_gla_normalized_decode_step", "normalized_decode_state_width",
            "gla_fused_recurrent", "simple_gla_fused_recurrent_bwd", "simple_gla_chunk_bwd", "gla_chunk", "ChunkSimpleGLAFunction",
-           "simple_gla_log_decay_total", "simple_gla_state_carry",
+           "simple_gla_log_decay_total", "simple_gla_state_carry", "simple_gla_chunk_final_state",
            "fwd_workspace_size", "varlen_workspace_size", "workspace_status", "noalloc_status", "library_path",
            "SglaError"]
 
@@ -287,6 +287,53 @@ def simple_gla_chunk(q, k, v, g=None, g_gamma=None, scale=None, initial_state=No
                                 vf, dt, _ptr(ws), ws.numel(), _stream())
     raise_for_status(st, "simple_gla_chunk")
     return (o.unsqueeze(0) if squeeze else o), ht
+
+
+@_on_tensor_device
+def simple_gla_chunk_final_state(k, v, g=None, g_gamma=None, initial_state=None, cu_seqlens=None, chunk_size=64,
+                                 workspace=None):
+    """The final state of the chunked forward without its output (the state pass of
+    section 3 alone): k [B,T,H,K], v [B,T,H,V] (or packed [1,T,H,*] / [T,H,*] with
+    cu_seqlens), g [B,T,H] or g_gamma [H].  Returns final_state [N,H,K,V] fp32."""
+    _common_checks(k, k, v, g, g_gamma, initial_state)
+    if cu_seqlens is not None:
+        _check_cuda("cu_seqlens", cu_seqlens, torch.int64, 1)
+        if k.dim() == 4:
+            if k.shape[0] != 1:
+                raise ValueError("with cu_seqlens the batch size must be 1 (flatten the batch first)")
+            k, v = k[0], v[0]
+            g = g[0] if g is not None else None
+        if k.dim() != 3 or v.dim() != 3 or v.shape[:2] != k.shape[:2]:
+            raise ValueError("k must be [T,H,K] and v [T,H,V] with cu_seqlens")
+        N = cu_seqlens.shape[0] - 1
+        if N < 1:
+            raise ValueError("cu_seqlens must hold at least two entries")
+        T, H, K = k.shape
+        V = v.shape[2]
+        if g is not None and tuple(g.shape) != (T, H):
+            raise ValueError("g must be [T,H] (or [1,T,H])")
+    else:
+        if k.dim() != 4 or v.dim() != 4 or v.shape[:3] != k.shape[:3]:
+            raise ValueError("k must be [B,T,H,K] and v [B,T,H,V]")
+        N, T, H, K = k.shape
+        V = v.shape[3]
+        if g is not None and tuple(g.shape) != (N, T, H):
+            raise ValueError(f"g must be [B,T,H] = {(N, T, H)}")
+    if g_gamma is not None and tuple(g_gamma.shape) != (H,):
+        raise ValueError("g_gamma must be [H]")
+    if initial_state is not None and tuple(initial_state.shape) != (N, H, K, V):
+        raise ValueError(f"initial_state must be {(N, H, K, V)}")
+    dt = _DTYPES[k.dtype]
+    ht = torch.empty((N, H, K, V), dtype=torch.float32, device=k.device)
+    nbytes = int(lib().simple_gla_chunk_final_state_workspace_size(_ptr(cu_seqlens), N, T, H, K, V, chunk_size, dt))
+    if nbytes == 0:
+        raise_for_status(_size_status(K, V, chunk_size), "simple_gla_chunk_final_state")
+    ws = _workspace(nbytes, k.device, workspace)
+    st = lib().simple_gla_chunk_final_state(_ptr(k), _ptr(v), _ptr(g), _ptr(g_gamma), _ptr(initial_state), _ptr(ht),
+                                            _ptr(cu_seqlens), N, T, H, K, V, chunk_size, dt, _ptr(ws), ws.numel(),
+                                            _stream())
+    raise_for_status(st, "simple_gla_chunk_final_state")
+    return ht
 
 
 class ChunkSimpleGLAFunction(torch.autograd.Function):

@@ -58,6 +58,10 @@ _SIG = {
                    ctypes.c_size_t, _P], ctypes.c_int),
     "simple_gla_log_decay_total": ([_P, _P, _I64, _I64, _P, _P], ctypes.c_int),
     "simple_gla_state_carry": ([_P, _P, _P, _P, ctypes.c_int, _I64, _I64, _I64, _P], ctypes.c_int),
+    "simple_gla_chunk_final_state_workspace_size": ([_P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int],
+                                                    ctypes.c_size_t),
+    "simple_gla_chunk_final_state": ([_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int,
+                                      ctypes.c_int, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "sgla_workspace_status": ([_P, ctypes.POINTER(ctypes.c_int), _P], ctypes.c_int),
     "sgla_noalloc_status": ([ctypes.POINTER(ctypes.c_int), _P], ctypes.c_int),
     "simple_gla_normalized_workspace_size": ([_P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int],

@@ -99,7 +99,7 @@ sgla_status check_sizes(int64_t H, int64_t K, int64_t V, int chunk_size) {
 
 // varlen: N sequences, T = total tokens; dense: N = B, T = tokens per sequence.
 Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V, int C,
-               sgla_dtype dtype, bool per_token_gate, bool state_v_first = false) {
+               sgla_dtype dtype, bool per_token_gate, bool state_v_first = false, bool state_only = false) {
     Plan p;
     sgla_status st = check_sizes(H, K, V, C);
     if (st != SGLA_OK) { p.why = st; return p; }
@@ -143,12 +143,17 @@ Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t 
             const int64_t l = (nt + ns - 1) / ns, ns_eff = (nt + l - 1) / l;
             if (l < min_l) break;
             const double waves_walk = (double)((units * ns_eff + 147) / 148);
-            const double t_w = std::max(waves_walk * (double)(l + 2) * t_walk, walk_bytes / bw);
+            const double t_w = state_only ? 0.0 : std::max(waves_walk * (double)(l + 2) * t_walk, walk_bytes / bw);
             double t_s = 0.0;
-            if (ns_eff > 1) {
-                const double waves_state = (double)((state_units * (ns_eff - 1) + 147) / 148);
+            // the state pass covers every segment but the last (all of them on a
+            // state-only call, whose carry then reads each segment state once)
+            const int64_t ns_state = state_only ? ns_eff : ns_eff - 1;
+            if (ns_state > 0) {
+                const double waves_state = (double)((state_units * ns_state + 147) / 148);
                 t_s = std::max(waves_state * (double)(l + 1) * t_state,
-                               kv_bytes * (double)(ns_eff - 1) / (double)ns_eff / bw_state);
+                               kv_bytes * (double)ns_state / (double)ns_eff / bw_state);
+                if (state_only)
+                    t_s += (double)ns_eff * (double)N * (double)H * (double)K * (double)V * 4.0 / bw;
             }
             const double cost = t_w + t_s;
             if (cost < best - 1e-9) {
@@ -174,7 +179,7 @@ Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t 
         p.NS = (p.NT + p.L - 1) / p.L;
         p.max_chunks = N * p.NT;
         p.max_segs = N * p.NS;
-        p.multi_seg = p.NS > 1;
+        p.multi_seg = p.NS > 1 || state_only;
     }
     if (p.max_chunks >= kMaxTokens || p.max_segs * H >= kMaxTokens) { p.why = SGLA_ERR_UNSUPPORTED; return p; }
     size_t off = 256;  // status word
@@ -478,6 +483,72 @@ sgla_status simple_gla_chunk(const void *q, const void *k, const void *v, const 
     if (N < (varlen ? 1 : 0) || T < 0) return SGLA_ERR_INVALID_ARGUMENT;
     return run_forward(varlen, q, k, v, g, g_gamma, scale, cu_seqlens, N, T, initial_state, o, final_state,
                        H, K, V, chunk_size, dtype, workspace, workspace_bytes, stream, state_v_first != 0);
+}
+
+// State-only chunked pass ("Simple GLA in flash-linear-attention" section 3, the state
+// recurrence chunk_fwd_h on its own): every segment's local end state from zero
+// (tensor-core or SIMT segment-state pass over all segments), then one carry that
+// folds them onto the initial state into final_state.  No output, q not read.
+size_t simple_gla_chunk_final_state_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H,
+                                                   int64_t K, int64_t V, int chunk_size, sgla_dtype dtype) {
+    Plan p = make_plan(cu_seqlens != nullptr, N, T, H, K, V, chunk_size, dtype, true, false, true);
+    return p.valid ? p.bytes : 0;
+}
+
+sgla_status simple_gla_chunk_final_state(const void *k, const void *v, const float *g, const float *g_gamma,
+                                         const float *initial_state, float *final_state, const int64_t *cu_seqlens,
+                                         int64_t N, int64_t T, int64_t H, int64_t K, int64_t V, int chunk_size,
+                                         sgla_dtype dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    const bool varlen = cu_seqlens != nullptr;
+    if (N < (varlen ? 1 : 0) || T < 0) return SGLA_ERR_INVALID_ARGUMENT;
+    if (g && g_gamma) return SGLA_ERR_INVALID_ARGUMENT;
+    const int64_t tokens = varlen ? T : N * T;
+    if (!final_state || (tokens > 0 && (!k || !v))) return SGLA_ERR_INVALID_ARGUMENT;
+    for (const void *p : {k, v, (const void *)initial_state, (const void *)final_state})
+        if (!aligned(p, 16)) return SGLA_ERR_INVALID_ARGUMENT;
+    if (!aligned(g, 4) || !aligned(g_gamma, 4) || !aligned(cu_seqlens, 8)) return SGLA_ERR_INVALID_ARGUMENT;
+    const bool per_token = g != nullptr;
+    Plan p = make_plan(varlen, N, T, H, K, V, chunk_size, dtype, per_token, false, true);
+    if (!p.valid) return p.why;
+    if (!workspace || workspace_bytes < p.bytes) return SGLA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return SGLA_ERR_INVALID_ARGUMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+    FwdArgs a{};
+    a.k = k; a.v = v; a.g = g; a.g_gamma = g_gamma; a.scale = 1.f;
+    a.h0 = initial_state; a.hT = final_state;
+    a.H = (int)H; a.K = (int)K; a.V = (int)V;
+    a.gate_mode = g ? kGatePerToken : (g_gamma ? kGatePerHead : kGateNone);
+    a.bf16 = dtype == SGLA_BF16;
+    a.state_all = true;
+    a.gcum = per_token ? reinterpret_cast<float *>(ws + p.off_gcum) : nullptr;
+    a.gpos = per_token ? reinterpret_cast<int *>(ws + p.off_gpos) : nullptr;
+    a.seg_dec = reinterpret_cast<float *>(ws + p.off_seg_dec);
+    a.seg_state = reinterpret_cast<float *>(ws + p.off_seg_state);
+    SeqLayout &lay = a.lay;
+    lay.cu = varlen ? cu_seqlens : nullptr;
+    lay.chunk_off = varlen ? reinterpret_cast<int *>(ws + p.off_chunk_off) : nullptr;
+    lay.seg_off = varlen ? reinterpret_cast<int *>(ws + p.off_seg_off) : nullptr;
+    lay.status = reinterpret_cast<int *>(ws);
+    a.dev_status = reinterpret_cast<int *>(ws);
+    lay.T = T; lay.N = (int)N; lay.H = (int)H; lay.C = p.C; lay.L = p.L;
+    lay.NT = p.NT; lay.NS = p.NS;
+    lay.max_chunks = (int)p.max_chunks; lay.max_segs = (int)p.max_segs;
+    if (varlen) {
+        SGLA_LAUNCH("varlen_plan", launch_varlen_plan(cu_seqlens, (int)N, T, p.C, p.L,
+                                                      const_cast<int *>(lay.chunk_off),
+                                                      const_cast<int *>(lay.seg_off), reinterpret_cast<int *>(ws), st));
+    } else {
+        SGLA_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), st), "status reset");
+    }
+    if (N == 0) return SGLA_OK;
+    if (per_token && tokens > 0) SGLA_LAUNCH("chunk_cumsum", launch_chunk_cumsum(g, a.gcum, a.gpos, lay, st));
+    if (p.max_segs > 0 && tokens > 0) {
+        if (p.tc) SGLA_LAUNCH("segment_state_tc", tc_launch_segment_state(a, st));
+        else SGLA_LAUNCH("segment_state_simt", launch_segment_state_simt(a, st));
+    }
+    SGLA_LAUNCH("segment_carry", launch_segment_carry(a, true, st));
+    return SGLA_OK;
 }
 
 sgla_status simple_gla_decode_step(const void *q, const void *k, const void *v, const float *g,

@@ -22,7 +22,8 @@ constexpr int kSimtThreads = 256;
 
 // ---------------------------------------------------------------------------
 // Segment state: local end state (from zero) of one segment, for one 64x64 tile
-// of the K x V state; only segments that are not the last of their sequence.
+// of the K x V state; only segments that are not the last of their sequence (every
+// segment on a state-only call).
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(kSimtThreads)
@@ -32,7 +33,7 @@ segment_state_simt_kernel(FwdArgs a) {
     int n, s;
     if (!locate_segment(lay, blockIdx.x, n, s)) return;
     const int nseg = seq_segments(lay, n);
-    if (s == nseg - 1) return;
+    if (s == nseg - 1 && !a.state_all) return;
     const int h = blockIdx.y, H = a.H, K = a.K, V = a.V, C = lay.C;
     const int VT = (V + 63) / 64;
     const int k0 = (blockIdx.z / VT) * 64, v0 = (blockIdx.z % VT) * 64;

@@ -75,7 +75,7 @@ tc_segment_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_con
     int n, s;
     if (!locate_segment(lay, u, n, s)) return;
     const int nseg = seq_segments(lay, n);
-    if (s == nseg - 1) return;
+    if (s == nseg - 1 && !a.state_all) return;  // the last end state is needed on a state-only call
     const int h = blockIdx.y, H = a.H, V = a.V;
     int64_t t0, t1;
     seq_span(lay, n, t0, t1);

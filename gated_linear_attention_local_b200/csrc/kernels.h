@@ -26,6 +26,8 @@ struct FwdArgs {
     float *seg_dec;  // [max_segs, H] log2 total decay of each segment
     float *seg_state;// [max_segs, H, K, V] segment states (local end state, then entering state)
     int *dev_status; // writable status word (bounded device waits record time-outs here)
+    bool state_all;  // state-only call: every segment, the last one too, goes through the state
+                     // pass and the carry folds them all into hT (no output walk)
     SeqLayout lay;
 };
 

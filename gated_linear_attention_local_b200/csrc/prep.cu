@@ -182,7 +182,8 @@ cudaError_t launch_chunk_cumsum(const float *g, float *gcum, int *gpos, const Se
 // Cross-segment carry, one thread per 4 state elements of one (sequence, head).
 // seg_state[u] holds segment u's local end state (from zero) on entry and the
 // state ENTERING segment u+1 on exit; seg_dec[u] is segment u's log2 total decay.
-// Also writes final_state for empty sequences (initial state unchanged).
+// Also writes final_state for empty sequences (initial state unchanged).  On a
+// state-only call (a.state_all) it folds every segment into final_state instead.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 segment_carry_kernel(FwdArgs a, bool need_carry) {
@@ -201,8 +202,22 @@ segment_carry_kernel(FwdArgs a, bool need_carry) {
         }
         return;
     }
-    if (!need_carry || nseg == 1) return;
     const int first = seq_first_segment(lay, n);
+    if (a.state_all) {  // hT = the fold of every segment's (decay, local end state) onto h0
+        if (!a.hT) return;
+        float4 S = a.h0 ? *reinterpret_cast<const float4 *>(a.h0 + sidx) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < nseg; ++s) {
+            const float4 d = *reinterpret_cast<const float4 *>(a.seg_state + ((int64_t)(first + s) * a.H + h) * KV + e);
+            const float dec = exp2f(a.seg_dec[(int64_t)(first + s) * a.H + h]);
+            S.x = fmaf(dec, S.x, d.x);
+            S.y = fmaf(dec, S.y, d.y);
+            S.z = fmaf(dec, S.z, d.z);
+            S.w = fmaf(dec, S.w, d.w);
+        }
+        *reinterpret_cast<float4 *>(a.hT + sidx) = S;
+        return;
+    }
+    if (!need_carry || nseg == 1) return;
     float4 S = a.h0 ? *reinterpret_cast<const float4 *>(a.h0 + sidx) : make_float4(0.f, 0.f, 0.f, 0.f);
     // the loads of segment s+1 are in flight while segment s is combined
     auto slot_of = [&](int s) {

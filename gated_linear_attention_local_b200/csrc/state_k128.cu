@@ -57,7 +57,7 @@ tc_state_k128_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
     const int v0 = (blockIdx.x % VT) * 128;
     int n, s;
     if (!locate_segment(lay, u, n, s)) return;
-    if (s == seq_segments(lay, n) - 1) return;  // the last segment's end state is not needed
+    if (s == seq_segments(lay, n) - 1 && !a.state_all) return;  // needed only on a state-only call
     const int h = blockIdx.y, H = a.H, V = a.V;
     int64_t t0, t1;
     seq_span(lay, n, t0, t1);

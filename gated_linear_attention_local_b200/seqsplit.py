@@ -9,13 +9,15 @@ inter-chunk propagation is only a scalar multiplication of S), so one all-gather
 every rank's summary (total log decay, end state from a zero state) lets each rank
 fold the ranks before it:
 
-  phase A   forward of the local slice from a zero state -> S_r; its log decay D_r
+  phase A   end state of the local slice from a zero state -> S_r (the state pass
+            alone, no output); its log decay D_r
   exchange  all_gather of (D_r, S_r) over the group (NCCL on GPUs)
   phase C   h_r = exp(D_{r-1}) h_{r-1} + S_{r-1} (h_0 = the initial state), then the
             forward of the local slice from h_r
 
-Both forwards, the decay total and the fold run in the library's kernels; this
-module only orders the calls and moves the summaries (torch.distributed).
+The state pass, the forward, the decay total and the fold run in the library's
+kernels; this module only orders the calls and moves the summaries
+(torch.distributed).
 """
 from __future__ import annotations
 
@@ -26,17 +28,22 @@ import torch.distributed as dist
 
 
 def library_ops():
-    """The CUDA implementations of the three local steps."""
-    from . import chunk_simple_gla, simple_gla_log_decay_total, simple_gla_state_carry
+    """The CUDA implementations of the local steps."""
+    from . import (chunk_simple_gla, simple_gla_chunk_final_state, simple_gla_log_decay_total,
+                   simple_gla_state_carry)
 
     def forward(q, k, v, g, g_gamma, scale, initial_state, output_final_state, chunk_size):
         return chunk_simple_gla(q, k, v, g=g, g_gamma=g_gamma, scale=scale, initial_state=initial_state,
                                 output_final_state=output_final_state, chunk_size=chunk_size)
 
+    def final_state(k, v, g, g_gamma, chunk_size):
+        return simple_gla_chunk_final_state(k, v, g=g, g_gamma=g_gamma, chunk_size=chunk_size)
+
     def log_decay_total(g, g_gamma, T, H):
         return simple_gla_log_decay_total(g=g, g_gamma=g_gamma, T=T, H=H)
 
-    return SimpleNamespace(forward=forward, log_decay_total=log_decay_total, state_carry=simple_gla_state_carry)
+    return SimpleNamespace(forward=forward, final_state=final_state, log_decay_total=log_decay_total,
+                           state_carry=simple_gla_state_carry)
 
 
 def chunk_simple_gla_seq_split(q, k, v, g=None, g_gamma=None, scale=None, initial_state=None,
@@ -51,7 +58,7 @@ def chunk_simple_gla_seq_split(q, k, v, g=None, g_gamma=None, scale=None, initia
     rank = dist.get_rank(group)
     T, H = q.shape[1], q.shape[2]
     # phase A: this slice's summary
-    _, s_r = ops.forward(q, k, v, g, g_gamma, scale, None, True, chunk_size)
+    s_r = ops.final_state(k, v, g, g_gamma, chunk_size)
     d_r = ops.log_decay_total(g, g_gamma, T, H)
     # exchange
     d_all = [torch.empty_like(d_r) for _ in range(world)]

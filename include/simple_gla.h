@@ -356,6 +356,32 @@ SGLA_API sgla_status simple_gla_state_carry(const float *log_decay, const float 
                                             int64_t H, int64_t K, int64_t V, void *stream);
 
 /*
+ * The final state of the chunked forward without its output ("Simple GLA in
+ * flash-linear-attention: maths and kernels", section 3: the state recurrence
+ * chunk_fwd_h on its own).  For every sequence,
+ *   final_state = exp(G) initial_state + sum_t exp(G - G_t) k_t v_t^T,
+ * G_t the sum of the log gates up to and including token t and G the sequence total
+ * (g_gamma: G_t = (t+1) g_gamma[h]).  It is the phase-A summary of a sequence split
+ * across ranks (a slice's end state from a zero state) at the cost of the state pass
+ * alone: q is not read and no output is formed.
+ *   cu_seqlens == NULL: N sequences of T tokens, k [N,T,H,K], v [N,T,H,V], g [N,T,H].
+ *   cu_seqlens != NULL: DEVICE pointer to N+1 int64 (N >= 1), packed k [T,H,K],
+ *       v [T,H,V], g [T,H]; a cu_seqlens that is not non-decreasing from 0 to T is
+ *       reported through sgla_workspace_status() as for simple_gla_fwd_varlen.
+ *   initial_state (NULL = 0) and final_state (required): fp32 [N,H,K,V], DEVICE.
+ *   Sizes, dtype, chunk_size, alignment and errors as simple_gla_fwd; workspace: at
+ *   least simple_gla_chunk_final_state_workspace_size() bytes, 256-byte aligned.
+ */
+SGLA_API size_t simple_gla_chunk_final_state_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T,
+                                                            int64_t H, int64_t K, int64_t V, int chunk_size,
+                                                            sgla_dtype dtype);
+SGLA_API sgla_status simple_gla_chunk_final_state(const void *k, const void *v, const float *g, const float *g_gamma,
+                                                  const float *initial_state, float *final_state,
+                                                  const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H,
+                                                  int64_t K, int64_t V, int chunk_size, sgla_dtype dtype,
+                                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Read the device-side status word of the last forward call that used
  * `workspace` (SGLA_DEVICE_OK or SGLA_DEVICE_*).  Synchronises `stream`.
  * Returns SGLA_OK and fills *device_status, or an error status.

@@ -39,6 +39,10 @@ def _oracle_ops():
                                       output_final_state=True)
         return torch.from_numpy(np.asarray(o)), torch.from_numpy(np.asarray(ht))
 
+    def final_state(k, v, g, g_gamma, chunk_size):
+        q = torch.zeros_like(k)
+        return forward(q, k, v, g, g_gamma, None, None, True, chunk_size)[1]
+
     def log_decay_total(g, g_gamma, T_r, H_):
         if g is not None:
             return g[0].double().sum(0)
@@ -52,7 +56,8 @@ def _oracle_ops():
             h = torch.exp(d_all[r])[:, None, None] * h + s_all[r]
         return h
 
-    return SimpleNamespace(forward=forward, log_decay_total=log_decay_total, state_carry=state_carry)
+    return SimpleNamespace(forward=forward, final_state=final_state, log_decay_total=log_decay_total,
+                           state_carry=state_carry)
 
 
 def _slices(inp):
@@ -108,8 +113,8 @@ def test_seq_split_kernels_on_one_gpu(gate):
     sl = [{k_: (v_[:, bounds[r]:bounds[r + 1]].contiguous() if k_ in ("q", "k", "v", "g") and v_ is not None else v_)
            for k_, v_ in dev.items()} for r in range(len(lens))]
     summaries = []
-    for s in sl:  # phase A on every rank
-        _, s_r = sg.chunk_simple_gla(s["q"], s["k"], s["v"], g=s["g"], g_gamma=s["g_gamma"], output_final_state=True)
+    for s in sl:  # phase A on every rank: the state pass alone
+        s_r = sg.simple_gla_chunk_final_state(s["k"], s["v"], g=s["g"], g_gamma=s["g_gamma"])
         d_r = sg.simple_gla_log_decay_total(g=s["g"], g_gamma=s["g_gamma"], T=s["q"].shape[1], H=Hn)
         summaries.append((d_r, s_r[0]))
     d_all = torch.stack([d for d, _ in summaries])
