@@ -67,18 +67,20 @@ constexpr int kK512BV = 64;
 
 template <int KS>
 struct K512Cfg {
-    static constexpr int NU = 5;                        // Q/K ring: units of one 128-wide k slice of Q or K
-    static constexpr uint32_t UNIT = 2 * kRegion;       // [128 tokens x 128 k] as two 64-k regions
-    static constexpr uint32_t RING = 0;
-    static constexpr uint32_t HB = NU * UNIT;           // Hb: [128 k rows x 64 v] of one state block
-    static constexpr uint32_t V0 = HB + kRegion;        // V ring: 2 x [128 tokens x 64 v] (V_f in place)
-    static constexpr uint32_t VW = V0 + 2 * kRegion;    // V_w [128 tokens x 64 v]
-    static constexpr uint32_t GS = VW + kRegion;        // exact steps: [128] gates, [128] factors
+    static constexpr uint32_t QUNIT = 2 * kRegion;            // Q_s: two 64-k regions of 128 token rows
+    static constexpr uint32_t KREG = kRegion + kRegion / 2;   // 128 token rows of K_s and 64 rows of Hb_s^T
+    static constexpr uint32_t KUNIT = 2 * KREG;
+    static constexpr uint32_t QR = 0;                         // Q ring: 2 slots
+    static constexpr uint32_t KR = QR + 2 * QUNIT;            // K ring: 2 slots
+    static constexpr uint32_t V0 = KR + 2 * KUNIT;            // V ring: 2 x [128 tokens x 64 v] (V_f in place)
+    static constexpr uint32_t VW = V0 + 2 * kRegion;          // V_w ring: 2 x [128 tokens x 64 v]
+    static constexpr uint32_t GS = VW + 2 * kRegion;          // exact steps: [128] gates, [128] factors
     static constexpr uint32_t BARS = GS + 2 * 128 * 4;
-    static constexpr uint32_t MISC = BARS + 32 * 8;     // tmem address, abort flag
+    static constexpr uint32_t MISC = BARS + 32 * 8;           // tmem address, abort flag
     static constexpr uint32_t TOTAL = MISC + 16;
-    static constexpr size_t SMEM = TOTAL + 1024;        // + alignment slack
-    static constexpr uint32_t COL_S = 0, COL_O = 128, COL_H = 256;
+    static constexpr size_t SMEM = TOTAL + 1024;              // + alignment slack
+    // tensor memory: O of even steps, S (P' over its first 64 columns), O of odd steps, H
+    static constexpr uint32_t COL_OA = 0, COL_S = 64, COL_OB = 192, COL_H = 256;
     static constexpr uint32_t COLS = 512;
     static_assert(KS == 2 || KS == 4, "K = 256 or 512");
     static_assert(COL_H + KS * kK512BV <= COLS, "tensor memory budget");
@@ -110,36 +112,39 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     const bool last_seg = (s == nseg - 1);
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::BARS);
-    uint64_t *full_u = bars + 0, *empty_u = bars + 5;    // [NU] ring unit landed / released
+    uint64_t *full_q = bars + 0, *empty_q = bars + 2;    // [2] Q ring slot landed / released
+    uint64_t *full_k = bars + 4, *empty_k = bars + 6;    // [2] K rows of a K ring slot landed / slot released
+    uint64_t *b_hbt = bars + 8;     // [2] Hb_s^T written into a K ring slot, H_s decayed (WG_S, 128 arrivals)
     uint64_t *full_v = bars + 10, *empty_v = bars + 12;  // [2] V stage landed / released (P V done)
-    uint64_t *b_s = bars + 14;      // S(t) complete
-    uint64_t *b_p = bars + 15;      // P'(t) written over S (WG_P, 128 arrivals)
-    uint64_t *b_o1 = bars + 16;     // O1(t) complete
-    uint64_t *b_o1s = bars + 17;    // O1(t) rescaled (WG_O, 128 arrivals)
-    uint64_t *b_hb = bars + 18;     // Hb holds the next block and its H block is decayed (WG_S, 128 arrivals)
-    uint64_t *b_hbfree = bars + 19; // Hb read by its O1 products
-    uint64_t *b_hdone = bars + 20;  // [KS] H block s of the step complete
-    uint64_t *b_vw = bars + 24;     // V_w(t), V_f(t) ready (WG_S, 128 arrivals)
-    uint64_t *b_pv = bars + 25;     // P V(t) done
-    uint64_t *b_ofree = bars + 26;  // [2] O buffer read out (WG_O, 128 arrivals)
-    uint64_t *b_drain = bars + 28;  // every product retired
+    uint64_t *b_vw = bars + 14;     // [2] V_w, V_f of a step ready (WG_S, 128 arrivals)
+    uint64_t *b_s = bars + 16;      // S(t) and O1(t) complete
+    uint64_t *b_p = bars + 17;      // P'(t) written over S (WG_P, 128 arrivals)
+    uint64_t *b_o1s = bars + 18;    // O1(t) rescaled (WG_O, 128 arrivals)
+    uint64_t *b_hdone = bars + 19;  // [KS] H block s of the step complete
+    uint64_t *b_pv = bars + 23;     // P V(t) done
+    uint64_t *b_ofree = bars + 24;  // [2] O buffer read out (WG_O, 128 arrivals)
+    uint64_t *b_drain = bars + 26;  // every product retired
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + C::MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + C::MISC + 8);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int b = 0; b < 14; ++b) mbar_init(&bars[b], 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&full_q[b], 1);
+            mbar_init(&empty_q[b], 1);
+            mbar_init(&full_k[b], 1);
+            mbar_init(&empty_k[b], 1);
+            mbar_init(&b_hbt[b], 128);
+            mbar_init(&full_v[b], 1);
+            mbar_init(&empty_v[b], 1);
+            mbar_init(&b_vw[b], 128);
+            mbar_init(&b_ofree[b], 128);
+        }
         mbar_init(b_s, 1);
         mbar_init(b_p, 128);
-        mbar_init(b_o1, 1);
         mbar_init(b_o1s, 128);
-        mbar_init(b_hb, 128);
-        mbar_init(b_hbfree, 1);
         for (int b = 0; b < KS; ++b) mbar_init(&b_hdone[b], 1);
-        mbar_init(b_vw, 128);
         mbar_init(b_pv, 1);
-        mbar_init(&b_ofree[0], 128);
-        mbar_init(&b_ofree[1], 128);
         mbar_init(b_drain, 1);
         *abort_flag = 0;
         mbar_fence_init();
@@ -175,19 +180,20 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
 
     if (warp == 12) {
         // ---------------------------------------------------------------- TMA loads
-        // Unit x of the ring is the Q (x even) or K (x odd) slice sl of step t, q = x / 2 =
-        // t KS + sl, in slot x % NU.  V(t) goes out just before unit 2 t KS: its stage is
-        // freed by P V(t-2), which retires before the unit that load waits for.
+        // Slice q = t KS + sl: Q_s into Q slot q & 1, K_s into the K rows of K slot q & 1
+        // (after the 64 rows of Hb^T on even steps, before them on odd steps).  V(t) goes
+        // out just before slice t KS: its stage is freed by P V(t-2), which retires
+        // before the slot that slice waits for.
         if (lane == 0) {
             prefetch_tmap(&tq);
             prefetch_tmap(&tk);
             prefetch_tmap(&tv);
             int issued = 0, issued_v = 0;
-            const int total = nsteps * KS * 2;
-            for (int x = 0; x < total; ++x) {
-                const int q = x >> 1, t = q / KS, sl = q - t * KS, slot = x % C::NU;
+            const int total = nsteps * KS;
+            for (int q = 0; q < total; ++q) {
+                const int t = q / KS, sl = q - t * KS, st = q & 1;
                 const int tok = (int)(t0 + (int64_t)(cb + t) * kStep);
-                if (sl == 0 && (x & 1) == 0) {
+                if (sl == 0) {
                     const int vs = t & 1;
                     if (t >= 2 && !mbar_wait(&empty_v[vs], ((t >> 1) - 1) & 1, abort_flag)) break;
                     K512_STAMP(t, 28);
@@ -195,25 +201,37 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                     tma_load_3d(sm + C::V0 + vs * kRegion, &tv, &full_v[vs], v0, h, tok);
                     issued_v = t + 1;
                 }
-                if (x >= C::NU && !mbar_wait(&empty_u[slot], ((x / C::NU) - 1) & 1, abort_flag)) break;
-                if (sl == 0 && (x & 1) == 0) K512_STAMP(t, 27);
-                if (sl == KS - 1 && (x & 1)) K512_STAMP(t, 29);
-                const CUtensorMap *m = (x & 1) ? &tk : &tq;
-                unsigned char *dst = sm + C::RING + slot * C::UNIT;
-                mbar_arrive_expect_tx(&full_u[slot], C::UNIT);
-                tma_load_3d(dst, m, &full_u[slot], 128 * sl, h, tok);
-                tma_load_3d(dst + kRegion, m, &full_u[slot], 128 * sl + 64, h, tok);
-                issued = x + 1;
+                if (q >= 2 && !mbar_wait(&empty_q[st], ((q >> 1) - 1) & 1, abort_flag)) break;
+                if (sl == 0) K512_STAMP(t, 27);
+                unsigned char *dq = sm + C::QR + st * C::QUNIT;
+                mbar_arrive_expect_tx(&full_q[st], C::QUNIT);
+                tma_load_3d(dq, &tq, &full_q[st], 128 * sl, h, tok);
+                tma_load_3d(dq + kRegion, &tq, &full_q[st], 128 * sl + 64, h, tok);
+                issued = 2 * q + 1;
+                if (q >= 2 && !mbar_wait(&empty_k[st], ((q >> 1) - 1) & 1, abort_flag)) break;
+                if (sl == KS - 1) K512_STAMP(t, 29);
+                unsigned char *dk = sm + C::KR + st * C::KUNIT + ((t & 1) ? 0u : kRegion / 2);
+                mbar_arrive_expect_tx(&full_k[st], 2 * kRegion);
+                tma_load_3d(dk, &tk, &full_k[st], 128 * sl, h, tok);
+                tma_load_3d(dk + C::KREG, &tk, &full_k[st], 128 * sl + 64, h, tok);
+                issued = 2 * q + 2;
             }
-            if (*abort_flag) {
-                for (int x = max(0, issued - C::NU); x < issued; ++x) mbar_drain(&full_u[x % C::NU], (x / C::NU) & 1);
+            if (*abort_flag) {  // issued counts halves: Q of slice q is 2q, K is 2q + 1
+                for (int x = max(0, issued - 4); x < issued; ++x) {
+                    const int q = x >> 1;
+                    mbar_drain((x & 1) ? &full_k[q & 1] : &full_q[q & 1], (q >> 1) & 1);
+                }
                 for (int t = max(0, issued_v - 2); t < issued_v; ++t) mbar_drain(&full_v[t & 1], (t >> 1) & 1);
             }
         }
     } else if (warp == 13) {
         // ---------------------------------------------------------------- MMA issuer
+        // Per slice s one N = 192 product gives S and O1 together: A = Q_s, B = the K slot's
+        // 192 rows per 64-k region, [Hb_s^T ; K_s] on even steps (D = O_A | S) and
+        // [K_s ; Hb_s^T] on odd steps (D = S | O_B); then H_s += K_s^T V_w.  Slice 0 issues
+        // H first (S holds P' of the step before until that P V retires).
         if (lane == 0) {
-            const uint32_t idS = idesc_bf16_f32(128, 128, false, false);
+            const uint32_t idSO = idesc_bf16_f32(128, 192, false, false);
             const uint32_t idO = idesc_bf16_f32(128, BV, false, true);
             const uint32_t idH = idesc_bf16_f32(128, BV, true, true);
             const uint32_t sbase = smem_u32(sm);
@@ -221,70 +239,53 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
             auto wait = [&](uint64_t *bar, uint32_t ph) { return mbar_wait(bar, ph, abort_flag); };
             bool ok = true;
             for (int t = 0; ok && t < nsteps; ++t) {
-                const uint32_t od = tmem + C::COL_O + (t & 1) * BV;
-#pragma unroll 1
-                // products of slice s: O1 += Q_s Hb_s; S += Q_s K_s^T; H_s += K_s^T V_w.  Slice 0
-                // issues O1, H, S (S holds P'(t-1) until P V(t-1) is done); the others S, O1, H,
-                // which puts S(t) complete early in the last slice (the mask overlaps the rest
-                // of the step) and leaves the state pass of the next block the time of S and H
+                const bool ev = (t & 1) == 0;
+                const uint32_t dso = tmem + (ev ? C::COL_OA : C::COL_S);
+                const uint32_t od = tmem + (ev ? C::COL_OA : C::COL_OB);
+                const uint32_t koff = ev ? kRegion / 2 : 0u;  // K rows inside a K region
+                const uint32_t vw = sbase + C::VW + (t & 1) * kRegion;
 #pragma unroll 1
                 for (int sl = 0; sl < KS; ++sl) {
-                    const int q = t * KS + sl, use = q;
-                    const int xq = 2 * q, xk = 2 * q + 1;
-                    const int sq = xq % C::NU, sk = xk % C::NU;
-                    const uint32_t qa = sbase + C::RING + sq * C::UNIT, ka = sbase + C::RING + sk * C::UNIT;
+                    const int q = t * KS + sl, st = q & 1;
+                    const uint32_t ph = (q >> 1) & 1;
+                    const uint32_t qa = sbase + C::QR + st * C::QUNIT, ka = sbase + C::KR + st * C::KUNIT;
                     if (sl == 0) K512_STAMP(t, 0);
-                    if (!(ok = wait(&full_u[sq], (xq / C::NU) & 1))) break;
+                    if (!(ok = wait(&full_q[st], ph) && wait(&full_k[st], ph))) break;
                     K512_STAMP(t, sl == 0 ? 1 : 4 + sl);
-                    auto issue_o1 = [&]() -> bool {
-                        if (!wait(b_hb, use & 1)) return false;
-                        if (sl == 0 && t >= 2 && !wait(&b_ofree[t & 1], ((t >> 1) - 1) & 1)) return false;
-                        if (sl == 0) K512_STAMP(t, 2);
+                    if (!(ok = wait(&b_hbt[st], ph))) break;
+                    if (sl == 0) K512_STAMP(t, 2);
+                    auto issue_so = [&]() {
                         tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
-                            mma_bf16(od, kdesc(qa + off), mn64(sbase + C::HB + kk * 2048), idO, (sl > 0 || kk > 0) ? 1u : 0u);
+                            const uint32_t c = (kk & 3) * 32;
+                            mma_bf16(dso, kdesc(qa + (kk >> 2) * kRegion + c), kdesc(ka + (kk >> 2) * C::KREG + c), idSO,
+                                     (sl > 0 || kk > 0) ? 1u : 0u);
                         }
-                        mma_commit(b_hbfree);
-                        if (sl == KS - 1) mma_commit(b_o1);
-                        return true;
-                    };
-                    auto issue_s = [&]() {
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t off = (kk >> 2) * kRegion + (kk & 3) * 32;
-                            mma_bf16(tmem + C::COL_S, kdesc(qa + off), kdesc(ka + off), idS, (sl > 0 || kk > 0) ? 1u : 0u);
-                        }
+                        mma_commit(&empty_q[st]);
                         if (sl == KS - 1) mma_commit(b_s);
                     };
                     auto issue_h = [&]() {
                         tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            mma_bf16(tmem + C::COL_H + sl * BV, sdesc(ka + kk * 2048, kRegion, 1024, 2),
-                                     mn64(sbase + C::VW + kk * 2048), idH, 1u);
+                            mma_bf16(tmem + C::COL_H + sl * BV, sdesc(ka + koff + kk * 2048, C::KREG, 1024, 2),
+                                     mn64(vw + kk * 2048), idH, 1u);
                         mma_commit(&b_hdone[sl]);
                     };
                     if (sl == 0) {
-                        if (!(ok = issue_o1())) break;
-                        if (!(ok = wait(&full_u[sk], (xk / C::NU) & 1))) break;
-                        if (!(ok = wait(b_vw, t & 1))) break;
+                        if (!(ok = wait(&b_vw[t & 1], (t >> 1) & 1))) break;
                         K512_STAMP(t, 4);
                         issue_h();
                         if (t >= 1 && !(ok = wait(b_pv, (t - 1) & 1))) break;
+                        if (t >= 2 && !(ok = wait(&b_ofree[t & 1], ((t >> 1) - 1) & 1))) break;
                         K512_STAMP(t, 3);
-                        issue_s();
-                        mma_commit(&empty_u[sq]);
+                        issue_so();
                     } else {
-                        if (!(ok = wait(&full_u[sk], (xk / C::NU) & 1))) break;
-                        issue_s();
-                        if (!(ok = issue_o1())) break;
-                        mma_commit(&empty_u[sq]);
+                        issue_so();
                         issue_h();
                     }
-                    mma_commit(&empty_u[sk]);
+                    mma_commit(&empty_k[st]);
                 }
                 if (!ok) break;
                 K512_STAMP(t, 8);
@@ -419,7 +420,7 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         const int i = threadIdx.x - 128;
         const uint32_t hrow = tmem + ((uint32_t)((warp - 4) * 32) << 16) + C::COL_H;
         const int64_t KV = (int64_t)a.K * V;
-        // V(t) -> V_w = w ⊙ V (own buffer) and V_f = f ⊙ V (in place), 0 past the end;
+        // V(t) -> V_w = w ⊙ V (buffer t & 1) and V_f = f ⊙ V (in place), 0 past the end;
         // each product of a bf16 pair with an fp32 weight is rounded once
         auto v_pass = [&](int t) {
             const int st = t & 1;
@@ -435,7 +436,7 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                 const __nv_bfloat162 wh = __float2bfloat162_rn(w), wl = __float2bfloat162_rn(w - __low2float(wh));
                 const __nv_bfloat162 fh = __float2bfloat162_rn(f), fl = __float2bfloat162_rn(f - __low2float(fh));
                 uint4 *vrow = reinterpret_cast<uint4 *>(sm + C::V0 + st * kRegion + i * 128);
-                uint4 *wrow = reinterpret_cast<uint4 *>(sm + C::VW + i * 128);
+                uint4 *wrow = reinterpret_cast<uint4 *>(sm + C::VW + st * kRegion + i * 128);
                 // thread i starts at chunk i % 8, so a quarter-warp's 16-byte accesses fall in
                 // different bank groups (the row is scaled as a whole, the swizzle is irrelevant)
 #pragma unroll
@@ -456,35 +457,52 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                 }
                 fence_proxy_async_smem();
             }
-            mbar_arrive(b_vw);
+            mbar_arrive(&b_vw[st]);
         };
-        // block sl of the state entering step t (x: its row i, 64 columns in two pieces)
-        // -> Hb (bf16) and H block sl (times the decay of step t)
-        auto block_out = [&](int sl, int pc, float (&x)[32], float gam) {
-            store_row32_bf16<128>(sm + C::HB, i, 32 * pc, x);
+        // columns 32 pc .. 32 pc + 31 of row i of state block s (x) -> the transposed bf16
+        // block Hb_s^T in the K slot: row v of Hb^T holds k = 128 s + 0..127 over the two
+        // 64-k regions, after the K rows (odd steps) or before them (even steps).  Lanes i
+        // and i ^ 1 swap one value per pair of rows (v, v ^ 4) so that each lane stores one
+        // 32-bit pair of adjacent k and a warp's store covers two rows in disjoint banks.
+        auto hbt_piece = [&](unsigned char *slot, bool ev, int pc, const float (&x)[32]) {
+            unsigned char *reg = slot + (i >> 6) * C::KREG;
+            const int row0 = ev ? 0 : 128, c = (i & 63) & ~1;
+            const bool odd = i & 1;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] *= gam;
-            tmem_st32(hrow + sl * BV + 32 * pc, x);
+            for (int j = 0; j < 16; ++j) {
+                const int a = (j & 3) | ((j >> 2) << 3);  // bit 2 clear: rows a and a | 4
+                const float send = odd ? x[a] : x[a | 4];
+                const float keep = odd ? x[a | 4] : x[a];
+                const float r = __shfl_xor_sync(0xffffffffu, send, 1);
+                const uint32_t w2 = odd ? pack_bf16(r, keep) : pack_bf16(keep, r);
+                const int row = row0 + 32 * pc + (odd ? (a | 4) : a);
+                const uint32_t off = row * 128 + ((((c >> 3) ^ row) & 7) << 4) + (c & 7) * 2;
+                *reinterpret_cast<uint32_t *>(reg + off) = w2;
+            }
         };
-        auto block_done = [&]() {
-            tmem_wait_st();
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(b_hb);
-        };
+        const float *src = nullptr;  // state entering the segment
+        if (s == 0) src = a.h0 ? a.h0 + ((int64_t)n * H + h) * KV : nullptr;
+        else src = a.seg_state + ((int64_t)(u - 1) * H + h) * KV;
         bool ok = true;
-        if (nsteps > 0) {  // step 0: the state entering the segment
-            const float *src = nullptr;
-            if (s == 0) src = a.h0 ? a.h0 + ((int64_t)n * H + h) * KV : nullptr;
-            else src = a.seg_state + ((int64_t)(u - 1) * H + h) * KV;
-            const float gam = exp2f(last_gate(0));
+        if (nsteps > 0) v_pass(0);
+        for (int t = 0; ok && t < nsteps; ++t) {
+            const float gam = exp2f(last_gate(t));  // decay of step t, applied to the entering state
+            const bool ev = (t & 1) == 0;
 #pragma unroll 1
             for (int sl = 0; sl < KS; ++sl) {
-                if (sl >= 1 && !(ok = mbar_wait(b_hbfree, (sl - 1) & 1, abort_flag))) break;
+                const int q = t * KS + sl, st = q & 1;
+                if (t >= 1 && !(ok = mbar_wait(&b_hdone[sl], (t - 1) & 1, abort_flag))) break;
+                if (q >= 2 && !(ok = mbar_wait(&empty_k[st], ((q >> 1) - 1) & 1, abort_flag))) break;
+                if (i == 0) K512_STAMP(t, 14 + 2 * sl);
+                tc_fence_after();
+                unsigned char *slot = sm + C::KR + st * C::KUNIT;
 #pragma unroll 1
                 for (int pc = 0; pc < 2; ++pc) {
                     float x[32];
-                    if (src) {
+                    if (t >= 1) {
+                        tmem_ld32(hrow + sl * BV + 32 * pc, x);
+                        tmem_wait_ld();
+                    } else if (src) {
                         const float4 *p4 =
                             reinterpret_cast<const float4 *>(src + (int64_t)(128 * sl + i) * V + v0 + 32 * pc);
 #pragma unroll
@@ -496,37 +514,21 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
 #pragma unroll
                         for (int e = 0; e < 32; ++e) x[e] = 0.f;
                     }
-                    block_out(sl, pc, x, gam);
+                    hbt_piece(slot, ev, pc, x);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[e] *= gam;
+                    tmem_st32(hrow + sl * BV + 32 * pc, x);
                 }
-                block_done();
-                if (sl == 0) v_pass(0);
-            }
-        }
-        // later steps: block sl once H_sl of the previous step is done and Hb has been read
-        // by the O1 products of the block before; V_w(t) once H(t-1) is done
-        for (int t = 1; ok && t < nsteps; ++t) {
-            const float gam = exp2f(last_gate(t));  // decay of step t, applied to the entering state
-#pragma unroll 1
-            for (int sl = 0; sl < KS; ++sl) {
-                const int use = t * KS + sl;
-                if (!(ok = mbar_wait(&b_hdone[sl], (t - 1) & 1, abort_flag))) break;
-                if (!(ok = mbar_wait(b_hbfree, (use - 1) & 1, abort_flag))) break;
-                if (i == 0) K512_STAMP(t, 14 + 2 * sl);
-                tc_fence_after();
-#pragma unroll 1
-                for (int pc = 0; pc < 2; ++pc) {
-                    float x[32];
-                    tmem_ld32(hrow + sl * BV + 32 * pc, x);
-                    tmem_wait_ld();
-                    block_out(sl, pc, x, gam);
-                }
-                block_done();
+                tmem_wait_st();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&b_hbt[st]);
                 if (i == 0) K512_STAMP(t, 15 + 2 * sl);
-                if (sl == 0) {
-                    if (!(ok = mbar_wait(&b_hdone[KS - 1], (t - 1) & 1, abort_flag))) break;
-                    v_pass(t);
-                    if (i == 0) K512_STAMP(t, 22);
-                }
+            }
+            // V_w(t+1) goes to the buffer H(t-1) read, which the block passes above waited for
+            if (ok && t + 1 < nsteps) {
+                v_pass(t + 1);
+                if (i == 0) K512_STAMP(t + 1, 22);
             }
         }
         // the state after the segment's last step
@@ -552,16 +554,16 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     } else if (warp < 12) {
         // ---------------------------------------------------------------- WG_O: output rows
         const int i = threadIdx.x - 256;
-        const uint32_t trow = tmem + ((uint32_t)((warp - 8) * 32) << 16) + C::COL_O;
+        const uint32_t trow = tmem + ((uint32_t)((warp - 8) * 32) << 16);
         const bool o32 = (reinterpret_cast<uintptr_t>(a.o) & 31) == 0;  // 32-byte row segments
         float gnext = nsteps > 0 ? gate_of(0, i) : 0.f;
         for (int t = 0; t < nsteps; ++t) {
             const StepSpan sp = step_span(t0, t1, cb + t);
             const float gi = gnext;
             gnext = (t + 1 < nsteps) ? gate_of(t + 1, i) : 0.f;
-            const uint32_t orow = trow + (t & 1) * BV;
+            const uint32_t orow = trow + ((t & 1) ? C::COL_OB : C::COL_OA);
             // O1 row i times scale 2^G~_i, in place, before P' V_f accumulates onto it
-            if (!mbar_wait(b_o1, t & 1, abort_flag)) break;
+            if (!mbar_wait(b_s, t & 1, abort_flag)) break;
             if (i == 0) K512_STAMP(t, 23);
             tc_fence_after();
             {
