@@ -83,7 +83,8 @@ struct Plan {
     int C = 0, L = 1, NT = 0, NS = 0;
     int64_t max_chunks = 0, max_segs = 0;
     bool multi_seg = false;    // some sequence may have more than one segment
-    size_t off_chunk_off = 0, off_seg_off = 0, off_gcum = 0, off_gpos = 0, off_seg_dec = 0, off_seg_state = 0;
+    size_t off_chunk_off = 0, off_seg_off = 0, off_seg_order = 0, off_gcum = 0, off_gpos = 0, off_seg_dec = 0,
+           off_seg_state = 0;
     size_t off_state_in = 0, off_state_out = 0;  // [K,V] copies of [V,K] states (state_v_first)
     size_t bytes = 0;
 };
@@ -142,6 +143,35 @@ Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t 
         for (int64_t ns = 1; ns <= std::min<int64_t>(nt, 512); ++ns) {
             const int64_t l = (nt + ns - 1) / ns, ns_eff = (nt + l - 1) / l;
             if (l < min_l) break;
+            if (varlen) {
+                // packed batches: the segments of unequal sequences are dispatched longest
+                // first (seg_order) as SMs free up, so the walk takes the larger of its
+                // longest segment and its total work spread over the SMs; sequences of a
+                // uniform length mix hold mean/l + 1/2 segments each
+                const double mean_steps = (double)T / ((double)std::max<int64_t>(N, 1) * (double)C);
+                const double segs = (double)N * std::max(1.0, mean_steps / (double)l + 0.5);
+                const double steps = (double)T / (double)C;
+                const double t_w = state_only ? 0.0
+                                   : std::max({(double)(l + 2) * t_walk,
+                                               (double)units / (double)std::max<int64_t>(N, 1) *
+                                                   (steps + 2.0 * segs) * t_walk / 148.0,
+                                               walk_bytes / bw});
+                const double seg_state = state_only ? segs : std::max(0.0, segs - (double)N);
+                double t_s = 0.0;
+                if (seg_state > 0.0) {
+                    const double frac = std::min(1.0, seg_state * (double)l / std::max(steps, 1.0));
+                    t_s = std::max({(double)(l + 1) * t_state,
+                                    (double)state_units / (double)std::max<int64_t>(N, 1) * seg_state *
+                                        (double)(l + 1) * t_state / 148.0,
+                                    kv_bytes * frac / bw_state});
+                    if (state_only) t_s += segs * (double)H * (double)K * (double)V * 4.0 / bw;
+                }
+                if (t_w + t_s < best - 1e-9) {
+                    best = t_w + t_s;
+                    L = l;
+                }
+                continue;
+            }
             const double waves_walk = (double)((units * ns_eff + 147) / 148);
             const double t_w = state_only ? 0.0 : std::max(waves_walk * (double)(l + 2) * t_walk, walk_bytes / bw);
             double t_s = 0.0;
@@ -181,13 +211,16 @@ Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t 
         p.max_segs = N * p.NS;
         p.multi_seg = p.NS > 1 || state_only;
     }
-    if (p.max_chunks >= kMaxTokens || p.max_segs * H >= kMaxTokens) { p.why = SGLA_ERR_UNSUPPORTED; return p; }
+    // segment grids are flattened over (segment, head, tile), at most 32 tiles
+    if (p.max_chunks >= kMaxTokens || p.max_segs * H * 32 >= kMaxTokens) { p.why = SGLA_ERR_UNSUPPORTED; return p; }
     size_t off = 256;  // status word
     if (varlen) {
         p.off_chunk_off = off;
         off = align_up(off + sizeof(int) * (size_t)(N + 1), 256);
         p.off_seg_off = off;
         off = align_up(off + sizeof(int) * (size_t)(N + 1), 256);
+        p.off_seg_order = off;
+        off = align_up(off + sizeof(int) * (size_t)p.max_segs, 256);
     }
     if (per_token_gate) {
         p.off_gcum = off;
@@ -252,6 +285,7 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
     lay.cu = varlen ? cu : nullptr;
     lay.chunk_off = varlen ? reinterpret_cast<int *>(ws + p.off_chunk_off) : nullptr;
     lay.seg_off = varlen ? reinterpret_cast<int *>(ws + p.off_seg_off) : nullptr;
+    lay.seg_order = varlen ? reinterpret_cast<int *>(ws + p.off_seg_order) : nullptr;
     lay.status = reinterpret_cast<int *>(ws);
     a.dev_status = reinterpret_cast<int *>(ws);
     lay.T = T; lay.N = (int)N; lay.H = (int)H; lay.C = p.C; lay.L = p.L;
@@ -259,9 +293,10 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
     lay.max_chunks = (int)p.max_chunks; lay.max_segs = (int)p.max_segs;
 
     if (varlen) {
-        SGLA_LAUNCH("varlen_plan", launch_varlen_plan(cu, (int)N, T, p.C, p.L, const_cast<int *>(lay.chunk_off),
-                                                      const_cast<int *>(lay.seg_off),
-                                                      reinterpret_cast<int *>(ws), st));
+        SGLA_LAUNCH("varlen_plan", launch_varlen_plan(cu, (int)N, T, p.C, p.L, (int)p.max_segs,
+                                                      const_cast<int *>(lay.chunk_off), const_cast<int *>(lay.seg_off),
+                                                      const_cast<int *>(lay.seg_order), reinterpret_cast<int *>(ws),
+                                                      a.h0, (p.tc && !state_v_first) ? a.hT : nullptr, H * K * V, st));
     } else {
         SGLA_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), st), "status reset");
     }
@@ -274,7 +309,13 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
         else SGLA_LAUNCH("segment_state_simt", launch_segment_state_simt(a, st));
     }
     const bool empty_dense = !varlen && p.NT == 0;
-    if (p.multi_seg || (empty_dense && hT)) SGLA_LAUNCH("segment_carry", launch_segment_carry(a, p.multi_seg, st));
+    // the tensor-core walks form their entering states from the segment states
+    // themselves, and the plan kernel writes the final states of empty packed sequences
+    // (with the [V,K] layout that copy waits for the transposed initial state: the carry
+    // pass does it)
+    if (p.multi_seg && !p.tc) SGLA_LAUNCH("segment_carry", launch_segment_carry(a, true, st));
+    else if (hT && (empty_dense || (varlen && state_v_first)))
+        SGLA_LAUNCH("segment_carry", launch_segment_carry(a, false, st));
     if (tokens > 0 && p.max_segs > 0) {
         if (p.tc) SGLA_LAUNCH("chunk_output_tc", tc_launch_chunk_output(a, st));
         else SGLA_LAUNCH("chunk_output_simt", launch_chunk_output_simt(a, st));
@@ -529,15 +570,17 @@ sgla_status simple_gla_chunk_final_state(const void *k, const void *v, const flo
     lay.cu = varlen ? cu_seqlens : nullptr;
     lay.chunk_off = varlen ? reinterpret_cast<int *>(ws + p.off_chunk_off) : nullptr;
     lay.seg_off = varlen ? reinterpret_cast<int *>(ws + p.off_seg_off) : nullptr;
+    lay.seg_order = varlen ? reinterpret_cast<int *>(ws + p.off_seg_order) : nullptr;
     lay.status = reinterpret_cast<int *>(ws);
     a.dev_status = reinterpret_cast<int *>(ws);
     lay.T = T; lay.N = (int)N; lay.H = (int)H; lay.C = p.C; lay.L = p.L;
     lay.NT = p.NT; lay.NS = p.NS;
     lay.max_chunks = (int)p.max_chunks; lay.max_segs = (int)p.max_segs;
     if (varlen) {
-        SGLA_LAUNCH("varlen_plan", launch_varlen_plan(cu_seqlens, (int)N, T, p.C, p.L,
-                                                      const_cast<int *>(lay.chunk_off),
-                                                      const_cast<int *>(lay.seg_off), reinterpret_cast<int *>(ws), st));
+        SGLA_LAUNCH("varlen_plan", launch_varlen_plan(cu_seqlens, (int)N, T, p.C, p.L, (int)p.max_segs,
+                                                      const_cast<int *>(lay.chunk_off), const_cast<int *>(lay.seg_off),
+                                                      const_cast<int *>(lay.seg_order), reinterpret_cast<int *>(ws),
+                                                      nullptr, nullptr, 0, st));
     } else {
         SGLA_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), st), "status reset");
     }
@@ -671,9 +714,9 @@ sgla_status gla_chunk(const void *q, const void *k, const void *v, const float *
     lay.T = T; lay.N = (int)N; lay.H = (int)H; lay.C = L.C; lay.L = 1; lay.NT = L.NT; lay.NS = L.NT;
     lay.max_chunks = (int)L.max_chunks; lay.max_segs = (int)L.max_chunks;
     if (varlen) {
-        SGLA_LAUNCH("varlen_plan", launch_varlen_plan(cu_seqlens, (int)N, T, L.C, 1, const_cast<int *>(lay.chunk_off),
-                                                      const_cast<int *>(lay.seg_off), reinterpret_cast<int *>(ws),
-                                                      st));
+        SGLA_LAUNCH("varlen_plan", launch_varlen_plan(cu_seqlens, (int)N, T, L.C, 1, 0, const_cast<int *>(lay.chunk_off),
+                                                      const_cast<int *>(lay.seg_off), nullptr,
+                                                      reinterpret_cast<int *>(ws), nullptr, nullptr, 0, st));
     } else {
         SGLA_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), st), "status reset");
     }

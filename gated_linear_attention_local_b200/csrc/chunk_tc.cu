@@ -68,15 +68,15 @@ tc_segment_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_con
     const SeqLayout &lay = a.lay;
     if (device_failed(lay)) return;
     const int VT = a.V / kStateBV, KB = a.K / 128;
-    const int u = blockIdx.x / (VT * KB);
-    const int rem = blockIdx.x % (VT * KB);
+    const SegWork wk = seg_work(lay, blockIdx.x, VT * KB);
+    const int u = wk.u, rem = wk.tile;
     const int kb = rem / VT;
     const int v0 = (rem % VT) * kStateBV;
     int n, s;
     if (!locate_segment(lay, u, n, s)) return;
     const int nseg = seq_segments(lay, n);
     if (s == nseg - 1 && !a.state_all) return;  // the last end state is needed on a state-only call
-    const int h = blockIdx.y, H = a.H, V = a.V;
+    const int h = wk.h, H = a.H, V = a.V;
     int64_t t0, t1;
     seq_span(lay, n, t0, t1);
     const int nt = (int)((t1 - t0 + kStep - 1) / kStep);
@@ -257,7 +257,7 @@ cudaError_t tc_launch_segment_state(const FwdArgs &a, cudaStream_t st) {
     if ((e = cudaFuncSetAttribute(tc_segment_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kStateSmem)) != cudaSuccess)
         return e;
-    dim3 grid(a.lay.max_segs * (a.V / kStateBV) * (a.K / 128), a.H);
+    dim3 grid(a.lay.max_segs * a.H * (a.V / kStateBV) * (a.K / 128));
     tc_segment_state_kernel<<<grid, kStateThreads, kStateSmem, st>>>(tk, tv, a);
     return cudaGetLastError();
 }

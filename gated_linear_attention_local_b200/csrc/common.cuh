@@ -70,6 +70,7 @@ struct SeqLayout {
     const int64_t *cu;     // varlen: device [N+1]; dense: nullptr
     const int *chunk_off;  // varlen: [N+1] prefix sums of chunks per sequence (workspace)
     const int *seg_off;    // varlen: [N+1] prefix sums of segments per sequence (workspace)
+    const int *seg_order;  // varlen: [max_segs] segment units, longest first (workspace); dense: nullptr
     const int *status;     // device status word (workspace)
     int64_t T;             // dense: tokens per sequence; varlen: total tokens
     int N;                 // sequences
@@ -122,6 +123,23 @@ __device__ __forceinline__ bool locate_segment(const SeqLayout &s, int u, int &n
     n = upper_index(s.seg_off, s.N, u);
     seg = u - s.seg_off[n];
     return true;
+}
+
+// Work item `idx` of a segment-level grid flattened as [rank][head][tile]: the segment
+// unit (the rank-th longest segment of a packed batch, or segment `rank` of a dense
+// one), its head and its tile.  The block scheduler starts blocks in index order, so
+// every head's longest segments start first and the short ones fill in behind them.
+struct SegWork {
+    int u, h, tile;
+};
+__device__ __forceinline__ SegWork seg_work(const SeqLayout &s, int idx, int tiles) {
+    const int per_rank = s.H * tiles;
+    const int r = idx / per_rank, rem = idx - r * per_rank;
+    SegWork w;
+    w.h = rem / tiles;
+    w.tile = rem - w.h * tiles;
+    w.u = (s.seg_order && r < s.max_segs) ? s.seg_order[r] : r;
+    return w;
 }
 
 // Global chunk index u -> (sequence n, chunk c within it).  False past the end.

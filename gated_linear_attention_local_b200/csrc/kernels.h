@@ -31,9 +31,13 @@ struct FwdArgs {
     SeqLayout lay;
 };
 
-// Plan for packed batches: validate cu_seqlens, fill chunk_off / seg_off, set status.
-cudaError_t launch_varlen_plan(const int64_t *cu, int N, int64_t T_total, int C, int L,
-                               int *chunk_off, int *seg_off, int *status, cudaStream_t st);
+// Plan for packed batches: validate cu_seqlens, fill chunk_off / seg_off and the
+// longest-first dispatch order of the segments (seg_order), set status; when hT is
+// given, write the final state of every empty sequence (its initial state h0, or 0;
+// state_elems = H K V floats per sequence).
+cudaError_t launch_varlen_plan(const int64_t *cu, int N, int64_t T_total, int C, int L, int max_segs,
+                               int *chunk_off, int *seg_off, int *seg_order, int *status, const float *h0, float *hT,
+                               int64_t state_elems, cudaStream_t st);
 
 // Chunk-local inclusive cumsum of g times 1/ln2 (warp-shuffle scan).
 cudaError_t launch_chunk_cumsum(const float *g, float *gcum, int *gpos, const SeqLayout &lay, cudaStream_t st);

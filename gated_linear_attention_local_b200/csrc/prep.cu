@@ -15,6 +15,7 @@ namespace sgla {
 // zero (so no kernel finds work) and the status word records the failure.
 // ---------------------------------------------------------------------------
 constexpr int kPlanThreads = 1024;
+constexpr int kLptMaxL = 1024;  // longest segment (chunks) the dispatch-order sort takes
 
 __device__ __forceinline__ int block_exclusive_scan(int x, int &total, int *warp_sums) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -45,10 +46,12 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int &total, int *warp
 }
 
 __global__ void __launch_bounds__(kPlanThreads)
-varlen_plan_kernel(const int64_t *__restrict__ cu, int N, int64_t T_total, int C, int L,
-                   int *__restrict__ chunk_off, int *__restrict__ seg_off, int *__restrict__ status) {
+varlen_plan_kernel(const int64_t *__restrict__ cu, int N, int64_t T_total, int C, int L, int max_segs,
+                   int *__restrict__ chunk_off, int *__restrict__ seg_off, int *__restrict__ seg_order,
+                   int *__restrict__ status, const float *__restrict__ h0, float *__restrict__ hT, int64_t state_elems) {
     __shared__ int warp_sums[33];
     __shared__ int bad;
+    __shared__ int cursor[kLptMaxL + 1];
     if (threadIdx.x == 0) bad = (cu[0] != 0 || cu[N] != T_total) ? 1 : 0;
     __syncthreads();
     for (int n = threadIdx.x; n < N; n += blockDim.x)
@@ -79,11 +82,55 @@ varlen_plan_kernel(const int64_t *__restrict__ cu, int N, int64_t T_total, int C
         seg_off[N] = run_s;
         *status = ok ? kDevOk : kDevBadCuSeqlens;
     }
+    // the final state of an empty sequence is its initial state (no walk runs for it)
+    if (ok && hT)
+        for (int n = 0; n < N; ++n)
+            if (cu[n + 1] == cu[n]) {
+                const int64_t base = (int64_t)n * state_elems;
+                for (int64_t e = threadIdx.x; e < state_elems; e += blockDim.x) hT[base + e] = h0 ? h0[base + e] : 0.f;
+            }
+    if (!seg_order) return;
+    // dispatch order of the segments, longest first: a counting sort on the length in
+    // chunks (every segment but the last of its sequence has L chunks); ranks past the
+    // last segment map to themselves, which locate_segment() rejects
+    const bool lpt = ok && L <= kLptMaxL;
+    for (int i = threadIdx.x; i <= kLptMaxL; i += blockDim.x) cursor[i] = 0;
+    __syncthreads();
+    if (lpt)
+        for (int n = threadIdx.x; n < N; n += blockDim.x) {
+            const int nc = (int)((cu[n + 1] - cu[n] + C - 1) / C), ns = (nc + L - 1) / L;
+            if (ns == 0) continue;
+            if (ns > 1) atomicAdd(&cursor[L], ns - 1);
+            atomicAdd(&cursor[nc - (ns - 1) * L], 1);
+        }
+    __syncthreads();
+    if (threadIdx.x == 0 && lpt) {  // bucket starts, longest bucket first
+        int run = 0;
+        for (int len = L; len >= 1; --len) {
+            const int c = cursor[len];
+            cursor[len] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    if (lpt)
+        for (int n = threadIdx.x; n < N; n += blockDim.x) {
+            const int nc = (int)((cu[n + 1] - cu[n] + C - 1) / C), ns = (nc + L - 1) / L;
+            const int first = seg_off[n];
+            for (int s = 0; s < ns; ++s) {
+                const int len = (s < ns - 1) ? L : nc - (ns - 1) * L;
+                seg_order[atomicAdd(&cursor[len], 1)] = first + s;
+            }
+        }
+    const int from = lpt ? run_s : 0;
+    for (int r = from + threadIdx.x; r < max_segs; r += blockDim.x) seg_order[r] = r;
 }
 
-cudaError_t launch_varlen_plan(const int64_t *cu, int N, int64_t T_total, int C, int L,
-                               int *chunk_off, int *seg_off, int *status, cudaStream_t st) {
-    varlen_plan_kernel<<<1, kPlanThreads, 0, st>>>(cu, N, T_total, C, L, chunk_off, seg_off, status);
+cudaError_t launch_varlen_plan(const int64_t *cu, int N, int64_t T_total, int C, int L, int max_segs,
+                               int *chunk_off, int *seg_off, int *seg_order, int *status, const float *h0, float *hT,
+                               int64_t state_elems, cudaStream_t st) {
+    varlen_plan_kernel<<<1, kPlanThreads, 0, st>>>(cu, N, T_total, C, L, max_segs, chunk_off, seg_off, seg_order,
+                                                   status, h0, hT, state_elems);
     return cudaGetLastError();
 }
 
@@ -179,7 +226,8 @@ cudaError_t launch_chunk_cumsum(const float *g, float *gcum, int *gpos, const Se
 }
 
 // ---------------------------------------------------------------------------
-// Cross-segment carry, one thread per 4 state elements of one (sequence, head).
+// Cross-segment carry, one thread per 4 state elements of one (sequence, head), for
+// the CUDA-core walk (the tensor-core walks fold the segment states themselves).
 // seg_state[u] holds segment u's local end state (from zero) on entry and the
 // state ENTERING segment u+1 on exit; seg_dec[u] is segment u's log2 total decay.
 // Also writes final_state for empty sequences (initial state unchanged).  On a

@@ -53,12 +53,12 @@ tc_state_k128_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
     const SeqLayout &lay = a.lay;
     if (device_failed(lay)) return;
     const int VT = a.V / 128;
-    const int u = blockIdx.x / VT;
-    const int v0 = (blockIdx.x % VT) * 128;
+    const SegWork wk = seg_work(lay, blockIdx.x, VT);
+    const int u = wk.u, v0 = wk.tile * 128;
     int n, s;
     if (!locate_segment(lay, u, n, s)) return;
     if (s == seq_segments(lay, n) - 1 && !a.state_all) return;  // needed only on a state-only call
-    const int h = blockIdx.y, H = a.H, V = a.V;
+    const int h = wk.h, H = a.H, V = a.V;
     int64_t t0, t1;
     seq_span(lay, n, t0, t1);
     const int nt = (int)((t1 - t0 + kStep - 1) / kStep);
@@ -193,7 +193,7 @@ cudaError_t tc_launch_state_k128(const FwdArgs &a, cudaStream_t st) {
     if ((e = cudaFuncSetAttribute(tc_state_k128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)S128Cfg::SMEM)) != cudaSuccess)
         return e;
-    dim3 grid(a.lay.max_segs * (a.V / 128), a.H);
+    dim3 grid(a.lay.max_segs * a.H * (a.V / 128));
     tc_state_k128_kernel<<<grid, kS128Threads, S128Cfg::SMEM, st>>>(tk, tv, a);
     return cudaGetLastError();
 }

@@ -45,6 +45,11 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
 // K-major 128-byte-swizzled operand (Q, K as the B of Q K^T): 8-row atoms 1024 B apart.
 __device__ __forceinline__ uint64_t kdesc(uint32_t saddr) { return sdesc(saddr, 16, 1024, 2); }
 
+// The descriptor of an operand `bytes` further into shared memory: the start address
+// is the low 14-bit field in 16-byte units, and every shared-memory address here is
+// below 2^18, so the field never carries into the next one.
+__device__ __forceinline__ uint64_t desc_at(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
 __device__ __forceinline__ unsigned char *align1024(unsigned char *p) {
     return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
@@ -148,6 +153,41 @@ __device__ __forceinline__ StepSpan step_span(int64_t t0, int64_t t1, int step) 
 }
 
 __device__ __forceinline__ void record_timeout(const FwdArgs &a) { atomicCAS(a.dev_status, kDevOk, kDevTimeout); }
+
+// Columns c0 .. c0 + 31 of row `row` of the state entering segment s of sequence n
+// (head h): the initial state (or 0) folded with the local end states of segments
+// 0 .. s-1 that the state pass left in seg_state, h <- 2^(log2 decay) h + S_p, one fma
+// per element and segment in segment order (the scalar-decay carry of the article's
+// section 3).  A walk forms its own entering state this way, so no separate carry pass
+// runs between the state pass and the walk.
+__device__ __forceinline__ void entering_state_row32(const FwdArgs &a, int n, int s, int first_seg, int h,
+                                                     int64_t row, int c0, float (&x)[32]) {
+    const int64_t KV = (int64_t)a.K * a.V, off = row * a.V + c0;
+    if (a.h0) {
+        const float4 *p4 = reinterpret_cast<const float4 *>(a.h0 + ((int64_t)n * a.H + h) * KV + off);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float4 f = p4[e];
+            x[4 * e] = f.x; x[4 * e + 1] = f.y; x[4 * e + 2] = f.z; x[4 * e + 3] = f.w;
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = 0.f;
+    }
+    for (int p = 0; p < s; ++p) {
+        const int64_t seg = first_seg + p;
+        const float dec = exp2f(a.seg_dec[seg * a.H + h]);
+        const float4 *d4 = reinterpret_cast<const float4 *>(a.seg_state + (seg * a.H + h) * KV + off);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float4 d = d4[e];
+            x[4 * e] = fmaf(dec, x[4 * e], d.x);
+            x[4 * e + 1] = fmaf(dec, x[4 * e + 1], d.y);
+            x[4 * e + 2] = fmaf(dec, x[4 * e + 2], d.z);
+            x[4 * e + 3] = fmaf(dec, x[4 * e + 3], d.w);
+        }
+    }
+}
 
 }  // namespace
 }  // namespace sgla

@@ -119,12 +119,12 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     const SeqLayout &lay = a.lay;
     if (device_failed(lay)) return;
     const int VT = a.V / BV;
-    const int u = blockIdx.x / VT;            // V tiles of one (segment, head) are adjacent
-    const int v0 = (blockIdx.x % VT) * BV;
+    const SegWork wk = seg_work(lay, blockIdx.x, VT);  // longest segments first, V tiles adjacent
+    const int u = wk.u, v0 = wk.tile * BV;
     int n, s;
     if (!locate_segment(lay, u, n, s)) return;
     const int nseg = seq_segments(lay, n);
-    const int h = blockIdx.y, H = a.H, V = a.V;
+    const int h = wk.h, H = a.H, V = a.V;
     int64_t t0, t1;
     seq_span(lay, n, t0, t1);
     const int nt = (int)((t1 - t0 + kStep - 1) / kStep);
@@ -477,24 +477,12 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         };
         // state entering the segment -> Hb (bf16) and H (times the first step's decay)
         {
-            const float *src = nullptr;
-            if (s == 0) src = a.h0 ? a.h0 + ((int64_t)n * H + h) * KV : nullptr;
-            else src = a.seg_state + ((int64_t)(u - 1) * H + h) * KV;
+            const int first = u - s;  // segment units of a sequence are consecutive
             const float gam = nsteps > 0 ? exp2f(last_gate(0)) : 1.f;
 #pragma unroll 1
             for (int pc = 0; pc < C::NP; ++pc) {
                 float x[32];
-                if (src) {
-                    const float4 *p4 = reinterpret_cast<const float4 *>(src + (int64_t)i * V + v0 + 32 * pc);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float4 f = p4[e];
-                        x[4 * e] = f.x; x[4 * e + 1] = f.y; x[4 * e + 2] = f.z; x[4 * e + 3] = f.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] = 0.f;
-                }
+                entering_state_row32(a, n, s, first, h, i, v0 + 32 * pc, x);
                 hb_piece(pc, x);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) x[e] *= gam;
@@ -700,7 +688,7 @@ cudaError_t launch_k128(const FwdArgs &a, cudaStream_t st) {
     auto kern = tc_walk_k128_kernel<BV>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM)) != cudaSuccess)
         return e;
-    dim3 grid(a.lay.max_segs * (a.V / BV), a.H);
+    dim3 grid(a.lay.max_segs * a.H * (a.V / BV));
     kern<<<grid, kK128Threads, C::SMEM, st>>>(tq, tk, tv, to, a);
     return cudaGetLastError();
 }

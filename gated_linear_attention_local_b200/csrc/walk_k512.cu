@@ -98,12 +98,12 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     const SeqLayout &lay = a.lay;
     if (device_failed(lay)) return;
     const int VT = a.V / BV;
-    const int u = blockIdx.x / VT;            // V tiles of one (segment, head) are adjacent
-    const int v0 = (blockIdx.x % VT) * BV;
+    const SegWork wk = seg_work(lay, blockIdx.x, VT);  // longest segments first, V tiles adjacent
+    const int u = wk.u, v0 = wk.tile * BV;
     int n, s;
     if (!locate_segment(lay, u, n, s)) return;
     const int nseg = seq_segments(lay, n);
-    const int h = blockIdx.y, H = a.H, V = a.V;
+    const int h = wk.h, H = a.H, V = a.V;
     int64_t t0, t1;
     seq_span(lay, n, t0, t1);
     const int nt = (int)((t1 - t0 + kStep - 1) / kStep);
@@ -181,46 +181,66 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     if (warp == 12) {
         // ---------------------------------------------------------------- TMA loads
         // Slice q = t KS + sl: Q_s into Q slot q & 1, K_s into the K rows of K slot q & 1
-        // (after the 64 rows of Hb^T on even steps, before them on odd steps).  V(t) goes
-        // out just before slice t KS: its stage is freed by P V(t-2), which retires
-        // before the slot that slice waits for.
+        // (after the 64 rows of Hb^T on even steps, before them on odd steps); slice 0 of
+        // a step loads K first (its H product, issued first, needs only K).  The copies
+        // of an SM land roughly in issue order, so V(t) goes out two slices ahead of step
+        // t (after slice t KS - 2; its stage was freed by P V(t-2), which retired before
+        // that slice's slots).
         if (lane == 0) {
             prefetch_tmap(&tq);
             prefetch_tmap(&tk);
             prefetch_tmap(&tv);
-            int issued = 0, issued_v = 0;
+            int issued_q = 0, issued_k = 0, issued_v = 0;  // loads issued so far (slices, steps)
             const int total = nsteps * KS;
-            for (int q = 0; q < total; ++q) {
+            auto load_v = [&](int t) -> bool {
+                const int vs = t & 1;
+                if (t >= 2 && !mbar_wait(&empty_v[vs], ((t >> 1) - 1) & 1, abort_flag)) return false;
+                K512_STAMP(t, 28);
+                const int tok = (int)(t0 + (int64_t)(cb + t) * kStep);
+                mbar_arrive_expect_tx(&full_v[vs], kRegion);
+                tma_load_3d(sm + C::V0 + vs * kRegion, &tv, &full_v[vs], v0, h, tok);
+                issued_v = t + 1;
+                return true;
+            };
+            bool ok = nsteps > 0 ? load_v(0) : true;
+            for (int q = 0; ok && q < total; ++q) {
                 const int t = q / KS, sl = q - t * KS, st = q & 1;
                 const int tok = (int)(t0 + (int64_t)(cb + t) * kStep);
-                if (sl == 0) {
-                    const int vs = t & 1;
-                    if (t >= 2 && !mbar_wait(&empty_v[vs], ((t >> 1) - 1) & 1, abort_flag)) break;
-                    K512_STAMP(t, 28);
-                    mbar_arrive_expect_tx(&full_v[vs], kRegion);
-                    tma_load_3d(sm + C::V0 + vs * kRegion, &tv, &full_v[vs], v0, h, tok);
-                    issued_v = t + 1;
+                auto load_q = [&]() -> bool {
+                    if (q >= 2 && !mbar_wait(&empty_q[st], ((q >> 1) - 1) & 1, abort_flag)) return false;
+                    if (sl == 0) K512_STAMP(t, 27);
+                    unsigned char *dq = sm + C::QR + st * C::QUNIT;
+                    mbar_arrive_expect_tx(&full_q[st], C::QUNIT);
+                    tma_load_3d(dq, &tq, &full_q[st], 128 * sl, h, tok);
+                    tma_load_3d(dq + kRegion, &tq, &full_q[st], 128 * sl + 64, h, tok);
+                    issued_q = q + 1;
+                    return true;
+                };
+                auto load_k = [&]() -> bool {
+                    if (q >= 2 && !mbar_wait(&empty_k[st], ((q >> 1) - 1) & 1, abort_flag)) return false;
+                    if (sl == KS - 1) K512_STAMP(t, 29);
+                    if (sl == 0) K512_STAMP(t, 25);
+                    unsigned char *dk = sm + C::KR + st * C::KUNIT + ((t & 1) ? 0u : kRegion / 2);
+                    mbar_arrive_expect_tx(&full_k[st], 2 * kRegion);
+                    tma_load_3d(dk, &tk, &full_k[st], 128 * sl, h, tok);
+                    tma_load_3d(dk + C::KREG, &tk, &full_k[st], 128 * sl + 64, h, tok);
+                    issued_k = q + 1;
+                    return true;
+                };
+                ok = (sl == 0) ? (load_k() && load_q()) : (load_q() && load_k());
+#ifdef SGLA_DEVICE_TRACE
+                if (ok && sl == 0 && blockIdx.x == 0 && blockIdx.y == 0) {  // landing times of slice 0
+                    mbar_wait(&full_k[st], (q >> 1) & 1, abort_flag);
+                    K512_STAMP(t, 30);
+                    mbar_wait(&full_q[st], (q >> 1) & 1, abort_flag);
+                    K512_STAMP(t, 31);
                 }
-                if (q >= 2 && !mbar_wait(&empty_q[st], ((q >> 1) - 1) & 1, abort_flag)) break;
-                if (sl == 0) K512_STAMP(t, 27);
-                unsigned char *dq = sm + C::QR + st * C::QUNIT;
-                mbar_arrive_expect_tx(&full_q[st], C::QUNIT);
-                tma_load_3d(dq, &tq, &full_q[st], 128 * sl, h, tok);
-                tma_load_3d(dq + kRegion, &tq, &full_q[st], 128 * sl + 64, h, tok);
-                issued = 2 * q + 1;
-                if (q >= 2 && !mbar_wait(&empty_k[st], ((q >> 1) - 1) & 1, abort_flag)) break;
-                if (sl == KS - 1) K512_STAMP(t, 29);
-                unsigned char *dk = sm + C::KR + st * C::KUNIT + ((t & 1) ? 0u : kRegion / 2);
-                mbar_arrive_expect_tx(&full_k[st], 2 * kRegion);
-                tma_load_3d(dk, &tk, &full_k[st], 128 * sl, h, tok);
-                tma_load_3d(dk + C::KREG, &tk, &full_k[st], 128 * sl + 64, h, tok);
-                issued = 2 * q + 2;
+#endif
+                if (ok && sl == KS - 2 && t + 1 < nsteps) ok = load_v(t + 1);
             }
-            if (*abort_flag) {  // issued counts halves: Q of slice q is 2q, K is 2q + 1
-                for (int x = max(0, issued - 4); x < issued; ++x) {
-                    const int q = x >> 1;
-                    mbar_drain((x & 1) ? &full_k[q & 1] : &full_q[q & 1], (q >> 1) & 1);
-                }
+            if (*abort_flag) {
+                for (int q = max(0, issued_q - 2); q < issued_q; ++q) mbar_drain(&full_q[q & 1], (q >> 1) & 1);
+                for (int q = max(0, issued_k - 2); q < issued_k; ++q) mbar_drain(&full_k[q & 1], (q >> 1) & 1);
                 for (int t = max(0, issued_v - 2); t < issued_v; ++t) mbar_drain(&full_v[t & 1], (t >> 1) & 1);
             }
         }
@@ -250,16 +270,19 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                     const uint32_t ph = (q >> 1) & 1;
                     const uint32_t qa = sbase + C::QR + st * C::QUNIT, ka = sbase + C::KR + st * C::KUNIT;
                     if (sl == 0) K512_STAMP(t, 0);
-                    if (!(ok = wait(&full_q[st], ph) && wait(&full_k[st], ph))) break;
-                    K512_STAMP(t, sl == 0 ? 1 : 4 + sl);
+                    if (!(ok = wait(&full_k[st], ph))) break;
+                    if (sl == 0) K512_STAMP(t, 26);
                     if (!(ok = wait(&b_hbt[st], ph))) break;
                     if (sl == 0) K512_STAMP(t, 2);
+                    // descriptors built once per slice, moved along by constant offsets
+                    const uint64_t qd = kdesc(qa), kd = kdesc(ka);
+                    const uint64_t hd = sdesc(ka + koff, C::KREG, 1024, 2), wd = mn64(vw);
                     auto issue_so = [&]() {
                         tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
                             const uint32_t c = (kk & 3) * 32;
-                            mma_bf16(dso, kdesc(qa + (kk >> 2) * kRegion + c), kdesc(ka + (kk >> 2) * C::KREG + c), idSO,
+                            mma_bf16(dso, desc_at(qd, (kk >> 2) * kRegion + c), desc_at(kd, (kk >> 2) * C::KREG + c), idSO,
                                      (sl > 0 || kk > 0) ? 1u : 0u);
                         }
                         mma_commit(&empty_q[st]);
@@ -267,21 +290,25 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                     };
                     auto issue_h = [&]() {
                         tc_fence_after();
+                        const uint32_t hcol = tmem + C::COL_H + sl * BV;
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            mma_bf16(tmem + C::COL_H + sl * BV, sdesc(ka + koff + kk * 2048, C::KREG, 1024, 2),
-                                     mn64(vw + kk * 2048), idH, 1u);
+                            mma_bf16(hcol, desc_at(hd, kk * 2048), desc_at(wd, kk * 2048), idH, 1u);
                         mma_commit(&b_hdone[sl]);
                     };
                     if (sl == 0) {
                         if (!(ok = wait(&b_vw[t & 1], (t >> 1) & 1))) break;
                         K512_STAMP(t, 4);
                         issue_h();
+                        if (!(ok = wait(&full_q[st], ph))) break;
+                        K512_STAMP(t, 1);
                         if (t >= 1 && !(ok = wait(b_pv, (t - 1) & 1))) break;
                         if (t >= 2 && !(ok = wait(&b_ofree[t & 1], ((t >> 1) - 1) & 1))) break;
                         K512_STAMP(t, 3);
                         issue_so();
                     } else {
+                        if (!(ok = wait(&full_q[st], ph))) break;
+                        K512_STAMP(t, 4 + sl);
                         issue_so();
                         issue_h();
                     }
@@ -295,10 +322,10 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                 if (!(ok = wait(b_o1s, t & 1))) break;
                 K512_STAMP(t, 10);
                 tc_fence_after();
-                const uint32_t vf = sbase + C::V0 + (t & 1) * kRegion;
+                const uint64_t vfd = mn64(sbase + C::V0 + (t & 1) * kRegion);
 #pragma unroll
                 for (int jj = 0; jj < kStep / 16; ++jj)
-                    mma_bf16_tmem_a(od, tmem + C::COL_S + jj * 8, mn64(vf + jj * 2048), idO, 1u);
+                    mma_bf16_tmem_a(od, tmem + C::COL_S + jj * 8, desc_at(vfd, jj * 2048), idO, 1u);
                 mma_commit(b_pv);
                 mma_commit(&empty_v[t & 1]);
                 K512_STAMP(t, 11);
@@ -480,9 +507,7 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                 *reinterpret_cast<uint32_t *>(reg + off) = w2;
             }
         };
-        const float *src = nullptr;  // state entering the segment
-        if (s == 0) src = a.h0 ? a.h0 + ((int64_t)n * H + h) * KV : nullptr;
-        else src = a.seg_state + ((int64_t)(u - 1) * H + h) * KV;
+        const int first = u - s;  // segment units of a sequence are consecutive
         bool ok = true;
         if (nsteps > 0) v_pass(0);
         for (int t = 0; ok && t < nsteps; ++t) {
@@ -502,17 +527,8 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                     if (t >= 1) {
                         tmem_ld32(hrow + sl * BV + 32 * pc, x);
                         tmem_wait_ld();
-                    } else if (src) {
-                        const float4 *p4 =
-                            reinterpret_cast<const float4 *>(src + (int64_t)(128 * sl + i) * V + v0 + 32 * pc);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float4 f = p4[e];
-                            x[4 * e] = f.x; x[4 * e + 1] = f.y; x[4 * e + 2] = f.z; x[4 * e + 3] = f.w;
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) x[e] = 0.f;
+                    } else {  // the state entering the segment
+                        entering_state_row32(a, n, s, first, h, 128 * sl + i, v0 + 32 * pc, x);
                     }
                     hbt_piece(slot, ev, pc, x);
 #pragma unroll
@@ -650,7 +666,7 @@ cudaError_t launch_k512(const FwdArgs &a, cudaStream_t st) {
     auto kern = tc_walk_k512_kernel<KS>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM)) != cudaSuccess)
         return e;
-    dim3 grid(a.lay.max_segs * (a.V / kK512BV), a.H);
+    dim3 grid(a.lay.max_segs * a.H * (a.V / kK512BV));
     kern<<<grid, kK512Threads, C::SMEM, st>>>(tq, tk, tv, a);
     return cudaGetLastError();
 }

@@ -352,3 +352,27 @@ def test_call_runs_on_the_device_of_its_tensors():
         assert o.device == dev and ht.device == dev
         torch.cuda.synchronize(dev)
     check(inp, (host(o), host(ht)), oracle_fwd(inp), torch.bfloat16, "second device")
+
+
+@pytest.mark.parametrize("vf", [False, True])
+def test_tensor_core_varlen_empty_sequences_both_state_layouts(vf):
+    """Packed batch with empty sequences (their final state is their initial state) and
+    long ones split into segments, through the chunked entry point in either state
+    layout: the plan pass writes the empty sequences' final states in the [K,V] layout,
+    the carry pass in the [V,K] one."""
+    cu_list = [0, 0, 3000, 3000, 3001, 7200, 7200]
+    cu = torch.tensor(cu_list, dtype=torch.int64)
+    inp = random_inputs(1, cu_list[-1], 2, 128, 128, torch.bfloat16, gate="g", h0=True, seed=43, cu_seqlens=cu)
+    h0 = inp["h0"].transpose(-1, -2).contiguous() if vf else inp["h0"]
+    o, ht = sg.chunk_simple_gla(to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"]), g=to_dev(inp["g"]),
+                                initial_state=to_dev(h0), output_final_state=True, cu_seqlens=to_dev(cu),
+                                state_v_first=vf)
+    torch.cuda.synchronize()
+    ht = host(ht)
+    if vf:
+        ht = np.swapaxes(ht, -1, -2)
+    ro, rh = oracle_fwd(inp, cu=cu)
+    check(inp, (host(o), ht), (ro, rh), torch.bfloat16, f"varlen empty sequences vf={vf}")
+    for n in range(len(cu_list) - 1):
+        if cu_list[n + 1] == cu_list[n]:
+            np.testing.assert_array_equal(ht[n], inp["h0"][n].numpy())
