@@ -303,7 +303,10 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
     if (N == 0) return SGLA_OK;
     if (state_v_first && h0)
         SGLA_LAUNCH("state_transpose", launch_state_transpose(h0, const_cast<float *>(a.h0), N * H, (int)V, (int)K, st));
-    if (per_token && tokens > 0) SGLA_LAUNCH("chunk_cumsum", launch_chunk_cumsum(g, a.gcum, a.gpos, lay, st));
+    // the K = 256 / 512 walk and the k-block state pass form the chunk-local cumsum of the
+    // gates themselves; the K = 128 kernels read it from this pass
+    if (per_token && tokens > 0 && (!p.tc || K == 128))
+        SGLA_LAUNCH("chunk_cumsum", launch_chunk_cumsum(g, a.gcum, a.gpos, lay, st));
     if (p.multi_seg && p.max_segs > 0) {
         if (p.tc) SGLA_LAUNCH("segment_state_tc", tc_launch_segment_state(a, st));
         else SGLA_LAUNCH("segment_state_simt", launch_segment_state_simt(a, st));
@@ -585,7 +588,10 @@ sgla_status simple_gla_chunk_final_state(const void *k, const void *v, const flo
         SGLA_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), st), "status reset");
     }
     if (N == 0) return SGLA_OK;
-    if (per_token && tokens > 0) SGLA_LAUNCH("chunk_cumsum", launch_chunk_cumsum(g, a.gcum, a.gpos, lay, st));
+    // the K = 256 / 512 walk and the k-block state pass form the chunk-local cumsum of the
+    // gates themselves; the K = 128 kernels read it from this pass
+    if (per_token && tokens > 0 && (!p.tc || K == 128))
+        SGLA_LAUNCH("chunk_cumsum", launch_chunk_cumsum(g, a.gcum, a.gpos, lay, st));
     if (p.max_segs > 0 && tokens > 0) {
         if (p.tc) SGLA_LAUNCH("segment_state_tc", tc_launch_segment_state(a, st));
         else SGLA_LAUNCH("segment_state_simt", launch_segment_state_simt(a, st));

@@ -155,11 +155,22 @@ tc_segment_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_con
         const int i = threadIdx.x;
         const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
         float lsuf = 0.f;  // log2 decay from the end of the current step to the end of the segment
+        const float head_l2 = (a.gate_mode == kGatePerHead) ? fmaxf(a.g_gamma[h], kMinLogGate) * kRcpLn2 : 0.f;
+        StepGateLoads ld{};
+        if (nsteps > 0 && a.gate_mode == kGatePerToken) {
+            const StepSpan sp0 = step_span(t0, t1, cb + nsteps - 1);
+            ld = step_gates_load(a.g, sp0.ta, sp0.len, h, H, i);
+        }
         for (int r = 0; r < nsteps; ++r) {
             const int st = r % kStateStages;
             const StepSpan sp = step_span(t0, t1, cb + nsteps - 1 - r);
-            const float gi = (i < sp.len) ? chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + i, i, h, H) : 0.f;
-            const float glast = chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + sp.len - 1, sp.len - 1, h, H);
+            const StepGates q = (a.gate_mode == kGatePerToken) ? step_gates_finish(ld, sp.len, i)
+                                                               : step_gates_head(head_l2, sp.len, i, kDecayStep);
+            const float gi = q.g, glast = q.last;
+            if (r + 1 < nsteps && a.gate_mode == kGatePerToken) {  // the next step's loads, a step ahead
+                const StepSpan spn = step_span(t0, t1, cb + nsteps - 2 - r);
+                ld = step_gates_load(a.g, spn.ta, spn.len, h, H, i);
+            }
             mbar_wait(&full[st], (r / kStateStages) & 1, abort_flag);
             const float w = (i < sp.len) ? fast_exp2(lsuf + (glast - gi)) : 0.f;
             scale_row<128>(sm + st * ss::STAGE + ss::V, sm + st * ss::STAGE + ss::VW, i, w);

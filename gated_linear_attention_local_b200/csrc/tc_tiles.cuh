@@ -145,6 +145,96 @@ struct StepSpan {
     int len;     // tokens in the step (<= 128)
 };
 
+// The chunk-local cumulative log gates of one 128-token step as the thread that owns
+// token i of a 4-warp group sees them (G~, log2 units, 0 past the step's end) and the
+// step's DecayMode.
+struct StepGates {
+    float g;        // G~ of token i
+    float tile[4];  // G~ of the last token of each 32-token tile, clipped to the step
+    float last;     // G~ of the step's last token
+    int mode;       // DecayMode
+};
+
+// Per-token gates: the inclusive sum of max(g, kMinLogGate) from the step's first token,
+// times 1/ln2 ("Simple GLA in flash-linear-attention" section 3: the chunk-local cumsum
+// of g, prescaled by RCP_LN2), and the decay mode: kDecayTile when the step spans more
+// than kMaxTileSpan, kDecayExact when a 32-token tile does, kDecaySigned when a log gate
+// is positive, else kDecayStep.  Every warp of the group sums all four tiles itself (one
+// strided load per tile and lane, a shuffle reduction broadcast from lane 0) and scans
+// its own tile, so the group needs no shared memory and no barrier; every caller gets
+// the same value for a token.  The loads (step_gates_load) are issued apart from the
+// arithmetic (step_gates_finish), so their latency hides behind other work; all 32
+// lanes of a warp call step_gates_finish together.
+struct StepGateLoads {
+    float x[4];  // max(g, kMinLogGate) of tokens lane, lane + 32, lane + 64, lane + 96 (0 past the end)
+};
+__device__ __forceinline__ StepGateLoads step_gates_load(const float *g, int64_t ta, int len, int h, int H, int i) {
+    const int lane = i & 31;
+    StepGateLoads ld;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int j = 32 * c + lane;
+        ld.x[c] = (j < len) ? g[(ta + j) * H + h] : 0.f;
+    }
+    return ld;
+}
+__device__ __forceinline__ StepGates step_gates_finish(const StepGateLoads &ld, int len, int i) {
+    const int lane = i & 31, w = i >> 5;
+    float x[4];
+    bool positive = false;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        x[c] = (32 * c + lane < len) ? fmaxf(ld.x[c], kMinLogGate) : 0.f;
+        positive |= x[c] > 0.f;
+    }
+    float pre[5];  // sums of the tiles before tile c (nats)
+    float first[4];
+    pre[0] = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        float s = x[c];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_down_sync(0xffffffffu, s, off);
+        pre[c + 1] = pre[c] + __shfl_sync(0xffffffffu, s, 0);
+        first[c] = __shfl_sync(0xffffffffu, x[c], 0);
+    }
+    float v = w == 0 ? x[0] : w == 1 ? x[1] : w == 2 ? x[2] : x[3];
+    float incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    const float base = w == 0 ? pre[0] : w == 1 ? pre[1] : w == 2 ? pre[2] : pre[3];
+    StepGates q;
+    q.g = (i < len) ? (base + incl) * kRcpLn2 : 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) q.tile[c] = pre[c + 1] * kRcpLn2;
+    q.last = pre[4] * kRcpLn2;
+    int mode = ((first[0] * kRcpLn2) - q.last > kMaxTileSpan) ? kDecayTile : kDecayStep;
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        if (32 * c < len && (pre[c] + first[c]) * kRcpLn2 - q.tile[c] > kMaxTileSpan) mode = kDecayExact;
+    if (__any_sync(0xffffffffu, positive)) mode = kDecaySigned;
+    q.mode = mode;
+    return q;
+}
+__device__ __forceinline__ StepGates step_gates_token(const float *g, int64_t ta, int len, int h, int H, int i) {
+    return step_gates_finish(step_gates_load(g, ta, len, h, H, i), len, i);
+}
+
+// The same for a per-head decay (G~_pos = (pos + 1) gamma, gamma in log2 units) or no
+// gate (gamma = 0), with the mode the caller has chosen for the head.
+__device__ __forceinline__ StepGates step_gates_head(float gamma, int len, int i, int mode) {
+    StepGates q;
+    q.g = (i < len) ? (float)(i + 1) * gamma : 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) q.tile[c] = (float)min(32 * c + 32, len) * gamma;
+    q.last = (float)len * gamma;
+    q.mode = mode;
+    return q;
+}
+
 __device__ __forceinline__ StepSpan step_span(int64_t t0, int64_t t1, int step) {
     StepSpan s;
     s.ta = t0 + (int64_t)step * kStep;

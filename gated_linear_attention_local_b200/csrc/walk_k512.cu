@@ -163,20 +163,23 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     const int head_mode = (a.o_f32 || head_l2 > 0.f || -31.f * head_l2 > kMaxTileSpan) ? kDecayExact
                           : (-127.f * head_l2 > kMaxTileSpan)                          ? kDecayTile
                                                                                        : kDecayStep;
-    const int64_t chunk0 = (lay.cu ? (int64_t)lay.chunk_off[n] : (int64_t)n * lay.NT) + cb;
-    auto step_mode = [&](int t) -> int {
-        if (a.gate_mode != kGatePerToken) return head_mode;
-        const int m = a.gpos[(chunk0 + t) * H + h];
-        return a.o_f32 ? max(m, (int)kDecayExact) : m;
-    };
-    auto gate_of = [&](int t, int pos) -> float {  // G~ of position pos of local step t (0 past the end)
+    // the gates of local step t as the warpgroup thread owning token i sees them; all 32
+    // lanes of a warp call it together (per-token gates are summed with shuffles)
+    // (gates_load issues the per-token loads early, gates_finish does the arithmetic)
+    auto gates_load = [&](int t, int i) -> StepGateLoads {
         const StepSpan sp = step_span(t0, t1, cb + t);
-        return (pos < sp.len) ? chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + pos, pos, h, H) : 0.f;
+        if (a.gate_mode != kGatePerToken) return StepGateLoads{};
+        return step_gates_load(a.g, sp.ta, sp.len, h, H, i);
     };
-    auto last_gate = [&](int t) -> float {
+    auto gates_finish = [&](int t, int i, const StepGateLoads &ld) -> StepGates {
         const StepSpan sp = step_span(t0, t1, cb + t);
-        return chunk_gate(a.gate_mode, a.gcum, a.g_gamma, sp.ta + sp.len - 1, sp.len - 1, h, H);
+        if (a.gate_mode != kGatePerToken) return step_gates_head(head_l2, sp.len, i, head_mode);
+        StepGates q = step_gates_finish(ld, sp.len, i);
+        if (a.o_f32) q.mode = max(q.mode, (int)kDecayExact);
+        return q;
     };
+    auto gates = [&](int t, int i) -> StepGates { return gates_finish(t, i, gates_load(t, i)); };
+    auto warp_all = [](bool ok) { return __all_sync(0xffffffffu, ok) != 0; };  // a warp-uniform exit
 
     if (warp == 12) {
         // ---------------------------------------------------------------- TMA loads
@@ -348,18 +351,7 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         float *fs = gs + 128;
         const bool per_token = a.gate_mode == kGatePerToken;
         if (!per_token) gs[i] = a.scale * exp2f((float)i * head_l2);  // per-head decay table
-        struct StepGates {
-            float g, gl, gr[4];
-            int mode;
-        };
-        auto load_step = [&](int t, StepGates &q) {
-            const StepSpan sp = step_span(t0, t1, cb + t);
-            q.g = gate_of(t, i);
-            q.gl = last_gate(t);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) q.gr[c] = gate_of(t, min(32 * c + 31, sp.len - 1));
-            q.mode = step_mode(t);
-        };
+        auto load_step = [&](int t, StepGates &q) { q = gates(t, i); };
         const float log2_scale = log2f(a.scale);
         StepGates cur{}, nxt{};
         if (nsteps > 0) load_step(0, cur);
@@ -368,10 +360,11 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         // step; once the CTA has given up, every wait returns at once
         for (int t = 0; t < nsteps; ++t) {
             const StepSpan sp = step_span(t0, t1, cb + t);
-            if (t + 1 < nsteps) load_step(t + 1, nxt);
+            StepGateLoads ldn{};  // the next step's gates, finished once this step's mask is out
+            if (t + 1 < nsteps) ldn = gates_load(t + 1, i);
             const bool exact = cur.mode >= kDecayExact;
             if (per_token && exact) {
-                const float gri = quarter == 0 ? cur.gr[0] : quarter == 1 ? cur.gr[1] : quarter == 2 ? cur.gr[2] : cur.gr[3];
+                const float gri = quarter == 0 ? cur.tile[0] : quarter == 1 ? cur.tile[1] : quarter == 2 ? cur.tile[2] : cur.tile[3];
                 gs[i] = cur.g;
                 fs[i] = (i < sp.len) ? fast_exp2(gri - cur.g) : 0.f;
             }
@@ -388,8 +381,8 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                     for (int e = 0; e < 32; ++e) x[e] = 0.f;
                 } else {
                     tmem_ld32(srow + 32 * c, x);
-                    const float grc = cur.mode == kDecayStep ? cur.gl
-                                      : c == 0 ? cur.gr[0] : c == 1 ? cur.gr[1] : c == 2 ? cur.gr[2] : cur.gr[3];
+                    const float grc = cur.mode == kDecayStep ? cur.last
+                                      : c == 0 ? cur.tile[0] : c == 1 ? cur.tile[1] : c == 2 ? cur.tile[2] : cur.tile[3];
                     const float R = a.scale * fast_exp2(cur.g - grc);
                     tmem_wait_ld();
                     if (!exact) {
@@ -438,6 +431,7 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
             mbar_arrive(b_p);
             if (i == 0) K512_STAMP(t, 13);
             named_sync(1, 128);  // every row is done with this step's gates and factors
+            if (t + 1 < nsteps) nxt = gates_finish(t + 1, i, ldn);
             cur = nxt;
         }
     } else if (warp < 8) {
@@ -449,16 +443,23 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         const int64_t KV = (int64_t)a.K * V;
         // V(t) -> V_w = w ⊙ V (buffer t & 1) and V_f = f ⊙ V (in place), 0 past the end;
         // each product of a bf16 pair with an fp32 weight is rounded once
-        auto v_pass = [&](int t) {
+        struct RowGates {  // what this thread needs of a step's gates
+            float g, ref, last;  // G~ of token i, of the last token of its tile, of the step's last
+            int mode;
+        };
+        auto row_gates = [&](int t, const StepGateLoads &ld) -> RowGates {
+            const StepGates q = gates_finish(t, i, ld);
+            const int wt = i >> 5;
+            return {q.g, wt == 0 ? q.tile[0] : wt == 1 ? q.tile[1] : wt == 2 ? q.tile[2] : q.tile[3], q.last, q.mode};
+        };
+        auto v_pass = [&](int t, const RowGates &q) {
             const int st = t & 1;
             if (mbar_wait(&full_v[st], (t >> 1) & 1, abort_flag)) {
-                const int mode = step_mode(t);
+                const int mode = q.mode;
                 const StepSpan sp = step_span(t0, t1, cb + t);
-                const float gi = gate_of(t, i);
-                const float w = (i < sp.len) ? fast_exp2(last_gate(t) - gi) : 0.f;
-                const float f = mode == kDecayStep ? w
-                                : (i < sp.len)     ? fast_exp2(gate_of(t, min(i | 31, sp.len - 1)) - gi)
-                                                   : 0.f;
+                const float gi = q.g, gref = q.ref;
+                const float w = (i < sp.len) ? fast_exp2(q.last - gi) : 0.f;
+                const float f = mode == kDecayStep ? w : (i < sp.len) ? fast_exp2(gref - gi) : 0.f;
                 const bool write_f = mode < kDecayExact;
                 const __nv_bfloat162 wh = __float2bfloat162_rn(w), wl = __float2bfloat162_rn(w - __low2float(wh));
                 const __nv_bfloat162 fh = __float2bfloat162_rn(f), fl = __float2bfloat162_rn(f - __low2float(fh));
@@ -509,15 +510,21 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         };
         const int first = u - s;  // segment units of a sequence are consecutive
         bool ok = true;
-        if (nsteps > 0) v_pass(0);
+        float glast = 0.f;  // G~_last of step t
+        if (nsteps > 0) {
+            const RowGates q0 = row_gates(0, gates_load(0, i));
+            glast = q0.last;
+            v_pass(0, q0);
+        }
         for (int t = 0; ok && t < nsteps; ++t) {
-            const float gam = exp2f(last_gate(t));  // decay of step t, applied to the entering state
+            const float gam = exp2f(glast);  // decay of step t, applied to the entering state
+            const StepGateLoads ldn = t + 1 < nsteps ? gates_load(t + 1, i) : StepGateLoads{};
             const bool ev = (t & 1) == 0;
 #pragma unroll 1
             for (int sl = 0; sl < KS; ++sl) {
                 const int q = t * KS + sl, st = q & 1;
-                if (t >= 1 && !(ok = mbar_wait(&b_hdone[sl], (t - 1) & 1, abort_flag))) break;
-                if (q >= 2 && !(ok = mbar_wait(&empty_k[st], ((q >> 1) - 1) & 1, abort_flag))) break;
+                if (t >= 1 && !(ok = warp_all(mbar_wait(&b_hdone[sl], (t - 1) & 1, abort_flag)))) break;
+                if (q >= 2 && !(ok = warp_all(mbar_wait(&empty_k[st], ((q >> 1) - 1) & 1, abort_flag)))) break;
                 if (i == 0) K512_STAMP(t, 14 + 2 * sl);
                 tc_fence_after();
                 unsigned char *slot = sm + C::KR + st * C::KUNIT;
@@ -543,7 +550,9 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
             }
             // V_w(t+1) goes to the buffer H(t-1) read, which the block passes above waited for
             if (ok && t + 1 < nsteps) {
-                v_pass(t + 1);
+                const RowGates qn = row_gates(t + 1, ldn);
+                glast = qn.last;
+                v_pass(t + 1, qn);
                 if (i == 0) K512_STAMP(t + 1, 22);
             }
         }
@@ -572,14 +581,14 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         const int i = threadIdx.x - 256;
         const uint32_t trow = tmem + ((uint32_t)((warp - 8) * 32) << 16);
         const bool o32 = (reinterpret_cast<uintptr_t>(a.o) & 31) == 0;  // 32-byte row segments
-        float gnext = nsteps > 0 ? gate_of(0, i) : 0.f;
+        StepGateLoads ldn = nsteps > 0 ? gates_load(0, i) : StepGateLoads{};  // loaded an iteration ahead
         for (int t = 0; t < nsteps; ++t) {
             const StepSpan sp = step_span(t0, t1, cb + t);
-            const float gi = gnext;
-            gnext = (t + 1 < nsteps) ? gate_of(t + 1, i) : 0.f;
+            const float gi = gates_finish(t, i, ldn).g;
+            if (t + 1 < nsteps) ldn = gates_load(t + 1, i);
             const uint32_t orow = trow + ((t & 1) ? C::COL_OB : C::COL_OA);
             // O1 row i times scale 2^G~_i, in place, before P' V_f accumulates onto it
-            if (!mbar_wait(b_s, t & 1, abort_flag)) break;
+            if (!warp_all(mbar_wait(b_s, t & 1, abort_flag))) break;
             if (i == 0) K512_STAMP(t, 23);
             tc_fence_after();
             {
@@ -598,7 +607,7 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
                 mbar_arrive(b_o1s);
             }
             // o = O (scale is in it) after P' V_f
-            if (!mbar_wait(b_pv, t & 1, abort_flag)) break;
+            if (!warp_all(mbar_wait(b_pv, t & 1, abort_flag))) break;
             if (i == 0) K512_STAMP(t, 24);
             tc_fence_after();
             const bool store = i < sp.len && !*abort_flag;
