@@ -307,19 +307,34 @@ sgla_status run_forward(bool varlen, const void *q, const void *k, const void *v
     // gates themselves; the K = 128 kernels read it from this pass
     if (per_token && tokens > 0 && (!p.tc || K == 128))
         SGLA_LAUNCH("chunk_cumsum", launch_chunk_cumsum(g, a.gcum, a.gpos, lay, st));
+    bool state_pass_tc = false;
     if (p.multi_seg && p.max_segs > 0) {
         if (p.tc) SGLA_LAUNCH("segment_state_tc", tc_launch_segment_state(a, st));
         else SGLA_LAUNCH("segment_state_simt", launch_segment_state_simt(a, st));
+        state_pass_tc = p.tc;
     }
     const bool empty_dense = !varlen && p.NT == 0;
     // the tensor-core walks form their entering states from the segment states
     // themselves, and the plan kernel writes the final states of empty packed sequences
     // (with the [V,K] layout that copy waits for the transposed initial state: the carry
     // pass does it)
-    if (p.multi_seg && !p.tc) SGLA_LAUNCH("segment_carry", launch_segment_carry(a, true, st));
-    else if (hT && (empty_dense || (varlen && state_v_first)))
+    bool carry = false;
+    if (p.multi_seg && !p.tc) {
+        SGLA_LAUNCH("segment_carry", launch_segment_carry(a, true, st));
+        carry = true;
+    } else if (hT && (empty_dense || (varlen && state_v_first))) {
         SGLA_LAUNCH("segment_carry", launch_segment_carry(a, false, st));
+        carry = true;
+    }
     if (tokens > 0 && p.max_segs > 0) {
+        // On a packed batch the walk starts while the tensor-core state pass runs: its
+        // first CTAs (longest first) are mostly first segments, which need nothing from
+        // that pass and walk on the SMs it leaves idle; the others wait for it.  Every
+        // other input was written by launches that completed before the state pass
+        // started.  A dense batch's first segments are no longer than the rest, so there
+        // an early start only competes with the state pass for bandwidth.  Not while
+        // per-kernel events are recorded: each kernel is then timed alone.
+        a.overlap_state = varlen && state_pass_tc && !carry && !g_prof_on;
         if (p.tc) SGLA_LAUNCH("chunk_output_tc", tc_launch_chunk_output(a, st));
         else SGLA_LAUNCH("chunk_output_simt", launch_chunk_output_simt(a, st));
     }

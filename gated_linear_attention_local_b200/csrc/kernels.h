@@ -28,6 +28,9 @@ struct FwdArgs {
     int *dev_status; // writable status word (bounded device waits record time-outs here)
     bool state_all;  // state-only call: every segment, the last one too, goes through the state
                      // pass and the carry folds them all into hT (no output walk)
+    bool overlap_state;  // the output walk is launched while the state pass it follows still
+                         // runs (programmatic dependent launch): a CTA that folds segment
+                         // states waits for that grid first; the others start at once
     SeqLayout lay;
 };
 

@@ -51,6 +51,7 @@ tc_state_k128_kernel(const __grid_constant__ CUtensorMap tk, const __grid_consta
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = align1024(smem_raw);
     const SeqLayout &lay = a.lay;
+    griddep_launch_dependents();  // an output walk launched behind this pass may start now
     if (device_failed(lay)) return;
     const int VT = a.V / 128;
     const SegWork wk = seg_work(lay, blockIdx.x, VT);

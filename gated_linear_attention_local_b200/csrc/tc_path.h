@@ -3,9 +3,30 @@
 
 #include <cuda.h>
 
+#include <utility>
+
 #include "kernels.h"
 
 namespace sgla {
+
+// Launch an output walk; with `overlap` set it may start while the grid launched just
+// before it (the state pass, which releases it at its start) still runs.  The walk
+// then waits for that grid before it reads what that grid writes.
+template <typename... P, typename... A>
+cudaError_t tc_launch_walk(void (*kern)(P...), dim3 grid, int threads, size_t smem, cudaStream_t st,
+                           bool overlap, A &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = overlap ? attr : nullptr;
+    cfg.numAttrs = overlap ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
 
 // True when the tensor-core kernels cover these sizes (bf16 operands only).
 bool tc_path_supports(bool bf16, int K, int V, int C);

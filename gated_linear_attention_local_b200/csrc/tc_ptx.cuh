@@ -179,6 +179,16 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
 }
 
 // ---------------------------------------------------------------- fences
+// Programmatic dependent launch (PTX griddepcontrol).  launch_dependents lets a grid
+// launched after this one with programmatic stream serialisation start before this
+// grid ends; wait blocks the calling thread until every grid this one depends on has
+// completed and its writes are visible (it returns at once in a grid launched the
+// ordinary way, whose predecessors completed before it started).
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

@@ -479,6 +479,9 @@ tc_walk_k128_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         {
             const int first = u - s;  // segment units of a sequence are consecutive
             const float gam = nsteps > 0 ? exp2f(last_gate(0)) : 1.f;
+            // the earlier segments' states come from the state pass, which may still run
+            // when this walk starts
+            if (s > 0) griddep_wait();
 #pragma unroll 1
             for (int pc = 0; pc < C::NP; ++pc) {
                 float x[32];
@@ -689,8 +692,7 @@ cudaError_t launch_k128(const FwdArgs &a, cudaStream_t st) {
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM)) != cudaSuccess)
         return e;
     dim3 grid(a.lay.max_segs * a.H * (a.V / BV));
-    kern<<<grid, kK128Threads, C::SMEM, st>>>(tq, tk, tv, to, a);
-    return cudaGetLastError();
+    return tc_launch_walk(kern, grid, kK128Threads, C::SMEM, st, a.overlap_state, tq, tk, tv, to, a);
 }
 
 }  // namespace

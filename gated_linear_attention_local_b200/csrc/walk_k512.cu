@@ -516,6 +516,9 @@ tc_walk_k512_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
             glast = q0.last;
             v_pass(0, q0);
         }
+        // the segment states of the sequence's earlier segments come from the state pass,
+        // which may still run when this walk starts
+        if (s > 0) griddep_wait();
         for (int t = 0; ok && t < nsteps; ++t) {
             const float gam = exp2f(glast);  // decay of step t, applied to the entering state
             const StepGateLoads ldn = t + 1 < nsteps ? gates_load(t + 1, i) : StepGateLoads{};
@@ -676,8 +679,7 @@ cudaError_t launch_k512(const FwdArgs &a, cudaStream_t st) {
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM)) != cudaSuccess)
         return e;
     dim3 grid(a.lay.max_segs * a.H * (a.V / kK512BV));
-    kern<<<grid, kK512Threads, C::SMEM, st>>>(tq, tk, tv, a);
-    return cudaGetLastError();
+    return tc_launch_walk(kern, grid, kK512Threads, C::SMEM, st, a.overlap_state, tq, tk, tv, a);
 }
 
 }  // namespace

@@ -376,3 +376,44 @@ def test_tensor_core_varlen_empty_sequences_both_state_layouts(vf):
     for n in range(len(cu_list) - 1):
         if cu_list[n + 1] == cu_list[n]:
             np.testing.assert_array_equal(ht[n], inp["h0"][n].numpy())
+
+
+# On packed batches the output walk starts while the segment-state pass that precedes
+# it still runs: the CTAs of first segments begin at once, the others wait for that pass
+# before they fold the earlier segments' states.  Sizes give long sequences many
+# segments and short ones a single segment each.
+OVERLAP_CASES = [
+    ("varlen", 128, 128, "g"),
+    ("varlen", 128, 128, "gamma"),
+    ("varlen", 512, 128, "g"),
+    ("dense", 128, 128, "gamma"),  # launched the ordinary way
+]
+
+
+@pytest.mark.parametrize("case", OVERLAP_CASES)
+def test_walk_started_under_the_state_pass_is_repeatable(case):
+    kind, K, V, gate = case
+    if kind == "varlen":
+        T = 12000 if K == 128 else 4000
+        cu = torch.tensor([0, 3 * T // 4, 3 * T // 4 + 100, 3 * T // 4 + 101, T], dtype=torch.int64)
+        inp = random_inputs(1, T, 2, K, V, torch.bfloat16, gate=gate, h0=True, seed=61, cu_seqlens=cu)
+        call = lambda d: sg.simple_gla_fwd_varlen(d["q"], d["k"], d["v"], d["cu"], g=d["g"], g_gamma=d["g_gamma"],
+                                                  initial_state=d["h0"], output_final_state=True)
+        ref = oracle_fwd(inp, cu=cu)
+    else:
+        cu = None
+        T = 12000 if K == 128 else 3000
+        inp = random_inputs(1, T, 2 if K == 128 else 1, K, V, torch.bfloat16, gate=gate, h0=True, seed=62)
+        call = lambda d: sg.simple_gla_fwd(d["q"], d["k"], d["v"], g=d["g"], g_gamma=d["g_gamma"],
+                                           initial_state=d["h0"], output_final_state=True)
+        ref = oracle_fwd(inp)
+    d = {k_: to_dev(inp[k_]) for k_ in ("q", "k", "v", "g", "g_gamma", "h0")}
+    d["cu"] = to_dev(cu)
+    runs = []
+    for _ in range(4):
+        o, ht = call(d)
+        runs.append((o.clone(), ht.clone()))
+    torch.cuda.synchronize()
+    for o, ht in runs[1:]:
+        assert torch.equal(o, runs[0][0]) and torch.equal(ht, runs[0][1]), "calls differ"
+    check(inp, (host(runs[0][0]), host(runs[0][1])), ref, torch.bfloat16, "walk under the state pass")
