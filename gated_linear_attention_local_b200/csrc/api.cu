@@ -140,38 +140,57 @@ Plan make_plan(bool varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t 
         double best = 1e300;
         L = nt;
         const int64_t min_l = std::min<int64_t>(nt, 4);
-        for (int64_t ns = 1; ns <= std::min<int64_t>(nt, 512); ++ns) {
-            const int64_t l = (nt + ns - 1) / ns, ns_eff = (nt + l - 1) / l;
-            if (l < min_l) break;
-            if (varlen) {
-                // packed batches: the segments of unequal sequences are dispatched longest
-                // first (seg_order) as SMs free up, so the walk takes the larger of its
-                // longest segment and its total work spread over the SMs; sequences of a
-                // uniform length mix hold mean/l + 1/2 segments each
-                const double mean_steps = (double)T / ((double)std::max<int64_t>(N, 1) * (double)C);
+        if (varlen) {
+            // Packed batches: the segments of unequal sequences are dispatched longest first
+            // (seg_order) as SMs free up, so the walk takes the larger of its longest
+            // segment and its total work spread over the SMs; sequences of a uniform length
+            // mix hold mean/l + 1/2 segments each.  Unless the [V,K] layout puts a carry
+            // pass between them, the walk starts under the state pass: first segments at
+            // once, later ones when the pass ends, so the call takes the longest of those
+            // two chains, the work of both kernels spread over the SMs and their bytes.
+            const bool overlap = !state_only && !state_v_first;
+            const double per_seq = (double)std::max<int64_t>(N, 1);
+            const double mean_steps = (double)T / (per_seq * (double)C);
+            const double steps = (double)T / (double)C;
+            auto varlen_cost = [&](int64_t l) {
                 const double segs = (double)N * std::max(1.0, mean_steps / (double)l + 0.5);
-                const double steps = (double)T / (double)C;
-                const double t_w = state_only ? 0.0
-                                   : std::max({(double)(l + 2) * t_walk,
-                                               (double)units / (double)std::max<int64_t>(N, 1) *
-                                                   (steps + 2.0 * segs) * t_walk / 148.0,
-                                               walk_bytes / bw});
                 const double seg_state = state_only ? segs : std::max(0.0, segs - (double)N);
+                const double frac = std::min(1.0, seg_state * (double)l / std::max(steps, 1.0));
+                const double walk_work = (double)units / per_seq * (steps + 2.0 * segs) * t_walk;
+                const double state_work = (double)state_units / per_seq * seg_state * (double)(l + 1) * t_state;
                 double t_s = 0.0;
                 if (seg_state > 0.0) {
-                    const double frac = std::min(1.0, seg_state * (double)l / std::max(steps, 1.0));
-                    t_s = std::max({(double)(l + 1) * t_state,
-                                    (double)state_units / (double)std::max<int64_t>(N, 1) * seg_state *
-                                        (double)(l + 1) * t_state / 148.0,
-                                    kv_bytes * frac / bw_state});
+                    t_s = std::max({(double)(l + 1) * t_state, state_work / 148.0, kv_bytes * frac / bw_state});
                     if (state_only) t_s += segs * (double)H * (double)K * (double)V * 4.0 / bw;
                 }
-                if (t_w + t_s < best - 1e-9) {
-                    best = t_w + t_s;
+                if (state_only) return t_s;
+                if (overlap) {
+                    const double first = (double)(std::min(l, nt) + 2) * t_walk;
+                    const double later = nt > l ? t_s + (double)(std::min(l, nt - l) + 2) * t_walk : 0.0;
+                    return std::max({first, later, (walk_work + state_work) / 148.0,
+                                     (walk_bytes + kv_bytes * frac) / bw});
+                }
+                return std::max({(double)(l + 2) * t_walk, walk_work / 148.0, walk_bytes / bw}) + t_s;
+            };
+            auto consider = [&](int64_t l) {
+                const double cost = varlen_cost(l);
+                if (cost < best - 1e-9) {
+                    best = cost;
                     L = l;
                 }
-                continue;
+            };
+            // the lengths above 1024 steps that split the longest sequence evenly, then
+            // every length from 1024 steps down
+            for (int64_t ns = 1; ns <= std::min<int64_t>(nt, 512); ++ns) {
+                const int64_t l = (nt + ns - 1) / ns;
+                if (l <= 1024) break;
+                consider(l);
             }
+            for (int64_t l = std::min<int64_t>(nt, 1024); l >= min_l; --l) consider(l);
+        }
+        for (int64_t ns = 1; !varlen && ns <= std::min<int64_t>(nt, 512); ++ns) {
+            const int64_t l = (nt + ns - 1) / ns, ns_eff = (nt + l - 1) / l;
+            if (l < min_l) break;
             const double waves_walk = (double)((units * ns_eff + 147) / 148);
             const double t_w = state_only ? 0.0 : std::max(waves_walk * (double)(l + 2) * t_walk, walk_bytes / bw);
             double t_s = 0.0;
