@@ -622,8 +622,8 @@ sgla_status simple_gla_chunk_final_state(const void *k, const void *v, const flo
         SGLA_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), st), "status reset");
     }
     if (N == 0) return SGLA_OK;
-    // the K = 256 / 512 walk and the k-block state pass form the chunk-local cumsum of the
-    // gates themselves; the K = 128 kernels read it from this pass
+    // the k-block state pass (K = 256 / 512) forms the chunk-local cumsum of the gates
+    // itself; the K = 128 and CUDA-core passes read it from this pass
     if (per_token && tokens > 0 && (!p.tc || K == 128))
         SGLA_LAUNCH("chunk_cumsum", launch_chunk_cumsum(g, a.gcum, a.gpos, lay, st));
     if (p.max_segs > 0 && tokens > 0) {

@@ -4,8 +4,9 @@
 // section 3: the state is carried between chunks by one scalar decay and the k^T v of
 // the chunk, so the state a segment of the sequence leaves behind, starting from zero,
 // is the decay-weighted sum  sum_j 2^(G_end - G_j) k_j v_j^T  over its tokens.  The
-// carry kernel combines these local end states across segments; the walk of every
-// segment but the first then starts from the carried state.
+// walk of every later segment folds these local end states onto the initial state (the
+// scalar-decay carry) to form the state it starts from; on a state-only call the carry
+// kernel folds all of them into the final state.
 //
 // One CTA per (non-final segment, head, 128-wide V tile) walks its segment BACKWARDS,
 // 128 tokens per step, so the decay from a token to the segment end is a running
