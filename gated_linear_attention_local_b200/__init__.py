@@ -40,6 +40,7 @@ import os
 
 import torch
 
+from . import _lib as _lib_mod
 from ._lib import (SGLA_BF16, SGLA_FP32, SGLA_OK, SglaError, lib, library_path,  # noqa: F401
                    raise_for_status)
 
@@ -48,6 +49,7 @@ __all__ = ["simple_gla_fwd", "simple_gla_fwd_noalloc", "simple_gla_fwd_varlen", 
            "simple_gla_normalized", "simple_gla_normalized_decode_step", "normalized_decode_state_width",
            "gla_fused_recurrent", "simple_gla_fused_recurrent_bwd", "simple_gla_chunk_bwd", "gla_chunk", "ChunkSimpleGLAFunction",
            "simple_gla_log_decay_total", "simple_gla_state_carry", "simple_gla_chunk_final_state",
+           "simple_gla_chunk_plan",
            "fwd_workspace_size", "varlen_workspace_size", "workspace_status", "noalloc_status", "library_path",
            "SglaError"]
 
@@ -290,6 +292,23 @@ def simple_gla_chunk(q, k, v, g=None, g_gamma=None, scale=None, initial_state=No
 
 
 @_on_tensor_device
+def simple_gla_chunk_plan(N, T, H, K, V, varlen=False, chunk_size=64, per_token_gate=True, state_v_first=False,
+                          dtype=torch.bfloat16):
+    """The plan a chunked forward makes for these sizes (host only, no device needed):
+    {"tensor_cores", "step_tokens", "segment_steps", "max_segments", "workspace_bytes"}.
+    varlen: N packed sequences in T tokens, else N sequences of T tokens."""
+    if dtype not in _DTYPES:
+        raise TypeError("dtype must be torch.bfloat16 or torch.float32")
+    out = _lib_mod.ChunkPlan()
+    st = lib().simple_gla_chunk_plan(int(bool(varlen)), int(N), int(T), int(H), int(K), int(V), int(chunk_size),
+                                     int(bool(per_token_gate)), int(bool(state_v_first)), _DTYPES[dtype],
+                                     ctypes.byref(out))
+    raise_for_status(st, "simple_gla_chunk_plan")
+    return {"tensor_cores": bool(out.tensor_cores), "step_tokens": out.step_tokens,
+            "segment_steps": out.segment_steps, "max_segments": out.max_segments,
+            "workspace_bytes": out.workspace_bytes}
+
+
 def simple_gla_chunk_final_state(k, v, g=None, g_gamma=None, initial_state=None, cu_seqlens=None, chunk_size=64,
                                  workspace=None):
     """The final state of the chunked forward without its output (the state pass of

@@ -83,6 +83,17 @@ _SIG = {
 _lib = None
 
 
+class ChunkPlan(ctypes.Structure):
+    """sgla_chunk_plan of include/simple_gla.h."""
+    _fields_ = [("tensor_cores", ctypes.c_int32), ("step_tokens", ctypes.c_int32),
+                ("segment_steps", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("max_segments", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
+
+
+_SIG["simple_gla_chunk_plan"] = ([ctypes.c_int, _I64, _I64, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
+                                  ctypes.c_int, ctypes.c_int, ctypes.POINTER(ChunkPlan)], ctypes.c_int)
+
+
 class SglaError(RuntimeError):
     def __init__(self, status, where, detail=""):
         self.status = status

@@ -552,6 +552,22 @@ size_t simple_gla_chunk_workspace_size(const int64_t *cu_seqlens, int64_t N, int
     return p.valid ? p.bytes : 0;
 }
 
+sgla_status simple_gla_chunk_plan(int varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V,
+                                  int chunk_size, int per_token_gate, int state_v_first, sgla_dtype dtype,
+                                  sgla_chunk_plan *out) {
+    if (!out) return SGLA_ERR_INVALID_ARGUMENT;
+    if (N < (varlen ? 1 : 0) || T < 0) return SGLA_ERR_INVALID_ARGUMENT;
+    const Plan p = make_plan(varlen != 0, N, T, H, K, V, chunk_size, dtype, per_token_gate != 0, state_v_first != 0);
+    if (!p.valid) return p.why;
+    out->tensor_cores = p.tc ? 1 : 0;
+    out->step_tokens = p.C;
+    out->segment_steps = p.L;
+    out->reserved = 0;
+    out->max_segments = p.max_segs;
+    out->workspace_bytes = (int64_t)p.bytes;
+    return SGLA_OK;
+}
+
 sgla_status simple_gla_chunk(const void *q, const void *k, const void *v, const float *g, const float *g_gamma,
                              float scale, const float *initial_state, void *o, float *final_state,
                              const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V,

@@ -275,6 +275,31 @@ SGLA_API sgla_status simple_gla_chunk_bwd(const void *q, const void *k, const vo
 SGLA_API size_t simple_gla_chunk_workspace_size(const int64_t *cu_seqlens, int64_t N, int64_t T, int64_t H,
                                                 int64_t K, int64_t V, int chunk_size, int state_v_first,
                                                 sgla_dtype dtype);
+
+/*
+ * The plan a chunked forward makes for these sizes, for inspection: host-only, it
+ * reads no device memory and launches nothing.  A sequence is cut into segments of
+ * segment_steps steps of step_tokens tokens each (article section 3: the state
+ * passes between chunks through one scalar decay, so the segments of one sequence
+ * run side by side and their end states are combined by that carry); the walk runs
+ * one CTA per (segment, head, V tile).  varlen != 0 plans a packed batch of N
+ * sequences in T tokens (as simple_gla_fwd_varlen), else N sequences of T tokens;
+ * per_token_gate != 0 for a per-token g; state_v_first as simple_gla_chunk.  Fills
+ * *out and returns SGLA_OK, or returns the status the forward would return for these
+ * sizes (out untouched).  out == NULL -> SGLA_ERR_INVALID_ARGUMENT.
+ */
+typedef struct {
+    int32_t tensor_cores;    /* 1: tcgen05 kernels (bf16), 0: CUDA-core kernels */
+    int32_t step_tokens;     /* tokens per step of the chunk kernels */
+    int32_t segment_steps;   /* steps per segment */
+    int32_t reserved;        /* 0 */
+    int64_t max_segments;    /* segments planned for (an upper bound for a packed batch) */
+    int64_t workspace_bytes; /* what this call needs (simple_gla_chunk_workspace_size with
+                                a per-token gate is an upper bound of it) */
+} sgla_chunk_plan;
+SGLA_API sgla_status simple_gla_chunk_plan(int varlen, int64_t N, int64_t T, int64_t H, int64_t K, int64_t V,
+                                           int chunk_size, int per_token_gate, int state_v_first,
+                                           sgla_dtype dtype, sgla_chunk_plan *out);
 SGLA_API sgla_status simple_gla_chunk(const void *q, const void *k, const void *v, const float *g,
                              const float *g_gamma, float scale, const float *initial_state, void *o,
                              float *final_state, const int64_t *cu_seqlens, int64_t N, int64_t T,

@@ -278,3 +278,66 @@ def test_every_compute_entry_point_has_a_binding_of_the_same_name():
     assert {"simple_gla_fwd", "simple_gla_fwd_varlen", "simple_gla_decode_step"} <= set(compute)
     missing = [n for n in compute if not callable(getattr(sg, n, None))]
     assert not missing, missing
+
+
+def test_chunk_plan_of_the_measured_workloads(lib):
+    """The plan the chunked forward makes for the measured workloads, read on the host:
+    the path, the step, the segment length the cost model picks (one segment per
+    sequence at K = V = 512, four per sequence on the long per-head-decay workload, and
+    the length that balances the walk started under the state pass on the packed
+    batch), and the workspace against the size queries."""
+    import gated_linear_attention_local_b200 as sg
+    p = sg.simple_gla_chunk_plan(4, 2048, 4, 512, 512)  # dense_prefill
+    assert p["tensor_cores"] and p["step_tokens"] == 128
+    assert p["segment_steps"] == 16 and p["max_segments"] == 4
+    assert p["workspace_bytes"] == sg.fwd_workspace_size(4, 2048, 4, 512, 512)
+    p = sg.simple_gla_chunk_plan(1, 65536, 32, 128, 128, per_token_gate=False)  # long_gamma
+    assert p["segment_steps"] == 128 and p["max_segments"] == 4
+    p = sg.simple_gla_chunk_plan(8, 18062, 16, 128, 128, varlen=True)  # varlen_prefill
+    assert p["segment_steps"] == 20
+    assert p["workspace_bytes"] == sg.varlen_workspace_size(8, 18062, 16, 128, 128)
+    p = sg.simple_gla_chunk_plan(1, 256, 2, 64, 64, dtype=torch.float32)  # tiny_fp32
+    assert not p["tensor_cores"] and p["step_tokens"] == 64
+
+
+def test_chunk_plan_agrees_with_the_workspace_query(lib):
+    """Over random sizes: the plan's workspace is what simple_gla_chunk_workspace_size
+    reports (per-token gate, either state layout), its segments cover every chunk of a
+    dense batch exactly, and a packed plan bounds the segments any split can need."""
+    import random
+
+    import gated_linear_attention_local_b200 as sg
+    rng = random.Random(5)
+    for _ in range(300):
+        varlen = rng.random() < 0.5
+        N = rng.randint(1, 48)
+        T = rng.randint(0, 300000)
+        H = rng.choice([1, 2, 4, 16, 32])
+        K, V = rng.choice([(64, 64), (128, 128), (128, 64), (256, 128), (512, 512), (96, 40)])
+        chunk = rng.choice([16, 32, 64, 128])
+        vf = rng.random() < 0.3
+        dtype = rng.choice([torch.bfloat16, torch.float32])
+        p = sg.simple_gla_chunk_plan(N, T, H, K, V, varlen=varlen, chunk_size=chunk, state_v_first=vf,
+                                     dtype=dtype)
+        cu = ctypes.c_void_p(8) if varlen else None  # the size query only tests it against NULL
+        want = lib.simple_gla_chunk_workspace_size(cu, N, T, H, K, V, chunk, int(vf), sg._DTYPES[dtype])
+        assert p["workspace_bytes"] == want
+        C, L = p["step_tokens"], p["segment_steps"]
+        assert C in (16, 32, 64, 128) and L >= 1
+        if varlen:
+            # every sequence of n tokens needs ceil(ceil(n / C) / L) segments; the sum over
+            # any split of T tokens into N sequences is at most T // (C L) + N
+            assert p["max_segments"] == T // (C * L) + N
+        else:
+            assert p["max_segments"] == N * -(-(-(-T // C)) // L)
+
+
+def test_chunk_plan_rejects_what_the_forward_rejects(lib):
+    import gated_linear_attention_local_b200 as sg
+    with pytest.raises(ValueError):
+        sg.simple_gla_chunk_plan(1, 256, 2, 64, 64, chunk_size=48)
+    with pytest.raises(NotImplementedError):
+        sg.simple_gla_chunk_plan(1, 256, 2, 64, 64, chunk_size=256)
+    with pytest.raises(ValueError):
+        sg.simple_gla_chunk_plan(0, 256, 2, 64, 64, varlen=True)
+    assert lib.simple_gla_chunk_plan(0, 1, 256, 2, 64, 64, 64, 1, 0, L.SGLA_BF16, None) == L.SGLA_ERR_INVALID_ARGUMENT
